@@ -1,0 +1,383 @@
+/*
+ * moe_oracle.c -- float64 CPU reference for the forward pass of a sparse
+ * Mixture-of-Experts feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE. Only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark load this library. The product path (the CUDA library)
+ * never links, loads or calls it, and the two share no code.
+ *
+ * Style rules this file keeps so that a reader can check it against the pages:
+ *   - one plain loop nest per formula, single thread, no blocking, no fusion;
+ *   - every sum runs in ascending order of its reduction index;
+ *   - all arithmetic is float64; BF16 / FP32 inputs are upcast exactly.
+ *
+ * Sources (page title, section / equation):
+ *   [ZM]  "Zen MoDE: Mixture of Distilled Experts Architecture"
+ *         §3.1 Router Architecture (eq. router_standard), §5.2 Auxiliary Load
+ *         Balancing Loss (eq. L_balance), §5.3 Adaptive Capacity Factors
+ *         (capacity_e), §6.2 Expert Utilization (table tab:utilization),
+ *         §7.1 Compute Budget (FLOPs ratio).
+ *   [ZX]  "Zen-Max: Maximum Capability via Mixture-of-Experts Architecture"
+ *         §2.2 Fine-Grained Expert Architecture (Expert_i, shared experts),
+ *         §2.3 Auxiliary-Loss-Free Load Balancing (s_ij = softmax(x W_g)_j + b_j),
+ *         §3.2 MoE-Specific Training Stability (router z-loss).
+ *   [SE]  "Scaling with experts" (jeff-ong.com), sections "The gating network",
+ *         "A balance penalty", "A budget", "A shared expert".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Element type codes for inputs handed to the oracle. */
+enum { ORC_F64 = 0, ORC_F32 = 1, ORC_BF16 = 2 };
+
+/* Bias placement for selection (see oracle_select). */
+enum { ORC_BIAS_PROB = 0, ORC_BIAS_LOGIT = 1 };
+
+/* Bytes per element of an input type code. */
+static size_t esz(int dt) { return dt == ORC_F64 ? 8 : dt == ORC_F32 ? 4 : 2; }
+
+/* Exact upcast of element i of an input array to float64.  BF16 is the upper
+ * half of an IEEE float32, so shifting it up 16 bits gives the float exactly. */
+static double ld(const void* p, int dt, int64_t i) {
+    if (dt == ORC_F64) return ((const double*)p)[i];
+    if (dt == ORC_F32) return (double)((const float*)p)[i];
+    uint32_t bits = ((uint32_t)((const uint16_t*)p)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* ---------------------------------------------------------------------------
+ * Gate logits.  [ZM] §3.1: the standard router applies a linear projection
+ * W_r to the token; [SE] "The gating network": one score per expert.
+ *   logits[t,e] = sum_j x[t,j] * Wg[e,j]   (+ offset[e] when given)
+ * Wg is stored as [E, d] (one row per expert).  The optional additive offset
+ * is an input of the layer (used to impose a popularity prior on experts).
+ * ------------------------------------------------------------------------- */
+void oracle_gate_logits(int64_t T, int32_t d, int32_t E,
+                        const void* x, int32_t x_dt,
+                        const void* wg, int32_t wg_dt,
+                        const float* offset, double* logits) {
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int32_t j = 0; j < d; ++j)
+                acc += ld(x, x_dt, t * (int64_t)d + j) * ld(wg, wg_dt, (int64_t)e * d + j);
+            if (offset) acc += (double)offset[e];
+            logits[t * E + e] = acc;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Softmax over all E experts of one token.  [ZM] §3.1 eq. router_standard:
+ * softmax(W_r x).  Shifted by the row maximum (the value is unchanged).
+ *   p[t,e] = exp(l[t,e] - m_t) / sum_e' exp(l[t,e'] - m_t)
+ * ------------------------------------------------------------------------- */
+void oracle_softmax(int64_t T, int32_t E, const double* logits, double* p) {
+    for (int64_t t = 0; t < T; ++t) {
+        const double* l = logits + t * E;
+        double m = l[0];
+        for (int32_t e = 1; e < E; ++e)
+            if (l[e] > m) m = l[e];
+        double z = 0.0;
+        for (int32_t e = 0; e < E; ++e) z += exp(l[e] - m);
+        for (int32_t e = 0; e < E; ++e) p[t * E + e] = exp(l[e] - m) / z;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Top-K selection and renormalised gate weights.
+ *
+ * Selection score s[e]:
+ *   no bias            : s = logit            (softmax is monotone, so this
+ *                                              is TopK(softmax(W_r x)) of [ZM] §3.1)
+ *   bias, BIAS_PROB    : s = p + b            ([ZX] §2.3: softmax(x W_g)_j + b_j)
+ *   bias, BIAS_LOGIT   : s = logit + b        (variant: bias in logit space)
+ * The bias steers selection only; gate weights never see it.
+ * The K chosen experts are those with the largest s; equal scores go to the
+ * lower expert index; they are listed in that order (largest s first).
+ *
+ * Gate weights ([SE] "The gating network": keep the top-k scores, zero the
+ * rest, renormalise the survivors to sum to one):
+ *   w[t,k] = p[t, idx[t,k]] / sum_k' p[t, idx[t,k']]
+ * which equals a softmax taken over the selected logits only.
+ *
+ * Returns 0, or -1 when K is outside [1, E].
+ * ------------------------------------------------------------------------- */
+int oracle_select(int64_t T, int32_t E, int32_t K,
+                  const double* logits, const double* p,
+                  const float* bias, int32_t bias_mode,
+                  int32_t* idx, double* w) {
+    if (K < 1 || K > E) return -1;
+    double* s = (double*)malloc(sizeof(double) * (size_t)E);
+    char* taken = (char*)malloc((size_t)E);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t e = 0; e < E; ++e) {
+            double v = logits[t * E + e];
+            if (bias) {
+                if (bias_mode == ORC_BIAS_LOGIT) v = logits[t * E + e] + (double)bias[e];
+                else                             v = p[t * E + e] + (double)bias[e];
+            }
+            s[e] = v;
+            taken[e] = 0;
+        }
+        /* K passes; each takes the best remaining expert (strictly greater score
+         * wins, so on a tie the earlier, i.e. lower, index is kept). */
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || s[e] > s[best]) best = e;
+            }
+            taken[best] = 1;
+            idx[t * K + k] = best;
+        }
+        double denom = 0.0;
+        for (int32_t k = 0; k < K; ++k) denom += p[t * E + idx[t * K + k]];
+        for (int32_t k = 0; k < K; ++k) w[t * K + k] = p[t * E + idx[t * K + k]] / denom;
+    }
+    free(s);
+    free(taken);
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Per-expert capacity.  [ZM] §5.3: capacity_e = C * (batch*seq) / N_E, the
+ * Switch top-1 form.  With top-K routing each token makes K assignments, so
+ * the budget that keeps a uniform load whole is C * T * K / E; it is rounded
+ * up to a whole number of rows.  C <= 0 means no limit (returns -1).
+ * Computed in float64 as (C * (T*K)) / E, then ceil.
+ * ------------------------------------------------------------------------- */
+int64_t oracle_capacity(int64_t T, int32_t K, int32_t E, float C) {
+    if (!(C > 0.0f)) return -1;
+    double v = ((double)C * (double)(T * (int64_t)K)) / (double)E;
+    return (int64_t)ceil(v);
+}
+
+/* ---------------------------------------------------------------------------
+ * Capacity-limited dispatch.  [SE] "A budget": each expert takes a limited
+ * number of tokens per batch; tokens past the budget are dropped (their expert
+ * update is skipped and they continue through the residual).
+ *
+ *   counts[e]  = number of (t,k) with idx[t,k] == e               (pre-capacity)
+ *   kept[e]    = min(counts[e], cap)        (counts[e] if cap < 0)
+ *   seg_off    = exclusive prefix sum of kept; seg_off[E] = total kept rows
+ *   rank(t,k)  = number of tokens t' < t that also chose e = idx[t,k]
+ *   kept iff rank < kept[e]; then slot_of[t,k] = seg_off[e] + rank and
+ *   perm[slot] = t*K + k; otherwise slot_of[t,k] = -1.
+ * Tokens are served in ascending token order (first come, first served).
+ * Returns 0, or -1 on an expert index outside [0, E).
+ * ------------------------------------------------------------------------- */
+int oracle_dispatch(int64_t T, int32_t K, int32_t E, int64_t cap,
+                    const int32_t* idx,
+                    int32_t* counts, int32_t* kept, int32_t* seg_off,
+                    int32_t* slot_of, int32_t* perm) {
+    for (int32_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t i = 0; i < T * (int64_t)K; ++i) {
+        if (idx[i] < 0 || idx[i] >= E) return -1;
+        counts[idx[i]] += 1;
+    }
+    for (int32_t e = 0; e < E; ++e)
+        kept[e] = (cap < 0 || counts[e] < cap) ? counts[e] : (int32_t)cap;
+    seg_off[0] = 0;
+    for (int32_t e = 0; e < E; ++e) seg_off[e + 1] = seg_off[e] + kept[e];
+
+    int32_t* seen = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t e = idx[t * K + k];
+            int32_t rank = seen[e];
+            seen[e] += 1;
+            if (rank < kept[e]) {
+                int32_t slot = seg_off[e] + rank;
+                slot_of[t * K + k] = slot;
+                perm[slot] = (int32_t)(t * K + k);
+            } else {
+                slot_of[t * K + k] = -1;
+            }
+        }
+    }
+    free(seen);
+    return 0;
+}
+
+/* SiLU, [ZX] §2.2 (activation): silu(z) = z * sigmoid(z) = z / (1 + e^-z). */
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* ---------------------------------------------------------------------------
+ * One SwiGLU expert applied to one token.  [ZX] §2.2 eq. Expert_i:
+ *   Expert(x) = (SiLU(x W_gate) (.) x W_up) W_down
+ * Storage ("linear [out, in]"): w13 is [2F, d] with rows 0..F-1 the gate
+ * projection and rows F..2F-1 the up projection; w2 is [d, F].
+ *   g[f] = sum_j w13[f, j]   x[j]
+ *   u[f] = sum_j w13[F+f, j] x[j]
+ *   h[f] = silu(g[f]) * u[f]
+ *   out[i] += scale * sum_f w2[i, f] h[f]
+ * h is caller scratch of F doubles.
+ * ------------------------------------------------------------------------- */
+void oracle_swiglu_accumulate(int32_t d, int32_t F, const double* x,
+                              const void* w13, const void* w2, int32_t w_dt,
+                              double scale, double* h, double* out) {
+    for (int32_t f = 0; f < F; ++f) {
+        double g = 0.0, u = 0.0;
+        for (int32_t j = 0; j < d; ++j) {
+            g += ld(w13, w_dt, (int64_t)f * d + j) * x[j];
+            u += ld(w13, w_dt, (int64_t)(F + f) * d + j) * x[j];
+        }
+        h[f] = silu(g) * u;
+    }
+    for (int32_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int32_t f = 0; f < F; ++f) acc += ld(w2, w_dt, (int64_t)i * F + f) * h[f];
+        out[i] += scale * acc;
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * The layer output for a list of tokens, given the routing.
+ *   y[t] = sum_{s < N_s} Expert^shared_s(x_t)
+ *        + sum_{k : slot_of[t,k] >= 0} w[t,k] * Expert_{idx[t,k]}(x_t)
+ * Shared experts: always active, added unweighted ([ZX] §2.2; [SE] "A shared
+ * expert").  Routed part: gate-weighted sum ([SE] "The gating network":
+ * y = g1 Expert1(x) + g2 Expert2(x)).  A dropped pair contributes nothing and
+ * the survivors are not renormalised again ([SE] "A budget").  The residual
+ * add is outside the layer.
+ * Layouts: x [T, d]; w13 [E, 2F, d]; w2 [E, d, F]; shared weights
+ * [N_s, 2F, d] / [N_s, d, F]; y rows written for the listed tokens only:
+ * y[r * d + i] for r = 0..n_rows-1 (row r is token rows[r]).
+ * Returns 0, or -1 on an out-of-range token or expert.
+ * ------------------------------------------------------------------------- */
+int oracle_layer_rows(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32_t n_shared,
+                      const void* x, int32_t x_dt,
+                      const void* w13, const void* w2,
+                      const void* w13_sh, const void* w2_sh, int32_t w_dt,
+                      const int32_t* idx, const double* w, const int32_t* slot_of,
+                      int64_t n_rows, const int64_t* rows, double* y) {
+    double* xr = (double*)malloc(sizeof(double) * (size_t)d);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    const int64_t w13_stride = 2 * (int64_t)F * d;
+    const int64_t w2_stride = (int64_t)d * F;
+    int rc = 0;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t t = rows[r];
+        if (t < 0 || t >= T) { rc = -1; break; }
+        for (int32_t j = 0; j < d; ++j) xr[j] = ld(x, x_dt, t * d + j);
+        double* yr = y + r * d;
+        for (int32_t i = 0; i < d; ++i) yr[i] = 0.0;
+        for (int32_t s = 0; s < n_shared; ++s) {
+            const char* a = (const char*)w13_sh + (size_t)(s * w13_stride) * esz(w_dt);
+            const char* b = (const char*)w2_sh + (size_t)(s * w2_stride) * esz(w_dt);
+            oracle_swiglu_accumulate(d, F, xr, a, b, w_dt, 1.0, h, yr);
+        }
+        for (int32_t k = 0; k < K; ++k) {
+            if (slot_of[t * K + k] < 0) continue;
+            int32_t e = idx[t * K + k];
+            if (e < 0 || e >= E) { rc = -1; break; }
+            const char* a = (const char*)w13 + (size_t)(e * w13_stride) * esz(w_dt);
+            const char* b = (const char*)w2 + (size_t)(e * w2_stride) * esz(w_dt);
+            oracle_swiglu_accumulate(d, F, xr, a, b, w_dt, w[t * K + k], h, yr);
+        }
+        if (rc) break;
+    }
+    free(xr);
+    free(h);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Switch balance statistics.  [ZM] §5.2 eq. L_balance and [SE] "A balance
+ * penalty":  L = alpha * N * sum_e f_e P_e, with
+ *   f_e = counts[e] / (T*K)   fraction of the batch's assignments sent to e
+ *                             (counted before the capacity cut)
+ *   P_e = (1/T) sum_t p[t,e]  average routing probability of e
+ * With uniform routing (f_e = P_e = 1/E) the loss is exactly alpha.
+ * ------------------------------------------------------------------------- */
+void oracle_balance(int64_t T, int32_t E, int32_t K, const int32_t* counts,
+                    const double* p, double alpha, double* f, double* P, double* loss) {
+    double acc = 0.0;
+    for (int32_t e = 0; e < E; ++e) {
+        f[e] = (double)counts[e] / (double)(T * (int64_t)K);
+        double s = 0.0;
+        for (int64_t t = 0; t < T; ++t) s += p[t * E + e];
+        P[e] = s / (double)T;
+    }
+    for (int32_t e = 0; e < E; ++e) acc += f[e] * P[e];
+    *loss = alpha * (double)E * acc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Router z-loss.  [ZX] §3.2: L_z = (1/B) sum_x (log sum_j e^{x_j})^2 over the
+ * router logits of the B tokens.  (Coefficient applied by the caller.)
+ * ------------------------------------------------------------------------- */
+double oracle_router_zloss(int64_t T, int32_t E, const double* logits) {
+    double acc = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        const double* l = logits + t * E;
+        double m = l[0];
+        for (int32_t e = 1; e < E; ++e)
+            if (l[e] > m) m = l[e];
+        double z = 0.0;
+        for (int32_t e = 0; e < E; ++e) z += exp(l[e] - m);
+        double lse = m + log(z);
+        acc += lse * lse;
+    }
+    return acc / (double)T;
+}
+
+/* ---------------------------------------------------------------------------
+ * Expert utilisation statistics, [ZM] §6.2 table tab:utilization, from the
+ * per-expert assignment counts (n = sum counts):
+ *   out[0] entropy in bits of the load distribution q_e = counts[e]/n
+ *          (0 log 0 = 0; at most log2 E, "max 7 bits" for 128 experts)
+ *   out[1] coefficient of variation of counts (population std / mean)
+ *   out[2] token drop rate: dropped assignments / n
+ *   out[3] experts whose load is below 50% of the mean
+ *   out[4] experts whose load is above 200% of the mean
+ * ------------------------------------------------------------------------- */
+void oracle_utilization(int32_t E, const int32_t* counts, const int32_t* kept, double* out) {
+    double n = 0.0, dropped = 0.0;
+    for (int32_t e = 0; e < E; ++e) {
+        n += counts[e];
+        dropped += (double)(counts[e] - kept[e]);
+    }
+    double mean = n / (double)E;
+    double ent = 0.0, var = 0.0, below = 0.0, above = 0.0;
+    for (int32_t e = 0; e < E; ++e) {
+        if (counts[e] > 0) {
+            double q = (double)counts[e] / n;
+            ent -= q * log2(q);
+        }
+        double dv = (double)counts[e] - mean;
+        var += dv * dv;
+        if ((double)counts[e] < 0.5 * mean) below += 1.0;
+        if ((double)counts[e] > 2.0 * mean) above += 1.0;
+    }
+    var /= (double)E;
+    out[0] = ent;
+    out[1] = mean > 0.0 ? sqrt(var) / mean : 0.0;
+    out[2] = n > 0.0 ? dropped / n : 0.0;
+    out[3] = below;
+    out[4] = above;
+}
+
+/* ---------------------------------------------------------------------------
+ * Algorithmic FLOPs of one layer forward (multiply-add = 2 FLOPs):
+ *   router   2 T d E
+ *   experts  6 d F per kept (t,k) pair (three d x F projections)
+ *   shared   6 d F N_s per token
+ * and the ratio of expert FLOPs to the dense-equivalent cost of running every
+ * expert on every token, T E 6 d F.  With no drops the ratio is
+ * (K + N_s) / E, the [ZM] §7.1 compute-budget ratio (12/128 there).
+ * out[0] = total FLOPs, out[1] = expert FLOPs, out[2] = the ratio.
+ * ------------------------------------------------------------------------- */
+void oracle_flops(int64_t T, int32_t d, int32_t E, int32_t F, int32_t n_shared,
+                  int64_t kept_pairs, double* out) {
+    double router = 2.0 * (double)T * d * E;
+    double expert = 6.0 * (double)d * F * (double)kept_pairs + 6.0 * (double)d * F * n_shared * (double)T;
+    out[0] = router + expert;
+    out[1] = expert;
+    out[2] = expert / (6.0 * (double)d * F * (double)E * (double)T);
+}
