@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse-MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+
+One step = one moe_layer_forward (router -> dispatch -> routed SwiGLU experts
+-> shared experts -> combine, plus balance statistics) over one batch of T
+tokens of seeded synthetic input, weights resident in HBM.  The metric is
+tokens per second; for N > 1 (launched with torchrun, one rank per GPU) every
+rank runs its own independent batch (no collective on the data path: the layer
+does not shard), and value = N * T / (max over ranks of the step time).
+
+Printed (rank 0): one JSON line with the device-timed value, the end-to-end
+value through the public API with host buffers (H2D of x and D2H of y and the
+statistics inside the timed region), the roofline of the dominant kernel (the
+routed up/gate SwiGLU GEMM) timed with CUDA events on its own stream, per-stage
+times, SM clocks sampled during the timed region, and the float64 oracle timed
+on a bounded sample on the host's cores.
+
+--impl reference times the oracle itself (the CPU reference), a bounded
+sample of tokens per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_04_b200 import MoeLayer, api  # noqa: E402
+from sparse_mixture_experts_04_b200 import _lib  # noqa: E402
+from sparse_mixture_experts_04_b200.synth import CONFIGS, extra_activations, generate  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s (BF16, 1 B200); expert GEMM % peak; dispatch GB/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# oracle tokens per reference step / in the cpu_baseline sample (about 0.5-1 s each)
+REF_TOKENS = {"tiny_fp32": 64, "mixtral": 1, "zen_fine": 4, "skewed": 8, "decode": 2}
+CPU_SAMPLE_TOKENS = {"tiny_fp32": 64, "mixtral": 16, "zen_fine": 48, "skewed": 96, "decode": 16}
+
+
+def workload_desc(cfg) -> str:
+    return cfg.description
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(os.path.join(ROOT, "sparse_mixture_experts_04_b200", "csrc", "expert_gemm.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the up/gate GEMM from the committed ncu summary,
+    or None when absent or taken on an older version of the kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get("expert_up_swiglu")
+    if not e or e.get("source_sha256_16") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every few ms."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.err = [], 0, None
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hi = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hi)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hi
+            self.h = h if h is not None else pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML unavailable: report, do not fail the benchmark
+            self.h, self.err = None, f"{type(e).__name__}: {e}"
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.h is not None:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if self.h is None:
+            return {"error": self.err}
+        names = sorted(n for bit, n in self.REASONS.items() if self.reasons & bit)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+    def rejected(self) -> bool:
+        if self.h is None or not self.samples:
+            return False
+        bad = {"hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown"}
+        if bad & set(self.summary()["reasons"]):
+            return True
+        med = statistics.median(self.samples)
+        return self.max_mhz is not None and med < 0.6 * self.max_mhz and not (self.reasons & 0x4)
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_config(cfg, rank: int):
+    """Each rank runs its own independent batch: seed shifted by the rank."""
+    return cfg.replace(seed=cfg.seed + 1000 * rank)
+
+
+def algorithmic_flops(cfg, kept_pairs: int) -> dict:
+    d, F, E, T, Ns = cfg.d_model, cfg.d_ff, cfg.n_experts, cfg.T, cfg.n_shared
+    return {"router": 2.0 * T * d * E, "up": 4.0 * d * F * kept_pairs, "down": 2.0 * d * F * kept_pairs,
+            "shared": 6.0 * d * F * Ns * T}
+
+
+def dispatch_bytes(cfg, kept_pairs: int) -> float:
+    """topk_idx read twice (histogram, rank) + slot_of / perm written + x rows read + x_perm written."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    TK = cfg.T * cfg.top_k
+    return 4.0 * TK * 2 + 4.0 * TK + 4.0 * kept_pairs + 2.0 * kept_pairs * cfg.d_model * es
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_tokens_per_s(cfg, inp, n_tokens: int, offset: int = 0):
+    """The float64 oracle's full pipeline on n_tokens tokens of the workload
+    (gate logits, softmax/top-K, dispatch, SwiGLU experts, combine).  The sample
+    is routed as a batch of its own with no capacity limit (so every sampled
+    token does its full K experts of work).  Returns (tokens/s, seconds)."""
+    import oracle
+    from sparse_mixture_experts_04_b200.synth import bf16_bits
+
+    def host_np(t):
+        if t is None or isinstance(t, np.ndarray):
+            return t
+        return bf16_bits(t) if t.dtype == torch.bfloat16 else t.contiguous().numpy()
+
+    rows = (np.arange(n_tokens) + offset) % cfg.T
+    x = host_np(inp["x"])[rows]
+    t0 = time.perf_counter()
+    l = oracle.gate_logits(x, host_np(inp["w_gate"]), inp["logit_offset"])
+    idx, w, p = oracle.select(l, cfg.top_k, bias=inp["sel_bias"])
+    disp = oracle.dispatch(idx, cfg.n_experts, -1)
+    oracle.layer_rows(x, host_np(inp["w13"]), host_np(inp["w2"]), idx, w, disp["slot_of"],
+                      w13_shared=host_np(inp.get("w13_shared")), w2_shared=host_np(inp.get("w2_shared")))
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt
+
+
+def run_reference(args, cfg):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = generate(cfg)
+    for i in range(args.warmup):
+        oracle_tokens_per_s(cfg, inp, REF_TOKENS[cfg.name], offset=i)
+    times = []
+    for i in range(args.steps):
+        _, dt = oracle_tokens_per_s(cfg, inp, REF_TOKENS[cfg.name], offset=args.warmup + i)
+        times.append(dt)
+    step_s = sum(times) / len(times)
+    value = REF_TOKENS[cfg.name] / step_s
+    sample = (f"{REF_TOKENS[cfg.name]} token(s) of the {cfg.name} workload per step through the float64 oracle "
+              "(gate logits, top-K, dispatch, SwiGLU experts, combine), one thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, cfg):
+    rank, world, local_rank = dist_env()
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    rcfg = rank_config(cfg, rank)
+    inp = generate(rcfg)
+    layer = MoeLayer.from_inputs(inp)
+    T = cfg.T
+    x_bytes = T * cfg.d_model * (2 if cfg.dtype == "bf16" else 4)
+    n_x = max(2, math.ceil(2 * L2_BYTES / x_bytes) + 1)
+    n_x = min(n_x, 64)
+    xs_host = [inp["x"]] + extra_activations(rcfg, n_x - 1)
+    xs = [x.cuda() for x in xs_host]
+    y = torch.empty((T, cfg.d_model), dtype=layer.dtype, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i, events=None):
+        if events is None:
+            return api.moe_layer_forward(layer.prob, xs[i % n_x], layer.weights, y, layer.routing, layer.stats,
+                                         layer.ws, stream)
+        return api.moe_layer_forward_profiled(layer.prob, xs[i % n_x], layer.weights, y, layer.routing,
+                                              layer.stats, layer.ws, events, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    status = api.read_device_status(layer.ws)
+    if status:
+        raise RuntimeError(f"device status {status:#x} after warm-up")
+
+    def timed_region():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(_lib.NUM_EVENTS)] for _ in range(args.steps)]
+        for row in evs:       # create the underlying events before they are handed to the library
+            for e in row:
+                e.record(stream)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        n_k = 0
+        with ClockSampler(local_rank) as clk:
+            start.record(stream)
+            for i in range(args.steps):
+                n_k += step(args.warmup + i, evs[i])
+            end.record(stream)
+            torch.cuda.synchronize()
+        barrier(world)
+        ms = start.elapsed_time(end) / args.steps
+        stage = {}
+        for j in range(1, _lib.NUM_EVENTS):
+            stage[_lib.EVENT_NAMES[j]] = sum(evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(args.steps)) / args.steps
+        return ms, stage, n_k, clk
+
+    ms, stage, n_kernels, clk = timed_region()
+    remeasured = False
+    if clk.rejected():
+        ms, stage, n_kernels, clk = timed_region()
+        remeasured = True
+    ms_max = max_over_ranks(ms, world)
+    up_ms_max = max_over_ranks(stage["up"], world)
+
+    # end to end through the public API: pinned host x in, y and statistics out
+    xh = [x.pin_memory() for x in xs_host[: min(n_x, 4)]]
+    yh = torch.empty((T, cfg.d_model), dtype=layer.dtype).pin_memory()
+    sh = torch.empty_like(layer.stats, device="cpu").pin_memory()
+    xd = torch.empty_like(xs[0])
+    for i in range(2):
+        xd.copy_(xh[i % len(xh)], non_blocking=True)
+        layer.forward(xd, y)
+        yh.copy_(y, non_blocking=True)
+        sh.copy_(layer.stats, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for i in range(args.steps):
+        xd.copy_(xh[i % len(xh)], non_blocking=True)
+        layer.forward(xd, y)
+        yh.copy_(y, non_blocking=True)
+        sh.copy_(layer.stats, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world)
+    h2d = xd.numel() * xd.element_size()
+    d2h = y.numel() * y.element_size() + layer.stats.numel() * 4
+
+    kept = int(layer.routing["seg_off"][-1].item())
+    flops = algorithmic_flops(cfg, kept)
+    peaks, peak_src = load_peaks()
+    up_tflops = flops["up"] / (stage["up"] * 1e-3) / 1e12
+    gemm_ms = stage["up"] + stage["down"]
+    gemm_tflops = (flops["up"] + flops["down"]) / (gemm_ms * 1e-3) / 1e12
+    disp_gbs = dispatch_bytes(cfg, kept) / (stage["dispatched"] * 1e-3) / 1e9
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        n = CPU_SAMPLE_TOKENS[cfg.name]
+        v, dt = oracle_tokens_per_s(cfg, inp, n)
+        cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} tokens of the {cfg.name} workload through the float64 oracle's full pipeline "
+                         f"(no capacity limit within the sample), one thread, {dt:.1f} s"}
+    total_flops = sum(flops.values())
+    line = {
+        "metric": METRIC, "value": world * T / (ms_max * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+        "data": "synthetic: seeded N(0,1) activations, random-init N(0,1/d_in) weights",
+        "config": {"workload": workload_desc(cfg), "T": cfg.T, "d_model": cfg.d_model, "n_experts": cfg.n_experts,
+                   "top_k": cfg.top_k, "d_ff": cfg.d_ff, "n_shared": cfg.n_shared,
+                   "capacity_factor": cfg.capacity_factor, "global_batch": world * cfg.T,
+                   "parallelism": f"replicas x{world} (independent batch per GPU, no data-path collective)",
+                   "l2": f"{n_x} rotating activation batches ({n_x * x_bytes / 2**20:.0f} MiB) and "
+                         f"{sum(v.numel() * v.element_size() for v in layer.weights.values() if v is not None) / 2**30:.2f}"
+                         " GiB of weights per step, both larger than the 126 MB L2; no flush"},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "roofline": {"kernel": "routed up/gate GEMM with SwiGLU epilogue (tcgen05)", "bound": "tensor",
+                     "achieved": up_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": up_tflops / peaks["bf16_tflops"],
+                     "traffic": ncu_traffic(cfg.name),
+                     "algorithmic_flops_per_launch": flops["up"], "launch_ms": stage["up"],
+                     "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
+                     else "fallback 1.59 PFLOP/s"},
+        "cpu_baseline": cpu,
+        "gpu_launches": n_kernels,
+        "clocks": {**clk.summary(), "remeasured": remeasured},
+        "stages_ms": stage,
+        "kept_pairs": kept, "dropped_pairs": cfg.T * cfg.top_k - kept,
+        "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
+        "dispatch_gbs": disp_gbs, "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral", choices=list(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps, always
+    cfg = CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

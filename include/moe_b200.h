@@ -1,0 +1,256 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts FFN
+ * forward library (libmoe_b200.so).
+ *
+ * The layer (per token x_t, t < T):
+ *   logits  = W_g x_t (+ logit_offset)                 one score per expert
+ *   p       = softmax(logits)
+ *   chosen  = the K experts with the largest selection score
+ *             (logit; or p + b with a selection bias b)
+ *   w_k     = p[chosen_k] / sum_k' p[chosen_k']        renormalised gates
+ *   dispatch: each expert serves at most `cap` (t,k) pairs, first come first
+ *             served in token order; the rest are dropped
+ *   y_t     = sum_s SharedExpert_s(x_t) + sum_{kept k} w_k Expert_{chosen_k}(x_t)
+ *   Expert(x) = W_down (SiLU(W_gate x) * (W_up x))
+ * plus the Switch statistics f_e, P_e and alpha * E * sum_e f_e P_e.
+ * The residual add is the caller's.
+ *
+ * Sources (page title, section / equation):
+ *   "Zen MoDE: Mixture of Distilled Experts Architecture": §3.1 Router
+ *     Architecture (eq. router_standard, TopK(softmax(W_r x), K)); §5.2 Auxiliary
+ *     Load Balancing Loss (eq. L_balance, f_e, P_e, alpha = 0.01); §5.3 Adaptive
+ *     Capacity Factors (capacity_e = C * batch * seq / N_E).
+ *   "Zen-Max: Maximum Capability via Mixture-of-Experts Architecture": §2.2
+ *     Fine-Grained Expert Architecture (eq. Expert_i, SwiGLU; shared experts added
+ *     to the routed outputs); §2.3 Auxiliary-Loss-Free Load Balancing
+ *     (s_ij = softmax(x_i W_g)_j + b_j).
+ *   "Scaling with experts" (jeff-ong.com): "The gating network" (softmax over
+ *     the top-k logits, renormalised survivors, y = g1 E1(x) + g2 E2(x));
+ *     "A balance penalty"; "A budget" (capacity, dropped tokens skip the expert
+ *     and continue through the residual); "A shared expert".
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, row-major, densely packed, owned
+ *     by the caller.  The library never allocates or frees device memory and
+ *     keeps no state between calls; scratch space is the caller's workspace
+ *     `ws` of `ws_bytes` bytes (size from moe_workspace_size; 256-byte aligned).
+ *   - Every call only enqueues work on `stream` and returns; nothing
+ *     synchronises with the host (except moe_read_device_status).
+ *   - Activations and weights are BF16 (MOE_DTYPE_BF16) or FP32 (MOE_DTYPE_F32);
+ *     router logits, gate weights, offsets, biases and statistics are FP32.
+ *     BF16 math: BF16 operands, FP32 accumulation, one rounding per stored
+ *     intermediate (expert hidden activations, expert outputs, layer output).
+ *   - Weight storage ("linear [out, in]" rows):
+ *       w_gate [E, d]; w13 [E, 2F, d] (rows 0..F-1 gate proj, F..2F-1 up proj);
+ *       w2 [E, d, F]; shared: w13 [N_s, 2F, d], w2 [N_s, d, F].
+ *   - Alignment: every pointer 16-byte aligned; d_model and d_ff multiples of 8.
+ *   - Return value: MOE_OK (0) or a negative moe_status.  Arguments are checked
+ *     on the host before anything is enqueued; a rejected call enqueues nothing.
+ *     Kernels that find bad data (an expert index outside [0, E)) or give up a
+ *     bounded wait do not trap: they skip the access and set a bit in the
+ *     device status word at the start of `ws` (see moe_read_device_status).
+ *   - Thread safety: calls are independent; concurrent calls need distinct
+ *     workspaces.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,  /* bad shape, NULL pointer, misalignment, K > E, ... */
+    MOE_ERR_UNSUPPORTED = -2,  /* valid problem this build does not handle (e.g. E > 256) */
+    MOE_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
+    MOE_ERR_DEVICE_CHECK = -4, /* a kernel reported bad data (see moe_read_device_status) */
+    MOE_ERR_WORKSPACE = -5     /* ws too small or misaligned */
+} moe_status;
+
+typedef enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 } moe_dtype;
+
+/* moe_problem_t.flags */
+#define MOE_FLAG_LOGITS_GIVEN 0x1u /* moe_route / moe_layer_forward read the logits
+                                      instead of computing them from x and w_gate */
+#define MOE_FLAG_BIAS_LOGIT 0x2u   /* selection bias added to the logit, not to p */
+
+/* Device status bits (moe_read_device_status). */
+#define MOE_DEV_BAD_EXPERT 0x1     /* an expert index outside [0, E) was skipped */
+#define MOE_DEV_WAIT_TIMEOUT 0x2   /* a pipeline wait gave up; results invalid */
+
+/* The problem, in the pages' terms: T = batch * seq tokens of width d_model;
+ * E routed experts ("N_E"), top_k ("K"), n_shared always-on experts, each
+ * expert a SwiGLU of inner width d_ff; capacity factor C; alpha of the
+ * balance loss.  Limits of this build: 1 <= top_k <= min(E, 32); E <= 256;
+ * 1 <= T < 2^31 / max(E, top_k). */
+typedef struct moe_problem {
+    int64_t T;
+    int32_t d_model;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t n_shared;
+    int32_t d_ff;
+    float capacity_factor; /* <= 0: no capacity limit; else cap = ceil(C*T*K/E) */
+    int32_t dtype;         /* moe_dtype */
+    uint32_t flags;        /* MOE_FLAG_* */
+    float alpha;           /* balance-loss coefficient, e.g. 0.01 */
+} moe_problem_t;
+
+/* Weights of one layer (device pointers, layouts above). */
+typedef struct moe_weights {
+    const void* w_gate;        /* [E, d]; unused with MOE_FLAG_LOGITS_GIVEN */
+    const float* logit_offset; /* [E] additive logit offset, or NULL */
+    const float* sel_bias;     /* [E] selection-only bias, or NULL */
+    const void* w13;           /* [E, 2F, d] */
+    const void* w2;            /* [E, d, F] */
+    const void* w13_shared;    /* [N_s, 2F, d], NULL iff n_shared == 0 */
+    const void* w2_shared;     /* [N_s, d, F],  NULL iff n_shared == 0 */
+} moe_weights_t;
+
+/* Optional routing outputs of moe_layer_forward (device pointers; each may be
+ * NULL, in which case the array lives in the workspace).  `logits` is an INPUT
+ * when MOE_FLAG_LOGITS_GIVEN is set (then it must not be NULL). */
+typedef struct moe_routing {
+    float* logits;     /* [T, E] */
+    int32_t* topk_idx; /* [T, K] */
+    float* topk_w;     /* [T, K] */
+    int32_t* counts;   /* [E]   assignments per expert before the capacity cut */
+    int32_t* kept;     /* [E]   min(counts, cap) */
+    int32_t* seg_off;  /* [E+1] exclusive prefix sum of kept */
+    int32_t* slot_of;  /* [T, K] row of (t,k) in the expert-grouped arrays, or -1 if dropped */
+    int32_t* perm;     /* [moe_max_rows] perm[slot] = t*K + k for slot < seg_off[E] */
+} moe_routing_t;
+
+/* ABI version of the loaded library (MOE_ABI_VERSION). */
+int moe_abi_version(void);
+
+/* Human-readable name of a moe_status value (static string). */
+const char* moe_status_string(int code);
+
+/* Per-expert capacity of `p`: ceil(C * T * K / E) computed in float64 as
+ * (C * (T*K)) / E, or -1 when capacity_factor <= 0 (no limit).
+ * Zen MoDE §5.3 capacity_e, scaled by K for top-K routing.  Pure host
+ * function; returns -2 for a NULL or invalid problem. */
+int64_t moe_capacity(const moe_problem_t* p);
+
+/* Upper bound on kept (t,k) rows: min(T*K, E*cap) (T*K without a limit).
+ * Rows of perm / x_perm / y_perm.  Returns -2 for an invalid problem. */
+int64_t moe_max_rows(const moe_problem_t* p);
+
+/* Workspace bytes every entry point below needs for problem `p` (one size for
+ * all of them).  Pure host function. */
+int moe_workspace_size(const moe_problem_t* p, size_t* bytes);
+
+/* Zero the device status word at the start of `ws` (async on stream). */
+int moe_reset_device_status(void* ws, moe_stream_t stream);
+
+/* Synchronise `stream`, then copy the device status word into *bits.
+ * Returns MOE_ERR_DEVICE_CHECK if any bit is set, MOE_OK otherwise. */
+int moe_read_device_status(const void* ws, moe_stream_t stream, uint32_t* bits);
+
+/* Router.  Zen MoDE §3.1 eq. router_standard; Zen-Max §2.3 (selection bias);
+ * "Scaling with experts", The gating network / A balance penalty.
+ *   x            [T, d]  activations (ignored with MOE_FLAG_LOGITS_GIVEN)
+ *   w_gate       [E, d]  (ignored with MOE_FLAG_LOGITS_GIVEN)
+ *   logit_offset [E] or NULL: added to every token's logits
+ *   sel_bias     [E] or NULL: added to the selection score only
+ *                (to p, or to the logit with MOE_FLAG_BIAS_LOGIT)
+ *   logits       [T, E] fp32: output, or input with MOE_FLAG_LOGITS_GIVEN
+ *                (then already including any offset; logit_offset is ignored)
+ *   topk_idx     [T, K] out: chosen experts, best first; equal scores go to
+ *                the lower index.  Without a bias the score is the fp32 logit;
+ *                with a bias it is computed in float64.
+ *   topk_w       [T, K] out: renormalised gate weights (sum to 1 per token)
+ *   stats        [2E+1] out or NULL: f_e = counts_e / (T*K) (before the
+ *                capacity cut), P_e = mean_t p[t,e], loss = alpha*E*sum f_e P_e */
+int moe_route(const moe_problem_t* p, const void* x, const void* w_gate,
+              const float* logit_offset, const float* sel_bias, float* logits,
+              int32_t* topk_idx, float* topk_w, float* stats,
+              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Capacity-limited dispatch: group the (t,k) pairs by expert and gather rows.
+ * "Scaling with experts", A budget; Zen MoDE §5.3.
+ *   topk_idx [T, K] in (an index outside [0, E) is skipped and flagged)
+ *   x        [T, d] in
+ *   counts [E], kept [E], seg_off [E+1], slot_of [T, K], perm [moe_max_rows] out
+ *            (definitions in moe_routing_t; rank of (t,k) within its expert =
+ *            number of earlier tokens that chose the same expert; kept iff
+ *            rank < cap; slot = seg_off[e] + rank; perm entries past
+ *            seg_off[E] are left untouched)
+ *   x_perm   [moe_max_rows, d] out: x_perm[slot] = x[perm[slot] / K] for
+ *            slot < seg_off[E]; later rows untouched.  May be NULL (no gather). */
+int moe_dispatch(const moe_problem_t* p, const int32_t* topk_idx, const void* x,
+                 int32_t* counts, int32_t* kept, int32_t* seg_off,
+                 int32_t* slot_of, int32_t* perm, void* x_perm,
+                 void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Expert SwiGLU FFNs (Zen-Max §2.2 eq. Expert_i).
+ * mode MOE_FFN_ROUTED: x_rows [n_rows, d] grouped by expert; rows
+ *   seg_off[e] .. seg_off[e+1]-1 go through expert e (w13 [E,2F,d],
+ *   w2 [E,d,F]); y_rows [n_rows, d]; rows >= seg_off[E] untouched.
+ *   n_rows is the allocated row count (>= seg_off[E], <= moe_max_rows).
+ * mode MOE_FFN_SHARED: every row goes through all n_shared experts
+ *   (w13 [N_s,2F,d], w2 [N_s,d,F]) and the outputs are summed, unweighted
+ *   ("Scaling with experts", A shared expert); seg_off is ignored;
+ *   1 <= n_rows <= T. */
+#define MOE_FFN_ROUTED 0
+#define MOE_FFN_SHARED 1
+int moe_expert_ffn(const moe_problem_t* p, int32_t mode, const void* x_rows, int64_t n_rows,
+                   const int32_t* seg_off, const void* w13, const void* w2, void* y_rows,
+                   void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Gate-weighted combine back to token order ("Scaling with experts", The
+ * gating network: y = g1 E1(x) + g2 E2(x); A budget: dropped pairs add 0).
+ *   y[t] = y_shared[t] + sum_{k: slot_of[t,k] >= 0} topk_w[t,k] * y_perm[slot_of[t,k]]
+ * summed in fp32 in that order (shared first, then k ascending), rounded once.
+ *   y_perm [*, d]; slot_of [T, K]; topk_w [T, K]; y_shared [T, d] or NULL
+ *   (required iff n_shared > 0); y [T, d] out. */
+int moe_combine(const moe_problem_t* p, const void* y_perm, const int32_t* slot_of,
+                const float* topk_w, const void* y_shared, void* y,
+                void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* The whole layer: route -> dispatch -> routed experts -> shared experts ->
+ * combine, plus statistics, enqueued on one stream with no host sync.
+ *   x [T, d] in; w weights; y [T, d] out;
+ *   routing: optional outputs (NULL or any subset; logits is an input with
+ *   MOE_FLAG_LOGITS_GIVEN); stats [2E+1] or NULL (as moe_route).
+ * Resets the device status word first. */
+int moe_layer_forward(const moe_problem_t* p, const void* x, const moe_weights_t* w,
+                      void* y, const moe_routing_t* routing, float* stats,
+                      void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Stage boundaries recorded by moe_layer_forward_profiled. */
+#define MOE_EV_START 0   /* before the router */
+#define MOE_EV_ROUTED 1  /* after gate logits, selection and statistics */
+#define MOE_EV_DISPATCHED 2 /* after histogram, scan, rank and gather */
+#define MOE_EV_UP 3      /* after the routed up/gate projection with SwiGLU */
+#define MOE_EV_DOWN 4    /* after the routed down projection */
+#define MOE_EV_SHARED 5  /* after the shared experts */
+#define MOE_EV_END 6     /* after the combine */
+#define MOE_NUM_EVENTS 7
+
+/* moe_layer_forward, instrumented: additionally records events[i]
+ * (cudaEvent_t handles the caller created on the stream's device; NULL
+ * entries are skipped) on `stream` at the MOE_EV_* boundaries, so that the
+ * time between two events is the time of that stage's kernels.  Stages that
+ * do not run for this problem record their event at the same point as the
+ * previous one.  *n_kernels (if not NULL) receives the number of kernels the
+ * call enqueued.  Same arguments, results and errors as moe_layer_forward. */
+int moe_layer_forward_profiled(const moe_problem_t* p, const void* x, const moe_weights_t* w,
+                               void* y, const moe_routing_t* routing, float* stats,
+                               void* ws, size_t ws_bytes, moe_stream_t stream,
+                               void* const* events, int32_t* n_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -17,6 +17,7 @@ Parity pins (what ties each function to something other than itself) are in
   capacity       exact integer cases printed in the configs' arithmetic
   dispatch       brute force per-expert queues; bijection and order invariants
   swiglu         one-hot weights reduce each output to silu(a) * b closed form
+  combine        grouped SwiGLU outputs combined equal layer_rows; hand example
   layer_rows     E=1, K=1 reduces to one dense SwiGLU; shared experts equal one
                  SwiGLU of concatenated width; dropped pairs contribute nothing
   balance        uniform routing gives exactly alpha
@@ -75,6 +76,8 @@ def _L():
         lib.oracle_layer_rows.argtypes = [i64, i32, i32, i32, i32, i32, P, i32, P, P, P, P, i32,
                                           P, P, P, i64, P, P]
         lib.oracle_layer_rows.restype = ctypes.c_int
+        lib.oracle_combine.argtypes = [i64, i32, i32, P, i32, P, P, P, i32, P]
+        lib.oracle_combine.restype = None
         lib.oracle_balance.argtypes = [i64, i32, i32, P, P, f64, P, P, P]
         lib.oracle_balance.restype = None
         lib.oracle_router_zloss.argtypes = [i64, i32, P]
@@ -224,6 +227,24 @@ def layer_rows(x, w13, w2, idx, w, slot_of, rows=None, w13_shared=None, w2_share
                                 _ptr(ia), _ptr(wa), _ptr(sa), r.shape[0], _ptr(r), _ptr(y))
     if rc != 0:
         raise ValueError("token or expert index out of range")
+    return y
+
+
+def combine(y_perm, slot_of, w, y_shared=None):
+    """y[t] = y_shared[t] + sum over kept k of w[t,k] * y_perm[slot_of[t,k]]
+    ("Scaling with experts", The gating network / A budget / A shared expert).
+    Returns float64 [T, d]."""
+    ya, ydt = _as_input(y_perm)
+    sa = np.ascontiguousarray(slot_of, dtype=np.int32)
+    wa = np.ascontiguousarray(w, dtype=np.float64)
+    T, K = sa.shape
+    d = ya.shape[1]
+    if y_shared is not None:
+        sh, sdt = _as_input(y_shared)
+    else:
+        sh, sdt = None, F64
+    y = np.empty((T, d), np.float64)
+    _L().oracle_combine(T, d, K, _ptr(ya), ydt, _ptr(sa), _ptr(wa), _ptr(sh), sdt, _ptr(y))
     return y
 
 

@@ -288,6 +288,29 @@ int oracle_layer_rows(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int
 }
 
 /* ---------------------------------------------------------------------------
+ * Combine expert-grouped outputs back to token order ([SE] "The gating
+ * network": y = g1 Expert1(x) + g2 Expert2(x); "A budget": dropped pairs add
+ * nothing; shared-expert output added unweighted):
+ *   y[t, i] = y_shared[t, i] + sum_{k : slot_of[t,k] >= 0} w[t,k] * y_perm[slot_of[t,k], i]
+ * y_perm rows and y_shared are inputs of any element type; y_shared may be NULL.
+ * ------------------------------------------------------------------------- */
+void oracle_combine(int64_t T, int32_t d, int32_t K,
+                    const void* y_perm, int32_t yp_dt, const int32_t* slot_of, const double* w,
+                    const void* y_shared, int32_t ys_dt, double* y) {
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t i = 0; i < d; ++i) {
+            double acc = y_shared ? ld(y_shared, ys_dt, t * d + i) : 0.0;
+            for (int32_t k = 0; k < K; ++k) {
+                int32_t slot = slot_of[t * K + k];
+                if (slot < 0) continue;
+                acc += w[t * K + k] * ld(y_perm, yp_dt, (int64_t)slot * d + i);
+            }
+            y[t * d + i] = acc;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * Switch balance statistics.  [ZM] §5.2 eq. L_balance and [SE] "A balance
  * penalty":  L = alpha * N * sum_e f_e P_e, with
  *   f_e = counts[e] / (T*K)   fraction of the batch's assignments sent to e

@@ -1,0 +1,137 @@
+"""Python binding of the C ABI, with the same entry-point names.
+
+Argument marshalling only: every function passes torch device tensors' data
+pointers (and the current CUDA stream) to libmoe_b200.so and raises MoeError
+on a non-zero status.  No step of the layer is computed here.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (DTYPE_BF16, DTYPE_F32, FFN_ROUTED, FFN_SHARED, FLAG_BIAS_LOGIT, FLAG_LOGITS_GIVEN, MoeError,
+                   MoeProblem, MoeRouting, MoeWeights)
+
+__all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
+           "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+           "moe_layer_forward_profiled",
+           "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
+           "FFN_ROUTED", "FFN_SHARED", "DTYPE_BF16", "DTYPE_F32"]
+
+
+def make_problem(T, d_model, n_experts, top_k, d_ff, n_shared=0, capacity_factor=0.0, dtype="bf16", flags=0,
+                 alpha=0.01) -> MoeProblem:
+    dt = {"bf16": DTYPE_BF16, "f32": DTYPE_F32, DTYPE_BF16: DTYPE_BF16, DTYPE_F32: DTYPE_F32}[dtype]
+    return MoeProblem(int(T), int(d_model), int(n_experts), int(top_k), int(n_shared), int(d_ff),
+                      float(capacity_factor), dt, int(flags), float(alpha))
+
+
+def _p(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def workspace_size(prob: MoeProblem) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check("moe_workspace_size", _lib.lib().moe_workspace_size(ctypes.byref(prob), ctypes.byref(n)))
+    return int(n.value)
+
+
+def capacity(prob: MoeProblem) -> int:
+    return int(_lib.lib().moe_capacity(ctypes.byref(prob)))
+
+
+def max_rows(prob: MoeProblem) -> int:
+    return int(_lib.lib().moe_max_rows(ctypes.byref(prob)))
+
+
+def alloc_workspace(prob: MoeProblem, device="cuda") -> torch.Tensor:
+    """A caller-owned workspace (torch's allocator returns 256-byte aligned blocks)."""
+    return torch.empty(workspace_size(prob), dtype=torch.uint8, device=device)
+
+
+def reset_device_status(ws: torch.Tensor, stream=None) -> None:
+    _lib.check("moe_reset_device_status", _lib.lib().moe_reset_device_status(_p(ws), _stream(stream)))
+
+
+def read_device_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream; returns the device status bits (0 = clean)."""
+    bits = ctypes.c_uint32(0)
+    rc = _lib.lib().moe_read_device_status(_p(ws), _stream(stream), ctypes.byref(bits))
+    if rc not in (0, -4):
+        raise MoeError("moe_read_device_status", rc)
+    return int(bits.value)
+
+
+def moe_route(prob, x, w_gate, logit_offset, sel_bias, logits, topk_idx, topk_w, stats, ws, stream=None):
+    rc = _lib.lib().moe_route(ctypes.byref(prob), _p(x), _p(w_gate), _p(logit_offset), _p(sel_bias), _p(logits),
+                              _p(topk_idx), _p(topk_w), _p(stats), _p(ws), ws.numel(), _stream(stream))
+    _lib.check("moe_route", rc)
+
+
+def moe_dispatch(prob, topk_idx, x, counts, kept, seg_off, slot_of, perm, x_perm, ws, stream=None):
+    rc = _lib.lib().moe_dispatch(ctypes.byref(prob), _p(topk_idx), _p(x), _p(counts), _p(kept), _p(seg_off),
+                                 _p(slot_of), _p(perm), _p(x_perm), _p(ws), ws.numel(), _stream(stream))
+    _lib.check("moe_dispatch", rc)
+
+
+def moe_expert_ffn(prob, mode, x_rows, n_rows, seg_off, w13, w2, y_rows, ws, stream=None):
+    rc = _lib.lib().moe_expert_ffn(ctypes.byref(prob), int(mode), _p(x_rows), int(n_rows), _p(seg_off), _p(w13),
+                                   _p(w2), _p(y_rows), _p(ws), ws.numel(), _stream(stream))
+    _lib.check("moe_expert_ffn", rc)
+
+
+def moe_combine(prob, y_perm, slot_of, topk_w, y_shared, y, ws, stream=None):
+    rc = _lib.lib().moe_combine(ctypes.byref(prob), _p(y_perm), _p(slot_of), _p(topk_w), _p(y_shared), _p(y),
+                                _p(ws), ws.numel(), _stream(stream))
+    _lib.check("moe_combine", rc)
+
+
+def _weights_struct(w: dict) -> MoeWeights:
+    return MoeWeights(_p(w.get("w_gate")), _p(w.get("logit_offset")), _p(w.get("sel_bias")), _p(w["w13"]),
+                      _p(w["w2"]), _p(w.get("w13_shared")), _p(w.get("w2_shared")))
+
+
+def _routing_struct(r: dict | None) -> MoeRouting | None:
+    if r is None:
+        return None
+    return MoeRouting(_p(r.get("logits")), _p(r.get("topk_idx")), _p(r.get("topk_w")), _p(r.get("counts")),
+                      _p(r.get("kept")), _p(r.get("seg_off")), _p(r.get("slot_of")), _p(r.get("perm")))
+
+
+def moe_layer_forward(prob, x, weights: dict, y, routing: dict | None, stats, ws, stream=None):
+    w = _weights_struct(weights)
+    r = _routing_struct(routing)
+    rc = _lib.lib().moe_layer_forward(ctypes.byref(prob), _p(x), ctypes.byref(w), _p(y),
+                                      ctypes.byref(r) if r is not None else None, _p(stats), _p(ws), ws.numel(),
+                                      _stream(stream))
+    _lib.check("moe_layer_forward", rc)
+
+
+def moe_layer_forward_profiled(prob, x, weights: dict, y, routing: dict | None, stats, ws, events, stream=None) -> int:
+    """moe_layer_forward that also records `events` (7 torch.cuda.Event, or None
+    entries) at the stage boundaries; returns the number of kernels enqueued."""
+    w = _weights_struct(weights)
+    r = _routing_struct(routing)
+    handles = (ctypes.c_void_p * _lib.NUM_EVENTS)()
+    for i, ev in enumerate(events):
+        handles[i] = None if ev is None else ev.cuda_event
+    n = ctypes.c_int32(0)
+    rc = _lib.lib().moe_layer_forward_profiled(ctypes.byref(prob), _p(x), ctypes.byref(w), _p(y),
+                                               ctypes.byref(r) if r is not None else None, _p(stats), _p(ws),
+                                               ws.numel(), _stream(stream), handles, ctypes.byref(n))
+    _lib.check("moe_layer_forward_profiled", rc)
+    return int(n.value)

@@ -1,0 +1,102 @@
+// Gate-weighted combine back to token order.
+//
+//   Scaling with experts, "The gating network": y = g1 * Expert1(x) + g2 * Expert2(x)
+//   with g the renormalised gate weights; "A budget": a dropped pair adds
+//   nothing; "A shared expert" / Zen-Max §2.2: shared experts are added unweighted.
+//
+//   y[t] = y_shared[t] + sum_{k : slot_of[t,k] >= 0} w[t,k] * y_perm[slot_of[t,k]]
+// accumulated in fp32 in that order (shared first, then k ascending) and
+// rounded once.  One warp per token, 16-byte vectors along d.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+template <typename T>
+struct Pack16;
+template <>
+struct Pack16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const void* p, float (&v)[8]) {
+    const uint4 q = *static_cast<const uint4*>(p);
+    v[0] = bf16_lo(q.x); v[1] = bf16_hi(q.x); v[2] = bf16_lo(q.y); v[3] = bf16_hi(q.y);
+    v[4] = bf16_lo(q.z); v[5] = bf16_hi(q.z); v[6] = bf16_lo(q.w); v[7] = bf16_hi(q.w);
+  }
+  __device__ static void store(void* p, const float (&v)[8]) {
+    uint4 q;
+    q.x = pack_bf16x2(v[0], v[1]); q.y = pack_bf16x2(v[2], v[3]);
+    q.z = pack_bf16x2(v[4], v[5]); q.w = pack_bf16x2(v[6], v[7]);
+    *static_cast<uint4*>(p) = q;
+  }
+};
+template <>
+struct Pack16<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const void* p, float (&v)[4]) {
+    const float4 q = *static_cast<const float4*>(p);
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  __device__ static void store(void* p, const float (&v)[4]) {
+    *static_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ slot_of,
+                                                      const float* __restrict__ topk_w,
+                                                      const T* __restrict__ y_shared, T* __restrict__ y,
+                                                      int64_t Tn, int d, int K, int64_t n_perm_rows) {
+  constexpr int V = Pack16<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int nvec = d / V;
+  for (int64_t t = warp0; t < Tn; t += n_warps) {
+    // lane k holds (slot, weight) of pair k
+    int my_slot = -1;
+    float my_w = 0.f;
+    if (lane < K) {
+      my_slot = slot_of[t * K + lane];
+      my_w = topk_w[t * K + lane];
+    }
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[V];
+      if (y_shared) {
+        Pack16<T>::load(y_shared + t * d + v * V, acc);
+      } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] = 0.f;
+      }
+      for (int k = 0; k < K; ++k) {
+        const int slot = __shfl_sync(0xffffffffu, my_slot, k);
+        const float w = __shfl_sync(0xffffffffu, my_w, k);
+        if (slot >= 0 && slot < n_perm_rows) {
+          float r[V];
+          Pack16<T>::load(y_perm + static_cast<int64_t>(slot) * d + v * V, r);
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[i] = fmaf(w, r[i], acc[i]);
+        }
+      }
+      Pack16<T>::store(y + t * d + v * V, acc);
+    }
+  }
+}
+
+cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
+                           const void* y_shared, void* y, cudaStream_t st) {
+  int64_t blocks = (p.T + 7) / 8;
+  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  if (p.dtype == kBF16)
+    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(y_perm), slot_of, topk_w, static_cast<const __nv_bfloat16*>(y_shared),
+        static_cast<__nv_bfloat16*>(y), p.T, p.d, p.K, p.max_rows);
+  else
+    combine_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const float*>(y_perm), slot_of, topk_w, static_cast<const float*>(y_shared),
+        static_cast<float*>(y), p.T, p.d, p.K, p.max_rows);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,213 @@
+// Capacity-limited dispatch: group the (token, k) assignments by expert.
+//
+//   Scaling with experts, "A budget": each expert takes a limited number of
+//   tokens per batch; tokens past the budget are dropped (the expert update is
+//   skipped; the token continues through the residual).
+//   Zen MoDE, §5.3 Adaptive Capacity Factors: capacity_e = C * batch*seq / N_E
+//   (scaled here by K for top-K routing).
+//
+// Order: first come, first served in token order.  rank(t,k) = number of tokens
+// t' < t that chose the same expert; (t,k) is kept iff rank < cap.  The result
+// is independent of thread scheduling: ranks are counted, never claimed by
+// racing atomics.
+//
+// Kernels (all multi-pass, no CTA waits on another):
+//   1. hist  : per 256-token chunk, per-expert counts
+//   2. scan  : per expert, exclusive prefix over chunks; totals, kept, seg_off
+//   3. rank  : per chunk, each warp builds a lane mask per expert (which of its
+//              32 tokens chose it); rank = chunk base + earlier warps' counts +
+//              popcount of the lower lanes' bits
+//   4. gather: x_perm[slot] = x[perm[slot] / K]
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) dispatch_hist_kernel(const int32_t* __restrict__ idx, int64_t T, int K,
+                                                            int E, int32_t* __restrict__ chunk_counts,
+                                                            unsigned* status) {
+  __shared__ int hist[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t begin = static_cast<int64_t>(blockIdx.x) * kDispatchChunk * K;
+  int64_t end = begin + static_cast<int64_t>(kDispatchChunk) * K;
+  if (end > T * K) end = T * K;
+  for (int64_t i = begin + threadIdx.x; i < end; i += blockDim.x) {
+    const int e = idx[i];
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E))
+      atomicAdd(&hist[e], 1);
+    else
+      raise_status(status, kDevBadExpert);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// One block of 1024 threads.  Thread (e, s) owns a contiguous run of chunks
+// for expert e; runs are summed, scanned per expert, then re-walked to write
+// each chunk's base.
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts,
+                                                             int n_chunks, int E, long long cap,
+                                                             int32_t* __restrict__ chunk_base,
+                                                             int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ kept,
+                                                             int32_t* __restrict__ seg_off) {
+  __shared__ int part[1024];
+  __shared__ int s_kept[kMaxExperts];
+  int S = 1024 / E;
+  if (S > n_chunks) S = n_chunks;
+  if (S < 1) S = 1;
+  const int per = (n_chunks + S - 1) / S;
+  const int tid = threadIdx.x;
+  const int e = tid / S;
+  const int s = tid - e * S;
+  const bool active = e < E;
+  int c0 = s * per, c1 = c0 + per;
+  if (c1 > n_chunks) c1 = n_chunks;
+  int local = 0;
+  if (active)
+    for (int c = c0; c < c1; ++c) local += chunk_counts[static_cast<int64_t>(c) * E + e];
+  part[tid] = local;
+  __syncthreads();
+  if (active && s == 0) {
+    int run = 0;
+    for (int i = 0; i < S; ++i) {
+      const int v = part[tid + i];
+      part[tid + i] = run;
+      run += v;
+    }
+    counts[e] = run;
+    const int k = (cap < 0 || run < cap) ? run : static_cast<int>(cap);
+    kept[e] = k;
+    s_kept[e] = k;
+  }
+  __syncthreads();
+  if (active) {
+    int run = part[tid];
+    for (int c = c0; c < c1; ++c) {
+      chunk_base[static_cast<int64_t>(c) * E + e] = run;
+      run += chunk_counts[static_cast<int64_t>(c) * E + e];
+    }
+  }
+  // seg_off = exclusive prefix of kept over experts (warp 0; 8 experts per lane)
+  if (tid < 32) {
+    constexpr int kPer = kMaxExperts / 32;
+    int v[kPer];
+    int loc = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int ee = tid * kPer + i;
+      v[i] = ee < E ? s_kept[ee] : 0;
+      loc += v[i];
+    }
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (tid >= o) incl += y;
+    }
+    int run = incl - loc;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int ee = tid * kPer + i;
+      if (ee < E) seg_off[ee] = run;
+      run += v[i];
+    }
+    if (tid == 31) seg_off[E] = incl;
+  }
+}
+
+__global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __restrict__ idx, int64_t T, int K,
+                                                            int E, const int32_t* __restrict__ chunk_base,
+                                                            const int32_t* __restrict__ kept,
+                                                            const int32_t* __restrict__ seg_off,
+                                                            int32_t* __restrict__ slot_of,
+                                                            int32_t* __restrict__ perm) {
+  __shared__ uint32_t mask[8][kMaxExperts];
+  __shared__ int wbase[8][kMaxExperts];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) mask[i / E][i % E] = 0u;
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchChunk + warp * 32 + lane;
+  const bool tok_ok = t < T;
+  if (tok_ok) {
+    for (int k = 0; k < K; ++k) {
+      const int e = idx[t * K + k];
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicOr(&mask[warp][e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = chunk_base[static_cast<int64_t>(blockIdx.x) * E + e];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w][e] = run;
+      run += __popc(mask[w][e]);
+    }
+  }
+  __syncthreads();
+  if (tok_ok) {
+    const uint32_t lower = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int64_t pair = t * K + k;
+      const int e = idx[pair];
+      int slot = -1;
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+        const int rank = wbase[warp][e] + __popc(mask[warp][e] & lower);
+        if (rank < kept[e]) {
+          slot = seg_off[e] + rank;
+          perm[slot] = static_cast<int32_t>(pair);
+        }
+      }
+      slot_of[pair] = slot;
+    }
+  }
+}
+
+cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* counts, int32_t* kept,
+                            int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
+                            int32_t* chunk_base, unsigned* status, cudaStream_t st) {
+  const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
+  dispatch_hist_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_counts, status);
+  dispatch_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, n_chunks, p.E, static_cast<long long>(p.cap),
+                                           chunk_base, counts, kept, seg_off);
+  dispatch_rank_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_base, kept, seg_off, slot_of, perm);
+  return cudaGetLastError();
+}
+
+// Row gather: one warp per destination row, 16-byte vectors.  Rows at or past
+// seg_off[E] (the kept total) are left untouched.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                          const int32_t* __restrict__ perm,
+                                                          const int32_t* __restrict__ seg_off, int E, int K,
+                                                          int64_t T, int vec_per_row, int64_t max_rows,
+                                                          uint4* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n_rows = seg_off[E];
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t r = warp0; r < n_rows && r < max_rows; r += n_warps) {
+    const int64_t tok = perm[r] / K;
+    if (tok < 0 || tok >= T) continue;
+    const uint4* src = x + tok * vec_per_row;
+    uint4* dst = x_perm + r * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+  }
+}
+
+cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
+                          void* x_perm, cudaStream_t st) {
+  if (p.max_rows <= 0) return cudaSuccess;
+  const int vec_per_row = static_cast<int>(p.d * p.esize() / 16);
+  int64_t blocks = (p.max_rows + 7) / 8;
+  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const uint4*>(x), perm, seg_off, p.E, p.K, p.T, vec_per_row, p.max_rows,
+      static_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,639 @@
+// Expert FFNs: grouped GEMMs on the 5th-generation tensor cores (tcgen05.mma,
+// accumulators in TMEM, operands staged by TMA), with SwiGLU fused into the
+// epilogue of the up/gate projection.
+//
+//   Zen-Max: Maximum Capability via Mixture-of-Experts Architecture, §2.2
+//   Fine-Grained Expert Architecture, eq. Expert_i:
+//       Expert_i(x) = (SiLU(x W_gate,i) (.) x W_up,i) W_down,i
+//   Shared experts (always active) are added to the routed outputs
+//   (same section; Scaling with experts, "A shared expert").
+//
+// One kernel template, three epilogues:
+//   EPI_SWIGLU : H[r, n] = silu(A W_gate^T)[r, n] * (A W_up^T)[r, n]   (BF16 out)
+//                the B tile stacks 128 gate rows over 128 up rows, so one
+//                M=128 x N=256 MMA chain yields both halves for the same n.
+//   EPI_BF16   : Y = A W_down^T                                          (BF16 out)
+//   EPI_F32    : logits = A W_g^T + offset                               (FP32 out)
+//
+// Work decomposition: a "group" is a block of A rows that shares one B
+// matrix (an expert).  Routed groups are the expert segments of the
+// expert-grouped rows [seg_off[g], seg_off[g+1]) (read on the device, so no
+// host sync); shared groups all cover rows [0, n_rows).  Tiles are 128 rows x
+// (128 or 256) columns, enumerated group-major, then column tile, then row
+// tile, so CTAs running at the same time share weight tiles through L2.
+// Persistent CTAs (one per SM) walk the tile list with a stride of the grid.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring of
+// shared-memory stages; warp 1 allocates TMEM and issues the MMAs from one
+// thread; warps 2-5 drain the TMEM accumulator (double-buffered, so the
+// epilogue of tile i overlaps the main loop of tile i+1) and store.
+// Every wait is bounded (see mbar_wait); on a timeout the kernel records
+// MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+enum { EPI_SWIGLU = 0, EPI_BF16 = 1, EPI_F32 = 2 };
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // 64 BF16 = 128 bytes: one 128-byte swizzle row
+constexpr int kGemmThreads = 192;
+constexpr int kMaxGroups = 256;
+
+struct GemmArgs {
+  int n_groups;
+  const int32_t* seg_off;  // [n_groups + 1] row offsets, or nullptr: every group covers [0, n_rows)
+  int n_rows;
+  int N;               // valid output columns of one group
+  int K;               // valid reduction length of one B matrix
+  int k_groups;        // B matrices summed along the reduction (A row holds k_groups * K)
+  void* out;
+  int64_t ldo;         // output row stride, elements
+  int out_col_stride;  // output column offset per group
+  const float* col_add;  // EPI_F32: per-column offset, or nullptr
+  unsigned* status;
+};
+
+template <int EPI, int BN>
+struct TileCfg {
+  static constexpr int kOutCols = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                   : (2 * BN <= 256) ? 256 : 512;
+};
+
+template <int EPI, int BN, int STAGES>
+constexpr int gemm_smem_bytes() {
+  return STAGES * TileCfg<EPI, BN>::kStageBytes + 256 /*barriers + flags*/ + 4 * (kMaxGroups + 1) +
+         1024 /*alignment slack*/;
+}
+
+struct TileInfo {
+  int g, row0, row_end, n0;
+};
+
+// Rows [base, base + return) of group g, clamped to the allocated rows
+// [0, n_rows) whatever seg_off holds, so no tile reads or writes outside them.
+__device__ __forceinline__ int group_rows(const GemmArgs& a, int g, int* base) {
+  if (a.seg_off) {
+    const int b = min(max(a.seg_off[g], 0), a.n_rows);
+    const int e = min(max(a.seg_off[g + 1], b), a.n_rows);
+    *base = b;
+    return e - b;
+  }
+  *base = 0;
+  return a.n_rows;
+}
+
+__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const GemmArgs& a, int n_tiles_n,
+                                                int out_cols) {
+  int lo = 0, hi = a.n_groups - 1;
+  while (lo < hi) {  // largest g with prefix[g] <= tile (that group is never empty)
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.g = lo;
+  int base;
+  const int rows = group_rows(a, lo, &base);
+  const int mt = (rows + kBM - 1) / kBM;
+  const int local = tile - prefix[lo];
+  const int n_idx = local / mt;
+  const int m_idx = local - n_idx * mt;
+  ti.row0 = base + m_idx * kBM;
+  ti.row_end = base + rows;
+  ti.n0 = n_idx * out_cols;
+  (void)n_tiles_n;
+  return ti;
+}
+
+template <int EPI, int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const GemmArgs args) {
+  using C = TileCfg<EPI, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::kBBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tiles_n = (args.N + C::kOutCols - 1) / C::kOutCols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    // tile prefix over groups: lane l owns groups [l*per, (l+1)*per)
+    const int per = (args.n_groups + 31) / 32;
+    int local = 0;
+    for (int i = 0; i < per; ++i) {
+      const int g = lane * per + i;
+      if (g < args.n_groups) {
+        int base;
+        const int rows = group_rows(args, g, &base);
+        local += ((rows + kBM - 1) / kBM) * n_tiles_n;
+      }
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int i = 0; i < per; ++i) {
+      const int g = lane * per + i;
+      if (g < args.n_groups) {
+        prefix[g] = run;
+        int base;
+        const int rows = group_rows(args, g, &base);
+        run += ((rows + kBM - 1) / kBM) * n_tiles_n;
+      }
+    }
+    if (lane == 31) prefix[args.n_groups] = incl;
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = prefix[args.n_groups];
+  const int nkb_g = (args.K + kBK - 1) / kBK;
+  const int nkb = nkb_g * args.k_groups;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(tile, prefix, args, n_tiles_n, C::kOutCols);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int kg = kb / nkb_g;
+          const int kk = (kb - kg * nkb_g) * kBK;
+          uint8_t* a_dst = sA + stage * C::kABytes;
+          uint8_t* b_dst = sB + stage * C::kBBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(a_dst, &tmA, &full[stage], kg * args.K + kk, ti.row0);
+          if (EPI == EPI_SWIGLU) {
+            tma_load_3d(b_dst, &tmB, &full[stage], kk, ti.n0, 2 * ti.g);
+            tma_load_3d(b_dst + C::kBBytes / 2, &tmB, &full[stage], kk, ti.n0, 2 * ti.g + 1);
+          } else if (EPI == EPI_BF16) {
+            tma_load_3d(b_dst, &tmB, &full[stage], kk, ti.n0, ti.g * args.k_groups + kg);
+          } else {
+            tma_load_3d(b_dst, &tmB, &full[stage], kk, 0, 0);
+          }
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {  // let every copy this thread started land before exit
+        int never = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if ((issued >> s) & 1u) mbar_wait(&full[s], (last_par >> s) & 1u, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint64_t adesc = smem_desc_k128(smem_addr(sA + stage * C::kABytes));
+          const uint64_t bdesc = smem_desc_k128(smem_addr(sB + stage * C::kBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)  // advance 16 elements = 32 bytes = 2 descriptor units
+            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      if (*abort_flag) {  // wait for every MMA this thread issued before TMEM is freed
+        umma_commit(drain);
+        int never = 0;
+        mbar_wait(drain, 0, &never);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter+32) are this warp's
+    const int r = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile(tile, prefix, args, n_tiles_n, C::kOutCols);
+      const int acc = it & 1;
+      const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+      // every lane waits; the result is made warp-uniform (and the warp
+      // reconverged) before the .sync.aligned TMEM loads below
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_par, abort_flag));
+      if (!ready) break;
+      tc_fence_after_sync();
+      const int row = ti.row0 + r;
+      const bool row_ok = row < ti.row_end;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      if (EPI == EPI_SWIGLU) {
+        __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
+                                 static_cast<int64_t>(ti.g) * args.out_col_stride;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t gr[32], ur[32];
+          tmem_load_32x32(t_row + c, gr);
+          tmem_load_32x32(t_row + BN / 2 + c, ur);
+          tmem_load_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = ti.n0 + c + q * 8;
+              if (col < args.N) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float g0 = __uint_as_float(gr[q * 8 + 2 * j]), g1 = __uint_as_float(gr[q * 8 + 2 * j + 1]);
+                  const float u0 = __uint_as_float(ur[q * 8 + 2 * j]), u1 = __uint_as_float(ur[q * 8 + 2 * j + 1]);
+                  const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                  const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                  pk[j] = pack_bf16x2(h0, h1);
+                }
+                *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          }
+        }
+      } else if (EPI == EPI_BF16) {
+        __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
+                                 static_cast<int64_t>(ti.g) * args.out_col_stride;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t vr[32];
+          tmem_load_32x32(t_row + c, vr);
+          tmem_load_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int col = ti.n0 + c + q * 8;
+              if (col < args.N) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  pk[j] = pack_bf16x2(__uint_as_float(vr[q * 8 + 2 * j]), __uint_as_float(vr[q * 8 + 2 * j + 1]));
+                *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              }
+            }
+          }
+        }
+      } else {
+        float* out_row = static_cast<float*>(args.out) + static_cast<int64_t>(row) * args.ldo;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t vr[32];
+          tmem_load_32x32(t_row + c, vr);
+          tmem_load_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int col = c + j;
+              if (col < args.N)
+                out_row[col] = __uint_as_float(vr[j]) + (args.col_add ? args.col_add[col] : 0.f);
+            }
+          }
+        }
+      }
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) raise_status(args.status, kDevWaitTimeout);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ============================================================================
+// Host side: tensor maps and launches.
+// ============================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// BF16 tensor map: dims[0] innermost (contiguous), 128-byte swizzle, zero fill
+// out of bounds.  Box inner extent is always 64 elements (128 bytes).
+static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3], gstr[2];
+  cuuint32_t bdim[3], estr[3] = {1, 1, 1};
+  uint64_t stride = 2;
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    if (i > 0) gstr[i - 1] = stride;
+    stride *= dims[i];
+  }
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gdim, gstr, bdim, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, int BN, int STAGES>
+static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int64_t tile_bound,
+                    cudaStream_t st) {
+  constexpr int smem = gemm_smem_bytes<EPI, BN, STAGES>();
+  // the dynamic shared-memory opt-in is per device: set it once per device
+  static std::mutex mu;
+  static uint64_t done = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!((done >> dev) & 1u)) {
+      if (cudaFuncSetAttribute(grouped_gemm_tc_kernel<EPI, BN, STAGES>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return -3;
+      done |= uint64_t(1) << dev;
+    }
+  }
+  if (tile_bound <= 0) return 0;
+  int64_t grid = num_sms();
+  if (grid > tile_bound) grid = tile_bound;
+  grouped_gemm_tc_kernel<EPI, BN, STAGES><<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(ta, tb, a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset,
+                          float* logits, unsigned* status, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.T)};
+  const uint32_t ba[2] = {kBK, kBM};
+  if (!make_map(&ta, x, 2, da, ba)) return -3;
+  const int bn = p.E <= 32 ? 32 : p.E <= 64 ? 64 : p.E <= 128 ? 128 : 256;
+  const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.E), 1};
+  const uint32_t bb[3] = {kBK, static_cast<uint32_t>(bn), 1};
+  if (!make_map(&tb, w_gate, 3, db, bb)) return -3;
+  GemmArgs a{};
+  a.n_groups = 1;
+  a.seg_off = nullptr;
+  a.n_rows = static_cast<int>(p.T);
+  a.N = p.E;
+  a.K = p.d;
+  a.k_groups = 1;
+  a.out = logits;
+  a.ldo = p.E;
+  a.out_col_stride = 0;
+  a.col_add = offset;
+  a.status = status;
+  const int64_t tiles = cdiv(p.T, kBM);
+  switch (bn) {
+    case 32: return run_gemm<EPI_F32, 32, 8>(ta, tb, a, tiles, st);
+    case 64: return run_gemm<EPI_F32, 64, 8>(ta, tb, a, tiles, st);
+    case 128: return run_gemm<EPI_F32, 128, 6>(ta, tb, a, tiles, st);
+    default: return run_gemm<EPI_F32, 256, 4>(ta, tb, a, tiles, st);
+  }
+}
+
+// ============================================================================
+// FP32 path on CUDA cores (tensor-core TF32 would not meet an FP32 tolerance).
+// C[r, n] = sum_k A[r, k] * B[n, k] over 32x32 output tiles; SWIGLU mode
+// computes gate and up accumulators together and writes silu(g) * u.
+// grid = (column tiles, row tiles of the largest group, groups).
+// ============================================================================
+template <bool SWIGLU>
+__global__ void __launch_bounds__(256) ffn_simt_kernel(const float* __restrict__ A, int lda,
+                                                       const float* __restrict__ B, const GemmArgs args,
+                                                       int64_t b_group_stride, int64_t b_up_offset) {
+  __shared__ float As[32][33];
+  __shared__ float Bg[32][33];
+  __shared__ float Bu[SWIGLU ? 32 : 1][33];
+  const int g = blockIdx.z;
+  int base;
+  const int rows = group_rows(args, g, &base);
+  const int m0 = blockIdx.y * 32;
+  if (m0 >= rows) return;
+  const int n0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // ty: 8 row groups of 4 rows
+  float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int kg = 0; kg < args.k_groups; ++kg) {
+    const float* Bm = B + static_cast<int64_t>(g * args.k_groups + kg) * b_group_stride;
+    for (int k0 = 0; k0 < args.K; k0 += 32) {
+      for (int i = threadIdx.x; i < 32 * 32; i += 256) {
+        const int rr = i / 32, kc = i % 32;
+        const int arow = base + m0 + rr, acol = k0 + kc;
+        As[rr][kc] = (m0 + rr < rows && acol < args.K) ? A[static_cast<int64_t>(arow) * lda + kg * args.K + acol] : 0.f;
+        const int bn = n0 + rr;
+        const bool bok = bn < args.N && acol < args.K;
+        Bg[rr][kc] = bok ? Bm[static_cast<int64_t>(bn) * args.K + acol] : 0.f;
+        if (SWIGLU) Bu[rr][kc] = bok ? Bm[b_up_offset + static_cast<int64_t>(bn) * args.K + acol] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int kc = 0; kc < 32; ++kc) {
+        const float bg = Bg[tx][kc];
+        const float bu = SWIGLU ? Bu[tx][kc] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float av = As[ty * 4 + i][kc];
+          accg[i] = fmaf(av, bg, accg[i]);
+          if (SWIGLU) accu[i] = fmaf(av, bu, accu[i]);
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int n = n0 + tx;
+  if (n >= args.N) return;
+  float* out = static_cast<float*>(args.out);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int rr = m0 + ty * 4 + i;
+    if (rr < rows) {
+      float v = accg[i];
+      if (SWIGLU) v = v / (1.0f + expf(-v)) * accu[i];
+      out[static_cast<int64_t>(base + rr) * args.ldo + static_cast<int64_t>(g) * args.out_col_stride + n] = v;
+    }
+  }
+}
+
+static int ffn_simt(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
+                    const void* w13, const void* w2, void* h, void* y_rows, cudaStream_t st, cudaEvent_t after_up) {
+  const bool routed = mode == 0;
+  const int G = routed ? p.E : p.Ns;
+  int64_t max_group_rows = routed ? (p.cap < 0 ? p.T : (p.cap < p.T ? p.cap : p.T)) : n_rows;
+  if (max_group_rows > n_rows) max_group_rows = n_rows;
+  if (max_group_rows <= 0) return 0;
+  GemmArgs up{};
+  up.n_groups = G;
+  up.seg_off = routed ? seg_off : nullptr;
+  up.n_rows = static_cast<int>(n_rows);
+  up.N = p.F;
+  up.K = p.d;
+  up.k_groups = 1;
+  up.out = h;
+  up.ldo = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+  up.out_col_stride = routed ? 0 : p.F;
+  dim3 g1(static_cast<unsigned>(cdiv(p.F, 32)), static_cast<unsigned>(cdiv(max_group_rows, 32)), G);
+  ffn_simt_kernel<true><<<g1, 256, 0, st>>>(static_cast<const float*>(x_rows), p.d, static_cast<const float*>(w13),
+                                            up, 2LL * p.F * p.d, static_cast<int64_t>(p.F) * p.d);
+  if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
+  GemmArgs dn{};
+  dn.n_groups = routed ? p.E : 1;
+  dn.seg_off = routed ? seg_off : nullptr;
+  dn.n_rows = static_cast<int>(n_rows);
+  dn.N = p.d;
+  dn.K = p.F;
+  dn.k_groups = routed ? 1 : p.Ns;
+  dn.out = y_rows;
+  dn.ldo = p.d;
+  dn.out_col_stride = 0;
+  dim3 g2(static_cast<unsigned>(cdiv(p.d, 32)), static_cast<unsigned>(cdiv(max_group_rows, 32)), dn.n_groups);
+  ffn_simt_kernel<false><<<g2, 256, 0, st>>>(static_cast<const float*>(h), static_cast<int>(up.ldo),
+                                             static_cast<const float*>(w2), dn, static_cast<int64_t>(p.d) * p.F, 0);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+// mode 0: routed (groups = experts over seg_off); mode 1: shared (every row
+// through all N_s experts, summed).  h is scratch: [n_rows, F] (routed) or
+// [n_rows, N_s * F] (shared).
+int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
+                      const void* w13, const void* w2, void* h, void* y_rows, unsigned* status, cudaStream_t st,
+                      cudaEvent_t after_up, int* n_kernels) {
+  if (n_rows <= 0) return 0;
+  if (n_kernels) *n_kernels += 2;
+  if (p.dtype == kF32) return ffn_simt(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, st, after_up);
+  const bool routed = mode == 0;
+  const int G = routed ? p.E : p.Ns;
+  const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+
+  // up/gate projection + SwiGLU: A = x_rows [n_rows, d], B = w13 viewed as (d, F, 2G)
+  CUtensorMap ta, tb;
+  {
+    const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
+    const uint32_t ba[2] = {kBK, kBM};
+    const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.F), static_cast<uint64_t>(2 * G)};
+    const uint32_t bb[3] = {kBK, 128, 1};
+    if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
+    GemmArgs a{};
+    a.n_groups = G;
+    a.seg_off = routed ? seg_off : nullptr;
+    a.n_rows = static_cast<int>(n_rows);
+    a.N = p.F;
+    a.K = p.d;
+    a.k_groups = 1;
+    a.out = h;
+    a.ldo = h_cols;
+    a.out_col_stride = routed ? 0 : p.F;
+    a.status = status;
+    const int64_t m_tiles = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
+    const int rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, m_tiles * cdiv(p.F, 128), st);
+    if (rc) return rc;
+    if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
+  }
+  // down projection: A = h [n_rows, k_groups * F], B = w2 viewed as (F, d, G)
+  {
+    const uint64_t da[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
+    const uint32_t ba[2] = {kBK, kBM};
+    const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
+    const uint32_t bb[3] = {kBK, 256, 1};
+    if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
+    GemmArgs a{};
+    a.n_groups = routed ? G : 1;
+    a.seg_off = routed ? seg_off : nullptr;
+    a.n_rows = static_cast<int>(n_rows);
+    a.N = p.d;
+    a.K = p.F;
+    a.k_groups = routed ? 1 : p.Ns;
+    a.out = y_rows;
+    a.ldo = p.d;
+    a.out_col_stride = 0;
+    a.status = status;
+    const int64_t m_tiles = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
+    const int rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, m_tiles * cdiv(p.d, 256), st);
+    if (rc) return rc;
+  }
+  return 0;
+}
+
+}  // namespace moe

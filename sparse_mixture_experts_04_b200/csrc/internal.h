@@ -1,0 +1,70 @@
+// Internal declarations of libmoe_b200: the validated problem, the workspace
+// layout and the kernel launchers each .cu file provides.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTopK = 32;
+constexpr int kDispatchChunk = 256;  // tokens per block in the dispatch kernels
+constexpr int kSelectTokens = 64;    // tokens per block in the selection kernel
+
+enum Dtype { kBF16 = 0, kF32 = 1 };
+
+struct Problem {
+  int64_t T;
+  int d, E, K, Ns, F;
+  int64_t cap;       // effective per-expert capacity, min(cap_raw, T); -1: no limit
+  int64_t cap_raw;   // ceil(C*T*K/E) as defined
+  int64_t max_rows;  // upper bound on kept rows
+  int dtype;
+  uint32_t flags;
+  float alpha;
+  size_t esize() const { return dtype == kBF16 ? 2 : 4; }
+};
+
+// Byte offsets of every scratch array inside the caller's workspace.
+struct WsLayout {
+  size_t status, logits, topk_idx, topk_w, counts, kept, seg_off, slot_of, perm;
+  size_t chunk_counts, chunk_base, sel_psum, sel_count;
+  size_t x_perm, h_routed, y_perm, h_shared, y_shared;
+  size_t total;
+  int n_chunks, n_sel_blocks;
+};
+WsLayout make_layout(const Problem& p);
+
+// router.cu
+cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void* w_gate,
+                                    const float* offset, float* logits, cudaStream_t st);
+cudaError_t launch_route_select(const Problem& p, const float* logits, const float* sel_bias,
+                                int32_t* topk_idx, float* topk_w, float* psum, int32_t* pcount,
+                                unsigned* status, cudaStream_t st);
+cudaError_t launch_route_stats(const Problem& p, const float* psum, const int32_t* pcount, int n_blocks,
+                               float* stats, cudaStream_t st);
+
+// dispatch.cu
+cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* counts, int32_t* kept,
+                            int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
+                            int32_t* chunk_base, unsigned* status, cudaStream_t st);
+cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
+                          void* x_perm, cudaStream_t st);
+
+// expert_gemm.cu -- returns a moe_status value
+int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset,
+                          float* logits, unsigned* status, cudaStream_t st);
+int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
+                      const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
+                      cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr);
+
+// combine.cu
+cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
+                           const void* y_shared, void* y, cudaStream_t st);
+
+// device properties (cached per device)
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,349 @@
+// C ABI of libmoe_b200 (declared in include/moe_b200.h): argument checks,
+// workspace layout and the launch sequence of each entry point.  Host code
+// only; every step of the layer runs in the kernels of router.cu, dispatch.cu,
+// expert_gemm.cu and combine.cu.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/moe_b200.h"
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+WsLayout make_layout(const Problem& p) {
+  WsLayout L{};
+  const size_t es = p.esize();
+  const size_t TK = static_cast<size_t>(p.T) * p.K;
+  const size_t R = static_cast<size_t>(p.max_rows);
+  L.n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
+  L.n_sel_blocks = static_cast<int>((p.T + kSelectTokens - 1) / kSelectTokens);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + (bytes ? bytes : 1));
+    return o;
+  };
+  L.status = take(256);
+  L.logits = take(static_cast<size_t>(p.T) * p.E * 4);
+  L.topk_idx = take(TK * 4);
+  L.topk_w = take(TK * 4);
+  L.counts = take(static_cast<size_t>(p.E) * 4);
+  L.kept = take(static_cast<size_t>(p.E) * 4);
+  L.seg_off = take(static_cast<size_t>(p.E + 1) * 4);
+  L.slot_of = take(TK * 4);
+  L.perm = take(R * 4);
+  L.chunk_counts = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
+  L.chunk_base = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
+  L.sel_psum = take(static_cast<size_t>(L.n_sel_blocks) * p.E * 4);
+  L.sel_count = take(static_cast<size_t>(L.n_sel_blocks) * p.E * 4);
+  L.x_perm = take(R * p.d * es);
+  L.h_routed = take(R * p.F * es);
+  L.y_perm = take(R * p.d * es);
+  L.h_shared = take(static_cast<size_t>(p.T) * p.Ns * p.F * es);
+  L.y_shared = take(p.Ns > 0 ? static_cast<size_t>(p.T) * p.d * es : 0);
+  L.total = off;
+  return L;
+}
+
+static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+// Validate the problem and derive cap / max_rows.  Returns MOE_OK or an error.
+static int to_problem(const moe_problem_t* in, Problem* out) {
+  if (!in) return MOE_ERR_INVALID_ARG;
+  const moe_problem_t& q = *in;
+  if (q.T < 1 || q.d_model < 8 || q.d_ff < 8 || (q.d_model % 8) || (q.d_ff % 8)) return MOE_ERR_INVALID_ARG;
+  if (q.n_experts < 1 || q.top_k < 1 || q.top_k > q.n_experts || q.n_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (q.dtype != MOE_DTYPE_BF16 && q.dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
+  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT)) return MOE_ERR_INVALID_ARG;
+  if (!(q.alpha == q.alpha) || !(q.capacity_factor == q.capacity_factor)) return MOE_ERR_INVALID_ARG;
+  if (q.n_experts > kMaxExperts || q.top_k > kMaxTopK || q.n_shared > 256) return MOE_ERR_UNSUPPORTED;
+  const int64_t lim = static_cast<int64_t>(1) << 31;
+  if (q.T >= lim / q.top_k || q.T >= lim / q.n_experts) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(q.d_ff) * (q.n_shared > 0 ? q.n_shared : 1) >= lim) return MOE_ERR_UNSUPPORTED;
+  Problem p{};
+  p.T = q.T;
+  p.d = q.d_model;
+  p.E = q.n_experts;
+  p.K = q.top_k;
+  p.Ns = q.n_shared;
+  p.F = q.d_ff;
+  p.dtype = q.dtype;
+  p.flags = q.flags;
+  p.alpha = q.alpha;
+  // capacity: ceil(C * (T*K) / E) evaluated in float64; C <= 0 means no limit
+  if (q.capacity_factor > 0.0f) {
+    const double v = (static_cast<double>(q.capacity_factor) * static_cast<double>(q.T * q.top_k)) /
+                     static_cast<double>(q.n_experts);
+    const double c = ceil(v);
+    p.cap_raw = c >= 4611686018427387904.0 ? (static_cast<int64_t>(1) << 62) : static_cast<int64_t>(c);
+    // an expert serves at most T tokens (a token picks it at most once)
+    p.cap = p.cap_raw >= q.T ? q.T : p.cap_raw;
+  } else {
+    p.cap = p.cap_raw = -1;
+  }
+  const int64_t TK = q.T * q.top_k;
+  p.max_rows = (p.cap < 0) ? TK : (p.cap * q.n_experts < TK ? p.cap * q.n_experts : TK);
+  *out = p;
+  return MOE_OK;
+}
+
+static int check_ws(const Problem& p, void* ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < make_layout(p).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <typename T>
+static T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Router body shared by moe_route and moe_layer_forward.
+static int route_impl(const Problem& p, const void* x, const void* w_gate, const float* offset,
+                      const float* sel_bias, float* logits, int32_t* idx, float* w, float* stats, void* ws,
+                      const WsLayout& L, cudaStream_t st) {
+  unsigned* status = at<unsigned>(ws, L.status);
+  if (!(p.flags & MOE_FLAG_LOGITS_GIVEN)) {
+    if (p.dtype == kBF16 && p.E > 16) {
+      const int rc = launch_gate_logits_tc(p, x, w_gate, offset, logits, status, st);
+      if (rc) return MOE_ERR_CUDA;
+    } else {
+      if (cudaError_t e = launch_gate_logits_simt(p, x, w_gate, offset, logits, st)) return cuda_rc(e);
+    }
+  }
+  float* psum = at<float>(ws, L.sel_psum);
+  int32_t* pcount = at<int32_t>(ws, L.sel_count);
+  if (cudaError_t e = launch_route_select(p, logits, sel_bias, idx, w, psum, pcount, status, st))
+    return cuda_rc(e);
+  if (stats) {
+    if (cudaError_t e = launch_route_stats(p, psum, pcount, L.n_sel_blocks, stats, st)) return cuda_rc(e);
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(int code) {
+  switch (code) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: problem outside this build's limits";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call failed";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a kernel reported bad data";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, too small or not 256-byte aligned";
+    default: return "unknown moe_status";
+  }
+}
+
+int64_t moe_capacity(const moe_problem_t* q) {
+  Problem p;
+  if (to_problem(q, &p) != MOE_OK) return -2;
+  return p.cap_raw;
+}
+
+int64_t moe_max_rows(const moe_problem_t* q) {
+  Problem p;
+  if (to_problem(q, &p) != MOE_OK) return -2;
+  return p.max_rows;
+}
+
+int moe_workspace_size(const moe_problem_t* q, size_t* bytes) {
+  Problem p;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  if (int rc = to_problem(q, &p)) return rc;
+  *bytes = make_layout(p).total;
+  return MOE_OK;
+}
+
+int moe_reset_device_status(void* ws, moe_stream_t stream) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  return cuda_rc(cudaMemsetAsync(ws, 0, sizeof(unsigned), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_read_device_status(const void* ws, moe_stream_t stream, uint32_t* bits) {
+  if (!ws || !bits) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(unsigned), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  *bits = v;
+  return v ? MOE_ERR_DEVICE_CHECK : MOE_OK;
+}
+
+int moe_route(const moe_problem_t* q, const void* x, const void* w_gate, const float* logit_offset,
+              const float* sel_bias, float* logits, int32_t* topk_idx, float* topk_w, float* stats, void* ws,
+              size_t ws_bytes, moe_stream_t stream) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (int rc = check_ws(p, ws, ws_bytes)) return rc;
+  const bool given = p.flags & MOE_FLAG_LOGITS_GIVEN;
+  if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!given && (!x || !w_gate || !aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  return route_impl(p, x, w_gate, given ? nullptr : logit_offset, sel_bias, logits, topk_idx, topk_w, stats, ws,
+                    L, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch(const moe_problem_t* q, const int32_t* topk_idx, const void* x, int32_t* counts, int32_t* kept,
+                 int32_t* seg_off, int32_t* slot_of, int32_t* perm, void* x_perm, void* ws, size_t ws_bytes,
+                 moe_stream_t stream) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (int rc = check_ws(p, ws, ws_bytes)) return rc;
+  if (!topk_idx || !counts || !kept || !seg_off || !slot_of || !perm) return MOE_ERR_INVALID_ARG;
+  if (x_perm && (!x || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaError_t e = launch_dispatch(p, topk_idx, counts, kept, seg_off, slot_of, perm,
+                                      at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base),
+                                      at<unsigned>(ws, L.status), st))
+    return cuda_rc(e);
+  if (x_perm) {
+    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
+  }
+  return MOE_OK;
+}
+
+int moe_expert_ffn(const moe_problem_t* q, int32_t mode, const void* x_rows, int64_t n_rows,
+                   const int32_t* seg_off, const void* w13, const void* w2, void* y_rows, void* ws, size_t ws_bytes,
+                   moe_stream_t stream) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (int rc = check_ws(p, ws, ws_bytes)) return rc;
+  if (mode != MOE_FFN_ROUTED && mode != MOE_FFN_SHARED) return MOE_ERR_INVALID_ARG;
+  if (!x_rows || !w13 || !w2 || !y_rows || n_rows < 1) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(w13) || !aligned16(w2) || !aligned16(y_rows)) return MOE_ERR_INVALID_ARG;
+  if (mode == MOE_FFN_ROUTED && (!seg_off || n_rows > p.max_rows)) return MOE_ERR_INVALID_ARG;
+  if (mode == MOE_FFN_SHARED && (p.Ns < 1 || n_rows > p.T)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  void* h = at<void>(ws, mode == MOE_FFN_ROUTED ? L.h_routed : L.h_shared);
+  const int rc = launch_expert_ffn(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, at<unsigned>(ws, L.status),
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return rc ? MOE_ERR_CUDA : MOE_OK;
+}
+
+int moe_combine(const moe_problem_t* q, const void* y_perm, const int32_t* slot_of, const float* topk_w,
+                const void* y_shared, void* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (int rc = check_ws(p, ws, ws_bytes)) return rc;
+  if (!slot_of || !topk_w || !y || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (p.max_rows > 0 && (!y_perm || !aligned16(y_perm))) return MOE_ERR_INVALID_ARG;
+  if ((p.Ns > 0) != (y_shared != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (y_shared && !aligned16(y_shared)) return MOE_ERR_INVALID_ARG;
+  return cuda_rc(launch_combine(p, y_perm, slot_of, topk_w, y_shared, y, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
+                              const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes,
+                              moe_stream_t stream, void* const* events, int32_t* n_kernels) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (int rc = check_ws(p, ws, ws_bytes)) return rc;
+  const bool given = p.flags & MOE_FLAG_LOGITS_GIVEN;
+  if (!x || !w || !y || !aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (!w->w13 || !w->w2 || !aligned16(w->w13) || !aligned16(w->w2)) return MOE_ERR_INVALID_ARG;
+  if (!given && (!w->w_gate || !aligned16(w->w_gate))) return MOE_ERR_INVALID_ARG;
+  if (given && (!routing || !routing->logits)) return MOE_ERR_INVALID_ARG;
+  if (p.Ns > 0 && (!w->w13_shared || !w->w2_shared || !aligned16(w->w13_shared) || !aligned16(w->w2_shared)))
+    return MOE_ERR_INVALID_ARG;
+  if (p.Ns == 0 && (w->w13_shared || w->w2_shared)) return MOE_ERR_INVALID_ARG;
+
+  const WsLayout L = make_layout(p);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto mark = [&](int i) -> cudaError_t {
+    if (!events || !events[i]) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
+  };
+  int kernels = 0;
+  moe_routing_t r{};
+  if (routing) r = *routing;
+  float* logits = r.logits ? r.logits : at<float>(ws, L.logits);
+  int32_t* idx = r.topk_idx ? r.topk_idx : at<int32_t>(ws, L.topk_idx);
+  float* gw = r.topk_w ? r.topk_w : at<float>(ws, L.topk_w);
+  int32_t* counts = r.counts ? r.counts : at<int32_t>(ws, L.counts);
+  int32_t* kept = r.kept ? r.kept : at<int32_t>(ws, L.kept);
+  int32_t* seg_off = r.seg_off ? r.seg_off : at<int32_t>(ws, L.seg_off);
+  int32_t* slot_of = r.slot_of ? r.slot_of : at<int32_t>(ws, L.slot_of);
+  int32_t* perm = r.perm ? r.perm : at<int32_t>(ws, L.perm);
+  unsigned* status = at<unsigned>(ws, L.status);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  void* y_sh = p.Ns > 0 ? at<void>(ws, L.y_shared) : nullptr;
+
+  if (cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st)) return cuda_rc(e);
+  if (cudaError_t e = mark(MOE_EV_START)) return cuda_rc(e);
+  if (int rc = route_impl(p, x, w->w_gate, given ? nullptr : w->logit_offset, w->sel_bias, logits, idx, gw, stats,
+                          ws, L, st))
+    return rc;
+  kernels += (given ? 0 : 1) + 1 + (stats ? 1 : 0);
+  if (cudaError_t e = mark(MOE_EV_ROUTED)) return cuda_rc(e);
+  if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, at<int32_t>(ws, L.chunk_counts),
+                                      at<int32_t>(ws, L.chunk_base), status, st))
+    return cuda_rc(e);
+  kernels += 3;
+  if (p.max_rows > 0) {
+    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
+    kernels += 1;
+  }
+  if (cudaError_t e = mark(MOE_EV_DISPATCHED)) return cuda_rc(e);
+  if (p.max_rows > 0) {
+    cudaEvent_t up_ev = (events && events[MOE_EV_UP]) ? static_cast<cudaEvent_t>(events[MOE_EV_UP]) : nullptr;
+    if (launch_expert_ffn(p, MOE_FFN_ROUTED, x_perm, p.max_rows, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed),
+                          y_perm, status, st, up_ev, &kernels))
+      return MOE_ERR_CUDA;
+  } else if (cudaError_t e = mark(MOE_EV_UP)) {
+    return cuda_rc(e);
+  }
+  if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
+  if (p.Ns > 0) {
+    if (launch_expert_ffn(p, MOE_FFN_SHARED, x, p.T, nullptr, w->w13_shared, w->w2_shared,
+                          at<void>(ws, L.h_shared), y_sh, status, st, nullptr, &kernels))
+      return MOE_ERR_CUDA;
+  }
+  if (cudaError_t e = mark(MOE_EV_SHARED)) return cuda_rc(e);
+  if (cudaError_t e = launch_combine(p, y_perm, slot_of, gw, y_sh, y, st)) return cuda_rc(e);
+  kernels += 1;
+  if (cudaError_t e = mark(MOE_EV_END)) return cuda_rc(e);
+  if (n_kernels) *n_kernels = kernels;
+  return MOE_OK;
+}
+
+int moe_layer_forward(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
+                      const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, nullptr, nullptr);
+}
+
+int moe_layer_forward_profiled(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
+                               const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes,
+                               moe_stream_t stream, void* const* events, int32_t* n_kernels) {
+  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, events, n_kernels);
+}
+
+}  // extern "C"

@@ -1,0 +1,336 @@
+// Router: gate logits, softmax, top-K selection with optional selection bias,
+// renormalised gate weights, and the Switch balance statistics.
+//
+//   Zen MoDE: Mixture of Distilled Experts Architecture, §3.1 Router
+//     Architecture, eq. router_standard: TopK(softmax(W_r x), K).
+//   Zen-Max, §2.3 Auxiliary-Loss-Free Load Balancing: s_ij = softmax(x_i W_g)_j + b_j
+//     (the bias steers selection; gate weights use the unbiased softmax).
+//   Scaling with experts, "The gating network": keep the top-k, zero the rest,
+//     renormalise the survivors to sum to one.  "A balance penalty":
+//     alpha * N * sum f_i P_i.  Zen MoDE §5.2 eq. L_balance.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// ----------------------------------------------------------------------------
+// Gate logits on CUDA cores: logits[t, e] = sum_j x[t, j] * Wg[e, j] + off[e].
+// One warp handles TPW tokens at a time; lanes stride over d in 16-byte
+// vectors; each lane keeps TPW x EB partial sums (so every Wg vector it loads
+// serves TPW tokens), then a butterfly reduction gives every lane the sums.
+// Experts are processed in blocks of EB (several passes when E > EB).
+// Used for FP32 problems and for BF16 problems with few experts.
+// ----------------------------------------------------------------------------
+template <typename Tin>
+struct Vec16;
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float (&v)[4]) {
+    float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+    uint4 q = *reinterpret_cast<const uint4*>(p);
+    v[0] = bf16_lo(q.x); v[1] = bf16_hi(q.x); v[2] = bf16_lo(q.y); v[3] = bf16_hi(q.y);
+    v[4] = bf16_lo(q.z); v[5] = bf16_hi(q.z); v[6] = bf16_lo(q.w); v[7] = bf16_hi(q.w);
+  }
+};
+
+template <typename Tin, int EB, int TPW>
+__global__ void __launch_bounds__(256) gate_logits_simt_kernel(const Tin* __restrict__ x,
+                                                               const Tin* __restrict__ wg,
+                                                               const float* __restrict__ off,
+                                                               float* __restrict__ logits, int64_t T, int d,
+                                                               int E) {
+  constexpr int V = Vec16<Tin>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t n_groups = (T + TPW - 1) / TPW;
+
+  for (int64_t grp = warp_global; grp < n_groups; grp += n_warps) {
+    const int64_t t0 = grp * TPW;
+    for (int eb = 0; eb < E; eb += EB) {
+      float acc[TPW][EB];
+#pragma unroll
+      for (int i = 0; i < TPW; ++i)
+#pragma unroll
+        for (int e = 0; e < EB; ++e) acc[i][e] = 0.f;
+
+      for (int j = lane * V; j < d; j += 32 * V) {
+        float xv[TPW][V];
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          if (t0 + i < T) {
+            Vec16<Tin>::load(x + (t0 + i) * d + j, xv[i]);
+          } else {
+#pragma unroll
+            for (int v = 0; v < V; ++v) xv[i][v] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < EB; ++e) {
+          if (eb + e < E) {
+            float wv[V];
+            Vec16<Tin>::load(wg + static_cast<int64_t>(eb + e) * d + j, wv);
+#pragma unroll
+            for (int i = 0; i < TPW; ++i)
+#pragma unroll
+              for (int v = 0; v < V; ++v) acc[i][e] = fmaf(xv[i][v], wv[v], acc[i][e]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < TPW; ++i)
+#pragma unroll
+        for (int e = 0; e < EB; ++e) acc[i][e] = warp_sum(acc[i][e]);
+#pragma unroll
+      for (int i = 0; i < TPW; ++i) {
+#pragma unroll
+        for (int e = 0; e < EB; ++e) {
+          if (lane == e && t0 + i < T && eb + e < E)
+            logits[(t0 + i) * E + eb + e] = acc[i][e] + (off ? off[eb + e] : 0.f);
+        }
+      }
+    }
+  }
+}
+
+template <typename Tin, int EB, int TPW>
+static cudaError_t gate_simt(const Problem& p, const void* x, const void* wg, const float* off, float* logits,
+                             cudaStream_t st) {
+  const int64_t warps = (p.T + TPW - 1) / TPW;
+  int64_t blocks = (warps + 7) / 8;
+  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  gate_logits_simt_kernel<Tin, EB, TPW><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const Tin*>(x), static_cast<const Tin*>(wg), off, logits, p.T, p.d, p.E);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void* wg, const float* off,
+                                    float* logits, cudaStream_t st) {
+  if (p.dtype == kBF16) {
+    if (p.E <= 8) return gate_simt<__nv_bfloat16, 8, 4>(p, x, wg, off, logits, st);
+    if (p.E <= 16) return gate_simt<__nv_bfloat16, 16, 2>(p, x, wg, off, logits, st);
+    return gate_simt<__nv_bfloat16, 32, 1>(p, x, wg, off, logits, st);
+  }
+  if (p.E <= 8) return gate_simt<float, 8, 4>(p, x, wg, off, logits, st);
+  if (p.E <= 16) return gate_simt<float, 16, 2>(p, x, wg, off, logits, st);
+  return gate_simt<float, 32, 1>(p, x, wg, off, logits, st);
+}
+
+// ----------------------------------------------------------------------------
+// Selection.  One warp per token; lane l holds experts l, l+32, ... (EPL of
+// them).  Per token:
+//   m = max logit; ex_e = exp(l_e - m) (fp32); Z = sum ex; p_e = ex_e / Z
+//   score_e (float64): l_e, or p64_e + b_e (bias on p), or l_e + b_e (bias on logit),
+//     p64 = exp(l - m) / sum exp(l - m) evaluated in float64
+//   K rounds of warp arg-max over (score desc, expert index asc)
+//   w_k = ex_{idx_k} / sum_k ex_{idx_k}    (= renormalised softmax over the chosen)
+// Per block: sum over its tokens of p_e (fp32, fixed order) and the number of
+// times each expert was chosen (integer), for the balance statistics.
+// ----------------------------------------------------------------------------
+template <int EPL>
+__global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ logits,
+                                                           const float* __restrict__ sel_bias, int bias_on_logit,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w, float* __restrict__ psum,
+                                                           int32_t* __restrict__ pcount, int64_t T, int E,
+                                                           int K) {
+  __shared__ float s_psum[8][32 * EPL];
+  __shared__ int s_count[32 * EPL];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < 32 * EPL; e += blockDim.x) s_count[e] = 0;
+  __syncthreads();
+
+  float pacc[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) pacc[i] = 0.f;
+
+  const int64_t tok_begin = static_cast<int64_t>(blockIdx.x) * kSelectTokens;
+  constexpr int kPerWarp = kSelectTokens / 8;
+  for (int n = 0; n < kPerWarp; ++n) {
+    const int64_t t = tok_begin + warp * kPerWarp + n;
+    if (t >= T) break;
+    float lg[EPL];
+    float mloc = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      lg[i] = (e < E) ? logits[t * E + e] : -INFINITY;
+      mloc = fmaxf(mloc, lg[i]);
+    }
+    const float m = warp_max(mloc);
+    float ex[EPL];
+    float zloc = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      ex[i] = (e < E) ? expf(lg[i] - m) : 0.f;
+      zloc += ex[i];
+    }
+    const float Z = warp_sum(zloc);
+    const float invZ = 1.0f / Z;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) pacc[i] += ex[i] * invZ;
+
+    double score[EPL];
+    if (sel_bias == nullptr) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) score[i] = static_cast<double>(lg[i]);
+    } else if (bias_on_logit) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        score[i] = (e < E) ? static_cast<double>(lg[i]) + static_cast<double>(sel_bias[e]) : -INFINITY;
+      }
+    } else {
+      const double m64 = static_cast<double>(m);
+      double ex64[EPL];
+      double z64loc = 0.0;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        ex64[i] = (e < E) ? exp(static_cast<double>(lg[i]) - m64) : 0.0;
+        z64loc += ex64[i];
+      }
+      const double z64 = warp_sum(z64loc);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        score[i] = (e < E) ? ex64[i] / z64 + static_cast<double>(sel_bias[e]) : -INFINITY;
+      }
+    }
+
+    // NaN scores rank lowest, so (score, index) is a total order and every
+    // lane agrees on each round's winner, which is always a valid expert.
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+      if (score[i] != score[i]) score[i] = -INFINITY;
+    bool taken[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) taken[i] = (lane + 32 * i) >= E;
+    int my_e = -1;
+    float my_ex = 0.f;
+    for (int k = 0; k < K; ++k) {
+      double best = -INFINITY;
+      int best_e = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        if (!taken[i] && (best_e == 0x7fffffff || score[i] > best)) {
+          best = score[i];
+          best_e = lane + 32 * i;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, best_e, o);
+        if (ob > best || (ob == best && oe < best_e)) {
+          best = ob;
+          best_e = oe;
+        }
+      }
+      // best_e is now the same on every lane
+      const int slot = best_e >> 5;
+      float ex_sel = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (i == slot) ex_sel = ex[i];
+      ex_sel = __shfl_sync(0xffffffffu, ex_sel, best_e & 31);
+      if (lane == (best_e & 31)) {
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (i == slot) taken[i] = true;
+      }
+      if (lane == k) {
+        my_e = best_e;
+        my_ex = ex_sel;
+      }
+    }
+    const float wsum = warp_sum(lane < K ? my_ex : 0.f);
+    if (lane < K) {
+      topk_idx[t * K + lane] = my_e;
+      topk_w[t * K + lane] = my_ex / wsum;
+      if (static_cast<unsigned>(my_e) < static_cast<unsigned>(E)) atomicAdd(&s_count[my_e], 1);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) s_psum[warp][lane + 32 * i] = pacc[i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += s_psum[w][e];
+    psum[static_cast<int64_t>(blockIdx.x) * E + e] = s;
+    pcount[static_cast<int64_t>(blockIdx.x) * E + e] = s_count[e];
+  }
+}
+
+cudaError_t launch_route_select(const Problem& p, const float* logits, const float* sel_bias, int32_t* topk_idx,
+                                float* topk_w, float* psum, int32_t* pcount, unsigned* /*status*/,
+                                cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>((p.T + kSelectTokens - 1) / kSelectTokens);
+  const int bias_on_logit = (p.flags & 0x2u) ? 1 : 0;
+  if (p.E <= 32)
+    route_select_kernel<1><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K);
+  else if (p.E <= 64)
+    route_select_kernel<2><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K);
+  else if (p.E <= 128)
+    route_select_kernel<4><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K);
+  else
+    route_select_kernel<8><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// Balance statistics from the per-block partials (fixed summation order):
+//   f_e = count_e / (T K),  P_e = (1/T) sum_t p[t,e],  loss = alpha E sum_e f_e P_e
+// stats layout: [f_0 .. f_{E-1}, P_0 .. P_{E-1}, loss].
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) route_stats_kernel(const float* __restrict__ psum,
+                                                          const int32_t* __restrict__ pcount, int n_blocks,
+                                                          int64_t T, int E, int K, float alpha,
+                                                          float* __restrict__ stats) {
+  __shared__ double s_fp[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    long long c = 0;
+    double s = 0.0;
+    for (int b = 0; b < n_blocks; ++b) {
+      c += pcount[static_cast<int64_t>(b) * E + e];
+      s += static_cast<double>(psum[static_cast<int64_t>(b) * E + e]);
+    }
+    const double f = static_cast<double>(c) / (static_cast<double>(T) * K);
+    const double P = s / static_cast<double>(T);
+    stats[e] = static_cast<float>(f);
+    stats[E + e] = static_cast<float>(P);
+    s_fp[e] = f * P;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double acc = 0.0;
+    for (int e = 0; e < E; ++e) acc += s_fp[e];
+    stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
+  }
+}
+
+cudaError_t launch_route_stats(const Problem& p, const float* psum, const int32_t* pcount, int n_blocks,
+                               float* stats, cudaStream_t st) {
+  route_stats_kernel<<<1, 256, 0, st>>>(psum, pcount, n_blocks, p.T, p.E, p.K, p.alpha, stats);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

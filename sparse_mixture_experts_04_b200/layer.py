@@ -1,0 +1,56 @@
+"""MoeLayer: one layer's weights, workspace and routing buffers on the device,
+with forward() = one moe_layer_forward call.  Allocation (through torch) and
+argument marshalling only."""
+from __future__ import annotations
+
+import torch
+
+from . import api
+
+
+class MoeLayer:
+    def __init__(self, prob: api.MoeProblem, weights: dict, device="cuda", keep_routing: bool = True):
+        self.prob = prob
+        self.device = torch.device(device)
+        self.weights = weights
+        self.ws = api.alloc_workspace(prob, self.device)
+        self.dtype = torch.bfloat16 if prob.dtype == api.DTYPE_BF16 else torch.float32
+        T, E, K = prob.T, prob.n_experts, prob.top_k
+        self.routing = None
+        if keep_routing:
+            i32 = dict(dtype=torch.int32, device=self.device)
+            self.routing = dict(
+                logits=torch.empty((T, E), dtype=torch.float32, device=self.device),
+                topk_idx=torch.empty((T, K), **i32), topk_w=torch.empty((T, K), dtype=torch.float32, device=self.device),
+                counts=torch.empty(E, **i32), kept=torch.empty(E, **i32), seg_off=torch.empty(E + 1, **i32),
+                slot_of=torch.empty((T, K), **i32), perm=torch.empty(max(api.max_rows(prob), 1), **i32))
+        self.stats = torch.empty(2 * E + 1, dtype=torch.float32, device=self.device)
+
+    @classmethod
+    def from_inputs(cls, inputs: dict, device="cuda", flags: int = 0, keep_routing: bool = True) -> "MoeLayer":
+        """Build from synth.generate() output (CPU tensors are copied to the device)."""
+        cfg = inputs["cfg"]
+        prob = api.make_problem(cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.n_shared,
+                                cfg.capacity_factor, cfg.dtype, flags, cfg.alpha)
+        dev = torch.device(device)
+
+        def to_dev(v):
+            if v is None:
+                return None
+            t = torch.as_tensor(v)
+            return t.to(dev).contiguous()
+
+        w = {k: to_dev(inputs.get(k)) for k in ("w_gate", "w13", "w2", "w13_shared", "w2_shared")}
+        w["sel_bias"] = to_dev(inputs.get("sel_bias"))
+        w["logit_offset"] = to_dev(inputs.get("logit_offset"))
+        return cls(prob, w, dev, keep_routing)
+
+    def forward(self, x: torch.Tensor, y: torch.Tensor | None = None, with_stats: bool = True,
+                stream=None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty((self.prob.T, self.prob.d_model), dtype=self.dtype, device=self.device)
+        api.moe_layer_forward(self.prob, x, self.weights, y, self.routing, self.stats if with_stats else None,
+                              self.ws, stream)
+        return y
+
+    __call__ = forward

@@ -7,8 +7,9 @@ shapes and distributions of the five workloads and rounds them to the storage
 type.  (The Zipf logit offsets of the skewed workload are an input
 distribution, not part of the method.)
 
-Recipe (every tensor has its own PCG64 stream, keyed by (seed, tensor id), so
-a tensor does not change when another tensor's size changes):
+Recipe (every tensor has its own PCG64 stream, keyed by (seed, tensor id) --
+and per expert matrix by (seed, tensor id, expert) -- so a tensor does not
+change when another tensor's size changes):
   x          N(0, x_std^2)                              [T, d]
   w_gate     N(0, 1/d)                                   [E, d]
   w13        N(0, 1/d)   rows 0..F-1 gate, F..2F-1 up    [E, 2F, d]
@@ -24,8 +25,10 @@ BF16 tensors are float32 draws rounded to nearest-even BF16 (via torch).
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
 import math
+import os
 from dataclasses import dataclass
 
 import numpy as np
@@ -100,12 +103,18 @@ def _normal(rng: np.random.Generator, shape, std: float, dtype: str) -> torch.Te
 
 
 def _normal_stack(seed, tensor_id, n, shape, std, dtype) -> torch.Tensor:
-    """n independent matrices drawn one at a time (bounded float32 temporaries)."""
-    rng = _rng(seed, tensor_id)
+    """n independent matrices, matrix i from stream (seed, tensor_id, i); drawn
+    on a few threads (the generator's fill releases the GIL)."""
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     out = torch.empty((n,) + tuple(shape), dtype=tdt)
-    for i in range(n):
+
+    def one(i):
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), int(tensor_id), i])))
         out[i] = _normal(rng, shape, std, dtype)
+
+    workers = max(1, min(n, os.cpu_count() or 1, 16))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        list(ex.map(one, range(n)))
     return out
 
 
@@ -133,6 +142,12 @@ def generate(cfg: MoeConfig, with_weights: bool = True) -> dict:
                        if cfg.bias_range > 0 else None)
     out["logit_offset"] = zipf_offsets(cfg) if cfg.zipf_s > 0 else None
     return out
+
+
+def extra_activations(cfg: MoeConfig, n: int) -> list:
+    """n further activation batches x [T, d] with the recipe of x, from streams
+    (seed, 100 + i); used to rotate inputs between timed steps."""
+    return [_normal(_rng(cfg.seed, 100 + i), (cfg.T, cfg.d_model), cfg.x_std, cfg.dtype) for i in range(n)]
 
 
 def given_logits(cfg: MoeConfig, T: int | None = None) -> np.ndarray:

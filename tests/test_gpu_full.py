@@ -1,0 +1,81 @@
+"""The five workloads at full size, in the launch configuration the benchmark
+times (one moe_layer_forward per step through MoeLayer).
+
+Routing outputs are compared bit-exactly over every token (both sides fed the
+same float32 logits); layer outputs on sampled tokens the oracle computes one
+by one; the GPU's own gate logits on sampled tokens; and the GPU's end-to-end
+routing against the oracle's own float64 routing."""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import dev, generate, given_logits, host_np, oracle_layer, oracle_routing, rel_err, sample_rows, tol
+from sparse_mixture_experts_04_b200 import MoeLayer, api
+from sparse_mixture_experts_04_b200.synth import CONFIGS
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+N_SAMPLE = {"tiny_fp32": 64, "mixtral": 6, "zen_fine": 16, "skewed": 24, "decode": 32}
+
+
+@pytest.fixture(scope="module", params=list(CONFIGS))
+def workload(request):
+    name = request.param
+    cfg = CONFIGS[name]
+    inp = generate(cfg)
+    yield name, cfg, inp
+    del inp
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_full_size_given_logits(workload):
+    name, cfg, inp = workload
+    logits32 = given_logits(cfg)
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN)
+    layer.routing["logits"].copy_(torch.as_tensor(logits32))
+    y = layer.forward(dev(inp["x"]))
+    assert api.read_device_status(layer.ws) == 0
+    r = {k: v.cpu().numpy() for k, v in layer.routing.items()}
+    assert (r["topk_idx"] == ref["idx"]).all()
+    assert np.max(np.abs(r["topk_w"] - ref["w"])) <= 1e-6
+    for k in ("counts", "kept", "seg_off", "slot_of"):
+        assert (r[k] == ref[k]).all(), k
+    S = int(ref["seg_off"][-1])
+    assert (r["perm"][:S] == ref["perm"]).all()
+    st = layer.stats.cpu().numpy()
+    E = cfg.n_experts
+    assert (st[:E] == ref["f"].astype(np.float32)).all()
+    assert np.max(np.abs(st[E:2 * E] - ref["P"])) <= 1e-6
+    assert abs(st[2 * E] - ref["loss"]) <= 1e-6 * max(1.0, ref["loss"])
+    # sampled outputs, including tokens with dropped pairs when there are any
+    dropped = np.nonzero((ref["slot_of"] < 0).any(1))[0][:4]
+    rows = sample_rows(cfg.T, N_SAMPLE[name], seed=cfg.seed, extra=tuple(int(t) for t in dropped))
+    want = oracle_layer(inp, ref, rows=rows)
+    got = y.float().cpu().numpy()[rows]
+    assert rel_err(got, want) <= tol(cfg)
+
+
+def test_full_size_end_to_end(workload):
+    name, cfg, inp = workload
+    layer = MoeLayer.from_inputs(inp)
+    y = layer.forward(dev(inp["x"]))
+    assert api.read_device_status(layer.ws) == 0
+    g_logits = layer.routing["logits"].cpu().numpy().astype(np.float64)
+    l64 = oracle.gate_logits(host_np(inp["x"]), host_np(inp["w_gate"]), inp["logit_offset"])
+    bound = (1e-5 if cfg.dtype == "f32" else 1e-3) * max(1.0, float(np.max(np.abs(l64))))
+    assert np.max(np.abs(g_logits - l64)) <= bound
+    ref = oracle_routing(cfg, l64, inp["sel_bias"])
+    g_idx = layer.routing["topk_idx"].cpu().numpy()
+    g_slot = layer.routing["slot_of"].cpu().numpy()
+    same = (g_idx == ref["idx"]).all(1) & ((g_slot >= 0) == (ref["slot_of"] >= 0)).all(1)
+    assert same.mean() >= 0.99, f"routing agreed on {same.mean():.4f} of tokens"
+    rows = sample_rows(cfg.T, N_SAMPLE[name], seed=cfg.seed + 100)
+    rows = rows[same[rows]]
+    want = oracle_layer(inp, ref, rows=rows)
+    got = y.float().cpu().numpy()[rows]
+    assert rel_err(got, want) <= tol(cfg)

@@ -322,6 +322,34 @@ def test_layer_rows_subset_matches_full():
     assert (sub == full[rows]).all()
 
 
+def test_combine_of_grouped_expert_outputs_equals_layer():
+    # Run every kept (t,k) row through its expert, lay the results out in slot
+    # order, combine: must equal layer_rows, which evaluates per token.
+    rng = np.random.default_rng(9)
+    T, d, E, F, Ns = 13, 8, 4, 6, 2
+    x, w13, w2, (w13s, w2s) = _rand_layer(rng, T, d, E, F, Ns)
+    idx, w, _ = oracle.select(rng.normal(size=(T, E)), 2)
+    disp = oracle.dispatch(idx, E, 5)
+    S = int(disp["seg_off"][-1])
+    y_perm = np.zeros((S, d))
+    for s_ in range(S):
+        t, k = divmod(int(disp["perm"][s_]), 2)
+        y_perm[s_] = oracle.swiglu(x[t], w13[idx[t, k]], w2[idx[t, k]])
+    y_sh = np.stack([sum(oracle.swiglu(x[t], w13s[s], w2s[s]) for s in range(Ns)) for t in range(T)])
+    y = oracle.combine(y_perm, disp["slot_of"], w, y_sh)
+    want = oracle.layer_rows(x, w13, w2, idx, w, disp["slot_of"], w13_shared=w13s, w2_shared=w2s)
+    assert np.allclose(y, want, rtol=0, atol=1e-13)
+
+
+def test_combine_hand_example():
+    y_perm = np.array([[1.0, 2.0], [10.0, 20.0], [100.0, 200.0]])
+    slot_of = np.array([[2, -1], [0, 1]], np.int32)
+    w = np.array([[0.5, 0.5], [0.25, 0.75]])
+    y = oracle.combine(y_perm, slot_of, w, y_shared=np.array([[1.0, 1.0], [0.0, 0.0]]))
+    assert y.tolist() == [[51.0, 101.0], [7.75, 15.5]]
+    assert oracle.combine(y_perm, slot_of, w).tolist() == [[50.0, 100.0], [7.75, 15.5]]
+
+
 # --------------------------------------------------------------- balance stats
 def test_balance_uniform_routing_gives_exactly_alpha():
     g = golden("balance_alpha.json")
