@@ -46,8 +46,8 @@ METRIC = "MoE layer fwd tokens/s (BF16, 1 B200); expert GEMM % peak; dispatch GB
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # oracle tokens per reference step / in the cpu_baseline sample (about 0.5-1 s each)
-REF_TOKENS = {"tiny_fp32": 64, "mixtral": 1, "zen_fine": 4, "skewed": 8, "decode": 2}
-CPU_SAMPLE_TOKENS = {"tiny_fp32": 64, "mixtral": 16, "zen_fine": 48, "skewed": 96, "decode": 16}
+REF_TOKENS = {"tiny_fp32": 256, "mixtral": 2, "zen_fine": 8, "skewed": 16, "decode": 2}
+CPU_SAMPLE_TOKENS = {"tiny_fp32": 2048, "mixtral": 64, "zen_fine": 192, "skewed": 384, "decode": 64}
 
 
 def workload_desc(cfg) -> str:

@@ -59,8 +59,9 @@ def max_rows(prob: MoeProblem) -> int:
 
 
 def alloc_workspace(prob: MoeProblem, device="cuda") -> torch.Tensor:
-    """A caller-owned workspace (torch's allocator returns 256-byte aligned blocks)."""
-    return torch.empty(workspace_size(prob), dtype=torch.uint8, device=device)
+    """A caller-owned workspace (torch's allocator returns 256-byte aligned
+    blocks), zero-filled once so that its device status word starts clean."""
+    return torch.zeros(workspace_size(prob), dtype=torch.uint8, device=device)
 
 
 def reset_device_status(ws: torch.Tensor, stream=None) -> None:

@@ -6,7 +6,7 @@
 //
 //   y[t] = y_shared[t] + sum_{k : slot_of[t,k] >= 0} w[t,k] * y_perm[slot_of[t,k]]
 // accumulated in fp32 in that order (shared first, then k ascending) and
-// rounded once.  One warp per token, 16-byte vectors along d.
+// rounded once.  16-byte vectors along d.
 #include "common.cuh"
 #include "internal.h"
 
@@ -41,59 +41,76 @@ struct Pack16<float> {
   }
 };
 
+constexpr int kCombineThreads = 128;
+constexpr int kCombineVPT = 4;  // 16-byte vectors per thread per pass
+
+// One block per token (grid-stride).  The token's K (slot, weight) pairs are
+// staged in shared memory; each thread owns kCombineVPT vectors of the row and
+// issues all their loads before the arithmetic.
 template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(const T* __restrict__ y_perm,
-                                                      const int32_t* __restrict__ slot_of,
-                                                      const float* __restrict__ topk_w,
-                                                      const T* __restrict__ y_shared, T* __restrict__ y,
-                                                      int64_t Tn, int d, int K, int64_t n_perm_rows) {
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const T* __restrict__ y_perm,
+                                                                  const int32_t* __restrict__ slot_of,
+                                                                  const float* __restrict__ topk_w,
+                                                                  const T* __restrict__ y_shared,
+                                                                  T* __restrict__ y, int64_t Tn, int d, int K,
+                                                                  int64_t n_perm_rows) {
   constexpr int V = Pack16<T>::N;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  __shared__ int s_slot[kMaxTopK];
+  __shared__ float s_w[kMaxTopK];
   const int nvec = d / V;
-  for (int64_t t = warp0; t < Tn; t += n_warps) {
-    // lane k holds (slot, weight) of pair k
-    int my_slot = -1;
-    float my_w = 0.f;
-    if (lane < K) {
-      my_slot = slot_of[t * K + lane];
-      my_w = topk_w[t * K + lane];
+  for (int64_t t = blockIdx.x; t < Tn; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < K) {
+      const int slot = slot_of[t * K + threadIdx.x];
+      s_slot[threadIdx.x] = (slot >= 0 && slot < n_perm_rows) ? slot : -1;
+      s_w[threadIdx.x] = topk_w[t * K + threadIdx.x];
     }
-    for (int v = lane; v < nvec; v += 32) {
-      float acc[V];
-      if (y_shared) {
-        Pack16<T>::load(y_shared + t * d + v * V, acc);
-      } else {
+    __syncthreads();
+    for (int v0 = 0; v0 < nvec; v0 += kCombineThreads * kCombineVPT) {
+      float acc[kCombineVPT][V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = 0.f;
+      for (int j = 0; j < kCombineVPT; ++j) {
+        const int v = v0 + j * kCombineThreads + threadIdx.x;
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[j][i] = 0.f;
+        if (y_shared && v < nvec) Pack16<T>::load(y_shared + t * d + v * V, acc[j]);
       }
       for (int k = 0; k < K; ++k) {
-        const int slot = __shfl_sync(0xffffffffu, my_slot, k);
-        const float w = __shfl_sync(0xffffffffu, my_w, k);
-        if (slot >= 0 && slot < n_perm_rows) {
-          float r[V];
-          Pack16<T>::load(y_perm + static_cast<int64_t>(slot) * d + v * V, r);
+        const int slot = s_slot[k];
+        if (slot < 0) continue;
+        const float w = s_w[k];
+        const T* row = y_perm + static_cast<int64_t>(slot) * d;
+        float r[kCombineVPT][V];
 #pragma unroll
-          for (int i = 0; i < V; ++i) acc[i] = fmaf(w, r[i], acc[i]);
+        for (int j = 0; j < kCombineVPT; ++j) {
+          const int v = v0 + j * kCombineThreads + threadIdx.x;
+          if (v < nvec) Pack16<T>::load(row + v * V, r[j]);
         }
+#pragma unroll
+        for (int j = 0; j < kCombineVPT; ++j)
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[j][i] = fmaf(w, r[j][i], acc[j][i]);
       }
-      Pack16<T>::store(y + t * d + v * V, acc);
+#pragma unroll
+      for (int j = 0; j < kCombineVPT; ++j) {
+        const int v = v0 + j * kCombineThreads + threadIdx.x;
+        if (v < nvec) Pack16<T>::store(y + t * d + v * V, acc[j]);
+      }
     }
   }
 }
 
 cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
                            const void* y_shared, void* y, cudaStream_t st) {
-  int64_t blocks = (p.T + 7) / 8;
-  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
+  int64_t blocks = p.T;
+  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 32;
   if (blocks > cap_blocks) blocks = cap_blocks;
   if (p.dtype == kBF16)
-    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCombineThreads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(y_perm), slot_of, topk_w, static_cast<const __nv_bfloat16*>(y_shared),
         static_cast<__nv_bfloat16*>(y), p.T, p.d, p.K, p.max_rows);
   else
-    combine_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+    combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineThreads, 0, st>>>(
         static_cast<const float*>(y_perm), slot_of, topk_w, static_cast<const float*>(y_shared),
         static_cast<float*>(y), p.T, p.d, p.K, p.max_rows);
   return cudaGetLastError();

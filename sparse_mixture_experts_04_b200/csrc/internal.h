@@ -11,7 +11,7 @@ namespace moe {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 32;
 constexpr int kDispatchChunk = 256;  // tokens per block in the dispatch kernels
-constexpr int kSelectTokens = 64;    // tokens per block in the selection kernel
+constexpr int kSelectTokens = 32;    // tokens per block in the selection kernel (4 per warp)
 
 enum Dtype { kBF16 = 0, kF32 = 1 };
 

@@ -124,7 +124,7 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
                       const WsLayout& L, cudaStream_t st) {
   unsigned* status = at<unsigned>(ws, L.status);
   if (!(p.flags & MOE_FLAG_LOGITS_GIVEN)) {
-    if (p.dtype == kBF16 && p.E > 16) {
+    if (p.dtype == kBF16) {
       const int rc = launch_gate_logits_tc(p, x, w_gate, offset, logits, status, st);
       if (rc) return MOE_ERR_CUDA;
     } else {

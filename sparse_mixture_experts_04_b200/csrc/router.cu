@@ -297,39 +297,61 @@ cudaError_t launch_route_select(const Problem& p, const float* logits, const flo
 }
 
 // ----------------------------------------------------------------------------
-// Balance statistics from the per-block partials (fixed summation order):
+// Balance statistics from the per-block partials:
 //   f_e = count_e / (T K),  P_e = (1/T) sum_t p[t,e],  loss = alpha E sum_e f_e P_e
 // stats layout: [f_0 .. f_{E-1}, P_0 .. P_{E-1}, loss].
+// One block of 1024 threads: thread (e, s) sums every S-th block partial of
+// expert e; the S sub-sums are then added in a fixed order, so the result
+// does not depend on scheduling.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) route_stats_kernel(const float* __restrict__ psum,
-                                                          const int32_t* __restrict__ pcount, int n_blocks,
-                                                          int64_t T, int E, int K, float alpha,
-                                                          float* __restrict__ stats) {
+__global__ void __launch_bounds__(1024) route_stats_kernel(const float* __restrict__ psum,
+                                                           const int32_t* __restrict__ pcount, int n_blocks,
+                                                           int64_t T, int E, int K, float alpha,
+                                                           float* __restrict__ stats) {
+  __shared__ double s_p[1024];
+  __shared__ long long s_c[1024];
   __shared__ double s_fp[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    long long c = 0;
-    double s = 0.0;
-    for (int b = 0; b < n_blocks; ++b) {
+  int S = 1024 / E;
+  if (S > n_blocks) S = n_blocks;
+  if (S < 1) S = 1;
+  const int tid = threadIdx.x;
+  const int e = tid / S, s = tid - (tid / S) * S;
+  double ps = 0.0;
+  long long c = 0;
+  if (e < E) {
+    for (int b = s; b < n_blocks; b += S) {
       c += pcount[static_cast<int64_t>(b) * E + e];
-      s += static_cast<double>(psum[static_cast<int64_t>(b) * E + e]);
+      ps += static_cast<double>(psum[static_cast<int64_t>(b) * E + e]);
     }
-    const double f = static_cast<double>(c) / (static_cast<double>(T) * K);
-    const double P = s / static_cast<double>(T);
+  }
+  s_p[tid] = ps;
+  s_c[tid] = c;
+  __syncthreads();
+  if (e < E && s == 0) {
+    double P = 0.0;
+    long long n = 0;
+    for (int i = 0; i < S; ++i) {
+      P += s_p[tid + i];
+      n += s_c[tid + i];
+    }
+    const double f = static_cast<double>(n) / (static_cast<double>(T) * K);
+    P /= static_cast<double>(T);
     stats[e] = static_cast<float>(f);
     stats[E + e] = static_cast<float>(P);
     s_fp[e] = f * P;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (tid < 32) {  // loss: fixed-order warp reduction over experts
     double acc = 0.0;
-    for (int e = 0; e < E; ++e) acc += s_fp[e];
-    stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
+    for (int i = tid; i < E; i += 32) acc += s_fp[i];
+    acc = warp_sum(acc);
+    if (tid == 0) stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
   }
 }
 
 cudaError_t launch_route_stats(const Problem& p, const float* psum, const int32_t* pcount, int n_blocks,
                                float* stats, cudaStream_t st) {
-  route_stats_kernel<<<1, 256, 0, st>>>(psum, pcount, n_blocks, p.T, p.E, p.K, p.alpha, stats);
+  route_stats_kernel<<<1, 1024, 0, st>>>(psum, pcount, n_blocks, p.T, p.E, p.K, p.alpha, stats);
   return cudaGetLastError();
 }
 

@@ -65,6 +65,7 @@ def _route_given(cfg, logits32, sel_bias, flags=api.FLAG_LOGITS_GIVEN):
     idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
     w = torch.empty((T, K), dtype=torch.float32, device="cuda")
     stats = torch.empty(2 * E + 1, dtype=torch.float32, device="cuda")
+    api.reset_device_status(ws)
     api.moe_route(prob, None, None, None, dev(sel_bias), lg, idx, w, stats, ws)
     assert api.read_device_status(ws) == 0
     return idx.cpu().numpy(), w.cpu().numpy(), stats.cpu().numpy()
@@ -132,9 +133,6 @@ def test_gate_logits_match_oracle(name):
     want = oracle.gate_logits(host_np(inp["x"]), host_np(inp["w_gate"]), inp["logit_offset"])
     bound = (1e-5 if cfg.dtype == "f32" else 1e-3) * max(1.0, float(np.max(np.abs(want))))
     assert np.max(np.abs(got - want)) <= bound
-    # the GPU's own selection on its own logits: bit-exact against the oracle fed the same logits
-    ref = oracle_routing(cfg, got, inp["sel_bias"])
-    assert (idx.cpu().numpy() == ref["idx"]).all()
 
 
 # ------------------------------------------------------------------ dispatch
@@ -153,6 +151,7 @@ def test_dispatch_is_bit_exact(name):
     perm = torch.full((R,), -7, **i32)
     x = dev(inp["x"])
     x_perm = torch.zeros((R, cfg.d_model), dtype=x.dtype, device="cuda")
+    api.reset_device_status(ws)
     api.moe_dispatch(prob, dev(ref["idx"]), x, counts, kept, seg, slot_of, perm, x_perm, ws)
     assert api.read_device_status(ws) == 0
     assert (counts.cpu().numpy() == ref["counts"]).all()
@@ -204,6 +203,7 @@ def test_routed_expert_ffn_matches_oracle(name):
     x_rows = torch.zeros((R, cfg.d_model), dtype=x.dtype)
     x_rows[:S] = x[torch.as_tensor(tok)]
     y_rows = torch.zeros((R, cfg.d_model), dtype=x.dtype, device="cuda")
+    api.reset_device_status(ws)
     api.moe_expert_ffn(prob, api.FFN_ROUTED, dev(x_rows), R, dev(ref["seg_off"]), dev(inp["w13"]), dev(inp["w2"]),
                        y_rows, ws)
     assert api.read_device_status(ws) == 0
@@ -242,7 +242,7 @@ def test_shared_expert_ffn_matches_oracle(name):
 
 
 # ------------------------------------------------------------------ combine
-@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "ragged_f32", "tiny_capacity"])
+@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "ragged_f32", "ragged_bf16", "tiny_capacity"])
 def test_combine_matches_oracle(name):
     cfg = SMALL[name]
     inp = inputs(name)
