@@ -30,6 +30,8 @@
 // Every wait is bounded (see mbar_wait); on a timeout the kernel records
 // MOE_DEV_WAIT_TIMEOUT, drains its own copies and MMAs, frees TMEM and exits.
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -92,8 +94,8 @@ __device__ __forceinline__ int group_rows(const GemmArgs& a, int g, int* base) {
   return a.n_rows;
 }
 
-__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const GemmArgs& a, int n_tiles_n,
-                                                int out_cols) {
+template <int BM>
+__device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const GemmArgs& a, int out_cols) {
   int lo = 0, hi = a.n_groups - 1;
   while (lo < hi) {  // largest g with prefix[g] <= tile (that group is never empty)
     const int mid = (lo + hi + 1) >> 1;
@@ -103,15 +105,119 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   ti.g = lo;
   int base;
   const int rows = group_rows(a, lo, &base);
-  const int mt = (rows + kBM - 1) / kBM;
+  const int mt = (rows + BM - 1) / BM;
   const int local = tile - prefix[lo];
   const int n_idx = local / mt;
   const int m_idx = local - n_idx * mt;
-  ti.row0 = base + m_idx * kBM;
+  ti.row0 = base + m_idx * BM;
   ti.row_end = base + rows;
   ti.n0 = n_idx * out_cols;
-  (void)n_tiles_n;
   return ti;
+}
+
+// Tile prefix over groups (one warp): lane l owns groups [l*per, (l+1)*per).
+// prefix[g] = first tile of group g; prefix[n_groups] = total tiles.
+template <int BM>
+__device__ __forceinline__ void tile_prefix_warp(const GemmArgs& args, int n_tiles_n, int* prefix, int lane) {
+  const int per = (args.n_groups + 31) / 32;
+  int local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int g = lane * per + i;
+    if (g < args.n_groups) {
+      int base;
+      local += ((group_rows(args, g, &base) + BM - 1) / BM) * n_tiles_n;
+    }
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - local;
+  for (int i = 0; i < per; ++i) {
+    const int g = lane * per + i;
+    if (g < args.n_groups) {
+      prefix[g] = run;
+      int base;
+      run += ((group_rows(args, g, &base) + BM - 1) / BM) * n_tiles_n;
+    }
+  }
+  if (lane == 31) prefix[args.n_groups] = incl;
+}
+
+// Drain one accumulator (this warp's 32 TMEM lanes, BN columns starting at
+// t_row) and store the thread's row.  Every lane must call it (the TMEM loads
+// are warp-collective); row_ok masks only the stores.
+template <int EPI, int BN>
+__device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int row, bool row_ok, int n0,
+                                              uint32_t t_row) {
+  if (EPI == EPI_SWIGLU) {
+    __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
+                             static_cast<int64_t>(g) * args.out_col_stride;
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 32) {
+      uint32_t gr[32], ur[32];
+      tmem_load_32x32(t_row + c, gr);
+      tmem_load_32x32(t_row + BN / 2 + c, ur);
+      tmem_load_wait();
+      if (row_ok) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int col = n0 + c + q * 8;
+          if (col < args.N) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float g0 = __uint_as_float(gr[q * 8 + 2 * j]), g1 = __uint_as_float(gr[q * 8 + 2 * j + 1]);
+              const float u0 = __uint_as_float(ur[q * 8 + 2 * j]), u1 = __uint_as_float(ur[q * 8 + 2 * j + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+              pk[j] = pack_bf16x2(h0, h1);
+            }
+            *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+    }
+  } else if (EPI == EPI_BF16) {
+    __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
+                             static_cast<int64_t>(g) * args.out_col_stride;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t vr[32];
+      tmem_load_32x32(t_row + c, vr);
+      tmem_load_wait();
+      if (row_ok) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int col = n0 + c + q * 8;
+          if (col < args.N) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              pk[j] = pack_bf16x2(__uint_as_float(vr[q * 8 + 2 * j]), __uint_as_float(vr[q * 8 + 2 * j + 1]));
+            *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+    }
+  } else {
+    float* out_row = static_cast<float*>(args.out) + static_cast<int64_t>(row) * args.ldo;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t vr[32];
+      tmem_load_32x32(t_row + c, vr);
+      tmem_load_wait();
+      if (row_ok) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int col = c + j;
+          if (col < args.N) out_row[col] = __uint_as_float(vr[j]) + (args.col_add ? args.col_add[col] : 0.f);
+        }
+      }
+    }
+  }
 }
 
 template <int EPI, int BN, int STAGES>
@@ -157,36 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 2) {
-    // tile prefix over groups: lane l owns groups [l*per, (l+1)*per)
-    const int per = (args.n_groups + 31) / 32;
-    int local = 0;
-    for (int i = 0; i < per; ++i) {
-      const int g = lane * per + i;
-      if (g < args.n_groups) {
-        int base;
-        const int rows = group_rows(args, g, &base);
-        local += ((rows + kBM - 1) / kBM) * n_tiles_n;
-      }
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - local;
-    for (int i = 0; i < per; ++i) {
-      const int g = lane * per + i;
-      if (g < args.n_groups) {
-        prefix[g] = run;
-        int base;
-        const int rows = group_rows(args, g, &base);
-        run += ((rows + kBM - 1) / kBM) * n_tiles_n;
-      }
-    }
-    if (lane == 31) prefix[args.n_groups] = incl;
-  }
+  if (warp == 2) tile_prefix_warp<kBM>(args, n_tiles_n, prefix, lane);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -202,7 +279,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, prefix, args, n_tiles_n, C::kOutCols);
+        const TileInfo ti = decode_tile<kBM>(tile, prefix, args, C::kOutCols);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -285,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = quarter * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile(tile, prefix, args, n_tiles_n, C::kOutCols);
+      const TileInfo ti = decode_tile<kBM>(tile, prefix, args, C::kOutCols);
       const int acc = it & 1;
       const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
       // every lane waits; the result is made warp-uniform (and the warp
@@ -294,75 +371,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ready) break;
       tc_fence_after_sync();
       const int row = ti.row0 + r;
-      const bool row_ok = row < ti.row_end;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      if (EPI == EPI_SWIGLU) {
-        __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
-                                 static_cast<int64_t>(ti.g) * args.out_col_stride;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t gr[32], ur[32];
-          tmem_load_32x32(t_row + c, gr);
-          tmem_load_32x32(t_row + BN / 2 + c, ur);
-          tmem_load_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int col = ti.n0 + c + q * 8;
-              if (col < args.N) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const float g0 = __uint_as_float(gr[q * 8 + 2 * j]), g1 = __uint_as_float(gr[q * 8 + 2 * j + 1]);
-                  const float u0 = __uint_as_float(ur[q * 8 + 2 * j]), u1 = __uint_as_float(ur[q * 8 + 2 * j + 1]);
-                  const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-                  const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-                  pk[j] = pack_bf16x2(h0, h1);
-                }
-                *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
-            }
-          }
-        }
-      } else if (EPI == EPI_BF16) {
-        __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
-                                 static_cast<int64_t>(ti.g) * args.out_col_stride;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t vr[32];
-          tmem_load_32x32(t_row + c, vr);
-          tmem_load_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int col = ti.n0 + c + q * 8;
-              if (col < args.N) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  pk[j] = pack_bf16x2(__uint_as_float(vr[q * 8 + 2 * j]), __uint_as_float(vr[q * 8 + 2 * j + 1]));
-                *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
-            }
-          }
-        }
-      } else {
-        float* out_row = static_cast<float*>(args.out) + static_cast<int64_t>(row) * args.ldo;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t vr[32];
-          tmem_load_32x32(t_row + c, vr);
-          tmem_load_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int col = c + j;
-              if (col < args.N)
-                out_row[col] = __uint_as_float(vr[j]) + (args.col_add ? args.col_add[col] : 0.f);
-            }
-          }
-        }
-      }
+      epilogue_rows<EPI, BN>(args, ti.g, row, row < ti.row_end, ti.n0, t_row);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -375,6 +385,208 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ============================================================================
+// Pair kernel: the same grouped GEMM on CTA pairs (clusters of 2) with M=256
+// tiles.  Each CTA stages its own 128 A rows and HALF of the B tile (for
+// SwiGLU: CTA 0 the 128 gate rows, CTA 1 the 128 up rows; otherwise B rows
+// n0..n0+127 and n0+128..n0+255), so per FLOP each SM pulls 2/3 of the bytes
+// a 128x256 one-CTA tile needs.  The leader (rank 0) issues the MMAs for both
+// CTAs; every accumulator row lands in the TMEM of the CTA that owns it.
+//   full[s]   (leader)  one arrive (leader, with both CTAs' bytes) + TMA bytes
+//   empty[s]  (each)    one arrive from the leader's multicast commit
+//   tfull[a]  (each)    one arrive from the leader's multicast commit
+//   tempty[a] (leader)  8 arrives: 4 epilogue warps in each CTA
+// Tiles are 256 rows; a group with r rows spans ceil(r/256) row tiles.
+// ============================================================================
+constexpr int kPairBM = 256;
+constexpr int kPairBN = 256;  // MMA N: both halves of B
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = 128 * kBK * 2;
+constexpr int kPairBBytes = 128 * kBK * 2;  // this CTA's half of B
+constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
+
+constexpr int pair_smem_bytes() {
+  return kPairStages * kPairStageBytes + 256 + 4 * (kMaxGroups + 1) + 1024;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const GemmArgs args) {
+  constexpr int kOutCols = (EPI == EPI_SWIGLU) ? kPairBN / 2 : kPairBN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kPairStages * kPairABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  uint64_t* empty = full + kPairStages;
+  uint64_t* tfull = empty + kPairStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int n_tiles_n = (args.N + kOutCols - 1) / kOutCols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2) tile_prefix_warp<kPairBM>(args, n_tiles_n, prefix, lane);
+  tc_fence_before_sync();
+  cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total_tiles = prefix[args.n_groups];
+  const int nkb_g = (args.K + kBK - 1) / kBK;
+  const int nkb = nkb_g * args.k_groups;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint32_t full_leader = mapa_shared(smem_addr(&full[0]), 0);
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
+        const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int kg = kb / nkb_g;
+          const int kk = (kb - kg * nkb_g) * kBK;
+          const uint32_t bar = full_leader + static_cast<uint32_t>(stage * 8);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
+          tma_load_2d_pair(sA + stage * kPairABytes, &tmA, bar, kg * args.K + kk,
+                           ti.row0 + 128 * static_cast<int>(rank));
+          uint8_t* b_dst = sB + stage * kPairBBytes;
+          if (EPI == EPI_SWIGLU)
+            tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
+          else
+            tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank),
+                             ti.g * args.k_groups + kg);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (*abort_flag) {
+        int never = 0;
+        if (rank == 0) {  // the leader's full barriers count both CTAs' bytes
+          for (int s = 0; s < kPairStages; ++s)
+            if ((issued >> s) & 1u) mbar_wait(&full[s], (last_par >> s) & 1u, &never);
+        } else {  // the peer cannot observe its copies: give them a bounded time to land
+          const unsigned long long t0 = global_ns();
+          while (global_ns() - t0 < 1000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairBN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint64_t adesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes));
+          const uint64_t bdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes));
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k)
+            umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair_multicast(&empty[stage], 0x3);
+          if (++stage == kPairStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_multicast(&tfull[acc], 0x3);
+      }
+      if (*abort_flag) {
+        umma_commit_pair_multicast(drain, 0x1);
+        int never = 0;
+        mbar_wait(drain, 0, &never);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t tempty_leader = mapa_shared(smem_addr(&tempty[0]), 0);
+    int it = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs, ++it) {
+      const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
+      const int acc = it & 1;
+      const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_par, abort_flag));
+      if (!ready) break;
+      tc_fence_after_sync();
+      const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kPairBN);
+      epilogue_rows<EPI, kPairBN>(args, ti.g, row, row < ti.row_end, ti.n0, t_row);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(acc * 8));
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before_sync();
+  cluster_sync();  // no CTA leaves while its peer may still touch its shared memory or TMEM
+  if (threadIdx.x == 0 && *abort_flag) raise_status(args.status, kDevWaitTimeout);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 
@@ -442,7 +654,53 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
   return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
 
+template <int EPI>
+static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int64_t tile_bound,
+                         cudaStream_t st) {
+  constexpr int smem = pair_smem_bytes();
+  static std::mutex mu;
+  static int max_pairs[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -3;
+  int pairs;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (max_pairs[dev] == 0) {
+      if (cudaFuncSetAttribute(grouped_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return -3;
+      // a persistent grid must fit at once: ask how many 2-CTA clusters can be co-resident
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<EPI>, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms() / 2;
+      }
+      max_pairs[dev] = n;
+    }
+    pairs = max_pairs[dev];
+  }
+  if (tile_bound <= 0) return 0;
+  if (pairs > tile_bound) pairs = static_cast<int>(tile_bound);
+  grouped_gemm_pair_kernel<EPI><<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(ta, tb, a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Tile shape of the expert GEMMs: 256-row tiles on CTA pairs when groups are
+// expected to be large (small groups waste too much of a 256-row tile),
+// 128-row tiles on single CTAs otherwise.  MOE_B200_GEMM_TILE=128|256
+// forces one shape (both are complete implementations; used by the tests).
+static bool use_pair_tiles(int64_t expected_rows_per_group, int64_t threshold) {
+  const char* e = getenv("MOE_B200_GEMM_TILE");
+  if (e && !strcmp(e, "128")) return false;
+  if (e && !strcmp(e, "256")) return true;
+  return expected_rows_per_group >= threshold;
+}
 
 int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset,
                           float* logits, unsigned* status, cudaStream_t st) {
@@ -586,6 +844,11 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
   const bool routed = mode == 0;
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+  // routed loads are uneven (a skewed router leaves most experts far below the
+  // mean), so routed groups need a larger expected size than shared ones
+  int64_t expected = routed ? (p.T * p.K) / p.E : n_rows;
+  if (routed && p.cap >= 0 && p.cap < expected) expected = p.cap;
+  const bool pair = use_pair_tiles(expected, routed ? 768 : 512);
 
   // up/gate projection + SwiGLU: A = x_rows [n_rows, d], B = w13 viewed as (d, F, 2G)
   CUtensorMap ta, tb;
@@ -606,8 +869,11 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.ldo = h_cols;
     a.out_col_stride = routed ? 0 : p.F;
     a.status = status;
-    const int64_t m_tiles = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
-    const int rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, m_tiles * cdiv(p.F, 128), st);
+    const int rc = pair
+        ? run_pair_gemm<EPI_SWIGLU>(ta, tb, a, (routed ? cdiv(n_rows, kPairBM) + G : G * cdiv(n_rows, kPairBM)) *
+                                                   cdiv(p.F, 128), st)
+        : run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, (routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM)) *
+                                                      cdiv(p.F, 128), st);
     if (rc) return rc;
     if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
   }
@@ -616,7 +882,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint64_t da[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
-    const uint32_t bb[3] = {kBK, 256, 1};
+    const uint32_t bb[3] = {kBK, pair ? 128u : 256u, 1};  // a pair CTA stages half of the 256 B rows
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
     GemmArgs a{};
     a.n_groups = routed ? G : 1;
@@ -629,8 +895,11 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.ldo = p.d;
     a.out_col_stride = 0;
     a.status = status;
-    const int64_t m_tiles = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
-    const int rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, m_tiles * cdiv(p.d, 256), st);
+    const int rc = pair
+        ? run_pair_gemm<EPI_BF16>(ta, tb, a, (routed ? cdiv(n_rows, kPairBM) + G : cdiv(n_rows, kPairBM)) *
+                                                 cdiv(p.d, 256), st)
+        : run_gemm<EPI_BF16, 256, 4>(ta, tb, a, (routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM)) *
+                                                    cdiv(p.d, 256), st);
     if (rc) return rc;
   }
   return 0;

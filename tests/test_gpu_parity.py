@@ -334,3 +334,21 @@ def test_layer_stats_match_oracle_and_uniform_routing_gives_alpha():
     idx, w, stats = _route_given(cfg, np.zeros((96, 8), np.float32), None)
     assert np.allclose(stats[:8], 1 / 8, atol=0) and np.allclose(stats[8:16], 1 / 8, atol=1e-7)
     assert abs(stats[16] - 0.01) <= 1e-8
+
+
+# --------------------------------------------------- both GEMM tile shapes
+@pytest.mark.parametrize("tile", ["128", "256"])
+@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "ragged_bf16", "mini_skewed", "mini_decode"])
+def test_layer_forward_both_tile_shapes(name, tile, monkeypatch):
+    """The 128-row single-CTA and 256-row CTA-pair expert GEMMs, each forced,
+    against the oracle (the library picks one per problem size otherwise)."""
+    monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
+    cfg = SMALL[name]
+    inp = inputs(name)
+    logits32 = given_logits(cfg)
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN)
+    layer.routing["logits"].copy_(torch.as_tensor(logits32))
+    y = layer.forward(dev(inp["x"]))
+    assert api.read_device_status(layer.ws) == 0
+    assert rel_err(y.float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
