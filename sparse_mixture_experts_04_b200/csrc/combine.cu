@@ -41,12 +41,15 @@ struct Pack16<float> {
   }
 };
 
+// 2-D grid: blockIdx.x selects a chunk of kCombineVPT * blockDim.x vectors of
+// a row, blockIdx.y (grid-stride) the token.  A thread owns kCombineVPT
+// vectors kCombineThreads apart and issues all their loads before the
+// arithmetic, so many requests are in flight per thread; index math is 32-bit.
+// The token's (slot, weight) pairs are the same for every thread of the block
+// (broadcast loads).
 constexpr int kCombineThreads = 128;
-constexpr int kCombineVPT = 4;  // 16-byte vectors per thread per pass
+constexpr int kCombineVPT = 2;
 
-// One block per token (grid-stride).  The token's K (slot, weight) pairs are
-// staged in shared memory; each thread owns kCombineVPT vectors of the row and
-// issues all their loads before the arithmetic.
 template <typename T>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const T* __restrict__ y_perm,
                                                                   const int32_t* __restrict__ slot_of,
@@ -55,62 +58,55 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const T* __res
                                                                   T* __restrict__ y, int64_t Tn, int d, int K,
                                                                   int64_t n_perm_rows) {
   constexpr int V = Pack16<T>::N;
-  __shared__ int s_slot[kMaxTopK];
-  __shared__ float s_w[kMaxTopK];
   const int nvec = d / V;
-  for (int64_t t = blockIdx.x; t < Tn; t += gridDim.x) {
-    __syncthreads();
-    if (threadIdx.x < K) {
-      const int slot = slot_of[t * K + threadIdx.x];
-      s_slot[threadIdx.x] = (slot >= 0 && slot < n_perm_rows) ? slot : -1;
-      s_w[threadIdx.x] = topk_w[t * K + threadIdx.x];
+  const int v0 = blockIdx.x * (kCombineThreads * kCombineVPT) + threadIdx.x;
+  for (int64_t t = blockIdx.y; t < Tn; t += gridDim.y) {
+    float acc[kCombineVPT][V];
+#pragma unroll
+    for (int j = 0; j < kCombineVPT; ++j) {
+      const int v = v0 + j * kCombineThreads;
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[j][i] = 0.f;
+      if (y_shared && v < nvec) Pack16<T>::load(y_shared + t * d + v * V, acc[j]);
     }
-    __syncthreads();
-    for (int v0 = 0; v0 < nvec; v0 += kCombineThreads * kCombineVPT) {
-      float acc[kCombineVPT][V];
+    for (int k = 0; k < K; ++k) {
+      const int slot = slot_of[t * K + k];
+      if (slot < 0 || slot >= n_perm_rows) continue;
+      const float w = topk_w[t * K + k];
+      const T* row = y_perm + static_cast<int64_t>(slot) * d;
+      float r[kCombineVPT][V];
 #pragma unroll
       for (int j = 0; j < kCombineVPT; ++j) {
-        const int v = v0 + j * kCombineThreads + threadIdx.x;
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[j][i] = 0.f;
-        if (y_shared && v < nvec) Pack16<T>::load(y_shared + t * d + v * V, acc[j]);
-      }
-      for (int k = 0; k < K; ++k) {
-        const int slot = s_slot[k];
-        if (slot < 0) continue;
-        const float w = s_w[k];
-        const T* row = y_perm + static_cast<int64_t>(slot) * d;
-        float r[kCombineVPT][V];
-#pragma unroll
-        for (int j = 0; j < kCombineVPT; ++j) {
-          const int v = v0 + j * kCombineThreads + threadIdx.x;
-          if (v < nvec) Pack16<T>::load(row + v * V, r[j]);
-        }
-#pragma unroll
-        for (int j = 0; j < kCombineVPT; ++j)
-#pragma unroll
-          for (int i = 0; i < V; ++i) acc[j][i] = fmaf(w, r[j][i], acc[j][i]);
+        const int v = v0 + j * kCombineThreads;
+        if (v < nvec) Pack16<T>::load(row + v * V, r[j]);
       }
 #pragma unroll
-      for (int j = 0; j < kCombineVPT; ++j) {
-        const int v = v0 + j * kCombineThreads + threadIdx.x;
-        if (v < nvec) Pack16<T>::store(y + t * d + v * V, acc[j]);
-      }
+      for (int j = 0; j < kCombineVPT; ++j)
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[j][i] = fmaf(w, r[j][i], acc[j][i]);
+    }
+#pragma unroll
+    for (int j = 0; j < kCombineVPT; ++j) {
+      const int v = v0 + j * kCombineThreads;
+      if (v < nvec) Pack16<T>::store(y + t * d + v * V, acc[j]);
     }
   }
 }
 
 cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
                            const void* y_shared, void* y, cudaStream_t st) {
-  int64_t blocks = p.T;
-  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 32;
-  if (blocks > cap_blocks) blocks = cap_blocks;
+  const int V = p.dtype == kBF16 ? 8 : 4;
+  const int nvec = p.d / V;
+  const unsigned gx = static_cast<unsigned>((nvec + kCombineThreads * kCombineVPT - 1) / (kCombineThreads * kCombineVPT));
+  int64_t gy = p.T;
+  if (gy > 65535) gy = 65535;
+  const dim3 grid(gx, static_cast<unsigned>(gy));
   if (p.dtype == kBF16)
-    combine_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCombineThreads, 0, st>>>(
+    combine_kernel<__nv_bfloat16><<<grid, kCombineThreads, 0, st>>>(
         static_cast<const __nv_bfloat16*>(y_perm), slot_of, topk_w, static_cast<const __nv_bfloat16*>(y_shared),
         static_cast<__nv_bfloat16*>(y), p.T, p.d, p.K, p.max_rows);
   else
-    combine_kernel<float><<<static_cast<unsigned>(blocks), kCombineThreads, 0, st>>>(
+    combine_kernel<float><<<grid, kCombineThreads, 0, st>>>(
         static_cast<const float*>(y_perm), slot_of, topk_w, static_cast<const float*>(y_shared),
         static_cast<float*>(y), p.T, p.d, p.K, p.max_rows);
   return cudaGetLastError();

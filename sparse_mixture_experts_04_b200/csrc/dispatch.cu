@@ -168,14 +168,16 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
 
 cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
-                            int32_t* chunk_base, unsigned* status, cudaStream_t st) {
+                            int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready) {
   const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
-  dispatch_hist_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_counts, status);
+  if (!counts_ready) dispatch_hist_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_counts, status);
   dispatch_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, n_chunks, p.E, static_cast<long long>(p.cap),
                                            chunk_base, counts, kept, seg_off);
   dispatch_rank_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_base, kept, seg_off, slot_of, perm);
   return cudaGetLastError();
 }
+
+constexpr int kGatherUnroll = 8;
 
 // Row gather: one warp per destination row, 16-byte vectors.  Rows at or past
 // seg_off[E] (the kept total) are left untouched.
@@ -193,7 +195,16 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
     if (tok < 0 || tok >= T) continue;
     const uint4* src = x + tok * vec_per_row;
     uint4* dst = x_perm + r * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
+    // up to kGatherUnroll 16-byte loads in flight per lane before any store
+    for (int v0 = lane; v0 < vec_per_row; v0 += 32 * kGatherUnroll) {
+      uint4 buf[kGatherUnroll];
+#pragma unroll
+      for (int j = 0; j < kGatherUnroll; ++j)
+        if (v0 + 32 * j < vec_per_row) buf[j] = __ldg(src + v0 + 32 * j);
+#pragma unroll
+      for (int j = 0; j < kGatherUnroll; ++j)
+        if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = buf[j];
+    }
   }
 }
 

@@ -59,7 +59,26 @@ struct GemmArgs {
   int out_col_stride;  // output column offset per group
   const float* col_add;  // EPI_F32: per-column offset, or nullptr
   unsigned* status;
+  // split-K (EPI_F32 only): group g reduces k in [g*k_split, (g+1)*k_split)
+  // and writes its partial sums at out + g*out_group_stride (0: no split)
+  int k_split;
+  int64_t out_group_stride;
+  // which rows of each group this launch covers: 0 all, 1 the head (rows
+  // rounded down to a multiple of 256), 2 the tail (the rest)
+  int row_mode;
 };
+
+// Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
+__device__ __forceinline__ void tile_k_range(const GemmArgs& a, int g, int* k0, int* nkb) {
+  if (a.k_split > 0) {
+    *k0 = g * a.k_split;
+    const int len = min(a.K - *k0, a.k_split);
+    *nkb = (len + 63) / 64;
+  } else {
+    *k0 = 0;
+    *nkb = ((a.K + 63) / 64) * a.k_groups;
+  }
+}
 
 template <int EPI, int BN>
 struct TileCfg {
@@ -81,17 +100,23 @@ struct TileInfo {
   int g, row0, row_end, n0;
 };
 
-// Rows [base, base + return) of group g, clamped to the allocated rows
-// [0, n_rows) whatever seg_off holds, so no tile reads or writes outside them.
+// Rows [base, base + return) of group g (the part row_mode selects), clamped
+// to the allocated rows [0, n_rows) whatever seg_off holds, so no tile reads
+// or writes outside them.
 __device__ __forceinline__ int group_rows(const GemmArgs& a, int g, int* base) {
+  int b = 0, rows = a.n_rows;
   if (a.seg_off) {
-    const int b = min(max(a.seg_off[g], 0), a.n_rows);
-    const int e = min(max(a.seg_off[g + 1], b), a.n_rows);
-    *base = b;
-    return e - b;
+    b = min(max(a.seg_off[g], 0), a.n_rows);
+    rows = min(max(a.seg_off[g + 1], b), a.n_rows) - b;
   }
-  *base = 0;
-  return a.n_rows;
+  const int head = rows & ~255;
+  if (a.row_mode == 1) rows = head;
+  if (a.row_mode == 2) {
+    b += head;
+    rows -= head;
+  }
+  *base = b;
+  return rows;
 }
 
 template <int BM>
@@ -203,7 +228,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
       }
     }
   } else {
-    float* out_row = static_cast<float*>(args.out) + static_cast<int64_t>(row) * args.ldo;
+    float* out_row = static_cast<float*>(args.out) + static_cast<int64_t>(g) * args.out_group_stride +
+                     static_cast<int64_t>(row) * args.ldo;
+    const float* add = (g == 0) ? args.col_add : nullptr;  // a split-K offset goes into slice 0 only
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t vr[32];
@@ -213,7 +240,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int col = c + j;
-          if (col < args.N) out_row[col] = __uint_as_float(vr[j]) + (args.col_add ? args.col_add[col] : 0.f);
+          if (col < args.N) out_row[col] = __uint_as_float(vr[j]) + (add ? add[col] : 0.f);
         }
       }
     }
@@ -270,7 +297,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = prefix[args.n_groups];
   const int nkb_g = (args.K + kBK - 1) / kBK;
-  const int nkb = nkb_g * args.k_groups;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -280,13 +306,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         const TileInfo ti = decode_tile<kBM>(tile, prefix, args, C::kOutCols);
+        int k0, nkb;
+        tile_k_range(args, ti.g, &k0, &nkb);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           const int kg = kb / nkb_g;
-          const int kk = (kb - kg * nkb_g) * kBK;
+          const int kk = k0 + (kb - kg * nkb_g) * kBK;
           uint8_t* a_dst = sA + stage * C::kABytes;
           uint8_t* b_dst = sB + stage * C::kBBytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
@@ -324,6 +352,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+        int k0, nkb;
+        tile_k_range(args, decode_tile<kBM>(tile, prefix, args, C::kOutCols).g, &k0, &nkb);
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -465,7 +495,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = prefix[args.n_groups];
   const int nkb_g = (args.K + kBK - 1) / kBK;
-  const int nkb = nkb_g * args.k_groups;
+  const int nkb = nkb_g * args.k_groups;  // no split-K on the pair path
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -691,19 +721,47 @@ static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Tile shape of the expert GEMMs: 256-row tiles on CTA pairs when groups are
-// expected to be large (small groups waste too much of a 256-row tile),
-// 128-row tiles on single CTAs otherwise.  MOE_B200_GEMM_TILE=128|256
-// forces one shape (both are complete implementations; used by the tests).
-static bool use_pair_tiles(int64_t expected_rows_per_group, int64_t threshold) {
+// Tile shape of the expert GEMMs:
+//   single     128-row tiles on single CTAs
+//   pair+tail  each group's rows rounded down to a multiple of 256 as 256-row
+//              tiles on CTA pairs, the rest (under 256 rows) as 128-row tiles
+//              on single CTAs (second launch): padding as with 128-row tiles
+//   pair       every group on 256-row pair tiles (padding up to 255 rows)
+// Measured choice: routed groups use the pure pair shape when they are large
+// (>= 768 expected rows) and the load is not skewed by a logit offset or a
+// selection bias, single CTAs otherwise; shared experts (every token, so the
+// rows are known) use pair+tail from 512 rows.
+// MOE_B200_GEMM_TILE=128|256|256all forces single, pair+tail or pair (all
+// complete implementations; the tests run each).
+enum TileMode { kTileSingle = 0, kTilePairTail = 1, kTilePair = 2 };
+
+static int tile_mode(int64_t expected_rows_per_group, bool routed, bool skewed) {
   const char* e = getenv("MOE_B200_GEMM_TILE");
-  if (e && !strcmp(e, "128")) return false;
-  if (e && !strcmp(e, "256")) return true;
-  return expected_rows_per_group >= threshold;
+  if (e && !strcmp(e, "128")) return kTileSingle;
+  if (e && !strcmp(e, "256")) return kTilePairTail;
+  if (e && !strcmp(e, "256all")) return kTilePair;
+  if (!routed) return expected_rows_per_group >= 512 ? kTilePairTail : kTileSingle;
+  return (expected_rows_per_group >= 768 && !skewed) ? kTilePair : kTileSingle;
 }
 
-int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset,
-                          float* logits, unsigned* status, cudaStream_t st) {
+int router_k_splits(const Problem& p) {
+  // as many slices as keep every (row tile, slice) in one wave of CTAs
+  const int64_t tiles = cdiv(p.T, kBM);
+  int64_t s = num_sms() / tiles;
+  const int64_t max_by_k = p.d / 256;  // keep at least four 64-wide k-blocks per slice
+  if (s > max_by_k) s = max_by_k;
+  if (s > 8) s = 8;
+  if (s < 1) s = 1;
+  const int64_t len = cdiv(cdiv(p.d, s), kBK) * kBK;
+  return static_cast<int>(cdiv(p.d, len));
+}
+
+// Gate logits on the tensor cores: A = x [T, d], B = w_gate [E, d] padded to
+// BN rows.  With n_splits > 1 the reduction over d is split into slices; slice
+// s writes its partial logits at out + s*T*E (the offset goes into slice 0) and
+// the selection kernel adds the slices in order.
+int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset, float* out,
+                          int n_splits, unsigned* status, cudaStream_t st) {
   CUtensorMap ta, tb;
   const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.T)};
   const uint32_t ba[2] = {kBK, kBM};
@@ -713,18 +771,20 @@ int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, c
   const uint32_t bb[3] = {kBK, static_cast<uint32_t>(bn), 1};
   if (!make_map(&tb, w_gate, 3, db, bb)) return -3;
   GemmArgs a{};
-  a.n_groups = 1;
+  a.n_groups = n_splits;
   a.seg_off = nullptr;
   a.n_rows = static_cast<int>(p.T);
   a.N = p.E;
   a.K = p.d;
   a.k_groups = 1;
-  a.out = logits;
+  a.out = out;
   a.ldo = p.E;
   a.out_col_stride = 0;
   a.col_add = offset;
   a.status = status;
-  const int64_t tiles = cdiv(p.T, kBM);
+  a.k_split = n_splits > 1 ? static_cast<int>(cdiv(cdiv(p.d, n_splits), kBK) * kBK) : 0;
+  a.out_group_stride = p.T * p.E;
+  const int64_t tiles = cdiv(p.T, kBM) * n_splits;
   switch (bn) {
     case 32: return run_gemm<EPI_F32, 32, 8>(ta, tb, a, tiles, st);
     case 64: return run_gemm<EPI_F32, 64, 8>(ta, tb, a, tiles, st);
@@ -839,8 +899,10 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status, cudaStream_t st,
                       cudaEvent_t after_up, int* n_kernels) {
   if (n_rows <= 0) return 0;
-  if (n_kernels) *n_kernels += 2;
-  if (p.dtype == kF32) return ffn_simt(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, st, after_up);
+  if (p.dtype == kF32) {
+    if (n_kernels) *n_kernels += 2;
+    return ffn_simt(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, st, after_up);
+  }
   const bool routed = mode == 0;
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
@@ -848,7 +910,10 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
   // mean), so routed groups need a larger expected size than shared ones
   int64_t expected = routed ? (p.T * p.K) / p.E : n_rows;
   if (routed && p.cap >= 0 && p.cap < expected) expected = p.cap;
-  const bool pair = use_pair_tiles(expected, routed ? 768 : 512);
+  const int mode_t = tile_mode(expected, routed, p.skewed_load);
+  const bool pair = mode_t != kTileSingle;
+  const bool tail = mode_t == kTilePairTail;
+  if (n_kernels) *n_kernels += tail ? 4 : 2;
 
   // up/gate projection + SwiGLU: A = x_rows [n_rows, d], B = w13 viewed as (d, F, 2G)
   CUtensorMap ta, tb;
@@ -869,12 +934,20 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.ldo = h_cols;
     a.out_col_stride = routed ? 0 : p.F;
     a.status = status;
-    const int rc = pair
-        ? run_pair_gemm<EPI_SWIGLU>(ta, tb, a, (routed ? cdiv(n_rows, kPairBM) + G : G * cdiv(n_rows, kPairBM)) *
-                                                   cdiv(p.F, 128), st)
-        : run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, (routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM)) *
-                                                      cdiv(p.F, 128), st);
-    if (rc) return rc;
+    const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
+    if (pair) {
+      a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
+      int rc = run_pair_gemm<EPI_SWIGLU>(ta, tb, a, (mt / 2 + G) * cdiv(p.F, 128), st);
+      if (rc) return rc;
+      if (tail) {
+        a.row_mode = 2;  // the rest (under 256 rows per group) on single CTAs
+        rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, 2 * G * cdiv(p.F, 128), st);
+        if (rc) return rc;
+      }
+    } else {
+      const int rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, mt * cdiv(p.F, 128), st);
+      if (rc) return rc;
+    }
     if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
   }
   // down projection: A = h [n_rows, k_groups * F], B = w2 viewed as (F, d, G)
@@ -882,8 +955,11 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint64_t da[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
-    const uint32_t bb[3] = {kBK, pair ? 128u : 256u, 1};  // a pair CTA stages half of the 256 B rows
+    const uint32_t bb[3] = {kBK, 256, 1};
+    const uint32_t bb_half[3] = {kBK, 128, 1};  // a pair CTA stages half of the 256 B rows
+    CUtensorMap tb_half;
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
+    if (pair && !make_map(&tb_half, w2, 3, db, bb_half)) return -3;
     GemmArgs a{};
     a.n_groups = routed ? G : 1;
     a.seg_off = routed ? seg_off : nullptr;
@@ -895,12 +971,20 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.ldo = p.d;
     a.out_col_stride = 0;
     a.status = status;
-    const int rc = pair
-        ? run_pair_gemm<EPI_BF16>(ta, tb, a, (routed ? cdiv(n_rows, kPairBM) + G : cdiv(n_rows, kPairBM)) *
-                                                 cdiv(p.d, 256), st)
-        : run_gemm<EPI_BF16, 256, 4>(ta, tb, a, (routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM)) *
-                                                    cdiv(p.d, 256), st);
-    if (rc) return rc;
+    const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
+    if (pair) {
+      a.row_mode = tail ? 1 : 0;
+      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, a, (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
+      if (rc) return rc;
+      if (tail) {
+        a.row_mode = 2;
+        rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.d, 256), st);
+        if (rc) return rc;
+      }
+    } else {
+      const int rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, mt * cdiv(p.d, 256), st);
+      if (rc) return rc;
+    }
   }
   return 0;
 }

@@ -11,7 +11,7 @@ namespace moe {
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 32;
 constexpr int kDispatchChunk = 256;  // tokens per block in the dispatch kernels
-constexpr int kSelectTokens = 32;    // tokens per block in the selection kernel (4 per warp)
+constexpr int kSelectTokens = 8;     // tokens per block in the selection kernel (one per warp)
 
 enum Dtype { kBF16 = 0, kF32 = 1 };
 
@@ -24,13 +24,14 @@ struct Problem {
   int dtype;
   uint32_t flags;
   float alpha;
+  bool skewed_load;  // the router has a logit offset or selection bias: expect uneven expert loads
   size_t esize() const { return dtype == kBF16 ? 2 : 4; }
 };
 
 // Byte offsets of every scratch array inside the caller's workspace.
 struct WsLayout {
   size_t status, logits, topk_idx, topk_w, counts, kept, seg_off, slot_of, perm;
-  size_t chunk_counts, chunk_base, sel_psum, sel_count;
+  size_t chunk_counts, chunk_base, sel_psum, sel_count, logit_parts, stats_scratch;
   size_t x_perm, h_routed, y_perm, h_shared, y_shared;
   size_t total;
   int n_chunks, n_sel_blocks;
@@ -40,22 +41,31 @@ WsLayout make_layout(const Problem& p);
 // router.cu
 cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void* w_gate,
                                     const float* offset, float* logits, cudaStream_t st);
-cudaError_t launch_route_select(const Problem& p, const float* logits, const float* sel_bias,
-                                int32_t* topk_idx, float* topk_w, float* psum, int32_t* pcount,
-                                unsigned* status, cudaStream_t st);
+// logits [T, E] are read, or (n_parts > 0) summed from n_parts slices at
+// parts + s*T*E in slice order and written to logits.
+// chunk_counts (or nullptr): zeroed [n_chunks, E] array that receives the
+// per-dispatch-chunk expert histogram of the chosen experts (integer atomics)
+cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
+                                const float* sel_bias, int32_t* topk_idx, float* topk_w, float* psum,
+                                int32_t* pcount, unsigned* stats_ticket, int32_t* chunk_counts,
+                                cudaStream_t st);
+// scratch: E doubles + one ticket word (zeroed by the selection kernel)
 cudaError_t launch_route_stats(const Problem& p, const float* psum, const int32_t* pcount, int n_blocks,
-                               float* stats, cudaStream_t st);
+                               float* stats, void* scratch, cudaStream_t st);
 
 // dispatch.cu
+// counts_ready: chunk_counts already hold the per-chunk expert histogram (the
+// selection kernel adds it when given a zeroed chunk_counts)
 cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
-                            int32_t* chunk_base, unsigned* status, cudaStream_t st);
+                            int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready = false);
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
                           void* x_perm, cudaStream_t st);
 
 // expert_gemm.cu -- returns a moe_status value
-int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset,
-                          float* logits, unsigned* status, cudaStream_t st);
+int router_k_splits(const Problem& p);  // slices of the tensor-core gate GEMM's reduction
+int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset, float* out,
+                          int n_splits, unsigned* status, cudaStream_t st);
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
                       cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr);

@@ -41,7 +41,9 @@ WsLayout make_layout(const Problem& p) {
     off = align256(off + (bytes ? bytes : 1));
     return o;
   };
-  L.status = take(256);
+  L.status = 0;  // status word, then the chunk histogram: one memset clears both
+  L.chunk_counts = 256;
+  off = align256(256 + static_cast<size_t>(L.n_chunks) * p.E * 4);
   L.logits = take(static_cast<size_t>(p.T) * p.E * 4);
   L.topk_idx = take(TK * 4);
   L.topk_w = take(TK * 4);
@@ -50,10 +52,12 @@ WsLayout make_layout(const Problem& p) {
   L.seg_off = take(static_cast<size_t>(p.E + 1) * 4);
   L.slot_of = take(TK * 4);
   L.perm = take(R * 4);
-  L.chunk_counts = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
   L.chunk_base = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
   L.sel_psum = take(static_cast<size_t>(L.n_sel_blocks) * p.E * 4);
   L.sel_count = take(static_cast<size_t>(L.n_sel_blocks) * p.E * 4);
+  const int splits = (p.dtype == kBF16) ? router_k_splits(p) : 1;
+  L.logit_parts = take(splits > 1 ? static_cast<size_t>(splits) * p.T * p.E * 4 : 0);
+  L.stats_scratch = take(kMaxExperts * 8 + 16);
   L.x_perm = take(R * p.d * es);
   L.h_routed = take(R * p.F * es);
   L.y_perm = take(R * p.d * es);
@@ -121,11 +125,18 @@ static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_C
 // Router body shared by moe_route and moe_layer_forward.
 static int route_impl(const Problem& p, const void* x, const void* w_gate, const float* offset,
                       const float* sel_bias, float* logits, int32_t* idx, float* w, float* stats, void* ws,
-                      const WsLayout& L, cudaStream_t st) {
+                      const WsLayout& L, cudaStream_t st, int32_t* chunk_counts = nullptr) {
   unsigned* status = at<unsigned>(ws, L.status);
+  int n_parts = 0;
+  float* parts = nullptr;
   if (!(p.flags & MOE_FLAG_LOGITS_GIVEN)) {
     if (p.dtype == kBF16) {
-      const int rc = launch_gate_logits_tc(p, x, w_gate, offset, logits, status, st);
+      const int splits = router_k_splits(p);
+      if (splits > 1) {
+        parts = at<float>(ws, L.logit_parts);
+        n_parts = splits;
+      }
+      const int rc = launch_gate_logits_tc(p, x, w_gate, offset, splits > 1 ? parts : logits, splits, status, st);
       if (rc) return MOE_ERR_CUDA;
     } else {
       if (cudaError_t e = launch_gate_logits_simt(p, x, w_gate, offset, logits, st)) return cuda_rc(e);
@@ -133,10 +144,14 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
   }
   float* psum = at<float>(ws, L.sel_psum);
   int32_t* pcount = at<int32_t>(ws, L.sel_count);
-  if (cudaError_t e = launch_route_select(p, logits, sel_bias, idx, w, psum, pcount, status, st))
+  double* stats_fp = at<double>(ws, L.stats_scratch);
+  unsigned* ticket = reinterpret_cast<unsigned*>(stats_fp + kMaxExperts);
+  if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, psum, pcount,
+                                          stats ? ticket : nullptr, chunk_counts, st))
     return cuda_rc(e);
   if (stats) {
-    if (cudaError_t e = launch_route_stats(p, psum, pcount, L.n_sel_blocks, stats, st)) return cuda_rc(e);
+    if (cudaError_t e = launch_route_stats(p, psum, pcount, L.n_sel_blocks, stats, stats_fp, st))
+      return cuda_rc(e);
   }
   return MOE_OK;
 }
@@ -275,6 +290,7 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     return MOE_ERR_INVALID_ARG;
   if (p.Ns == 0 && (w->w13_shared || w->w2_shared)) return MOE_ERR_INVALID_ARG;
 
+  p.skewed_load = (!given && w->logit_offset) || w->sel_bias;
   const WsLayout L = make_layout(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t {
@@ -297,17 +313,20 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   void* y_perm = at<void>(ws, L.y_perm);
   void* y_sh = p.Ns > 0 ? at<void>(ws, L.y_shared) : nullptr;
 
-  if (cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st)) return cuda_rc(e);
+  // status word and chunk histogram (contiguous at the start of ws) start at zero
+  if (cudaError_t e = cudaMemsetAsync(ws, 0, L.chunk_counts + static_cast<size_t>(L.n_chunks) * p.E * 4, st))
+    return cuda_rc(e);
   if (cudaError_t e = mark(MOE_EV_START)) return cuda_rc(e);
+  int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
   if (int rc = route_impl(p, x, w->w_gate, given ? nullptr : w->logit_offset, w->sel_bias, logits, idx, gw, stats,
-                          ws, L, st))
+                          ws, L, st, chunk_counts))
     return rc;
   kernels += (given ? 0 : 1) + 1 + (stats ? 1 : 0);
   if (cudaError_t e = mark(MOE_EV_ROUTED)) return cuda_rc(e);
-  if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, at<int32_t>(ws, L.chunk_counts),
-                                      at<int32_t>(ws, L.chunk_base), status, st))
+  if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, chunk_counts,
+                                      at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true))
     return cuda_rc(e);
-  kernels += 3;
+  kernels += 2;
   if (p.max_rows > 0) {
     if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
     kernels += 1;

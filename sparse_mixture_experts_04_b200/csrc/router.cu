@@ -139,12 +139,15 @@ cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void*
 // times each expert was chosen (integer), for the balance statistics.
 // ----------------------------------------------------------------------------
 template <int EPL>
-__global__ void __launch_bounds__(256) route_select_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ logits,
+                                                           const float* __restrict__ parts, int n_parts,
                                                            const float* __restrict__ sel_bias, int bias_on_logit,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ topk_w, float* __restrict__ psum,
                                                            int32_t* __restrict__ pcount, int64_t T, int E,
-                                                           int K) {
+                                                           int K, unsigned* stats_ticket,
+                                                           int32_t* __restrict__ chunk_counts) {
+  if (stats_ticket && blockIdx.x == 0 && threadIdx.x == 0) *stats_ticket = 0u;  // for route_stats_kernel
   __shared__ float s_psum[8][32 * EPL];
   __shared__ int s_count[32 * EPL];
   const int lane = threadIdx.x & 31;
@@ -166,7 +169,18 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      lg[i] = (e < E) ? logits[t * E + e] : -INFINITY;
+      if (e < E) {
+        if (n_parts > 0) {  // split-K gate GEMM: add the slices in order
+          float v = 0.f;
+          for (int sl = 0; sl < n_parts; ++sl) v += parts[static_cast<int64_t>(sl) * T * E + t * E + e];
+          logits[t * E + e] = v;
+          lg[i] = v;
+        } else {
+          lg[i] = logits[t * E + e];
+        }
+      } else {
+        lg[i] = -INFINITY;
+      }
       mloc = fmaxf(mloc, lg[i]);
     }
     const float m = warp_max(mloc);
@@ -273,26 +287,31 @@ __global__ void __launch_bounds__(256) route_select_kernel(const float* __restri
     for (int w = 0; w < 8; ++w) s += s_psum[w][e];
     psum[static_cast<int64_t>(blockIdx.x) * E + e] = s;
     pcount[static_cast<int64_t>(blockIdx.x) * E + e] = s_count[e];
+    // this block's tokens all lie in one dispatch chunk (kDispatchChunk is a
+    // multiple of kSelectTokens); integer adds commute, so the total is exact
+    if (chunk_counts && s_count[e])
+      atomicAdd(&chunk_counts[(tok_begin / kDispatchChunk) * E + e], s_count[e]);
   }
 }
 
-cudaError_t launch_route_select(const Problem& p, const float* logits, const float* sel_bias, int32_t* topk_idx,
-                                float* topk_w, float* psum, int32_t* pcount, unsigned* /*status*/,
+cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
+                                const float* sel_bias, int32_t* topk_idx, float* topk_w, float* psum,
+                                int32_t* pcount, unsigned* stats_ticket, int32_t* chunk_counts,
                                 cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>((p.T + kSelectTokens - 1) / kSelectTokens);
   const int bias_on_logit = (p.flags & 0x2u) ? 1 : 0;
   if (p.E <= 32)
-    route_select_kernel<1><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K);
+    route_select_kernel<1><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
   else if (p.E <= 64)
-    route_select_kernel<2><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K);
+    route_select_kernel<2><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
   else if (p.E <= 128)
-    route_select_kernel<4><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K);
+    route_select_kernel<4><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
   else
-    route_select_kernel<8><<<blocks, 256, 0, st>>>(logits, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K);
+    route_select_kernel<8><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
+                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
   return cudaGetLastError();
 }
 
@@ -300,58 +319,66 @@ cudaError_t launch_route_select(const Problem& p, const float* logits, const flo
 // Balance statistics from the per-block partials:
 //   f_e = count_e / (T K),  P_e = (1/T) sum_t p[t,e],  loss = alpha E sum_e f_e P_e
 // stats layout: [f_0 .. f_{E-1}, P_0 .. P_{E-1}, loss].
-// One block of 1024 threads: thread (e, s) sums every S-th block partial of
-// expert e; the S sub-sums are then added in a fixed order, so the result
-// does not depend on scheduling.
+// One block per expert: each thread sums a fixed stride of the partials, then
+// a fixed-shape tree adds the threads' sums, so the result does not depend on
+// scheduling.  The block that finishes last (ticket) adds the E products in
+// expert order for the loss; the ticket is zeroed by the selection kernel.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) route_stats_kernel(const float* __restrict__ psum,
-                                                           const int32_t* __restrict__ pcount, int n_blocks,
-                                                           int64_t T, int E, int K, float alpha,
-                                                           float* __restrict__ stats) {
-  __shared__ double s_p[1024];
-  __shared__ long long s_c[1024];
-  __shared__ double s_fp[kMaxExperts];
-  int S = 1024 / E;
-  if (S > n_blocks) S = n_blocks;
-  if (S < 1) S = 1;
+static_assert(kDispatchChunk % kSelectTokens == 0, "a selection block must not straddle dispatch chunks");
+constexpr int kStatsThreads = 256;
+
+__global__ void __launch_bounds__(kStatsThreads) route_stats_kernel(const float* __restrict__ psum,
+                                                                    const int32_t* __restrict__ pcount,
+                                                                    int n_blocks, int64_t T, int E, int K,
+                                                                    float alpha, float* __restrict__ stats,
+                                                                    double* __restrict__ fp,
+                                                                    unsigned* __restrict__ ticket) {
+  __shared__ double s_p[kStatsThreads];
+  __shared__ long long s_c[kStatsThreads];
+  __shared__ bool s_last;
+  const int e = blockIdx.x;
   const int tid = threadIdx.x;
-  const int e = tid / S, s = tid - (tid / S) * S;
   double ps = 0.0;
   long long c = 0;
-  if (e < E) {
-    for (int b = s; b < n_blocks; b += S) {
-      c += pcount[static_cast<int64_t>(b) * E + e];
-      ps += static_cast<double>(psum[static_cast<int64_t>(b) * E + e]);
-    }
+  for (int b = tid; b < n_blocks; b += kStatsThreads) {
+    c += pcount[static_cast<int64_t>(b) * E + e];
+    ps += static_cast<double>(psum[static_cast<int64_t>(b) * E + e]);
   }
   s_p[tid] = ps;
   s_c[tid] = c;
   __syncthreads();
-  if (e < E && s == 0) {
-    double P = 0.0;
-    long long n = 0;
-    for (int i = 0; i < S; ++i) {
-      P += s_p[tid + i];
-      n += s_c[tid + i];
+#pragma unroll
+  for (int w = kStatsThreads / 2; w > 0; w >>= 1) {
+    if (tid < w) {
+      s_p[tid] += s_p[tid + w];
+      s_c[tid] += s_c[tid + w];
     }
-    const double f = static_cast<double>(n) / (static_cast<double>(T) * K);
-    P /= static_cast<double>(T);
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const double f = static_cast<double>(s_c[0]) / (static_cast<double>(T) * K);
+    const double P = s_p[0] / static_cast<double>(T);
     stats[e] = static_cast<float>(f);
     stats[E + e] = static_cast<float>(P);
-    s_fp[e] = f * P;
+    fp[e] = f * P;
+    __threadfence();
+    s_last = atomicAdd(ticket, 1u) == static_cast<unsigned>(E - 1);
   }
   __syncthreads();
-  if (tid < 32) {  // loss: fixed-order warp reduction over experts
+  if (s_last && tid == 0) {
+    __threadfence();
     double acc = 0.0;
-    for (int i = tid; i < E; i += 32) acc += s_fp[i];
-    acc = warp_sum(acc);
-    if (tid == 0) stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
+    for (int i = 0; i < E; ++i) acc += static_cast<volatile double*>(fp)[i];
+    stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
   }
 }
 
 cudaError_t launch_route_stats(const Problem& p, const float* psum, const int32_t* pcount, int n_blocks,
-                               float* stats, cudaStream_t st) {
-  route_stats_kernel<<<1, 1024, 0, st>>>(psum, pcount, n_blocks, p.T, p.E, p.K, p.alpha, stats);
+                               float* stats, void* scratch, cudaStream_t st) {
+  double* fp = static_cast<double*>(scratch);
+  unsigned* ticket = reinterpret_cast<unsigned*>(fp + kMaxExperts);
+  route_stats_kernel<<<p.E, kStatsThreads, 0, st>>>(psum, pcount, n_blocks, p.T, p.E, p.K, p.alpha, stats, fp,
+                                                   ticket);
   return cudaGetLastError();
 }
 

@@ -337,7 +337,7 @@ def test_layer_stats_match_oracle_and_uniform_routing_gives_alpha():
 
 
 # --------------------------------------------------- both GEMM tile shapes
-@pytest.mark.parametrize("tile", ["128", "256"])
+@pytest.mark.parametrize("tile", ["128", "256", "256all"])
 @pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "ragged_bf16", "mini_skewed", "mini_decode"])
 def test_layer_forward_both_tile_shapes(name, tile, monkeypatch):
     """The 128-row single-CTA and 256-row CTA-pair expert GEMMs, each forced,
