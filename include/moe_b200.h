@@ -227,6 +227,25 @@ int moe_layer_forward(const moe_problem_t* p, const void* x, const moe_weights_t
                       void* y, const moe_routing_t* routing, float* stats,
                       void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_dispatch for callers that cannot give the library device memory for
+ * scratch: a program whose device-memory budget is fixed up front (all of it
+ * owned by its own pool or planner), or a host without a caching allocator,
+ * for which a cudaMalloc / cudaFree around each call would synchronise the
+ * device.  Same inputs, outputs and results as moe_dispatch, without ws: the
+ * scratch (per-chunk histogram and chunk bases) lives in a 1 MiB array of
+ * device memory that the library declares, which every GPU that loads the
+ * library holds until the process exits.  Limit: 2 * ceil(T/256) * E <= 262144
+ * (e.g. T <= 131072 at E = 256, T <= 524288 at E = 64); larger problems return
+ * MOE_ERR_UNSUPPORTED and enqueue nothing.  All calls on a GPU share the array:
+ * calls whose work overlaps on the GPU race, so serialise them.  The first call
+ * on a device looks the array's address up (device current); make it before
+ * any stream capture.  Expert indices outside [0, E) are skipped (slot -1) but
+ * not reported (there is no status word).  The pages have no counterpart of
+ * this entry point. */
+int moe_dispatch_noalloc(const moe_problem_t* p, const int32_t* topk_idx, const void* x,
+                         int32_t* counts, int32_t* kept, int32_t* seg_off,
+                         int32_t* slot_of, int32_t* perm, void* x_perm, moe_stream_t stream);
+
 /* Stage boundaries recorded by moe_layer_forward_profiled. */
 #define MOE_EV_START 0   /* before the router */
 #define MOE_EV_ROUTED 1  /* after gate logits, selection and statistics */

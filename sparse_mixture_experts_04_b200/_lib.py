@@ -22,7 +22,8 @@ DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
 # every symbol include/moe_b200.h declares
 EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
             "moe_reset_device_status", "moe_read_device_status", "moe_route", "moe_dispatch",
-            "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled")
+            "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
+            "moe_dispatch_noalloc")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
 
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_forward_profiled.argtypes = [PP, P, ctypes.POINTER(MoeWeights), P, ctypes.POINTER(MoeRouting), P,
                                              P, sz, P, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(i32)]
     L.moe_layer_forward_profiled.restype = ctypes.c_int
+    L.moe_dispatch_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P]
+    L.moe_dispatch_noalloc.restype = ctypes.c_int
     _lib = L
     return L
 

@@ -16,7 +16,7 @@ from ._lib import (DTYPE_BF16, DTYPE_F32, FFN_ROUTED, FFN_SHARED, FLAG_BIAS_LOGI
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-           "moe_layer_forward_profiled",
+           "moe_layer_forward_profiled", "moe_dispatch_noalloc",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
            "FFN_ROUTED", "FFN_SHARED", "DTYPE_BF16", "DTYPE_F32"]
 
@@ -87,6 +87,14 @@ def moe_dispatch(prob, topk_idx, x, counts, kept, seg_off, slot_of, perm, x_perm
     rc = _lib.lib().moe_dispatch(ctypes.byref(prob), _p(topk_idx), _p(x), _p(counts), _p(kept), _p(seg_off),
                                  _p(slot_of), _p(perm), _p(x_perm), _p(ws), ws.numel(), _stream(stream))
     _lib.check("moe_dispatch", rc)
+
+
+def moe_dispatch_noalloc(prob, topk_idx, x, counts, kept, seg_off, slot_of, perm, x_perm, stream=None):
+    """moe_dispatch without a workspace, for callers that cannot provide device
+    scratch memory (the library's own fixed array is used; see the header)."""
+    rc = _lib.lib().moe_dispatch_noalloc(ctypes.byref(prob), _p(topk_idx), _p(x), _p(counts), _p(kept),
+                                         _p(seg_off), _p(slot_of), _p(perm), _p(x_perm), _stream(stream))
+    _lib.check("moe_dispatch_noalloc", rc)
 
 
 def moe_expert_ffn(prob, mode, x_rows, n_rows, seg_off, w13, w2, y_rows, ws, stream=None):

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+struct moe_problem;  // include/moe_b200.h
+
 namespace moe {
 
 constexpr int kMaxExperts = 256;
@@ -37,6 +39,9 @@ struct WsLayout {
   int n_chunks, n_sel_blocks;
 };
 WsLayout make_layout(const Problem& p);
+
+// The ABI problem validated and converted (cap, max_rows derived); a moe_status.
+int problem_from_abi(const ::moe_problem* in, Problem* out);
 
 // router.cu
 cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void* w_gate,

@@ -109,6 +109,8 @@ static int to_problem(const moe_problem_t* in, Problem* out) {
   return MOE_OK;
 }
 
+int problem_from_abi(const moe_problem_t* in, Problem* out) { return to_problem(in, out); }
+
 static int check_ws(const Problem& p, void* ws, size_t ws_bytes) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < make_layout(p).total) return MOE_ERR_WORKSPACE;
