@@ -8,8 +8,8 @@
  *   chosen  = the K experts with the largest selection score
  *             (logit; or p + b with a selection bias b)
  *   w_k     = p[chosen_k] / sum_k' p[chosen_k']        renormalised gates
- *   dispatch: each expert serves at most `cap` (t,k) pairs, first come first
- *             served in token order; the rest are dropped
+ *   dispatch: each expert serves at most `cap` (t,k) pairs, earlier tokens
+ *             first; the rest are dropped
  *   y_t     = sum_s SharedExpert_s(x_t) + sum_{kept k} w_k Expert_{chosen_k}(x_t)
  *   Expert(x) = W_down (SiLU(W_gate x) * (W_up x))
  * plus the Switch statistics f_e, P_e and alpha * E * sum_e f_e P_e.
@@ -24,10 +24,10 @@
  *     Fine-Grained Expert Architecture (eq. Expert_i, SwiGLU; shared experts added
  *     to the routed outputs); §2.3 Auxiliary-Loss-Free Load Balancing
  *     (s_ij = softmax(x_i W_g)_j + b_j).
- *   "Scaling with experts" (jeff-ong.com): "The gating network" (softmax over
- *     the top-k logits, renormalised survivors, y = g1 E1(x) + g2 E2(x));
- *     "A balance penalty"; "A budget" (capacity, dropped tokens skip the expert
- *     and continue through the residual); "A shared expert".
+ *   "Scaling with experts" (jeff-ong.com): "The gating network" (the k best
+ *     gates kept and rescaled to add up to 1; output = gate-weighted sum of the
+ *     chosen experts); "A balance penalty"; "A budget" (per-expert capacity;
+ *     a dropped assignment is not processed by its expert); "A shared expert".
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers, row-major, densely packed, owned

@@ -22,7 +22,7 @@ Parity pins (what ties each function to something other than itself) are in
                  SwiGLU of concatenated width; dropped pairs contribute nothing
   balance        uniform routing gives exactly alpha
   router_zloss   all-equal logits give (l + ln E)^2
-  utilization    uniform counts give log2 E bits ("max 7 bits" for 128)
+  utilization    uniform counts give log2 E bits (7 bits for 128 experts, the table's bound)
   flops          K=8, N_s=4, E=128 gives 12/128 (the compute-budget ratio)
 """
 from __future__ import annotations

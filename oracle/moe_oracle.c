@@ -100,8 +100,8 @@ void oracle_softmax(int64_t T, int32_t E, const double* logits, double* p) {
  * The K chosen experts are those with the largest s; equal scores go to the
  * lower expert index; they are listed in that order (largest s first).
  *
- * Gate weights ([SE] "The gating network": keep the top-k scores, zero the
- * rest, renormalise the survivors to sum to one):
+ * Gate weights ([SE] "The gating network": only the k best scores stay
+ * non-zero and they are rescaled so that they add up to 1):
  *   w[t,k] = p[t, idx[t,k]] / sum_k' p[t, idx[t,k']]
  * which equals a softmax taken over the selected logits only.
  *
@@ -158,9 +158,9 @@ int64_t oracle_capacity(int64_t T, int32_t K, int32_t E, float C) {
 }
 
 /* ---------------------------------------------------------------------------
- * Capacity-limited dispatch.  [SE] "A budget": each expert takes a limited
- * number of tokens per batch; tokens past the budget are dropped (their expert
- * update is skipped and they continue through the residual).
+ * Capacity-limited dispatch.  [SE] "A budget": an expert accepts a bounded
+ * number of tokens per batch; an assignment beyond that bound is dropped, so
+ * the expert does not process that token, which keeps only its residual path.
  *
  *   counts[e]  = number of (t,k) with idx[t,k] == e               (pre-capacity)
  *   kept[e]    = min(counts[e], cap)        (counts[e] if cap < 0)
@@ -243,7 +243,7 @@ void oracle_swiglu_accumulate(int32_t d, int32_t F, const double* x,
  * Shared experts: always active, added unweighted ([ZX] §2.2; [SE] "A shared
  * expert").  Routed part: gate-weighted sum ([SE] "The gating network":
  * y = g1 Expert1(x) + g2 Expert2(x)).  A dropped pair contributes nothing and
- * the survivors are not renormalised again ([SE] "A budget").  The residual
+ * the kept pairs are not rescaled again ([SE] "A budget").  The residual
  * add is outside the layer.
  * Layouts: x [T, d]; w13 [E, 2F, d]; w2 [E, d, F]; shared weights
  * [N_s, 2F, d] / [N_s, d, F]; y rows written for the listed tokens only:
@@ -315,7 +315,7 @@ void oracle_combine(int64_t T, int32_t d, int32_t K,
  * penalty":  L = alpha * N * sum_e f_e P_e, with
  *   f_e = counts[e] / (T*K)   fraction of the batch's assignments sent to e
  *                             (counted before the capacity cut)
- *   P_e = (1/T) sum_t p[t,e]  average routing probability of e
+ *   P_e = (1/T) sum_t p[t,e]  mean softmax probability of e over the batch
  * With uniform routing (f_e = P_e = 1/E) the loss is exactly alpha.
  * ------------------------------------------------------------------------- */
 void oracle_balance(int64_t T, int32_t E, int32_t K, const int32_t* counts,
@@ -354,7 +354,7 @@ double oracle_router_zloss(int64_t T, int32_t E, const double* logits) {
  * Expert utilisation statistics, [ZM] §6.2 table tab:utilization, from the
  * per-expert assignment counts (n = sum counts):
  *   out[0] entropy in bits of the load distribution q_e = counts[e]/n
- *          (0 log 0 = 0; at most log2 E, "max 7 bits" for 128 experts)
+ *          (0 log 0 = 0; at most log2 E, i.e. 7 bits for 128 experts)
  *   out[1] coefficient of variation of counts (population std / mean)
  *   out[2] token drop rate: dropped assignments / n
  *   out[3] experts whose load is below 50% of the mean

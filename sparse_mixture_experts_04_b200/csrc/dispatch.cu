@@ -1,12 +1,12 @@
 // Capacity-limited dispatch: group the (token, k) assignments by expert.
 //
-//   Scaling with experts, "A budget": each expert takes a limited number of
-//   tokens per batch; tokens past the budget are dropped (the expert update is
-//   skipped; the token continues through the residual).
+//   Scaling with experts, "A budget": an expert accepts a bounded number of
+//   tokens per batch; an assignment beyond the bound is dropped (the expert
+//   does not process that token, which keeps only its residual path).
 //   Zen MoDE, §5.3 Adaptive Capacity Factors: capacity_e = C * batch*seq / N_E
 //   (scaled here by K for top-K routing).
 //
-// Order: first come, first served in token order.  rank(t,k) = number of tokens
+// Order: earlier tokens are served first.  rank(t,k) = number of tokens
 // t' < t that chose the same expert; (t,k) is kept iff rank < cap.  The result
 // is independent of thread scheduling: ranks are counted, never claimed by
 // racing atomics.

@@ -5,8 +5,8 @@
 //     Architecture, eq. router_standard: TopK(softmax(W_r x), K).
 //   Zen-Max, §2.3 Auxiliary-Loss-Free Load Balancing: s_ij = softmax(x_i W_g)_j + b_j
 //     (the bias steers selection; gate weights use the unbiased softmax).
-//   Scaling with experts, "The gating network": keep the top-k, zero the rest,
-//     renormalise the survivors to sum to one.  "A balance penalty":
+//   Scaling with experts, "The gating network": only the k best scores stay
+//     non-zero, rescaled to add up to 1.  "A balance penalty":
 //     alpha * N * sum f_i P_i.  Zen MoDE §5.2 eq. L_balance.
 #include <math.h>
 
