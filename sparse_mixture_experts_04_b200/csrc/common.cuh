@@ -263,6 +263,35 @@ __device__ __forceinline__ void umma_commit_pair_multicast(uint64_t* bar, uint16
       : "memory");
 }
 
+// ------------------------------------------- balance statistics (shared)
+// Per-expert probability sums travel as unsigned fixed-point integers (exact,
+// order-independent integer adds).  Scale 2^s with s = min(40, 62 - ceil(log2 T))
+// keeps T tokens' sum (each p <= 1) below 2^62; resolution 2^-s per token.
+__host__ __device__ inline double p_fixed_scale(int64_t T) {
+  int bits = 0;
+  while ((static_cast<int64_t>(1) << bits) < T) ++bits;
+  int s = 62 - bits;
+  if (s > 40) s = 40;
+  return static_cast<double>(static_cast<int64_t>(1) << s);
+}
+
+// Writes f_e and P_e of expert e into stats and returns f_e * P_e.
+__device__ __forceinline__ double balance_stats_expert(long long count, unsigned long long psum_fixed, int64_t T,
+                                                       int E, int K, int e, float* stats) {
+  const double f = static_cast<double>(count) / (static_cast<double>(T) * K);
+  const double P = static_cast<double>(psum_fixed) / p_fixed_scale(T) / static_cast<double>(T);
+  stats[e] = static_cast<float>(f);
+  stats[E + e] = static_cast<float>(P);
+  return f * P;
+}
+
+// loss = alpha * E * sum_e f_e P_e, summed in expert order (one thread).
+__device__ __forceinline__ void balance_loss(const double* fp, int E, float alpha, float* stats) {
+  double acc = 0.0;
+  for (int e = 0; e < E; ++e) acc += fp[e];
+  stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
+}
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -47,14 +47,22 @@ __global__ void __launch_bounds__(256) dispatch_hist_kernel(const int32_t* __res
 // One block of 1024 threads.  Thread (e, s) owns a contiguous run of chunks
 // for expert e; runs are summed, scanned per expert, then re-walked to write
 // each chunk's base.
+// With stats != nullptr it also finalises the balance statistics from the
+// chunk histogram and the chunk probability sums (fixed point) that the
+// selection kernel added: f_e, P_e and the loss (see balance_stats_expert).
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __restrict__ chunk_counts,
                                                              int n_chunks, int E, long long cap,
                                                              int32_t* __restrict__ chunk_base,
                                                              int32_t* __restrict__ counts,
                                                              int32_t* __restrict__ kept,
-                                                             int32_t* __restrict__ seg_off) {
+                                                             int32_t* __restrict__ seg_off,
+                                                             const unsigned long long* __restrict__ chunk_psum,
+                                                             float* __restrict__ stats, int64_t T, int K,
+                                                             float alpha) {
   __shared__ int part[1024];
+  __shared__ unsigned long long ppart[1024];
   __shared__ int s_kept[kMaxExperts];
+  __shared__ double s_fp[kMaxExperts];
   int S = 1024 / E;
   if (S > n_chunks) S = n_chunks;
   if (S < 1) S = 1;
@@ -66,23 +74,32 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
   int c0 = s * per, c1 = c0 + per;
   if (c1 > n_chunks) c1 = n_chunks;
   int local = 0;
-  if (active)
+  unsigned long long plocal = 0;
+  if (active) {
     for (int c = c0; c < c1; ++c) local += chunk_counts[static_cast<int64_t>(c) * E + e];
+    if (stats)
+      for (int c = c0; c < c1; ++c) plocal += chunk_psum[static_cast<int64_t>(c) * E + e];
+  }
   part[tid] = local;
+  ppart[tid] = plocal;
   __syncthreads();
   if (active && s == 0) {
     int run = 0;
+    unsigned long long prun = 0;
     for (int i = 0; i < S; ++i) {
       const int v = part[tid + i];
       part[tid + i] = run;
       run += v;
+      prun += ppart[tid + i];
     }
     counts[e] = run;
     const int k = (cap < 0 || run < cap) ? run : static_cast<int>(cap);
     kept[e] = k;
     s_kept[e] = k;
+    if (stats) s_fp[e] = balance_stats_expert(run, prun, T, E, K, e, stats);
   }
   __syncthreads();
+  if (stats && tid == 32) balance_loss(s_fp, E, alpha, stats);
   if (active) {
     int run = part[tid];
     for (int c = c0; c < c1; ++c) {
@@ -168,11 +185,13 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
 
 cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
-                            int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready) {
+                            int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready,
+                            const unsigned long long* chunk_psum, float* stats) {
   const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
   if (!counts_ready) dispatch_hist_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_counts, status);
   dispatch_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, n_chunks, p.E, static_cast<long long>(p.cap),
-                                           chunk_base, counts, kept, seg_off);
+                                           chunk_base, counts, kept, seg_off, chunk_psum,
+                                           chunk_psum ? stats : nullptr, p.T, p.K, p.alpha);
   dispatch_rank_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_base, kept, seg_off, slot_of, perm);
   return cudaGetLastError();
 }

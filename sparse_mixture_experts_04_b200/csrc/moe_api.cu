@@ -34,16 +34,19 @@ WsLayout make_layout(const Problem& p) {
   const size_t TK = static_cast<size_t>(p.T) * p.K;
   const size_t R = static_cast<size_t>(p.max_rows);
   L.n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
-  L.n_sel_blocks = static_cast<int>((p.T + kSelectTokens - 1) / kSelectTokens);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off = align256(off + (bytes ? bytes : 1));
     return o;
   };
-  L.status = 0;  // status word, then the chunk histogram: one memset clears both
-  L.chunk_counts = 256;
-  off = align256(256 + static_cast<size_t>(L.n_chunks) * p.E * 4);
+  // status word, chunk histogram and chunk p sums first: one memset clears them
+  const size_t ce = static_cast<size_t>(L.n_chunks) * p.E;
+  L.status = 0;
+  L.chunk_psum = 256;                              // 8-byte entries
+  L.chunk_counts = align256(L.chunk_psum + ce * 8);
+  L.zero_bytes = L.chunk_counts + ce * 4;
+  off = align256(L.zero_bytes);
   L.logits = take(static_cast<size_t>(p.T) * p.E * 4);
   L.topk_idx = take(TK * 4);
   L.topk_w = take(TK * 4);
@@ -53,11 +56,8 @@ WsLayout make_layout(const Problem& p) {
   L.slot_of = take(TK * 4);
   L.perm = take(R * 4);
   L.chunk_base = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
-  L.sel_psum = take(static_cast<size_t>(L.n_sel_blocks) * p.E * 4);
-  L.sel_count = take(static_cast<size_t>(L.n_sel_blocks) * p.E * 4);
   const int splits = (p.dtype == kBF16) ? router_k_splits(p) : 1;
   L.logit_parts = take(splits > 1 ? static_cast<size_t>(splits) * p.T * p.E * 4 : 0);
-  L.stats_scratch = take(kMaxExperts * 8 + 16);
   L.x_perm = take(R * p.d * es);
   L.h_routed = take(R * p.F * es);
   L.y_perm = take(R * p.d * es);
@@ -125,9 +125,11 @@ static T* at(void* ws, size_t off) {
 static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // Router body shared by moe_route and moe_layer_forward.
+// chunk_totals_cleared: the caller already zeroed the chunk totals;
+// stats_in_route: finalise the statistics here (else the dispatch scan does).
 static int route_impl(const Problem& p, const void* x, const void* w_gate, const float* offset,
                       const float* sel_bias, float* logits, int32_t* idx, float* w, float* stats, void* ws,
-                      const WsLayout& L, cudaStream_t st, int32_t* chunk_counts = nullptr) {
+                      const WsLayout& L, cudaStream_t st, bool chunk_totals_cleared, bool stats_in_route) {
   unsigned* status = at<unsigned>(ws, L.status);
   int n_parts = 0;
   float* parts = nullptr;
@@ -144,16 +146,18 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
       if (cudaError_t e = launch_gate_logits_simt(p, x, w_gate, offset, logits, st)) return cuda_rc(e);
     }
   }
-  float* psum = at<float>(ws, L.sel_psum);
-  int32_t* pcount = at<int32_t>(ws, L.sel_count);
-  double* stats_fp = at<double>(ws, L.stats_scratch);
-  unsigned* ticket = reinterpret_cast<unsigned*>(stats_fp + kMaxExperts);
-  if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, psum, pcount,
-                                          stats ? ticket : nullptr, chunk_counts, st))
-    return cuda_rc(e);
-  if (stats) {
-    if (cudaError_t e = launch_route_stats(p, psum, pcount, L.n_sel_blocks, stats, stats_fp, st))
+  // the chunk totals start at zero: the layer forward clears them with the
+  // status word; a standalone call clears them here
+  if (!chunk_totals_cleared) {
+    if (cudaError_t e = cudaMemsetAsync(at<char>(ws, L.chunk_psum), 0, L.zero_bytes - L.chunk_psum, st))
       return cuda_rc(e);
+  }
+  int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
+  unsigned long long* chunk_psum = at<unsigned long long>(ws, L.chunk_psum);
+  if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, chunk_counts, chunk_psum, st))
+    return cuda_rc(e);
+  if (stats && stats_in_route) {
+    if (cudaError_t e = launch_route_stats(p, chunk_counts, chunk_psum, L.n_chunks, stats, st)) return cuda_rc(e);
   }
   return MOE_OK;
 }
@@ -224,7 +228,8 @@ int moe_route(const moe_problem_t* q, const void* x, const void* w_gate, const f
   if (!given && (!x || !w_gate || !aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
   return route_impl(p, x, w_gate, given ? nullptr : logit_offset, sel_bias, logits, topk_idx, topk_w, stats, ws,
-                    L, reinterpret_cast<cudaStream_t>(stream));
+                    L, reinterpret_cast<cudaStream_t>(stream), /*chunk_totals_cleared=*/false,
+                    /*stats_in_route=*/true);
 }
 
 int moe_dispatch(const moe_problem_t* q, const int32_t* topk_idx, const void* x, int32_t* counts, int32_t* kept,
@@ -315,18 +320,18 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   void* y_perm = at<void>(ws, L.y_perm);
   void* y_sh = p.Ns > 0 ? at<void>(ws, L.y_shared) : nullptr;
 
-  // status word and chunk histogram (contiguous at the start of ws) start at zero
-  if (cudaError_t e = cudaMemsetAsync(ws, 0, L.chunk_counts + static_cast<size_t>(L.n_chunks) * p.E * 4, st))
-    return cuda_rc(e);
+  // status word, chunk histogram and chunk p sums (contiguous at offset 0) start at zero
+  if (cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, st)) return cuda_rc(e);
   if (cudaError_t e = mark(MOE_EV_START)) return cuda_rc(e);
-  int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
   if (int rc = route_impl(p, x, w->w_gate, given ? nullptr : w->logit_offset, w->sel_bias, logits, idx, gw, stats,
-                          ws, L, st, chunk_counts))
+                          ws, L, st, /*chunk_totals_cleared=*/true, /*stats_in_route=*/false))
     return rc;
-  kernels += (given ? 0 : 1) + 1 + (stats ? 1 : 0);
+  kernels += (given ? 0 : 1) + 1;
   if (cudaError_t e = mark(MOE_EV_ROUTED)) return cuda_rc(e);
-  if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, chunk_counts,
-                                      at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true))
+  // the scan also finalises the balance statistics from the chunk totals
+  if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, at<int32_t>(ws, L.chunk_counts),
+                                      at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true,
+                                      at<unsigned long long>(ws, L.chunk_psum), stats))
     return cuda_rc(e);
   kernels += 2;
   if (p.max_rows > 0) {

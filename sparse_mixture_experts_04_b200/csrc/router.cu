@@ -143,13 +143,14 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
                                                            const float* __restrict__ parts, int n_parts,
                                                            const float* __restrict__ sel_bias, int bias_on_logit,
                                                            int32_t* __restrict__ topk_idx,
-                                                           float* __restrict__ topk_w, float* __restrict__ psum,
-                                                           int32_t* __restrict__ pcount, int64_t T, int E,
-                                                           int K, unsigned* stats_ticket,
-                                                           int32_t* __restrict__ chunk_counts) {
-  if (stats_ticket && blockIdx.x == 0 && threadIdx.x == 0) *stats_ticket = 0u;  // for route_stats_kernel
+                                                           float* __restrict__ topk_w, int64_t T, int E, int K,
+                                                           int32_t* __restrict__ chunk_counts,
+                                                           unsigned long long* __restrict__ chunk_psum,
+                                                           double pscale) {
   __shared__ float s_psum[8][32 * EPL];
   __shared__ int s_count[32 * EPL];
+  // the fixed-point block sums below cover at most kSelectTokens tokens
+  static_assert(kDispatchChunk % kSelectTokens == 0, "a selection block must not straddle dispatch chunks");
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < 32 * EPL; e += blockDim.x) s_count[e] = 0;
@@ -281,104 +282,63 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
 #pragma unroll
   for (int i = 0; i < EPL; ++i) s_psum[warp][lane + 32 * i] = pacc[i];
   __syncthreads();
+  // Per-dispatch-chunk totals (this block's tokens lie in one chunk, since
+  // kDispatchChunk is a multiple of kSelectTokens): the expert histogram and
+  // the sum of p as a fixed-point integer (scale p_fixed_scale(T)).  Integer adds commute, so the
+  // totals do not depend on the order in which blocks arrive.
+  const int64_t chunk = tok_begin / kDispatchChunk;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += s_psum[w][e];
-    psum[static_cast<int64_t>(blockIdx.x) * E + e] = s;
-    pcount[static_cast<int64_t>(blockIdx.x) * E + e] = s_count[e];
-    // this block's tokens all lie in one dispatch chunk (kDispatchChunk is a
-    // multiple of kSelectTokens); integer adds commute, so the total is exact
-    if (chunk_counts && s_count[e])
-      atomicAdd(&chunk_counts[(tok_begin / kDispatchChunk) * E + e], s_count[e]);
+    if (s_count[e]) atomicAdd(&chunk_counts[chunk * E + e], s_count[e]);
+    if (s > 0.f) atomicAdd(&chunk_psum[chunk * E + e], __double2ull_rn(static_cast<double>(s) * pscale));
   }
 }
 
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
-                                const float* sel_bias, int32_t* topk_idx, float* topk_w, float* psum,
-                                int32_t* pcount, unsigned* stats_ticket, int32_t* chunk_counts,
-                                cudaStream_t st) {
+                                const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
+                                unsigned long long* chunk_psum, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>((p.T + kSelectTokens - 1) / kSelectTokens);
   const int bias_on_logit = (p.flags & 0x2u) ? 1 : 0;
   if (p.E <= 32)
-    route_select_kernel<1><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
+    route_select_kernel<1><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   else if (p.E <= 64)
-    route_select_kernel<2><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
+    route_select_kernel<2><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   else if (p.E <= 128)
-    route_select_kernel<4><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
+    route_select_kernel<4><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   else
-    route_select_kernel<8><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, psum,
-                                                   pcount, p.T, p.E, p.K, stats_ticket, chunk_counts);
+    route_select_kernel<8><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   return cudaGetLastError();
 }
 
 // ----------------------------------------------------------------------------
-// Balance statistics from the per-block partials:
+// Balance statistics from the per-chunk totals the selection kernel adds:
 //   f_e = count_e / (T K),  P_e = (1/T) sum_t p[t,e],  loss = alpha E sum_e f_e P_e
-// stats layout: [f_0 .. f_{E-1}, P_0 .. P_{E-1}, loss].
-// One block per expert: each thread sums a fixed stride of the partials, then
-// a fixed-shape tree adds the threads' sums, so the result does not depend on
-// scheduling.  The block that finishes last (ticket) adds the E products in
-// expert order for the loss; the ticket is zeroed by the selection kernel.
+// stats layout: [f_0 .. f_{E-1}, P_0 .. P_{E-1}, loss].  Used by moe_route;
+// the layer forward finalises the same statistics inside the dispatch scan.
 // ----------------------------------------------------------------------------
-static_assert(kDispatchChunk % kSelectTokens == 0, "a selection block must not straddle dispatch chunks");
-constexpr int kStatsThreads = 256;
-
-__global__ void __launch_bounds__(kStatsThreads) route_stats_kernel(const float* __restrict__ psum,
-                                                                    const int32_t* __restrict__ pcount,
-                                                                    int n_blocks, int64_t T, int E, int K,
-                                                                    float alpha, float* __restrict__ stats,
-                                                                    double* __restrict__ fp,
-                                                                    unsigned* __restrict__ ticket) {
-  __shared__ double s_p[kStatsThreads];
-  __shared__ long long s_c[kStatsThreads];
-  __shared__ bool s_last;
-  const int e = blockIdx.x;
-  const int tid = threadIdx.x;
-  double ps = 0.0;
-  long long c = 0;
-  for (int b = tid; b < n_blocks; b += kStatsThreads) {
-    c += pcount[static_cast<int64_t>(b) * E + e];
-    ps += static_cast<double>(psum[static_cast<int64_t>(b) * E + e]);
-  }
-  s_p[tid] = ps;
-  s_c[tid] = c;
-  __syncthreads();
-#pragma unroll
-  for (int w = kStatsThreads / 2; w > 0; w >>= 1) {
-    if (tid < w) {
-      s_p[tid] += s_p[tid + w];
-      s_c[tid] += s_c[tid + w];
+__global__ void __launch_bounds__(1024) route_stats_kernel(const int32_t* __restrict__ chunk_counts,
+                                                           const unsigned long long* __restrict__ chunk_psum,
+                                                           int n_chunks, int64_t T, int E, int K, float alpha,
+                                                           float* __restrict__ stats) {
+  __shared__ double s_fp[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    long long c = 0;
+    unsigned long long ps = 0;
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      c += chunk_counts[static_cast<int64_t>(ch) * E + e];
+      ps += chunk_psum[static_cast<int64_t>(ch) * E + e];
     }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    const double f = static_cast<double>(s_c[0]) / (static_cast<double>(T) * K);
-    const double P = s_p[0] / static_cast<double>(T);
-    stats[e] = static_cast<float>(f);
-    stats[E + e] = static_cast<float>(P);
-    fp[e] = f * P;
-    __threadfence();
-    s_last = atomicAdd(ticket, 1u) == static_cast<unsigned>(E - 1);
+    s_fp[e] = balance_stats_expert(c, ps, T, E, K, e, stats);
   }
   __syncthreads();
-  if (s_last && tid == 0) {
-    __threadfence();
-    double acc = 0.0;
-    for (int i = 0; i < E; ++i) acc += static_cast<volatile double*>(fp)[i];
-    stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
-  }
+  if (threadIdx.x == 0) balance_loss(s_fp, E, alpha, stats);
 }
 
-cudaError_t launch_route_stats(const Problem& p, const float* psum, const int32_t* pcount, int n_blocks,
-                               float* stats, void* scratch, cudaStream_t st) {
-  double* fp = static_cast<double*>(scratch);
-  unsigned* ticket = reinterpret_cast<unsigned*>(fp + kMaxExperts);
-  route_stats_kernel<<<p.E, kStatsThreads, 0, st>>>(psum, pcount, n_blocks, p.T, p.E, p.K, p.alpha, stats, fp,
-                                                   ticket);
+cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, const unsigned long long* chunk_psum,
+                               int n_chunks, float* stats, cudaStream_t st) {
+  route_stats_kernel<<<1, 1024, 0, st>>>(chunk_counts, chunk_psum, n_chunks, p.T, p.E, p.K, p.alpha, stats);
   return cudaGetLastError();
 }
 
