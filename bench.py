@@ -89,21 +89,26 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
     def __init__(self, device_index: int):
-        self.samples, self.reasons, self.err = [], 0, None
+        self.samples, self.power, self.reasons, self.err = [], [], 0, None
         self._stop = threading.Event()
         self.max_mhz = None
+        self.match = None
         try:
             import pynvml
             pynvml.nvmlInit()
-            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid).lower().replace("gpu-", "")
             h = None
-            for i in range(pynvml.nvmlDeviceGetCount()):
+            n = pynvml.nvmlDeviceGetCount()
+            for i in range(n):
                 hi = pynvml.nvmlDeviceGetHandleByIndex(i)
                 u = pynvml.nvmlDeviceGetUUID(hi)
-                u = u.decode() if isinstance(u, bytes) else u
-                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
-                    h = hi
-            self.h = h if h is not None else pynvml.nvmlDeviceGetHandleByIndex(device_index)
+                u = (u.decode() if isinstance(u, bytes) else u).lower().replace("gpu-", "")
+                if u == uuid:
+                    h, self.match = hi, f"uuid (nvml index {i} of {n})"
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index if n > 1 else 0)
+                self.match = f"index fallback (nvml index {device_index if n > 1 else 0} of {n})"
+            self.h = h
             self.nv = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception as e:  # NVML unavailable: report, do not fail the benchmark
@@ -114,6 +119,7 @@ class ClockSampler:
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
                 self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                self.power.append(self.nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
             except Exception as e:
                 self.err = str(e)
                 return
@@ -135,7 +141,9 @@ class ClockSampler:
             return {"error": self.err}
         names = sorted(n for bit, n in self.REASONS.items() if self.reasons & bit)
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+                "sm_mhz_min": min(self.samples) if self.samples else None,
+                "power_w_max": max(self.power) if self.power else None,
+                "reasons": names, "samples": len(self.samples), "device": self.match}
 
     def rejected(self) -> bool:
         if self.h is None or not self.samples:
@@ -271,11 +279,22 @@ def run_ours(args, cfg):
     if status:
         raise RuntimeError(f"device status {status:#x} after warm-up")
 
-    def timed_region():
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(_lib.NUM_EVENTS)] for _ in range(args.steps)]
+    def make_events(n, which):
+        evs = [[torch.cuda.Event(enable_timing=True) if j in which else None for j in range(_lib.NUM_EVENTS)]
+               for _ in range(n)]
         for row in evs:       # create the underlying events before they are handed to the library
             for e in row:
-                e.record(stream)
+                if e is not None:
+                    e.record(stream)
+        return evs
+
+    UP = (_lib.EVENT_NAMES.index("dispatched"), _lib.EVENT_NAMES.index("up"))
+
+    def timed_region():
+        # Inside the timed region only the two events around the dominant kernel
+        # (the routed up/gate GEMM) are recorded, so the kernels of a forward
+        # otherwise follow each other directly on the stream.
+        evs = make_events(args.steps, UP)
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         barrier(world)
@@ -289,18 +308,25 @@ def run_ours(args, cfg):
             torch.cuda.synchronize()
         barrier(world)
         ms = start.elapsed_time(end) / args.steps
-        stage = {}
-        for j in range(1, _lib.NUM_EVENTS):
-            stage[_lib.EVENT_NAMES[j]] = sum(evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(args.steps)) / args.steps
-        return ms, stage, n_k, clk
+        up_ms = sum(evs[i][UP[0]].elapsed_time(evs[i][UP[1]]) for i in range(args.steps)) / args.steps
+        return ms, up_ms, n_k, clk
 
-    ms, stage, n_kernels, clk = timed_region()
+    ms, up_ms, n_kernels, clk = timed_region()
     remeasured = False
     if clk.rejected():
-        ms, stage, n_kernels, clk = timed_region()
+        ms, up_ms, n_kernels, clk = timed_region()
         remeasured = True
     ms_max = max_over_ranks(ms, world)
-    up_ms_max = max_over_ranks(stage["up"], world)
+
+    # per-stage breakdown: a separate short pass with an event at every stage boundary
+    n_prof = min(args.steps, 10)
+    evs = make_events(n_prof, set(range(_lib.NUM_EVENTS)))
+    for i in range(n_prof):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    stage = {}
+    for j in range(1, _lib.NUM_EVENTS):
+        stage[_lib.EVENT_NAMES[j]] = sum(evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(n_prof)) / n_prof
 
     # end to end through the public API: pinned host x in, y and statistics out
     xh = [x.pin_memory() for x in xs_host[: min(n_x, 4)]]
@@ -331,7 +357,7 @@ def run_ours(args, cfg):
     kept = int(layer.routing["seg_off"][-1].item())
     flops = algorithmic_flops(cfg, kept)
     peaks, peak_src = load_peaks()
-    up_tflops = flops["up"] / (stage["up"] * 1e-3) / 1e12
+    up_tflops = flops["up"] / (up_ms * 1e-3) / 1e12
     gemm_ms = stage["up"] + stage["down"]
     gemm_tflops = (flops["up"] + flops["down"]) / (gemm_ms * 1e-3) / 1e12
     disp_gbs = dispatch_bytes(cfg, kept) / (stage["dispatched"] * 1e-3) / 1e9
@@ -367,13 +393,13 @@ def run_ours(args, cfg):
                      "achieved": up_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": up_tflops / peaks["bf16_tflops"],
                      "traffic": ncu_traffic(cfg.name),
-                     "algorithmic_flops_per_launch": flops["up"], "launch_ms": stage["up"],
+                     "algorithmic_flops_per_launch": flops["up"], "launch_ms": up_ms,
                      "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
                      else "fallback 1.59 PFLOP/s"},
         "cpu_baseline": cpu,
         "gpu_launches": n_kernels,
         "clocks": {**clk.summary(), "remeasured": remeasured},
-        "stages_ms": stage,
+        "stages_ms": stage, "stages_note": "separate pass with an event at every stage boundary",
         "kept_pairs": kept, "dropped_pairs": cfg.T * cfg.top_k - kept,
         "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
         "dispatch_gbs": disp_gbs, "layer_tflops": total_flops / (ms * 1e-3) / 1e12,

@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const T* __res
                                                                   T* __restrict__ y, int64_t Tn, int d, int K,
                                                                   int64_t n_perm_rows) {
   constexpr int V = Pack16<T>::N;
+  pdl_wait();
+  pdl_trigger();
   const int nvec = d / V;
   const int v0 = blockIdx.x * (kCombineThreads * kCombineVPT) + threadIdx.x;
   for (int64_t t = blockIdx.y; t < Tn; t += gridDim.y) {
@@ -102,13 +104,14 @@ cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* 
   if (gy > 65535) gy = 65535;
   const dim3 grid(gx, static_cast<unsigned>(gy));
   if (p.dtype == kBF16)
-    combine_kernel<__nv_bfloat16><<<grid, kCombineThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(y_perm), slot_of, topk_w, static_cast<const __nv_bfloat16*>(y_shared),
-        static_cast<__nv_bfloat16*>(y), p.T, p.d, p.K, p.max_rows);
+    return launch_k(combine_kernel<__nv_bfloat16>, grid, dim3(kCombineThreads), 0, st,
+                    static_cast<const __nv_bfloat16*>(y_perm), slot_of, topk_w,
+                    static_cast<const __nv_bfloat16*>(y_shared), static_cast<__nv_bfloat16*>(y), p.T, p.d, p.K,
+                    p.max_rows);
   else
-    combine_kernel<float><<<grid, kCombineThreads, 0, st>>>(
-        static_cast<const float*>(y_perm), slot_of, topk_w, static_cast<const float*>(y_shared),
-        static_cast<float*>(y), p.T, p.d, p.K, p.max_rows);
+    return launch_k(combine_kernel<float>, grid, dim3(kCombineThreads), 0, st, static_cast<const float*>(y_perm),
+                    slot_of, topk_w, static_cast<const float*>(y_shared), static_cast<float*>(y), p.T, p.d, p.K,
+                    p.max_rows);
   return cudaGetLastError();
 }
 

@@ -292,6 +292,34 @@ __device__ __forceinline__ void balance_loss(const double* fp, int E, float alph
   stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Kernels of one forward are launched with programmatic stream serialisation:
+// a kernel may be scheduled while its predecessor on the stream is finishing.
+// Every kernel calls pdl_wait() before it reads anything the predecessor wrote
+// (and every kernel calls it, so completion stays transitive along the
+// stream), and pdl_trigger() once it no longer needs to hold back its
+// successor's launch.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+bool pdl_enabled();  // MOE_B200_PDL=0 turns the attribute off (moe_api.cu)
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256) dispatch_hist_kernel(const int32_t* __res
                                                             int E, int32_t* __restrict__ chunk_counts,
                                                             unsigned* status) {
   __shared__ int hist[kMaxExperts];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int64_t begin = static_cast<int64_t>(blockIdx.x) * kDispatchChunk * K;
@@ -63,6 +65,8 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
   __shared__ unsigned long long ppart[1024];
   __shared__ int s_kept[kMaxExperts];
   __shared__ double s_fp[kMaxExperts];
+  pdl_wait();
+  pdl_trigger();
   int S = 1024 / E;
   if (S > n_chunks) S = n_chunks;
   if (S < 1) S = 1;
@@ -143,6 +147,8 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
                                                             int32_t* __restrict__ perm) {
   __shared__ uint32_t mask[8][kMaxExperts];
   __shared__ int wbase[8][kMaxExperts];
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) mask[i / E][i % E] = 0u;
@@ -188,12 +194,19 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready,
                             const unsigned long long* chunk_psum, float* stats) {
   const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
-  if (!counts_ready) dispatch_hist_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_counts, status);
-  dispatch_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, n_chunks, p.E, static_cast<long long>(p.cap),
-                                           chunk_base, counts, kept, seg_off, chunk_psum,
-                                           chunk_psum ? stats : nullptr, p.T, p.K, p.alpha);
-  dispatch_rank_kernel<<<n_chunks, 256, 0, st>>>(idx, p.T, p.K, p.E, chunk_base, kept, seg_off, slot_of, perm);
-  return cudaGetLastError();
+  if (!counts_ready) {
+    if (cudaError_t e = launch_k(dispatch_hist_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
+                                 chunk_counts, status))
+      return e;
+  }
+  if (cudaError_t e = launch_k(dispatch_scan_kernel, dim3(1), dim3(1024), 0, st,
+                               static_cast<const int32_t*>(chunk_counts), n_chunks, p.E, static_cast<long long>(p.cap),
+                               chunk_base, counts, kept, seg_off, chunk_psum, chunk_psum ? stats : nullptr, p.T,
+                               p.K, p.alpha))
+    return e;
+  return launch_k(dispatch_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
+                  static_cast<const int32_t*>(chunk_base), static_cast<const int32_t*>(kept),
+                  static_cast<const int32_t*>(seg_off), slot_of, perm);
 }
 
 constexpr int kGatherUnroll = 8;
@@ -206,6 +219,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           int64_t T, int vec_per_row, int64_t max_rows,
                                                           uint4* __restrict__ x_perm) {
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   const int64_t n_rows = seg_off[E];
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -234,10 +249,9 @@ cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, 
   int64_t blocks = (p.max_rows + 7) / 8;
   const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
   if (blocks > cap_blocks) blocks = cap_blocks;
-  gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const uint4*>(x), perm, seg_off, p.E, p.K, p.T, vec_per_row, p.max_rows,
-      static_cast<uint4*>(x_perm));
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                  static_cast<const uint4*>(x), perm, seg_off, p.E, p.K, p.T, vec_per_row, p.max_rows,
+                  static_cast<uint4*>(x_perm));
 }
 
 }  // namespace moe

@@ -290,6 +290,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
+  pdl_wait();  // everything above is local set-up; from here on the predecessor's outputs are read
+  pdl_trigger();
   if (warp == 2) tile_prefix_warp<kBM>(args, n_tiles_n, prefix, lane);
   tc_fence_before_sync();
   __syncthreads();
@@ -488,6 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
+  pdl_wait();  // everything above is local set-up; from here on the predecessor's outputs are read
+  pdl_trigger();
   if (warp == 2) tile_prefix_warp<kPairBM>(args, n_tiles_n, prefix, lane);
   tc_fence_before_sync();
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
@@ -680,8 +684,8 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
   if (tile_bound <= 0) return 0;
   int64_t grid = num_sms();
   if (grid > tile_bound) grid = tile_bound;
-  grouped_gemm_tc_kernel<EPI, BN, STAGES><<<static_cast<unsigned>(grid), kGemmThreads, smem, st>>>(ta, tb, a);
-  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+  return launch_k(grouped_gemm_tc_kernel<EPI, BN, STAGES>, dim3(static_cast<unsigned>(grid)), dim3(kGemmThreads),
+                  smem, st, ta, tb, a) == cudaSuccess ? 0 : -3;
 }
 
 template <int EPI>
@@ -715,8 +719,8 @@ static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   }
   if (tile_bound <= 0) return 0;
   if (pairs > tile_bound) pairs = static_cast<int>(tile_bound);
-  grouped_gemm_pair_kernel<EPI><<<static_cast<unsigned>(2 * pairs), kGemmThreads, smem, st>>>(ta, tb, a);
-  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+  return launch_k(grouped_gemm_pair_kernel<EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads), smem,
+                  st, ta, tb, a) == cudaSuccess ? 0 : -3;
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -806,6 +810,8 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const float* __restrict__
   __shared__ float As[32][33];
   __shared__ float Bg[32][33];
   __shared__ float Bu[SWIGLU ? 32 : 1][33];
+  pdl_wait();
+  pdl_trigger();
   const int g = blockIdx.z;
   int base;
   const int rows = group_rows(args, g, &base);
@@ -873,8 +879,9 @@ static int ffn_simt(const Problem& p, int mode, const void* x_rows, int64_t n_ro
   up.ldo = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
   up.out_col_stride = routed ? 0 : p.F;
   dim3 g1(static_cast<unsigned>(cdiv(p.F, 32)), static_cast<unsigned>(cdiv(max_group_rows, 32)), G);
-  ffn_simt_kernel<true><<<g1, 256, 0, st>>>(static_cast<const float*>(x_rows), p.d, static_cast<const float*>(w13),
-                                            up, 2LL * p.F * p.d, static_cast<int64_t>(p.F) * p.d);
+  if (launch_k(ffn_simt_kernel<true>, g1, dim3(256), 0, st, static_cast<const float*>(x_rows), p.d,
+               static_cast<const float*>(w13), up, 2LL * p.F * p.d, static_cast<int64_t>(p.F) * p.d) != cudaSuccess)
+    return -3;
   if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
   GemmArgs dn{};
   dn.n_groups = routed ? p.E : 1;
@@ -887,9 +894,9 @@ static int ffn_simt(const Problem& p, int mode, const void* x_rows, int64_t n_ro
   dn.ldo = p.d;
   dn.out_col_stride = 0;
   dim3 g2(static_cast<unsigned>(cdiv(p.d, 32)), static_cast<unsigned>(cdiv(max_group_rows, 32)), dn.n_groups);
-  ffn_simt_kernel<false><<<g2, 256, 0, st>>>(static_cast<const float*>(h), static_cast<int>(up.ldo),
-                                             static_cast<const float*>(w2), dn, static_cast<int64_t>(p.d) * p.F, 0);
-  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+  return launch_k(ffn_simt_kernel<false>, g2, dim3(256), 0, st, static_cast<const float*>(h),
+                  static_cast<int>(up.ldo), static_cast<const float*>(w2), dn, static_cast<int64_t>(p.d) * p.F,
+                  static_cast<int64_t>(0)) == cudaSuccess ? 0 : -3;
 }
 
 // mode 0: routed (groups = experts over seg_off); mode 1: shared (every row

@@ -3,11 +3,13 @@
 // only; every step of the layer runs in the kernels of router.cu, dispatch.cu,
 // expert_gemm.cu and combine.cu.
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
 
 #include "../../include/moe_b200.h"
+#include "common.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -24,6 +26,14 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("MOE_B200_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 static size_t align256(size_t v) { return (v + 255) & ~size_t(255); }

@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(256) gate_logits_simt_kernel(const Tin* __rest
                                                                float* __restrict__ logits, int64_t T, int d,
                                                                int E) {
   constexpr int V = Vec16<Tin>::N;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -110,9 +112,8 @@ static cudaError_t gate_simt(const Problem& p, const void* x, const void* wg, co
   int64_t blocks = (warps + 7) / 8;
   const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
   if (blocks > cap_blocks) blocks = cap_blocks;
-  gate_logits_simt_kernel<Tin, EB, TPW><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<const Tin*>(x), static_cast<const Tin*>(wg), off, logits, p.T, p.d, p.E);
-  return cudaGetLastError();
+  return launch_k(gate_logits_simt_kernel<Tin, EB, TPW>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                  static_cast<const Tin*>(x), static_cast<const Tin*>(wg), off, logits, p.T, p.d, p.E);
 }
 
 cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void* wg, const float* off,
@@ -153,6 +154,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   static_assert(kDispatchChunk % kSelectTokens == 0, "a selection block must not straddle dispatch chunks");
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < 32 * EPL; e += blockDim.x) s_count[e] = 0;
   __syncthreads();
 
@@ -302,14 +305,17 @@ cudaError_t launch_route_select(const Problem& p, float* logits, const float* pa
   const unsigned blocks = static_cast<unsigned>((p.T + kSelectTokens - 1) / kSelectTokens);
   const int bias_on_logit = (p.flags & 0x2u) ? 1 : 0;
   if (p.E <= 32)
-    route_select_kernel<1><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+    return launch_k(route_select_kernel<1>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   else if (p.E <= 64)
-    route_select_kernel<2><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+    return launch_k(route_select_kernel<2>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   else if (p.E <= 128)
-    route_select_kernel<4><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+    return launch_k(route_select_kernel<4>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
   else
-    route_select_kernel<8><<<blocks, 256, 0, st>>>(logits, parts, n_parts, sel_bias, bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
-  return cudaGetLastError();
+    return launch_k(route_select_kernel<8>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
 }
 
 // ----------------------------------------------------------------------------
@@ -323,6 +329,8 @@ __global__ void __launch_bounds__(1024) route_stats_kernel(const int32_t* __rest
                                                            int n_chunks, int64_t T, int E, int K, float alpha,
                                                            float* __restrict__ stats) {
   __shared__ double s_fp[kMaxExperts];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     long long c = 0;
     unsigned long long ps = 0;
@@ -338,8 +346,8 @@ __global__ void __launch_bounds__(1024) route_stats_kernel(const int32_t* __rest
 
 cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, const unsigned long long* chunk_psum,
                                int n_chunks, float* stats, cudaStream_t st) {
-  route_stats_kernel<<<1, 1024, 0, st>>>(chunk_counts, chunk_psum, n_chunks, p.T, p.E, p.K, p.alpha, stats);
-  return cudaGetLastError();
+  return launch_k(route_stats_kernel, dim3(1), dim3(1024), 0, st, chunk_counts, chunk_psum, n_chunks, p.T, p.E,
+                  p.K, p.alpha, stats);
 }
 
 }  // namespace moe
