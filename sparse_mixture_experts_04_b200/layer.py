@@ -1,6 +1,7 @@
 """MoeLayer: one layer's weights, workspace and routing buffers on the device,
-with forward() = one moe_layer_forward call.  Allocation (through torch) and
-argument marshalling only."""
+with forward() = one moe_layer_forward call, and forward_host() for batches
+that live in (pinned) host memory.  Allocation (through torch), stream
+bookkeeping and argument marshalling only."""
 from __future__ import annotations
 
 import torch
@@ -54,3 +55,48 @@ class MoeLayer:
         return y
 
     __call__ = forward
+
+    def forward_host(self, xs_host, ys_host, stats_host=None, stream=None):
+        """Run one layer forward per host batch: xs_host[i] [T, d] -> ys_host[i].
+
+        Host tensors should be pinned.  The host->device copy of batch i+1 and
+        the device->host copy of batch i-1 run on their own streams while batch
+        i computes (two device buffers each for x and y), so the copy engines
+        overlap the kernels.  stats_host[i] (optional) receives the [2E+1]
+        statistics of batch i.  Returns after every copy has landed."""
+        n = len(xs_host)
+        if n == 0:
+            return
+        dev = self.device
+        comp = stream if stream is not None else torch.cuda.current_stream(dev)
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        T, d = self.prob.T, self.prob.d_model
+        xb = [torch.empty((T, d), dtype=self.dtype, device=dev) for _ in range(2)]
+        yb = [torch.empty((T, d), dtype=self.dtype, device=dev) for _ in range(2)]
+        sb = [torch.empty_like(self.stats) for _ in range(2)]
+        ev = lambda: torch.cuda.Event()
+        copied_in = [ev() for _ in range(n)]
+        computed = [ev() for _ in range(n)]
+        copied_out = [ev() for _ in range(n)]
+        h2d.wait_stream(comp)
+        d2h.wait_stream(comp)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(h2d):
+                if i >= 2:
+                    h2d.wait_event(computed[i - 2])       # x buffer b is free again
+                xb[b].copy_(xs_host[i], non_blocking=True)
+                copied_in[i].record(h2d)
+            comp.wait_event(copied_in[i])
+            if i >= 2:
+                comp.wait_event(copied_out[i - 2])        # y / stats buffers b are free again
+            api.moe_layer_forward(self.prob, xb[b], self.weights, yb[b], self.routing, sb[b], self.ws, comp)
+            computed[i].record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(computed[i])
+                ys_host[i].copy_(yb[b], non_blocking=True)
+                if stats_host is not None:
+                    stats_host[i].copy_(sb[b], non_blocking=True)
+                copied_out[i].record(d2h)
+        comp.wait_stream(d2h)
+        comp.synchronize()

@@ -352,3 +352,20 @@ def test_layer_forward_both_tile_shapes(name, tile, monkeypatch):
     y = layer.forward(dev(inp["x"]))
     assert api.read_device_status(layer.ws) == 0
     assert rel_err(y.float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
+
+
+def test_forward_host_pipelined_matches_device_forward():
+    """MoeLayer.forward_host (host batches in and out, copies overlapped with
+    the kernels on side streams) gives the same bytes as forward() per batch."""
+    cfg = SMALL["mini_zen"]
+    inp = inputs("mini_zen")
+    layer = MoeLayer.from_inputs(inp)
+    gen = torch.Generator().manual_seed(3)
+    xs = [(torch.randn((cfg.T, cfg.d_model), generator=gen)).to(torch.bfloat16).pin_memory() for _ in range(5)]
+    ys = [torch.empty((cfg.T, cfg.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    st = [torch.empty(2 * cfg.n_experts + 1, dtype=torch.float32).pin_memory() for _ in range(5)]
+    layer.forward_host(xs, ys, st)
+    for i in range(5):
+        y = layer.forward(xs[i].cuda())
+        assert torch.equal(ys[i], y.cpu()), i
+        assert torch.equal(st[i], layer.stats.cpu()), i
