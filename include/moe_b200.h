@@ -81,6 +81,9 @@ typedef enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 } moe_dtype;
 #define MOE_FLAG_LOGITS_GIVEN 0x1u /* moe_route / moe_layer_forward read the logits
                                       instead of computing them from x and w_gate */
 #define MOE_FLAG_BIAS_LOGIT 0x2u   /* selection bias added to the logit, not to p */
+#define MOE_FLAG_EXTENDED_STATS 0x4u /* stats has 2E+7 entries: after the 2E+1 balance
+                                        entries, the router z-loss and utilisation
+                                        statistics (see moe_route) */
 
 /* Device status bits (moe_read_device_status). */
 #define MOE_DEV_BAD_EXPERT 0x1     /* an expert index outside [0, E) was skipped */
@@ -170,7 +173,16 @@ int moe_read_device_status(const void* ws, moe_stream_t stream, uint32_t* bits);
  *                with a bias it is computed in float64.
  *   topk_w       [T, K] out: renormalised gate weights (sum to 1 per token)
  *   stats        [2E+1] out or NULL: f_e = counts_e / (T*K) (before the
- *                capacity cut), P_e = mean_t p[t,e], loss = alpha*E*sum f_e P_e */
+ *                capacity cut), P_e = mean_t p[t,e], loss = alpha*E*sum f_e P_e.
+ *                With MOE_FLAG_EXTENDED_STATS, [2E+7]: then
+ *                [2E+1] router z-loss (1/T) sum_t (log sum_e exp l[t,e])^2
+ *                       (Zen-Max §3.2; the coefficient is the caller's),
+ *                [2E+2] entropy in bits of the load shares counts_e / (T*K),
+ *                [2E+3] coefficient of variation of counts (population std / mean),
+ *                [2E+4] drop rate sum(counts - kept) / (T*K), kept = min(counts, cap),
+ *                [2E+5] number of experts with load below 50% of the mean,
+ *                [2E+6] number above 200% of the mean
+ *                (Zen MoDE §6.2, table tab:utilization). */
 int moe_route(const moe_problem_t* p, const void* x, const void* w_gate,
               const float* logit_offset, const float* sel_bias, float* logits,
               int32_t* topk_idx, float* topk_w, float* stats,
@@ -221,7 +233,8 @@ int moe_combine(const moe_problem_t* p, const void* y_perm, const int32_t* slot_
  * combine, plus statistics, enqueued on one stream with no host sync.
  *   x [T, d] in; w weights; y [T, d] out;
  *   routing: optional outputs (NULL or any subset; logits is an input with
- *   MOE_FLAG_LOGITS_GIVEN); stats [2E+1] or NULL (as moe_route).
+ *   MOE_FLAG_LOGITS_GIVEN); stats [2E+1] ([2E+7] with MOE_FLAG_EXTENDED_STATS)
+ *   or NULL (as moe_route).
  * Resets the device status word first. */
 int moe_layer_forward(const moe_problem_t* p, const void* x, const moe_weights_t* w,
                       void* y, const moe_routing_t* routing, float* stats,

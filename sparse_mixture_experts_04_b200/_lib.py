@@ -15,7 +15,8 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_CUDA",
                 -4: "MOE_ERR_DEVICE_CHECK", -5: "MOE_ERR_WORKSPACE"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
-FLAG_LOGITS_GIVEN, FLAG_BIAS_LOGIT = 0x1, 0x2
+FLAG_LOGITS_GIVEN, FLAG_BIAS_LOGIT, FLAG_EXTENDED_STATS = 0x1, 0x2, 0x4
+EXTENDED_STATS = ("z_loss", "entropy_bits", "cv", "drop_rate", "n_below_half", "n_above_double")
 FFN_ROUTED, FFN_SHARED = 0, 1
 DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
 

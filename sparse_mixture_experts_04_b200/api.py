@@ -11,13 +11,14 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (DTYPE_BF16, DTYPE_F32, FFN_ROUTED, FFN_SHARED, FLAG_BIAS_LOGIT, FLAG_LOGITS_GIVEN, MoeError,
-                   MoeProblem, MoeRouting, MoeWeights)
+from ._lib import (DTYPE_BF16, DTYPE_F32, EXTENDED_STATS, FFN_ROUTED, FFN_SHARED, FLAG_BIAS_LOGIT,
+                   FLAG_EXTENDED_STATS, FLAG_LOGITS_GIVEN, MoeError, MoeProblem, MoeRouting, MoeWeights)
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_profiled", "moe_dispatch_noalloc",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
+           "FLAG_EXTENDED_STATS", "EXTENDED_STATS", "stats_size",
            "FFN_ROUTED", "FFN_SHARED", "DTYPE_BF16", "DTYPE_F32"]
 
 
@@ -42,6 +43,11 @@ def _stream(stream) -> int | None:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def stats_size(prob: MoeProblem) -> int:
+    """Entries of the stats array: 2E+1, or 2E+7 with FLAG_EXTENDED_STATS."""
+    return 2 * prob.n_experts + (7 if prob.flags & FLAG_EXTENDED_STATS else 1)
 
 
 def workspace_size(prob: MoeProblem) -> int:

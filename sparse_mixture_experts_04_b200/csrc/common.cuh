@@ -320,6 +320,44 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
 }
 
+// Extended statistics (written after the 2E+1 balance entries when requested):
+//   stats[2E+1] router z-loss  (1/T) sum_t (logsumexp_t)^2   (from zsum = sum of the squares)
+//   stats[2E+2] entropy in bits of the load shares counts_e / sum(counts)
+//   stats[2E+3] coefficient of variation of counts (population std / mean)
+//   stats[2E+4] drop rate: sum(counts - kept) / sum(counts)
+//   stats[2E+5] experts below 50% of the mean load; stats[2E+6] above 200%
+// counts / kept are read from shared or global memory; one thread, expert order.
+constexpr int kExtendedStats = 6;
+
+__device__ __forceinline__ void utilisation_stats(const int* counts, const int* kept, int E, int64_t T,
+                                                  double zsum, float* stats) {
+  double n = 0.0, dropped = 0.0;
+  for (int e = 0; e < E; ++e) {
+    n += counts[e];
+    dropped += static_cast<double>(counts[e] - kept[e]);
+  }
+  const double mean = n / E;
+  double ent = 0.0, var = 0.0, below = 0.0, above = 0.0;
+  for (int e = 0; e < E; ++e) {
+    if (counts[e] > 0) {
+      const double q = counts[e] / n;
+      ent -= q * log2(q);
+    }
+    const double dv = counts[e] - mean;
+    var += dv * dv;
+    if (counts[e] < 0.5 * mean) below += 1.0;
+    if (counts[e] > 2.0 * mean) above += 1.0;
+  }
+  var /= E;
+  float* x = stats + 2 * E + 1;
+  x[0] = static_cast<float>(zsum / static_cast<double>(T));
+  x[1] = static_cast<float>(ent);
+  x[2] = static_cast<float>(mean > 0.0 ? sqrt(var) / mean : 0.0);
+  x[3] = static_cast<float>(n > 0.0 ? dropped / n : 0.0);
+  x[4] = static_cast<float>(below);
+  x[5] = static_cast<float>(above);
+}
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

@@ -60,11 +60,14 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
                                                              int32_t* __restrict__ seg_off,
                                                              const unsigned long long* __restrict__ chunk_psum,
                                                              float* __restrict__ stats, int64_t T, int K,
-                                                             float alpha) {
+                                                             float alpha, const float* __restrict__ zpart,
+                                                             int n_zpart) {
   __shared__ int part[1024];
   __shared__ unsigned long long ppart[1024];
   __shared__ int s_kept[kMaxExperts];
+  __shared__ int s_count[kMaxExperts];
   __shared__ double s_fp[kMaxExperts];
+  __shared__ double s_zsum[1024];
   pdl_wait();
   pdl_trigger();
   int S = 1024 / E;
@@ -100,10 +103,25 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
     const int k = (cap < 0 || run < cap) ? run : static_cast<int>(cap);
     kept[e] = k;
     s_kept[e] = k;
+    s_count[e] = run;
     if (stats) s_fp[e] = balance_stats_expert(run, prun, T, E, K, e, stats);
   }
+  if (stats && zpart) {  // router z-loss partials: strided per thread, then a fixed-shape tree
+    double z = 0.0;
+    for (int b = tid; b < n_zpart; b += 1024) z += zpart[b];
+    s_zsum[tid] = z;
+  }
   __syncthreads();
-  if (stats && tid == 32) balance_loss(s_fp, E, alpha, stats);
+  if (stats && zpart) {
+    for (int w = 512; w > 0; w >>= 1) {
+      if (tid < w) s_zsum[tid] += s_zsum[tid + w];
+      __syncthreads();
+    }
+  }
+  if (stats && tid == 32) {
+    balance_loss(s_fp, E, alpha, stats);
+    if (zpart) utilisation_stats(s_count, s_kept, E, T, s_zsum[0], stats);
+  }
   if (active) {
     int run = part[tid];
     for (int c = c0; c < c1; ++c) {
@@ -192,7 +210,7 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
 cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready,
-                            const unsigned long long* chunk_psum, float* stats) {
+                            const unsigned long long* chunk_psum, float* stats, const float* zpart, int n_zpart) {
   const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
   if (!counts_ready) {
     if (cudaError_t e = launch_k(dispatch_hist_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
@@ -202,7 +220,7 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
   if (cudaError_t e = launch_k(dispatch_scan_kernel, dim3(1), dim3(1024), 0, st,
                                static_cast<const int32_t*>(chunk_counts), n_chunks, p.E, static_cast<long long>(p.cap),
                                chunk_base, counts, kept, seg_off, chunk_psum, chunk_psum ? stats : nullptr, p.T,
-                               p.K, p.alpha))
+                               p.K, p.alpha, zpart, n_zpart))
     return e;
   return launch_k(dispatch_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
                   static_cast<const int32_t*>(chunk_base), static_cast<const int32_t*>(kept),

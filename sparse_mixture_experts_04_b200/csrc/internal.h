@@ -33,11 +33,11 @@ struct Problem {
 // Byte offsets of every scratch array inside the caller's workspace.
 struct WsLayout {
   size_t status, logits, topk_idx, topk_w, counts, kept, seg_off, slot_of, perm;
-  size_t chunk_counts, chunk_psum, chunk_base, logit_parts;
+  size_t chunk_counts, chunk_psum, chunk_base, logit_parts, zpart;
   size_t zero_bytes;  // status word + chunk histogram + chunk p sums: cleared together at offset 0
   size_t x_perm, h_routed, y_perm, h_shared, y_shared;
   size_t total;
-  int n_chunks;
+  int n_chunks, n_sel_blocks;
 };
 WsLayout make_layout(const Problem& p);
 
@@ -52,22 +52,27 @@ cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void*
 // chunk_counts / chunk_psum: zeroed [n_chunks, E] arrays that receive, per
 // dispatch chunk, the histogram of the chosen experts and the sum of p in
 // fixed point (p_fixed_scale; integer atomics: exact and order-independent)
+// zpart (or nullptr): [n_selection_blocks] sums of logsumexp^2 (router z-loss)
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
                                 const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
-                                unsigned long long* chunk_psum, cudaStream_t st);
-// f, P and the loss from those chunk totals (moe_route's statistics)
+                                unsigned long long* chunk_psum, float* zpart, cudaStream_t st);
+// f, P and the loss from those chunk totals (moe_route's statistics); with
+// zpart also the extended statistics (kept = min(counts, cap))
 cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, const unsigned long long* chunk_psum,
-                               int n_chunks, float* stats, cudaStream_t st);
+                               int n_chunks, const float* zpart, int n_zpart, float* stats, cudaStream_t st);
 
 // dispatch.cu
 // counts_ready: chunk_counts already hold the per-chunk expert histogram (the
 // selection kernel adds it when given a zeroed chunk_counts)
 // chunk_psum / stats: when both are given, the scan also finalises the
 // balance statistics from the selection kernel's chunk totals.
+// zpart / n_zpart: per-selection-block sums of logsumexp^2; given with stats,
+// the extended statistics are written too.
 cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready = false,
-                            const unsigned long long* chunk_psum = nullptr, float* stats = nullptr);
+                            const unsigned long long* chunk_psum = nullptr, float* stats = nullptr,
+                            const float* zpart = nullptr, int n_zpart = 0);
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
                           void* x_perm, cudaStream_t st);
 

@@ -44,6 +44,7 @@ WsLayout make_layout(const Problem& p) {
   const size_t TK = static_cast<size_t>(p.T) * p.K;
   const size_t R = static_cast<size_t>(p.max_rows);
   L.n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
+  L.n_sel_blocks = static_cast<int>((p.T + kSelectTokens - 1) / kSelectTokens);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -68,6 +69,7 @@ WsLayout make_layout(const Problem& p) {
   L.chunk_base = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
   const int splits = (p.dtype == kBF16) ? router_k_splits(p) : 1;
   L.logit_parts = take(splits > 1 ? static_cast<size_t>(splits) * p.T * p.E * 4 : 0);
+  L.zpart = take(static_cast<size_t>(L.n_sel_blocks) * 4);
   L.x_perm = take(R * p.d * es);
   L.h_routed = take(R * p.F * es);
   L.y_perm = take(R * p.d * es);
@@ -86,7 +88,7 @@ static int to_problem(const moe_problem_t* in, Problem* out) {
   if (q.T < 1 || q.d_model < 8 || q.d_ff < 8 || (q.d_model % 8) || (q.d_ff % 8)) return MOE_ERR_INVALID_ARG;
   if (q.n_experts < 1 || q.top_k < 1 || q.top_k > q.n_experts || q.n_shared < 0) return MOE_ERR_INVALID_ARG;
   if (q.dtype != MOE_DTYPE_BF16 && q.dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
-  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT)) return MOE_ERR_INVALID_ARG;
+  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT | MOE_FLAG_EXTENDED_STATS)) return MOE_ERR_INVALID_ARG;
   if (!(q.alpha == q.alpha) || !(q.capacity_factor == q.capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (q.n_experts > kMaxExperts || q.top_k > kMaxTopK || q.n_shared > 256) return MOE_ERR_UNSUPPORTED;
   const int64_t lim = static_cast<int64_t>(1) << 31;
@@ -164,10 +166,13 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
   }
   int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
   unsigned long long* chunk_psum = at<unsigned long long>(ws, L.chunk_psum);
-  if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, chunk_counts, chunk_psum, st))
+  float* zpart = (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr;
+  if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, chunk_counts, chunk_psum,
+                                          zpart, st))
     return cuda_rc(e);
   if (stats && stats_in_route) {
-    if (cudaError_t e = launch_route_stats(p, chunk_counts, chunk_psum, L.n_chunks, stats, st)) return cuda_rc(e);
+    if (cudaError_t e = launch_route_stats(p, chunk_counts, chunk_psum, L.n_chunks, zpart, L.n_sel_blocks, stats, st))
+      return cuda_rc(e);
   }
   return MOE_OK;
 }
@@ -341,7 +346,9 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   // the scan also finalises the balance statistics from the chunk totals
   if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, at<int32_t>(ws, L.chunk_counts),
                                       at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true,
-                                      at<unsigned long long>(ws, L.chunk_psum), stats))
+                                      at<unsigned long long>(ws, L.chunk_psum), stats,
+                                      (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr,
+                                      L.n_sel_blocks))
     return cuda_rc(e);
   kernels += 2;
   if (p.max_rows > 0) {

@@ -147,9 +147,10 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
                                                            float* __restrict__ topk_w, int64_t T, int E, int K,
                                                            int32_t* __restrict__ chunk_counts,
                                                            unsigned long long* __restrict__ chunk_psum,
-                                                           double pscale) {
+                                                           double pscale, float* __restrict__ zpart) {
   __shared__ float s_psum[8][32 * EPL];
   __shared__ int s_count[32 * EPL];
+  __shared__ float s_z[8];
   // the fixed-point block sums below cover at most kSelectTokens tokens
   static_assert(kDispatchChunk % kSelectTokens == 0, "a selection block must not straddle dispatch chunks");
   const int lane = threadIdx.x & 31;
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   float pacc[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) pacc[i] = 0.f;
+  float zacc = 0.f;  // sum over this warp's tokens of logsumexp^2 (router z-loss)
 
   const int64_t tok_begin = static_cast<int64_t>(blockIdx.x) * kSelectTokens;
   constexpr int kPerWarp = kSelectTokens / 8;
@@ -198,6 +200,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
     }
     const float Z = warp_sum(zloc);
     const float invZ = 1.0f / Z;
+    const float lse = m + logf(Z);
+    zacc += lse * lse;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) pacc[i] += ex[i] * invZ;
 
@@ -284,12 +288,19 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   }
 #pragma unroll
   for (int i = 0; i < EPL; ++i) s_psum[warp][lane + 32 * i] = pacc[i];
+  if (lane == 0) s_z[warp] = zacc;
   __syncthreads();
   // Per-dispatch-chunk totals (this block's tokens lie in one chunk, since
   // kDispatchChunk is a multiple of kSelectTokens): the expert histogram and
   // the sum of p as a fixed-point integer (scale p_fixed_scale(T)).  Integer adds commute, so the
   // totals do not depend on the order in which blocks arrive.
   const int64_t chunk = tok_begin / kDispatchChunk;
+  if (zpart && threadIdx.x == 0) {
+    float z = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) z += s_z[w];
+    zpart[blockIdx.x] = z;
+  }
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     float s = 0.f;
 #pragma unroll
@@ -301,21 +312,21 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
 
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
                                 const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
-                                unsigned long long* chunk_psum, cudaStream_t st) {
+                                unsigned long long* chunk_psum, float* zpart, cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>((p.T + kSelectTokens - 1) / kSelectTokens);
   const int bias_on_logit = (p.flags & 0x2u) ? 1 : 0;
   if (p.E <= 32)
     return launch_k(route_select_kernel<1>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
   else if (p.E <= 64)
     return launch_k(route_select_kernel<2>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
   else if (p.E <= 128)
     return launch_k(route_select_kernel<4>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
   else
     return launch_k(route_select_kernel<8>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T));
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
 }
 
 // ----------------------------------------------------------------------------
@@ -327,8 +338,12 @@ cudaError_t launch_route_select(const Problem& p, float* logits, const float* pa
 __global__ void __launch_bounds__(1024) route_stats_kernel(const int32_t* __restrict__ chunk_counts,
                                                            const unsigned long long* __restrict__ chunk_psum,
                                                            int n_chunks, int64_t T, int E, int K, float alpha,
-                                                           float* __restrict__ stats) {
+                                                           long long cap, const float* __restrict__ zpart,
+                                                           int n_zpart, float* __restrict__ stats) {
   __shared__ double s_fp[kMaxExperts];
+  __shared__ int s_c[kMaxExperts];
+  __shared__ int s_k[kMaxExperts];
+  __shared__ double s_zsum[1024];
   pdl_wait();
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -339,15 +354,31 @@ __global__ void __launch_bounds__(1024) route_stats_kernel(const int32_t* __rest
       ps += chunk_psum[static_cast<int64_t>(ch) * E + e];
     }
     s_fp[e] = balance_stats_expert(c, ps, T, E, K, e, stats);
+    s_c[e] = static_cast<int>(c);
+    s_k[e] = (cap < 0 || c < cap) ? static_cast<int>(c) : static_cast<int>(cap);
+  }
+  if (zpart) {  // router z-loss partials: strided per thread, then a fixed-shape tree
+    double z = 0.0;
+    for (int b = threadIdx.x; b < n_zpart; b += blockDim.x) z += zpart[b];
+    s_zsum[threadIdx.x] = z;
   }
   __syncthreads();
-  if (threadIdx.x == 0) balance_loss(s_fp, E, alpha, stats);
+  if (zpart) {
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (threadIdx.x < w) s_zsum[threadIdx.x] += s_zsum[threadIdx.x + w];
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x == 0) {
+    balance_loss(s_fp, E, alpha, stats);
+    if (zpart) utilisation_stats(s_c, s_k, E, T, s_zsum[0], stats);
+  }
 }
 
 cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, const unsigned long long* chunk_psum,
-                               int n_chunks, float* stats, cudaStream_t st) {
+                               int n_chunks, const float* zpart, int n_zpart, float* stats, cudaStream_t st) {
   return launch_k(route_stats_kernel, dim3(1), dim3(1024), 0, st, chunk_counts, chunk_psum, n_chunks, p.T, p.E,
-                  p.K, p.alpha, stats);
+                  p.K, p.alpha, static_cast<long long>(p.cap), zpart, n_zpart, stats);
 }
 
 }  // namespace moe

@@ -25,7 +25,7 @@ class MoeLayer:
                 topk_idx=torch.empty((T, K), **i32), topk_w=torch.empty((T, K), dtype=torch.float32, device=self.device),
                 counts=torch.empty(E, **i32), kept=torch.empty(E, **i32), seg_off=torch.empty(E + 1, **i32),
                 slot_of=torch.empty((T, K), **i32), perm=torch.empty(max(api.max_rows(prob), 1), **i32))
-        self.stats = torch.empty(2 * E + 1, dtype=torch.float32, device=self.device)
+        self.stats = torch.empty(api.stats_size(prob), dtype=torch.float32, device=self.device)
 
     @classmethod
     def from_inputs(cls, inputs: dict, device="cuda", flags: int = 0, keep_routing: bool = True) -> "MoeLayer":

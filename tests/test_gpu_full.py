@@ -36,7 +36,7 @@ def test_full_size_given_logits(workload):
     name, cfg, inp = workload
     logits32 = given_logits(cfg)
     ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
-    layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN)
+    layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN | api.FLAG_EXTENDED_STATS)
     layer.routing["logits"].copy_(torch.as_tensor(logits32))
     y = layer.forward(dev(inp["x"]))
     assert api.read_device_status(layer.ws) == 0
@@ -52,6 +52,13 @@ def test_full_size_given_logits(workload):
     assert (st[:E] == ref["f"].astype(np.float32)).all()
     assert np.max(np.abs(st[E:2 * E] - ref["P"])) <= 1e-6
     assert abs(st[2 * E] - ref["loss"]) <= 1e-6 * max(1.0, ref["loss"])
+    z = oracle.router_zloss(logits32.astype(np.float64))
+    u = oracle.utilization(ref["counts"], ref["kept"])
+    x = st[2 * E + 1:]
+    assert abs(x[0] - z) <= 1e-5 * max(1.0, z)
+    assert abs(x[1] - u["entropy_bits"]) <= 1e-5 * max(1.0, u["entropy_bits"])
+    assert abs(x[2] - u["cv"]) <= 1e-5 * max(1.0, u["cv"]) and abs(x[3] - u["drop_rate"]) <= 1e-6
+    assert x[4] == u["n_below_half"] and x[5] == u["n_above_double"]
     # sampled outputs, including tokens with dropped pairs when there are any
     dropped = np.nonzero((ref["slot_of"] < 0).any(1))[0][:4]
     rows = sample_rows(cfg.T, N_SAMPLE[name], seed=cfg.seed, extra=tuple(int(t) for t in dropped))

@@ -369,3 +369,51 @@ def test_forward_host_pipelined_matches_device_forward():
         y = layer.forward(xs[i].cuda())
         assert torch.equal(ys[i], y.cpu()), i
         assert torch.equal(st[i], layer.stats.cpu()), i
+
+
+# ------------------------------------------------- extended statistics (f1)
+def _check_extended(stats, E, logits64, counts, kept):
+    x = stats[2 * E + 1:]
+    z = oracle.router_zloss(logits64)
+    u = oracle.utilization(counts, kept)
+    assert abs(x[0] - z) <= 1e-5 * max(1.0, abs(z))
+    assert abs(x[1] - u["entropy_bits"]) <= 1e-5 * max(1.0, u["entropy_bits"])
+    assert abs(x[2] - u["cv"]) <= 1e-5 * max(1.0, u["cv"])
+    assert abs(x[3] - u["drop_rate"]) <= 1e-6
+    assert x[4] == u["n_below_half"] and x[5] == u["n_above_double"]
+
+
+@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "mini_skewed", "tiny_capacity", "wide_e256"])
+def test_route_extended_stats_match_oracle(name):
+    cfg = SMALL[name]
+    inp = inputs(name)
+    logits32 = given_logits(cfg)
+    flags = api.FLAG_LOGITS_GIVEN | api.FLAG_EXTENDED_STATS
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    prob = problem(cfg, flags)
+    ws = api.alloc_workspace(prob)
+    T, E, K = cfg.T, cfg.n_experts, cfg.top_k
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    stats = torch.empty(api.stats_size(prob), dtype=torch.float32, device="cuda")
+    api.moe_route(prob, None, None, None, dev(inp["sel_bias"]), dev(logits32), idx, w, stats, ws)
+    st = stats.cpu().numpy()
+    assert (st[:E] == ref["f"].astype(np.float32)).all()
+    _check_extended(st, E, logits32.astype(np.float64), ref["counts"], ref["kept"])
+
+
+@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "ragged_f32", "tiny_capacity"])
+def test_layer_extended_stats_match_oracle(name):
+    cfg = SMALL[name]
+    inp = inputs(name)
+    logits32 = given_logits(cfg)
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN | api.FLAG_EXTENDED_STATS)
+    layer.routing["logits"].copy_(torch.as_tensor(logits32))
+    layer.forward(dev(inp["x"]))
+    st = layer.stats.cpu().numpy()
+    E = cfg.n_experts
+    assert st.shape[0] == 2 * E + 7
+    assert np.max(np.abs(st[E:2 * E] - ref["P"])) <= 1e-6
+    assert abs(st[2 * E] - ref["loss"]) <= 1e-6 * max(1.0, ref["loss"])
+    _check_extended(st, E, logits32.astype(np.float64), ref["counts"], ref["kept"])
