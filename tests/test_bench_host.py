@@ -1,0 +1,40 @@
+"""Host-side arithmetic of bench.py: the roofline's bound and byte counts."""
+import os
+import sys
+
+import pytest
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+from sparse_mixture_experts_04_b200.synth import CONFIGS  # noqa: E402
+
+PEAKS = {"hbm_gbs": 6540.8, "bf16_tflops": 1641.2, "bf16_tflops_sustained": 1380.6}
+
+
+def test_up_gemm_bytes_counts_touched_experts_rows_and_h():
+    cfg = CONFIGS["mixtral"]
+    kept = [1024] * 7 + [0]
+    d, F = cfg.d_model, cfg.d_ff
+    want = 2 * (7 * 2 * F * d + 7 * 1024 * d + 7 * 1024 * F)
+    assert bench.up_gemm_bytes(cfg, kept) == want
+
+
+def test_roofline_is_tensor_bound_for_large_groups():
+    cfg = CONFIGS["mixtral"]
+    kept = [1024] * 8
+    flops = bench.algorithmic_flops(cfg, sum(kept))["up"]
+    r = bench.roofline(cfg, flops, bench.up_gemm_bytes(cfg, kept), 1.5, PEAKS, "measured", None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(flops / 1.5e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
+
+
+def test_roofline_is_hbm_bound_when_weights_dominate():
+    cfg = CONFIGS["decode"]
+    kept = [2] * cfg.n_experts          # a few rows per expert: weight streaming
+    flops = bench.algorithmic_flops(cfg, sum(kept))["up"]
+    nbytes = bench.up_gemm_bytes(cfg, kept)
+    r = bench.roofline(cfg, flops, nbytes, 0.5, PEAKS, "fallback", None)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(nbytes / 0.5e-3 / 1e9)
+    assert r["peak"] == PEAKS["hbm_gbs"] and "fallback" in r["peak_source"]
