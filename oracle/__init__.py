@@ -16,6 +16,11 @@ Parity pins (what ties each function to something other than itself) are in
   select         brute-force full sort on tiny inputs; tie rule; renormalisation
   capacity       exact integer cases printed in the configs' arithmetic
   dispatch       brute force per-expert queues; bijection and order invariants
+  dispatch_caps  brute force per-expert queues with a different capacity per expert
+  bias_update    hand-worked loads: overloaded down, underloaded up, balanced unchanged;
+                 proportional steps sum to zero; a fixed routing drives the biases apart
+  adaptive_capacity  hand-worked C_e / cap_e; gamma = 0 and a uniform window give the
+                 uniform capacity; window mean; clamps to [0, T]; monotone in the load
   swiglu         one-hot weights reduce each output to silu(a) * b closed form
   combine        grouped SwiGLU outputs combined equal layer_rows; hand example
   layer_rows     E=1, K=1 reduces to one dense SwiGLU; shared experts equal one
@@ -71,6 +76,12 @@ def _L():
         lib.oracle_capacity.restype = i64
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i64, P, P, P, P, P, P]
         lib.oracle_dispatch.restype = ctypes.c_int
+        lib.oracle_dispatch_caps.argtypes = [i64, i32, i32, P, P, P, P, P, P, P]
+        lib.oracle_dispatch_caps.restype = ctypes.c_int
+        lib.oracle_bias_update.argtypes = [i32, i64, P, P, f32, i32]
+        lib.oracle_bias_update.restype = None
+        lib.oracle_adaptive_capacity.argtypes = [i64, i32, i32, P, i32, f32, f32, P]
+        lib.oracle_adaptive_capacity.restype = None
         lib.oracle_swiglu_accumulate.argtypes = [i32, i32, P, P, P, i32, f64, P, P]
         lib.oracle_swiglu_accumulate.restype = None
         lib.oracle_layer_rows.argtypes = [i64, i32, i32, i32, i32, i32, P, i32, P, P, P, P, i32,
@@ -180,6 +191,49 @@ def dispatch(idx, E, cap):
         raise ValueError("expert index out of range")
     return dict(counts=counts, kept=kept, seg_off=seg_off, slot_of=slot_of,
                 perm=perm[: int(seg_off[E])].copy())
+
+
+def dispatch_caps(idx, E, caps):
+    """dispatch() with one capacity per expert (caps[e] < 0: no limit), Zen MoDE
+    §5.3 capacity_e per expert."""
+    ia = np.ascontiguousarray(idx, dtype=np.int32)
+    T, K = ia.shape
+    ca = np.ascontiguousarray(caps, dtype=np.int64)
+    assert ca.shape == (E,)
+    counts = np.empty(E, np.int32)
+    kept = np.empty(E, np.int32)
+    seg_off = np.empty(E + 1, np.int32)
+    slot_of = np.empty((T, K), np.int32)
+    perm = np.full(max(T * K, 1), -1, np.int32)
+    rc = _L().oracle_dispatch_caps(T, K, E, _ptr(ca), _ptr(ia), _ptr(counts), _ptr(kept), _ptr(seg_off),
+                                   _ptr(slot_of), _ptr(perm))
+    if rc != 0:
+        raise ValueError("expert index out of range")
+    return dict(counts=counts, kept=kept, seg_off=seg_off, slot_of=slot_of,
+                perm=perm[: int(seg_off[E])].copy())
+
+
+BIAS_UPDATE_SIGN, BIAS_UPDATE_PROPORTIONAL = 0, 1
+
+
+def bias_update(counts, TK, bias, rate, mode=BIAS_UPDATE_SIGN):
+    """One selection-bias update after a step (Zen-Max §2.3): overloaded experts'
+    biases go down, underloaded ones' up.  Returns the new float32 biases."""
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    b = np.array(bias, dtype=np.float32, copy=True)
+    assert b.shape == c.shape
+    _L().oracle_bias_update(int(c.shape[0]), int(TK), _ptr(c), _ptr(b), float(rate), int(mode))
+    return b
+
+
+def adaptive_capacity(T, K, hist, c_base, gamma):
+    """Per-expert capacities from the counts of the last n batches, hist [n, E]
+    (Zen MoDE §5.3 Adaptive Capacity Factors).  Returns int64 [E]."""
+    h = np.ascontiguousarray(hist, dtype=np.int32)
+    n, E = h.shape
+    caps = np.empty(E, np.int64)
+    _L().oracle_adaptive_capacity(int(T), int(K), int(E), _ptr(h), int(n), float(c_base), float(gamma), _ptr(caps))
+    return caps
 
 
 def swiglu(x_row, w13, w2):

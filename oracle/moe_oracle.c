@@ -161,9 +161,11 @@ int64_t oracle_capacity(int64_t T, int32_t K, int32_t E, float C) {
  * Capacity-limited dispatch.  [SE] "A budget": an expert accepts a bounded
  * number of tokens per batch; an assignment beyond that bound is dropped, so
  * the expert does not process that token, which keeps only its residual path.
+ * [ZM] §5.3 lets that bound differ per expert (capacity_e), so it is given
+ * here per expert:
  *
  *   counts[e]  = number of (t,k) with idx[t,k] == e               (pre-capacity)
- *   kept[e]    = min(counts[e], cap)        (counts[e] if cap < 0)
+ *   kept[e]    = min(counts[e], caps[e])    (counts[e] if caps[e] < 0)
  *   seg_off    = exclusive prefix sum of kept; seg_off[E] = total kept rows
  *   rank(t,k)  = number of tokens t' < t that also chose e = idx[t,k]
  *   kept iff rank < kept[e]; then slot_of[t,k] = seg_off[e] + rank and
@@ -171,17 +173,17 @@ int64_t oracle_capacity(int64_t T, int32_t K, int32_t E, float C) {
  * Tokens are served in ascending token order (first come, first served).
  * Returns 0, or -1 on an expert index outside [0, E).
  * ------------------------------------------------------------------------- */
-int oracle_dispatch(int64_t T, int32_t K, int32_t E, int64_t cap,
-                    const int32_t* idx,
-                    int32_t* counts, int32_t* kept, int32_t* seg_off,
-                    int32_t* slot_of, int32_t* perm) {
+int oracle_dispatch_caps(int64_t T, int32_t K, int32_t E, const int64_t* caps,
+                         const int32_t* idx,
+                         int32_t* counts, int32_t* kept, int32_t* seg_off,
+                         int32_t* slot_of, int32_t* perm) {
     for (int32_t e = 0; e < E; ++e) counts[e] = 0;
     for (int64_t i = 0; i < T * (int64_t)K; ++i) {
         if (idx[i] < 0 || idx[i] >= E) return -1;
         counts[idx[i]] += 1;
     }
     for (int32_t e = 0; e < E; ++e)
-        kept[e] = (cap < 0 || counts[e] < cap) ? counts[e] : (int32_t)cap;
+        kept[e] = (caps[e] < 0 || counts[e] < caps[e]) ? counts[e] : (int32_t)caps[e];
     seg_off[0] = 0;
     for (int32_t e = 0; e < E; ++e) seg_off[e + 1] = seg_off[e] + kept[e];
 
@@ -202,6 +204,69 @@ int oracle_dispatch(int64_t T, int32_t K, int32_t E, int64_t cap,
     }
     free(seen);
     return 0;
+}
+
+/* The same dispatch with one capacity for every expert (cap < 0: no limit). */
+int oracle_dispatch(int64_t T, int32_t K, int32_t E, int64_t cap,
+                    const int32_t* idx,
+                    int32_t* counts, int32_t* kept, int32_t* seg_off,
+                    int32_t* slot_of, int32_t* perm) {
+    int64_t* caps = (int64_t*)malloc((size_t)E * sizeof(int64_t));
+    for (int32_t e = 0; e < E; ++e) caps[e] = cap;
+    int rc = oracle_dispatch_caps(T, K, E, caps, idx, counts, kept, seg_off, slot_of, perm);
+    free(caps);
+    return rc;
+}
+
+/* ---------------------------------------------------------------------------
+ * Selection-bias update.  [ZX] §2.3 Auxiliary-Loss-Free Load Balancing: after
+ * a training step each expert's bias b_e moves against the deviation of its
+ * load from the target: an overloaded expert's bias goes down, an underloaded
+ * one's up.  The page gives neither the load measure nor the step size; the
+ * reading taken here: load = counts[e] (assignments before the capacity cut),
+ * target = T*K / E (the mean load), step size `rate`, and either
+ *   mode 0 (sign):          b_e += rate * sign(T*K - E*counts[e])
+ *   mode 1 (proportional):  b_e += rate * (T*K - E*counts[e]) / (T*K)
+ * (mode 1 is the relative deviation (target - load) / target).  Each update is
+ * evaluated in float64 and rounded once to the float32 bias.  TK = T*K.
+ * ------------------------------------------------------------------------- */
+void oracle_bias_update(int32_t E, int64_t TK, const int32_t* counts, float* bias,
+                        float rate, int32_t mode) {
+    for (int32_t e = 0; e < E; ++e) {
+        int64_t dev = TK - (int64_t)E * (int64_t)counts[e];   /* E * (target - load) */
+        double step;
+        if (mode == 0)
+            step = (double)rate * (double)((dev > 0) - (dev < 0));
+        else
+            step = (double)rate * ((double)dev / (double)TK);
+        bias[e] = (float)((double)bias[e] + step);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * Adaptive per-expert capacity.  [ZM] §5.3 Adaptive Capacity Factors:
+ *   C_e = C_base + gamma * (fbar_e - 1/N_E)
+ * with fbar_e the expert's load fraction over a rolling window of recent
+ * batches, so an expert that has been receiving less than its share gets a
+ * smaller budget and one receiving more gets a larger one.  Reading: fbar_e is
+ * the mean over the last n batches of f_e = counts[e] / (T*K) (the balance
+ * statistic's f, pre-capacity); hist holds those n batches' counts, [n, E]
+ * row-major (T and K fixed, so the mean of the fractions is the window's
+ * summed counts over n*T*K).  The capacity is then capacity_e with C_e in
+ * place of C, K-scaled like the uniform one:
+ *   cap_e = ceil(C_e * (T*K) / E), clamped to [0, T].
+ * ------------------------------------------------------------------------- */
+void oracle_adaptive_capacity(int64_t T, int32_t K, int32_t E, const int32_t* hist, int32_t n,
+                              float c_base, float gamma, int64_t* caps) {
+    int64_t TK = T * (int64_t)K;
+    for (int32_t e = 0; e < E; ++e) {
+        int64_t s = 0;
+        for (int32_t i = 0; i < n; ++i) s += hist[(int64_t)i * E + e];
+        double fbar = (double)s / ((double)n * (double)TK);
+        double ce = (double)c_base + (double)gamma * (fbar - 1.0 / (double)E);
+        double v = ceil((ce * (double)TK) / (double)E);
+        caps[e] = v <= 0.0 ? 0 : (v >= (double)T ? T : (int64_t)v);
+    }
 }
 
 /* SiLU, [ZX] §2.2 (activation): silu(z) = z * sigmoid(z) = z / (1 + e^-z). */

@@ -163,13 +163,15 @@ def test_capacity_closed_forms():
 
 # -------------------------------------------------------------------- dispatch
 def _brute_dispatch(idx, E, cap):
+    """cap: one capacity for all experts, or a list with one per expert (< 0: no limit)."""
+    caps = list(cap) if hasattr(cap, "__len__") else [cap] * E
     T, K = idx.shape
     queues = [[] for _ in range(E)]
     for t in range(T):
         for k in range(K):
             queues[idx[t, k]].append((t, k))
     counts = [len(q) for q in queues]
-    kept = [c if cap < 0 else min(c, cap) for c in counts]
+    kept = [c if cp < 0 else min(c, cp) for c, cp in zip(counts, caps)]
     seg = [0]
     for e in range(E):
         seg.append(seg[-1] + kept[e])
@@ -202,6 +204,20 @@ def test_dispatch_matches_per_expert_queues(T, E, K, cap):
     kept_mask = got["slot_of"] >= 0
     assert kept_mask.sum() == seg[-1]
     assert sorted(got["slot_of"][kept_mask].tolist()) == list(range(seg[-1]))
+
+
+@pytest.mark.parametrize("T,E,K", [(1, 1, 1), (37, 5, 2), (257, 7, 3), (64, 16, 4)])
+def test_dispatch_caps_matches_per_expert_queues(T, E, K):
+    rng = np.random.default_rng(7 * T + E)
+    pr = 1.0 / np.arange(1, E + 1) ** 1.2
+    pr /= pr.sum()
+    idx = np.stack([rng.choice(E, size=K, replace=False, p=pr) for _ in range(T)]).astype(np.int32)
+    caps = rng.integers(-1, max(2, T // 2), size=E)          # includes no-limit (-1) and 0
+    got = oracle.dispatch_caps(idx, E, caps)
+    counts, kept, seg, slot_of, perm = _brute_dispatch(idx, E, caps.tolist())
+    assert list(got["counts"]) == counts and list(got["kept"]) == kept and list(got["seg_off"]) == seg
+    assert (got["slot_of"] == slot_of).all()
+    assert list(got["perm"]) == perm
 
 
 def test_dispatch_rejects_out_of_range_expert():
@@ -414,3 +430,86 @@ def test_flops_ratio_golden_compute_budget():
     assert ratio == g["ratio_numerator"] / g["ratio_denominator"]
     assert round(100 * ratio, 1) == g["printed_percent"]
     assert expert == 6.0 * 7168 * 2048 * (K + Ns) * T
+
+
+# ----------------------------------------------------- bias update (Zen-Max §2.3)
+def test_bias_update_sign_hand_example():
+    # E=4, T*K=8: target load 2.  Loads 4, 2, 1, 1: overloaded, balanced, under, under.
+    b = oracle.bias_update([4, 2, 1, 1], 8, [0.0, 0.0, 0.0, 0.0], 0.125, oracle.BIAS_UPDATE_SIGN)
+    assert b.tolist() == [-0.125, 0.0, 0.125, 0.125]
+    b2 = oracle.bias_update([4, 2, 1, 1], 8, b, 0.125, oracle.BIAS_UPDATE_SIGN)
+    assert b2.tolist() == [-0.25, 0.0, 0.25, 0.25]
+
+
+def test_bias_update_proportional_hand_example_and_zero_sum():
+    # relative deviation (target - load) / target = (2 - c) / 2
+    b = oracle.bias_update([4, 2, 1, 1], 8, [1.0, 1.0, 1.0, 1.0], 0.5, oracle.BIAS_UPDATE_PROPORTIONAL)
+    assert b.tolist() == [0.5, 1.0, 1.25, 1.25]
+    rng = np.random.default_rng(3)
+    for E in (3, 8, 64):
+        counts = rng.multinomial(1000, np.ones(E) / E).astype(np.int32)
+        d = oracle.bias_update(counts, 1000, np.zeros(E), 1.0, oracle.BIAS_UPDATE_PROPORTIONAL)
+        # the steps are E*(target - load)/TK: they sum to zero up to one rounding each
+        assert abs(float(np.sum(d.astype(np.float64)))) <= E * 2.0 ** -23
+
+
+def test_bias_update_balanced_load_leaves_bias_unchanged():
+    for mode in (oracle.BIAS_UPDATE_SIGN, oracle.BIAS_UPDATE_PROPORTIONAL):
+        b0 = np.array([0.3, -0.2, 0.0, 1e-3], np.float32)
+        assert (oracle.bias_update([5, 5, 5, 5], 20, b0, 0.01, mode) == b0).all()
+
+
+def test_bias_update_closes_the_loop_on_a_fixed_router():
+    # Fixed probabilities favouring expert 0; top-1 selection on p + b.  Repeated
+    # updates must pull the selection towards a balanced load (the page's purpose).
+    rng = np.random.default_rng(11)
+    T, E, K = 512, 4, 1
+    logits = rng.normal(size=(T, E)) + np.array([1.0, 0.0, 0.0, 0.0])
+    b = np.zeros(E, np.float32)
+    first = None
+    for step in range(200):
+        idx, _, _ = oracle.select(logits, K, bias=b)
+        counts = np.bincount(idx.ravel(), minlength=E).astype(np.int32)
+        if first is None:
+            first = counts.max() - counts.min()
+        b = oracle.bias_update(counts, T * K, b, 0.002, oracle.BIAS_UPDATE_SIGN)
+    assert first > 150 and counts.max() - counts.min() < first / 4
+    assert b[0] < 0 < min(b[1:])
+
+
+# ----------------------------------------- adaptive capacity (Zen MoDE §5.3)
+def test_adaptive_capacity_hand_example():
+    # T=8, K=1, E=4, one batch with loads 4, 2, 1, 1: fbar = .5, .25, .125, .125
+    # C_e = 1 + 2 (fbar - 1/4) = 1.5, 1, .75, .75; cap = ceil(C_e * 8 / 4) = 3, 2, 2, 2
+    caps = oracle.adaptive_capacity(8, 1, [[4, 2, 1, 1]], 1.0, 2.0)
+    assert caps.tolist() == [3, 2, 2, 2]
+
+
+def test_adaptive_capacity_reduces_to_uniform_capacity():
+    # gamma = 0, or a window whose mean load is uniform: every expert gets ceil(C T K / E)
+    hist = np.array([[1100, 990, 1010, 996, 1000, 1024, 1000, 1072]], np.int32)   # sums to 8192
+    assert oracle.adaptive_capacity(4096, 2, hist, 1.25, 0.0).tolist() == [1280] * 8
+    flat = np.array([[1024] * 8, [1024] * 8], np.int32)
+    assert oracle.adaptive_capacity(4096, 2, flat, 1.25, 3.0).tolist() == [1280] * 8
+
+
+def test_adaptive_capacity_window_mean_and_clamps():
+    # two batches that average to a uniform load: the window sees no skew
+    hist = [[4, 2, 1, 1], [0, 2, 3, 3]]
+    assert oracle.adaptive_capacity(8, 1, hist, 1.0, 2.0).tolist() == [2, 2, 2, 2]
+    # everything on expert 0: C = 1 + 5 (1 - 1/4) = 4.75 -> ceil(9.5) = 10 -> clamped to T = 8;
+    # the others: 1 - 5/4 < 0 -> 0
+    assert oracle.adaptive_capacity(8, 1, [[8, 0, 0, 0]], 1.0, 5.0).tolist() == [8, 0, 0, 0]
+
+
+def test_adaptive_capacity_monotone_in_load():
+    rng = np.random.default_rng(5)
+    E = 16
+    hist = rng.multinomial(4096, rng.dirichlet(np.ones(E)), size=3).astype(np.int32)
+    caps = oracle.adaptive_capacity(2048, 2, hist, 1.0, 4.0)
+    load = hist.sum(0)
+    order = np.argsort(load, kind="stable")
+    assert (np.diff(caps[order]) >= 0).all()
+    # under-used experts lose budget, over-used gain it (page: prevents drops under skew)
+    base = oracle.capacity(2048, 2, E, 1.0)
+    assert (caps[load < load.mean()] <= base).all() and (caps[load > load.mean()] >= base).all()
