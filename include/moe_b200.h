@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
 
@@ -84,6 +84,11 @@ typedef enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 } moe_dtype;
 #define MOE_FLAG_EXTENDED_STATS 0x4u /* stats has 2E+7 entries: after the 2E+1 balance
                                         entries, the router z-loss and utilisation
                                         statistics (see moe_route) */
+#define MOE_FLAG_EXPERT_CAPACITY 0x8u /* per-expert capacities from a device array
+                                         (moe_weights_t.expert_capacity, or the
+                                         argument of moe_dispatch_capacity) instead
+                                         of the uniform ceil(C*T*K/E); the row
+                                         bound moe_max_rows becomes T*K */
 
 /* Device status bits (moe_read_device_status). */
 #define MOE_DEV_BAD_EXPERT 0x1     /* an expert index outside [0, E) was skipped */
@@ -116,6 +121,9 @@ typedef struct moe_weights {
     const void* w2;            /* [E, d, F] */
     const void* w13_shared;    /* [N_s, 2F, d], NULL iff n_shared == 0 */
     const void* w2_shared;     /* [N_s, d, F],  NULL iff n_shared == 0 */
+    const int32_t* expert_capacity; /* [E] with MOE_FLAG_EXPERT_CAPACITY (expert e
+                                       keeps at most expert_capacity[e] pairs; a
+                                       negative entry: no limit), else ignored */
 } moe_weights_t;
 
 /* Optional routing outputs of moe_layer_forward (device pointers; each may be
@@ -182,7 +190,10 @@ int moe_read_device_status(const void* ws, moe_stream_t stream, uint32_t* bits);
  *                [2E+4] drop rate sum(counts - kept) / (T*K), kept = min(counts, cap),
  *                [2E+5] number of experts with load below 50% of the mean,
  *                [2E+6] number above 200% of the mean
- *                (Zen MoDE §6.2, table tab:utilization). */
+ *                (Zen MoDE §6.2, table tab:utilization).
+ *                moe_route knows only the uniform capacity: MOE_FLAG_EXTENDED_STATS
+ *                together with MOE_FLAG_EXPERT_CAPACITY is MOE_ERR_INVALID_ARG here
+ *                (moe_layer_forward reports them for the per-expert capacities). */
 int moe_route(const moe_problem_t* p, const void* x, const void* w_gate,
               const float* logit_offset, const float* sel_bias, float* logits,
               int32_t* topk_idx, float* topk_w, float* stats,
@@ -198,7 +209,8 @@ int moe_route(const moe_problem_t* p, const void* x, const void* w_gate,
  *            rank < cap; slot = seg_off[e] + rank; perm entries past
  *            seg_off[E] are left untouched)
  *   x_perm   [moe_max_rows, d] out: x_perm[slot] = x[perm[slot] / K] for
- *            slot < seg_off[E]; later rows untouched.  May be NULL (no gather). */
+ *            slot < seg_off[E]; later rows untouched.  May be NULL (no gather).
+ * With MOE_FLAG_EXPERT_CAPACITY use moe_dispatch_capacity (here: MOE_ERR_INVALID_ARG). */
 int moe_dispatch(const moe_problem_t* p, const int32_t* topk_idx, const void* x,
                  int32_t* counts, int32_t* kept, int32_t* seg_off,
                  int32_t* slot_of, int32_t* perm, void* x_perm,
@@ -253,11 +265,57 @@ int moe_layer_forward(const moe_problem_t* p, const void* x, const moe_weights_t
  * calls whose work overlaps on the GPU race, so serialise them.  The first call
  * on a device looks the array's address up (device current); make it before
  * any stream capture.  Expert indices outside [0, E) are skipped (slot -1) but
- * not reported (there is no status word).  The pages have no counterpart of
+ * not reported (there is no status word).  MOE_FLAG_EXPERT_CAPACITY is not
+ * accepted here (MOE_ERR_INVALID_ARG).  The pages have no counterpart of
  * this entry point. */
 int moe_dispatch_noalloc(const moe_problem_t* p, const int32_t* topk_idx, const void* x,
                          int32_t* counts, int32_t* kept, int32_t* seg_off,
                          int32_t* slot_of, int32_t* perm, void* x_perm, moe_stream_t stream);
+
+/* moe_dispatch with one capacity per expert (Zen MoDE §5.3: capacity_e may
+ * differ per expert).  Requires MOE_FLAG_EXPERT_CAPACITY in p (the workspace
+ * and moe_max_rows are then sized for T*K rows).
+ *   expert_capacity [E] int32 in: expert e keeps the first expert_capacity[e]
+ *            of its pairs in token order (negative: no limit); kept[e] =
+ *            min(counts[e], expert_capacity[e]).
+ * Everything else as moe_dispatch. */
+int moe_dispatch_capacity(const moe_problem_t* p, const int32_t* topk_idx, const int32_t* expert_capacity,
+                          const void* x, int32_t* counts, int32_t* kept, int32_t* seg_off,
+                          int32_t* slot_of, int32_t* perm, void* x_perm,
+                          void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Load-balancing update after a step, from that step's pre-capacity counts
+ * [E] (moe_routing_t.counts).  One kernel, no workspace; either part may be
+ * skipped by passing NULL for its output.
+ *
+ * Selection bias (Zen-Max §2.3 Auxiliary-Loss-Free Load Balancing: after each
+ * step an overloaded expert's bias is lowered and an underloaded one's raised;
+ * the page fixes neither the load measure nor the step).  Load = counts[e],
+ * target = T*K/E, in float64 and rounded once into the float32 bias:
+ *   MOE_BIAS_UPDATE_SIGN:         sel_bias[e] += bias_rate * sign(target - load)
+ *   MOE_BIAS_UPDATE_PROPORTIONAL: sel_bias[e] += bias_rate * (target - load) / target
+ *
+ * Adaptive capacity (Zen MoDE §5.3 Adaptive Capacity Factors,
+ * C_e = C_base + gamma * (fbar_e - 1/N_E)): count_hist is a ring of hist_len
+ * rows of E int32 that this call owns between calls; `step` (0, 1, 2, ...
+ * counted by the caller) selects row step % hist_len, where counts are
+ * stored.  fbar_e = mean of counts[e] / (T*K) over the min(step+1, hist_len)
+ * rows written so far; then
+ *   expert_capacity[e] = clamp(ceil(C_e * T*K / E), 0, T)     (float64)
+ * for the next step's MOE_FLAG_EXPERT_CAPACITY dispatch.  c_base > 0.
+ *
+ * Pointers are device pointers (16-byte aligned); sel_bias and
+ * expert_capacity are updated in place / written.  Errors: MOE_ERR_INVALID_ARG
+ * for NULL counts, both outputs NULL, a non-finite rate / c_base / gamma,
+ * c_base <= 0, hist_len < 1, step < 0, an unknown bias_mode, or
+ * expert_capacity without count_hist. */
+#define MOE_BIAS_UPDATE_SIGN 0
+#define MOE_BIAS_UPDATE_PROPORTIONAL 1
+int moe_balance_update(const moe_problem_t* p, const int32_t* counts,
+                       float* sel_bias, float bias_rate, int32_t bias_mode,
+                       int32_t* count_hist, int32_t hist_len, int64_t step,
+                       float c_base, float gamma, int32_t* expert_capacity,
+                       moe_stream_t stream);
 
 /* Stage boundaries recorded by moe_layer_forward_profiled. */
 #define MOE_EV_START 0   /* before the router */

@@ -15,7 +15,9 @@ MOE_OK = 0
 STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_CUDA",
                 -4: "MOE_ERR_DEVICE_CHECK", -5: "MOE_ERR_WORKSPACE"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
-FLAG_LOGITS_GIVEN, FLAG_BIAS_LOGIT, FLAG_EXTENDED_STATS = 0x1, 0x2, 0x4
+FLAG_LOGITS_GIVEN, FLAG_BIAS_LOGIT, FLAG_EXTENDED_STATS, FLAG_EXPERT_CAPACITY = 0x1, 0x2, 0x4, 0x8
+BIAS_UPDATE_SIGN, BIAS_UPDATE_PROPORTIONAL = 0, 1
+ABI_VERSION = 2
 EXTENDED_STATS = ("z_loss", "entropy_bits", "cv", "drop_rate", "n_below_half", "n_above_double")
 FFN_ROUTED, FFN_SHARED = 0, 1
 DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
@@ -24,7 +26,7 @@ DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
 EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
             "moe_reset_device_status", "moe_read_device_status", "moe_route", "moe_dispatch",
             "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
-            "moe_dispatch_noalloc")
+            "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
 
@@ -39,7 +41,7 @@ class MoeProblem(ctypes.Structure):
 class MoeWeights(ctypes.Structure):
     _fields_ = [("w_gate", ctypes.c_void_p), ("logit_offset", ctypes.c_void_p), ("sel_bias", ctypes.c_void_p),
                 ("w13", ctypes.c_void_p), ("w2", ctypes.c_void_p), ("w13_shared", ctypes.c_void_p),
-                ("w2_shared", ctypes.c_void_p)]
+                ("w2_shared", ctypes.c_void_p), ("expert_capacity", ctypes.c_void_p)]
 
 
 class MoeRouting(ctypes.Structure):
@@ -90,6 +92,14 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_forward_profiled.restype = ctypes.c_int
     L.moe_dispatch_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P]
     L.moe_dispatch_noalloc.restype = ctypes.c_int
+    L.moe_dispatch_capacity.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, sz, P]
+    L.moe_dispatch_capacity.restype = ctypes.c_int
+    L.moe_balance_update.argtypes = [PP, P, P, ctypes.c_float, i32, P, i32, i64, ctypes.c_float, ctypes.c_float,
+                                     P, P]
+    L.moe_balance_update.restype = ctypes.c_int
+    if L.moe_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"{LIB_PATH} has ABI version {L.moe_abi_version()}, this binding expects {ABI_VERSION}: "
+                           "rebuild it")
     _lib = L
     return L
 

@@ -11,14 +11,16 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (DTYPE_BF16, DTYPE_F32, EXTENDED_STATS, FFN_ROUTED, FFN_SHARED, FLAG_BIAS_LOGIT,
-                   FLAG_EXTENDED_STATS, FLAG_LOGITS_GIVEN, MoeError, MoeProblem, MoeRouting, MoeWeights)
+from ._lib import (BIAS_UPDATE_PROPORTIONAL, BIAS_UPDATE_SIGN, DTYPE_BF16, DTYPE_F32, EXTENDED_STATS, FFN_ROUTED,
+                   FFN_SHARED, FLAG_BIAS_LOGIT, FLAG_EXPERT_CAPACITY, FLAG_EXTENDED_STATS, FLAG_LOGITS_GIVEN,
+                   MoeError, MoeProblem, MoeRouting, MoeWeights)
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-           "moe_layer_forward_profiled", "moe_dispatch_noalloc",
+           "moe_layer_forward_profiled", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
-           "FLAG_EXTENDED_STATS", "EXTENDED_STATS", "stats_size",
+           "FLAG_EXTENDED_STATS", "FLAG_EXPERT_CAPACITY", "EXTENDED_STATS", "stats_size",
+           "BIAS_UPDATE_SIGN", "BIAS_UPDATE_PROPORTIONAL",
            "FFN_ROUTED", "FFN_SHARED", "DTYPE_BF16", "DTYPE_F32"]
 
 
@@ -103,6 +105,25 @@ def moe_dispatch_noalloc(prob, topk_idx, x, counts, kept, seg_off, slot_of, perm
     _lib.check("moe_dispatch_noalloc", rc)
 
 
+def moe_dispatch_capacity(prob, topk_idx, expert_capacity, x, counts, kept, seg_off, slot_of, perm, x_perm, ws,
+                          stream=None):
+    rc = _lib.lib().moe_dispatch_capacity(ctypes.byref(prob), _p(topk_idx), _p(expert_capacity), _p(x), _p(counts),
+                                          _p(kept), _p(seg_off), _p(slot_of), _p(perm), _p(x_perm), _p(ws),
+                                          ws.numel(), _stream(stream))
+    _lib.check("moe_dispatch_capacity", rc)
+
+
+def moe_balance_update(prob, counts, sel_bias=None, bias_rate=0.0, bias_mode=BIAS_UPDATE_SIGN, count_hist=None,
+                       step=0, c_base=1.0, gamma=0.0, expert_capacity=None, stream=None):
+    """Selection-bias update and/or adaptive per-expert capacity from one step's
+    counts (see moe_balance_update in the header); count_hist [W, E] int32."""
+    hist_len = 0 if count_hist is None else int(count_hist.shape[0])
+    rc = _lib.lib().moe_balance_update(ctypes.byref(prob), _p(counts), _p(sel_bias), float(bias_rate), int(bias_mode),
+                                       _p(count_hist), hist_len, int(step), float(c_base), float(gamma),
+                                       _p(expert_capacity), _stream(stream))
+    _lib.check("moe_balance_update", rc)
+
+
 def moe_expert_ffn(prob, mode, x_rows, n_rows, seg_off, w13, w2, y_rows, ws, stream=None):
     rc = _lib.lib().moe_expert_ffn(ctypes.byref(prob), int(mode), _p(x_rows), int(n_rows), _p(seg_off), _p(w13),
                                    _p(w2), _p(y_rows), _p(ws), ws.numel(), _stream(stream))
@@ -117,7 +138,7 @@ def moe_combine(prob, y_perm, slot_of, topk_w, y_shared, y, ws, stream=None):
 
 def _weights_struct(w: dict) -> MoeWeights:
     return MoeWeights(_p(w.get("w_gate")), _p(w.get("logit_offset")), _p(w.get("sel_bias")), _p(w["w13"]),
-                      _p(w["w2"]), _p(w.get("w13_shared")), _p(w.get("w2_shared")))
+                      _p(w["w2"]), _p(w.get("w13_shared")), _p(w.get("w2_shared")), _p(w.get("expert_capacity")))
 
 
 def _routing_struct(r: dict | None) -> MoeRouting | None:

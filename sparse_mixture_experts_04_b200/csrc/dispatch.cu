@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
                                                              const unsigned long long* __restrict__ chunk_psum,
                                                              float* __restrict__ stats, int64_t T, int K,
                                                              float alpha, const float* __restrict__ zpart,
-                                                             int n_zpart) {
+                                                             int n_zpart, const int32_t* __restrict__ expert_cap) {
   __shared__ int part[1024];
   __shared__ unsigned long long ppart[1024];
   __shared__ int s_kept[kMaxExperts];
@@ -100,7 +100,9 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
       prun += ppart[tid + i];
     }
     counts[e] = run;
-    const int k = (cap < 0 || run < cap) ? run : static_cast<int>(cap);
+    long long ce = cap;
+    if (expert_cap) ce = expert_cap[e];   // per-expert capacity (Zen MoDE §5.3 capacity_e)
+    const int k = (ce < 0 || run < ce) ? run : static_cast<int>(ce);
     kept[e] = k;
     s_kept[e] = k;
     s_count[e] = run;
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
 cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready,
-                            const unsigned long long* chunk_psum, float* stats, const float* zpart, int n_zpart) {
+                            const unsigned long long* chunk_psum, float* stats, const float* zpart, int n_zpart,
+                            const int32_t* expert_cap) {
   const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
   if (!counts_ready) {
     if (cudaError_t e = launch_k(dispatch_hist_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
@@ -220,7 +223,7 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
   if (cudaError_t e = launch_k(dispatch_scan_kernel, dim3(1), dim3(1024), 0, st,
                                static_cast<const int32_t*>(chunk_counts), n_chunks, p.E, static_cast<long long>(p.cap),
                                chunk_base, counts, kept, seg_off, chunk_psum, chunk_psum ? stats : nullptr, p.T,
-                               p.K, p.alpha, zpart, n_zpart))
+                               p.K, p.alpha, zpart, n_zpart, expert_cap))
     return e;
   return launch_k(dispatch_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
                   static_cast<const int32_t*>(chunk_base), static_cast<const int32_t*>(kept),

@@ -66,6 +66,7 @@ extern "C" int moe_dispatch_noalloc(const moe_problem_t* q, const int32_t* topk_
                                     void* x_perm, moe_stream_t stream) {
   Problem p;
   if (int rc = problem_from_abi(q, &p)) return rc;
+  if (p.flags & MOE_FLAG_EXPERT_CAPACITY) return MOE_ERR_INVALID_ARG;
   if (!topk_idx || !counts || !kept || !seg_off || !slot_of || !perm) return MOE_ERR_INVALID_ARG;
   if (x_perm && (!x || (reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u)))
     return MOE_ERR_INVALID_ARG;

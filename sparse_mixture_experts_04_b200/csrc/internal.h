@@ -68,13 +68,21 @@ cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, co
 // balance statistics from the selection kernel's chunk totals.
 // zpart / n_zpart: per-selection-block sums of logsumexp^2; given with stats,
 // the extended statistics are written too.
+// expert_cap (or nullptr): [E] per-expert capacities (negative: no limit)
+// instead of p.cap.
 cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready = false,
                             const unsigned long long* chunk_psum = nullptr, float* stats = nullptr,
-                            const float* zpart = nullptr, int n_zpart = 0);
+                            const float* zpart = nullptr, int n_zpart = 0, const int32_t* expert_cap = nullptr);
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
                           void* x_perm, cudaStream_t st);
+
+// balance.cu: selection-bias update and adaptive capacity from one step's
+// counts (see moe_balance_update).  bias / caps may be nullptr.
+cudaError_t launch_balance_update(const Problem& p, const int32_t* counts, float* bias, float rate, int mode,
+                                  int32_t* hist, int hist_slot, int hist_rows, float c_base, float gamma,
+                                  int32_t* caps, cudaStream_t st);
 
 // expert_gemm.cu -- returns a moe_status value
 int router_k_splits(const Problem& p);  // slices of the tensor-core gate GEMM's reduction

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "../../include/moe_b200.h"
@@ -88,7 +89,8 @@ static int to_problem(const moe_problem_t* in, Problem* out) {
   if (q.T < 1 || q.d_model < 8 || q.d_ff < 8 || (q.d_model % 8) || (q.d_ff % 8)) return MOE_ERR_INVALID_ARG;
   if (q.n_experts < 1 || q.top_k < 1 || q.top_k > q.n_experts || q.n_shared < 0) return MOE_ERR_INVALID_ARG;
   if (q.dtype != MOE_DTYPE_BF16 && q.dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
-  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT | MOE_FLAG_EXTENDED_STATS)) return MOE_ERR_INVALID_ARG;
+  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT | MOE_FLAG_EXTENDED_STATS | MOE_FLAG_EXPERT_CAPACITY))
+    return MOE_ERR_INVALID_ARG;
   if (!(q.alpha == q.alpha) || !(q.capacity_factor == q.capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (q.n_experts > kMaxExperts || q.top_k > kMaxTopK || q.n_shared > 256) return MOE_ERR_UNSUPPORTED;
   const int64_t lim = static_cast<int64_t>(1) << 31;
@@ -116,7 +118,9 @@ static int to_problem(const moe_problem_t* in, Problem* out) {
     p.cap = p.cap_raw = -1;
   }
   const int64_t TK = q.T * q.top_k;
-  p.max_rows = (p.cap < 0) ? TK : (p.cap * q.n_experts < TK ? p.cap * q.n_experts : TK);
+  // per-expert capacities can give any expert up to T rows: only T*K bounds the total
+  const bool uniform = !(q.flags & MOE_FLAG_EXPERT_CAPACITY);
+  p.max_rows = (p.cap < 0 || !uniform) ? TK : (p.cap * q.n_experts < TK ? p.cap * q.n_experts : TK);
   *out = p;
   return MOE_OK;
 }
@@ -240,6 +244,8 @@ int moe_route(const moe_problem_t* q, const void* x, const void* w_gate, const f
   if (int rc = check_ws(p, ws, ws_bytes)) return rc;
   const bool given = p.flags & MOE_FLAG_LOGITS_GIVEN;
   if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  // the drop figures of the extended statistics need the capacities the dispatch will use
+  if ((p.flags & MOE_FLAG_EXTENDED_STATS) && (p.flags & MOE_FLAG_EXPERT_CAPACITY)) return MOE_ERR_INVALID_ARG;
   if (!given && (!x || !w_gate || !aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
   return route_impl(p, x, w_gate, given ? nullptr : logit_offset, sel_bias, logits, topk_idx, topk_w, stats, ws,
@@ -247,24 +253,64 @@ int moe_route(const moe_problem_t* q, const void* x, const void* w_gate, const f
                     /*stats_in_route=*/true);
 }
 
-int moe_dispatch(const moe_problem_t* q, const int32_t* topk_idx, const void* x, int32_t* counts, int32_t* kept,
-                 int32_t* seg_off, int32_t* slot_of, int32_t* perm, void* x_perm, void* ws, size_t ws_bytes,
-                 moe_stream_t stream) {
+static int dispatch_entry(const moe_problem_t* q, const int32_t* topk_idx, const int32_t* expert_cap,
+                          const void* x, int32_t* counts, int32_t* kept, int32_t* seg_off, int32_t* slot_of,
+                          int32_t* perm, void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
   Problem p;
   if (int rc = to_problem(q, &p)) return rc;
   if (int rc = check_ws(p, ws, ws_bytes)) return rc;
   if (!topk_idx || !counts || !kept || !seg_off || !slot_of || !perm) return MOE_ERR_INVALID_ARG;
   if (x_perm && (!x || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (((p.flags & MOE_FLAG_EXPERT_CAPACITY) != 0) != (expert_cap != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (expert_cap && !aligned16(expert_cap)) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaError_t e = launch_dispatch(p, topk_idx, counts, kept, seg_off, slot_of, perm,
                                       at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.chunk_base),
-                                      at<unsigned>(ws, L.status), st))
+                                      at<unsigned>(ws, L.status), st, false, nullptr, nullptr, nullptr, 0,
+                                      expert_cap))
     return cuda_rc(e);
   if (x_perm) {
     if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
   }
   return MOE_OK;
+}
+
+int moe_dispatch(const moe_problem_t* q, const int32_t* topk_idx, const void* x, int32_t* counts, int32_t* kept,
+                 int32_t* seg_off, int32_t* slot_of, int32_t* perm, void* x_perm, void* ws, size_t ws_bytes,
+                 moe_stream_t stream) {
+  return dispatch_entry(q, topk_idx, nullptr, x, counts, kept, seg_off, slot_of, perm, x_perm, ws, ws_bytes, stream);
+}
+
+int moe_dispatch_capacity(const moe_problem_t* q, const int32_t* topk_idx, const int32_t* expert_capacity,
+                          const void* x, int32_t* counts, int32_t* kept, int32_t* seg_off, int32_t* slot_of,
+                          int32_t* perm, void* x_perm, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!expert_capacity) return MOE_ERR_INVALID_ARG;
+  return dispatch_entry(q, topk_idx, expert_capacity, x, counts, kept, seg_off, slot_of, perm, x_perm, ws, ws_bytes,
+                        stream);
+}
+
+int moe_balance_update(const moe_problem_t* q, const int32_t* counts, float* sel_bias, float bias_rate,
+                       int32_t bias_mode, int32_t* count_hist, int32_t hist_len, int64_t step, float c_base,
+                       float gamma, int32_t* expert_capacity, moe_stream_t stream) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (!counts || !aligned16(counts) || (!sel_bias && !expert_capacity)) return MOE_ERR_INVALID_ARG;
+  if (sel_bias) {
+    if (!aligned16(sel_bias) || !std::isfinite(bias_rate)) return MOE_ERR_INVALID_ARG;
+    if (bias_mode != MOE_BIAS_UPDATE_SIGN && bias_mode != MOE_BIAS_UPDATE_PROPORTIONAL) return MOE_ERR_INVALID_ARG;
+  }
+  int slot = 0, rows = 0;
+  if (expert_capacity) {
+    if (!aligned16(expert_capacity) || !count_hist || !aligned16(count_hist)) return MOE_ERR_INVALID_ARG;
+    if (hist_len < 1 || step < 0 || !std::isfinite(c_base) || !(c_base > 0.0f) || !std::isfinite(gamma))
+      return MOE_ERR_INVALID_ARG;
+    slot = static_cast<int>(step % hist_len);
+    rows = step + 1 < hist_len ? static_cast<int>(step + 1) : hist_len;
+  }
+  return cuda_rc(launch_balance_update(p, counts, sel_bias, bias_rate, bias_mode, expert_capacity ? count_hist : nullptr,
+                                       slot, rows, c_base, gamma, expert_capacity,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int moe_expert_ffn(const moe_problem_t* q, int32_t mode, const void* x_rows, int64_t n_rows,
@@ -311,6 +357,8 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   if (p.Ns > 0 && (!w->w13_shared || !w->w2_shared || !aligned16(w->w13_shared) || !aligned16(w->w2_shared)))
     return MOE_ERR_INVALID_ARG;
   if (p.Ns == 0 && (w->w13_shared || w->w2_shared)) return MOE_ERR_INVALID_ARG;
+  const int32_t* expert_cap = (p.flags & MOE_FLAG_EXPERT_CAPACITY) ? w->expert_capacity : nullptr;
+  if ((p.flags & MOE_FLAG_EXPERT_CAPACITY) && (!expert_cap || !aligned16(expert_cap))) return MOE_ERR_INVALID_ARG;
 
   p.skewed_load = (!given && w->logit_offset) || w->sel_bias;
   const WsLayout L = make_layout(p);
@@ -348,7 +396,7 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
                                       at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true,
                                       at<unsigned long long>(ws, L.chunk_psum), stats,
                                       (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr,
-                                      L.n_sel_blocks))
+                                      L.n_sel_blocks, expert_cap))
     return cuda_rc(e);
   kernels += 2;
   if (p.max_rows > 0) {

@@ -26,6 +26,13 @@ class MoeLayer:
                 counts=torch.empty(E, **i32), kept=torch.empty(E, **i32), seg_off=torch.empty(E + 1, **i32),
                 slot_of=torch.empty((T, K), **i32), perm=torch.empty(max(api.max_rows(prob), 1), **i32))
         self.stats = torch.empty(api.stats_size(prob), dtype=torch.float32, device=self.device)
+        if prob.flags & api.FLAG_EXPERT_CAPACITY and weights.get("expert_capacity") is None:
+            # start from the uniform capacity (no limit: -1)
+            cap = api.capacity(prob)
+            cap = -1 if cap < 0 else min(cap, T)
+            weights["expert_capacity"] = torch.full((E,), cap, dtype=torch.int32, device=self.device)
+        self._balance_step = 0
+        self._count_hist = None
 
     @classmethod
     def from_inputs(cls, inputs: dict, device="cuda", flags: int = 0, keep_routing: bool = True) -> "MoeLayer":
@@ -55,6 +62,31 @@ class MoeLayer:
         return y
 
     __call__ = forward
+
+    def balance_update(self, bias_rate: float = 0.0, bias_mode: int = api.BIAS_UPDATE_SIGN, c_base: float | None = None,
+                       gamma: float = 0.0, window: int = 8, stream=None) -> None:
+        """Between steps: move the selection bias against the last forward's
+        load (when the layer has one and bias_rate != 0) and, for a layer built
+        with FLAG_EXPERT_CAPACITY, set the next forward's per-expert capacities
+        from the last `window` forwards' loads (c_base defaults to the
+        problem's capacity factor).  One kernel on the stream."""
+        if self.routing is None:
+            raise ValueError("balance_update needs the routing outputs (keep_routing=True)")
+        bias = self.weights.get("sel_bias") if bias_rate != 0.0 else None
+        caps = self.weights.get("expert_capacity") if self.prob.flags & api.FLAG_EXPERT_CAPACITY else None
+        if bias is None and caps is None:
+            return
+        hist = None
+        if caps is not None:
+            if self._count_hist is None or self._count_hist.shape[0] != window:
+                self._count_hist = torch.zeros((window, self.prob.n_experts), dtype=torch.int32, device=self.device)
+                self._balance_step = 0
+            hist = self._count_hist
+        cb = self.prob.capacity_factor if c_base is None else c_base
+        api.moe_balance_update(self.prob, self.routing["counts"], bias, bias_rate, bias_mode, hist,
+                               self._balance_step, cb, gamma, caps, stream)
+        if caps is not None:
+            self._balance_step += 1
 
     def forward_host(self, xs_host, ys_host, stats_host=None, stream=None):
         """Run one layer forward per host batch: xs_host[i] [T, d] -> ys_host[i].

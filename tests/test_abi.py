@@ -29,7 +29,7 @@ def declared_functions():
     return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\**\s+\**(moe_\w+)\s*\(", src, flags=re.M)))
 
 
-def test_header_declares_the_north_star_entry_points():
+def test_header_declares_the_layer_entry_points():
     names = declared_functions()
     for n in ("moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward"):
         assert n in names
@@ -39,7 +39,7 @@ def test_header_declares_the_north_star_entry_points():
 def test_library_exports_every_declared_symbol(L):
     for n in declared_functions():
         assert hasattr(L, n), n
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == _lib.ABI_VERSION == 2
 
 
 def test_status_strings(L):
@@ -72,7 +72,7 @@ def _ret(fn, *args):
 
 @pytest.mark.parametrize("field,value,code", [
     ("T", 0, -1), ("d_model", 12, -1), ("d_ff", 4, -1), ("n_experts", 0, -1), ("top_k", 0, -1),
-    ("top_k", 9, -1), ("n_shared", -1, -1), ("dtype", 7, -1), ("flags", 0x10, -1),
+    ("top_k", 9, -1), ("n_shared", -1, -1), ("dtype", 7, -1), ("flags", 0x10, -1), ("flags", 0x20, -1),
     ("n_experts", 300, -2), ("top_k", 33, -2)])
 def test_invalid_problems_are_rejected(L, field, value, code):
     prob = api.make_problem(64, 64, 8, 2, 128)
@@ -94,8 +94,10 @@ def test_entry_points_reject_bad_workspace_before_launching(L):
     assert L.moe_dispatch(P, fake, fake, fake, fake, fake, fake, fake, None, None, 0, None) == -5
     assert L.moe_expert_ffn(P, 0, fake, 8, fake, fake, fake, fake, None, 0, None) == -5
     assert L.moe_combine(P, fake, fake, fake, None, fake, None, 0, None) == -5
-    w = _lib.MoeWeights(fake, None, None, fake, fake, None, None)
+    w = _lib.MoeWeights(fake, None, None, fake, fake, None, None, None)
     assert L.moe_layer_forward(P, fake, ctypes.byref(w), fake, None, None, None, 0, None) == -5
+    prob.flags = api.FLAG_EXPERT_CAPACITY
+    assert L.moe_dispatch_capacity(P, fake, fake, fake, fake, fake, fake, fake, fake, None, None, 0, None) == -5
 
 
 def test_entry_points_reject_bad_arguments_before_launching(L):
@@ -119,11 +121,11 @@ def test_entry_points_reject_bad_arguments_before_launching(L):
     assert L.moe_combine(P, fake, fake, fake, fake, fake, ws, big, None) == -1
     # layer: logits-given mode needs routing.logits
     prob.flags = api.FLAG_LOGITS_GIVEN
-    w = _lib.MoeWeights(None, None, None, fake, fake, None, None)
+    w = _lib.MoeWeights(None, None, None, fake, fake, None, None, None)
     assert L.moe_layer_forward(P, fake, ctypes.byref(w), fake, None, None, ws, big, None) == -1
     # layer: shared weights given although n_shared == 0
     prob.flags = 0
-    w = _lib.MoeWeights(fake, None, None, fake, fake, fake, fake)
+    w = _lib.MoeWeights(fake, None, None, fake, fake, fake, fake, None)
     assert L.moe_layer_forward(P, fake, ctypes.byref(w), fake, None, None, ws, big, None) == -1
 
 
@@ -132,3 +134,52 @@ def test_python_binding_raises_on_error(L):
     prob.top_k = 0
     with pytest.raises(api.MoeError):
         api.workspace_size(prob)
+
+
+def test_expert_capacity_flag_sizes_for_all_pairs_and_checks_its_array(L):
+    prob = api.make_problem(64, 64, 8, 2, 128, capacity_factor=0.5, flags=api.FLAG_EXPERT_CAPACITY)
+    P = ctypes.byref(prob)
+    assert api.capacity(prob) == 8          # the uniform capacity is still reported
+    assert api.max_rows(prob) == 64 * 2     # but any expert may be given up to T rows
+    n = ctypes.c_size_t(0)
+    assert L.moe_workspace_size(P, ctypes.byref(n)) == 0
+    ws, big, fake = 1 << 20, n.value, 4096
+    # moe_dispatch has no capacity array: the flag needs moe_dispatch_capacity
+    assert L.moe_dispatch(P, fake, fake, fake, fake, fake, fake, fake, None, ws, big, None) == -1
+    assert L.moe_dispatch_capacity(P, fake, None, fake, fake, fake, fake, fake, fake, None, ws, big, None) == -1
+    assert L.moe_dispatch_capacity(P, fake, fake + 4, fake, fake, fake, fake, fake, fake, None, ws, big, None) == -1
+    # the layer reads the array from the weights
+    w = _lib.MoeWeights(fake, None, None, fake, fake, None, None, None)
+    assert L.moe_layer_forward(P, fake, ctypes.byref(w), fake, None, None, ws, big, None) == -1
+    # moe_route cannot report drop figures for capacities it does not know
+    prob.flags |= api.FLAG_EXTENDED_STATS
+    assert L.moe_route(P, fake, fake, None, None, fake, fake, fake, fake, ws, big, None) == -1
+    # moe_dispatch_capacity without the flag, and the no-workspace dispatch with it
+    prob.flags = 0
+    assert L.moe_dispatch_capacity(P, fake, fake, fake, fake, fake, fake, fake, fake, None, ws, big, None) == -1
+    prob.flags = api.FLAG_EXPERT_CAPACITY
+    assert L.moe_dispatch_noalloc(P, fake, fake, fake, fake, fake, fake, fake, None, None) == -1
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(counts=None), "no counts"),
+    (dict(sel_bias=None, expert_capacity=None), "nothing to update"),
+    (dict(bias_rate=float("nan")), "non-finite rate"),
+    (dict(bias_mode=2), "unknown mode"),
+    (dict(count_hist=None), "capacity without history"),
+    (dict(hist_len=0), "empty history"),
+    (dict(step=-1), "negative step"),
+    (dict(c_base=0.0), "no base capacity"),
+    (dict(gamma=float("inf")), "non-finite gamma"),
+    (dict(sel_bias=4096 + 8), "misaligned bias"),
+])
+def test_balance_update_rejects_bad_arguments(L, kw, why):
+    prob = api.make_problem(64, 64, 8, 2, 128, capacity_factor=1.0)
+    fake = 4096
+    a = dict(counts=fake, sel_bias=fake, bias_rate=0.01, bias_mode=0, count_hist=fake, hist_len=4, step=0,
+             c_base=1.0, gamma=0.5, expert_capacity=fake)
+    a.update(kw)
+    rc = L.moe_balance_update(ctypes.byref(prob), a["counts"], a["sel_bias"], a["bias_rate"], a["bias_mode"],
+                              a["count_hist"], a["hist_len"], a["step"], a["c_base"], a["gamma"],
+                              a["expert_capacity"], None)
+    assert rc == -1, why
