@@ -66,6 +66,9 @@ struct GemmArgs {
   // which rows of each group this launch covers: 0 all, 1 the head (rows
   // rounded down to a multiple of 256), 2 the tail (the rest)
   int row_mode;
+  // pair kernel: a group's last row tile with at most swap_max rows (0: never)
+  // is computed operand-swapped (see grouped_gemm_pair_kernel)
+  int swap_max;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -98,6 +101,7 @@ constexpr int gemm_smem_bytes() {
 
 struct TileInfo {
   int g, row0, row_end, n0;
+  bool swap;  // operand-swapped remainder tile (pair kernel only)
 };
 
 // Rows [base, base + return) of group g (the part row_mode selects), clamped
@@ -137,6 +141,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   ti.row0 = base + m_idx * BM;
   ti.row_end = base + rows;
   ti.n0 = n_idx * out_cols;
+  ti.swap = m_idx == mt - 1 && rows - m_idx * BM <= a.swap_max;
   return ti;
 }
 
@@ -440,13 +445,90 @@ constexpr int kPairABytes = 128 * kBK * 2;
 constexpr int kPairBBytes = 128 * kBK * 2;  // this CTA's half of B
 constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
 
+// Swap-tile epilogues transpose through shared memory, 32 tokens at a time:
+// xbuf[token][TMEM lane] (row stride 132 floats keeps 16-byte alignment).
+constexpr int kSwapXStride = 132;
+constexpr int kSwapXBytes = 32 * kSwapXStride * 4;
+// A swap tile with at most this many tokens per CTA loads them with a 64-row box.
+constexpr int kSwapSmallRows = 64;
+
 constexpr int pair_smem_bytes() {
-  return kPairStages * kPairStageBytes + 256 + 4 * (kMaxGroups + 1) + 1024;
+  return kPairStages * kPairStageBytes + 256 + 4 * (kMaxGroups + 1) + kSwapXBytes + 1024;
+}
+
+// MMA N of a swap tile covering `rows` (1..256) token rows: a multiple of 16.
+__device__ __forceinline__ int swap_n(int rows) { return (rows + 15) & ~15; }
+
+// Epilogue of a swap tile (all four epilogue warps, uniform control flow):
+// TMEM lane = weight row of this CTA, column = token of the tile.  Each
+// 32-token chunk goes through xbuf so that every thread then stores 8
+// consecutive outputs of one token (16 bytes).
+//   SwiGLU: lanes 0..63 hold gate features n0 + 64*rank + (0..63), lanes
+//   64..127 the same up features: h = silu(g) * u.
+//   BF16: lane = output column n0 + 128*rank + lane.
+template <int EPI>
+__device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileInfo& ti, uint32_t rank, int quarter,
+                                              int lane, int et, uint32_t t_lane, float* xbuf) {
+  const int rows = ti.row_end - ti.row0;
+  const int n = swap_n(rows);
+  const int my_lane = quarter * 32 + lane;
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(ti.row0) * args.ldo +
+                       static_cast<int64_t>(ti.g) * args.out_col_stride;
+#pragma unroll 1
+  for (int c = 0; c < n; c += 32) {
+    uint32_t v[32];
+    tmem_load_32x32(t_lane + c, v);
+    tmem_load_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) xbuf[j * kSwapXStride + my_lane] = __uint_as_float(v[j]);
+    named_bar_sync(1, 128);
+    if (EPI == EPI_SWIGLU) {
+      // 64 features = 8 groups of 8: 16 tokens per pass
+      const int fg = et & 7;
+      const int f = ti.n0 + 64 * static_cast<int>(rank) + 8 * fg;
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const int j = pass * 16 + (et >> 3);
+        if (c + j < rows && f < args.N) {
+          const float4* gp = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 8 * fg);
+          const float4* up = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 64 + 8 * fg);
+          const float4 g0 = gp[0], g1 = gp[1], u0 = up[0], u1 = up[1];
+          const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          uint32_t pk[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float h0 = g[2 * q] / (1.0f + __expf(-g[2 * q])) * u[2 * q];
+            const float h1 = g[2 * q + 1] / (1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
+            pk[q] = pack_bf16x2(h0, h1);
+          }
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c + j) * args.ldo + f) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+    } else {
+      // 128 columns = 16 groups of 8: 8 tokens per pass
+      const int fg = et & 15;
+      const int col = ti.n0 + 128 * static_cast<int>(rank) + 8 * fg;
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int j = pass * 8 + (et >> 4);
+        if (c + j < rows && col < args.N) {
+          const float4* vp = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 8 * fg);
+          const float4 a = vp[0], b = vp[1];
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c + j) * args.ldo + col) =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+        }
+      }
+    }
+    named_bar_sync(1, 128);
+  }
 }
 
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             const __grid_constant__ CUtensorMap tmA64, const __grid_constant__ CUtensorMap tmB64,
                              const GemmArgs args) {
   constexpr int kOutCols = (EPI == EPI_SWIGLU) ? kPairBN / 2 : kPairBN;
   extern __shared__ uint8_t smem_raw[];
@@ -461,6 +543,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
+  float* xbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(prefix + kMaxGroups + 1) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -485,6 +568,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmA64);
+    if (EPI == EPI_SWIGLU) prefetch_tensormap(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -518,11 +603,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const int kg = kb / nkb_g;
           const int kk = (kb - kg * nkb_g) * kBK;
           const uint32_t bar = full_leader + static_cast<uint32_t>(stage * 8);
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kPairStageBytes);
-          tma_load_2d_pair(sA + stage * kPairABytes, &tmA, bar, kg * args.K + kk,
-                           ti.row0 + 128 * static_cast<int>(rank));
+          // a swap tile's N token rows are split N/2 per CTA; the box (64 or
+          // 128 rows) may load more, the MMA reads the first N/2
+          const int half_n = ti.swap ? swap_n(ti.row_end - ti.row0) / 2 : 128;
+          const bool small = half_n <= kSwapSmallRows;
+          if (rank == 0)
+            mbar_arrive_expect_tx(&full[stage], 2 * (kPairBBytes + (small ? kSwapSmallRows * kBK * 2 : kPairABytes)));
+          const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
+          tma_load_2d_pair(sA + stage * kPairABytes, small ? &tmA64 : &tmA, bar, kg * args.K + kk, a_row);
           uint8_t* b_dst = sB + stage * kPairBBytes;
-          if (EPI == EPI_SWIGLU)
+          if (EPI == EPI_SWIGLU && ti.swap) {
+            // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
+            const int f = ti.n0 + 64 * static_cast<int>(rank);
+            tma_load_3d_pair(b_dst, &tmB64, bar, kk, f, 2 * ti.g);
+            tma_load_3d_pair(b_dst + kPairBBytes / 2, &tmB64, bar, kk, f, 2 * ti.g + 1);
+          } else if (EPI == EPI_SWIGLU)
             tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
           else
             tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank),
@@ -550,12 +645,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kPairBM, kPairBN);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
+        const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
+        // normal tile: A = token rows (M = 256), B = weight rows (N = 256);
+        // swap tile: A = weight rows (M = 256), B = the tile's N token rows
+        const uint32_t idesc = idesc_bf16_f32(kPairBM, ti.swap ? swap_n(ti.row_end - ti.row0) : kPairBN);
         const int acc = it & 1;
         const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
@@ -570,8 +668,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after_sync();
-          const uint64_t adesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes));
-          const uint64_t bdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes));
+          const uint64_t tdesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes));
+          const uint64_t wdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes));
+          const uint64_t adesc = ti.swap ? wdesc : tdesc;
+          const uint64_t bdesc = ti.swap ? tdesc : wdesc;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k)
             umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
@@ -600,13 +700,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
       const int acc = it & 1;
       const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
-      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_par, abort_flag));
+      // all four epilogue warps take the same decision (a swap tile's
+      // epilogue synchronises them), even when a wait gives up
+      const bool ready = named_bar_and(2, 128, mbar_wait(&tfull[acc], acc_par, abort_flag));
       if (!ready) break;
       tc_fence_after_sync();
-      const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kPairBN);
-      epilogue_rows<EPI, kPairBN>(args, ti.g, row, row < ti.row_end, ti.n0, t_row);
+      if (ti.swap) {
+        epilogue_swap<EPI>(args, ti, rank, quarter, lane, (warp - 2) * 32 + lane, t_row, xbuf);
+      } else {
+        const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
+        epilogue_rows<EPI, kPairBN>(args, ti.g, row, row < ti.row_end, ti.n0, t_row);
+      }
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(acc * 8));
@@ -689,8 +795,8 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
 }
 
 template <int EPI>
-static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int64_t tile_bound,
-                         cudaStream_t st) {
+static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64, const CUtensorMap& tb64,
+                         const GemmArgs& a, int64_t tile_bound, cudaStream_t st) {
   constexpr int smem = pair_smem_bytes();
   static std::mutex mu;
   static int max_pairs[64] = {0};
@@ -720,7 +826,7 @@ static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   if (tile_bound <= 0) return 0;
   if (pairs > tile_bound) pairs = static_cast<int>(tile_bound);
   return launch_k(grouped_gemm_pair_kernel<EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads), smem,
-                  st, ta, tb, a) == cudaSuccess ? 0 : -3;
+                  st, ta, tb, ta64, tb64, a) == cudaSuccess ? 0 : -3;
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -731,21 +837,35 @@ static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 //              tiles on CTA pairs, the rest (under 256 rows) as 128-row tiles
 //              on single CTAs (second launch): padding as with 128-row tiles
 //   pair       every group on 256-row pair tiles (padding up to 255 rows)
-// Measured choice: routed groups use the pure pair shape when they are large
-// (>= 768 expected rows) and the load is not skewed by a logit offset or a
-// selection bias, single CTAs otherwise; shared experts (every token, so the
-// rows are known) use pair+tail from 512 rows.
+// Measured choice: the pair shape, with operand-swapped remainder tiles, for
+// groups of at least 256 expected rows (routed: T*K/E capped by the capacity;
+// shared: every row), single CTAs below (decode-sized groups, where the
+// weights' HBM stream bounds both shapes).
 // MOE_B200_GEMM_TILE=128|256|256all forces single, pair+tail or pair (all
 // complete implementations; the tests run each).
 enum TileMode { kTileSingle = 0, kTilePairTail = 1, kTilePair = 2 };
 
-static int tile_mode(int64_t expected_rows_per_group, bool routed, bool skewed) {
+// Largest last row tile of a group that the pair kernel computes operand-
+// swapped (weights as the 256-row M operand, the tile's tokens as N): its MMAs
+// cost in proportion to the rows it has, not to 256.  MOE_B200_SWAP_MAX
+// (0..255) overrides; 0 turns swap tiles off.  Measured: with at most 128
+// rows a swap tile is clearly cheaper than a 256-row tile; near 256 rows it
+// is not (the transposing epilogue costs more than the padding saves).
+static int swap_max_rows() {
+  const char* e = getenv("MOE_B200_SWAP_MAX");
+  if (e && *e) {
+    const int v = atoi(e);
+    return v < 0 ? 0 : v > 255 ? 255 : v;
+  }
+  return 128;
+}
+
+static int tile_mode(int64_t expected_rows_per_group) {
   const char* e = getenv("MOE_B200_GEMM_TILE");
   if (e && !strcmp(e, "128")) return kTileSingle;
   if (e && !strcmp(e, "256")) return kTilePairTail;
   if (e && !strcmp(e, "256all")) return kTilePair;
-  if (!routed) return expected_rows_per_group >= 512 ? kTilePairTail : kTileSingle;
-  return (expected_rows_per_group >= 768 && !skewed) ? kTilePair : kTileSingle;
+  return expected_rows_per_group >= 256 ? kTilePair : kTileSingle;
 }
 
 int router_k_splits(const Problem& p) {
@@ -913,11 +1033,10 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
   const bool routed = mode == 0;
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
-  // routed loads are uneven (a skewed router leaves most experts far below the
-  // mean), so routed groups need a larger expected size than shared ones
+  // expected rows per group: routed T*K/E (at most the capacity), shared all rows
   int64_t expected = routed ? (p.T * p.K) / p.E : n_rows;
   if (routed && p.cap >= 0 && p.cap < expected) expected = p.cap;
-  const int mode_t = tile_mode(expected, routed, p.skewed_load);
+  const int mode_t = tile_mode(expected);
   const bool pair = mode_t != kTileSingle;
   const bool tail = mode_t == kTilePairTail;
   if (n_kernels) *n_kernels += tail ? 4 : 2;
@@ -929,7 +1048,11 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.F), static_cast<uint64_t>(2 * G)};
     const uint32_t bb[3] = {kBK, 128, 1};
+    const uint32_t bb64[3] = {kBK, 64, 1};  // swap tiles: 64 gate and 64 up rows per CTA
+    const uint32_t ba64[2] = {kBK, 64};     // swap tiles: up to 64 token rows per CTA
+    CUtensorMap ta64, tb64;
     if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
+    if (pair && (!make_map(&ta64, x_rows, 2, da, ba64) || !make_map(&tb64, w13, 3, db, bb64))) return -3;
     GemmArgs a{};
     a.n_groups = G;
     a.seg_off = routed ? seg_off : nullptr;
@@ -941,13 +1064,15 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.ldo = h_cols;
     a.out_col_stride = routed ? 0 : p.F;
     a.status = status;
+    a.swap_max = swap_max_rows();
     const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
     if (pair) {
       a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
-      int rc = run_pair_gemm<EPI_SWIGLU>(ta, tb, a, (mt / 2 + G) * cdiv(p.F, 128), st);
+      int rc = run_pair_gemm<EPI_SWIGLU>(ta, tb, ta64, tb64, a, (mt / 2 + G) * cdiv(p.F, 128), st);
       if (rc) return rc;
       if (tail) {
         a.row_mode = 2;  // the rest (under 256 rows per group) on single CTAs
+        a.swap_max = 0;
         rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, 2 * G * cdiv(p.F, 128), st);
         if (rc) return rc;
       }
@@ -964,9 +1089,10 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
     const uint32_t bb[3] = {kBK, 256, 1};
     const uint32_t bb_half[3] = {kBK, 128, 1};  // a pair CTA stages half of the 256 B rows
-    CUtensorMap tb_half;
+    const uint32_t ba64[2] = {kBK, 64};
+    CUtensorMap tb_half, ta64;
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
-    if (pair && !make_map(&tb_half, w2, 3, db, bb_half)) return -3;
+    if (pair && (!make_map(&tb_half, w2, 3, db, bb_half) || !make_map(&ta64, h, 2, da, ba64))) return -3;
     GemmArgs a{};
     a.n_groups = routed ? G : 1;
     a.seg_off = routed ? seg_off : nullptr;
@@ -978,13 +1104,15 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.ldo = p.d;
     a.out_col_stride = 0;
     a.status = status;
+    a.swap_max = swap_max_rows();
     const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
     if (pair) {
       a.row_mode = tail ? 1 : 0;
-      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, a, (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
+      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, ta64, tb_half, a, (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
       if (rc) return rc;
       if (tail) {
         a.row_mode = 2;
+        a.swap_max = 0;
         rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.d, 256), st);
         if (rc) return rc;
       }

@@ -26,7 +26,6 @@ struct Problem {
   int dtype;
   uint32_t flags;
   float alpha;
-  bool skewed_load;  // the router has a logit offset or selection bias: expect uneven expert loads
   size_t esize() const { return dtype == kBF16 ? 2 : 4; }
 };
 

@@ -360,7 +360,6 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   const int32_t* expert_cap = (p.flags & MOE_FLAG_EXPERT_CAPACITY) ? w->expert_capacity : nullptr;
   if ((p.flags & MOE_FLAG_EXPERT_CAPACITY) && (!expert_cap || !aligned16(expert_cap))) return MOE_ERR_INVALID_ARG;
 
-  p.skewed_load = (!given && w->logit_offset) || w->sel_bias;
   const WsLayout L = make_layout(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   auto mark = [&](int i) -> cudaError_t {

@@ -217,6 +217,39 @@ def test_routed_expert_ffn_matches_oracle(name):
     assert rel_err(got[rows], want) <= tol(cfg)
 
 
+@pytest.mark.parametrize("tile,swap", [("256all", ""), ("256all", "0"), ("256all", "100"), ("128", "")])
+def test_routed_ffn_every_remainder_shape(tile, swap, monkeypatch):
+    """Groups whose last 256-row tile holds 1..256 rows (every swap-tile MMA
+    width class, ragged F across two column tiles), every row against the
+    oracle's SwiGLU of its expert."""
+    monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
+    monkeypatch.setenv("MOE_B200_SWAP_MAX", swap)
+    sizes = [1, 15, 16, 17, 31, 33, 100, 128, 129, 200, 255, 256, 257, 300, 513, 0, 48]
+    E, d, F = len(sizes), 256, 200
+    T = sum(sizes)
+    prob = api.make_problem(T, d, E, 1, F, 0, 0.0, "bf16")
+    ws = api.alloc_workspace(prob)
+    R = api.max_rows(prob)
+    g = torch.Generator().manual_seed(21)
+    x_rows = torch.randn((R, d), generator=g).to(torch.bfloat16)
+    w13 = (torch.randn((E, 2 * F, d), generator=g) / d ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn((E, d, F), generator=g) / F ** 0.5).to(torch.bfloat16)
+    seg_off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    y_rows = torch.zeros((R, d), dtype=torch.bfloat16, device="cuda")
+    api.reset_device_status(ws)
+    api.moe_expert_ffn(prob, api.FFN_ROUTED, dev(x_rows), R, dev(seg_off), dev(w13), dev(w2), y_rows, ws)
+    assert api.read_device_status(ws) == 0
+    got = y_rows.float().cpu().numpy()
+    xs, a, b = host_np(x_rows), host_np(w13), host_np(w2)
+    e_of = np.repeat(np.arange(E), sizes)
+    want = np.stack([oracle.swiglu(_row64(xs, r, torch.bfloat16), a[e_of[r]], b[e_of[r]]) for r in range(T)])
+    assert rel_err(got[:T], want) <= 2e-2
+    for e in range(E):   # per group too, so a small group is not hidden by a large one
+        lo, hi = seg_off[e], seg_off[e + 1]
+        if hi > lo:
+            assert rel_err(got[lo:hi], want[lo:hi]) <= 2e-2, (e, sizes[e])
+
+
 def _row64(xs, t, dtype):
     if dtype == torch.bfloat16:
         return (xs[t].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
@@ -337,12 +370,14 @@ def test_layer_stats_match_oracle_and_uniform_routing_gives_alpha():
 
 
 # --------------------------------------------------- both GEMM tile shapes
-@pytest.mark.parametrize("tile", ["128", "256", "256all"])
+@pytest.mark.parametrize("tile,swap", [("128", ""), ("256", ""), ("256all", "0"), ("256all", "64"), ("256all", "")])
 @pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "ragged_bf16", "mini_skewed", "mini_decode"])
-def test_layer_forward_both_tile_shapes(name, tile, monkeypatch):
+def test_layer_forward_both_tile_shapes(name, tile, swap, monkeypatch):
     """The 128-row single-CTA and 256-row CTA-pair expert GEMMs, each forced,
-    against the oracle (the library picks one per problem size otherwise)."""
+    the pair kernel with and without operand-swapped remainder tiles, against
+    the oracle (the library picks one per problem size otherwise)."""
     monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
+    monkeypatch.setenv("MOE_B200_SWAP_MAX", swap)
     cfg = SMALL[name]
     inp = inputs(name)
     logits32 = given_logits(cfg)
