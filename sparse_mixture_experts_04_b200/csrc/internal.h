@@ -51,7 +51,9 @@ cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void*
 // chunk_counts / chunk_psum: zeroed [n_chunks, E] arrays that receive, per
 // dispatch chunk, the histogram of the chosen experts and the sum of p in
 // fixed point (p_fixed_scale; integer atomics: exact and order-independent)
-// zpart (or nullptr): [n_selection_blocks] sums of logsumexp^2 (router z-loss)
+// zpart (or nullptr): [route_select_zparts(p)] partial sums of logsumexp^2
+// (router z-loss), at most n_sel_blocks of them
+int route_select_zparts(const Problem& p);
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
                                 const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
                                 unsigned long long* chunk_psum, float* zpart, cudaStream_t st);

@@ -143,25 +143,13 @@ static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_C
 // Router body shared by moe_route and moe_layer_forward.
 // chunk_totals_cleared: the caller already zeroed the chunk totals;
 // stats_in_route: finalise the statistics here (else the dispatch scan does).
+// *n_zpart: number of z-loss partials written (for the statistics);
+// *n_kernels (if given) += kernels enqueued.
 static int route_impl(const Problem& p, const void* x, const void* w_gate, const float* offset,
                       const float* sel_bias, float* logits, int32_t* idx, float* w, float* stats, void* ws,
-                      const WsLayout& L, cudaStream_t st, bool chunk_totals_cleared, bool stats_in_route) {
+                      const WsLayout& L, cudaStream_t st, bool chunk_totals_cleared, bool stats_in_route,
+                      int* n_zpart, int* n_kernels) {
   unsigned* status = at<unsigned>(ws, L.status);
-  int n_parts = 0;
-  float* parts = nullptr;
-  if (!(p.flags & MOE_FLAG_LOGITS_GIVEN)) {
-    if (p.dtype == kBF16) {
-      const int splits = router_k_splits(p);
-      if (splits > 1) {
-        parts = at<float>(ws, L.logit_parts);
-        n_parts = splits;
-      }
-      const int rc = launch_gate_logits_tc(p, x, w_gate, offset, splits > 1 ? parts : logits, splits, status, st);
-      if (rc) return MOE_ERR_CUDA;
-    } else {
-      if (cudaError_t e = launch_gate_logits_simt(p, x, w_gate, offset, logits, st)) return cuda_rc(e);
-    }
-  }
   // the chunk totals start at zero: the layer forward clears them with the
   // status word; a standalone call clears them here
   if (!chunk_totals_cleared) {
@@ -171,13 +159,36 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
   int32_t* chunk_counts = at<int32_t>(ws, L.chunk_counts);
   unsigned long long* chunk_psum = at<unsigned long long>(ws, L.chunk_psum);
   float* zpart = (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr;
-  if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, chunk_counts, chunk_psum,
-                                          zpart, st))
-    return cuda_rc(e);
-  if (stats && stats_in_route) {
-    if (cudaError_t e = launch_route_stats(p, chunk_counts, chunk_psum, L.n_chunks, zpart, L.n_sel_blocks, stats, st))
+  int kernels = 0;
+  {
+    int n_parts = 0;
+    float* parts = nullptr;
+    if (!(p.flags & MOE_FLAG_LOGITS_GIVEN)) {
+      if (p.dtype == kBF16) {
+        const int splits = router_k_splits(p);
+        if (splits > 1) {
+          parts = at<float>(ws, L.logit_parts);
+          n_parts = splits;
+        }
+        const int rc = launch_gate_logits_tc(p, x, w_gate, offset, splits > 1 ? parts : logits, splits, status, st);
+        if (rc) return MOE_ERR_CUDA;
+      } else {
+        if (cudaError_t e = launch_gate_logits_simt(p, x, w_gate, offset, logits, st)) return cuda_rc(e);
+      }
+      kernels += 1;
+    }
+    if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, chunk_counts, chunk_psum,
+                                            zpart, st))
       return cuda_rc(e);
+    kernels += 1;
+    *n_zpart = route_select_zparts(p);
   }
+  if (stats && stats_in_route) {
+    if (cudaError_t e = launch_route_stats(p, chunk_counts, chunk_psum, L.n_chunks, zpart, *n_zpart, stats, st))
+      return cuda_rc(e);
+    kernels += 1;
+  }
+  if (n_kernels) *n_kernels += kernels;
   return MOE_OK;
 }
 
@@ -248,9 +259,10 @@ int moe_route(const moe_problem_t* q, const void* x, const void* w_gate, const f
   if ((p.flags & MOE_FLAG_EXTENDED_STATS) && (p.flags & MOE_FLAG_EXPERT_CAPACITY)) return MOE_ERR_INVALID_ARG;
   if (!given && (!x || !w_gate || !aligned16(x) || !aligned16(w_gate))) return MOE_ERR_INVALID_ARG;
   const WsLayout L = make_layout(p);
+  int n_zpart = 0;
   return route_impl(p, x, w_gate, given ? nullptr : logit_offset, sel_bias, logits, topk_idx, topk_w, stats, ws,
                     L, reinterpret_cast<cudaStream_t>(stream), /*chunk_totals_cleared=*/false,
-                    /*stats_in_route=*/true);
+                    /*stats_in_route=*/true, &n_zpart, nullptr);
 }
 
 static int dispatch_entry(const moe_problem_t* q, const int32_t* topk_idx, const int32_t* expert_cap,
@@ -385,17 +397,17 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   // status word, chunk histogram and chunk p sums (contiguous at offset 0) start at zero
   if (cudaError_t e = cudaMemsetAsync(ws, 0, L.zero_bytes, st)) return cuda_rc(e);
   if (cudaError_t e = mark(MOE_EV_START)) return cuda_rc(e);
+  int n_zpart = 0;
   if (int rc = route_impl(p, x, w->w_gate, given ? nullptr : w->logit_offset, w->sel_bias, logits, idx, gw, stats,
-                          ws, L, st, /*chunk_totals_cleared=*/true, /*stats_in_route=*/false))
+                          ws, L, st, /*chunk_totals_cleared=*/true, /*stats_in_route=*/false, &n_zpart, &kernels))
     return rc;
-  kernels += (given ? 0 : 1) + 1;
   if (cudaError_t e = mark(MOE_EV_ROUTED)) return cuda_rc(e);
   // the scan also finalises the balance statistics from the chunk totals
   if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, at<int32_t>(ws, L.chunk_counts),
                                       at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true,
                                       at<unsigned long long>(ws, L.chunk_psum), stats,
                                       (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr,
-                                      L.n_sel_blocks, expert_cap))
+                                      n_zpart, expert_cap))
     return cuda_rc(e);
   kernels += 2;
   if (p.max_rows > 0) {

@@ -310,6 +310,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   }
 }
 
+int route_select_zparts(const Problem& p) { return static_cast<int>((p.T + kSelectTokens - 1) / kSelectTokens); }
+
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
                                 const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
                                 unsigned long long* chunk_psum, float* zpart, cudaStream_t st) {

@@ -160,6 +160,21 @@ def given_logits(cfg: MoeConfig, T: int | None = None) -> np.ndarray:
     return l
 
 
+def exact_router_inputs(T: int, d: int, E: int, seed: int) -> dict:
+    """Router inputs whose gate logits are exact in float32: x entries k/8 with
+    k in [-4, 4], w_gate integers in [-3, 3], offsets multiples of 1/8 in
+    [-1, 1].  Every product is a multiple of 1/8 of magnitude <= 1.5, so every
+    partial sum (d <= 4096) is a multiple of 1/8 below 2^13 in magnitude and
+    exact in float32: any summation order gives the same float32 (and float64)
+    value, and many logits tie exactly."""
+    assert d <= 4096
+    rng = np.random.default_rng(seed)
+    x = torch.from_numpy(rng.integers(-4, 5, size=(T, d)).astype(np.float32) / 8).to(torch.bfloat16)
+    w = torch.from_numpy(rng.integers(-3, 4, size=(E, d)).astype(np.float32)).to(torch.bfloat16)
+    off = (rng.integers(-8, 9, size=E) / 8).astype(np.float32)
+    return {"x": x, "w_gate": w, "logit_offset": off}
+
+
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Raw BF16 bits of a CPU bfloat16 tensor, as uint16 numpy (for the oracle)."""
     assert t.dtype == torch.bfloat16
