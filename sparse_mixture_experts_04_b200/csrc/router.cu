@@ -134,7 +134,8 @@ cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void*
 //   m = max logit; ex_e = exp(l_e - m) (fp32); Z = sum ex; p_e = ex_e / Z
 //   score_e (float64): l_e, or p64_e + b_e (bias on p), or l_e + b_e (bias on logit),
 //     p64 = exp(l - m) / sum exp(l - m) evaluated in float64
-//   K rounds of warp arg-max over (score desc, expert index asc)
+//   K rounds of warp arg-max over (score desc, expert index asc), each three
+//   redux.sync reductions over order-preserving 64-bit keys
 //   w_k = ex_{idx_k} / sum_k ex_{idx_k}    (= renormalised softmax over the chosen)
 // Per block: sum over its tokens of p_e (fp32, fixed order) and the number of
 // times each expert was chosen (integer), for the balance statistics.
@@ -205,78 +206,169 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
 #pragma unroll
     for (int i = 0; i < EPL; ++i) pacc[i] += ex[i] * invZ;
 
-    double score[EPL];
-    if (sel_bias == nullptr) {
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) score[i] = static_cast<double>(lg[i]);
-    } else if (bias_on_logit) {
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        score[i] = (e < E) ? static_cast<double>(lg[i]) + static_cast<double>(sel_bias[e]) : -INFINITY;
-      }
-    } else {
-      const double m64 = static_cast<double>(m);
-      double ex64[EPL];
-      double z64loc = 0.0;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        ex64[i] = (e < E) ? exp(static_cast<double>(lg[i]) - m64) : 0.0;
-        z64loc += ex64[i];
-      }
-      const double z64 = warp_sum(z64loc);
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        score[i] = (e < E) ? ex64[i] / z64 + static_cast<double>(sel_bias[e]) : -INFINITY;
-      }
-    }
-
-    // NaN scores rank lowest, so (score, index) is a total order and every
-    // lane agrees on each round's winner, which is always a valid expert.
-#pragma unroll
-    for (int i = 0; i < EPL; ++i)
-      if (score[i] != score[i]) score[i] = -INFINITY;
-    bool taken[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) taken[i] = (lane + 32 * i) >= E;
     int my_e = -1;
     float my_ex = 0.f;
-    for (int k = 0; k < K; ++k) {
-      double best = -INFINITY;
-      int best_e = 0x7fffffff;
+    bool done = false;
+    if (sel_bias != nullptr && !bias_on_logit) {
+      // Bias on p: rank the float32 scores s = ex/Z + b first (K+1 rounds over
+      // 32-bit keys).  Each is within d = (E+8) eps p + eps (|s| + 1) of the
+      // exact p + b (eps = 2^-23; terms: expf's 2 ulp, the sum Z, 1/Z, the
+      // product, the add, and the rounding of l - m, whose effect on p is at
+      // most eps |l - m| p / 2 <= eps / (2e)); if every gap between
+      // consecutive ones of the best K+1 exceeds 2d, the exact ranking of the
+      // top K is the same, else the token is ranked again in float64 below.
+      unsigned k32[EPL];
+      float s32[EPL];
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        if (!taken[i] && (best_e == 0x7fffffff || score[i] > best)) {
-          best = score[i];
-          best_e = lane + 32 * i;
-        }
+        const int e = lane + 32 * i;
+        float sc = (e < E) ? ex[i] * invZ + sel_bias[e] : 0.f;
+        if (sc != sc) sc = -INFINITY;
+        sc += 0.0f;
+        s32[i] = sc;
+        const unsigned b = __float_as_uint(sc);
+        k32[i] = e >= E ? 0u : ((b >> 31) ? ~b : (b | 0x80000000u));
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, best_e, o);
-        if (ob > best || (ob == best && oe < best_e)) {
-          best = ob;
-          best_e = oe;
-        }
-      }
-      // best_e is now the same on every lane
-      const int slot = best_e >> 5;
-      float ex_sel = 0.f;
+      unsigned bk = 0;
+      int bi = 0;
 #pragma unroll
       for (int i = 0; i < EPL; ++i)
-        if (i == slot) ex_sel = ex[i];
-      ex_sel = __shfl_sync(0xffffffffu, ex_sel, best_e & 31);
-      if (lane == (best_e & 31)) {
+        if (k32[i] > bk) {
+          bk = k32[i];
+          bi = i;
+        }
+      float my_s = 0.f, my_p = 0.f;
+      for (int r = 0; r <= K && r < 32; ++r) {
+        const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
+        const int best_e = __reduce_min_sync(0xffffffffu, (bk != 0u && bk == kmax) ? lane + 32 * bi : 0x7fffffff);
+        const int wl = best_e & 31;
+        float ex_mine = 0.f, s_mine = 0.f;
 #pragma unroll
         for (int i = 0; i < EPL; ++i)
-          if (i == slot) taken[i] = true;
+          if (i == bi) {
+            ex_mine = ex[i];
+            s_mine = s32[i];
+          }
+        const float ex_sel = __shfl_sync(0xffffffffu, ex_mine, wl);
+        const float s_sel = __shfl_sync(0xffffffffu, s_mine, wl);
+        if (lane == wl) {
+          bk = 0;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i)
+            if (i == bi) k32[i] = 0u;
+          bi = 0;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i)
+            if (k32[i] > bk) {
+              bk = k32[i];
+              bi = i;
+            }
+        }
+        if (lane == r) {
+          my_e = best_e;
+          my_ex = ex_sel;
+          my_s = s_sel;
+          my_p = ex_sel * invZ;
+        }
+        if (best_e == 0x7fffffff) break;  // fewer than K+1 experts (K == E)
       }
-      if (lane == k) {
-        my_e = best_e;
-        my_ex = ex_sel;
+      const float s_next = __shfl_down_sync(0xffffffffu, my_s, 1);
+      const float p_next = __shfl_down_sync(0xffffffffu, my_p, 1);
+      const float eps = 1.1920928955078125e-7f;  // 2^-23
+      const float d = (static_cast<float>(E) + 8.0f) * eps * fmaxf(my_p, p_next) +
+                      eps * (fmaxf(fabsf(my_s), fabsf(s_next)) + 1.0f);
+      // with K == E there is no (K+1)-th score: the last gap only orders the set
+      const bool last_ok = lane == K - 1 && K == E;
+      const bool gap_ok = lane >= K || last_ok || (my_s - s_next > 2.0f * d);
+      done = __all_sync(0xffffffffu, gap_ok);
+      if (!done) {
+        my_e = -1;
+        my_ex = 0.f;
+      }
+    }
+    if (!done) {
+      double score[EPL];
+      if (sel_bias == nullptr) {
+  #pragma unroll
+        for (int i = 0; i < EPL; ++i) score[i] = static_cast<double>(lg[i]);
+      } else if (bias_on_logit) {
+  #pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          score[i] = (e < E) ? static_cast<double>(lg[i]) + static_cast<double>(sel_bias[e]) : -INFINITY;
+        }
+      } else {
+        const double m64 = static_cast<double>(m);
+        double ex64[EPL];
+        double z64loc = 0.0;
+  #pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          ex64[i] = (e < E) ? exp(static_cast<double>(lg[i]) - m64) : 0.0;
+          z64loc += ex64[i];
+        }
+        const double z64 = warp_sum(z64loc);
+  #pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          score[i] = (e < E) ? ex64[i] / z64 + static_cast<double>(sel_bias[e]) : -INFINITY;
+        }
+      }
+
+      // Order-preserving 64-bit keys: a larger key is a larger score (NaN ranks
+      // as -inf, -0 as +0); padding lanes and chosen experts get key 0, below
+      // every real score.  (key, index ascending) is a total order, so every
+      // lane agrees on each round's winner, which is always a valid expert.
+      unsigned long long key[EPL];
+  #pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        double sc = score[i];
+        if (sc != sc) sc = -INFINITY;
+        sc += 0.0;
+        const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(sc));
+        key[i] = (lane + 32 * i) >= E ? 0ull : ((b >> 63) ? ~b : (b | 0x8000000000000000ull));
+      }
+      // this lane's best remaining entry (equal keys: the lower slot, i.e. expert)
+      unsigned long long bk = 0;
+      int bi = 0;
+  #pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (key[i] > bk) {
+          bk = key[i];
+          bi = i;
+        }
+      for (int k = 0; k < K; ++k) {
+        // warp arg-max: high word, then low word among the maxima, then the
+        // lowest expert index among equal keys
+        const unsigned hi = static_cast<unsigned>(bk >> 32), lo = static_cast<unsigned>(bk);
+        const unsigned hmax = __reduce_max_sync(0xffffffffu, hi);
+        const unsigned lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? lo : 0u);
+        const bool cand = bk != 0ull && hi == hmax && lo == lmax;
+        const int best_e = __reduce_min_sync(0xffffffffu, cand ? lane + 32 * bi : 0x7fffffff);
+        const int wl = best_e & 31;
+        float ex_mine = 0.f;
+  #pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (i == bi) ex_mine = ex[i];
+        const float ex_sel = __shfl_sync(0xffffffffu, ex_mine, wl);
+        if (lane == wl) {  // the winner's lane drops it and finds its next best
+          bk = 0;
+  #pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            if (i == bi) key[i] = 0ull;
+          }
+          bi = 0;
+  #pragma unroll
+          for (int i = 0; i < EPL; ++i)
+            if (key[i] > bk) {
+              bk = key[i];
+              bi = i;
+            }
+        }
+        if (lane == k) {
+          my_e = best_e;
+          my_ex = ex_sel;
+        }
       }
     }
     const float wsum = warp_sum(lane < K ? my_ex : 0.f);
