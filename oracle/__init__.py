@@ -29,6 +29,10 @@ Parity pins (what ties each function to something other than itself) are in
   router_zloss   all-equal logits give (l + ln E)^2
   utilization    uniform counts give log2 E bits (7 bits for 128 experts, the table's bound)
   flops          K=8, N_s=4, E=128 gives 12/128 (the compute-budget ratio)
+  layer_backward central finite differences of the forward (layer_rows, select,
+                 balance, router_zloss) with the routing held fixed, for every
+                 input and weight element; offset gradients sum to zero
+                 without the z-loss
 """
 from __future__ import annotations
 
@@ -82,6 +86,9 @@ def _L():
         lib.oracle_bias_update.restype = None
         lib.oracle_adaptive_capacity.argtypes = [i64, i32, i32, P, i32, f32, f32, P]
         lib.oracle_adaptive_capacity.restype = None
+        lib.oracle_layer_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, i32, P, P, P, P, P, i32,
+                                              P, P, P, P, P, f64, P, f64, f64, P, P, P, P, P, P, P]
+        lib.oracle_layer_backward.restype = ctypes.c_int
         lib.oracle_swiglu_accumulate.argtypes = [i32, i32, P, P, P, i32, f64, P, P]
         lib.oracle_swiglu_accumulate.restype = None
         lib.oracle_layer_rows.argtypes = [i64, i32, i32, i32, i32, i32, P, i32, P, P, P, P, i32,
@@ -340,3 +347,43 @@ def flops(T, d, E, F, n_shared, kept_pairs):
     out = np.empty(3, np.float64)
     _L().oracle_flops(int(T), int(d), int(E), int(F), int(n_shared), int(kept_pairs), _ptr(out))
     return float(out[0]), float(out[1]), float(out[2])
+
+
+def layer_backward(x, wg, w13, w2, logits, idx, w, slot_of, counts, alpha, dy, c_bal=1.0, c_z=0.0,
+                   w13_shared=None, w2_shared=None):
+    """Gradients of the layer for training (routing held fixed): dJ/dy = dy,
+    dJ/dL_balance = c_bal, dJ/dL_z = c_z.  Zen-Max §2.2 (experts), "Scaling with
+    experts" (The gating network, A balance penalty), Zen-Max §3.2 (z-loss).
+    Returns float64 arrays dx, dw13, dw2, dw13_shared, dw2_shared, dwg, doff."""
+    xa, xdt = _as_input(x)
+    ga, gdt = _as_input(wg)
+    a, wdt = _as_input(w13)
+    b, bdt = _as_input(w2)
+    assert gdt == wdt == bdt
+    T, d = xa.shape
+    E, F2, _ = a.shape
+    F = F2 // 2
+    K = np.asarray(idx).shape[1]
+    Ns = 0 if w13_shared is None else np.asarray(w13_shared).shape[0]
+    sa = sb = None
+    if Ns:
+        sa, sdt = _as_input(w13_shared)
+        sb, _ = _as_input(w2_shared)
+        assert sdt == wdt
+    la = np.ascontiguousarray(logits, dtype=np.float64)
+    ia = np.ascontiguousarray(idx, dtype=np.int32)
+    wa = np.ascontiguousarray(w, dtype=np.float64)
+    so = np.ascontiguousarray(slot_of, dtype=np.int32)
+    ca = np.ascontiguousarray(counts, dtype=np.int32)
+    dya = np.ascontiguousarray(dy, dtype=np.float64)
+    out = dict(dx=np.empty((T, d)), dw13=np.empty((E, 2 * F, d)), dw2=np.empty((E, d, F)),
+               dw13_shared=np.empty((Ns, 2 * F, d)), dw2_shared=np.empty((Ns, d, F)), dwg=np.empty((E, d)),
+               doff=np.empty(E))
+    rc = _L().oracle_layer_backward(T, d, E, K, F, Ns, _ptr(xa), xdt, _ptr(ga), _ptr(a), _ptr(b), _ptr(sa), _ptr(sb),
+                                    wdt, _ptr(la), _ptr(ia), _ptr(wa), _ptr(so), _ptr(ca), float(alpha), _ptr(dya),
+                                    float(c_bal), float(c_z), _ptr(out["dx"]), _ptr(out["dw13"]), _ptr(out["dw2"]),
+                                    _ptr(out["dw13_shared"]), _ptr(out["dw2_shared"]), _ptr(out["dwg"]),
+                                    _ptr(out["doff"]))
+    if rc != 0:
+        raise ValueError("expert index out of range")
+    return out

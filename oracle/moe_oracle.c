@@ -469,3 +469,169 @@ void oracle_flops(int64_t T, int32_t d, int32_t E, int32_t F, int32_t n_shared,
     out[1] = expert;
     out[2] = expert / (6.0 * (double)d * F * (double)E * (double)T);
 }
+
+/* ---------------------------------------------------------------------------
+ * Backward of the layer, for training.  [SE] "The gating network": a token's
+ * output is the gate-weighted sum of the experts it was sent to, so the loss
+ * reaches an expert only through the tokens it processed and reaches the
+ * router through those gates; [SE] "A balance penalty" and [ZX] §3.2 add two
+ * scalar terms computed from the router's probabilities.
+ *
+ * Given dy = dJ/dy for the forward's output y, and c_bal, c_z = dJ/dL for the
+ * balance loss L = alpha E sum_e f_e P_e and the router z-loss Lz =
+ * (1/T) sum_t lse_t^2, with the routing held fixed (the choice of experts and
+ * the capacity cut are piecewise constant, so they carry no gradient):
+ *   kept pair (t,k), e = idx[t,k]:  g = Wgate_e x, u = Wup_e x, h = silu(g) u,
+ *                                   o = Wdown_e h
+ *     dw_k = <dy_t, o>,  do = w_k dy_t
+ *     dWdown_e += do h^T;  dh = Wdown_e^T do
+ *     dg = dh u silu'(g);  du = dh silu(g);  silu'(g) = s (1 + g (1 - s)), s = sigmoid(g)
+ *     dWgate_e += dg x^T;  dWup_e += du x^T;  dx_t += Wgate_e^T dg + Wup_e^T du
+ *   dropped pair: dw_k = 0
+ *   shared expert s: the same with weight 1, for every token
+ *   router (w = softmax over the K chosen logits, p = softmax over all E):
+ *     dl_{i_k} += w_k (dw_k - sum_k' w_k' dw_k')
+ *     dl_e += p_e (q_e - sum_j p_j q_j),  q_e = c_bal alpha E f_e / T
+ *     dl_e += c_z (2 / T) lse_t p_e
+ *     dWg += dl x^T;  doffset += dl;  dx_t += Wg^T dl
+ * f_e = counts[e] / (T K) as in the forward statistics.  Outputs are
+ * overwritten, all in float64: dx [T,d], dw13 [E,2F,d], dw2 [E,d,F],
+ * dw13_sh [Ns,2F,d], dw2_sh [Ns,d,F], dwg [E,d], doff [E].  logits [T,E] are
+ * the forward's (offset included).  Returns 0, or -1 on a bad expert index.
+ * ------------------------------------------------------------------------- */
+int oracle_layer_backward(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32_t n_shared,
+                          const void* x, int32_t x_dt, const void* wg, const void* w13, const void* w2,
+                          const void* w13_sh, const void* w2_sh, int32_t w_dt,
+                          const double* logits, const int32_t* idx, const double* w, const int32_t* slot_of,
+                          const int32_t* counts, double alpha, const double* dy, double c_bal, double c_z,
+                          double* dx, double* dw13, double* dw2, double* dw13_sh, double* dw2_sh,
+                          double* dwg, double* doff) {
+    const int64_t w13_stride = 2 * (int64_t)F * d;
+    const int64_t w2_stride = (int64_t)d * F;
+    for (int64_t i = 0; i < T * d; ++i) dx[i] = 0.0;
+    for (int64_t i = 0; i < E * w13_stride; ++i) dw13[i] = 0.0;
+    for (int64_t i = 0; i < E * w2_stride; ++i) dw2[i] = 0.0;
+    for (int64_t i = 0; i < n_shared * w13_stride; ++i) dw13_sh[i] = 0.0;
+    for (int64_t i = 0; i < n_shared * w2_stride; ++i) dw2_sh[i] = 0.0;
+    for (int64_t i = 0; i < (int64_t)E * d; ++i) dwg[i] = 0.0;
+    for (int32_t e = 0; e < E; ++e) doff[e] = 0.0;
+
+    double* xr = (double*)malloc(sizeof(double) * (size_t)d);
+    double* g = (double*)malloc(sizeof(double) * (size_t)F);
+    double* u = (double*)malloc(sizeof(double) * (size_t)F);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)F);
+    double* dz = (double*)malloc(sizeof(double) * (size_t)F);   /* dg */
+    double* dv = (double*)malloc(sizeof(double) * (size_t)F);   /* du */
+    double* dwk = (double*)malloc(sizeof(double) * (size_t)K);
+    double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    double* dl = (double*)malloc(sizeof(double) * (size_t)E);
+    double* q = (double*)malloc(sizeof(double) * (size_t)E);
+    int rc = 0;
+    for (int32_t e = 0; e < E; ++e)
+        q[e] = c_bal * alpha * (double)E * ((double)counts[e] / ((double)T * (double)K)) / (double)T;
+
+    for (int64_t t = 0; t < T && rc == 0; ++t) {
+        for (int32_t j = 0; j < d; ++j) xr[j] = ld(x, x_dt, t * d + j);
+        const double* dyt = dy + t * d;
+        double* dxt = dx + t * d;
+        /* experts: n_shared shared ones (weight 1), then the token's K pairs */
+        for (int32_t r = 0; r < n_shared + K; ++r) {
+            const void *a, *b;
+            double* da;
+            double* db;
+            double scale;
+            if (r < n_shared) {
+                a = (const char*)w13_sh + (size_t)(r * w13_stride) * esz(w_dt);
+                b = (const char*)w2_sh + (size_t)(r * w2_stride) * esz(w_dt);
+                da = dw13_sh + r * w13_stride;
+                db = dw2_sh + r * w2_stride;
+                scale = 1.0;
+            } else {
+                int32_t k = r - n_shared;
+                dwk[k] = 0.0;
+                if (slot_of[t * K + k] < 0) continue;
+                int32_t e = idx[t * K + k];
+                if (e < 0 || e >= E) { rc = -1; break; }
+                a = (const char*)w13 + (size_t)(e * w13_stride) * esz(w_dt);
+                b = (const char*)w2 + (size_t)(e * w2_stride) * esz(w_dt);
+                da = dw13 + e * w13_stride;
+                db = dw2 + e * w2_stride;
+                scale = w[t * K + k];
+            }
+            for (int32_t f = 0; f < F; ++f) {
+                double gg = 0.0, uu = 0.0;
+                for (int32_t j = 0; j < d; ++j) {
+                    gg += ld(a, w_dt, (int64_t)f * d + j) * xr[j];
+                    uu += ld(a, w_dt, (int64_t)(F + f) * d + j) * xr[j];
+                }
+                g[f] = gg;
+                u[f] = uu;
+                h[f] = silu(gg) * uu;
+            }
+            if (r >= n_shared) {   /* dw_k = <dy_t, o>, o = Wdown h */
+                double acc = 0.0;
+                for (int32_t i = 0; i < d; ++i) {
+                    double o = 0.0;
+                    for (int32_t f = 0; f < F; ++f) o += ld(b, w_dt, (int64_t)i * F + f) * h[f];
+                    acc += dyt[i] * o;
+                }
+                dwk[r - n_shared] = acc;
+            }
+            /* do = scale dy_t */
+            for (int32_t f = 0; f < F; ++f) dh[f] = 0.0;
+            for (int32_t i = 0; i < d; ++i) {
+                double doi = scale * dyt[i];
+                for (int32_t f = 0; f < F; ++f) {
+                    db[(int64_t)i * F + f] += doi * h[f];
+                    dh[f] += ld(b, w_dt, (int64_t)i * F + f) * doi;
+                }
+            }
+            for (int32_t f = 0; f < F; ++f) {
+                double sg = 1.0 / (1.0 + exp(-g[f]));
+                dz[f] = dh[f] * u[f] * (sg * (1.0 + g[f] * (1.0 - sg)));
+                dv[f] = dh[f] * silu(g[f]);
+            }
+            for (int32_t f = 0; f < F; ++f) {
+                for (int32_t j = 0; j < d; ++j) {
+                    da[(int64_t)f * d + j] += dz[f] * xr[j];
+                    da[(int64_t)(F + f) * d + j] += dv[f] * xr[j];
+                    dxt[j] += ld(a, w_dt, (int64_t)f * d + j) * dz[f] + ld(a, w_dt, (int64_t)(F + f) * d + j) * dv[f];
+                }
+            }
+        }
+        if (rc) break;
+        /* router */
+        const double* lt = logits + t * E;
+        double m = lt[0];
+        for (int32_t e = 1; e < E; ++e) if (lt[e] > m) m = lt[e];
+        double zs = 0.0;
+        for (int32_t e = 0; e < E; ++e) { p[e] = exp(lt[e] - m); zs += p[e]; }
+        for (int32_t e = 0; e < E; ++e) p[e] /= zs;
+        double lse = m + log(zs);
+        for (int32_t e = 0; e < E; ++e) dl[e] = 0.0;
+        double wdw = 0.0;
+        for (int32_t k = 0; k < K; ++k) wdw += w[t * K + k] * dwk[k];
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t e = idx[t * K + k];
+            if (e < 0 || e >= E) { rc = -1; break; }
+            dl[e] += w[t * K + k] * (dwk[k] - wdw);
+        }
+        if (rc) break;
+        double pq = 0.0;
+        for (int32_t e = 0; e < E; ++e) pq += p[e] * q[e];
+        for (int32_t e = 0; e < E; ++e) {
+            dl[e] += p[e] * (q[e] - pq);
+            dl[e] += c_z * (2.0 / (double)T) * lse * p[e];
+        }
+        for (int32_t e = 0; e < E; ++e) {
+            doff[e] += dl[e];
+            for (int32_t j = 0; j < d; ++j) {
+                dwg[(int64_t)e * d + j] += dl[e] * xr[j];
+                dxt[j] += ld(wg, w_dt, (int64_t)e * d + j) * dl[e];
+            }
+        }
+    }
+    free(xr); free(g); free(u); free(h); free(dh); free(dz); free(dv); free(dwk); free(p); free(dl); free(q);
+    return rc;
+}

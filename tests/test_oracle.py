@@ -513,3 +513,94 @@ def test_adaptive_capacity_monotone_in_load():
     # under-used experts lose budget, over-used gain it (page: prevents drops under skew)
     base = oracle.capacity(2048, 2, E, 1.0)
     assert (caps[load < load.mean()] <= base).all() and (caps[load > load.mean()] >= base).all()
+
+
+# ---------------------------------------------- layer backward (training)
+def _fd_problem(seed=0, T=6, d=5, E=4, K=2, F=3, Ns=1, cap=3):
+    rng = np.random.default_rng(seed)
+    P = dict(x=rng.normal(size=(T, d)), wg=rng.normal(size=(E, d)) * 0.7, off=rng.normal(size=E).astype(np.float32),
+             w13=rng.normal(size=(E, 2 * F, d)) * 0.5, w2=rng.normal(size=(E, d, F)) * 0.5,
+             w13s=rng.normal(size=(Ns, 2 * F, d)) * 0.5, w2s=rng.normal(size=(Ns, d, F)) * 0.5)
+    R = rng.normal(size=(T, d))
+    return P, R, dict(T=T, d=d, E=E, K=K, F=F, Ns=Ns, cap=cap)
+
+
+def _objective(P, R, c, idx_fixed, slot_fixed, counts_fixed, c_bal, c_z, alpha=0.01):
+    """J = sum(R * y) + c_bal * L_balance + c_z * L_z through the oracle's own forward,
+    with the routing (chosen experts, capacity cut, counts) held fixed."""
+    logits = oracle.gate_logits(P["x"], P["wg"], P["off"])
+    idx, w, p = oracle.select(logits, c["K"])
+    assert (idx == idx_fixed).all(), "perturbation changed the routing"
+    y = oracle.layer_rows(P["x"], P["w13"], P["w2"], idx, w, slot_fixed,
+                          w13_shared=P["w13s"] if c["Ns"] else None, w2_shared=P["w2s"] if c["Ns"] else None)
+    _, _, loss = oracle.balance(counts_fixed, p, c["K"], alpha)
+    return float(np.sum(R * y)) + c_bal * loss + c_z * oracle.router_zloss(logits)
+
+
+@pytest.mark.parametrize("seed,c_bal,c_z,cap", [(0, 1.0, 0.0, 3), (1, 0.7, 0.3, 2), (2, 0.0, 1.0, -1)])
+def test_layer_backward_matches_finite_differences(seed, c_bal, c_z, cap):
+    P, R, c = _fd_problem(seed, cap=cap)
+    alpha = 0.01
+    logits = oracle.gate_logits(P["x"], P["wg"], P["off"])
+    idx, w, p = oracle.select(logits, c["K"])
+    disp = oracle.dispatch(idx, c["E"], cap)
+    assert cap < 0 or (disp["slot_of"] < 0).any() or cap >= c["T"]
+    g = oracle.layer_backward(P["x"], P["wg"], P["w13"], P["w2"], logits, idx, w, disp["slot_of"], disp["counts"],
+                              alpha, R, c_bal, c_z, P["w13s"], P["w2s"])
+    h = 1e-6
+    names = {"x": "dx", "wg": "dwg", "w13": "dw13", "w2": "dw2", "w13s": "dw13_shared", "w2s": "dw2_shared"}
+    for name, gname in names.items():
+        arr = P[name]
+        fd = np.empty_like(arr)
+        for i in np.ndindex(arr.shape):
+            keep = arr[i]
+            arr[i] = keep + h
+            jp = _objective(P, R, c, idx, disp["slot_of"], disp["counts"], c_bal, c_z, alpha)
+            arr[i] = keep - h
+            jm = _objective(P, R, c, idx, disp["slot_of"], disp["counts"], c_bal, c_z, alpha)
+            arr[i] = keep
+            fd[i] = (jp - jm) / (2 * h)
+        err = np.max(np.abs(fd - g[gname]))
+        assert err <= 1e-6 * max(1.0, float(np.max(np.abs(fd)))), (name, err)
+    # the offset (a float32 input) enters like a logit shared by all tokens; steps of
+    # 2^-12 are exact in float32 at these magnitudes, so the difference quotient is exact
+    fdo = np.empty(c["E"])
+    hs = np.float32(2.0 ** -12)
+    for e in range(c["E"]):
+        P2 = dict(P)
+        o = P["off"].copy(); o[e] += hs
+        P2["off"] = o
+        jp = _objective(P2, R, c, idx, disp["slot_of"], disp["counts"], c_bal, c_z, alpha)
+        o = P["off"].copy(); o[e] -= hs
+        P2["off"] = o
+        jm = _objective(P2, R, c, idx, disp["slot_of"], disp["counts"], c_bal, c_z, alpha)
+        fdo[e] = (jp - jm) / (2.0 * float(hs))
+    assert np.max(np.abs(fdo - g["doff"])) <= 1e-5 * max(1.0, float(np.max(np.abs(fdo))))
+
+
+def test_layer_backward_offset_gradient_sums_to_zero_without_zloss():
+    # the gate-weight and balance terms are softmax Jacobians: each token's dl sums to 0
+    P, R, c = _fd_problem(5, T=9, E=6, K=3)
+    logits = oracle.gate_logits(P["x"], P["wg"], P["off"])
+    idx, w, p = oracle.select(logits, c["K"])
+    disp = oracle.dispatch(idx, c["E"], -1)
+    g = oracle.layer_backward(P["x"], P["wg"], P["w13"], P["w2"], logits, idx, w, disp["slot_of"], disp["counts"],
+                              0.01, R, 1.0, 0.0, P["w13s"], P["w2s"])
+    assert abs(float(np.sum(g["doff"]))) <= 1e-12
+    g2 = oracle.layer_backward(P["x"], P["wg"], P["w13"], P["w2"], logits, idx, w, disp["slot_of"], disp["counts"],
+                               0.01, R, 1.0, 1.0, P["w13s"], P["w2s"])
+    # with the z-loss: sum_e dl_e = (2/T) lse_t per token
+    lse = np.log(np.sum(np.exp(logits - logits.max(1, keepdims=True)), 1)) + logits.max(1)
+    assert abs(float(np.sum(g2["doff"])) - float(np.sum(2.0 / c["T"] * lse))) <= 1e-12 * max(1.0, float(np.sum(np.abs(lse))))
+
+
+def test_layer_backward_dropped_pairs_give_their_expert_no_gradient():
+    P, R, c = _fd_problem(3, T=8, E=4, K=2, cap=1)
+    logits = oracle.gate_logits(P["x"], P["wg"], P["off"])
+    idx, w, p = oracle.select(logits, c["K"])
+    disp = oracle.dispatch(idx, c["E"], 1)
+    g = oracle.layer_backward(P["x"], P["wg"], P["w13"], P["w2"], logits, idx, w, disp["slot_of"], disp["counts"],
+                              0.01, R, 0.0, 0.0, P["w13s"], P["w2s"])
+    for e in range(c["E"]):
+        if disp["kept"][e] == 0:
+            assert not g["dw13"][e].any() and not g["dw2"][e].any()
