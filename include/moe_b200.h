@@ -317,6 +317,46 @@ int moe_balance_update(const moe_problem_t* p, const int32_t* counts,
                        float c_base, float gamma, int32_t* expert_capacity,
                        moe_stream_t stream);
 
+/* Gradients of the layer (device pointers, caller-owned).  FP32 weight
+ * gradients in the weights' layouts; each optional one may be NULL. */
+typedef struct moe_grads {
+    void* dx;            /* [T, d] activations dtype, or NULL */
+    float* dw13;         /* [E, 2F, d] (required) */
+    float* dw2;          /* [E, d, F] (required) */
+    float* dw13_shared;  /* [N_s, 2F, d], NULL iff n_shared == 0 */
+    float* dw2_shared;   /* [N_s, d, F],  NULL iff n_shared == 0 */
+    float* dw_gate;      /* [E, d] or NULL; must be NULL with MOE_FLAG_LOGITS_GIVEN */
+    float* d_offset;     /* [E] or NULL (gradient of logit_offset) */
+    float* d_logits;     /* [T, E] or NULL (gradient of the router logits) */
+} moe_grads_t;
+
+/* Scratch needed by moe_layer_backward (bytes).  Pure host function. */
+int moe_backward_workspace_size(const moe_problem_t* p, size_t* bytes);
+
+/* Backward of moe_layer_forward, for training.  Scaling with experts, "The
+ * gating network" (the gate-weighted sum; gradients reach an expert only
+ * through the tokens it processed), "A balance penalty"; Zen-Max §2.2
+ * (Expert_i), §3.2 (router z-loss).  The routing of the forward is held fixed:
+ * the choice of experts and the capacity cut carry no gradient, nor does the
+ * selection bias.
+ *   x, w     the forward's inputs (unchanged since)
+ *   routing  the forward's routing (any NULL member is read from fwd_ws, where
+ *            the forward then kept it)
+ *   fwd_ws   the forward's workspace, untouched since that call (it holds the
+ *            expert inputs, hidden activations and outputs the backward reads)
+ *   dy       [T, d] dJ/dy; d_loss, d_zloss: dJ/d(balance loss), dJ/d(z-loss)
+ *   grads    outputs (see moe_grads_t); the weight gradients are overwritten
+ *   ws       moe_backward_workspace_size bytes, 256-byte aligned
+ * Computes in BF16 with FP32 accumulation, like the forward: intermediate
+ * gradients (dO, dh -> dg/du, dx rows, the logit gradient fed to the tensor
+ * cores) are rounded to BF16, weight gradients accumulate in FP32 in TMEM.
+ * The gate and up projections are recomputed from the forward's expert
+ * inputs.  FP32 problems return MOE_ERR_UNSUPPORTED. */
+int moe_layer_backward(const moe_problem_t* p, const void* x, const moe_weights_t* w,
+                       const moe_routing_t* routing, const void* fwd_ws, size_t fwd_ws_bytes,
+                       const void* dy, float d_loss, float d_zloss, const moe_grads_t* grads,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Stage boundaries recorded by moe_layer_forward_profiled. */
 #define MOE_EV_START 0   /* before the router */
 #define MOE_EV_ROUTED 1  /* after gate logits, selection and statistics */

@@ -87,7 +87,7 @@ def _L():
         lib.oracle_adaptive_capacity.argtypes = [i64, i32, i32, P, i32, f32, f32, P]
         lib.oracle_adaptive_capacity.restype = None
         lib.oracle_layer_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, i32, P, P, P, P, P, i32,
-                                              P, P, P, P, P, f64, P, f64, f64, P, P, P, P, P, P, P]
+                                              P, P, P, P, P, f64, P, f64, f64, P, P, P, P, P, P, P, P]
         lib.oracle_layer_backward.restype = ctypes.c_int
         lib.oracle_swiglu_accumulate.argtypes = [i32, i32, P, P, P, i32, f64, P, P]
         lib.oracle_swiglu_accumulate.restype = None
@@ -354,7 +354,7 @@ def layer_backward(x, wg, w13, w2, logits, idx, w, slot_of, counts, alpha, dy, c
     """Gradients of the layer for training (routing held fixed): dJ/dy = dy,
     dJ/dL_balance = c_bal, dJ/dL_z = c_z.  Zen-Max §2.2 (experts), "Scaling with
     experts" (The gating network, A balance penalty), Zen-Max §3.2 (z-loss).
-    Returns float64 arrays dx, dw13, dw2, dw13_shared, dw2_shared, dwg, doff."""
+    Returns float64 arrays dx, dw13, dw2, dw13_shared, dw2_shared, dwg, doff, dlogits."""
     xa, xdt = _as_input(x)
     ga, gdt = _as_input(wg)
     a, wdt = _as_input(w13)
@@ -378,12 +378,12 @@ def layer_backward(x, wg, w13, w2, logits, idx, w, slot_of, counts, alpha, dy, c
     dya = np.ascontiguousarray(dy, dtype=np.float64)
     out = dict(dx=np.empty((T, d)), dw13=np.empty((E, 2 * F, d)), dw2=np.empty((E, d, F)),
                dw13_shared=np.empty((Ns, 2 * F, d)), dw2_shared=np.empty((Ns, d, F)), dwg=np.empty((E, d)),
-               doff=np.empty(E))
+               doff=np.empty(E), dlogits=np.empty((T, E)))
     rc = _L().oracle_layer_backward(T, d, E, K, F, Ns, _ptr(xa), xdt, _ptr(ga), _ptr(a), _ptr(b), _ptr(sa), _ptr(sb),
                                     wdt, _ptr(la), _ptr(ia), _ptr(wa), _ptr(so), _ptr(ca), float(alpha), _ptr(dya),
                                     float(c_bal), float(c_z), _ptr(out["dx"]), _ptr(out["dw13"]), _ptr(out["dw2"]),
                                     _ptr(out["dw13_shared"]), _ptr(out["dw2_shared"]), _ptr(out["dwg"]),
-                                    _ptr(out["doff"]))
+                                    _ptr(out["doff"]), _ptr(out["dlogits"]))
     if rc != 0:
         raise ValueError("expert index out of range")
     return out

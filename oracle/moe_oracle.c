@@ -496,8 +496,9 @@ void oracle_flops(int64_t T, int32_t d, int32_t E, int32_t F, int32_t n_shared,
  *     dWg += dl x^T;  doffset += dl;  dx_t += Wg^T dl
  * f_e = counts[e] / (T K) as in the forward statistics.  Outputs are
  * overwritten, all in float64: dx [T,d], dw13 [E,2F,d], dw2 [E,d,F],
- * dw13_sh [Ns,2F,d], dw2_sh [Ns,d,F], dwg [E,d], doff [E].  logits [T,E] are
- * the forward's (offset included).  Returns 0, or -1 on a bad expert index.
+ * dw13_sh [Ns,2F,d], dw2_sh [Ns,d,F], dwg [E,d], doff [E], and dlogits
+ * [T,E] (the dl above) when not NULL.  logits [T,E] are the forward's (offset
+ * included).  Returns 0, or -1 on a bad expert index.
  * ------------------------------------------------------------------------- */
 int oracle_layer_backward(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32_t n_shared,
                           const void* x, int32_t x_dt, const void* wg, const void* w13, const void* w2,
@@ -505,7 +506,7 @@ int oracle_layer_backward(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F,
                           const double* logits, const int32_t* idx, const double* w, const int32_t* slot_of,
                           const int32_t* counts, double alpha, const double* dy, double c_bal, double c_z,
                           double* dx, double* dw13, double* dw2, double* dw13_sh, double* dw2_sh,
-                          double* dwg, double* doff) {
+                          double* dwg, double* doff, double* dlogits) {
     const int64_t w13_stride = 2 * (int64_t)F * d;
     const int64_t w2_stride = (int64_t)d * F;
     for (int64_t i = 0; i < T * d; ++i) dx[i] = 0.0;
@@ -624,6 +625,8 @@ int oracle_layer_backward(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F,
             dl[e] += p[e] * (q[e] - pq);
             dl[e] += c_z * (2.0 / (double)T) * lse * p[e];
         }
+        if (dlogits)
+            for (int32_t e = 0; e < E; ++e) dlogits[t * E + e] = dl[e];
         for (int32_t e = 0; e < E; ++e) {
             doff[e] += dl[e];
             for (int32_t j = 0; j < d; ++j) {

@@ -26,7 +26,8 @@ DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
 EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
             "moe_reset_device_status", "moe_read_device_status", "moe_route", "moe_dispatch",
             "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
-            "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update")
+            "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update", "moe_backward_workspace_size",
+            "moe_layer_backward")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
 
@@ -48,6 +49,12 @@ class MoeRouting(ctypes.Structure):
     _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
                 ("counts", ctypes.c_void_p), ("kept", ctypes.c_void_p), ("seg_off", ctypes.c_void_p),
                 ("slot_of", ctypes.c_void_p), ("perm", ctypes.c_void_p)]
+
+
+class MoeGrads(ctypes.Structure):
+    _fields_ = [("dx", ctypes.c_void_p), ("dw13", ctypes.c_void_p), ("dw2", ctypes.c_void_p),
+                ("dw13_shared", ctypes.c_void_p), ("dw2_shared", ctypes.c_void_p), ("dw_gate", ctypes.c_void_p),
+                ("d_offset", ctypes.c_void_p), ("d_logits", ctypes.c_void_p)]
 
 
 class MoeError(RuntimeError):
@@ -97,6 +104,11 @@ def lib() -> ctypes.CDLL:
     L.moe_balance_update.argtypes = [PP, P, P, ctypes.c_float, i32, P, i32, i64, ctypes.c_float, ctypes.c_float,
                                      P, P]
     L.moe_balance_update.restype = ctypes.c_int
+    L.moe_backward_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
+    L.moe_backward_workspace_size.restype = ctypes.c_int
+    L.moe_layer_backward.argtypes = [PP, P, ctypes.POINTER(MoeWeights), ctypes.POINTER(MoeRouting), P, sz, P,
+                                     ctypes.c_float, ctypes.c_float, ctypes.POINTER(MoeGrads), P, sz, P]
+    L.moe_layer_backward.restype = ctypes.c_int
     if L.moe_abi_version() != ABI_VERSION:
         raise RuntimeError(f"{LIB_PATH} has ABI version {L.moe_abi_version()}, this binding expects {ABI_VERSION}: "
                            "rebuild it")

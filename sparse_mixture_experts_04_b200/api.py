@@ -13,11 +13,12 @@ import torch
 from . import _lib
 from ._lib import (BIAS_UPDATE_PROPORTIONAL, BIAS_UPDATE_SIGN, DTYPE_BF16, DTYPE_F32, EXTENDED_STATS, FFN_ROUTED,
                    FFN_SHARED, FLAG_BIAS_LOGIT, FLAG_EXPERT_CAPACITY, FLAG_EXTENDED_STATS, FLAG_LOGITS_GIVEN,
-                   MoeError, MoeProblem, MoeRouting, MoeWeights)
+                   MoeError, MoeGrads, MoeProblem, MoeRouting, MoeWeights)
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_profiled", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
+           "moe_layer_backward", "backward_workspace_size", "alloc_backward_workspace",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
            "FLAG_EXTENDED_STATS", "FLAG_EXPERT_CAPACITY", "EXTENDED_STATS", "stats_size",
            "BIAS_UPDATE_SIGN", "BIAS_UPDATE_PROPORTIONAL",
@@ -171,3 +172,28 @@ def moe_layer_forward_profiled(prob, x, weights: dict, y, routing: dict | None, 
                                                ws.numel(), _stream(stream), handles, ctypes.byref(n))
     _lib.check("moe_layer_forward_profiled", rc)
     return int(n.value)
+
+
+def backward_workspace_size(prob: MoeProblem) -> int:
+    n = ctypes.c_size_t(0)
+    _lib.check("moe_backward_workspace_size", _lib.lib().moe_backward_workspace_size(ctypes.byref(prob), ctypes.byref(n)))
+    return int(n.value)
+
+
+def alloc_backward_workspace(prob: MoeProblem, device="cuda") -> torch.Tensor:
+    return torch.zeros(backward_workspace_size(prob), dtype=torch.uint8, device=device)
+
+
+def moe_layer_backward(prob, x, weights: dict, routing: dict | None, fwd_ws, dy, d_loss, d_zloss, grads: dict, ws,
+                       stream=None):
+    """Gradients of the layer (see moe_layer_backward in the header); grads maps
+    dx, dw13, dw2, dw13_shared, dw2_shared, dw_gate, d_offset, d_logits to
+    tensors (missing or None: not computed; dw13 and dw2 required)."""
+    g = MoeGrads(*[_p(grads.get(k)) for k in ("dx", "dw13", "dw2", "dw13_shared", "dw2_shared", "dw_gate",
+                                               "d_offset", "d_logits")])
+    r = _routing_struct(routing)
+    rc = _lib.lib().moe_layer_backward(ctypes.byref(prob), _p(x), ctypes.byref(_weights_struct(weights)),
+                                       ctypes.byref(r) if r is not None else None, _p(fwd_ws), fwd_ws.numel(),
+                                       _p(dy), float(d_loss), float(d_zloss), ctypes.byref(g), _p(ws), ws.numel(),
+                                       _stream(stream))
+    _lib.check("moe_layer_backward", rc)

@@ -10,6 +10,10 @@
 
 namespace moe {
 
+// BF16 TMA tensor map (host): dims[0] innermost, 128-byte swizzle, box inner
+// extent 64 elements, zero fill out of bounds (expert_gemm.cu).
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box);
+
 // Status bits written into the first word of the caller's workspace.
 constexpr unsigned kDevBadExpert = 0x1u;
 constexpr unsigned kDevWaitTimeout = 0x2u;
@@ -163,6 +167,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (tcgen05.mma operands).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // named_bar_sync that also ANDs one predicate over the participating threads.
 __device__ __forceinline__ bool named_bar_and(int id, int threads, bool v) {
   uint32_t r;
@@ -188,6 +198,28 @@ __device__ __forceinline__ uint64_t smem_desc_k128(uint32_t saddr) {
   desc |= static_cast<uint64_t>(1) << 46;                  // descriptor version (sm_100)
   desc |= static_cast<uint64_t>(2) << 61;                  // 128-byte swizzle
   return desc;
+}
+
+// Shared-memory matrix descriptor, MN-major operand with 128-byte swizzle: rows
+// of 64 MN-elements (128 B) per K index, 8 K rows per 1024-byte atom.
+//   lbo: bytes between consecutive 64-element MN chunks
+//   sbo: bytes between consecutive groups of 8 K rows (1024 when the K rows
+//        of a chunk are contiguous)
+__device__ __forceinline__ uint64_t smem_desc_mn128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t desc = 0;
+  desc |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  desc |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  desc |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  desc |= static_cast<uint64_t>(1) << 46;
+  desc |= static_cast<uint64_t>(2) << 61;
+  return desc;
+}
+
+// Instruction descriptor: BF16 x BF16 -> FP32, M x N; a_mn / b_mn select the
+// MN-major ("transposed") layout for A / B (bits 15 / 16), else K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor: BF16 x BF16 -> FP32, both operands K-major, M x N.

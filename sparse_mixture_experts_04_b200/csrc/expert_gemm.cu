@@ -752,7 +752,7 @@ static EncodeTiledFn encode_fn() {
 
 // BF16 tensor map: dims[0] innermost (contiguous), 128-byte swizzle, zero fill
 // out of bounds.  Box inner extent is always 64 elements (128 bytes).
-static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box) {
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[3], gstr[2];
@@ -1017,6 +1017,36 @@ static int ffn_simt(const Problem& p, int mode, const void* x_rows, int64_t n_ro
   return launch_k(ffn_simt_kernel<false>, g2, dim3(256), 0, st, static_cast<const float*>(h),
                   static_cast<int>(up.ldo), static_cast<const float*>(w2), dn, static_cast<int64_t>(p.d) * p.F,
                   static_cast<int64_t>(0)) == cudaSuccess ? 0 : -3;
+}
+
+// The gate and up projections without SwiGLU, for the backward: gu = x W13^T
+// as BF16 (routed: [n_rows, 2F] per expert row; shared: [n_rows, N_s * 2F],
+// expert s in columns [2F s, 2F (s + 1))), columns 0..F-1 of a block the gate
+// projection, F..2F-1 the up projection.
+int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
+                          const void* w13, void* gu, unsigned* status, cudaStream_t st) {
+  if (n_rows <= 0) return 0;
+  const bool routed = mode == 0;
+  const int G = routed ? p.E : p.Ns;
+  CUtensorMap ta, tb;
+  const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
+  const uint32_t ba[2] = {kBK, kBM};
+  const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(2 * p.F), static_cast<uint64_t>(G)};
+  const uint32_t bb[3] = {kBK, 256, 1};
+  if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
+  GemmArgs a{};
+  a.n_groups = G;
+  a.seg_off = routed ? seg_off : nullptr;
+  a.n_rows = static_cast<int>(n_rows);
+  a.N = 2 * p.F;
+  a.K = p.d;
+  a.k_groups = 1;
+  a.out = gu;
+  a.ldo = routed ? 2 * static_cast<int64_t>(p.F) : 2 * static_cast<int64_t>(p.F) * p.Ns;
+  a.out_col_stride = routed ? 0 : 2 * p.F;
+  a.status = status;
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
+  return run_gemm<EPI_BF16, 256, 4>(ta, tb, a, mt * cdiv(2 * p.F, 256), st);
 }
 
 // mode 0: routed (groups = experts over seg_off); mode 1: shared (every row

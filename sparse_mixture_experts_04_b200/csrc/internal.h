@@ -93,6 +93,21 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
                       cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr);
 
+// expert_gemm.cu: gu = x W13^T (gate | up projections, BF16) for the backward
+int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
+                          const void* w13, void* gu, unsigned* status, cudaStream_t st);
+// grad_gemm.cu: backward of the expert FFNs (see there); returns a moe_status value
+int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, int64_t n_rows,
+                               const int32_t* seg_off, const void* w13, const void* w2, const void* dout,
+                               const void* h, void* gu, void* dgu, void* dx_rows, float* dw13, float* dw2,
+                               unsigned* status, cudaStream_t st);
+
+// grad_gemm.cu: router gradients through the gate GEMM from dl [T, e_pad] BF16
+int launch_router_dgrad(const Problem& p, const void* dl16, int e_pad, const void* w_gate, void* dx_r,
+                        unsigned* status, cudaStream_t st);
+int launch_router_wgrad(const Problem& p, const void* dl16, int e_pad, const void* x, float* dwg, unsigned* status,
+                        cudaStream_t st);
+
 // combine.cu
 cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
                            const void* y_shared, void* y, cudaStream_t st);

@@ -63,6 +63,28 @@ class MoeLayer:
 
     __call__ = forward
 
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, d_loss: float = 1.0, d_zloss: float = 0.0,
+                 stream=None) -> dict:
+        """Gradients of the last forward (same x; the workspace untouched since),
+        for dJ/dy = dy and dJ/d(balance loss) = d_loss, dJ/d(z-loss) = d_zloss.
+        Returns FP32 weight gradients and dx (activation dtype)."""
+        P, dev = self.prob, self.device
+        f32 = dict(dtype=torch.float32, device=dev)
+        E, d, F, Ns, T = P.n_experts, P.d_model, P.d_ff, P.n_shared, P.T
+        g = dict(dx=torch.empty((T, d), dtype=self.dtype, device=dev), dw13=torch.empty((E, 2 * F, d), **f32),
+                 dw2=torch.empty((E, d, F), **f32), d_offset=torch.empty(E, **f32),
+                 d_logits=torch.empty((T, E), **f32))
+        if not P.flags & api.FLAG_LOGITS_GIVEN:
+            g["dw_gate"] = torch.empty((E, d), **f32)
+        if Ns:
+            g["dw13_shared"] = torch.empty((Ns, 2 * F, d), **f32)
+            g["dw2_shared"] = torch.empty((Ns, d, F), **f32)
+        if getattr(self, "_bwd_ws", None) is None:
+            self._bwd_ws = api.alloc_backward_workspace(P, dev)
+        api.moe_layer_backward(P, x, self.weights, self.routing, self.ws, dy, d_loss, d_zloss, g, self._bwd_ws,
+                               stream)
+        return g
+
     def balance_update(self, bias_rate: float = 0.0, bias_mode: int = api.BIAS_UPDATE_SIGN, c_base: float | None = None,
                        gamma: float = 0.0, window: int = 8, stream=None) -> None:
         """Between steps: move the selection bias against the last forward's

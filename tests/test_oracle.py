@@ -604,3 +604,29 @@ def test_layer_backward_dropped_pairs_give_their_expert_no_gradient():
     for e in range(c["E"]):
         if disp["kept"][e] == 0:
             assert not g["dw13"][e].any() and not g["dw2"][e].any()
+
+
+def test_layer_backward_logit_gradient_matches_finite_differences():
+    P, R, c = _fd_problem(7, T=5, E=5, K=2, cap=2)
+    alpha, c_bal, c_z = 0.01, 0.9, 0.4
+    logits = oracle.gate_logits(P["x"], P["wg"], P["off"])
+    idx, w, p = oracle.select(logits, c["K"])
+    disp = oracle.dispatch(idx, c["E"], c["cap"])
+    g = oracle.layer_backward(P["x"], P["wg"], P["w13"], P["w2"], logits, idx, w, disp["slot_of"], disp["counts"],
+                              alpha, R, c_bal, c_z, P["w13s"], P["w2s"])
+
+    def J(l):
+        i2, w2, p2 = oracle.select(l, c["K"])
+        assert (i2 == idx).all()
+        y = oracle.layer_rows(P["x"], P["w13"], P["w2"], i2, w2, disp["slot_of"], w13_shared=P["w13s"],
+                              w2_shared=P["w2s"])
+        _, _, loss = oracle.balance(disp["counts"], p2, c["K"], alpha)
+        return float(np.sum(R * y)) + c_bal * loss + c_z * oracle.router_zloss(l)
+
+    fd = np.empty_like(logits)
+    for i in np.ndindex(logits.shape):
+        lp = logits.copy(); lp[i] += 1e-6
+        lm = logits.copy(); lm[i] -= 1e-6
+        fd[i] = (J(lp) - J(lm)) / 2e-6
+    assert np.max(np.abs(fd - g["dlogits"])) <= 1e-6 * max(1.0, float(np.max(np.abs(fd))))
+    assert np.allclose(g["dlogits"].sum(0), g["doff"], rtol=0, atol=1e-12)
