@@ -380,6 +380,36 @@ def run_ours(args, cfg):
     d2h = ys_e[0].numel() * ys_e[0].element_size() + layer.stats.numel() * 4
     y = torch.empty(0)
 
+    # training: the backward of a forward over the same batch (moe_layer_backward),
+    # timed on its own (not part of the forward metric); BF16 problems only
+    bwd = None
+    if cfg.dtype == "bf16" and not args.no_backward:
+        gen = torch.Generator(device="cuda").manual_seed(rcfg.seed)
+        dy = torch.randn((T, cfg.d_model), generator=gen, device="cuda").to(torch.bfloat16)
+        n_b = 3
+        b_ms = []
+        for i in range(n_b + 2):
+            api.moe_layer_forward(layer.prob, xs[0], layer.weights, torch.empty_like(xs[0]), layer.routing,
+                                  layer.stats, layer.ws, stream)
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            layer.backward(xs[0], dy, 1.0, 0.0)
+            b1.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                b_ms.append(b0.elapsed_time(b1))
+        if api.read_device_status(layer.ws):
+            raise RuntimeError("device status after the backward")
+        kept_b = int(layer.routing["seg_off"][-1].item())
+        bflops = 12.0 * cfg.d_model * cfg.d_ff * (kept_b + cfg.n_shared * T) + 4.0 * T * cfg.d_model * cfg.n_experts
+        bwd = {"ms": statistics.median(b_ms), "algorithmic_tflop": bflops / 1e12,
+               "tflops": bflops / (statistics.median(b_ms) * 1e-3) / 1e12,
+               "note": "moe_layer_backward after a forward of the same batch, median of 3; 12 d F FLOPs per "
+                       "expert row (dh, dx, dW13, dW2) + router 4 T d E; the recomputed gate/up projections "
+                       "are not counted"}
+        layer._bwd_ws = None
+        del dy
+
     kept = int(layer.routing["seg_off"][-1].item())
     up_bytes = up_gemm_bytes(cfg, layer.routing["kept"].tolist())
     flops = algorithmic_flops(cfg, kept)
@@ -423,6 +453,7 @@ def run_ours(args, cfg):
         "kept_pairs": kept, "dropped_pairs": cfg.T * cfg.top_k - kept,
         "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
         "dispatch_gbs": disp_gbs, "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
+        "backward": bwd,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -436,6 +467,7 @@ def main():
     ap.add_argument("--workload", default="mixtral", choices=list(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the (separately reported) backward timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps, always
     cfg = CONFIGS[args.workload]
