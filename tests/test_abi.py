@@ -183,3 +183,33 @@ def test_balance_update_rejects_bad_arguments(L, kw, why):
                               a["count_hist"], a["hist_len"], a["step"], a["c_base"], a["gamma"],
                               a["expert_capacity"], None)
     assert rc == -1, why
+
+
+def test_backward_rejects_bad_arguments_before_launching(L):
+    fake = 4096
+    prob = api.make_problem(64, 64, 8, 2, 128, capacity_factor=1.0)
+    P = ctypes.byref(prob)
+    n = ctypes.c_size_t(0)
+    assert L.moe_workspace_size(P, ctypes.byref(n)) == 0
+    fwd = n.value
+    assert L.moe_backward_workspace_size(P, ctypes.byref(n)) == 0 and n.value > 0
+    bwd = n.value
+    w = _lib.MoeWeights(fake, None, None, fake, fake, None, None, None)
+    good = _lib.MoeGrads(fake, fake, fake, None, None, fake, None, None)
+
+    def call(prob_=prob, x=fake, g=good, fws=fake, fbytes=fwd, dy=fake, ws=1 << 20, wbytes=bwd, d_loss=1.0):
+        return L.moe_layer_backward(ctypes.byref(prob_), x, ctypes.byref(w), None, fws, fbytes, dy, d_loss, 0.0,
+                                    ctypes.byref(g), ws, wbytes, None)
+
+    assert call(dy=None) == -1
+    assert call(x=fake + 4) == -1
+    assert call(d_loss=float("nan")) == -1
+    assert call(g=_lib.MoeGrads(fake, None, fake, None, None, None, None, None)) == -1   # dw13 required
+    assert call(g=_lib.MoeGrads(fake, fake, fake, fake, fake, None, None, None)) == -1   # shared grads, no shared
+    assert call(fbytes=fwd - 1) == -5
+    assert call(wbytes=bwd - 1) == -5
+    assert call(ws=(1 << 20) + 16) == -5
+    f32 = api.make_problem(64, 64, 8, 2, 128, dtype="f32")
+    assert call(prob_=f32) == -2
+    given = api.make_problem(64, 64, 8, 2, 128, flags=api.FLAG_LOGITS_GIVEN)
+    assert call(prob_=given) == -1   # dw_gate requested although the logits are given
