@@ -440,9 +440,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ============================================================================
 constexpr int kPairBM = 256;
 constexpr int kPairBN = 256;  // MMA N: both halves of B
-constexpr int kPairStages = 6;
-constexpr int kPairABytes = 128 * kBK * 2;
-constexpr int kPairBBytes = 128 * kBK * 2;  // this CTA's half of B
+// 128-deep stages (two 64-deep chunks, one TMA box per chunk and operand), 3
+// of them: half the barrier round trips of 64-deep stages for the same bytes
+// in flight; measured 6% faster on the up/gate GEMM than 6 stages of 64.
+constexpr int kPairKC = 2;
+constexpr int kPairStages = 3;
+constexpr int kPairChunk = 128 * kBK * 2;  // one 128-row, 64-deep chunk: 16 KB
+constexpr int kPairABytes = kPairKC * kPairChunk;
+constexpr int kPairBBytes = kPairKC * kPairChunk;  // this CTA's half of B
 constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
 
 // Swap-tile epilogues transpose through shared memory, 32 tokens at a time:
@@ -583,7 +588,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
   const int total_tiles = prefix[args.n_groups];
-  const int nkb_g = (args.K + kBK - 1) / kBK;
+  const int nkb_g = (args.K + kBK * kPairKC - 1) / (kBK * kPairKC);
   const int nkb = nkb_g * args.k_groups;  // no split-K on the pair path
 
   if (warp == 0) {
@@ -601,27 +606,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           const int kg = kb / nkb_g;
-          const int kk = (kb - kg * nkb_g) * kBK;
+          const int kk0 = (kb - kg * nkb_g) * kBK * kPairKC;
           const uint32_t bar = full_leader + static_cast<uint32_t>(stage * 8);
           // a swap tile's N token rows are split N/2 per CTA; the box (64 or
           // 128 rows) may load more, the MMA reads the first N/2
           const int half_n = ti.swap ? swap_n(ti.row_end - ti.row0) / 2 : 128;
           const bool small = half_n <= kSwapSmallRows;
           if (rank == 0)
-            mbar_arrive_expect_tx(&full[stage], 2 * (kPairBBytes + (small ? kSwapSmallRows * kBK * 2 : kPairABytes)));
+            mbar_arrive_expect_tx(&full[stage],
+                                  2 * kPairKC * (kPairChunk + (small ? kSwapSmallRows * kBK * 2 : kPairChunk)));
           const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
-          tma_load_2d_pair(sA + stage * kPairABytes, small ? &tmA64 : &tmA, bar, kg * args.K + kk, a_row);
-          uint8_t* b_dst = sB + stage * kPairBBytes;
-          if (EPI == EPI_SWIGLU && ti.swap) {
-            // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
-            const int f = ti.n0 + 64 * static_cast<int>(rank);
-            tma_load_3d_pair(b_dst, &tmB64, bar, kk, f, 2 * ti.g);
-            tma_load_3d_pair(b_dst + kPairBBytes / 2, &tmB64, bar, kk, f, 2 * ti.g + 1);
-          } else if (EPI == EPI_SWIGLU)
-            tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
-          else
-            tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank),
-                             ti.g * args.k_groups + kg);
+#pragma unroll
+          for (int c = 0; c < kPairKC; ++c) {
+            const int kk = kk0 + c * kBK;  // past K: the box reads zeros
+            tma_load_2d_pair(sA + stage * kPairABytes + c * kPairChunk, small ? &tmA64 : &tmA, bar,
+                             kg * args.K + kk, a_row);
+            uint8_t* b_dst = sB + stage * kPairBBytes + c * kPairChunk;
+            if (EPI == EPI_SWIGLU && ti.swap) {
+              // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
+              const int f = ti.n0 + 64 * static_cast<int>(rank);
+              tma_load_3d_pair(b_dst, &tmB64, bar, kk, f, 2 * ti.g);
+              tma_load_3d_pair(b_dst + kPairChunk / 2, &tmB64, bar, kk, f, 2 * ti.g + 1);
+            } else if (EPI == EPI_SWIGLU) {
+              tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
+            } else {
+              tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank),
+                               ti.g * args.k_groups + kg);
+            }
+          }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
           if (++stage == kPairStages) {
@@ -668,13 +680,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after_sync();
-          const uint64_t tdesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes));
-          const uint64_t wdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes));
-          const uint64_t adesc = ti.swap ? wdesc : tdesc;
-          const uint64_t bdesc = ti.swap ? tdesc : wdesc;
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int c = 0; c < kPairKC; ++c) {
+            const uint64_t tdesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes + c * kPairChunk));
+            const uint64_t wdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes + c * kPairChunk));
+            const uint64_t adesc = ti.swap ? wdesc : tdesc;
+            const uint64_t bdesc = ti.swap ? tdesc : wdesc;
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | c | k) != 0 ? 1u : 0u);
+          }
           umma_commit_pair_multicast(&empty[stage], 0x3);
           if (++stage == kPairStages) {
             stage = 0;
