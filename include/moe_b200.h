@@ -89,6 +89,10 @@ typedef enum moe_dtype { MOE_DTYPE_BF16 = 0, MOE_DTYPE_F32 = 1 } moe_dtype;
                                          argument of moe_dispatch_capacity) instead
                                          of the uniform ceil(C*T*K/E); the row
                                          bound moe_max_rows becomes T*K */
+#define MOE_FLAG_SAVE_GU 0x10u /* training (BF16): moe_layer_forward also keeps the
+                                  experts' gate and up projections in its
+                                  workspace (larger: moe_workspace_size), so that
+                                  moe_layer_backward does not recompute them */
 
 /* Device status bits (moe_read_device_status). */
 #define MOE_DEV_BAD_EXPERT 0x1     /* an expert index outside [0, E) was skipped */
@@ -350,8 +354,9 @@ int moe_backward_workspace_size(const moe_problem_t* p, size_t* bytes);
  * Computes in BF16 with FP32 accumulation, like the forward: intermediate
  * gradients (dO, dh -> dg/du, dx rows, the logit gradient fed to the tensor
  * cores) are rounded to BF16, weight gradients accumulate in FP32 in TMEM.
- * The gate and up projections are recomputed from the forward's expert
- * inputs.  FP32 problems return MOE_ERR_UNSUPPORTED. */
+ * The gate and up projections are read from fwd_ws when the forward ran with
+ * MOE_FLAG_SAVE_GU (same flags here), else recomputed from the forward's
+ * expert inputs.  FP32 problems return MOE_ERR_UNSUPPORTED. */
 int moe_layer_backward(const moe_problem_t* p, const void* x, const moe_weights_t* w,
                        const moe_routing_t* routing, const void* fwd_ws, size_t fwd_ws_bytes,
                        const void* dy, float d_loss, float d_zloss, const moe_grads_t* grads,

@@ -16,6 +16,7 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
                 -4: "MOE_ERR_DEVICE_CHECK", -5: "MOE_ERR_WORKSPACE"}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 FLAG_LOGITS_GIVEN, FLAG_BIAS_LOGIT, FLAG_EXTENDED_STATS, FLAG_EXPERT_CAPACITY = 0x1, 0x2, 0x4, 0x8
+FLAG_SAVE_GU = 0x10
 BIAS_UPDATE_SIGN, BIAS_UPDATE_PROPORTIONAL = 0, 1
 ABI_VERSION = 2
 EXTENDED_STATS = ("z_loss", "entropy_bits", "cv", "drop_rate", "n_below_half", "n_above_double")

@@ -13,6 +13,7 @@ import torch
 from . import _lib
 from ._lib import (BIAS_UPDATE_PROPORTIONAL, BIAS_UPDATE_SIGN, DTYPE_BF16, DTYPE_F32, EXTENDED_STATS, FFN_ROUTED,
                    FFN_SHARED, FLAG_BIAS_LOGIT, FLAG_EXPERT_CAPACITY, FLAG_EXTENDED_STATS, FLAG_LOGITS_GIVEN,
+                   FLAG_SAVE_GU,
                    MoeError, MoeGrads, MoeProblem, MoeRouting, MoeWeights)
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
@@ -20,7 +21,7 @@ __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity
            "moe_layer_forward_profiled", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
            "moe_layer_backward", "backward_workspace_size", "alloc_backward_workspace",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
-           "FLAG_EXTENDED_STATS", "FLAG_EXPERT_CAPACITY", "EXTENDED_STATS", "stats_size",
+           "FLAG_EXTENDED_STATS", "FLAG_EXPERT_CAPACITY", "FLAG_SAVE_GU", "EXTENDED_STATS", "stats_size",
            "BIAS_UPDATE_SIGN", "BIAS_UPDATE_PROPORTIONAL",
            "FFN_ROUTED", "FFN_SHARED", "DTYPE_BF16", "DTYPE_F32"]
 

@@ -211,10 +211,11 @@ static BwdLayout bwd_layout(const Problem& p) {
   B.dl = take(T * p.E * 4);
   B.dl16 = take(T * B.e_pad * 2);
   B.dout = take(R * p.d * 2);
-  B.gu = take(R * 2 * p.F * 2);
+  const bool saved = p.flags & MOE_FLAG_SAVE_GU;  // the forward kept g, u in its workspace
+  B.gu = take(saved ? 0 : R * 2 * p.F * 2);
   B.dgu = take(R * 2 * p.F * 2);
   B.dx_rows = take(R * p.d * 2);
-  B.gu_sh = take(T * 2 * p.F * p.Ns * 2);
+  B.gu_sh = take(saved ? 0 : T * 2 * p.F * p.Ns * 2);
   B.dgu_sh = take(T * 2 * p.F * p.Ns * 2);
   B.dx_sh = take(p.Ns > 0 ? T * p.d * 2 : 0);
   B.dx_r = take(T * p.d * 2);
@@ -269,6 +270,7 @@ int moe_layer_backward(const moe_problem_t* q, const void* x, const moe_weights_
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void* fws = const_cast<void*>(fwd_ws);
+  const bool saved = p.flags & MOE_FLAG_SAVE_GU;
   moe_routing_t r{};
   if (routing) r = *routing;
   const float* logits = r.logits ? r.logits : wsat<float>(fws, L.logits);
@@ -300,15 +302,16 @@ int moe_layer_backward(const moe_problem_t* q, const void* x, const moe_weights_
   // 2. routed experts
   if (p.max_rows > 0) {
     if (launch_expert_ffn_backward(p, 0, wsat<void>(fws, L.x_perm), p.max_rows, seg_off, w->w13, w->w2, dout,
-                                   wsat<void>(fws, L.h_routed), wsat<void>(ws, B.gu), wsat<void>(ws, B.dgu), dx_rows,
-                                   grads->dw13, grads->dw2, status, st))
+                                   wsat<void>(fws, L.h_routed), saved ? wsat<void>(fws, L.gu_routed) : wsat<void>(ws, B.gu),
+                                   wsat<void>(ws, B.dgu), dx_rows, grads->dw13, grads->dw2, status, st, saved))
       return MOE_ERR_CUDA;
   }
   // 3. shared experts: do = dy for every token
   if (p.Ns > 0) {
     if (launch_expert_ffn_backward(p, 1, x, p.T, nullptr, w->w13_shared, w->w2_shared, dy,
-                                   wsat<void>(fws, L.h_shared), wsat<void>(ws, B.gu_sh), wsat<void>(ws, B.dgu_sh),
-                                   dx_sh, grads->dw13_shared, grads->dw2_shared, status, st))
+                                   wsat<void>(fws, L.h_shared), saved ? wsat<void>(fws, L.gu_shared) : wsat<void>(ws, B.gu_sh),
+                                   wsat<void>(ws, B.dgu_sh), dx_sh, grads->dw13_shared, grads->dw2_shared, status, st,
+                                   saved))
       return MOE_ERR_CUDA;
   }
   // 4. through the gate GEMM

@@ -69,6 +69,12 @@ struct GemmArgs {
   // pair kernel: a group's last row tile with at most swap_max rows (0: never)
   // is computed operand-swapped (see grouped_gemm_pair_kernel)
   int swap_max;
+  // EPI_SWIGLU: when not null, the gate and up projections are also stored
+  // (BF16): row r, group g: g at gu + r*ld_gu + g*gu_col_stride + col, u at
+  // N columns further
+  void* gu;
+  int64_t ld_gu;
+  int gu_col_stride;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -196,7 +202,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
         for (int q = 0; q < 4; ++q) {
           const int col = n0 + c + q * 8;
           if (col < args.N) {
-            uint32_t pk[4];
+            uint32_t pk[4], gp[4], up[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const float g0 = __uint_as_float(gr[q * 8 + 2 * j]), g1 = __uint_as_float(gr[q * 8 + 2 * j + 1]);
@@ -204,8 +210,16 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
               const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
               const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
               pk[j] = pack_bf16x2(h0, h1);
+              gp[j] = pack_bf16x2(g0, g1);
+              up[j] = pack_bf16x2(u0, u1);
             }
             *reinterpret_cast<uint4*>(out_row + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (args.gu) {
+              __nv_bfloat16* gu_row = static_cast<__nv_bfloat16*>(args.gu) + static_cast<int64_t>(row) * args.ld_gu +
+                                      static_cast<int64_t>(g) * args.gu_col_stride;
+              *reinterpret_cast<uint4*>(gu_row + col) = make_uint4(gp[0], gp[1], gp[2], gp[3]);
+              *reinterpret_cast<uint4*>(gu_row + args.N + col) = make_uint4(up[0], up[1], up[2], up[3]);
+            }
           }
         }
       }
@@ -509,6 +523,17 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileIn
           }
           *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c + j) * args.ldo + f) =
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (args.gu) {
+            __nv_bfloat16* gu_row = static_cast<__nv_bfloat16*>(args.gu) +
+                                    static_cast<int64_t>(ti.row0 + c + j) * args.ld_gu +
+                                    static_cast<int64_t>(ti.g) * args.gu_col_stride;
+            *reinterpret_cast<uint4*>(gu_row + f) =
+                make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]),
+                           pack_bf16x2(g[6], g[7]));
+            *reinterpret_cast<uint4*>(gu_row + args.N + f) =
+                make_uint4(pack_bf16x2(u[0], u[1]), pack_bf16x2(u[2], u[3]), pack_bf16x2(u[4], u[5]),
+                           pack_bf16x2(u[6], u[7]));
+          }
         }
       }
     } else {
@@ -1069,7 +1094,7 @@ int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_
 // [n_rows, N_s * F] (shared).
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status, cudaStream_t st,
-                      cudaEvent_t after_up, int* n_kernels) {
+                      cudaEvent_t after_up, int* n_kernels, void* gu) {
   if (n_rows <= 0) return 0;
   if (p.dtype == kF32) {
     if (n_kernels) *n_kernels += 2;
@@ -1110,6 +1135,9 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     a.out_col_stride = routed ? 0 : p.F;
     a.status = status;
     a.swap_max = swap_max_rows();
+    a.gu = gu;  // kept for the backward (routed [rows, 2F]; shared [rows, N_s 2F])
+    a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
+    a.gu_col_stride = routed ? 0 : 2 * p.F;
     const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
     if (pair) {
       a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only

@@ -475,7 +475,7 @@ static int64_t gcdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, int64_t n_rows,
                                const int32_t* seg_off, const void* w13, const void* w2, const void* dout,
                                const void* h, void* gu, void* dgu, void* dx_rows, float* dw13, float* dw2,
-                               unsigned* status, cudaStream_t st) {
+                               unsigned* status, cudaStream_t st, bool gu_ready) {
   if (n_rows <= 0) return 0;
   const bool routed = mode == 0;
   const int G = routed ? p.E : p.Ns;
@@ -483,8 +483,8 @@ int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, i
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.F) * p.Ns;
   const int64_t row_tiles = routed ? gcdiv(n_rows, kGBM) + G : static_cast<int64_t>(G) * gcdiv(n_rows, kGBM);
 
-  // 1. g, u recomputed: GU = x W13^T (the forward's up projection without SwiGLU)
-  if (launch_up_projections(p, mode, x_rows, n_rows, seg_off, w13, gu, status, st)) return -3;
+  // 1. g, u: kept by the forward, or recomputed as GU = x W13^T (its up projection without SwiGLU)
+  if (!gu_ready && launch_up_projections(p, mode, x_rows, n_rows, seg_off, w13, gu, status, st)) return -3;
 
   // 2. dGU: dh = do W2 (B = W2 read MN-major), epilogue -> (dg | du)
   {

@@ -35,6 +35,7 @@ struct WsLayout {
   size_t chunk_counts, chunk_psum, chunk_base, logit_parts, zpart;
   size_t zero_bytes;  // status word + chunk histogram + chunk p sums: cleared together at offset 0
   size_t x_perm, h_routed, y_perm, h_shared, y_shared;
+  size_t gu_routed, gu_shared;  // with MOE_FLAG_SAVE_GU: the gate/up projections for the backward
   size_t total;
   int n_chunks, n_sel_blocks;
 };
@@ -91,16 +92,18 @@ int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, c
                           int n_splits, unsigned* status, cudaStream_t st);
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
-                      cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr);
+                      cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr,
+                      void* gu = nullptr);
 
 // expert_gemm.cu: gu = x W13^T (gate | up projections, BF16) for the backward
 int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                           const void* w13, void* gu, unsigned* status, cudaStream_t st);
 // grad_gemm.cu: backward of the expert FFNs (see there); returns a moe_status value
+// gu_ready: gu already holds the forward's gate/up projections (no recompute)
 int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, int64_t n_rows,
                                const int32_t* seg_off, const void* w13, const void* w2, const void* dout,
                                const void* h, void* gu, void* dgu, void* dx_rows, float* dw13, float* dw2,
-                               unsigned* status, cudaStream_t st);
+                               unsigned* status, cudaStream_t st, bool gu_ready);
 
 // grad_gemm.cu: router gradients through the gate GEMM from dl [T, e_pad] BF16
 int launch_router_dgrad(const Problem& p, const void* dl16, int e_pad, const void* w_gate, void* dx_r,

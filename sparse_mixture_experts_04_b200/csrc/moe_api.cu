@@ -76,6 +76,9 @@ WsLayout make_layout(const Problem& p) {
   L.y_perm = take(R * p.d * es);
   L.h_shared = take(static_cast<size_t>(p.T) * p.Ns * p.F * es);
   L.y_shared = take(p.Ns > 0 ? static_cast<size_t>(p.T) * p.d * es : 0);
+  const bool save_gu = (p.flags & MOE_FLAG_SAVE_GU) && p.dtype == kBF16;
+  L.gu_routed = take(save_gu ? R * 2 * p.F * es : 0);
+  L.gu_shared = take(save_gu ? static_cast<size_t>(p.T) * p.Ns * 2 * p.F * es : 0);
   L.total = off;
   return L;
 }
@@ -89,7 +92,8 @@ static int to_problem(const moe_problem_t* in, Problem* out) {
   if (q.T < 1 || q.d_model < 8 || q.d_ff < 8 || (q.d_model % 8) || (q.d_ff % 8)) return MOE_ERR_INVALID_ARG;
   if (q.n_experts < 1 || q.top_k < 1 || q.top_k > q.n_experts || q.n_shared < 0) return MOE_ERR_INVALID_ARG;
   if (q.dtype != MOE_DTYPE_BF16 && q.dtype != MOE_DTYPE_F32) return MOE_ERR_INVALID_ARG;
-  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT | MOE_FLAG_EXTENDED_STATS | MOE_FLAG_EXPERT_CAPACITY))
+  if (q.flags & ~(MOE_FLAG_LOGITS_GIVEN | MOE_FLAG_BIAS_LOGIT | MOE_FLAG_EXTENDED_STATS | MOE_FLAG_EXPERT_CAPACITY |
+                  MOE_FLAG_SAVE_GU))
     return MOE_ERR_INVALID_ARG;
   if (!(q.alpha == q.alpha) || !(q.capacity_factor == q.capacity_factor)) return MOE_ERR_INVALID_ARG;
   if (q.n_experts > kMaxExperts || q.top_k > kMaxTopK || q.n_shared > 256) return MOE_ERR_UNSUPPORTED;
@@ -417,16 +421,18 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   if (cudaError_t e = mark(MOE_EV_DISPATCHED)) return cuda_rc(e);
   if (p.max_rows > 0) {
     cudaEvent_t up_ev = (events && events[MOE_EV_UP]) ? static_cast<cudaEvent_t>(events[MOE_EV_UP]) : nullptr;
+    void* gu = (p.flags & MOE_FLAG_SAVE_GU) && p.dtype == kBF16 ? at<void>(ws, L.gu_routed) : nullptr;
     if (launch_expert_ffn(p, MOE_FFN_ROUTED, x_perm, p.max_rows, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed),
-                          y_perm, status, st, up_ev, &kernels))
+                          y_perm, status, st, up_ev, &kernels, gu))
       return MOE_ERR_CUDA;
   } else if (cudaError_t e = mark(MOE_EV_UP)) {
     return cuda_rc(e);
   }
   if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
   if (p.Ns > 0) {
+    void* gu = (p.flags & MOE_FLAG_SAVE_GU) && p.dtype == kBF16 ? at<void>(ws, L.gu_shared) : nullptr;
     if (launch_expert_ffn(p, MOE_FFN_SHARED, x, p.T, nullptr, w->w13_shared, w->w2_shared,
-                          at<void>(ws, L.h_shared), y_sh, status, st, nullptr, &kernels))
+                          at<void>(ws, L.h_shared), y_sh, status, st, nullptr, &kernels, gu))
       return MOE_ERR_CUDA;
   }
   if (cudaError_t e = mark(MOE_EV_SHARED)) return cuda_rc(e);

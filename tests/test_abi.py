@@ -72,7 +72,7 @@ def _ret(fn, *args):
 
 @pytest.mark.parametrize("field,value,code", [
     ("T", 0, -1), ("d_model", 12, -1), ("d_ff", 4, -1), ("n_experts", 0, -1), ("top_k", 0, -1),
-    ("top_k", 9, -1), ("n_shared", -1, -1), ("dtype", 7, -1), ("flags", 0x10, -1), ("flags", 0x20, -1),
+    ("top_k", 9, -1), ("n_shared", -1, -1), ("dtype", 7, -1), ("flags", 0x20, -1), ("flags", 0x40, -1),
     ("n_experts", 300, -2), ("top_k", 33, -2)])
 def test_invalid_problems_are_rejected(L, field, value, code):
     prob = api.make_problem(64, 64, 8, 2, 128)

@@ -46,9 +46,13 @@ def _inputs(name):
 
 
 @pytest.mark.parametrize("name", list(CASES))
-@pytest.mark.parametrize("d_loss,d_zloss", [(1.0, 0.0), (0.5, 2.0)])
-def test_layer_backward_matches_oracle(name, d_loss, d_zloss):
+@pytest.mark.parametrize("d_loss,d_zloss,save_gu", [(1.0, 0.0, False), (0.5, 2.0, False), (1.0, 0.5, True)])
+def test_layer_backward_matches_oracle(name, d_loss, d_zloss, save_gu):
+    """save_gu: the forward keeps the gate/up projections (MOE_FLAG_SAVE_GU)
+    instead of the backward recomputing them."""
     prob, inp, dy = _inputs(name)
+    if save_gu:
+        prob.flags |= api.FLAG_SAVE_GU
     T, d, E, K, F, Ns = prob.T, prob.d_model, prob.n_experts, prob.top_k, prob.d_ff, prob.n_shared
     w = {k: dev(inp.get(k)) for k in ("w_gate", "w13", "w2", "w13_shared", "w2_shared", "sel_bias", "logit_offset")}
     layer = MoeLayer(prob, w)
@@ -92,3 +96,18 @@ def test_layer_backward_is_deterministic():
     g2 = layer.backward(x, dev(dy), 1.0, 1.0)
     for k in g1:
         assert torch.equal(g1[k], g2[k]), k
+
+
+def test_saved_projections_give_the_same_gradients_as_recomputed():
+    prob, inp, dy = _inputs("drops_shared")
+    w = {k: dev(inp.get(k)) for k in ("w_gate", "w13", "w2", "w13_shared", "w2_shared", "sel_bias", "logit_offset")}
+    x = dev(inp["x"])
+    grads = []
+    for flags in (0, api.FLAG_SAVE_GU):
+        p2 = api.make_problem(prob.T, prob.d_model, prob.n_experts, prob.top_k, prob.d_ff, prob.n_shared,
+                              prob.capacity_factor, "bf16", prob.flags | flags, prob.alpha)
+        layer = MoeLayer(p2, w)
+        layer.forward(x)
+        grads.append({k: v.clone() for k, v in layer.backward(x, dev(dy), 1.0, 1.0).items()})
+    for k in grads[0]:
+        assert torch.equal(grads[0][k], grads[1][k]), k
