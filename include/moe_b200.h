@@ -384,6 +384,40 @@ int moe_layer_forward_profiled(const moe_problem_t* p, const void* x, const moe_
                                void* ws, size_t ws_bytes, moe_stream_t stream,
                                void* const* events, int32_t* n_kernels);
 
+/* Expert-parallel exchange plan.  "Scaling with experts", What you still pay
+ * for (experts partitioned over devices: a token travels to the device that
+ * holds its expert, the output travels back); Zen MoDE §7.2 Communication
+ * Overhead (all-to-all between the expert devices).
+ *
+ * HOST function: every pointer here is a HOST pointer; it enqueues nothing,
+ * needs no device and may be called from any thread.
+ *
+ * n_ranks G >= 1 devices, rank in [0, G); n_experts E with E % G == 0; rank q
+ * holds the global experts [q*E_l, (q+1)*E_l), E_l = E/G.  Each rank routes
+ * and dispatches its own T tokens with the full router (moe_route +
+ * moe_dispatch, the global E), so its kept rows for global expert e are
+ * x_perm[seg_off[e] .. seg_off[e+1]).
+ *   seg_off_all   [G, E+1] in: row s = rank s's seg_off (each starts at 0 and
+ *                 never decreases)
+ *   send          [E, 3] out: chunk e = {peer e / E_l, first row in this rank's
+ *                 x_perm (and, on the way back, y_perm), rows}
+ *   recv          [E_l * G, 3] out: chunk el*G + s = {peer s, first row in the
+ *                 local buffer, rows} for local expert el from source rank s
+ *   local_seg_off [E_l + 1] out: local expert el owns local rows
+ *                 [local_seg_off[el], local_seg_off[el+1]) -- sources in rank
+ *                 order inside each expert -- ready for moe_expert_ffn (ROUTED)
+ *                 with the rank's E_l expert weights
+ * Forward: send chunk e of x_perm to its peer, receive chunk (el, s) into the
+ * local buffer; back: send local chunk (el, s) of the expert outputs to s,
+ * receive chunk e into y_perm.  Between two ranks both sides list their chunks
+ * in ascending expert order, so point-to-point messages match in posting
+ * order.  Chunks with 0 rows may be skipped by both sides.
+ * Errors: MOE_ERR_INVALID_ARG for NULL pointers, G < 1, rank out of range,
+ * E % G != 0, offsets not starting at 0 or decreasing, more than INT32_MAX
+ * local rows. */
+int moe_ep_plan(int32_t n_ranks, int32_t rank, int32_t n_experts, const int32_t* seg_off_all,
+                int32_t* send, int32_t* recv, int32_t* local_seg_off);
+
 #ifdef __cplusplus
 }
 #endif

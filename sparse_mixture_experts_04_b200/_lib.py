@@ -28,7 +28,7 @@ EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_row
             "moe_reset_device_status", "moe_read_device_status", "moe_route", "moe_dispatch",
             "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
             "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update", "moe_backward_workspace_size",
-            "moe_layer_backward")
+            "moe_layer_backward", "moe_ep_plan")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_backward.argtypes = [PP, P, ctypes.POINTER(MoeWeights), ctypes.POINTER(MoeRouting), P, sz, P,
                                      ctypes.c_float, ctypes.c_float, ctypes.POINTER(MoeGrads), P, sz, P]
     L.moe_layer_backward.restype = ctypes.c_int
+    L.moe_ep_plan.argtypes = [i32, i32, i32, P, P, P, P]
+    L.moe_ep_plan.restype = ctypes.c_int
     if L.moe_abi_version() != ABI_VERSION:
         raise RuntimeError(f"{LIB_PATH} has ABI version {L.moe_abi_version()}, this binding expects {ABI_VERSION}: "
                            "rebuild it")

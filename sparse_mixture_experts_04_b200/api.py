@@ -19,7 +19,7 @@ from ._lib import (BIAS_UPDATE_PROPORTIONAL, BIAS_UPDATE_SIGN, DTYPE_BF16, DTYPE
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_profiled", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
-           "moe_layer_backward", "backward_workspace_size", "alloc_backward_workspace",
+           "moe_layer_backward", "backward_workspace_size", "alloc_backward_workspace", "moe_ep_plan",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
            "FLAG_EXTENDED_STATS", "FLAG_EXPERT_CAPACITY", "FLAG_SAVE_GU", "EXTENDED_STATS", "stats_size",
            "BIAS_UPDATE_SIGN", "BIAS_UPDATE_PROPORTIONAL",
@@ -198,3 +198,22 @@ def moe_layer_backward(prob, x, weights: dict, routing: dict | None, fwd_ws, dy,
                                        _p(dy), float(d_loss), float(d_zloss), ctypes.byref(g), _p(ws), ws.numel(),
                                        _stream(stream))
     _lib.check("moe_layer_backward", rc)
+
+
+def moe_ep_plan(n_ranks: int, rank: int, n_experts: int, seg_off_all) -> tuple:
+    """Expert-parallel exchange plan (host function, no device).  seg_off_all
+    [n_ranks, E+1] int32 (CPU) -> (send [E, 3], recv [E_l*n_ranks, 3],
+    local_seg_off [E_l+1]) int32 CPU tensors; see include/moe_b200.h."""
+    so = torch.as_tensor(seg_off_all, dtype=torch.int32).contiguous()
+    if so.device.type != "cpu":
+        raise ValueError("moe_ep_plan takes host (CPU) segment offsets")
+    G, E = int(n_ranks), int(n_experts)
+    El = E // G if G > 0 else 0
+    send = torch.empty((max(E, 1), 3), dtype=torch.int32)
+    recv = torch.empty((max(El * G, 1), 3), dtype=torch.int32)
+    local = torch.empty(El + 1, dtype=torch.int32)
+    if so.numel() != G * (E + 1):
+        raise ValueError(f"seg_off_all has {so.numel()} entries, expected {G}x{E + 1}")
+    rc = _lib.lib().moe_ep_plan(G, int(rank), E, so.data_ptr(), send.data_ptr(), recv.data_ptr(), local.data_ptr())
+    _lib.check("moe_ep_plan", rc)
+    return send[:E], recv[:El * G], local

@@ -1,0 +1,62 @@
+// Expert-parallel exchange plan (host code only; no device work).
+//
+// "Scaling with experts" (jeff-ong.com), What you still pay for: with the
+// experts partitioned over devices, a token travels to the device holding its
+// assigned expert and the expert's output travels back.  Zen MoDE §7.2
+// Communication Overhead (Distributed Training): that routing is an
+// all-to-all exchange between the expert devices.
+//
+// Rank q of G holds the global experts [q*E_l, (q+1)*E_l), E_l = E/G.  Every
+// rank routes and dispatches its own tokens exactly as a single device would
+// (so its capacity cut and statistics are its own batch's), which leaves the
+// kept rows of global expert e at x_perm[seg_off[e] .. seg_off[e+1]).  The plan
+// turns all ranks' segment offsets into
+//   - one send chunk per global expert (to the expert's owner), and
+//   - one receive chunk per (local expert, source rank), placed so that the
+//     local buffer is grouped by local expert, sources in rank order inside
+//     each expert: the grouped expert GEMM then runs on it unchanged.
+// The return trip is the same table read backwards.  Between one pair of
+// ranks, both sides list their chunks in ascending expert order, so
+// point-to-point messages between the pair match in posting order.
+
+#include <cstdint>
+
+#include "../../include/moe_b200.h"
+
+extern "C" int moe_ep_plan(int32_t n_ranks, int32_t rank, int32_t n_experts, const int32_t* seg_off_all,
+                           int32_t* send, int32_t* recv, int32_t* local_seg_off) {
+  if (n_ranks < 1 || n_experts < 1 || rank < 0 || rank >= n_ranks || n_experts % n_ranks != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!seg_off_all || !send || !recv || !local_seg_off) return MOE_ERR_INVALID_ARG;
+  const int G = n_ranks, E = n_experts, El = E / G;
+  // every rank's offsets must start at 0 and never decrease
+  for (int s = 0; s < G; ++s) {
+    const int32_t* so = seg_off_all + static_cast<int64_t>(s) * (E + 1);
+    if (so[0] != 0) return MOE_ERR_INVALID_ARG;
+    for (int e = 0; e < E; ++e)
+      if (so[e + 1] < so[e]) return MOE_ERR_INVALID_ARG;
+  }
+  const int32_t* mine = seg_off_all + static_cast<int64_t>(rank) * (E + 1);
+  for (int e = 0; e < E; ++e) {
+    send[3 * e + 0] = e / El;
+    send[3 * e + 1] = mine[e];
+    send[3 * e + 2] = mine[e + 1] - mine[e];
+  }
+  int64_t off = 0;
+  for (int el = 0; el < El; ++el) {
+    local_seg_off[el] = static_cast<int32_t>(off);
+    const int e = rank * El + el;
+    for (int s = 0; s < G; ++s) {
+      const int32_t* so = seg_off_all + static_cast<int64_t>(s) * (E + 1);
+      const int32_t rows = so[e + 1] - so[e];
+      int32_t* c = recv + 3 * (static_cast<int64_t>(el) * G + s);
+      c[0] = s;
+      c[1] = static_cast<int32_t>(off);
+      c[2] = rows;
+      off += rows;
+      if (off > INT32_MAX) return MOE_ERR_INVALID_ARG;
+    }
+  }
+  local_seg_off[El] = static_cast<int32_t>(off);
+  return MOE_OK;
+}

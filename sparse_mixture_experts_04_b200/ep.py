@@ -1,0 +1,246 @@
+"""Expert-parallel forward of the MoE layer: the experts are partitioned over
+G devices and each token's rows travel to the device holding its expert and
+back ("Scaling with experts", What you still pay for; Zen MoDE §7.2
+Communication Overhead (Distributed Training): an all-to-all between the
+expert devices).
+
+Rank q holds the global experts [q*E_l, (q+1)*E_l), E_l = E/G, plus a copy
+of the router and of the shared experts.  One forward on rank q:
+
+  1. moe_route + moe_dispatch on its own T tokens with the full router, so the
+     capacity cut and the statistics are exactly those of a single device on
+     that batch; the kept rows of global expert e sit in x_perm at
+     seg_off[e] .. seg_off[e+1];
+  2. all-gather of the G segment-offset vectors (E+1 int32 each) and
+     moe_ep_plan (host): which rows go where;
+  3. exchange: chunk e of x_perm goes to the owner of expert e; the chunks
+     received land grouped by local expert, sources in rank order;
+  4. moe_expert_ffn (ROUTED) with the local E_l experts on the received rows;
+  5. exchange back: each output chunk returns to its source's y_perm, in the
+     place its input came from;
+  6. shared experts (local) and moe_combine, as on one device.
+
+Every step of the layer runs in libmoe_b200.so; this module allocates
+buffers, computes nothing and moves rows with torch.distributed point-to-point
+operations (NCCL between GPUs, gloo between CPU processes), or with device
+copies for the chunks a rank keeps for itself.  `forward_emulated` runs the
+same schedule for G ranks held in one process (every exchange a copy).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import api
+
+
+class CudaExperts:
+    """One rank's device state and kernels (C ABI): router + dispatch over the
+    global E experts, the rank's E_l local experts, shared experts, combine.
+
+    weights: w_gate [E, d], optional logit_offset / sel_bias [E],
+    expert_capacity [E] (with FLAG_EXPERT_CAPACITY), w13 [E_l, 2F, d],
+    w2 [E_l, d, F] (this rank's experts: global expert rank*E_l + i is local
+    expert i), optional w13_shared / w2_shared."""
+
+    def __init__(self, prob: api.MoeProblem, weights: dict, n_ranks: int, rank: int, device="cuda"):
+        E, T, K, d, F = prob.n_experts, prob.T, prob.top_k, prob.d_model, prob.d_ff
+        if n_ranks < 1 or not 0 <= rank < n_ranks or E % n_ranks:
+            raise ValueError(f"{E} experts cannot be split over {n_ranks} ranks (rank {rank})")
+        if prob.flags & api.FLAG_SAVE_GU:
+            raise ValueError("FLAG_SAVE_GU belongs to the training layer; the expert-parallel path is forward only")
+        self.prob, self.weights = prob, weights
+        self.n_ranks, self.rank = n_ranks, rank
+        self.n_local = E // n_ranks
+        self.device = torch.device(device)
+        self.dtype = torch.bfloat16 if prob.dtype == api.DTYPE_BF16 else torch.float32
+        self.d_model = d
+        if tuple(weights["w13"].shape) != (self.n_local, 2 * F, d) or tuple(weights["w2"].shape) != (self.n_local, d, F):
+            raise ValueError(f"rank {rank} needs w13 [{self.n_local}, {2 * F}, {d}] and w2 [{self.n_local}, {d}, {F}]")
+        self.capacity_flag = bool(prob.flags & api.FLAG_EXPERT_CAPACITY)
+        if self.capacity_flag and weights.get("expert_capacity") is None:
+            raise ValueError("FLAG_EXPERT_CAPACITY needs weights['expert_capacity'] [E]")
+        # rows one source can send here: at most T*K, at most T per expert, at most the capacity
+        cap = api.capacity(prob)
+        per_src = min(T * K, self.n_local * T)
+        if cap >= 0 and not self.capacity_flag:
+            per_src = min(per_src, self.n_local * cap)
+        self.max_local_rows = max(n_ranks * per_src, 1)
+        # the local experts' problem: max_local_rows rows over E_l groups (top_k 1, no capacity)
+        self.prob_local = api.make_problem(self.max_local_rows, d, self.n_local, 1, F, 0, 0.0, prob.dtype, 0,
+                                           prob.alpha)
+        dev = self.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.ws = api.alloc_workspace(prob, dev)
+        self.ws_local = api.alloc_workspace(self.prob_local, dev)
+        mr = max(api.max_rows(prob), 1)
+        self.logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+        self.topk_idx = torch.empty((T, K), **i32)
+        self.topk_w = torch.empty((T, K), dtype=torch.float32, device=dev)
+        self.counts, self.kept = torch.empty(E, **i32), torch.empty(E, **i32)
+        self.seg_off = torch.empty(E + 1, **i32)
+        self.slot_of = torch.empty((T, K), **i32)
+        self.perm = torch.empty(mr, **i32)
+        self.x_perm = torch.empty((mr, d), dtype=self.dtype, device=dev)
+        self.y_perm = torch.empty((mr, d), dtype=self.dtype, device=dev)
+        self.x_loc = torch.empty((self.max_local_rows, d), dtype=self.dtype, device=dev)
+        self.y_loc = torch.empty((self.max_local_rows, d), dtype=self.dtype, device=dev)
+        self.stats = torch.empty(api.stats_size(prob), dtype=torch.float32, device=dev)
+        self.y_shared = torch.empty((T, d), dtype=self.dtype, device=dev) if prob.n_shared > 0 else None
+
+    def route_dispatch(self, x: torch.Tensor) -> torch.Tensor:
+        w, P = self.weights, self.prob
+        api.moe_route(P, x, w.get("w_gate"), w.get("logit_offset"), w.get("sel_bias"), self.logits, self.topk_idx,
+                      self.topk_w, self.stats, self.ws)
+        if self.capacity_flag:
+            api.moe_dispatch_capacity(P, self.topk_idx, w["expert_capacity"], x, self.counts, self.kept,
+                                      self.seg_off, self.slot_of, self.perm, self.x_perm, self.ws)
+        else:
+            api.moe_dispatch(P, self.topk_idx, x, self.counts, self.kept, self.seg_off, self.slot_of, self.perm,
+                             self.x_perm, self.ws)
+        return self.seg_off
+
+    def experts(self, n_rows: int, local_seg_off: torch.Tensor) -> None:
+        if n_rows > 0:
+            seg = local_seg_off.to(self.device, non_blocking=False)
+            api.moe_expert_ffn(self.prob_local, api.FFN_ROUTED, self.x_loc, n_rows, seg, self.weights["w13"],
+                               self.weights["w2"], self.y_loc, self.ws_local)
+
+    def finish(self, x: torch.Tensor, y: torch.Tensor) -> None:
+        w, P = self.weights, self.prob
+        if self.y_shared is not None:
+            api.moe_expert_ffn(P, api.FFN_SHARED, x, P.T, None, w["w13_shared"], w["w2_shared"], self.y_shared,
+                               self.ws)
+        api.moe_combine(P, self.y_perm, self.slot_of, self.topk_w, self.y_shared, y, self.ws)
+
+
+class EpRank:
+    """The expert-parallel schedule of one rank, in phases (route, plan,
+    exchange lists, experts, combine) so that a process-group driver and the
+    in-process emulation share it.  `kernels` holds the rank's buffers
+    (x_perm, y_perm, x_loc, y_loc, seg_off) and its compute (CudaExperts)."""
+
+    def __init__(self, kernels):
+        self.k = kernels
+        self.send = self.recv = self.local_seg_off = None
+
+    def route(self, x: torch.Tensor) -> torch.Tensor:
+        """Steps 1: routing and dispatch; returns this rank's seg_off [E+1]."""
+        return self.k.route_dispatch(x)
+
+    def plan(self, seg_off_all: torch.Tensor) -> None:
+        """Step 2: seg_off_all [G, E+1] int32 (host) of every rank."""
+        self.send, self.recv, self.local_seg_off = api.moe_ep_plan(self.k.n_ranks, self.k.rank,
+                                                                   self.k.prob.n_experts, seg_off_all)
+        n = int(self.local_seg_off[-1])
+        if n > self.k.x_loc.shape[0]:
+            raise RuntimeError(f"rank {self.k.rank} would receive {n} rows, more than its bound "
+                               f"{self.k.x_loc.shape[0]}")
+
+    def _chunks(self, table, buf):
+        return [(int(p), buf[int(o): int(o) + int(r)]) for p, o, r in table.tolist() if r > 0]
+
+    def forward_lists(self):
+        """Step 3: (sends, recvs) as lists of (peer, rows view)."""
+        return self._chunks(self.send, self.k.x_perm), self._chunks(self.recv, self.k.x_loc)
+
+    def experts(self) -> None:
+        """Step 4."""
+        self.k.experts(int(self.local_seg_off[-1]), self.local_seg_off)
+
+    def backward_lists(self):
+        """Step 5: the outputs go back the way the inputs came."""
+        return self._chunks(self.recv, self.k.y_loc), self._chunks(self.send, self.k.y_perm)
+
+    def finish(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
+        """Step 6: shared experts and the gate-weighted combine."""
+        if y is None:
+            y = torch.empty((self.k.prob.T, self.k.d_model), dtype=self.k.dtype, device=self.k.device)
+        self.k.finish(x, y)
+        return y
+
+
+def _exchange(sends, recvs, rank: int, group=None) -> None:
+    """Point-to-point exchange of row chunks; chunks a rank sends to itself are
+    copied locally.  Messages between two ranks match in posting order."""
+    import torch.distributed as dist
+
+    def glob(r):
+        return r if group is None else dist.get_global_rank(group, r)
+
+    self_out = [t for p, t in sends if p == rank]
+    self_in = [t for p, t in recvs if p == rank]
+    if len(self_out) != len(self_in):
+        raise RuntimeError(f"rank {rank}: {len(self_out)} chunks to itself but {len(self_in)} expected")
+    for a, b in zip(self_out, self_in):
+        if a.shape != b.shape:
+            raise RuntimeError(f"rank {rank}: self chunk of {a.shape[0]} rows into a slot of {b.shape[0]}")
+        b.copy_(a)
+    ops = [dist.P2POp(dist.isend, t, glob(p), group) for p, t in sends if p != rank]
+    ops += [dist.P2POp(dist.irecv, t, glob(p), group) for p, t in recvs if p != rank]
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+
+
+def forward(rank_state: EpRank, x: torch.Tensor, y: torch.Tensor | None = None, group=None) -> torch.Tensor:
+    """One expert-parallel forward on this process's rank (torch.distributed
+    initialised; NCCL for CUDA tensors).  Every rank of the group calls it
+    with its own batch x [T, d]; returns this rank's layer output [T, d]."""
+    import torch.distributed as dist
+    k = rank_state.k
+    G = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if G != k.n_ranks or rank != k.rank:
+        raise RuntimeError(f"process group rank {rank}/{G} but the experts were placed for {k.rank}/{k.n_ranks}")
+    seg = rank_state.route(x)
+    parts = [torch.empty_like(seg) for _ in range(G)]
+    dist.all_gather(parts, seg, group=group)
+    rank_state.plan(torch.stack(parts).cpu())
+    _exchange(*rank_state.forward_lists(), rank, group)
+    rank_state.experts()
+    _exchange(*rank_state.backward_lists(), rank, group)
+    return rank_state.finish(x, y)
+
+
+def _emulated_exchange(lists) -> None:
+    G = len(lists)
+    for s in range(G):
+        for r in range(G):
+            out = [t for p, t in lists[s][0] if p == r]
+            inn = [t for p, t in lists[r][1] if p == s]
+            if len(out) != len(inn):
+                raise RuntimeError(f"{len(out)} chunks {s}->{r} but {len(inn)} expected")
+            for a, b in zip(out, inn):
+                if a.shape != b.shape:
+                    raise RuntimeError(f"chunk {s}->{r} of {a.shape[0]} rows into a slot of {b.shape[0]}")
+                b.copy_(a)
+
+
+def forward_emulated(ranks: list, xs: list) -> list:
+    """The schedule of `forward` for G ranks held in one process (for example
+    G ranks' expert sets on one device): every exchange is a copy.  Returns
+    the G layer outputs."""
+    if len(ranks) != len(xs):
+        raise ValueError("one batch per rank")
+    segs = [rk.route(x) for rk, x in zip(ranks, xs)]
+    host = torch.stack([s.cpu() for s in segs])
+    for rk in ranks:
+        rk.plan(host)
+    _emulated_exchange([rk.forward_lists() for rk in ranks])
+    for rk in ranks:
+        rk.experts()
+    _emulated_exchange([rk.backward_lists() for rk in ranks])
+    return [rk.finish(x) for rk, x in zip(ranks, xs)]
+
+
+def split_weights(weights: dict, n_ranks: int, rank: int) -> dict:
+    """This rank's share of a full weight set: its E/G routed experts (views),
+    the router and the shared experts whole."""
+    E = weights["w13"].shape[0]
+    if E % n_ranks:
+        raise ValueError(f"{E} experts cannot be split over {n_ranks} ranks")
+    El = E // n_ranks
+    out = {k: v for k, v in weights.items() if k not in ("w13", "w2")}
+    out["w13"] = weights["w13"][rank * El:(rank + 1) * El].contiguous()
+    out["w2"] = weights["w2"][rank * El:(rank + 1) * El].contiguous()
+    return out
