@@ -8,6 +8,8 @@ Modules:
   api    -- the C entry points with torch tensors (moe_route, moe_dispatch,
             moe_expert_ffn, moe_combine, moe_layer_forward, ...)
   layer  -- MoeLayer: weights + workspace held on the device, forward()
+  ep     -- expert-parallel forward: experts split over ranks, rows exchanged
+            with torch.distributed point-to-point (moe_ep_plan plans it)
   synth  -- seeded synthetic inputs of the five workloads
   build  -- nvcc build of the library
 """
