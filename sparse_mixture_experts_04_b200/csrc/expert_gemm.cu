@@ -75,6 +75,10 @@ struct GemmArgs {
   void* gu;
   int64_t ld_gu;
   int gu_col_stride;
+  // pair kernel: 1 when the tensor maps address both 64-deep chunks of a
+  // stage with one box (K a multiple of 64): A maps (64, rows, K/64), B maps
+  // (64, rows, groups, K/64); 0: one 2-D / 3-D box per chunk
+  int merged_k;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -468,8 +472,11 @@ constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
 // xbuf[token][TMEM lane] (row stride 132 floats keeps 16-byte alignment).
 constexpr int kSwapXStride = 132;
 constexpr int kSwapXBytes = 32 * kSwapXStride * 4;
-// A swap tile with at most this many tokens per CTA loads them with a 64-row box.
-constexpr int kSwapSmallRows = 64;
+// A swap tile loads its tokens with the smallest box (16, 32, 64 or 128
+// rows) that holds its N/2 tokens per CTA.
+__device__ __forceinline__ int swap_box_rows(int half_n) {
+  return half_n <= 16 ? 16 : half_n <= 32 ? 32 : half_n <= 64 ? 64 : 128;
+}
 
 constexpr int pair_smem_bytes() {
   return kPairStages * kPairStageBytes + 256 + 4 * (kMaxGroups + 1) + kSwapXBytes + 1024;
@@ -559,6 +566,7 @@ template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmA64, const __grid_constant__ CUtensorMap tmB64,
+                             const __grid_constant__ CUtensorMap tmA32, const __grid_constant__ CUtensorMap tmA16,
                              const GemmArgs args) {
   constexpr int kOutCols = (EPI == EPI_SWIGLU) ? kPairBN / 2 : kPairBN;
   extern __shared__ uint8_t smem_raw[];
@@ -599,6 +607,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmA64);
+    prefetch_tensormap(&tmA32);
+    prefetch_tensormap(&tmA16);
     if (EPI == EPI_SWIGLU) prefetch_tensormap(&tmB64);
   }
   if (warp == 1) {
@@ -633,30 +643,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const int kg = kb / nkb_g;
           const int kk0 = (kb - kg * nkb_g) * kBK * kPairKC;
           const uint32_t bar = full_leader + static_cast<uint32_t>(stage * 8);
-          // a swap tile's N token rows are split N/2 per CTA; the box (64 or
-          // 128 rows) may load more, the MMA reads the first N/2
+          // a swap tile's N token rows are split N/2 per CTA; the box (16, 32,
+          // 64 or 128 rows) may load more, the MMA reads the first N/2
           const int half_n = ti.swap ? swap_n(ti.row_end - ti.row0) / 2 : 128;
-          const bool small = half_n <= kSwapSmallRows;
-          if (rank == 0)
-            mbar_arrive_expect_tx(&full[stage],
-                                  2 * kPairKC * (kPairChunk + (small ? kSwapSmallRows * kBK * 2 : kPairChunk)));
+          const int a_box = ti.swap ? swap_box_rows(half_n) : 128;
+          const CUtensorMap* a_map = a_box == 16 ? &tmA16 : a_box == 32 ? &tmA32 : a_box == 64 ? &tmA64 : &tmA;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kPairKC * (kPairChunk + a_box * kBK * 2));
           const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
-#pragma unroll
-          for (int c = 0; c < kPairKC; ++c) {
-            const int kk = kk0 + c * kBK;  // past K: the box reads zeros
-            tma_load_2d_pair(sA + stage * kPairABytes + c * kPairChunk, small ? &tmA64 : &tmA, bar,
-                             kg * args.K + kk, a_row);
-            uint8_t* b_dst = sB + stage * kPairBBytes + c * kPairChunk;
+          uint8_t* a_dst = sA + stage * kPairABytes;
+          uint8_t* b_dst = sB + stage * kPairBBytes;
+          if (args.merged_k) {
+            // one box per operand covers both 64-deep chunks (chunk c of the
+            // tokens at c * a_box rows, of the weights at c * kPairChunk);
+            // chunks past K read zeros
+            const int kc = (kg * args.K + kk0) / kBK;
+            tma_load_3d_pair(a_dst, a_map, bar, 0, a_row, kc);
             if (EPI == EPI_SWIGLU && ti.swap) {
               // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
-              const int f = ti.n0 + 64 * static_cast<int>(rank);
-              tma_load_3d_pair(b_dst, &tmB64, bar, kk, f, 2 * ti.g);
-              tma_load_3d_pair(b_dst + kPairChunk / 2, &tmB64, bar, kk, f, 2 * ti.g + 1);
+              tma_load_4d_pair(b_dst, &tmB64, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
             } else if (EPI == EPI_SWIGLU) {
-              tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
+              tma_load_4d_pair(b_dst, &tmB, bar, 0, ti.n0, 2 * ti.g + static_cast<int>(rank), kk0 / kBK);
             } else {
-              tma_load_3d_pair(b_dst, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank),
-                               ti.g * args.k_groups + kg);
+              tma_load_4d_pair(b_dst, &tmB, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * args.k_groups + kg,
+                               kk0 / kBK);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kPairKC; ++c) {
+              const int kk = kk0 + c * kBK;  // past K: the box reads zeros
+              tma_load_2d_pair(a_dst + c * a_box * kBK * 2, a_map, bar, kg * args.K + kk, a_row);
+              uint8_t* bc = b_dst + c * kPairChunk;
+              if (EPI == EPI_SWIGLU && ti.swap) {
+                const int f = ti.n0 + 64 * static_cast<int>(rank);
+                tma_load_3d_pair(bc, &tmB64, bar, kk, f, 2 * ti.g);
+                tma_load_3d_pair(bc + kPairChunk / 2, &tmB64, bar, kk, f, 2 * ti.g + 1);
+              } else if (EPI == EPI_SWIGLU) {
+                tma_load_3d_pair(bc, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
+              } else {
+                tma_load_3d_pair(bc, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank), ti.g * args.k_groups + kg);
+              }
             }
           }
           issued |= 1u << stage;
@@ -691,6 +716,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // normal tile: A = token rows (M = 256), B = weight rows (N = 256);
         // swap tile: A = weight rows (M = 256), B = the tile's N token rows
         const uint32_t idesc = idesc_bf16_f32(kPairBM, ti.swap ? swap_n(ti.row_end - ti.row0) : kPairBN);
+        // the token operand's chunks sit a_box rows apart (see the producer)
+        const int a_chunk = (ti.swap ? swap_box_rows(swap_n(ti.row_end - ti.row0) / 2) : 128) * kBK * 2;
         const int acc = it & 1;
         const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
@@ -707,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tc_fence_after_sync();
 #pragma unroll
           for (int c = 0; c < kPairKC; ++c) {
-            const uint64_t tdesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes + c * kPairChunk));
+            const uint64_t tdesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes + c * a_chunk));
             const uint64_t wdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes + c * kPairChunk));
             const uint64_t adesc = ti.swap ? wdesc : tdesc;
             const uint64_t bdesc = ti.swap ? tdesc : wdesc;
@@ -809,6 +836,72 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// BF16 tensor map with explicit byte strides for dims 1..rank-1 (dim 0
+// contiguous), 128-byte swizzle, zero fill out of bounds.  Used for the
+// chunk-merged views: (64, rows, K/64) with the chunk stride 128 bytes.
+static bool make_map_strided(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                             const uint64_t* strides, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rank < 2 || rank > 5) return false;
+  cuuint64_t gdim[5], gstr[4];
+  cuuint32_t bdim[5], estr[5] = {1, 1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    if (i > 0) gstr[i - 1] = strides[i - 1];
+  }
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gdim, gstr, bdim, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Token maps of the pair kernel: row boxes of 128, 64, 32 and 16 rows.
+// merged: one box spans both 64-deep chunks of a stage, (64, rows, cols/64)
+// with the chunk stride 128 bytes; else a 2-D (cols, rows) map per chunk.
+static bool make_token_maps(CUtensorMap* t128, CUtensorMap* t64, CUtensorMap* t32, CUtensorMap* t16,
+                            const void* base, int64_t cols, int64_t rows, bool merged) {
+  CUtensorMap* maps[4] = {t128, t64, t32, t16};
+  const uint32_t heights[4] = {128, 64, 32, 16};
+  for (int i = 0; i < 4; ++i) {
+    if (merged) {
+      const uint64_t d[3] = {static_cast<uint64_t>(kBK), static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / kBK)};
+      const uint64_t st[2] = {static_cast<uint64_t>(cols) * 2, static_cast<uint64_t>(kBK) * 2};
+      const uint32_t b[3] = {kBK, heights[i], static_cast<uint32_t>(kPairKC)};
+      if (!make_map_strided(maps[i], base, 3, d, st, b)) return false;
+    } else {
+      const uint64_t d[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+      const uint32_t b[2] = {kBK, heights[i]};
+      if (!make_map(maps[i], base, 2, d, b)) return false;
+    }
+  }
+  return true;
+}
+
+// Weight map of the pair kernel over w [groups, rows, K] (row-major):
+// merged (64, rows, groups, K/64) with box (64, box_rows, box_groups, 2);
+// else (K, rows, groups) with box (64, box_rows, 1).
+static bool make_weight_map(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t groups,
+                            uint32_t box_rows, uint32_t box_groups, bool merged) {
+  if (merged) {
+    const uint64_t d[4] = {static_cast<uint64_t>(kBK), static_cast<uint64_t>(rows), static_cast<uint64_t>(groups),
+                           static_cast<uint64_t>(K / kBK)};
+    const uint64_t st[3] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K * rows) * 2,
+                            static_cast<uint64_t>(kBK) * 2};
+    const uint32_t b[4] = {kBK, box_rows, box_groups, static_cast<uint32_t>(kPairKC)};
+    return make_map_strided(m, base, 4, d, st, b);
+  }
+  const uint64_t d[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows), static_cast<uint64_t>(groups)};
+  const uint32_t b[3] = {kBK, box_rows, 1};
+  return make_map(m, base, 3, d, b);
+}
+
+// Chunk-merged boxes need whole 64-wide chunks; MOE_B200_MERGED_K=0 turns them off.
+static bool merged_k_ok(int64_t K) {
+  const char* e = getenv("MOE_B200_MERGED_K");
+  if (e && !strcmp(e, "0")) return false;
+  return K % kBK == 0;
+}
+
 template <int EPI, int BN, int STAGES>
 static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int64_t tile_bound,
                     cudaStream_t st) {
@@ -836,7 +929,8 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
 
 template <int EPI>
 static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64, const CUtensorMap& tb64,
-                         const GemmArgs& a, int64_t tile_bound, cudaStream_t st) {
+                         const CUtensorMap& ta32, const CUtensorMap& ta16, const GemmArgs& a, int64_t tile_bound,
+                         cudaStream_t st) {
   constexpr int smem = pair_smem_bytes();
   static std::mutex mu;
   static int max_pairs[64] = {0};
@@ -866,7 +960,7 @@ static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
   if (tile_bound <= 0) return 0;
   if (pairs > tile_bound) pairs = static_cast<int>(tile_bound);
   return launch_k(grouped_gemm_pair_kernel<EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads), smem,
-                  st, ta, tb, ta64, tb64, a) == cudaSuccess ? 0 : -3;
+                  st, ta, tb, ta64, tb64, ta32, ta16, a) == cudaSuccess ? 0 : -3;
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -1118,11 +1212,18 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.F), static_cast<uint64_t>(2 * G)};
     const uint32_t bb[3] = {kBK, 128, 1};
-    const uint32_t bb64[3] = {kBK, 64, 1};  // swap tiles: 64 gate and 64 up rows per CTA
-    const uint32_t ba64[2] = {kBK, 64};     // swap tiles: up to 64 token rows per CTA
-    CUtensorMap ta64, tb64;
-    if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
-    if (pair && (!make_map(&ta64, x_rows, 2, da, ba64) || !make_map(&tb64, w13, 3, db, bb64))) return -3;
+    CUtensorMap ta64, tb64, ta32, ta16;
+    const bool merged = pair && merged_k_ok(p.d);
+    if (pair) {
+      // w13 [G, 2F, d] as (d, F, 2G): gate rows of group g at 2g, up rows at 2g+1;
+      // swap tiles take 64 gate and the same 64 up rows per CTA
+      if (!make_token_maps(&ta, &ta64, &ta32, &ta16, x_rows, p.d, n_rows, merged) ||
+          !make_weight_map(&tb, w13, p.d, p.F, 2 * G, 128, 1, merged) ||
+          !make_weight_map(&tb64, w13, p.d, p.F, 2 * G, 64, merged ? 2 : 1, merged))
+        return -3;
+    } else if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) {
+      return -3;
+    }
     GemmArgs a{};
     a.n_groups = G;
     a.seg_off = routed ? seg_off : nullptr;
@@ -1141,11 +1242,14 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
     if (pair) {
       a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
-      int rc = run_pair_gemm<EPI_SWIGLU>(ta, tb, ta64, tb64, a, (mt / 2 + G) * cdiv(p.F, 128), st);
+      a.merged_k = merged ? 1 : 0;
+      int rc = run_pair_gemm<EPI_SWIGLU>(ta, tb, ta64, tb64, ta32, ta16, a, (mt / 2 + G) * cdiv(p.F, 128), st);
       if (rc) return rc;
       if (tail) {
         a.row_mode = 2;  // the rest (under 256 rows per group) on single CTAs
         a.swap_max = 0;
+        a.merged_k = 0;
+        if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
         rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, 2 * G * cdiv(p.F, 128), st);
         if (rc) return rc;
       }
@@ -1161,11 +1265,13 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
     const uint32_t bb[3] = {kBK, 256, 1};
-    const uint32_t bb_half[3] = {kBK, 128, 1};  // a pair CTA stages half of the 256 B rows
-    const uint32_t ba64[2] = {kBK, 64};
-    CUtensorMap tb_half, ta64;
+    CUtensorMap tb_half, ta64, ta32, ta16;
+    const bool merged = pair && merged_k_ok(p.F);
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
-    if (pair && (!make_map(&tb_half, w2, 3, db, bb_half) || !make_map(&ta64, h, 2, da, ba64))) return -3;
+    // w2 [G, d, F] as (F, d, G); a pair CTA stages half of the 256 B rows
+    if (pair && (!make_token_maps(&ta, &ta64, &ta32, &ta16, h, h_cols, n_rows, merged) ||
+                 !make_weight_map(&tb_half, w2, p.F, p.d, routed ? G : p.Ns, 128, 1, merged)))
+      return -3;
     GemmArgs a{};
     a.n_groups = routed ? G : 1;
     a.seg_off = routed ? seg_off : nullptr;
@@ -1181,11 +1287,15 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
     if (pair) {
       a.row_mode = tail ? 1 : 0;
-      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, ta64, tb_half, a, (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
+      a.merged_k = merged ? 1 : 0;
+      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, ta64, tb_half, ta32, ta16, a,
+                                       (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
       if (rc) return rc;
       if (tail) {
         a.row_mode = 2;
         a.swap_max = 0;
+        a.merged_k = 0;
+        if (!make_map(&ta, h, 2, da, ba)) return -3;
         rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.d, 256), st);
         if (rc) return rc;
       }
