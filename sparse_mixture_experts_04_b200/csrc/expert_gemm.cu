@@ -609,7 +609,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     prefetch_tensormap(&tmA64);
     prefetch_tensormap(&tmA32);
     prefetch_tensormap(&tmA16);
-    if (EPI == EPI_SWIGLU) prefetch_tensormap(&tmB64);
+    prefetch_tensormap(&tmB64);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -652,26 +652,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
           uint8_t* a_dst = sA + stage * kPairABytes;
           uint8_t* b_dst = sB + stage * kPairBBytes;
-          if (args.merged_k) {
-            // one box per operand covers both 64-deep chunks (chunk c of the
-            // tokens at c * a_box rows, of the weights at c * kPairChunk);
-            // chunks past K read zeros
-            const int kc = (kg * args.K + kk0) / kBK;
-            tma_load_3d_pair(a_dst, a_map, bar, 0, a_row, kc);
-            if (EPI == EPI_SWIGLU && ti.swap) {
-              // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
+          // Swap tiles are bound by the copies, not the MMAs: with merged maps
+          // (args.merged_k) each of their operands comes in one box spanning
+          // both 64-deep chunks (the tokens' chunk c at c * a_box rows, the
+          // weights' at c * kPairChunk; chunks past K read zeros).  Full tiles
+          // keep one box per chunk, which measured slightly faster for them.
+          const bool merge = args.merged_k && ti.swap;
+          if (merge && a_box <= 64) {
+            tma_load_3d_pair(a_dst, a_map, bar, 0, a_row, (kg * args.K + kk0) / kBK);
+          } else {
+#pragma unroll
+            for (int c = 0; c < kPairKC; ++c)  // past K: the box reads zeros
+              tma_load_2d_pair(a_dst + c * a_box * kBK * 2, a_box == 128 ? &tmA : a_map, bar,
+                               kg * args.K + kk0 + c * kBK, a_row);
+          }
+          if (merge) {
+            if (EPI == EPI_SWIGLU)  // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
               tma_load_4d_pair(b_dst, &tmB64, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
-            } else if (EPI == EPI_SWIGLU) {
-              tma_load_4d_pair(b_dst, &tmB, bar, 0, ti.n0, 2 * ti.g + static_cast<int>(rank), kk0 / kBK);
-            } else {
-              tma_load_4d_pair(b_dst, &tmB, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * args.k_groups + kg,
+            else
+              tma_load_4d_pair(b_dst, &tmB64, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * args.k_groups + kg,
                                kk0 / kBK);
-            }
           } else {
 #pragma unroll
             for (int c = 0; c < kPairKC; ++c) {
-              const int kk = kk0 + c * kBK;  // past K: the box reads zeros
-              tma_load_2d_pair(a_dst + c * a_box * kBK * 2, a_map, bar, kg * args.K + kk, a_row);
+              const int kk = kk0 + c * kBK;
               uint8_t* bc = b_dst + c * kPairChunk;
               if (EPI == EPI_SWIGLU && ti.swap) {
                 const int f = ti.n0 + 64 * static_cast<int>(rank);
@@ -855,23 +859,26 @@ static bool make_map_strided(CUtensorMap* m, const void* base, int rank, const u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Token maps of the pair kernel: row boxes of 128, 64, 32 and 16 rows.
-// merged: one box spans both 64-deep chunks of a stage, (64, rows, cols/64)
-// with the chunk stride 128 bytes; else a 2-D (cols, rows) map per chunk.
+// Token maps of the pair kernel: a 2-D (cols, rows) map with 128-row boxes,
+// and swap-tile maps with 64-, 32- and 16-row boxes: 2-D as well, or with
+// merged chunks one box spanning both 64-deep chunks of a stage,
+// (64, rows, cols/64) with the chunk stride 128 bytes.
 static bool make_token_maps(CUtensorMap* t128, CUtensorMap* t64, CUtensorMap* t32, CUtensorMap* t16,
                             const void* base, int64_t cols, int64_t rows, bool merged) {
-  CUtensorMap* maps[4] = {t128, t64, t32, t16};
-  const uint32_t heights[4] = {128, 64, 32, 16};
-  for (int i = 0; i < 4; ++i) {
+  const uint64_t d2[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint32_t b128[2] = {kBK, 128};
+  if (!make_map(t128, base, 2, d2, b128)) return false;
+  CUtensorMap* maps[3] = {t64, t32, t16};
+  const uint32_t heights[3] = {64, 32, 16};
+  for (int i = 0; i < 3; ++i) {
     if (merged) {
       const uint64_t d[3] = {static_cast<uint64_t>(kBK), static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / kBK)};
       const uint64_t st[2] = {static_cast<uint64_t>(cols) * 2, static_cast<uint64_t>(kBK) * 2};
       const uint32_t b[3] = {kBK, heights[i], static_cast<uint32_t>(kPairKC)};
       if (!make_map_strided(maps[i], base, 3, d, st, b)) return false;
     } else {
-      const uint64_t d[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
       const uint32_t b[2] = {kBK, heights[i]};
-      if (!make_map(maps[i], base, 2, d, b)) return false;
+      if (!make_map(maps[i], base, 2, d2, b)) return false;
     }
   }
   return true;
@@ -1218,7 +1225,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
       // w13 [G, 2F, d] as (d, F, 2G): gate rows of group g at 2g, up rows at 2g+1;
       // swap tiles take 64 gate and the same 64 up rows per CTA
       if (!make_token_maps(&ta, &ta64, &ta32, &ta16, x_rows, p.d, n_rows, merged) ||
-          !make_weight_map(&tb, w13, p.d, p.F, 2 * G, 128, 1, merged) ||
+          !make_weight_map(&tb, w13, p.d, p.F, 2 * G, 128, 1, false) ||
           !make_weight_map(&tb64, w13, p.d, p.F, 2 * G, 64, merged ? 2 : 1, merged))
         return -3;
     } else if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) {
@@ -1265,12 +1272,14 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
     const uint32_t bb[3] = {kBK, 256, 1};
-    CUtensorMap tb_half, ta64, ta32, ta16;
+    CUtensorMap tb_half, tb_swap, ta64, ta32, ta16;
     const bool merged = pair && merged_k_ok(p.F);
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
     // w2 [G, d, F] as (F, d, G); a pair CTA stages half of the 256 B rows
+    const int64_t wg = routed ? G : p.Ns;
     if (pair && (!make_token_maps(&ta, &ta64, &ta32, &ta16, h, h_cols, n_rows, merged) ||
-                 !make_weight_map(&tb_half, w2, p.F, p.d, routed ? G : p.Ns, 128, 1, merged)))
+                 !make_weight_map(&tb_half, w2, p.F, p.d, wg, 128, 1, false) ||
+                 !make_weight_map(&tb_swap, w2, p.F, p.d, wg, 128, 1, merged)))
       return -3;
     GemmArgs a{};
     a.n_groups = routed ? G : 1;
@@ -1288,7 +1297,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     if (pair) {
       a.row_mode = tail ? 1 : 0;
       a.merged_k = merged ? 1 : 0;
-      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, ta64, tb_half, ta32, ta16, a,
+      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, ta64, tb_swap, ta32, ta16, a,
                                        (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
       if (rc) return rc;
       if (tail) {
