@@ -13,6 +13,9 @@ namespace moe {
 // BF16 TMA tensor map (host): dims[0] innermost, 128-byte swizzle, box inner
 // extent 64 elements, zero fill out of bounds (expert_gemm.cu).
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box);
+// Same with explicit byte strides for dims 1..rank-1 (dim 0 contiguous).
+bool make_map_strided(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                      const uint32_t* box);
 
 // Status bits written into the first word of the caller's workspace.
 constexpr unsigned kDevBadExpert = 0x1u;
@@ -90,6 +93,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+      "[%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
 

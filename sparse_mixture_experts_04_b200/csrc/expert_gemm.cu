@@ -211,8 +211,8 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
             for (int j = 0; j < 4; ++j) {
               const float g0 = __uint_as_float(gr[q * 8 + 2 * j]), g1 = __uint_as_float(gr[q * 8 + 2 * j + 1]);
               const float u0 = __uint_as_float(ur[q * 8 + 2 * j]), u1 = __uint_as_float(ur[q * 8 + 2 * j + 1]);
-              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
               pk[j] = pack_bf16x2(h0, h1);
               gp[j] = pack_bf16x2(g0, g1);
               up[j] = pack_bf16x2(u0, u1);
@@ -524,8 +524,8 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileIn
           uint32_t pk[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float h0 = g[2 * q] / (1.0f + __expf(-g[2 * q])) * u[2 * q];
-            const float h1 = g[2 * q + 1] / (1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
+            const float h0 = __fdividef(g[2 * q], 1.0f + __expf(-g[2 * q])) * u[2 * q];
+            const float h1 = __fdividef(g[2 * q + 1], 1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
             pk[q] = pack_bf16x2(h0, h1);
           }
           *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c + j) * args.ldo + f) =
@@ -843,8 +843,8 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
 // BF16 tensor map with explicit byte strides for dims 1..rank-1 (dim 0
 // contiguous), 128-byte swizzle, zero fill out of bounds.  Used for the
 // chunk-merged views: (64, rows, K/64) with the chunk stride 128 bytes.
-static bool make_map_strided(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                             const uint64_t* strides, const uint32_t* box) {
+bool make_map_strided(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+                      const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn || rank < 2 || rank > 5) return false;
   cuuint64_t gdim[5], gstr[4];

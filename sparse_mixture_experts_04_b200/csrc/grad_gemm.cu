@@ -23,6 +23,8 @@
 //          memory before its MMAs, so rows of the next group add nothing.
 //          Stores the FP32 weight gradient (zeros for a group without rows).
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -72,6 +74,9 @@ struct GradArgs {
   int gu_group_cols;         // gu_col = group * gu_group_cols
   int F;
   unsigned* status;
+  // 1: the MN-major operand's 64-column chunks of a k-block come in one box
+  // (maps (64, K rows, columns/64[, matrices]), chunk stride 128 bytes)
+  int merged_a, merged_b;
 };
 
 // Token rows [base, base + return) of group g, clamped to [0, n_rows).
@@ -312,17 +317,29 @@ __global__ void __launch_bounds__(kGThreads, 1)
             const int kg = kb / nkb_g;
             const int kk = (kb - kg * nkb_g) * kGBK;
             tma_load_2d(a_dst, &tmA, &full[stage], kg * args.kdim + kk, t.row_base + t.m0);
+            if (args.merged_b) {  // the four 64-column chunks in one box; chunks past N read zeros
+              tma_load_4d(b_dst, &tmB, &full[stage], 0, kk, t.n0 / 64, t.g * args.k_groups + kg);
+            } else {
 #pragma unroll
-            for (int c = 0; c < kGBN / 64; ++c)
-              tma_load_3d(b_dst + c * kGChunk, &tmB, &full[stage], t.n0 + 64 * c, kk, t.g * args.k_groups + kg);
+              for (int c = 0; c < kGBN / 64; ++c)
+                tma_load_3d(b_dst + c * kGChunk, &tmB, &full[stage], t.n0 + 64 * c, kk, t.g * args.k_groups + kg);
+            }
           } else {
             const int r0 = t.row_base + kb * kGBK;
+            if (args.merged_a) {
+              tma_load_3d(a_dst, &tmA, &full[stage], 0, r0, (t.g * args.a_col_group + t.m0) / 64);
+            } else {
 #pragma unroll
-            for (int c = 0; c < kGBM / 64; ++c)
-              tma_load_2d(a_dst + c * kGChunk, &tmA, &full[stage], t.g * args.a_col_group + t.m0 + 64 * c, r0);
+              for (int c = 0; c < kGBM / 64; ++c)
+                tma_load_2d(a_dst + c * kGChunk, &tmA, &full[stage], t.g * args.a_col_group + t.m0 + 64 * c, r0);
+            }
+            if (args.merged_b) {
+              tma_load_3d(b_dst, &tmB, &full[stage], 0, r0, (t.g * args.b_col_group + t.n0) / 64);
+            } else {
 #pragma unroll
-            for (int c = 0; c < kGBN / 64; ++c)
-              tma_load_2d(b_dst + c * kGChunk, &tmB, &full[stage], t.g * args.b_col_group + t.n0 + 64 * c, r0);
+              for (int c = 0; c < kGBN / 64; ++c)
+                tma_load_2d(b_dst + c * kGChunk, &tmB, &full[stage], t.g * args.b_col_group + t.n0 + 64 * c, r0);
+            }
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -465,6 +482,32 @@ static int run_grad(const CUtensorMap& ta, const CUtensorMap& tb, const GradArgs
 
 static int64_t gcdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// MN-major operand maps.  A matrix stack [mats, rows (the K index), cols]
+// read in 64-column chunks of 64 rows: chunked, one box holds `chunks`
+// consecutive chunks, (64, rows, cols/64, mats) with the chunk stride 128
+// bytes; else (cols, rows, mats) with 64 x 64 boxes.  Chunked needs cols a
+// multiple of 64 (MOE_B200_MERGED_K=0 turns it off).
+static bool mn_chunked_ok(int64_t cols) {
+  const char* e = getenv("MOE_B200_MERGED_K");
+  if (e && !strcmp(e, "0")) return false;
+  return cols % 64 == 0;
+}
+
+static bool make_mn_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t mats, int chunks,
+                        bool chunked, bool with_mats) {
+  const int rank = (chunked ? 3 : 2) + (with_mats ? 1 : 0);
+  if (chunked) {
+    const uint64_t d[4] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / 64),
+                           static_cast<uint64_t>(mats)};
+    const uint64_t st[3] = {static_cast<uint64_t>(cols) * 2, 128, static_cast<uint64_t>(cols * rows) * 2};
+    const uint32_t b[4] = {64, kGBK, static_cast<uint32_t>(chunks), 1};
+    return make_map_strided(m, base, rank, d, st, b);
+  }
+  const uint64_t d[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows), static_cast<uint64_t>(mats)};
+  const uint32_t b[3] = {64, kGBK, 1};
+  return make_map(m, base, rank, d, b);
+}
+
 // Backward of the expert FFNs, given do (the gradient at the experts' outputs,
 // per row: a routed row's token dy times its gate weight; for the shared
 // experts dy itself).  mode 0 routed (groups = experts over seg_off), 1 shared
@@ -491,10 +534,10 @@ int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, i
     CUtensorMap ta, tb;
     const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kGBK, kGBM};
-    const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
-    const uint32_t bb[3] = {64, kGBK, 1};
-    if (!make_map(&ta, dout, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
+    const bool mb = mn_chunked_ok(p.F);
+    if (!make_map(&ta, dout, 2, da, ba) || !make_mn_map(&tb, w2, p.F, p.d, G, kGBN / 64, mb, true)) return -3;
     GradArgs a{};
+    a.merged_b = mb;
     a.n_groups = G;
     a.seg_off = routed ? seg_off : nullptr;
     a.n_rows = static_cast<int>(n_rows);
@@ -516,10 +559,10 @@ int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, i
     CUtensorMap ta, tb;
     const uint64_t da[2] = {static_cast<uint64_t>(gu_cols), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kGBK, kGBM};
-    const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(2 * p.F), static_cast<uint64_t>(G)};
-    const uint32_t bb[3] = {64, kGBK, 1};
-    if (!make_map(&ta, dgu, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
+    const bool mb = mn_chunked_ok(p.d);
+    if (!make_map(&ta, dgu, 2, da, ba) || !make_mn_map(&tb, w13, p.d, 2 * p.F, G, kGBN / 64, mb, true)) return -3;
     GradArgs a{};
+    a.merged_b = mb;
     a.n_groups = routed ? G : 1;
     a.seg_off = routed ? seg_off : nullptr;
     a.n_rows = static_cast<int>(n_rows);
@@ -536,11 +579,13 @@ int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, i
   // 4. dW13[g] = dGU_g^T x (reduction over the group's rows)
   {
     CUtensorMap ta, tb;
-    const uint64_t da[2] = {static_cast<uint64_t>(gu_cols), static_cast<uint64_t>(n_rows)};
-    const uint64_t db[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
-    const uint32_t bx[2] = {64, kGBK};
-    if (!make_map(&ta, dgu, 2, da, bx) || !make_map(&tb, x_rows, 2, db, bx)) return -3;
+    const bool ma = mn_chunked_ok(gu_cols) && (2 * p.F) % 64 == 0, mb = mn_chunked_ok(p.d);
+    if (!make_mn_map(&ta, dgu, gu_cols, n_rows, 1, kGBM / 64, ma, false) ||
+        !make_mn_map(&tb, x_rows, p.d, n_rows, 1, kGBN / 64, mb, false))
+      return -3;
     GradArgs a{};
+    a.merged_a = ma;
+    a.merged_b = mb;
     a.n_groups = G;
     a.seg_off = routed ? seg_off : nullptr;
     a.n_rows = static_cast<int>(n_rows);
@@ -557,11 +602,13 @@ int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, i
   // 5. dW2[g] = do_g^T h_g
   {
     CUtensorMap ta, tb;
-    const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
-    const uint64_t db[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
-    const uint32_t bx[2] = {64, kGBK};
-    if (!make_map(&ta, dout, 2, da, bx) || !make_map(&tb, h, 2, db, bx)) return -3;
+    const bool ma = mn_chunked_ok(p.d), mb = mn_chunked_ok(h_cols) && p.F % 64 == 0;
+    if (!make_mn_map(&ta, dout, p.d, n_rows, 1, kGBM / 64, ma, false) ||
+        !make_mn_map(&tb, h, h_cols, n_rows, 1, kGBN / 64, mb, false))
+      return -3;
     GradArgs a{};
+    a.merged_a = ma;
+    a.merged_b = mb;
     a.n_groups = G;
     a.seg_off = routed ? seg_off : nullptr;
     a.n_rows = static_cast<int>(n_rows);
@@ -585,10 +632,10 @@ int launch_router_dgrad(const Problem& p, const void* dl16, int e_pad, const voi
   CUtensorMap ta, tb;
   const uint64_t da[2] = {static_cast<uint64_t>(e_pad), static_cast<uint64_t>(p.T)};
   const uint32_t ba[2] = {kGBK, kGBM};
-  const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.E), 1};
-  const uint32_t bb[3] = {64, kGBK, 1};
-  if (!make_map(&ta, dl16, 2, da, ba) || !make_map(&tb, w_gate, 3, db, bb)) return -3;
+  const bool mb = mn_chunked_ok(p.d);
+  if (!make_map(&ta, dl16, 2, da, ba) || !make_mn_map(&tb, w_gate, p.d, p.E, 1, kGBN / 64, mb, true)) return -3;
   GradArgs a{};
+  a.merged_b = mb;
   a.n_groups = 1;
   a.n_rows = static_cast<int>(p.T);
   a.n_dim = p.d;
@@ -604,11 +651,13 @@ int launch_router_dgrad(const Problem& p, const void* dl16, int e_pad, const voi
 int launch_router_wgrad(const Problem& p, const void* dl16, int e_pad, const void* x, float* dwg, unsigned* status,
                         cudaStream_t st) {
   CUtensorMap ta, tb;
-  const uint64_t da[2] = {static_cast<uint64_t>(e_pad), static_cast<uint64_t>(p.T)};
-  const uint64_t db[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.T)};
-  const uint32_t bx[2] = {64, kGBK};
-  if (!make_map(&ta, dl16, 2, da, bx) || !make_map(&tb, x, 2, db, bx)) return -3;
+  const bool ma = mn_chunked_ok(e_pad), mb = mn_chunked_ok(p.d);
+  if (!make_mn_map(&ta, dl16, e_pad, p.T, 1, kGBM / 64, ma, false) ||
+      !make_mn_map(&tb, x, p.d, p.T, 1, kGBN / 64, mb, false))
+    return -3;
   GradArgs a{};
+  a.merged_a = ma;
+  a.merged_b = mb;
   a.n_groups = 1;
   a.n_rows = static_cast<int>(p.T);
   a.m_dim = p.E;
