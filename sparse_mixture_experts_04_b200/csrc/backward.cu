@@ -191,7 +191,7 @@ namespace moe {
 // Backward scratch layout (bytes, 256-aligned): status, dl [T,E] f32,
 // dl16 [T, e_pad] bf16, then per-row BF16 buffers.
 struct BwdLayout {
-  size_t status, dl, dl16, dout, gu, dgu, dx_rows, gu_sh, dgu_sh, dx_sh, dx_r, total;
+  size_t status, dl, dl16, dout, gu, dgu, dx_rows, gu_sh, dgu_sh, dx_sh, dx_r, tail_a, tail_b, total;
   int e_pad;
 };
 
@@ -219,6 +219,8 @@ static BwdLayout bwd_layout(const Problem& p) {
   B.dgu_sh = take(T * 2 * p.F * p.Ns * 2);
   B.dx_sh = take(p.Ns > 0 ? T * p.d * 2 : 0);
   B.dx_r = take(T * p.d * 2);
+  B.tail_a = take(wgrad_tail_bytes(p, B.e_pad));
+  B.tail_b = take(wgrad_tail_bytes(p, B.e_pad));
   B.total = off;
   return B;
 }
@@ -303,21 +305,24 @@ int moe_layer_backward(const moe_problem_t* q, const void* x, const moe_weights_
   if (p.max_rows > 0) {
     if (launch_expert_ffn_backward(p, 0, wsat<void>(fws, L.x_perm), p.max_rows, seg_off, w->w13, w->w2, dout,
                                    wsat<void>(fws, L.h_routed), saved ? wsat<void>(fws, L.gu_routed) : wsat<void>(ws, B.gu),
-                                   wsat<void>(ws, B.dgu), dx_rows, grads->dw13, grads->dw2, status, st, saved))
+                                   wsat<void>(ws, B.dgu), dx_rows, grads->dw13, grads->dw2, wsat<void>(ws, B.tail_a),
+                                   wsat<void>(ws, B.tail_b), status, st, saved))
       return MOE_ERR_CUDA;
   }
   // 3. shared experts: do = dy for every token
   if (p.Ns > 0) {
     if (launch_expert_ffn_backward(p, 1, x, p.T, nullptr, w->w13_shared, w->w2_shared, dy,
                                    wsat<void>(fws, L.h_shared), saved ? wsat<void>(fws, L.gu_shared) : wsat<void>(ws, B.gu_sh),
-                                   wsat<void>(ws, B.dgu_sh), dx_sh, grads->dw13_shared, grads->dw2_shared, status, st,
-                                   saved))
+                                   wsat<void>(ws, B.dgu_sh), dx_sh, grads->dw13_shared, grads->dw2_shared,
+                                   wsat<void>(ws, B.tail_a), wsat<void>(ws, B.tail_b), status, st, saved))
       return MOE_ERR_CUDA;
   }
   // 4. through the gate GEMM
   const bool router_dx = grads->dx && !given;
   if (router_dx && launch_router_dgrad(p, dl16, B.e_pad, w->w_gate, dx_r, status, st)) return MOE_ERR_CUDA;
-  if (grads->dw_gate && launch_router_wgrad(p, dl16, B.e_pad, x, grads->dw_gate, status, st)) return MOE_ERR_CUDA;
+  if (grads->dw_gate && launch_router_wgrad(p, dl16, B.e_pad, x, grads->dw_gate, wsat<void>(ws, B.tail_a),
+                                            wsat<void>(ws, B.tail_b), status, st))
+    return MOE_ERR_CUDA;
   if (grads->d_offset) {
     if (launch_k(bwd_colsum_kernel, dim3(p.E), dim3(256), 0, st, static_cast<const float*>(dl), p.T, p.E,
                  grads->d_offset) != cudaSuccess)

@@ -100,16 +100,19 @@ int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_
                           const void* w13, void* gu, unsigned* status, cudaStream_t st);
 // grad_gemm.cu: backward of the expert FFNs (see there); returns a moe_status value
 // gu_ready: gu already holds the forward's gate/up projections (no recompute)
+// tail_a, tail_b: scratch of wgrad_tail_bytes each (the weight-gradient GEMMs'
+// zero-padded last k-blocks)
 int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, int64_t n_rows,
                                const int32_t* seg_off, const void* w13, const void* w2, const void* dout,
                                const void* h, void* gu, void* dgu, void* dx_rows, float* dw13, float* dw2,
-                               unsigned* status, cudaStream_t st, bool gu_ready);
+                               void* tail_a, void* tail_b, unsigned* status, cudaStream_t st, bool gu_ready);
+size_t wgrad_tail_bytes(const Problem& p, int e_pad);
 
 // grad_gemm.cu: router gradients through the gate GEMM from dl [T, e_pad] BF16
 int launch_router_dgrad(const Problem& p, const void* dl16, int e_pad, const void* w_gate, void* dx_r,
                         unsigned* status, cudaStream_t st);
-int launch_router_wgrad(const Problem& p, const void* dl16, int e_pad, const void* x, float* dwg, unsigned* status,
-                        cudaStream_t st);
+int launch_router_wgrad(const Problem& p, const void* dl16, int e_pad, const void* x, float* dwg, void* tail_a,
+                        void* tail_b, unsigned* status, cudaStream_t st);
 
 // combine.cu
 cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,

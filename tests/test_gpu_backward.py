@@ -26,6 +26,9 @@ CASES = {  # T, d, E, K, F, Ns, C, bias
     "fine_e64": (500, 192, 64, 6, 136, 1, 1.0, "logit"),
     "e7_ragged": (129, 264, 7, 3, 72, 1, 0.9, None),
     "single_expert": (64, 64, 1, 1, 64, 0, 0.0, None),
+    # groups of ~300 rows and d, F multiples of 64: the CTA-pair backward GEMMs
+    # (dgrad tiles of 256 rows, wgrad k-blocks of 128 rows with a tail)
+    "pairs_shared": (600, 256, 4, 2, 320, 1, 1.25, None),
 }
 
 
@@ -84,6 +87,26 @@ def test_layer_backward_matches_oracle(name, d_loss, d_zloss, save_gu):
     for e in range(E):
         if disp["kept"][e] == 0:
             assert not g["dw13"][e].any() and not g["dw2"][e].any()
+
+
+@pytest.mark.parametrize("name", ["pairs_shared", "mixtral_like"])
+def test_single_cta_and_pair_backward_gemms_agree(name, monkeypatch):
+    """The same backward with the CTA-pair GEMMs everywhere the shapes allow
+    (MOE_B200_GRAD_PAIR=all) and with the single-CTA ones (=0): both within the
+    oracle bar above; here they must agree to BF16 rounding of the stored
+    intermediates (dg/du, dx rows) and FP32 summation order (weights)."""
+    prob, inp, dy = _inputs(name)
+    w = {k: dev(inp.get(k)) for k in ("w_gate", "w13", "w2", "w13_shared", "w2_shared", "sel_bias", "logit_offset")}
+    x = dev(inp["x"])
+    out = []
+    for env in ("all", "0"):
+        monkeypatch.setenv("MOE_B200_GRAD_PAIR", env)
+        layer = MoeLayer(prob, w)
+        layer.forward(x)
+        out.append({k: v.float().clone() for k, v in layer.backward(x, dev(dy), 1.0, 0.5).items()})
+        assert api.read_device_status(layer.ws) == 0
+    for k in out[0]:
+        assert rel_err(out[0][k].cpu().numpy(), out[1][k].cpu().numpy().astype(np.float64)) <= 1e-2, k
 
 
 def test_layer_backward_is_deterministic():
