@@ -8,8 +8,8 @@
 //       dh = W_down^T do;  dg = dh u silu'(g);  du = dh silu(g)
 //       dx = W_gate^T dg + W_up^T du;  dW_down = do h^T;  dW_gate = dg x^T;  dW_up = du x^T
 //
-// Two shapes, one warp-specialised kernel (warp 0 TMA, warp 1 MMA, warps 2-5
-// epilogue; 128 x 256 tiles, 64-deep k-blocks, double-buffered TMEM):
+// Two shapes, one warp-specialised kernel (warp 0 TMA, warp 1 MMA, then 4 or 8
+// epilogue warps; 128 x 256 tiles, 64-deep k-blocks, double-buffered TMEM):
 //   dgrad  M = a group's token rows, N = output columns, K fixed:
 //          A = activations (token rows, K-major), B = the group's weights read
 //          MN-major (the weights are stored [out, in] for the forward, so the
@@ -43,7 +43,15 @@ constexpr int kGBM = 128;
 constexpr int kGBN = 256;
 constexpr int kGBK = 64;
 constexpr int kGStages = 4;
-constexpr int kGThreads = 192;
+// warp 0 TMA, warp 1 MMA, then the epilogue warps: 8 (two per TMEM lane
+// quarter, each taking half of the 256 accumulator columns) for the dSwiGLU
+// epilogue, whose loads and math set its pace; 4 for the others (8 measured
+// 16% slower on the FP32 weight gradients, 4% faster on the dSwiGLU dgrad)
+template <int EPI>
+constexpr int grad_epi_warps() { return EPI == GEPI_DSWIGLU ? 8 : 4; }
+template <int EPI>
+constexpr int grad_threads() { return 32 * (2 + grad_epi_warps<EPI>()); }
+constexpr int kGEpiWarpsMax = 8;
 constexpr int kGMaxGroups = 256;
 constexpr int kGABytes = kGBM * kGBK * 2;  // 16 KB
 constexpr int kGBBytes = kGBN * kGBK * 2;  // 32 KB: four 64-column MN chunks of 64 K rows
@@ -53,7 +61,7 @@ constexpr int kGChunk = 64 * kGBK * 2;  // one MN chunk (64 elements x 64 K rows
 // (17 KB), and a margin so that the operand descriptors of the last stage stay
 // inside the allocation whatever they address.
 constexpr int kGSlack = 32 * 1024;
-static_assert(4 * 32 * 33 * 4 <= kGSlack, "epilogue staging buffers do not fit");
+static_assert(kGEpiWarpsMax * 32 * 32 * 4 <= kGSlack, "epilogue staging buffers do not fit");
 
 constexpr int grad_smem_bytes() {
   return kGStages * kGStageBytes + kGSlack + 256 + 4 * (kGMaxGroups + 1) + 1024;
@@ -166,13 +174,15 @@ __device__ __forceinline__ int grad_nkb(const GradArgs& a, const GradTile& t) {
 }
 
 // Epilogue of one accumulator: this thread's TMEM lane r (0..127) holds row
-// m0 + r of the tile, 256 columns from t_lane.  Every lane calls it (the TMEM
-// loads are warp-collective); `zero` (wgrad, no rows in the group) stores
-// zeros without reading TMEM.  xw: this warp's 32 x 33 float staging buffer in
-// shared memory (FP32 weight gradients are written row-coalesced through it).
+// m0 + r of the tile, 256 columns from t_lane; this warp takes columns
+// [c_lo, c_hi).  Every lane calls it (the TMEM loads are warp-collective);
+// `zero` (wgrad, no rows in the group) stores zeros without reading TMEM.
+// xw: this warp's 32 x 32 float staging buffer in shared memory, element
+// (row, col) at row * 32 + (col ^ row) (conflict-free both ways); FP32 weight
+// gradients are written row-coalesced through it.
 template <int MODE, int EPI>
 __device__ __forceinline__ void grad_epilogue(const GradArgs& a, const GradTile& t, int r, uint32_t t_lane,
-                                              bool zero, float* xw) {
+                                              bool zero, float* xw, int c_lo, int c_hi) {
   const int lane = r & 31;
   if (EPI == GEPI_F32) {
     // each warp owns 32 rows; a 32 x 32 block goes lane-per-row into xw, then
@@ -181,14 +191,14 @@ __device__ __forceinline__ void grad_epilogue(const GradArgs& a, const GradTile&
     const int m_warp = t.m0 + (r & ~31);
     const int cq = (lane & 7) * 4;
 #pragma unroll 1
-    for (int c = 0; c < kGBN; c += 32) {
+    for (int c = c_lo; c < c_hi; c += 32) {
       uint32_t v[32];
       if (!zero) {
         tmem_load_32x32(t_lane + static_cast<uint32_t>(c), v);
         tmem_load_wait();
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) xw[lane * 33 + j] = zero ? 0.f : __uint_as_float(v[j]);
+      for (int j = 0; j < 32; ++j) xw[lane * 32 + (j ^ lane)] = zero ? 0.f : __uint_as_float(v[j]);
       __syncwarp();
       const int n = t.n0 + c + cq;
 #pragma unroll
@@ -196,9 +206,9 @@ __device__ __forceinline__ void grad_epilogue(const GradArgs& a, const GradTile&
         const int rr = i * 4 + (lane >> 3);
         const int m = m_warp + rr;
         if (m < a.m_dim && n < a.n_dim) {
-          const float* src = xw + rr * 33 + cq;
+          const float* row = xw + rr * 32;
           *reinterpret_cast<float4*>(obase + static_cast<int64_t>(m) * a.ldo + n) =
-              make_float4(src[0], src[1], src[2], src[3]);
+              make_float4(row[cq ^ rr], row[(cq + 1) ^ rr], row[(cq + 2) ^ rr], row[(cq + 3) ^ rr]);
         }
       }
       __syncwarp();
@@ -214,7 +224,7 @@ __device__ __forceinline__ void grad_epilogue(const GradArgs& a, const GradTile&
   if (EPI == GEPI_DSWIGLU)
     gurow = a.gu + static_cast<int64_t>(row_ok ? tok : 0) * a.ld_gu + static_cast<int64_t>(t.g) * a.gu_group_cols;
 #pragma unroll 1
-  for (int c = 0; c < kGBN; c += 32) {
+  for (int c = c_lo; c < c_hi; c += 32) {
     uint32_t v[32];
     uint4 gq[4], uq[4];
     if (EPI == GEPI_DSWIGLU) {
@@ -276,7 +286,7 @@ __device__ __forceinline__ void grad_epilogue(const GradArgs& a, const GradTile&
 // tmB: dgrad 3-D (N total, K, matrices) with 64 x 64 x 1 boxes (MN-major, four per k-block);
 //      wgrad 2-D (columns, rows) with 64 x 64 boxes (four per k-block).
 template <int MODE, int EPI>
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(grad_threads<EPI>(), 1)
     grad_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmAt, const __grid_constant__ CUtensorMap tmBt,
                      const GradArgs args) {
@@ -303,7 +313,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], grad_epi_warps<EPI>());
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -457,8 +467,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
       tc_fence_after_sync();
       const uint32_t t_lane =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kGBN);
+      constexpr int span = kGBN * 4 / grad_epi_warps<EPI>();  // columns per epilogue warp
+      const int part = (warp - 2) >> 2;
       grad_epilogue<MODE, EPI>(args, t, r, t_lane, grad_nkb<MODE, kGBK>(args, t) == 0,
-                               reinterpret_cast<float*>(smem + kGStages * kGStageBytes) + quarter * 32 * 33);
+                               reinterpret_cast<float*>(smem + kGStages * kGStageBytes) + (warp - 2) * 32 * 32,
+                               part * span, (part + 1) * span);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -498,7 +511,7 @@ constexpr int pgrad_smem_bytes() { return kPGStages * 2 * kPGHalf + kGSlack + 25
 static_assert(pgrad_smem_bytes() <= 232448, "exceeds the per-block shared-memory limit");
 
 template <int MODE, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(grad_threads<EPI>(), 1)
     grad_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmAt, const __grid_constant__ CUtensorMap tmBt,
                           const GradArgs args) {
@@ -528,7 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);
+      mbar_init(&tempty[a], 2 * grad_epi_warps<EPI>());
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -669,14 +682,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       const bool zero = grad_nkb<MODE, kPGBK>(args, t) == 0;
       const int acc = it & 1;
       const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
-      const bool ready = named_bar_and(2, 128, mbar_wait(&tfull[acc], acc_par, abort_flag));
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_par, abort_flag));
       if (!ready) break;
       tc_fence_after_sync();
       const uint32_t t_lane =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kGBN);
       t.m0 += 128 * static_cast<int>(rank);  // this CTA's accumulator rows
+      constexpr int span = kGBN * 4 / grad_epi_warps<EPI>();  // columns per epilogue warp
+      const int part = (warp - 2) >> 2;
       grad_epilogue<MODE, EPI>(args, t, r, t_lane, zero,
-                               reinterpret_cast<float*>(smem + kPGStages * 2 * kPGHalf) + quarter * 32 * 33);
+                               reinterpret_cast<float*>(smem + kPGStages * 2 * kPGHalf) + (warp - 2) * 32 * 32,
+                               part * span, (part + 1) * span);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>(acc * 8));
@@ -715,7 +731,8 @@ static int run_grad(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensor
   if (tile_bound <= 0) return 0;
   int64_t grid = num_sms();
   if (grid > tile_bound) grid = tile_bound;
-  return launch_k(grad_gemm_kernel<MODE, EPI>, dim3(static_cast<unsigned>(grid)), dim3(kGThreads), smem, st, ta, tb,
+  return launch_k(grad_gemm_kernel<MODE, EPI>, dim3(static_cast<unsigned>(grid)), dim3(grad_threads<EPI>()), smem, st,
+                  ta, tb,
                   tat, tbt, a) == cudaSuccess
              ? 0
              : -3;
@@ -768,7 +785,7 @@ static int run_grad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
       // a persistent grid must fit at once: ask how many 2-CTA clusters can be co-resident
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
-      cfg.blockDim = dim3(kGThreads, 1, 1);
+      cfg.blockDim = dim3(grad_threads<EPI>(), 1, 1);
       cfg.dynamicSmemBytes = smem;
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, grad_gemm_pair_kernel<MODE, EPI>, &cfg) != cudaSuccess || n <= 0) {
@@ -781,7 +798,8 @@ static int run_grad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
   }
   if (tile_bound <= 0) return 0;
   if (pairs > tile_bound) pairs = static_cast<int>(tile_bound);
-  return launch_k(grad_gemm_pair_kernel<MODE, EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGThreads), smem,
+  return launch_k(grad_gemm_pair_kernel<MODE, EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(grad_threads<EPI>()),
+                  smem,
                   st, ta, tb, tat, tbt, a) == cudaSuccess
              ? 0
              : -3;
