@@ -44,6 +44,7 @@ from sparse_mixture_experts_04_b200.synth import CONFIGS, extra_activations, gen
 
 METRIC = "MoE layer fwd tokens/s (BF16, 1 B200); expert GEMM % peak; dispatch GB/s"
 L2_BYTES = 126 * 1024 * 1024
+EP_RANKS = 8  # ranks of the emulated expert-parallel forward
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # oracle tokens per reference step / in the cpu_baseline sample (about 0.5-1 s each)
 REF_TOKENS = {"tiny_fp32": 256, "mixtral": 2, "zen_fine": 8, "skewed": 16, "decode": 2}
@@ -416,6 +417,41 @@ def run_ours(args, cfg):
                        "router 4 T d E"}
         del tlayer, dy
 
+    # the expert-parallel forward (experts split over EP_RANKS ranks), emulated on this one GPU:
+    # every rank's share of the experts and its own batch, every exchange a device copy
+    # (ep.forward_emulated); reported beside the metric, not part of it
+    epl = None
+    if world == 1 and cfg.dtype == "bf16" and not args.no_ep and cfg.n_experts % EP_RANKS == 0:
+        from sparse_mixture_experts_04_b200 import ep
+        G = EP_RANKS
+        ranks = [ep.EpRank(ep.CudaExperts(layer.prob, ep.split_weights(layer.weights, G, r), G, r)) for r in range(G)]
+        xb = [xs[r % n_x] for r in range(G)]
+        for _ in range(2):
+            ep.forward_emulated(ranks, xb)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_ep = 3
+        e0.record(stream)
+        for _ in range(n_ep):
+            ep.forward_emulated(ranks, xb)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ep_ms = e0.elapsed_time(e1) / n_ep
+        row_bytes = cfg.d_model * 2
+        # per rank and direction: its rows going out to other ranks plus the outputs it sends back
+        out_rows = [sum(n for p_, o_, n in rk.send.tolist() if p_ != rk.k.rank) +
+                    sum(n for p_, o_, n in rk.recv.tolist() if p_ != rk.k.rank) for rk in ranks]
+        xbytes = max(out_rows) * row_bytes
+        epl = {"ranks": G, "emulated_on_one_gpu": True, "ms_per_step_all_ranks": ep_ms,
+               "tokens_per_step": G * T, "tokens_per_s_on_one_gpu": G * T / (ep_ms * 1e-3),
+               "exchange_bytes_per_rank_per_direction_max": xbytes,
+               "modelled_exchange_ms_at_770GBps": xbytes / 770e9 * 1e3,
+               "note": f"{G} ranks' expert shares and batches run one after another on one GPU through "
+                       "ep.forward_emulated (route, dispatch, exchange as device copies, local experts, return, "
+                       "combine); includes a device-to-host copy of the segment offsets per step; the NVLink "
+                       "time is modelled from the bytes, not measured (one GPU per run)"}
+        del ranks
+
     kept = int(layer.routing["seg_off"][-1].item())
     up_bytes = up_gemm_bytes(cfg, layer.routing["kept"].tolist())
     flops = algorithmic_flops(cfg, kept)
@@ -460,6 +496,7 @@ def run_ours(args, cfg):
         "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
         "dispatch_gbs": disp_gbs, "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
         "backward": bwd,
+        "expert_parallel": epl,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -474,6 +511,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the (separately reported) backward timing")
+    ap.add_argument("--no-ep", action="store_true", help="skip the (separately reported) emulated expert-parallel timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps, always
     cfg = CONFIGS[args.workload]
