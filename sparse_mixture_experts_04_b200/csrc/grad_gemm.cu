@@ -808,20 +808,15 @@ static int run_grad_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
 // The pair kernel needs every operand chunk-merged (column counts multiples
 // of 64); dgrad also wants groups of at least 256 rows (else the 256-row tiles
 // are mostly padding).  Measured on the Mixtral shape (8 groups of ~1024 rows,
-// ncu per launch): wgrad dW13 2.01 -> 1.80 ms and dW2 0.90 -> 0.81 ms with
-// pairs, dX rows 1.52 -> 1.42 ms; the dSwiGLU dgrad 0.93 -> 0.98 ms (its
-// epilogue, not the operand stream, sets its pace, and 256-row tiles pad
-// more), so that one stays on single CTAs.  MOE_B200_GRAD_PAIR=0: single CTAs
-// everywhere; =all: pairs for the dSwiGLU dgrad too.
+// ncu per launch, single CTA -> pair): dW13 2.01 -> 1.74 ms, dW2 0.90 -> 0.80
+// ms, dX rows 1.52 -> 1.40 ms; whole backward with the dSwiGLU dgrad on pairs
+// too 2% faster (equal on the fine-grained and skewed workloads).
+// MOE_B200_GRAD_PAIR=0 keeps every backward GEMM on single CTAs.
 static bool grad_pair_ok() {
   const char* e = getenv("MOE_B200_GRAD_PAIR");
   if (e && !strcmp(e, "0")) return false;
   const char* m = getenv("MOE_B200_MERGED_K");
   return !(m && !strcmp(m, "0"));
-}
-static bool grad_pair_all() {
-  const char* e = getenv("MOE_B200_GRAD_PAIR");
-  return e && !strcmp(e, "all");
 }
 
 // K-major activation map of the pair dgrad: (64, rows, cols/64), box (64, 128, 2).
@@ -957,7 +952,7 @@ int launch_expert_ffn_backward(const Problem& p, int mode, const void* x_rows, i
   // 2. dGU: dh = do W2 (B = W2 read MN-major), epilogue -> (dg | du)
   {
     CUtensorMap ta, tb;
-    const bool pair = pair_rows && grad_pair_all() && p.d % 64 == 0 && p.F % 64 == 0;
+    const bool pair = pair_rows && p.d % 64 == 0 && p.F % 64 == 0;
     const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kGBK, kGBM};
     const bool mb = mn_chunked_ok(p.F);

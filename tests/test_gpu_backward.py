@@ -91,15 +91,15 @@ def test_layer_backward_matches_oracle(name, d_loss, d_zloss, save_gu):
 
 @pytest.mark.parametrize("name", ["pairs_shared", "mixtral_like"])
 def test_single_cta_and_pair_backward_gemms_agree(name, monkeypatch):
-    """The same backward with the CTA-pair GEMMs everywhere the shapes allow
-    (MOE_B200_GRAD_PAIR=all) and with the single-CTA ones (=0): both within the
+    """The same backward with the CTA-pair GEMMs (the default where the shapes
+    allow) and with the single-CTA ones (MOE_B200_GRAD_PAIR=0): both within the
     oracle bar above; here they must agree to BF16 rounding of the stored
     intermediates (dg/du, dx rows) and FP32 summation order (weights)."""
     prob, inp, dy = _inputs(name)
     w = {k: dev(inp.get(k)) for k in ("w_gate", "w13", "w2", "w13_shared", "w2_shared", "sel_bias", "logit_offset")}
     x = dev(inp["x"])
     out = []
-    for env in ("all", "0"):
+    for env in ("1", "0"):
         monkeypatch.setenv("MOE_B200_GRAD_PAIR", env)
         layer = MoeLayer(prob, w)
         layer.forward(x)
