@@ -18,7 +18,8 @@ of the router and of the shared experts.  One forward on rank q:
   4. moe_expert_ffn (ROUTED) with the local E_l experts on the received rows;
   5. exchange back: each output chunk returns to its source's y_perm, in the
      place its input came from;
-  6. shared experts (local) and moe_combine, as on one device.
+  6. shared experts (local; `forward` runs them while the rows of step 3 are
+     in flight) and moe_combine, as on one device.
 
 Every step of the layer runs in libmoe_b200.so; this module allocates
 buffers, computes nothing and moves rows with torch.distributed point-to-point
@@ -105,11 +106,15 @@ class CudaExperts:
             api.moe_expert_ffn(self.prob_local, api.FFN_ROUTED, self.x_loc, n_rows, seg, self.weights["w13"],
                                self.weights["w2"], self.y_loc, self.ws_local)
 
-    def finish(self, x: torch.Tensor, y: torch.Tensor) -> None:
+    def shared(self, x: torch.Tensor) -> None:
+        """The shared experts on this rank's batch (no routed rows needed)."""
         w, P = self.weights, self.prob
         if self.y_shared is not None:
             api.moe_expert_ffn(P, api.FFN_SHARED, x, P.T, None, w["w13_shared"], w["w2_shared"], self.y_shared,
                                self.ws)
+
+    def combine(self, y: torch.Tensor) -> None:
+        P = self.prob
         api.moe_combine(P, self.y_perm, self.slot_of, self.topk_w, self.y_shared, y, self.ws)
 
 
@@ -151,17 +156,28 @@ class EpRank:
         """Step 5: the outputs go back the way the inputs came."""
         return self._chunks(self.recv, self.k.y_loc), self._chunks(self.send, self.k.y_perm)
 
-    def finish(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
-        """Step 6: shared experts and the gate-weighted combine."""
+    def shared(self, x: torch.Tensor) -> None:
+        """Step 6a: the shared experts (independent of the exchange, so a
+        process-group forward runs them while the rows are in flight)."""
+        self.k.shared(x)
+
+    def combine(self, y: torch.Tensor | None = None) -> torch.Tensor:
+        """Step 6b: the gate-weighted combine."""
         if y is None:
             y = torch.empty((self.k.prob.T, self.k.d_model), dtype=self.k.dtype, device=self.k.device)
-        self.k.finish(x, y)
+        self.k.combine(y)
         return y
 
+    def finish(self, x: torch.Tensor, y: torch.Tensor | None = None) -> torch.Tensor:
+        """Step 6: shared experts and the gate-weighted combine."""
+        self.shared(x)
+        return self.combine(y)
 
-def _exchange(sends, recvs, rank: int, group=None) -> None:
+
+def _exchange(sends, recvs, rank: int, group=None, wait: bool = True):
     """Point-to-point exchange of row chunks; chunks a rank sends to itself are
-    copied locally.  Messages between two ranks match in posting order."""
+    copied locally.  Messages between two ranks match in posting order.  With
+    wait=False the requests are returned for the caller to wait on."""
     import torch.distributed as dist
 
     def glob(r):
@@ -177,9 +193,12 @@ def _exchange(sends, recvs, rank: int, group=None) -> None:
         b.copy_(a)
     ops = [dist.P2POp(dist.isend, t, glob(p), group) for p, t in sends if p != rank]
     ops += [dist.P2POp(dist.irecv, t, glob(p), group) for p, t in recvs if p != rank]
-    if ops:
-        for req in dist.batch_isend_irecv(ops):
+    reqs = dist.batch_isend_irecv(ops) if ops else []
+    if wait:
+        for req in reqs:
             req.wait()
+        return []
+    return reqs
 
 
 def forward(rank_state: EpRank, x: torch.Tensor, y: torch.Tensor | None = None, group=None) -> torch.Tensor:
@@ -196,10 +215,13 @@ def forward(rank_state: EpRank, x: torch.Tensor, y: torch.Tensor | None = None, 
     parts = [torch.empty_like(seg) for _ in range(G)]
     dist.all_gather(parts, seg, group=group)
     rank_state.plan(torch.stack(parts).cpu())
-    _exchange(*rank_state.forward_lists(), rank, group)
+    reqs = _exchange(*rank_state.forward_lists(), rank, group, wait=False)
+    rank_state.shared(x)  # overlaps the rows in flight
+    for req in reqs:
+        req.wait()
     rank_state.experts()
     _exchange(*rank_state.backward_lists(), rank, group)
-    return rank_state.finish(x, y)
+    return rank_state.combine(y)
 
 
 def _emulated_exchange(lists) -> None:

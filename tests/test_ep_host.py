@@ -142,15 +142,18 @@ class OracleExperts:
             for r in range(lso[el], lso[el + 1]):
                 self.y_loc[r] = torch.from_numpy(oracle.swiglu(self.x_loc[r].numpy(), self.w13[el], self.w2[el]))
 
-    def finish(self, x, y):
-        ysh = None
+    def shared(self, x):
+        self.ysh = None
         if self.cfg.n_shared:
             xs = x.numpy().astype(np.float64)
-            ysh = np.stack([sum(oracle.swiglu(xs[t], self.inp["w13_shared"][s].numpy(),
-                                              self.inp["w2_shared"][s].numpy()) for s in range(self.cfg.n_shared))
-                            for t in range(self.cfg.T)])
+            self.ysh = np.stack([sum(oracle.swiglu(xs[t], self.inp["w13_shared"][s].numpy(),
+                                                   self.inp["w2_shared"][s].numpy())
+                                     for s in range(self.cfg.n_shared)) for t in range(self.cfg.T)])
+
+    def combine(self, y):
         n = int(self.disp["seg_off"][-1])
-        y.copy_(torch.from_numpy(oracle.combine(self.y_perm[:max(n, 1)].numpy(), self.disp["slot_of"], self.w, ysh)))
+        y.copy_(torch.from_numpy(oracle.combine(self.y_perm[:max(n, 1)].numpy(), self.disp["slot_of"], self.w,
+                                                self.ysh)))
 
 
 def single_device_reference(cfg, inp, x):
