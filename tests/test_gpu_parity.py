@@ -217,15 +217,18 @@ def test_routed_expert_ffn_matches_oracle(name):
     assert rel_err(got[rows], want) <= tol(cfg)
 
 
+@pytest.mark.parametrize("F", [200, 320])
 @pytest.mark.parametrize("tile,swap", [("256all", ""), ("256all", "0"), ("256all", "100"), ("128", "")])
-def test_routed_ffn_every_remainder_shape(tile, swap, monkeypatch):
+def test_routed_ffn_every_remainder_shape(tile, swap, F, monkeypatch):
     """Groups whose last 256-row tile holds 1..256 rows (every swap-tile MMA
-    width class, ragged F across two column tiles), every row against the
-    oracle's SwiGLU of its expert."""
+    width class and token-box height, ragged F across two column tiles), every
+    row against the oracle's SwiGLU of its expert.  F = 320 (a multiple of 64)
+    takes the down projection's chunk-merged swap-tile boxes, F = 200 the
+    per-chunk ones (the up projection, d = 256, always merged)."""
     monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
     monkeypatch.setenv("MOE_B200_SWAP_MAX", swap)
     sizes = [1, 15, 16, 17, 31, 33, 100, 128, 129, 200, 255, 256, 257, 300, 513, 0, 48]
-    E, d, F = len(sizes), 256, 200
+    E, d = len(sizes), 256
     T = sum(sizes)
     prob = api.make_problem(T, d, E, 1, F, 0, 0.0, "bf16")
     ws = api.alloc_workspace(prob)
