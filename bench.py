@@ -410,8 +410,10 @@ def run_ours(args, cfg):
             raise RuntimeError("device status after the backward")
         kept_b = int(tlayer.routing["seg_off"][-1].item())
         bflops = 12.0 * cfg.d_model * cfg.d_ff * (kept_b + cfg.n_shared * T) + 4.0 * T * cfg.d_model * cfg.n_experts
+        b_tflops = bflops / (statistics.median(b_ms) * 1e-3) / 1e12
         bwd = {"ms": statistics.median(b_ms), "training_forward_ms": statistics.median(f_ms),
-               "algorithmic_tflop": bflops / 1e12, "tflops": bflops / (statistics.median(b_ms) * 1e-3) / 1e12,
+               "algorithmic_tflop": bflops / 1e12, "tflops": b_tflops,
+               "frac_of_bf16_peak": b_tflops / load_peaks()[0]["bf16_tflops"],
                "note": "moe_layer_backward after a MOE_FLAG_SAVE_GU forward of the same batch (which keeps the "
                        "gate/up projections), median of 3; 12 d F FLOPs per expert row (dh, dx, dW13, dW2) + "
                        "router 4 T d E"}
