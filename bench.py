@@ -381,6 +381,28 @@ def run_ours(args, cfg):
     d2h = ys_e[0].numel() * ys_e[0].element_size() + layer.stats.numel() * 4
     y = torch.empty(0)
 
+    # the same forward replayed from a CUDA graph (MoeLayer.capture): each step copies its
+    # batch into the graph's static input and replays; reported beside the metric
+    graph = None
+    if not args.no_graph:
+        layer.capture()
+        for i in range(args.warmup):
+            layer.forward_graphed(xs[i % n_x])
+        torch.cuda.synchronize()
+        barrier(world)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(args.steps):
+            layer.forward_graphed(xs[i % n_x])
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        g_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps, world)
+        graph = {"ms_per_step": g_ms, "tokens_per_s": world * T / (g_ms * 1e-3),
+                 "note": "one CUDA-graph replay of moe_layer_forward per step after a device copy of the "
+                         "step's batch into the graph's static input"}
+        layer._graph = None
+
     # training: the backward of a forward over the same batch (moe_layer_backward),
     # timed on its own (not part of the forward metric); BF16 problems only
     bwd = None
@@ -499,6 +521,7 @@ def run_ours(args, cfg):
         "dispatch_gbs": disp_gbs, "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
         "backward": bwd,
         "expert_parallel": epl,
+        "graph": graph,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -514,6 +537,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the (separately reported) backward timing")
     ap.add_argument("--no-ep", action="store_true", help="skip the (separately reported) emulated expert-parallel timing")
+    ap.add_argument("--no-graph", action="store_true", help="skip the (separately reported) CUDA-graph replay timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least 3 untimed warm-up steps, always
     cfg = CONFIGS[args.workload]

@@ -63,6 +63,35 @@ class MoeLayer:
 
     __call__ = forward
 
+    def capture(self, with_stats: bool = True) -> None:
+        """Capture one forward into a CUDA graph over static input/output
+        buffers (self.graph_x, self.graph_y); forward_graphed() replays it.  The
+        layer's launches (memset, kernels with programmatic dependent launch)
+        become one graph, so a replay costs one launch on the host.  One eager
+        forward runs first, outside the capture, to set the kernels' per-device
+        attributes."""
+        T, d = self.prob.T, self.prob.d_model
+        self.graph_x = torch.zeros((T, d), dtype=self.dtype, device=self.device)
+        self.graph_y = torch.empty((T, d), dtype=self.dtype, device=self.device)
+        self.forward(self.graph_x, self.graph_y, with_stats)
+        torch.cuda.synchronize(self.device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            api.moe_layer_forward(self.prob, self.graph_x, self.weights, self.graph_y, self.routing,
+                                  self.stats if with_stats else None, self.ws)
+        self._graph = g
+
+    def forward_graphed(self, x: torch.Tensor | None = None) -> torch.Tensor:
+        """Replay the captured forward (capture() first) on the current stream;
+        x (if given) is copied into the static input first.  Returns the static
+        output buffer, overwritten by the next replay."""
+        if getattr(self, "_graph", None) is None:
+            raise RuntimeError("MoeLayer.capture() has not been called")
+        if x is not None:
+            self.graph_x.copy_(x)
+        self._graph.replay()
+        return self.graph_y
+
     def backward(self, x: torch.Tensor, dy: torch.Tensor, d_loss: float = 1.0, d_zloss: float = 0.0,
                  stream=None) -> dict:
         """Gradients of the last forward (same x; the workspace untouched since),
