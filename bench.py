@@ -225,6 +225,21 @@ def dispatch_bytes(cfg, kept_pairs: int) -> float:
     return 4.0 * TK * 2 + 4.0 * TK + 4.0 * kept_pairs + 2.0 * kept_pairs * cfg.d_model * es
 
 
+def router_bytes(cfg) -> float:
+    """x read + W_g read + logits written + top-K indices and gates written."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    T, E, K, d = cfg.T, cfg.n_experts, cfg.top_k, cfg.d_model
+    return 1.0 * T * d * es + 1.0 * E * d * es + 4.0 * T * E + 8.0 * T * K
+
+
+def combine_bytes(cfg, kept_pairs: int) -> float:
+    """kept y_perm rows read + y_shared read (if any) + y written + slot_of and gates read."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    T, K, d = cfg.T, cfg.top_k, cfg.d_model
+    shared = 1.0 * T * d * es if cfg.n_shared > 0 else 0.0
+    return 1.0 * kept_pairs * d * es + shared + 1.0 * T * d * es + 8.0 * T * K
+
+
 # ------------------------------------------------------------------ oracle timing
 def oracle_tokens_per_s(cfg, inp, n_tokens: int, offset: int = 0):
     """The float64 oracle's full pipeline on n_tokens tokens of the workload
@@ -483,6 +498,8 @@ def run_ours(args, cfg):
     gemm_ms = stage["up"] + stage["down"]
     gemm_tflops = (flops["up"] + flops["down"]) / (gemm_ms * 1e-3) / 1e12
     disp_gbs = dispatch_bytes(cfg, kept) / (stage["dispatched"] * 1e-3) / 1e9
+    router_gbs = router_bytes(cfg) / (stage["routed"] * 1e-3) / 1e9
+    combine_gbs = combine_bytes(cfg, kept) / (stage["end"] * 1e-3) / 1e9
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -518,7 +535,12 @@ def run_ours(args, cfg):
         "stages_ms": stage, "stages_note": "separate pass with an event at every stage boundary",
         "kept_pairs": kept, "dropped_pairs": cfg.T * cfg.top_k - kept,
         "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
-        "dispatch_gbs": disp_gbs, "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
+        "dispatch_gbs": disp_gbs, "router_gbs": router_gbs, "combine_gbs": combine_gbs,
+        "hbm_frac": {"router": router_gbs / peaks["hbm_gbs"], "dispatch": disp_gbs / peaks["hbm_gbs"],
+                     "combine": combine_gbs / peaks["hbm_gbs"],
+                     "note": "algorithmic bytes / stage time (the bench's separate pass with an event at "
+                             "every stage boundary) / the measured HBM copy bandwidth"},
+        "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
         "backward": bwd,
         "expert_parallel": epl,
         "graph": graph,

@@ -38,3 +38,18 @@ def test_roofline_is_hbm_bound_when_weights_dominate():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(nbytes / 0.5e-3 / 1e9)
     assert r["peak"] == PEAKS["hbm_gbs"] and "fallback" in r["peak_source"]
+
+
+def test_router_and_combine_bytes_at_the_mixtral_shape():
+    """x (33.6 MB) dominates the router; the combine reads the 8192 kept rows
+    (67 MB) and writes y (33.5 MB): about 101 MB."""
+    cfg = CONFIGS["mixtral"]
+    T, d, E, K = cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k
+    assert bench.router_bytes(cfg) == 2 * T * d + 2 * E * d + 4 * T * E + 8 * T * K
+    assert 33.5e6 < bench.router_bytes(cfg) < 34.0e6
+    kept = T * K
+    assert bench.combine_bytes(cfg, kept) == 2 * kept * d + 2 * T * d + 8 * T * K
+    assert 100e6 < bench.combine_bytes(cfg, kept) < 101.5e6
+    # a shared expert adds its output rows to the combine's reads
+    z = CONFIGS["zen_fine"]
+    assert bench.combine_bytes(z, 0) == 2 * z.T * z.d_model * 2 + 8 * z.T * z.top_k
