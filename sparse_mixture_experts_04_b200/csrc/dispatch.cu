@@ -12,12 +12,16 @@
 // racing atomics.
 //
 // Kernels (all multi-pass, no CTA waits on another):
-//   1. hist  : per 256-token chunk, per-expert counts
-//   2. scan  : per expert, exclusive prefix over chunks; totals, kept, seg_off
-//   3. rank  : per chunk, each warp builds a lane mask per expert (which of its
-//              32 tokens chose it); rank = chunk base + earlier warps' counts +
-//              popcount of the lower lanes' bits
-//   4. gather: x_perm[slot] = x[perm[slot] / K]
+//   1. hist      : per 256-token chunk, per-expert counts (fused into the
+//                  selection kernel on the layer path)
+//   2. scan+rank : per chunk, the expert totals and the earlier chunks' counts
+//                  from the whole histogram, kept and seg_off; each warp builds
+//                  a lane mask per expert (which of its 32 tokens chose it);
+//                  rank = earlier chunks + earlier warps' counts + popcount of
+//                  the lower lanes' bits.  Large problems run it as two
+//                  kernels: scan (per expert, prefix over chunks, totals, kept,
+//                  seg_off) then rank.
+//   3. gather    : x_perm[slot] = x[perm[slot] / K]
 #include "common.cuh"
 #include "internal.h"
 
@@ -46,6 +50,7 @@ __global__ void __launch_bounds__(256) dispatch_hist_kernel(const int32_t* __res
     chunk_counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
 }
 
+// Large problems: scan (one block) then rank (one block per chunk).
 // One block of 1024 threads.  Thread (e, s) owns a contiguous run of chunks
 // for expert e; runs are summed, scanned per expert, then re-walked to write
 // each chunk's base.
@@ -209,6 +214,173 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
   }
 }
 
+// Fused scan+rank reads n_chunks^2 * E histogram words from L2 in all (every
+// block reads all of it); above this the separate scan is cheaper (measured
+// even at 256 chunks x 256 experts, 2^24 words).
+constexpr long long kFusedScanMaxReads = 1ll << 22;
+
+// Scan and rank in one kernel, one block per 256-token chunk (no block waits
+// on another): every block reads the whole [n_chunks, E] histogram (E x
+// n_chunks int32, a few KB, from L2) to get each expert's total and the count
+// in the chunks before its own, derives kept and seg_off itself, and ranks its
+// 256 tokens.  Block 0 also writes counts / kept / seg_off and, with stats !=
+// nullptr, finalises the balance statistics from the histogram and the chunk
+// probability sums (fixed point) that the selection kernel added: f_e, P_e,
+// the loss, and with zpart the z-loss and utilisation statistics.
+//   rank(t,k) = (tokens of earlier chunks for e) + (earlier warps of this
+//   chunk, by popcount of their lane masks) + popcount of the lower lanes
+__global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
+    const int32_t* __restrict__ idx, int64_t T, int K, int E, const int32_t* __restrict__ chunk_counts,
+    int n_chunks, long long cap, const int32_t* __restrict__ expert_cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ kept_out, int32_t* __restrict__ seg_off_out, int32_t* __restrict__ slot_of,
+    int32_t* __restrict__ perm, const unsigned long long* __restrict__ chunk_psum, float* __restrict__ stats,
+    float alpha, const float* __restrict__ zpart, int n_zpart) {
+  __shared__ int s_tot_part[256];
+  __shared__ int s_pre_part[256];
+  __shared__ int s_tot[kMaxExperts];
+  __shared__ int s_pre[kMaxExperts];
+  __shared__ int s_kept[kMaxExperts];
+  __shared__ int s_seg[kMaxExperts + 1];
+  __shared__ uint32_t mask[8][kMaxExperts];
+  __shared__ int wbase[8][kMaxExperts];
+  __shared__ double s_fp[kMaxExperts];
+  __shared__ double s_red[256];
+  pdl_wait();
+  pdl_trigger();
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int b = blockIdx.x;
+  // 1. per expert: total over all chunks and the count in chunks before b.
+  //    Thread (e, sl) sums a strided set of chunks; E <= 256 experts, S slices.
+  int S = 256 / E;
+  if (S > n_chunks) S = n_chunks;
+  if (S < 1) S = 1;
+  {
+    const int e = tid % E, sl = tid / E;
+    int tot = 0, pre = 0;
+    if (tid < E * S) {
+#pragma unroll 4
+      for (int c = sl; c < n_chunks; c += S) {
+        const int v = chunk_counts[static_cast<int64_t>(c) * E + e];
+        tot += v;
+        pre += c < b ? v : 0;
+      }
+    }
+    s_tot_part[tid] = tot;
+    s_pre_part[tid] = pre;
+  }
+  for (int i = tid; i < 8 * E; i += blockDim.x) mask[i / E][i % E] = 0u;
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int tot = 0, pre = 0;
+    for (int sl = 0; sl < S; ++sl) {
+      tot += s_tot_part[sl * E + e];
+      pre += s_pre_part[sl * E + e];
+    }
+    long long ce = expert_cap ? static_cast<long long>(expert_cap[e]) : cap;  // Zen MoDE §5.3 capacity_e
+    s_tot[e] = tot;
+    s_pre[e] = pre;
+    s_kept[e] = (ce < 0 || tot < ce) ? tot : static_cast<int>(ce);
+  }
+  __syncthreads();
+  // 2. seg_off = exclusive prefix of kept over experts (warp 0; 8 experts per lane)
+  if (warp == 0) {
+    constexpr int kPer = kMaxExperts / 32;
+    int v[kPer];
+    int loc = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int ee = lane * kPer + i;
+      v[i] = ee < E ? s_kept[ee] : 0;
+      loc += v[i];
+    }
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - loc;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int ee = lane * kPer + i;
+      if (ee < E) s_seg[ee] = run;
+      run += v[i];
+    }
+    if (lane == 31) s_seg[E] = incl;
+  }
+  // 3. this chunk's lane masks
+  const int64_t t = static_cast<int64_t>(b) * kDispatchChunk + warp * 32 + lane;
+  const bool tok_ok = t < T;
+  if (tok_ok) {
+    for (int k = 0; k < K; ++k) {
+      const int e = idx[t * K + k];
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicOr(&mask[warp][e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = s_pre[e];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w][e] = run;
+      run += __popc(mask[w][e]);
+    }
+  }
+  if (b == 0) {
+    for (int e = tid; e < E; e += blockDim.x) {
+      counts[e] = s_tot[e];
+      kept_out[e] = s_kept[e];
+    }
+    for (int e = tid; e <= E; e += blockDim.x) seg_off_out[e] = s_seg[e];
+  }
+  __syncthreads();
+  // 4. ranks and slots
+  if (tok_ok) {
+    const uint32_t lower = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int64_t pair = t * K + k;
+      const int e = idx[pair];
+      int slot = -1;
+      if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
+        const int rank = wbase[warp][e] + __popc(mask[warp][e] & lower);
+        if (rank < s_kept[e]) {
+          slot = s_seg[e] + rank;
+          perm[slot] = static_cast<int32_t>(pair);
+        }
+      }
+      slot_of[pair] = slot;
+    }
+  }
+  // 5. block 0: the balance statistics (f, P, loss; z-loss and utilisation with zpart)
+  if (b == 0 && stats) {
+    for (int e = tid; e < E; e += blockDim.x) {
+      unsigned long long ps = 0;
+      for (int c = 0; c < n_chunks; ++c) ps += chunk_psum[static_cast<int64_t>(c) * E + e];
+      s_fp[e] = balance_stats_expert(s_tot[e], ps, T, E, K, e, stats);
+    }
+    double z = 0.0;
+    if (zpart)
+      for (int i = tid; i < n_zpart; i += blockDim.x) z += zpart[i];
+    s_red[tid] = z;
+    __syncthreads();
+    for (int w = 128; w > 0; w >>= 1) {  // fixed-shape tree
+      if (tid < w) s_red[tid] += s_red[tid + w];
+      __syncthreads();
+    }
+    if (tid == 0) {
+      balance_loss(s_fp, E, alpha, stats);
+      if (zpart) utilisation_stats(s_tot, s_kept, E, T, s_red[0], stats);
+    }
+  }
+}
+
+bool dispatch_fused(const Problem& p) {
+  const long long n_chunks = (p.T + kDispatchChunk - 1) / kDispatchChunk;
+  return n_chunks * n_chunks * p.E <= kFusedScanMaxReads;
+}
+
 cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* counts, int32_t* kept,
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready,
@@ -220,6 +392,11 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
                                  chunk_counts, status))
       return e;
   }
+  if (dispatch_fused(p))
+    return launch_k(dispatch_scan_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
+                    static_cast<const int32_t*>(chunk_counts), n_chunks, static_cast<long long>(p.cap), expert_cap,
+                    counts, kept, seg_off, slot_of, perm, chunk_psum, chunk_psum ? stats : nullptr, p.alpha, zpart,
+                    n_zpart);
   if (cudaError_t e = launch_k(dispatch_scan_kernel, dim3(1), dim3(1024), 0, st,
                                static_cast<const int32_t*>(chunk_counts), n_chunks, p.E, static_cast<long long>(p.cap),
                                chunk_base, counts, kept, seg_off, chunk_psum, chunk_psum ? stats : nullptr, p.T,

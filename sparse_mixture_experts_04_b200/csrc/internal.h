@@ -64,6 +64,9 @@ cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, co
                                int n_chunks, const float* zpart, int n_zpart, float* stats, cudaStream_t st);
 
 // dispatch.cu
+// true when launch_dispatch ranks with one fused scan+rank kernel (else a
+// scan kernel and a rank kernel)
+bool dispatch_fused(const Problem& p);
 // counts_ready: chunk_counts already hold the per-chunk expert histogram (the
 // selection kernel adds it when given a zeroed chunk_counts)
 // chunk_psum / stats: when both are given, the scan also finalises the

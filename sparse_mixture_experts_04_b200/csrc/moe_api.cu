@@ -406,14 +406,15 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
                           ws, L, st, /*chunk_totals_cleared=*/true, /*stats_in_route=*/false, &n_zpart, &kernels))
     return rc;
   if (cudaError_t e = mark(MOE_EV_ROUTED)) return cuda_rc(e);
-  // the scan also finalises the balance statistics from the chunk totals
+  // scan+rank (the histogram came from the selection kernel); the scan also
+  // finalises the balance statistics from the chunk totals
   if (cudaError_t e = launch_dispatch(p, idx, counts, kept, seg_off, slot_of, perm, at<int32_t>(ws, L.chunk_counts),
                                       at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true,
                                       at<unsigned long long>(ws, L.chunk_psum), stats,
                                       (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr,
                                       n_zpart, expert_cap))
     return cuda_rc(e);
-  kernels += 2;
+  kernels += dispatch_fused(p) ? 1 : 2;
   if (p.max_rows > 0) {
     if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
     kernels += 1;

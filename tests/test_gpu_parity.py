@@ -186,6 +186,35 @@ def test_dispatch_flags_out_of_range_expert_without_faulting():
     assert counts.cpu().numpy()[0] == 39 and counts.cpu().numpy()[1] == 39
 
 
+@pytest.mark.parametrize("T,E,K", [(32768, 256, 4), (32769, 256, 4), (65536, 64, 4), (65537, 64, 4)])
+def test_layer_routing_and_stats_on_both_sides_of_the_fused_scan_limit(T, E, K):
+    """Dispatch ranks with one fused scan+rank kernel while ceil(T/256)^2 * E
+    <= 2^22 and with a scan kernel then a rank kernel above; each pair of
+    cases sits on the two sides of that limit.  Routing bit-exact and the
+    balance / extended statistics against the oracle, through the layer."""
+    cfg = MoeConfig(f"limit_{T}_{E}", T=T, d_model=64, n_experts=E, top_k=K, d_ff=64, n_shared=0,
+                    capacity_factor=1.0, dtype="bf16", seed=21, zipf_s=1.1)
+    inp = generate(cfg)
+    logits32 = given_logits(cfg)
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN | api.FLAG_EXTENDED_STATS)
+    layer.routing["logits"].copy_(torch.as_tensor(logits32))
+    layer.forward(dev(inp["x"]))
+    assert api.read_device_status(layer.ws) == 0
+    r = {k: v.cpu().numpy() for k, v in layer.routing.items()}
+    S = int(ref["seg_off"][-1])
+    assert 0 < S < T * K                                   # some pairs dropped
+    for k in ("counts", "kept", "seg_off"):
+        assert (r[k] == ref[k]).all(), k
+    assert (r["slot_of"].reshape(T, K) == ref["slot_of"]).all()
+    assert (r["perm"][:S] == ref["perm"]).all()
+    st = layer.stats.cpu().numpy()
+    assert (st[:E] == ref["f"].astype(np.float32)).all()
+    assert np.max(np.abs(st[E:2 * E] - ref["P"])) <= 1e-6
+    assert abs(st[2 * E] - ref["loss"]) <= 1e-6 * max(1.0, ref["loss"])
+    _check_extended(st, E, logits32.astype(np.float64), ref["counts"], ref["kept"])
+
+
 # ------------------------------------------------------------- expert FFNs
 @pytest.mark.parametrize("name", list(SMALL))
 def test_routed_expert_ffn_matches_oracle(name):
