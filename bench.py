@@ -188,6 +188,28 @@ def algorithmic_flops(cfg, kept_pairs: int) -> dict:
             "shared": 6.0 * d * F * Ns * T}
 
 
+def shared_mixed(cfg, prob) -> bool:
+    """True when the library runs the shared experts in the routed experts'
+    launches (BF16, shared experts, both on CTA-pair tiles: at least 256
+    expected rows per routed expert, T * K / E capped by the capacity, and
+    T >= 256), so the up and down stages cover both."""
+    if cfg.dtype != "bf16" or cfg.n_shared == 0 or os.environ.get("MOE_B200_MIX_SHARED", "1") == "0":
+        return False
+    expected = cfg.T * cfg.top_k // cfg.n_experts
+    cap = api.capacity(prob)
+    if cap >= 0:
+        expected = min(expected, cap)
+    return api.max_rows(prob) > 0 and expected >= 256 and cfg.T >= 256
+
+
+def shared_up_bytes(cfg) -> float:
+    """Algorithmic HBM bytes of the shared experts' up/gate projection: their
+    W13, x read once and their H written once."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    d, F, Ns, T = cfg.d_model, cfg.d_ff, cfg.n_shared, cfg.T
+    return es * (Ns * 2.0 * F * d + T * d + T * Ns * F)
+
+
 def up_gemm_bytes(cfg, kept_per_expert) -> float:
     """Algorithmic HBM bytes of the routed up/gate GEMM: the W13 slices of every
     expert that received a row, its x_perm rows read once and H written once."""
@@ -198,13 +220,14 @@ def up_gemm_bytes(cfg, kept_per_expert) -> float:
     return es * (touched * 2.0 * F * d + rows * d + rows * F)
 
 
-def roofline(cfg, flops: float, nbytes: float, launch_ms: float, peaks: dict, peak_src: str, traffic) -> dict:
+def roofline(cfg, flops: float, nbytes: float, launch_ms: float, peaks: dict, peak_src: str, traffic,
+             kernel: str = "routed up/gate GEMM with SwiGLU epilogue (tcgen05)") -> dict:
     """Bound = whichever of tensor time (flops / dense BF16 peak) and HBM time
     (bytes / copy bandwidth) is longer; achieved and peak are in that unit."""
     t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     src = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    r = {"kernel": "routed up/gate GEMM with SwiGLU epilogue (tcgen05)",
+    r = {"kernel": kernel,
          "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes, "launch_ms": launch_ms,
          "traffic": traffic}
     if t_tensor >= t_hbm:
@@ -495,8 +518,16 @@ def run_ours(args, cfg):
     up_bytes = up_gemm_bytes(cfg, layer.routing["kept"].tolist())
     flops = algorithmic_flops(cfg, kept)
     peaks, peak_src = load_peaks()
+    mixed = shared_mixed(cfg, layer.prob)
     gemm_ms = stage["up"] + stage["down"]
-    gemm_tflops = (flops["up"] + flops["down"]) / (gemm_ms * 1e-3) / 1e12
+    gemm_flops = flops["up"] + flops["down"] + (flops["shared"] if mixed else 0.0)
+    gemm_tflops = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    if mixed:   # the dominant launch computes the shared experts' up projection too
+        roof = roofline(cfg, flops["up"] + 4.0 * cfg.d_model * cfg.d_ff * cfg.n_shared * cfg.T,
+                        up_bytes + shared_up_bytes(cfg), up_ms, peaks, peak_src, ncu_traffic(cfg.name),
+                        kernel="routed + shared up/gate GEMM with SwiGLU epilogue, one launch (tcgen05)")
+    else:
+        roof = roofline(cfg, flops["up"], up_bytes, up_ms, peaks, peak_src, ncu_traffic(cfg.name))
     disp_gbs = dispatch_bytes(cfg, kept) / (stage["dispatched"] * 1e-3) / 1e9
     router_gbs = router_bytes(cfg) / (stage["routed"] * 1e-3) / 1e9
     combine_gbs = combine_bytes(cfg, kept) / (stage["end"] * 1e-3) / 1e9
@@ -528,11 +559,14 @@ def run_ours(args, cfg):
                          " GiB of weights per step, both larger than the 126 MB L2; no flush"},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "roofline": roofline(cfg, flops["up"], up_bytes, up_ms, peaks, peak_src, ncu_traffic(cfg.name)),
+        "roofline": roof,
         "cpu_baseline": cpu,
         "gpu_launches": n_kernels,
         "clocks": {**clk.summary(), "remeasured": remeasured},
-        "stages_ms": stage, "stages_note": "separate pass with an event at every stage boundary",
+        "stages_ms": stage,
+        "stages_note": "separate pass with an event at every stage boundary" +
+                       ("; the shared experts run in the up and down launches (the shared stage is empty)"
+                        if mixed else ""),
         "kept_pairs": kept, "dropped_pairs": cfg.T * cfg.top_k - kept,
         "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
         "dispatch_gbs": disp_gbs, "router_gbs": router_gbs, "combine_gbs": combine_gbs,

@@ -111,7 +111,8 @@ constexpr int gemm_smem_bytes() {
 
 struct TileInfo {
   int g, row0, row_end, n0;
-  bool swap;  // operand-swapped remainder tile (pair kernel only)
+  bool swap;    // operand-swapped remainder tile (pair kernel only)
+  bool second;  // tile of the pair kernel's second problem
 };
 
 // Rows [base, base + return) of group g (the part row_mode selects), clamped
@@ -152,6 +153,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   ti.row_end = base + rows;
   ti.n0 = n_idx * out_cols;
   ti.swap = m_idx == mt - 1 && rows - m_idx * BM <= a.swap_max;
+  ti.second = false;
   return ti;
 }
 
@@ -479,7 +481,27 @@ __device__ __forceinline__ int swap_box_rows(int half_n) {
 }
 
 constexpr int pair_smem_bytes() {
-  return kPairStages * kPairStageBytes + 256 + 4 * (kMaxGroups + 1) + kSwapXBytes + 1024;
+  return kPairStages * kPairStageBytes + 256 + 8 * (kMaxGroups + 1) + kSwapXBytes + 1024;
+}
+
+// Tile `tile` of a launch over two problems with t1 and total - t1 tiles: the
+// first problem's tiles are spread evenly through [0, total) (tile i is the
+// first problem's number floor(i t1 / total) when that count steps at i), so
+// every pair's strided walk mixes both kinds in proportion.
+__device__ __forceinline__ TileInfo decode_pair_tile(int tile, int t1, int total, const int* prefix,
+                                                     const int* prefix2, const GemmArgs& a1, const GemmArgs& a2,
+                                                     int out_cols) {
+  const int lo = static_cast<int>(static_cast<long long>(tile) * t1 / total);
+  const int hi = static_cast<int>(static_cast<long long>(tile + 1) * t1 / total);
+  if (hi > lo) return decode_tile<kPairBM>(lo, prefix, a1, out_cols);
+  TileInfo ti = decode_tile<kPairBM>(tile - lo, prefix2, a2, out_cols);
+  ti.second = true;
+  return ti;
+}
+
+// 128-deep k-blocks of one tile of a problem
+__device__ __forceinline__ int pair_nkb(const GemmArgs& a) {
+  return ((a.K + kBK * kPairKC - 1) / (kBK * kPairKC)) * a.k_groups;
 }
 
 // MMA N of a swap tile covering `rows` (1..256) token rows: a multiple of 16.
@@ -567,7 +589,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmA64, const __grid_constant__ CUtensorMap tmB64,
                              const __grid_constant__ CUtensorMap tmA32, const __grid_constant__ CUtensorMap tmA16,
-                             const GemmArgs args) {
+                             const __grid_constant__ GemmArgs args,
+                             const __grid_constant__ CUtensorMap tmA_2, const __grid_constant__ CUtensorMap tmB_2,
+                             const __grid_constant__ CUtensorMap tmA64_2, const __grid_constant__ CUtensorMap tmB64_2,
+                             const __grid_constant__ CUtensorMap tmA32_2, const __grid_constant__ CUtensorMap tmA16_2,
+                             const __grid_constant__ GemmArgs args2) {
   constexpr int kOutCols = (EPI == EPI_SWIGLU) ? kPairBN / 2 : kPairBN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -581,7 +607,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
-  float* xbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(prefix + kMaxGroups + 1) + 15) & ~uintptr_t(15));
+  int* prefix2 = prefix + kMaxGroups + 1;
+  float* xbuf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(prefix2 + kMaxGroups + 1) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -589,6 +616,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
   const int n_tiles_n = (args.N + kOutCols - 1) / kOutCols;
+  const int n_tiles_n2 = (args2.N + kOutCols - 1) / kOutCols;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPairStages; ++s) {
@@ -610,6 +638,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     prefetch_tensormap(&tmA32);
     prefetch_tensormap(&tmA16);
     prefetch_tensormap(&tmB64);
+    if (args2.n_groups > 0) {
+      prefetch_tensormap(&tmA_2);
+      prefetch_tensormap(&tmB_2);
+      prefetch_tensormap(&tmA64_2);
+      prefetch_tensormap(&tmA32_2);
+      prefetch_tensormap(&tmA16_2);
+      prefetch_tensormap(&tmB64_2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -618,13 +654,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   pdl_wait();  // everything above is local set-up; from here on the predecessor's outputs are read
   pdl_trigger();
   if (warp == 2) tile_prefix_warp<kPairBM>(args, n_tiles_n, prefix, lane);
+  if (warp == 3) {
+    if (args2.n_groups > 0)
+      tile_prefix_warp<kPairBM>(args2, n_tiles_n2, prefix2, lane);
+    else if (lane == 0)
+      prefix2[0] = 0;
+  }
   tc_fence_before_sync();
   cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const int total_tiles = prefix[args.n_groups];
-  const int nkb_g = (args.K + kBK * kPairKC - 1) / (kBK * kPairKC);
-  const int nkb = nkb_g * args.k_groups;  // no split-K on the pair path
+  const int tiles1 = prefix[args.n_groups];
+  const int total_tiles = tiles1 + prefix2[max(args2.n_groups, 0)];
+  // no split-K on the pair path
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -634,7 +676,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs) {
-        const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
+        const TileInfo ti = decode_pair_tile(tile, tiles1, total_tiles, prefix, prefix2, args, args2, kOutCols);
+        const GemmArgs& A = ti.second ? args2 : args;
+        const CUtensorMap* mA = ti.second ? &tmA_2 : &tmA;
+        const CUtensorMap* mB = ti.second ? &tmB_2 : &tmB;
+        const CUtensorMap* mB64 = ti.second ? &tmB64_2 : &tmB64;
+        const int nkb_g = (A.K + kBK * kPairKC - 1) / (kBK * kPairKC);
+        const int nkb = nkb_g * A.k_groups;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -647,7 +695,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           // 64 or 128 rows) may load more, the MMA reads the first N/2
           const int half_n = ti.swap ? swap_n(ti.row_end - ti.row0) / 2 : 128;
           const int a_box = ti.swap ? swap_box_rows(half_n) : 128;
-          const CUtensorMap* a_map = a_box == 16 ? &tmA16 : a_box == 32 ? &tmA32 : a_box == 64 ? &tmA64 : &tmA;
+          const CUtensorMap* a_map = a_box == 16   ? (ti.second ? &tmA16_2 : &tmA16)
+                                     : a_box == 32 ? (ti.second ? &tmA32_2 : &tmA32)
+                                     : a_box == 64 ? (ti.second ? &tmA64_2 : &tmA64)
+                                                   : mA;
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kPairKC * (kPairChunk + a_box * kBK * 2));
           const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
           uint8_t* a_dst = sA + stage * kPairABytes;
@@ -657,20 +708,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           // both 64-deep chunks (the tokens' chunk c at c * a_box rows, the
           // weights' at c * kPairChunk; chunks past K read zeros).  Full tiles
           // keep one box per chunk, which measured slightly faster for them.
-          const bool merge = args.merged_k && ti.swap;
+          const bool merge = A.merged_k && ti.swap;
           if (merge && a_box <= 64) {
-            tma_load_3d_pair(a_dst, a_map, bar, 0, a_row, (kg * args.K + kk0) / kBK);
+            tma_load_3d_pair(a_dst, a_map, bar, 0, a_row, (kg * A.K + kk0) / kBK);
           } else {
 #pragma unroll
             for (int c = 0; c < kPairKC; ++c)  // past K: the box reads zeros
-              tma_load_2d_pair(a_dst + c * a_box * kBK * 2, a_box == 128 ? &tmA : a_map, bar,
-                               kg * args.K + kk0 + c * kBK, a_row);
+              tma_load_2d_pair(a_dst + c * a_box * kBK * 2, a_box == 128 ? mA : a_map, bar, kg * A.K + kk0 + c * kBK,
+                               a_row);
           }
           if (merge) {
             if (EPI == EPI_SWIGLU)  // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
-              tma_load_4d_pair(b_dst, &tmB64, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
+              tma_load_4d_pair(b_dst, mB64, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
             else
-              tma_load_4d_pair(b_dst, &tmB64, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * args.k_groups + kg,
+              tma_load_4d_pair(b_dst, mB64, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * A.k_groups + kg,
                                kk0 / kBK);
           } else {
 #pragma unroll
@@ -679,12 +730,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               uint8_t* bc = b_dst + c * kPairChunk;
               if (EPI == EPI_SWIGLU && ti.swap) {
                 const int f = ti.n0 + 64 * static_cast<int>(rank);
-                tma_load_3d_pair(bc, &tmB64, bar, kk, f, 2 * ti.g);
-                tma_load_3d_pair(bc + kPairChunk / 2, &tmB64, bar, kk, f, 2 * ti.g + 1);
+                tma_load_3d_pair(bc, mB64, bar, kk, f, 2 * ti.g);
+                tma_load_3d_pair(bc + kPairChunk / 2, mB64, bar, kk, f, 2 * ti.g + 1);
               } else if (EPI == EPI_SWIGLU) {
-                tma_load_3d_pair(bc, &tmB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
+                tma_load_3d_pair(bc, mB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
               } else {
-                tma_load_3d_pair(bc, &tmB, bar, kk, ti.n0 + 128 * static_cast<int>(rank), ti.g * args.k_groups + kg);
+                tma_load_3d_pair(bc, mB, bar, kk, ti.n0 + 128 * static_cast<int>(rank), ti.g * A.k_groups + kg);
               }
             }
           }
@@ -716,7 +767,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       int it = 0;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
-        const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
+        const TileInfo ti = decode_pair_tile(tile, tiles1, total_tiles, prefix, prefix2, args, args2, kOutCols);
+        const int nkb = pair_nkb(ti.second ? args2 : args);
         // normal tile: A = token rows (M = 256), B = weight rows (N = 256);
         // swap tile: A = weight rows (M = 256), B = the tile's N token rows
         const uint32_t idesc = idesc_bf16_f32(kPairBM, ti.swap ? swap_n(ti.row_end - ti.row0) : kPairBN);
@@ -768,7 +820,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const uint32_t tempty_leader = mapa_shared(smem_addr(&tempty[0]), 0);
     int it = 0;
     for (int tile = pair; tile < total_tiles; tile += n_pairs, ++it) {
-      const TileInfo ti = decode_tile<kPairBM>(tile, prefix, args, kOutCols);
+      const TileInfo ti = decode_pair_tile(tile, tiles1, total_tiles, prefix, prefix2, args, args2, kOutCols);
+      const GemmArgs& A = ti.second ? args2 : args;
       const int acc = it & 1;
       const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
       // all four epilogue warps take the same decision (a swap tile's
@@ -779,10 +832,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kPairBN);
       if (ti.swap) {
-        epilogue_swap<EPI>(args, ti, rank, quarter, lane, (warp - 2) * 32 + lane, t_row, xbuf);
+        epilogue_swap<EPI>(A, ti, rank, quarter, lane, (warp - 2) * 32 + lane, t_row, xbuf);
       } else {
         const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
-        epilogue_rows<EPI, kPairBN>(args, ti.g, row, row < ti.row_end, ti.n0, t_row);
+        epilogue_rows<EPI, kPairBN>(A, ti.g, row, row < ti.row_end, ti.n0, t_row);
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -934,10 +987,18 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
                   smem, st, ta, tb, a) == cudaSuccess ? 0 : -3;
 }
 
+// One problem of a pair-kernel launch: its tensor maps (see the kernel's
+// parameters), arguments and an upper bound on its tiles.
+struct PairProblem {
+  CUtensorMap ta, tb, ta64, tb64, ta32, ta16;
+  GemmArgs a;
+  int64_t tile_bound;
+};
+
+// p2 (or nullptr): a second problem whose tiles the same launch interleaves
+// with p1's (same EPI and tile shape; see decode_pair_tile).
 template <int EPI>
-static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ta64, const CUtensorMap& tb64,
-                         const CUtensorMap& ta32, const CUtensorMap& ta16, const GemmArgs& a, int64_t tile_bound,
-                         cudaStream_t st) {
+static int run_pair_gemm(const PairProblem& p1, const PairProblem* p2, cudaStream_t st) {
   constexpr int smem = pair_smem_bytes();
   static std::mutex mu;
   static int max_pairs[64] = {0};
@@ -964,10 +1025,16 @@ static int run_pair_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
     }
     pairs = max_pairs[dev];
   }
+  const int64_t tile_bound = p1.tile_bound + (p2 ? p2->tile_bound : 0);
   if (tile_bound <= 0) return 0;
   if (pairs > tile_bound) pairs = static_cast<int>(tile_bound);
+  // without a second problem its maps are p1's (never read: no tiles)
+  const PairProblem& q = p2 ? *p2 : p1;
+  GemmArgs a2 = q.a;
+  if (!p2) a2.n_groups = 0;
   return launch_k(grouped_gemm_pair_kernel<EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads), smem,
-                  st, ta, tb, ta64, tb64, ta32, ta16, a) == cudaSuccess ? 0 : -3;
+                  st, p1.ta, p1.tb, p1.ta64, p1.tb64, p1.ta32, p1.ta16, p1.a, q.ta, q.tb, q.ta64, q.tb64, q.ta32,
+                  q.ta16, a2) == cudaSuccess ? 0 : -3;
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -1190,6 +1257,81 @@ int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_
   return run_gemm<EPI_BF16, 256, 4>(ta, tb, a, mt * cdiv(2 * p.F, 256), st);
 }
 
+// Tile shape of one FFN (routed: expected rows per group T*K/E capped by the
+// capacity; shared: every row).
+static int ffn_tile_mode(const Problem& p, bool routed, int64_t n_rows) {
+  int64_t expected = routed ? (p.T * p.K) / p.E : n_rows;
+  if (routed && p.cap >= 0 && p.cap < expected) expected = p.cap;
+  return tile_mode(expected);
+}
+
+// Pair-kernel problem of an up/gate projection + SwiGLU: A = x_rows [n_rows, d],
+// B = w13 [G, 2F, d] viewed as (d, F, 2G): gate rows of group g at 2g, up rows
+// at 2g+1; swap tiles take 64 gate and the same 64 up rows per CTA.
+static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, int64_t n_rows,
+                            const int32_t* seg_off, const void* w13, void* h, void* gu, unsigned* status, bool tail,
+                            PairProblem* q) {
+  const int G = routed ? p.E : p.Ns;
+  const bool merged = merged_k_ok(p.d);
+  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, x_rows, p.d, n_rows, merged) ||
+      !make_weight_map(&q->tb, w13, p.d, p.F, 2 * G, 128, 1, false) ||
+      !make_weight_map(&q->tb64, w13, p.d, p.F, 2 * G, 64, merged ? 2 : 1, merged))
+    return false;
+  GemmArgs& a = q->a;
+  a = GemmArgs{};
+  a.n_groups = G;
+  a.seg_off = routed ? seg_off : nullptr;
+  a.n_rows = static_cast<int>(n_rows);
+  a.N = p.F;
+  a.K = p.d;
+  a.k_groups = 1;
+  a.out = h;
+  a.ldo = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+  a.out_col_stride = routed ? 0 : p.F;
+  a.status = status;
+  a.swap_max = swap_max_rows();
+  a.gu = gu;  // kept for the backward (routed [rows, 2F]; shared [rows, N_s 2F])
+  a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
+  a.gu_col_stride = routed ? 0 : 2 * p.F;
+  a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
+  a.merged_k = merged ? 1 : 0;
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
+  q->tile_bound = (mt / 2 + G) * cdiv(p.F, 128);
+  return true;
+}
+
+// Pair-kernel problem of a down projection: A = h [n_rows, k_groups * F],
+// B = w2 [G, d, F] viewed as (F, d, G); a pair CTA stages half of the 256 B
+// rows.  Shared: one group whose reduction runs over all N_s experts.
+static bool down_pair_problem(const Problem& p, bool routed, const void* h, int64_t n_rows, const int32_t* seg_off,
+                              const void* w2, void* y_rows, unsigned* status, bool tail, PairProblem* q) {
+  const int G = routed ? p.E : p.Ns;
+  const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+  const bool merged = merged_k_ok(p.F);
+  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, h, h_cols, n_rows, merged) ||
+      !make_weight_map(&q->tb, w2, p.F, p.d, G, 128, 1, false) ||
+      !make_weight_map(&q->tb64, w2, p.F, p.d, G, 128, 1, merged))
+    return false;
+  GemmArgs& a = q->a;
+  a = GemmArgs{};
+  a.n_groups = routed ? G : 1;
+  a.seg_off = routed ? seg_off : nullptr;
+  a.n_rows = static_cast<int>(n_rows);
+  a.N = p.d;
+  a.K = p.F;
+  a.k_groups = routed ? 1 : p.Ns;
+  a.out = y_rows;
+  a.ldo = p.d;
+  a.out_col_stride = 0;
+  a.status = status;
+  a.swap_max = swap_max_rows();
+  a.row_mode = tail ? 1 : 0;
+  a.merged_k = merged ? 1 : 0;
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
+  q->tile_bound = (mt / 2 + a.n_groups) * cdiv(p.d, 256);
+  return true;
+}
+
 // mode 0: routed (groups = experts over seg_off); mode 1: shared (every row
 // through all N_s experts, summed).  h is scratch: [n_rows, F] (routed) or
 // [n_rows, N_s * F] (shared).
@@ -1204,55 +1346,25 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
   const bool routed = mode == 0;
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
-  // expected rows per group: routed T*K/E (at most the capacity), shared all rows
-  int64_t expected = routed ? (p.T * p.K) / p.E : n_rows;
-  if (routed && p.cap >= 0 && p.cap < expected) expected = p.cap;
-  const int mode_t = tile_mode(expected);
+  const int mode_t = ffn_tile_mode(p, routed, n_rows);
   const bool pair = mode_t != kTileSingle;
   const bool tail = mode_t == kTilePairTail;
   if (n_kernels) *n_kernels += tail ? 4 : 2;
 
-  // up/gate projection + SwiGLU: A = x_rows [n_rows, d], B = w13 viewed as (d, F, 2G)
-  CUtensorMap ta, tb;
+  // up/gate projection + SwiGLU
   {
     const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.F), static_cast<uint64_t>(2 * G)};
     const uint32_t bb[3] = {kBK, 128, 1};
-    CUtensorMap ta64, tb64, ta32, ta16;
-    const bool merged = pair && merged_k_ok(p.d);
+    CUtensorMap ta, tb;
     if (pair) {
-      // w13 [G, 2F, d] as (d, F, 2G): gate rows of group g at 2g, up rows at 2g+1;
-      // swap tiles take 64 gate and the same 64 up rows per CTA
-      if (!make_token_maps(&ta, &ta64, &ta32, &ta16, x_rows, p.d, n_rows, merged) ||
-          !make_weight_map(&tb, w13, p.d, p.F, 2 * G, 128, 1, false) ||
-          !make_weight_map(&tb64, w13, p.d, p.F, 2 * G, 64, merged ? 2 : 1, merged))
-        return -3;
-    } else if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) {
-      return -3;
-    }
-    GemmArgs a{};
-    a.n_groups = G;
-    a.seg_off = routed ? seg_off : nullptr;
-    a.n_rows = static_cast<int>(n_rows);
-    a.N = p.F;
-    a.K = p.d;
-    a.k_groups = 1;
-    a.out = h;
-    a.ldo = h_cols;
-    a.out_col_stride = routed ? 0 : p.F;
-    a.status = status;
-    a.swap_max = swap_max_rows();
-    a.gu = gu;  // kept for the backward (routed [rows, 2F]; shared [rows, N_s 2F])
-    a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
-    a.gu_col_stride = routed ? 0 : 2 * p.F;
-    const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
-    if (pair) {
-      a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
-      a.merged_k = merged ? 1 : 0;
-      int rc = run_pair_gemm<EPI_SWIGLU>(ta, tb, ta64, tb64, ta32, ta16, a, (mt / 2 + G) * cdiv(p.F, 128), st);
+      PairProblem q;
+      if (!up_pair_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, tail, &q)) return -3;
+      int rc = run_pair_gemm<EPI_SWIGLU>(q, nullptr, st);
       if (rc) return rc;
       if (tail) {
+        GemmArgs a = q.a;
         a.row_mode = 2;  // the rest (under 256 rows per group) on single CTAs
         a.swap_max = 0;
         a.merged_k = 0;
@@ -1261,59 +1373,97 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
         if (rc) return rc;
       }
     } else {
+      if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
+      GemmArgs a{};
+      a.n_groups = G;
+      a.seg_off = routed ? seg_off : nullptr;
+      a.n_rows = static_cast<int>(n_rows);
+      a.N = p.F;
+      a.K = p.d;
+      a.k_groups = 1;
+      a.out = h;
+      a.ldo = h_cols;
+      a.out_col_stride = routed ? 0 : p.F;
+      a.status = status;
+      a.swap_max = swap_max_rows();
+      a.gu = gu;
+      a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
+      a.gu_col_stride = routed ? 0 : 2 * p.F;
+      const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
       const int rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, mt * cdiv(p.F, 128), st);
       if (rc) return rc;
     }
     if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
   }
-  // down projection: A = h [n_rows, k_groups * F], B = w2 viewed as (F, d, G)
+  // down projection
   {
     const uint64_t da[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
     const uint32_t ba[2] = {kBK, kBM};
     const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
     const uint32_t bb[3] = {kBK, 256, 1};
-    CUtensorMap tb_half, tb_swap, ta64, ta32, ta16;
-    const bool merged = pair && merged_k_ok(p.F);
+    CUtensorMap ta, tb;
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
-    // w2 [G, d, F] as (F, d, G); a pair CTA stages half of the 256 B rows
-    const int64_t wg = routed ? G : p.Ns;
-    if (pair && (!make_token_maps(&ta, &ta64, &ta32, &ta16, h, h_cols, n_rows, merged) ||
-                 !make_weight_map(&tb_half, w2, p.F, p.d, wg, 128, 1, false) ||
-                 !make_weight_map(&tb_swap, w2, p.F, p.d, wg, 128, 1, merged)))
-      return -3;
-    GemmArgs a{};
-    a.n_groups = routed ? G : 1;
-    a.seg_off = routed ? seg_off : nullptr;
-    a.n_rows = static_cast<int>(n_rows);
-    a.N = p.d;
-    a.K = p.F;
-    a.k_groups = routed ? 1 : p.Ns;
-    a.out = y_rows;
-    a.ldo = p.d;
-    a.out_col_stride = 0;
-    a.status = status;
-    a.swap_max = swap_max_rows();
-    const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
     if (pair) {
-      a.row_mode = tail ? 1 : 0;
-      a.merged_k = merged ? 1 : 0;
-      int rc = run_pair_gemm<EPI_BF16>(ta, tb_half, ta64, tb_swap, ta32, ta16, a,
-                                       (mt / 2 + a.n_groups) * cdiv(p.d, 256), st);
+      PairProblem q;
+      if (!down_pair_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, tail, &q)) return -3;
+      int rc = run_pair_gemm<EPI_BF16>(q, nullptr, st);
       if (rc) return rc;
       if (tail) {
+        GemmArgs a = q.a;
         a.row_mode = 2;
         a.swap_max = 0;
         a.merged_k = 0;
-        if (!make_map(&ta, h, 2, da, ba)) return -3;
         rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.d, 256), st);
         if (rc) return rc;
       }
     } else {
+      GemmArgs a{};
+      a.n_groups = routed ? G : 1;
+      a.seg_off = routed ? seg_off : nullptr;
+      a.n_rows = static_cast<int>(n_rows);
+      a.N = p.d;
+      a.K = p.F;
+      a.k_groups = routed ? 1 : p.Ns;
+      a.out = y_rows;
+      a.ldo = p.d;
+      a.out_col_stride = 0;
+      a.status = status;
+      a.swap_max = swap_max_rows();
+      const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
       const int rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, mt * cdiv(p.d, 256), st);
       if (rc) return rc;
     }
   }
   return 0;
+}
+
+bool expert_ffn_mixed_ok(const Problem& p) {
+  const char* e = getenv("MOE_B200_MIX_SHARED");
+  if (e && e[0] == '0') return false;
+  return p.dtype == kBF16 && p.Ns > 0 && p.max_rows > 0 && ffn_tile_mode(p, true, p.max_rows) == kTilePair &&
+         ffn_tile_mode(p, false, p.T) == kTilePair;
+}
+
+// Routed and shared experts in the same two pair-kernel launches (up/gate +
+// SwiGLU for both, then both down projections): the routed tiles, bound by
+// the weight reads when the experts get few rows, share every SM's time with
+// the shared experts' tensor-core-bound tiles instead of running alone.
+int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t* seg_off, const void* w13,
+                            const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
+                            const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
+                            cudaStream_t st, cudaEvent_t after_up, int* n_kernels) {
+  if (!expert_ffn_mixed_ok(p)) return -3;
+  if (n_kernels) *n_kernels += 2;
+  PairProblem r, s;
+  if (!up_pair_problem(p, true, x_perm, p.max_rows, seg_off, w13, h, gu, status, false, &r) ||
+      !up_pair_problem(p, false, x, p.T, nullptr, w13_shared, h_shared, gu_shared, status, false, &s))
+    return -3;
+  if (int rc = run_pair_gemm<EPI_SWIGLU>(r, &s, st)) return rc;
+  if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
+  if (!down_pair_problem(p, true, h, p.max_rows, seg_off, w2, y_perm, status, false, &r) ||
+      !down_pair_problem(p, false, h_shared, p.T, nullptr, w2_shared, y_shared, status, false, &s))
+    return -3;
+  return run_pair_gemm<EPI_BF16>(r, &s, st);
 }
 
 }  // namespace moe

@@ -97,6 +97,16 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
                       cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr,
                       void* gu = nullptr);
+// Routed (x_perm over seg_off, p.max_rows rows) and shared (x, T rows)
+// experts in the same two launches, their tiles interleaved: requires
+// expert_ffn_mixed_ok(p) (BF16, shared experts, both on CTA-pair tiles;
+// MOE_B200_MIX_SHARED=0 turns it off).  gu / gu_shared: nullptr or the saved
+// gate and up projections.
+bool expert_ffn_mixed_ok(const Problem& p);
+int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t* seg_off, const void* w13,
+                            const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
+                            const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
+                            cudaStream_t st, cudaEvent_t after_up, int* n_kernels);
 
 // expert_gemm.cu: gu = x W13^T (gate | up projections, BF16) for the backward
 int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,

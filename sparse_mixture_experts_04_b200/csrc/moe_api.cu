@@ -420,21 +420,32 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     kernels += 1;
   }
   if (cudaError_t e = mark(MOE_EV_DISPATCHED)) return cuda_rc(e);
-  if (p.max_rows > 0) {
-    cudaEvent_t up_ev = (events && events[MOE_EV_UP]) ? static_cast<cudaEvent_t>(events[MOE_EV_UP]) : nullptr;
-    void* gu = (p.flags & MOE_FLAG_SAVE_GU) && p.dtype == kBF16 ? at<void>(ws, L.gu_routed) : nullptr;
-    if (launch_expert_ffn(p, MOE_FFN_ROUTED, x_perm, p.max_rows, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed),
-                          y_perm, status, st, up_ev, &kernels, gu))
+  const bool save_gu = (p.flags & MOE_FLAG_SAVE_GU) && p.dtype == kBF16;
+  cudaEvent_t up_ev = (events && events[MOE_EV_UP]) ? static_cast<cudaEvent_t>(events[MOE_EV_UP]) : nullptr;
+  if (expert_ffn_mixed_ok(p)) {
+    // routed and shared experts in the same two launches; the stage events
+    // UP and DOWN then cover both, SHARED follows DOWN at once
+    if (launch_expert_ffn_mixed(p, x_perm, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed), y_perm,
+                                save_gu ? at<void>(ws, L.gu_routed) : nullptr, x, w->w13_shared, w->w2_shared,
+                                at<void>(ws, L.h_shared), y_sh, save_gu ? at<void>(ws, L.gu_shared) : nullptr,
+                                status, st, up_ev, &kernels))
       return MOE_ERR_CUDA;
-  } else if (cudaError_t e = mark(MOE_EV_UP)) {
-    return cuda_rc(e);
-  }
-  if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
-  if (p.Ns > 0) {
-    void* gu = (p.flags & MOE_FLAG_SAVE_GU) && p.dtype == kBF16 ? at<void>(ws, L.gu_shared) : nullptr;
-    if (launch_expert_ffn(p, MOE_FFN_SHARED, x, p.T, nullptr, w->w13_shared, w->w2_shared,
-                          at<void>(ws, L.h_shared), y_sh, status, st, nullptr, &kernels, gu))
-      return MOE_ERR_CUDA;
+    if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
+  } else {
+    if (p.max_rows > 0) {
+      if (launch_expert_ffn(p, MOE_FFN_ROUTED, x_perm, p.max_rows, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed),
+                            y_perm, status, st, up_ev, &kernels, save_gu ? at<void>(ws, L.gu_routed) : nullptr))
+        return MOE_ERR_CUDA;
+    } else if (cudaError_t e = mark(MOE_EV_UP)) {
+      return cuda_rc(e);
+    }
+    if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
+    if (p.Ns > 0) {
+      if (launch_expert_ffn(p, MOE_FFN_SHARED, x, p.T, nullptr, w->w13_shared, w->w2_shared,
+                            at<void>(ws, L.h_shared), y_sh, status, st, nullptr, &kernels,
+                            save_gu ? at<void>(ws, L.gu_shared) : nullptr))
+        return MOE_ERR_CUDA;
+    }
   }
   if (cudaError_t e = mark(MOE_EV_SHARED)) return cuda_rc(e);
   if (cudaError_t e = launch_combine(p, y_perm, slot_of, gw, y_sh, y, st)) return cuda_rc(e);

@@ -53,3 +53,24 @@ def test_router_and_combine_bytes_at_the_mixtral_shape():
     # a shared expert adds its output rows to the combine's reads
     z = CONFIGS["zen_fine"]
     assert bench.combine_bytes(z, 0) == 2 * z.T * z.d_model * 2 + 8 * z.T * z.top_k
+
+
+@pytest.mark.parametrize("name,want", [("zen_fine", True), ("mixtral", False), ("skewed", False), ("decode", False),
+                                       ("tiny_fp32", False)])
+def test_shared_mixed_follows_the_library_rule(name, want, monkeypatch):
+    """The shared experts share the routed launches only with BF16, shared
+    experts and CTA-pair tiles for both (>= 256 expected rows per routed
+    expert after the capacity, T >= 256); MOE_B200_MIX_SHARED=0 turns it off."""
+    from sparse_mixture_experts_04_b200 import api
+    cfg = CONFIGS[name]
+    prob = api.make_problem(cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.n_shared,
+                            cfg.capacity_factor, cfg.dtype)
+    assert bench.shared_mixed(cfg, prob) is want
+    monkeypatch.setenv("MOE_B200_MIX_SHARED", "0")
+    assert bench.shared_mixed(cfg, prob) is False
+
+
+def test_shared_up_bytes_counts_weights_x_and_h():
+    cfg = CONFIGS["zen_fine"]
+    d, F, Ns, T = cfg.d_model, cfg.d_ff, cfg.n_shared, cfg.T
+    assert bench.shared_up_bytes(cfg) == 2 * (Ns * 2 * F * d + T * d + T * Ns * F)

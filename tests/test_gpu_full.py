@@ -86,3 +86,22 @@ def test_full_size_end_to_end(workload):
     want = oracle_layer(inp, ref, rows=rows)
     got = y.float().cpu().numpy()[rows]
     assert rel_err(got, want) <= tol(cfg)
+
+
+def test_full_size_mixed_shared_launch_is_bit_identical(workload, monkeypatch):
+    """Where the shared experts run in the routed experts' launches (zen_fine:
+    both on CTA-pair tiles), every tile is computed as in separate launches:
+    outputs and statistics are bit-identical with the mixing turned off."""
+    name, cfg, inp = workload
+    if cfg.dtype != "bf16" or cfg.n_shared == 0:
+        pytest.skip("no shared experts on the tensor-core path")
+    x = dev(inp["x"])
+    outs = []
+    for mix in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_MIX_SHARED", mix)
+        layer = MoeLayer.from_inputs(inp)
+        y = layer.forward(x)
+        assert api.read_device_status(layer.ws) == 0
+        outs.append((y.clone(), layer.stats.clone()))
+        del layer
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])

@@ -421,6 +421,29 @@ def test_layer_forward_both_tile_shapes(name, tile, swap, monkeypatch):
     assert rel_err(y.float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
 
 
+@pytest.mark.parametrize("name", ["mini_zen", "ragged_bf16", "mini_decode"])
+def test_mixed_shared_launch_is_bit_identical_to_separate_launches(name, monkeypatch):
+    """With CTA-pair tiles forced for both FFNs the shared experts run in the
+    routed experts' launches, their tiles interleaved with the routed ones;
+    each tile is computed as in separate launches, so the layer output and
+    the statistics are the same bytes.  Also against the oracle."""
+    monkeypatch.setenv("MOE_B200_GEMM_TILE", "256all")
+    cfg = SMALL[name]
+    inp = inputs(name)
+    logits32 = given_logits(cfg)
+    outs = []
+    for mix in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_MIX_SHARED", mix)
+        layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN)
+        layer.routing["logits"].copy_(torch.as_tensor(logits32))
+        y = layer.forward(dev(inp["x"]))
+        assert api.read_device_status(layer.ws) == 0
+        outs.append((y.clone(), layer.stats.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    assert rel_err(outs[0][0].float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
+
+
 def test_forward_host_pipelined_matches_device_forward():
     """MoeLayer.forward_host (host batches in and out, copies overlapped with
     the kernels on side streams) gives the same bytes as forward() per batch."""
