@@ -190,16 +190,17 @@ def algorithmic_flops(cfg, kept_pairs: int) -> dict:
 
 def shared_mixed(cfg, prob) -> bool:
     """True when the library runs the shared experts in the routed experts'
-    launches (BF16, shared experts, both on CTA-pair tiles: at least 256
-    expected rows per routed expert, T * K / E capped by the capacity, and
-    T >= 256), so the up and down stages cover both."""
+    launches (BF16, shared experts, both FFNs on the same tile shape: CTA
+    pairs for groups of at least 256 expected rows -- routed T * K / E capped
+    by the capacity, shared T -- single CTAs below), so the up and down stages
+    cover both."""
     if cfg.dtype != "bf16" or cfg.n_shared == 0 or os.environ.get("MOE_B200_MIX_SHARED", "1") == "0":
         return False
     expected = cfg.T * cfg.top_k // cfg.n_experts
     cap = api.capacity(prob)
     if cap >= 0:
         expected = min(expected, cap)
-    return api.max_rows(prob) > 0 and expected >= 256 and cfg.T >= 256
+    return api.max_rows(prob) > 0 and (expected >= 256) == (cfg.T >= 256)
 
 
 def shared_up_bytes(cfg) -> float:

@@ -105,7 +105,7 @@ struct TileCfg {
 
 template <int EPI, int BN, int STAGES>
 constexpr int gemm_smem_bytes() {
-  return STAGES * TileCfg<EPI, BN>::kStageBytes + 256 /*barriers + flags*/ + 4 * (kMaxGroups + 1) +
+  return STAGES * TileCfg<EPI, BN>::kStageBytes + 256 /*barriers + flags*/ + 8 * (kMaxGroups + 1) +
          1024 /*alignment slack*/;
 }
 
@@ -186,6 +186,22 @@ __device__ __forceinline__ void tile_prefix_warp(const GemmArgs& args, int n_til
     }
   }
   if (lane == 31) prefix[args.n_groups] = incl;
+}
+
+// Tile `tile` of a launch over two problems with t1 and total - t1 tiles: the
+// first problem's tiles are spread evenly through [0, total) (tile i is the
+// first problem's number floor(i t1 / total) when that count steps at i), so
+// every CTA's strided walk mixes both kinds in proportion.
+template <int BM>
+__device__ __forceinline__ TileInfo decode_mixed_tile(int tile, int t1, int total, const int* prefix,
+                                                      const int* prefix2, const GemmArgs& a1, const GemmArgs& a2,
+                                                      int out_cols) {
+  const int lo = static_cast<int>(static_cast<long long>(tile) * t1 / total);
+  const int hi = static_cast<int>(static_cast<long long>(tile + 1) * t1 / total);
+  if (hi > lo) return decode_tile<BM>(lo, prefix, a1, out_cols);
+  TileInfo ti = decode_tile<BM>(tile - lo, prefix2, a2, out_cols);
+  ti.second = true;
+  return ti;
 }
 
 // Drain one accumulator (this warp's 32 TMEM lanes, BN columns starting at
@@ -275,7 +291,8 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
 template <int EPI, int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const GemmArgs args) {
+                           const __grid_constant__ GemmArgs args, const __grid_constant__ CUtensorMap tmA_2,
+                           const __grid_constant__ CUtensorMap tmB_2, const __grid_constant__ GemmArgs args2) {
   using C = TileCfg<EPI, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -289,10 +306,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
+  int* prefix2 = prefix + kMaxGroups + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_tiles_n = (args.N + C::kOutCols - 1) / C::kOutCols;
+  const int n_tiles_n2 = (args2.N + C::kOutCols - 1) / C::kOutCols;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -310,6 +329,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    if (args2.n_groups > 0) {
+      prefetch_tensormap(&tmA_2);
+      prefetch_tensormap(&tmB_2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -318,12 +341,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_wait();  // everything above is local set-up; from here on the predecessor's outputs are read
   pdl_trigger();
   if (warp == 2) tile_prefix_warp<kBM>(args, n_tiles_n, prefix, lane);
+  if (warp == 3) {
+    if (args2.n_groups > 0)
+      tile_prefix_warp<kBM>(args2, n_tiles_n2, prefix2, lane);
+    else if (lane == 0)
+      prefix2[0] = 0;
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const int total_tiles = prefix[args.n_groups];
-  const int nkb_g = (args.K + kBK - 1) / kBK;
+  const int tiles1 = prefix[args.n_groups];
+  const int total_tiles = tiles1 + prefix2[max(args2.n_groups, 0)];
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -332,9 +361,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        const TileInfo ti = decode_tile<kBM>(tile, prefix, args, C::kOutCols);
+        const TileInfo ti = decode_mixed_tile<kBM>(tile, tiles1, total_tiles, prefix, prefix2, args, args2,
+                                                   C::kOutCols);
+        const GemmArgs& A = ti.second ? args2 : args;
+        const CUtensorMap* mA = ti.second ? &tmA_2 : &tmA;
+        const CUtensorMap* mB = ti.second ? &tmB_2 : &tmB;
+        const int nkb_g = (A.K + kBK - 1) / kBK;
         int k0, nkb;
-        tile_k_range(args, ti.g, &k0, &nkb);
+        tile_k_range(A, ti.g, &k0, &nkb);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
             ok = false;
@@ -345,14 +379,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* a_dst = sA + stage * C::kABytes;
           uint8_t* b_dst = sB + stage * C::kBBytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(a_dst, &tmA, &full[stage], kg * args.K + kk, ti.row0);
+          tma_load_2d(a_dst, mA, &full[stage], kg * A.K + kk, ti.row0);
           if (EPI == EPI_SWIGLU) {
-            tma_load_3d(b_dst, &tmB, &full[stage], kk, ti.n0, 2 * ti.g);
-            tma_load_3d(b_dst + C::kBBytes / 2, &tmB, &full[stage], kk, ti.n0, 2 * ti.g + 1);
+            tma_load_3d(b_dst, mB, &full[stage], kk, ti.n0, 2 * ti.g);
+            tma_load_3d(b_dst + C::kBBytes / 2, mB, &full[stage], kk, ti.n0, 2 * ti.g + 1);
           } else if (EPI == EPI_BF16) {
-            tma_load_3d(b_dst, &tmB, &full[stage], kk, ti.n0, ti.g * args.k_groups + kg);
+            tma_load_3d(b_dst, mB, &full[stage], kk, ti.n0, ti.g * A.k_groups + kg);
           } else {
-            tma_load_3d(b_dst, &tmB, &full[stage], kk, 0, 0);
+            tma_load_3d(b_dst, mB, &full[stage], kk, 0, 0);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -379,8 +413,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+        const TileInfo ti = decode_mixed_tile<kBM>(tile, tiles1, total_tiles, prefix, prefix2, args, args2,
+                                                   C::kOutCols);
         int k0, nkb;
-        tile_k_range(args, decode_tile<kBM>(tile, prefix, args, C::kOutCols).g, &k0, &nkb);
+        tile_k_range(ti.second ? args2 : args, ti.g, &k0, &nkb);
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
           ok = false;
           break;
@@ -419,7 +455,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int r = quarter * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile<kBM>(tile, prefix, args, C::kOutCols);
+      const TileInfo ti = decode_mixed_tile<kBM>(tile, tiles1, total_tiles, prefix, prefix2, args, args2,
+                                                 C::kOutCols);
       const int acc = it & 1;
       const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
       // every lane waits; the result is made warp-uniform (and the warp
@@ -429,7 +466,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after_sync();
       const int row = ti.row0 + r;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      epilogue_rows<EPI, BN>(args, ti.g, row, row < ti.row_end, ti.n0, t_row);
+      epilogue_rows<EPI, BN>(ti.second ? args2 : args, ti.g, row, row < ti.row_end, ti.n0, t_row);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -484,19 +521,10 @@ constexpr int pair_smem_bytes() {
   return kPairStages * kPairStageBytes + 256 + 8 * (kMaxGroups + 1) + kSwapXBytes + 1024;
 }
 
-// Tile `tile` of a launch over two problems with t1 and total - t1 tiles: the
-// first problem's tiles are spread evenly through [0, total) (tile i is the
-// first problem's number floor(i t1 / total) when that count steps at i), so
-// every pair's strided walk mixes both kinds in proportion.
 __device__ __forceinline__ TileInfo decode_pair_tile(int tile, int t1, int total, const int* prefix,
                                                      const int* prefix2, const GemmArgs& a1, const GemmArgs& a2,
                                                      int out_cols) {
-  const int lo = static_cast<int>(static_cast<long long>(tile) * t1 / total);
-  const int hi = static_cast<int>(static_cast<long long>(tile + 1) * t1 / total);
-  if (hi > lo) return decode_tile<kPairBM>(lo, prefix, a1, out_cols);
-  TileInfo ti = decode_tile<kPairBM>(tile - lo, prefix2, a2, out_cols);
-  ti.second = true;
-  return ti;
+  return decode_mixed_tile<kPairBM>(tile, t1, total, prefix, prefix2, a1, a2, out_cols);
 }
 
 // 128-deep k-blocks of one tile of a problem
@@ -962,9 +990,12 @@ static bool merged_k_ok(int64_t K) {
   return K % kBK == 0;
 }
 
+// (ta2, tb2, a2, tile_bound2): an optional second problem whose tiles the same
+// launch interleaves with the first's (see decode_mixed_tile).
 template <int EPI, int BN, int STAGES>
 static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& a, int64_t tile_bound,
-                    cudaStream_t st) {
+                    cudaStream_t st, const CUtensorMap* ta2 = nullptr, const CUtensorMap* tb2 = nullptr,
+                    const GemmArgs* a2 = nullptr, int64_t tile_bound2 = 0) {
   constexpr int smem = gemm_smem_bytes<EPI, BN, STAGES>();
   // the dynamic shared-memory opt-in is per device: set it once per device
   static std::mutex mu;
@@ -980,11 +1011,16 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
       done |= uint64_t(1) << dev;
     }
   }
+  const bool two = ta2 && tb2 && a2;
+  if (two) tile_bound += tile_bound2;
   if (tile_bound <= 0) return 0;
   int64_t grid = num_sms();
   if (grid > tile_bound) grid = tile_bound;
+  // without a second problem its maps are the first's (never read: no tiles)
+  GemmArgs b = two ? *a2 : a;
+  if (!two) b.n_groups = 0;
   return launch_k(grouped_gemm_tc_kernel<EPI, BN, STAGES>, dim3(static_cast<unsigned>(grid)), dim3(kGemmThreads),
-                  smem, st, ta, tb, a) == cudaSuccess ? 0 : -3;
+                  smem, st, ta, tb, a, two ? *ta2 : ta, two ? *tb2 : tb, b) == cudaSuccess ? 0 : -3;
 }
 
 // One problem of a pair-kernel launch: its tensor maps (see the kernel's
@@ -1332,6 +1368,76 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   return true;
 }
 
+// One problem of a single-CTA launch (128-row tiles).
+struct SingleProblem {
+  CUtensorMap ta, tb;
+  GemmArgs a;
+  int64_t tile_bound;
+};
+
+// Up/gate projection + SwiGLU on single CTAs: A = x_rows [n_rows, d], B = w13
+// [G, 2F, d] viewed as (d, F, 2G) with 128-row boxes (gate rows of group g at
+// 2g, up rows at 2g+1).
+static bool up_single_problem(const Problem& p, bool routed, const void* x_rows, int64_t n_rows,
+                              const int32_t* seg_off, const void* w13, void* h, void* gu, unsigned* status,
+                              SingleProblem* q) {
+  const int G = routed ? p.E : p.Ns;
+  const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
+  const uint32_t ba[2] = {kBK, kBM};
+  const uint64_t db[3] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.F), static_cast<uint64_t>(2 * G)};
+  const uint32_t bb[3] = {kBK, 128, 1};
+  if (!make_map(&q->ta, x_rows, 2, da, ba) || !make_map(&q->tb, w13, 3, db, bb)) return false;
+  GemmArgs& a = q->a;
+  a = GemmArgs{};
+  a.n_groups = G;
+  a.seg_off = routed ? seg_off : nullptr;
+  a.n_rows = static_cast<int>(n_rows);
+  a.N = p.F;
+  a.K = p.d;
+  a.k_groups = 1;
+  a.out = h;
+  a.ldo = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+  a.out_col_stride = routed ? 0 : p.F;
+  a.status = status;
+  a.swap_max = swap_max_rows();
+  a.gu = gu;
+  a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
+  a.gu_col_stride = routed ? 0 : 2 * p.F;
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
+  q->tile_bound = mt * cdiv(p.F, 128);
+  return true;
+}
+
+// Down projection on single CTAs: A = h [n_rows, k_groups * F], B = w2 [G, d, F]
+// viewed as (F, d, G) with 256-row boxes.
+static bool down_single_problem(const Problem& p, bool routed, const void* h, int64_t n_rows,
+                                const int32_t* seg_off, const void* w2, void* y_rows, unsigned* status,
+                                SingleProblem* q) {
+  const int G = routed ? p.E : p.Ns;
+  const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
+  const uint64_t da[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
+  const uint32_t ba[2] = {kBK, kBM};
+  const uint64_t db[3] = {static_cast<uint64_t>(p.F), static_cast<uint64_t>(p.d), static_cast<uint64_t>(G)};
+  const uint32_t bb[3] = {kBK, 256, 1};
+  if (!make_map(&q->ta, h, 2, da, ba) || !make_map(&q->tb, w2, 3, db, bb)) return false;
+  GemmArgs& a = q->a;
+  a = GemmArgs{};
+  a.n_groups = routed ? G : 1;
+  a.seg_off = routed ? seg_off : nullptr;
+  a.n_rows = static_cast<int>(n_rows);
+  a.N = p.d;
+  a.K = p.F;
+  a.k_groups = routed ? 1 : p.Ns;
+  a.out = y_rows;
+  a.ldo = p.d;
+  a.out_col_stride = 0;
+  a.status = status;
+  a.swap_max = swap_max_rows();
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
+  q->tile_bound = mt * cdiv(p.d, 256);
+  return true;
+}
+
 // mode 0: routed (groups = experts over seg_off); mode 1: shared (every row
 // through all N_s experts, summed).  h is scratch: [n_rows, F] (routed) or
 // [n_rows, N_s * F] (shared).
@@ -1373,24 +1479,9 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
         if (rc) return rc;
       }
     } else {
-      if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
-      GemmArgs a{};
-      a.n_groups = G;
-      a.seg_off = routed ? seg_off : nullptr;
-      a.n_rows = static_cast<int>(n_rows);
-      a.N = p.F;
-      a.K = p.d;
-      a.k_groups = 1;
-      a.out = h;
-      a.ldo = h_cols;
-      a.out_col_stride = routed ? 0 : p.F;
-      a.status = status;
-      a.swap_max = swap_max_rows();
-      a.gu = gu;
-      a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
-      a.gu_col_stride = routed ? 0 : 2 * p.F;
-      const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
-      const int rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, mt * cdiv(p.F, 128), st);
+      SingleProblem q;
+      if (!up_single_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, &q)) return -3;
+      const int rc = run_gemm<EPI_SWIGLU, 256, 4>(q.ta, q.tb, q.a, q.tile_bound, st);
       if (rc) return rc;
     }
     if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
@@ -1417,20 +1508,9 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
         if (rc) return rc;
       }
     } else {
-      GemmArgs a{};
-      a.n_groups = routed ? G : 1;
-      a.seg_off = routed ? seg_off : nullptr;
-      a.n_rows = static_cast<int>(n_rows);
-      a.N = p.d;
-      a.K = p.F;
-      a.k_groups = routed ? 1 : p.Ns;
-      a.out = y_rows;
-      a.ldo = p.d;
-      a.out_col_stride = 0;
-      a.status = status;
-      a.swap_max = swap_max_rows();
-      const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
-      const int rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, mt * cdiv(p.d, 256), st);
+      SingleProblem q;
+      if (!down_single_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, &q)) return -3;
+      const int rc = run_gemm<EPI_BF16, 256, 4>(q.ta, q.tb, q.a, q.tile_bound, st);
       if (rc) return rc;
     }
   }
@@ -1440,20 +1520,34 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
 bool expert_ffn_mixed_ok(const Problem& p) {
   const char* e = getenv("MOE_B200_MIX_SHARED");
   if (e && e[0] == '0') return false;
-  return p.dtype == kBF16 && p.Ns > 0 && p.max_rows > 0 && ffn_tile_mode(p, true, p.max_rows) == kTilePair &&
-         ffn_tile_mode(p, false, p.T) == kTilePair;
+  if (p.dtype != kBF16 || p.Ns <= 0 || p.max_rows <= 0) return false;
+  const int mr = ffn_tile_mode(p, true, p.max_rows), ms = ffn_tile_mode(p, false, p.T);
+  return mr == ms && mr != kTilePairTail;
 }
 
-// Routed and shared experts in the same two pair-kernel launches (up/gate +
-// SwiGLU for both, then both down projections): the routed tiles, bound by
-// the weight reads when the experts get few rows, share every SM's time with
-// the shared experts' tensor-core-bound tiles instead of running alone.
+// Routed and shared experts in the same two launches (up/gate + SwiGLU for
+// both, then both down projections), on CTA pairs or on single CTAs: no
+// launch of its own for the shared experts, whose few tiles (decode: one row
+// tile) would otherwise run on a handful of SMs while the rest wait.
 int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t* seg_off, const void* w13,
                             const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
                             const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
                             cudaStream_t st, cudaEvent_t after_up, int* n_kernels) {
   if (!expert_ffn_mixed_ok(p)) return -3;
   if (n_kernels) *n_kernels += 2;
+  if (ffn_tile_mode(p, true, p.max_rows) == kTileSingle) {
+    SingleProblem r, s;
+    if (!up_single_problem(p, true, x_perm, p.max_rows, seg_off, w13, h, gu, status, &r) ||
+        !up_single_problem(p, false, x, p.T, nullptr, w13_shared, h_shared, gu_shared, status, &s))
+      return -3;
+    if (int rc = run_gemm<EPI_SWIGLU, 256, 4>(r.ta, r.tb, r.a, r.tile_bound, st, &s.ta, &s.tb, &s.a, s.tile_bound))
+      return rc;
+    if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
+    if (!down_single_problem(p, true, h, p.max_rows, seg_off, w2, y_perm, status, &r) ||
+        !down_single_problem(p, false, h_shared, p.T, nullptr, w2_shared, y_shared, status, &s))
+      return -3;
+    return run_gemm<EPI_BF16, 256, 4>(r.ta, r.tb, r.a, r.tile_bound, st, &s.ta, &s.tb, &s.a, s.tile_bound);
+  }
   PairProblem r, s;
   if (!up_pair_problem(p, true, x_perm, p.max_rows, seg_off, w13, h, gu, status, false, &r) ||
       !up_pair_problem(p, false, x, p.T, nullptr, w13_shared, h_shared, gu_shared, status, false, &s))

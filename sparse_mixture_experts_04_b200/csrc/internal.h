@@ -99,8 +99,8 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
                       void* gu = nullptr);
 // Routed (x_perm over seg_off, p.max_rows rows) and shared (x, T rows)
 // experts in the same two launches, their tiles interleaved: requires
-// expert_ffn_mixed_ok(p) (BF16, shared experts, both on CTA-pair tiles;
-// MOE_B200_MIX_SHARED=0 turns it off).  gu / gu_shared: nullptr or the saved
+// expert_ffn_mixed_ok(p) (BF16, shared experts, both on the same tile shape:
+// CTA pairs or single CTAs; MOE_B200_MIX_SHARED=0 turns it off).  gu / gu_shared: nullptr or the saved
 // gate and up projections.
 bool expert_ffn_mixed_ok(const Problem& p);
 int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t* seg_off, const void* w13,

@@ -55,12 +55,13 @@ def test_router_and_combine_bytes_at_the_mixtral_shape():
     assert bench.combine_bytes(z, 0) == 2 * z.T * z.d_model * 2 + 8 * z.T * z.top_k
 
 
-@pytest.mark.parametrize("name,want", [("zen_fine", True), ("mixtral", False), ("skewed", False), ("decode", False),
+@pytest.mark.parametrize("name,want", [("zen_fine", True), ("mixtral", False), ("skewed", False), ("decode", True),
                                        ("tiny_fp32", False)])
 def test_shared_mixed_follows_the_library_rule(name, want, monkeypatch):
     """The shared experts share the routed launches only with BF16, shared
-    experts and CTA-pair tiles for both (>= 256 expected rows per routed
-    expert after the capacity, T >= 256); MOE_B200_MIX_SHARED=0 turns it off."""
+    experts and the same tile shape for both (CTA pairs: >= 256 expected rows
+    per routed expert after the capacity and T >= 256; single CTAs: both
+    below); MOE_B200_MIX_SHARED=0 turns it off."""
     from sparse_mixture_experts_04_b200 import api
     cfg = CONFIGS[name]
     prob = api.make_problem(cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.n_shared,

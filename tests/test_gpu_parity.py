@@ -421,13 +421,15 @@ def test_layer_forward_both_tile_shapes(name, tile, swap, monkeypatch):
     assert rel_err(y.float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
 
 
+@pytest.mark.parametrize("tile", ["256all", "128"])
 @pytest.mark.parametrize("name", ["mini_zen", "ragged_bf16", "mini_decode"])
-def test_mixed_shared_launch_is_bit_identical_to_separate_launches(name, monkeypatch):
-    """With CTA-pair tiles forced for both FFNs the shared experts run in the
-    routed experts' launches, their tiles interleaved with the routed ones;
-    each tile is computed as in separate launches, so the layer output and
-    the statistics are the same bytes.  Also against the oracle."""
-    monkeypatch.setenv("MOE_B200_GEMM_TILE", "256all")
+def test_mixed_shared_launch_is_bit_identical_to_separate_launches(name, tile, monkeypatch):
+    """With one tile shape forced for both FFNs (CTA pairs, or single CTAs)
+    the shared experts run in the routed experts' launches, their tiles
+    interleaved with the routed ones; each tile is computed as in separate
+    launches, so the layer output and the statistics are the same bytes.
+    Also against the oracle."""
+    monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
     cfg = SMALL[name]
     inp = inputs(name)
     logits32 = given_logits(cfg)
