@@ -1118,7 +1118,7 @@ int router_k_splits(const Problem& p) {
   int64_t s = num_sms() / tiles;
   const int64_t max_by_k = p.d / 256;  // keep at least four 64-wide k-blocks per slice
   if (s > max_by_k) s = max_by_k;
-  if (s > 8) s = 8;
+  if (s > kMaxLogitParts) s = kMaxLogitParts;
   if (s < 1) s = 1;
   const int64_t len = cdiv(cdiv(p.d, s), kBK) * kBK;
   return static_cast<int>(cdiv(p.d, len));

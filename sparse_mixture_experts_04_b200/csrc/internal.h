@@ -14,6 +14,7 @@ constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 32;
 constexpr int kDispatchChunk = 256;  // tokens per block in the dispatch kernels
 constexpr int kSelectTokens = 8;     // tokens per block in the selection kernel (one per warp)
+constexpr int kMaxLogitParts = 8;    // most slices of the split-K gate GEMM
 
 enum Dtype { kBF16 = 0, kF32 = 1 };
 

@@ -172,24 +172,41 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
     const int64_t t = tok_begin + warp * kPerWarp + n;
     if (t >= T) break;
     float lg[EPL];
+    float bias[EPL];
+    // every load of the token first (the slices, the biases), then the adds
+    // in slice order: the loads' latencies overlap instead of queueing
+    if (n_parts > 0) {  // split-K gate GEMM: add the slices in order
+      float pv[kMaxLogitParts][EPL];
+#pragma unroll
+      for (int sl = 0; sl < kMaxLogitParts; ++sl)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          pv[sl][i] = (sl < n_parts && e < E) ? parts[static_cast<int64_t>(sl) * T * E + t * E + e] : 0.f;
+        }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) bias[i] = (sel_bias && lane + 32 * i < E) ? sel_bias[lane + 32 * i] : 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        float v = 0.f;
+#pragma unroll
+        for (int sl = 0; sl < kMaxLogitParts; ++sl)
+          if (sl < n_parts) v += pv[sl][i];
+        if (e < E) logits[t * E + e] = v;
+        lg[i] = e < E ? v : -INFINITY;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        lg[i] = e < E ? logits[t * E + e] : -INFINITY;
+        bias[i] = (sel_bias && e < E) ? sel_bias[e] : 0.f;
+      }
+    }
     float mloc = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) {
-        if (n_parts > 0) {  // split-K gate GEMM: add the slices in order
-          float v = 0.f;
-          for (int sl = 0; sl < n_parts; ++sl) v += parts[static_cast<int64_t>(sl) * T * E + t * E + e];
-          logits[t * E + e] = v;
-          lg[i] = v;
-        } else {
-          lg[i] = logits[t * E + e];
-        }
-      } else {
-        lg[i] = -INFINITY;
-      }
-      mloc = fmaxf(mloc, lg[i]);
-    }
+    for (int i = 0; i < EPL; ++i) mloc = fmaxf(mloc, lg[i]);
     const float m = warp_max(mloc);
     float ex[EPL];
     float zloc = 0.f;
@@ -209,20 +226,23 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
     int my_e = -1;
     float my_ex = 0.f;
     bool done = false;
-    if (sel_bias != nullptr && !bias_on_logit) {
-      // Bias on p: rank the float32 scores s = ex/Z + b first (K+1 rounds over
-      // 32-bit keys).  Each is within d = (E+8) eps p + eps (|s| + 1) of the
-      // exact p + b (eps = 2^-23; terms: expf's 2 ulp, the sum Z, 1/Z, the
-      // product, the add, and the rounding of l - m, whose effect on p is at
-      // most eps |l - m| p / 2 <= eps / (2e)); if every gap between
-      // consecutive ones of the best K+1 exceeds 2d, the exact ranking of the
-      // top K is the same, else the token is ranked again in float64 below.
+    if (sel_bias == nullptr || !bias_on_logit) {
+      // Ranked on 32-bit keys of float32 scores.  Without a bias the score is
+      // the float32 logit itself, so this ranking is the exact one (K rounds).
+      // Bias on p: the float32 scores s = ex/Z + b (K+1 rounds).  Each is
+      // within d = (E+8) eps p + eps (|s| + 1) of the exact p + b (eps =
+      // 2^-23; terms: expf's 2 ulp, the sum Z, 1/Z, the product, the add, and
+      // the rounding of l - m, whose effect on p is at most eps |l - m| p / 2
+      // <= eps / (2e)); if every gap between consecutive ones of the best K+1
+      // exceeds 2d, the exact ranking of the top K is the same, else the
+      // token is ranked again in float64 below.
+      const bool biased = sel_bias != nullptr;
       unsigned k32[EPL];
       float s32[EPL];
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        float sc = (e < E) ? ex[i] * invZ + sel_bias[e] : 0.f;
+        float sc = (e < E) ? (biased ? ex[i] * invZ + bias[i] : lg[i]) : 0.f;
         if (sc != sc) sc = -INFINITY;
         sc += 0.0f;
         s32[i] = sc;
@@ -238,7 +258,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
           bi = i;
         }
       float my_s = 0.f, my_p = 0.f;
-      for (int r = 0; r <= K && r < 32; ++r) {
+      const int rounds = biased ? K + 1 : K;
+      for (int r = 0; r < rounds && r < 32; ++r) {
         const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
         const int best_e = __reduce_min_sync(0xffffffffu, (bk != 0u && bk == kmax) ? lane + 32 * bi : 0x7fffffff);
         const int wl = best_e & 31;
@@ -279,7 +300,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
                       eps * (fmaxf(fabsf(my_s), fabsf(s_next)) + 1.0f);
       // with K == E there is no (K+1)-th score: the last gap only orders the set
       const bool last_ok = lane == K - 1 && K == E;
-      const bool gap_ok = lane >= K || last_ok || (my_s - s_next > 2.0f * d);
+      const bool gap_ok = !biased || lane >= K || last_ok || (my_s - s_next > 2.0f * d);
       done = __all_sync(0xffffffffu, gap_ok);
       if (!done) {
         my_e = -1;
@@ -295,7 +316,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   #pragma unroll
         for (int i = 0; i < EPL; ++i) {
           const int e = lane + 32 * i;
-          score[i] = (e < E) ? static_cast<double>(lg[i]) + static_cast<double>(sel_bias[e]) : -INFINITY;
+          score[i] = (e < E) ? static_cast<double>(lg[i]) + static_cast<double>(bias[i]) : -INFINITY;
         }
       } else {
         const double m64 = static_cast<double>(m);
@@ -311,7 +332,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   #pragma unroll
         for (int i = 0; i < EPL; ++i) {
           const int e = lane + 32 * i;
-          score[i] = (e < E) ? ex64[i] / z64 + static_cast<double>(sel_bias[e]) : -INFINITY;
+          score[i] = (e < E) ? ex64[i] / z64 + static_cast<double>(bias[i]) : -INFINITY;
         }
       }
 
