@@ -103,10 +103,13 @@ struct TileCfg {
                                    : (2 * BN <= 256) ? 256 : 512;
 };
 
+// FP32 epilogue staging: one 32 x 32 float block per epilogue warp
+constexpr int kF32StageBytes = 4 * 32 * 32 * 4;
+
 template <int EPI, int BN, int STAGES>
 constexpr int gemm_smem_bytes() {
   return STAGES * TileCfg<EPI, BN>::kStageBytes + 256 /*barriers + flags*/ + 8 * (kMaxGroups + 1) +
-         1024 /*alignment slack*/;
+         (EPI == EPI_F32 ? kF32StageBytes + 16 : 0) + 1024 /*alignment slack*/;
 }
 
 struct TileInfo {
@@ -288,6 +291,35 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
   }
 }
 
+// FP32 epilogue through shared memory: each 32-column block of this warp's 32
+// accumulator rows goes lane-per-row into xw (XOR-swizzled, no bank
+// conflicts) and out lane-per-column, so every store instruction writes 32
+// consecutive floats of one row instead of one float of 32 rows.
+template <int BN>
+__device__ __forceinline__ void epilogue_f32_staged(const GemmArgs& args, int g, int row_base, int row_end,
+                                                    uint32_t t_row, int lane, float* xw) {
+  float* obase = static_cast<float*>(args.out) + static_cast<int64_t>(g) * args.out_group_stride;
+  const float* add = (g == 0) ? args.col_add : nullptr;  // a split-K offset goes into slice 0 only
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    uint32_t v[32];
+    tmem_load_32x32(t_row + c, v);
+    tmem_load_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) xw[lane * 32 + (j ^ lane)] = __uint_as_float(v[j]);
+    __syncwarp();
+    const int col = c + lane;
+    const bool col_ok = col < args.N;
+    const float ad = (add && col_ok) ? add[col] : 0.f;
+#pragma unroll 4
+    for (int rr = 0; rr < 32; ++rr) {
+      const int row = row_base + rr;
+      if (col_ok && row < row_end) obase[static_cast<int64_t>(row) * args.ldo + col] = xw[rr * 32 + (lane ^ rr)] + ad;
+    }
+    __syncwarp();
+  }
+}
+
 template <int EPI, int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -307,6 +339,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* prefix = reinterpret_cast<int*>(tmem_slot + 4);
   int* prefix2 = prefix + kMaxGroups + 1;
+  float* xw_all = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(prefix2 + kMaxGroups + 1) + 15) & ~uintptr_t(15));
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -466,7 +499,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after_sync();
       const int row = ti.row0 + r;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      epilogue_rows<EPI, BN>(ti.second ? args2 : args, ti.g, row, row < ti.row_end, ti.n0, t_row);
+      if (EPI == EPI_F32)
+        epilogue_f32_staged<BN>(ti.second ? args2 : args, ti.g, ti.row0 + quarter * 32, ti.row_end, t_row, lane,
+                                xw_all + quarter * 32 * 32);
+      else
+        epilogue_rows<EPI, BN>(ti.second ? args2 : args, ti.g, row, row < ti.row_end, ti.n0, t_row);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
