@@ -249,50 +249,58 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
         const unsigned b = __float_as_uint(sc);
         k32[i] = e >= E ? 0u : ((b >> 31) ? ~b : (b | 0x80000000u));
       }
-      unsigned bk = 0;
-      int bi = 0;
+      // this lane's keys in descending order with their slots (equal keys:
+      // the lower slot, i.e. expert, first): a round only pops the winner's head
+      unsigned hk[EPL];
+      int hs[EPL];
 #pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (k32[i] > bk) {
-          bk = k32[i];
-          bi = i;
-        }
-      float my_s = 0.f, my_p = 0.f;
+      for (int i = 0; i < EPL; ++i) {
+        hk[i] = k32[i];
+        hs[i] = i;
+      }
+#pragma unroll
+      for (int pass = 0; pass < EPL; ++pass)
+#pragma unroll
+        for (int i = pass & 1; i + 1 < EPL; i += 2)
+          if (hk[i + 1] > hk[i]) {  // slots start ascending and equal keys never swap
+            const unsigned tk = hk[i];
+            hk[i] = hk[i + 1];
+            hk[i + 1] = tk;
+            const int ts = hs[i];
+            hs[i] = hs[i + 1];
+            hs[i + 1] = ts;
+          }
       const int rounds = biased ? K + 1 : K;
       for (int r = 0; r < rounds && r < 32; ++r) {
-        const unsigned kmax = __reduce_max_sync(0xffffffffu, bk);
-        const int best_e = __reduce_min_sync(0xffffffffu, (bk != 0u && bk == kmax) ? lane + 32 * bi : 0x7fffffff);
-        const int wl = best_e & 31;
-        float ex_mine = 0.f, s_mine = 0.f;
+        const unsigned kmax = __reduce_max_sync(0xffffffffu, hk[0]);
+        const int best_e =
+            __reduce_min_sync(0xffffffffu, (hk[0] != 0u && hk[0] == kmax) ? lane + 32 * hs[0] : 0x7fffffff);
+        if (lane == (best_e & 31)) {
 #pragma unroll
-        for (int i = 0; i < EPL; ++i)
-          if (i == bi) {
-            ex_mine = ex[i];
-            s_mine = s32[i];
+          for (int i = 0; i + 1 < EPL; ++i) {
+            hk[i] = hk[i + 1];
+            hs[i] = hs[i + 1];
           }
-        const float ex_sel = __shfl_sync(0xffffffffu, ex_mine, wl);
-        const float s_sel = __shfl_sync(0xffffffffu, s_mine, wl);
-        if (lane == wl) {
-          bk = 0;
-#pragma unroll
-          for (int i = 0; i < EPL; ++i)
-            if (i == bi) k32[i] = 0u;
-          bi = 0;
-#pragma unroll
-          for (int i = 0; i < EPL; ++i)
-            if (k32[i] > bk) {
-              bk = k32[i];
-              bi = i;
-            }
+          hk[EPL - 1] = 0u;
         }
-        if (lane == r) {
-          my_e = best_e;
-          my_ex = ex_sel;
-          my_s = s_sel;
-          my_p = ex_sel * invZ;
-        }
+        if (lane == r) my_e = best_e;
         if (best_e == 0x7fffffff) break;  // fewer than K+1 experts (K == E)
       }
+      // the winners' ex and score: expert e sits in lane e & 31, slot e >> 5
+      float my_s = 0.f;
+      {
+        const int src = my_e & 31, slot = my_e >> 5;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const float a = __shfl_sync(0xffffffffu, ex[i], src);
+          const float b = __shfl_sync(0xffffffffu, s32[i], src);
+          if (i == slot) {
+            my_ex = a;
+            my_s = b;
+          }
+        }
+      }
+      const float my_p = my_ex * invZ;
       const float s_next = __shfl_down_sync(0xffffffffu, my_s, 1);
       const float p_next = __shfl_down_sync(0xffffffffu, my_p, 1);
       const float eps = 1.1920928955078125e-7f;  // 2^-23
