@@ -79,6 +79,9 @@ struct GemmArgs {
   // stage with one box (K a multiple of 64): A maps (64, rows, K/64), B maps
   // (64, rows, groups, K/64); 0: one 2-D / 3-D box per chunk
   int merged_k;
+  // pair kernel, merged maps: swap tiles of at most 64 token rows take
+  // 192-deep stages (tokens and weights of three chunks in one stage slot)
+  int deep_swap;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -543,6 +546,18 @@ constexpr int kPairChunk = 128 * kBK * 2;  // one 128-row, 64-deep chunk: 16 KB
 constexpr int kPairABytes = kPairKC * kPairChunk;
 constexpr int kPairBBytes = kPairKC * kPairChunk;  // this CTA's half of B
 constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
+// A deep swap stage (swap tiles of at most 64 token rows, merged maps): three
+// 64-deep chunks in one 64 KB stage slot, the tokens (3 x at most 32 rows per
+// CTA, 12 KB) at its start and the weights (3 x 16 KB) in its last 48 KB.
+// Copy-bound swap tiles then keep 1.7x the bytes in flight per SM.
+constexpr int kDeepKC = 3;
+constexpr int kDeepWOffset = kPairStageBytes - kDeepKC * kPairChunk;
+static_assert(kDeepKC * 32 * kBK * 2 <= kDeepWOffset, "deep swap tokens overlap the weights");
+
+// 64-deep chunks per stage of a tile whose token box is a_box rows
+__device__ __forceinline__ int pair_tile_kc(const GemmArgs& a, const TileInfo& ti, int a_box) {
+  return (a.deep_swap && a.merged_k && ti.swap && a_box <= 32) ? kDeepKC : kPairKC;
+}
 
 // Swap-tile epilogues transpose through shared memory, 32 tokens at a time:
 // xbuf[token][TMEM lane] (row stride 132 floats keeps 16-byte alignment).
@@ -564,9 +579,9 @@ __device__ __forceinline__ TileInfo decode_pair_tile(int tile, int t1, int total
   return decode_mixed_tile<kPairBM>(tile, t1, total, prefix, prefix2, a1, a2, out_cols);
 }
 
-// 128-deep k-blocks of one tile of a problem
-__device__ __forceinline__ int pair_nkb(const GemmArgs& a) {
-  return ((a.K + kBK * kPairKC - 1) / (kBK * kPairKC)) * a.k_groups;
+// k-blocks (kc chunks of 64 deep) of one tile of a problem
+__device__ __forceinline__ int pair_nkb(const GemmArgs& a, int kc) {
+  return ((a.K + kBK * kc - 1) / (kBK * kc)) * a.k_groups;
 }
 
 // MMA N of a swap tile covering `rows` (1..256) token rows: a multiple of 16.
@@ -658,13 +673,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                              const __grid_constant__ CUtensorMap tmA_2, const __grid_constant__ CUtensorMap tmB_2,
                              const __grid_constant__ CUtensorMap tmA64_2, const __grid_constant__ CUtensorMap tmB64_2,
                              const __grid_constant__ CUtensorMap tmA32_2, const __grid_constant__ CUtensorMap tmA16_2,
-                             const __grid_constant__ GemmArgs args2) {
+                             const __grid_constant__ GemmArgs args2,
+                             const __grid_constant__ CUtensorMap tmA32d, const __grid_constant__ CUtensorMap tmA16d,
+                             const __grid_constant__ CUtensorMap tmB64d, const __grid_constant__ CUtensorMap tmA32d_2,
+                             const __grid_constant__ CUtensorMap tmA16d_2, const __grid_constant__ CUtensorMap tmB64d_2) {
   constexpr int kOutCols = (EPI == EPI_SWIGLU) ? kPairBN / 2 : kPairBN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + kPairStages * kPairABytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kPairStages * kPairBBytes);
+  // stage s: smem + s * kPairStageBytes (tokens / A rows first, then weights)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
@@ -711,6 +728,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       prefetch_tensormap(&tmA16_2);
       prefetch_tensormap(&tmB64_2);
     }
+    if (args.deep_swap) {
+      prefetch_tensormap(&tmA32d);
+      prefetch_tensormap(&tmA16d);
+      prefetch_tensormap(&tmB64d);
+      if (args2.n_groups > 0) {
+        prefetch_tensormap(&tmA32d_2);
+        prefetch_tensormap(&tmA16d_2);
+        prefetch_tensormap(&tmB64d_2);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -746,7 +773,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const CUtensorMap* mA = ti.second ? &tmA_2 : &tmA;
         const CUtensorMap* mB = ti.second ? &tmB_2 : &tmB;
         const CUtensorMap* mB64 = ti.second ? &tmB64_2 : &tmB64;
-        const int nkb_g = (A.K + kBK * kPairKC - 1) / (kBK * kPairKC);
+        // a swap tile's N token rows are split N/2 per CTA; the box (16, 32,
+        // 64 or 128 rows) may load more, the MMA reads the first N/2
+        const int half_n = ti.swap ? swap_n(ti.row_end - ti.row0) / 2 : 128;
+        const int a_box = ti.swap ? swap_box_rows(half_n) : 128;
+        const int kc = pair_tile_kc(A, ti, a_box);
+        const bool deep = kc == kDeepKC;
+        const int nkb_g = (A.K + kBK * kc - 1) / (kBK * kc);
         const int nkb = nkb_g * A.k_groups;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
@@ -754,20 +787,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           const int kg = kb / nkb_g;
-          const int kk0 = (kb - kg * nkb_g) * kBK * kPairKC;
+          const int kk0 = (kb - kg * nkb_g) * kBK * kc;
           const uint32_t bar = full_leader + static_cast<uint32_t>(stage * 8);
-          // a swap tile's N token rows are split N/2 per CTA; the box (16, 32,
-          // 64 or 128 rows) may load more, the MMA reads the first N/2
-          const int half_n = ti.swap ? swap_n(ti.row_end - ti.row0) / 2 : 128;
-          const int a_box = ti.swap ? swap_box_rows(half_n) : 128;
-          const CUtensorMap* a_map = a_box == 16   ? (ti.second ? &tmA16_2 : &tmA16)
-                                     : a_box == 32 ? (ti.second ? &tmA32_2 : &tmA32)
+          const CUtensorMap* a_map = a_box == 16   ? (deep ? (ti.second ? &tmA16d_2 : &tmA16d) : (ti.second ? &tmA16_2 : &tmA16))
+                                     : a_box == 32 ? (deep ? (ti.second ? &tmA32d_2 : &tmA32d) : (ti.second ? &tmA32_2 : &tmA32))
                                      : a_box == 64 ? (ti.second ? &tmA64_2 : &tmA64)
                                                    : mA;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kPairKC * (kPairChunk + a_box * kBK * 2));
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kc * (kPairChunk + a_box * kBK * 2));
           const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
-          uint8_t* a_dst = sA + stage * kPairABytes;
-          uint8_t* b_dst = sB + stage * kPairBBytes;
+          uint8_t* a_dst = smem + stage * kPairStageBytes;
+          uint8_t* b_dst = a_dst + (deep ? kDeepWOffset : kPairABytes);
           // Swap tiles are bound by the copies, not the MMAs: with merged maps
           // (args.merged_k) each of their operands comes in one box spanning
           // both 64-deep chunks (the tokens' chunk c at c * a_box rows, the
@@ -783,10 +812,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                a_row);
           }
           if (merge) {
+            const CUtensorMap* wmap = deep ? (ti.second ? &tmB64d_2 : &tmB64d) : mB64;
             if (EPI == EPI_SWIGLU)  // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
-              tma_load_4d_pair(b_dst, mB64, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
+              tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
             else
-              tma_load_4d_pair(b_dst, mB64, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * A.k_groups + kg,
+              tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * A.k_groups + kg,
                                kk0 / kBK);
           } else {
 #pragma unroll
@@ -833,12 +863,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int it = 0;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
         const TileInfo ti = decode_pair_tile(tile, tiles1, total_tiles, prefix, prefix2, args, args2, kOutCols);
-        const int nkb = pair_nkb(ti.second ? args2 : args);
+        const int a_box = ti.swap ? swap_box_rows(swap_n(ti.row_end - ti.row0) / 2) : 128;
+        const int kc = pair_tile_kc(ti.second ? args2 : args, ti, a_box);
+        const int nkb = pair_nkb(ti.second ? args2 : args, kc);
+        const int w_off = kc == kDeepKC ? kDeepWOffset : kPairABytes;
         // normal tile: A = token rows (M = 256), B = weight rows (N = 256);
         // swap tile: A = weight rows (M = 256), B = the tile's N token rows
         const uint32_t idesc = idesc_bf16_f32(kPairBM, ti.swap ? swap_n(ti.row_end - ti.row0) : kPairBN);
         // the token operand's chunks sit a_box rows apart (see the producer)
-        const int a_chunk = (ti.swap ? swap_box_rows(swap_n(ti.row_end - ti.row0) / 2) : 128) * kBK * 2;
+        const int a_chunk = a_box * kBK * 2;
         const int acc = it & 1;
         const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
@@ -853,10 +886,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           tc_fence_after_sync();
+          uint8_t* st_base = smem + stage * kPairStageBytes;
 #pragma unroll
-          for (int c = 0; c < kPairKC; ++c) {
-            const uint64_t tdesc = smem_desc_k128(smem_addr(sA + stage * kPairABytes + c * a_chunk));
-            const uint64_t wdesc = smem_desc_k128(smem_addr(sB + stage * kPairBBytes + c * kPairChunk));
+          for (int c = 0; c < kDeepKC; ++c) {
+            if (c >= kc) break;
+            const uint64_t tdesc = smem_desc_k128(smem_addr(st_base + c * a_chunk));
+            const uint64_t wdesc = smem_desc_k128(smem_addr(st_base + w_off + c * kPairChunk));
             const uint64_t adesc = ti.swap ? wdesc : tdesc;
             const uint64_t bdesc = ti.swap ? tdesc : wdesc;
 #pragma unroll
@@ -982,7 +1017,8 @@ bool make_map_strided(CUtensorMap* m, const void* base, int rank, const uint64_t
 // merged chunks one box spanning both 64-deep chunks of a stage,
 // (64, rows, cols/64) with the chunk stride 128 bytes.
 static bool make_token_maps(CUtensorMap* t128, CUtensorMap* t64, CUtensorMap* t32, CUtensorMap* t16,
-                            const void* base, int64_t cols, int64_t rows, bool merged) {
+                            CUtensorMap* t32d, CUtensorMap* t16d, const void* base, int64_t cols, int64_t rows,
+                            bool merged) {
   const uint64_t d2[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
   const uint32_t b128[2] = {kBK, 128};
   if (!make_map(t128, base, 2, d2, b128)) return false;
@@ -999,6 +1035,21 @@ static bool make_token_maps(CUtensorMap* t128, CUtensorMap* t64, CUtensorMap* t3
       if (!make_map(maps[i], base, 2, d2, b)) return false;
     }
   }
+  // deep swap stages: 32- and 16-row boxes spanning three chunks (merged only;
+  // otherwise copies that no tile reads)
+  if (!merged) {
+    *t32d = *t32;
+    *t16d = *t16;
+    return true;
+  }
+  CUtensorMap* dmaps[2] = {t32d, t16d};
+  const uint32_t dheights[2] = {32, 16};
+  for (int i = 0; i < 2; ++i) {
+    const uint64_t d[3] = {static_cast<uint64_t>(kBK), static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / kBK)};
+    const uint64_t st[2] = {static_cast<uint64_t>(cols) * 2, static_cast<uint64_t>(kBK) * 2};
+    const uint32_t b[3] = {kBK, dheights[i], static_cast<uint32_t>(kDeepKC)};
+    if (!make_map_strided(dmaps[i], base, 3, d, st, b)) return false;
+  }
   return true;
 }
 
@@ -1006,13 +1057,13 @@ static bool make_token_maps(CUtensorMap* t128, CUtensorMap* t64, CUtensorMap* t3
 // merged (64, rows, groups, K/64) with box (64, box_rows, box_groups, 2);
 // else (K, rows, groups) with box (64, box_rows, 1).
 static bool make_weight_map(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int64_t groups,
-                            uint32_t box_rows, uint32_t box_groups, bool merged) {
+                            uint32_t box_rows, uint32_t box_groups, bool merged, int chunks = kPairKC) {
   if (merged) {
     const uint64_t d[4] = {static_cast<uint64_t>(kBK), static_cast<uint64_t>(rows), static_cast<uint64_t>(groups),
                            static_cast<uint64_t>(K / kBK)};
     const uint64_t st[3] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K * rows) * 2,
                             static_cast<uint64_t>(kBK) * 2};
-    const uint32_t b[4] = {kBK, box_rows, box_groups, static_cast<uint32_t>(kPairKC)};
+    const uint32_t b[4] = {kBK, box_rows, box_groups, static_cast<uint32_t>(chunks)};
     return make_map_strided(m, base, 4, d, st, b);
   }
   const uint64_t d[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(rows), static_cast<uint64_t>(groups)};
@@ -1064,6 +1115,7 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
 // parameters), arguments and an upper bound on its tiles.
 struct PairProblem {
   CUtensorMap ta, tb, ta64, tb64, ta32, ta16;
+  CUtensorMap ta32d, ta16d, tb64d;  // deep swap stages (three chunks per box)
   GemmArgs a;
   int64_t tile_bound;
 };
@@ -1107,7 +1159,7 @@ static int run_pair_gemm(const PairProblem& p1, const PairProblem* p2, cudaStrea
   if (!p2) a2.n_groups = 0;
   return launch_k(grouped_gemm_pair_kernel<EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads), smem,
                   st, p1.ta, p1.tb, p1.ta64, p1.tb64, p1.ta32, p1.ta16, p1.a, q.ta, q.tb, q.ta64, q.tb64, q.ta32,
-                  q.ta16, a2) == cudaSuccess ? 0 : -3;
+                  q.ta16, a2, p1.ta32d, p1.ta16d, p1.tb64d, q.ta32d, q.ta16d, q.tb64d) == cudaSuccess ? 0 : -3;
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -1132,6 +1184,13 @@ enum TileMode { kTileSingle = 0, kTilePairTail = 1, kTilePair = 2 };
 // (0..255) overrides; 0 turns swap tiles off.  Measured: with at most 128
 // rows a swap tile is clearly cheaper than a 256-row tile; near 256 rows it
 // is not (the transposing epilogue costs more than the padding saves).
+// Deep (192-deep) stages for swap tiles of at most 64 token rows
+// (MOE_B200_DEEP_SWAP=0 turns them off).
+static bool deep_swap_on() {
+  const char* e = getenv("MOE_B200_DEEP_SWAP");
+  return !(e && e[0] == '0');
+}
+
 static int swap_max_rows() {
   const char* e = getenv("MOE_B200_SWAP_MAX");
   if (e && *e) {
@@ -1346,10 +1405,15 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
                             PairProblem* q) {
   const int G = routed ? p.E : p.Ns;
   const bool merged = merged_k_ok(p.d);
-  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, x_rows, p.d, n_rows, merged) ||
+  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, x_rows, p.d, n_rows, merged) ||
       !make_weight_map(&q->tb, w13, p.d, p.F, 2 * G, 128, 1, false) ||
       !make_weight_map(&q->tb64, w13, p.d, p.F, 2 * G, 64, merged ? 2 : 1, merged))
     return false;
+  if (merged) {
+    if (!make_weight_map(&q->tb64d, w13, p.d, p.F, 2 * G, 64, 2, true, kDeepKC)) return false;
+  } else {
+    q->tb64d = q->tb64;
+  }
   GemmArgs& a = q->a;
   a = GemmArgs{};
   a.n_groups = G;
@@ -1368,6 +1432,7 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
   a.gu_col_stride = routed ? 0 : 2 * p.F;
   a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
   a.merged_k = merged ? 1 : 0;
+  a.deep_swap = merged && deep_swap_on() ? 1 : 0;
   const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
   q->tile_bound = (mt / 2 + G) * cdiv(p.F, 128);
   return true;
@@ -1381,10 +1446,15 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
   const bool merged = merged_k_ok(p.F);
-  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, h, h_cols, n_rows, merged) ||
+  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, h, h_cols, n_rows, merged) ||
       !make_weight_map(&q->tb, w2, p.F, p.d, G, 128, 1, false) ||
       !make_weight_map(&q->tb64, w2, p.F, p.d, G, 128, 1, merged))
     return false;
+  if (merged) {
+    if (!make_weight_map(&q->tb64d, w2, p.F, p.d, G, 128, 1, true, kDeepKC)) return false;
+  } else {
+    q->tb64d = q->tb64;
+  }
   GemmArgs& a = q->a;
   a = GemmArgs{};
   a.n_groups = routed ? G : 1;
@@ -1400,6 +1470,7 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   a.swap_max = swap_max_rows();
   a.row_mode = tail ? 1 : 0;
   a.merged_k = merged ? 1 : 0;
+  a.deep_swap = merged && deep_swap_on() ? 1 : 0;
   const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
   q->tile_bound = (mt / 2 + a.n_groups) * cdiv(p.d, 256);
   return true;

@@ -446,6 +446,29 @@ def test_mixed_shared_launch_is_bit_identical_to_separate_launches(name, tile, m
     assert rel_err(outs[0][0].float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
 
 
+@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "mini_skewed", "mini_decode", "ragged_bf16"])
+def test_deep_swap_stages_are_bit_identical(name, monkeypatch):
+    """Swap tiles of at most 64 token rows take 192-deep stages (three 64-deep
+    chunks per stage slot); the MMAs run in the same k order, so the layer
+    output is the same bytes as with 128-deep stages (MOE_B200_DEEP_SWAP=0),
+    with pair tiles forced and every remainder of up to 128 rows swapped."""
+    monkeypatch.setenv("MOE_B200_GEMM_TILE", "256all")
+    cfg = SMALL[name]
+    inp = inputs(name)
+    logits32 = given_logits(cfg)
+    outs = []
+    for deep in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_DEEP_SWAP", deep)
+        layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN)
+        layer.routing["logits"].copy_(torch.as_tensor(logits32))
+        y = layer.forward(dev(inp["x"]))
+        assert api.read_device_status(layer.ws) == 0
+        outs.append(y.clone())
+    assert torch.equal(outs[0], outs[1])
+    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
+    assert rel_err(outs[0].float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
+
+
 def test_forward_host_pipelined_matches_device_forward():
     """MoeLayer.forward_host (host batches in and out, copies overlapped with
     the kernels on side streams) gives the same bytes as forward() per batch."""
