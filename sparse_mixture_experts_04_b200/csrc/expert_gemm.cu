@@ -22,6 +22,9 @@
 // (128 or 256) columns, enumerated group-major, then column tile, then row
 // tile, so CTAs running at the same time share weight tiles through L2.
 // Persistent CTAs (one per SM) walk the tile list with a stride of the grid.
+// A launch may carry a second problem (its own tensor maps, arguments and
+// tile prefix; the layer puts the shared experts there): the first problem's
+// tiles are spread evenly through the combined tile list (decode_mixed_tile).
 //
 // Warp roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring of
 // shared-memory stages; warp 1 allocates TMEM and issues the MMAs from one
@@ -533,7 +536,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   empty[s]  (each)    one arrive from the leader's multicast commit
 //   tfull[a]  (each)    one arrive from the leader's multicast commit
 //   tempty[a] (leader)  8 arrives: 4 epilogue warps in each CTA
-// Tiles are 256 rows; a group with r rows spans ceil(r/256) row tiles.
+// Tiles are 256 rows; a group with r rows spans ceil(r/256) row tiles.  Stage
+// s occupies [s * 64 KB, (s + 1) * 64 KB): the token / A rows first, then the
+// weights (32 KB each; a deep swap stage: tokens, then 48 KB of weights).
 // ============================================================================
 constexpr int kPairBM = 256;
 constexpr int kPairBN = 256;  // MMA N: both halves of B
