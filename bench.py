@@ -232,9 +232,18 @@ def roofline(cfg, flops: float, nbytes: float, launch_ms: float, peaks: dict, pe
          "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes, "launch_ms": launch_ms,
          "traffic": traffic}
     if t_tensor >= t_hbm:
+        # the kernel is timed inside the timed loop of back-to-back forwards,
+        # under the power limit: the sustained GEMM figure is its peak; the
+        # burst figure (a GEMM timed alone) is reported beside it
         a = flops / (launch_ms * 1e-3) / 1e12
-        r.update(bound="tensor", achieved=a, peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                 frac=a / peaks["bf16_tflops"], peak_source=f"{src} bf16 dense burst")
+        sus = peaks.get("bf16_tflops_sustained")
+        if sus:
+            r.update(bound="tensor", achieved=a, peak=sus, unit="TFLOP/s", frac=a / sus,
+                     peak_source=f"{src} bf16 dense sustained (kernel timed inside the timed loop)",
+                     frac_of_burst=a / peaks["bf16_tflops"])
+        else:
+            r.update(bound="tensor", achieved=a, peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                     frac=a / peaks["bf16_tflops"], peak_source=f"{src} bf16 dense burst")
     else:
         a = nbytes / (launch_ms * 1e-3) / 1e9
         r.update(bound="hbm", achieved=a, peak=peaks["hbm_gbs"], unit="GB/s",
@@ -570,6 +579,8 @@ def run_ours(args, cfg):
                         if mixed else ""),
         "kept_pairs": kept, "dropped_pairs": cfg.T * cfg.top_k - kept,
         "expert_gemm_tflops": gemm_tflops, "expert_gemm_pct_peak": 100.0 * gemm_tflops / peaks["bf16_tflops"],
+        "expert_gemm_pct_sustained_peak": (100.0 * gemm_tflops / peaks["bf16_tflops_sustained"]
+                                           if peaks.get("bf16_tflops_sustained") else None),
         "dispatch_gbs": disp_gbs, "router_gbs": router_gbs, "combine_gbs": combine_gbs,
         "hbm_frac": {"router": router_gbs / peaks["hbm_gbs"], "dispatch": disp_gbs / peaks["hbm_gbs"],
                      "combine": combine_gbs / peaks["hbm_gbs"],

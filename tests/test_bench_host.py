@@ -26,7 +26,13 @@ def test_roofline_is_tensor_bound_for_large_groups():
     r = bench.roofline(cfg, flops, bench.up_gemm_bytes(cfg, kept), 1.5, PEAKS, "measured", None)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(flops / 1.5e-3 / 1e12)
-    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
+    # timed inside the loop of forwards: the sustained peak, the burst one beside it
+    assert r["peak"] == PEAKS["bf16_tflops_sustained"] and "sustained" in r["peak_source"]
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
+    assert r["frac_of_burst"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
+    burst_only = {k: v for k, v in PEAKS.items() if k != "bf16_tflops_sustained"}
+    r = bench.roofline(cfg, flops, bench.up_gemm_bytes(cfg, kept), 1.5, burst_only, "fallback", None)
+    assert r["peak"] == PEAKS["bf16_tflops"] and "burst" in r["peak_source"]
 
 
 def test_roofline_is_hbm_bound_when_weights_dominate():
