@@ -366,9 +366,11 @@ int moe_layer_backward(const moe_problem_t* p, const void* x, const moe_weights_
 #define MOE_EV_START 0   /* before the router */
 #define MOE_EV_ROUTED 1  /* after gate logits, selection and statistics */
 #define MOE_EV_DISPATCHED 2 /* after histogram, scan, rank and gather */
-#define MOE_EV_UP 3      /* after the routed up/gate projection with SwiGLU */
-#define MOE_EV_DOWN 4    /* after the routed down projection */
-#define MOE_EV_SHARED 5  /* after the shared experts */
+#define MOE_EV_UP 3      /* after the routed up/gate projection with SwiGLU (and the
+                            shared experts' one when they share its launch) */
+#define MOE_EV_DOWN 4    /* after the routed down projection (and the shared one, ditto) */
+#define MOE_EV_SHARED 5  /* after the shared experts (at MOE_EV_DOWN when they ran in
+                            the routed launches) */
 #define MOE_EV_END 6     /* after the combine */
 #define MOE_NUM_EVENTS 7
 
@@ -377,8 +379,12 @@ int moe_layer_backward(const moe_problem_t* p, const void* x, const moe_weights_
  * entries are skipped) on `stream` at the MOE_EV_* boundaries, so that the
  * time between two events is the time of that stage's kernels.  Stages that
  * do not run for this problem record their event at the same point as the
- * previous one.  *n_kernels (if not NULL) receives the number of kernels the
- * call enqueued.  Same arguments, results and errors as moe_layer_forward. */
+ * previous one.  With BF16, shared experts and the same expert-GEMM tile
+ * shape for the routed and the shared experts, the shared experts run inside
+ * the routed up and down launches (their tiles interleaved with the routed
+ * ones), so MOE_EV_UP and MOE_EV_DOWN cover both and the shared stage is
+ * empty.  *n_kernels (if not NULL) receives the number of kernels the call
+ * enqueued.  Same arguments, results and errors as moe_layer_forward. */
 int moe_layer_forward_profiled(const moe_problem_t* p, const void* x, const moe_weights_t* w,
                                void* y, const moe_routing_t* routing, float* stats,
                                void* ws, size_t ws_bytes, moe_stream_t stream,
