@@ -326,6 +326,48 @@ def test_layer_is_gate_weighted_sum_and_drops_contribute_nothing():
     assert (y[4:] == 0.0).all()
 
 
+def _pipeline(x, wg, w13, w2, K, C):
+    T, E = x.shape[0], wg.shape[0]
+    idx, w, _ = oracle.select(oracle.gate_logits(x, wg), K)
+    disp = oracle.dispatch(idx, E, oracle.capacity(T, K, E, C))
+    return oracle.layer_rows(x, w13, w2, idx, w, disp["slot_of"]), idx, disp
+
+
+def test_layer_is_unchanged_by_relabelling_the_experts():
+    # Expert j of the relabelled layer is expert pi[j] of the original (its gate
+    # row and weights move together): every token picks the same experts under
+    # new names, in the same order, each expert queues the same tokens, so the
+    # output -- drops under the capacity included -- is the same up to the
+    # rounding of sums over experts taken in another order (a slip in an expert
+    # index changes it by O(1)).
+    rng = np.random.default_rng(21)
+    T, d, E, K, F = 40, 12, 6, 2, 9
+    x, w13, w2, _ = _rand_layer(rng, T, d, E, F)
+    wg = rng.normal(size=(E, d)) / math.sqrt(d)
+    y, idx, disp = _pipeline(x, wg, w13, w2, K, 0.75)
+    assert int(disp["seg_off"][-1]) < T * K                    # the capacity drops pairs
+    pi = rng.permutation(E)
+    inv = np.argsort(pi)
+    y2, idx2, disp2 = _pipeline(x, wg[pi], w13[pi], w2[pi], K, 0.75)
+    assert (idx2 == inv[idx]).all()
+    assert ((disp2["slot_of"] >= 0) == (disp["slot_of"] >= 0)).all()
+    assert np.max(np.abs(y2 - y)) <= 1e-14 * np.max(np.abs(y))
+
+
+def test_layer_without_capacity_permutes_with_its_tokens():
+    # With no capacity limit nothing depends on the order of arrival: output row
+    # i of the permuted batch is output row sigma[i] of the original.
+    rng = np.random.default_rng(22)
+    T, d, E, K, F = 33, 10, 5, 3, 8
+    x, w13, w2, _ = _rand_layer(rng, T, d, E, F)
+    wg = rng.normal(size=(E, d)) / math.sqrt(d)
+    y, _, disp = _pipeline(x, wg, w13, w2, K, 0.0)
+    assert int(disp["seg_off"][-1]) == T * K
+    sigma = rng.permutation(T)
+    y2, _, _ = _pipeline(x[sigma], wg, w13, w2, K, 0.0)
+    assert np.array_equal(y2, y[sigma])
+
+
 def test_layer_rows_subset_matches_full():
     rng = np.random.default_rng(7)
     T, d, E, F = 11, 8, 4, 6
