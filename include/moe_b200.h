@@ -267,8 +267,9 @@ int moe_layer_forward(const moe_problem_t* p, const void* x, const moe_weights_t
  * (e.g. T <= 131072 at E = 256, T <= 524288 at E = 64); larger problems return
  * MOE_ERR_UNSUPPORTED and enqueue nothing.  All calls on a GPU share the array:
  * calls whose work overlaps on the GPU race, so serialise them.  The first call
- * on a device looks the array's address up (device current); make it before
- * any stream capture.  Expert indices outside [0, E) are skipped (slot -1) but
+ * on a device looks the array's address up (device current), and so does the
+ * first call after the device's context was reset (cudaDeviceReset); make
+ * such a call before any stream capture.  Expert indices outside [0, E) are skipped (slot -1) but
  * not reported (there is no status word).  MOE_FLAG_EXPERT_CAPACITY is not
  * accepted here (MOE_ERR_INVALID_ARG).  The pages have no counterpart of
  * this entry point. */

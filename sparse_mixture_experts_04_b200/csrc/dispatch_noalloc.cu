@@ -17,8 +17,9 @@
 // MOE_ERR_UNSUPPORTED before anything is enqueued.
 //
 // The first call on a device looks up the array's device address for that
-// device (with the device current); make that first call before any stream
-// capture begins.  Expert indices outside [0, E) are skipped (their slot is
+// device (with the device current), and so does the first call after the
+// device's context was reset; make that first call before any stream capture
+// begins.  Expert indices outside [0, E) are skipped (their slot is
 // -1) but, with no workspace, not reported.  The pages have no counterpart of
 // this entry point: it only changes where scratch memory comes from.
 #include <mutex>
@@ -33,25 +34,63 @@ constexpr size_t kNoAllocScratchWords = 262144;  // 1 MiB
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchWords];
 
-// Device address of g_noalloc_scratch on the current device (looked up once per
-// device).  In host code the array's name is only a host-side handle, never a
-// device pointer, so kernels get this address instead.
+// Device address of g_noalloc_scratch in the current context.  In host code
+// the array's name is only a host-side handle, never a device pointer, so
+// kernels get this address instead.  The address is looked up once per
+// context, keyed by the context's unique ID: after cudaDeviceReset (or any
+// other release of the primary context) the module is loaded again, possibly
+// elsewhere, and the next call looks the address up afresh.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+static bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 static int32_t* noalloc_scratch(int* rc) {
   static std::mutex mu;
+  static unsigned long long ctx_of[64] = {0};
   static int32_t* addr[64] = {nullptr};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    *rc = MOE_ERR_CUDA;
+  if (cudaError_t e = cudaGetDevice(&dev)) {
+    *rc = cuda_rc(e);
+    return nullptr;
+  }
+  if (dev < 0 || dev >= 64) {
+    *rc = MOE_ERR_UNSUPPORTED;
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  if (!addr[dev] || !have_ctx || ctx != ctx_of[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+    // makes the device's primary context current if no context was yet
+    if (cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) {
+      *rc = cuda_rc(e);
+      return nullptr;
+    }
+    if (!p || !current_context_id(&ctx)) {
       *rc = MOE_ERR_CUDA;
       return nullptr;
     }
     addr[dev] = static_cast<int32_t*>(p);
+    ctx_of[dev] = ctx;
   }
   *rc = MOE_OK;
   return addr[dev];
@@ -81,9 +120,11 @@ extern "C" int moe_dispatch_noalloc(const moe_problem_t* q, const int32_t* topk_
   int32_t* chunk_counts = scratch;
   int32_t* chunk_base = scratch + n_chunks * p.E;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (launch_dispatch(p, topk_idx, counts, kept, seg_off, slot_of, perm, chunk_counts, chunk_base,
-                      /*status=*/nullptr, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (x_perm && launch_gather(p, x, perm, seg_off, x_perm, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaError_t e = launch_dispatch(p, topk_idx, counts, kept, seg_off, slot_of, perm, chunk_counts, chunk_base,
+                                      /*status=*/nullptr, st))
+    return cuda_rc(e);
+  if (x_perm) {
+    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
+  }
   return MOE_OK;
 }

@@ -135,4 +135,7 @@ cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* 
 // device properties (cached per device)
 int num_sms();
 
+// moe_api.cu: the moe_status value reported for a CUDA error (MOE_OK for cudaSuccess)
+int cuda_rc(cudaError_t e);
+
 }  // namespace moe

@@ -23,15 +23,20 @@ def test_roofline_is_tensor_bound_for_large_groups():
     cfg = CONFIGS["mixtral"]
     kept = [1024] * 8
     flops = bench.algorithmic_flops(cfg, sum(kept))["up"]
-    r = bench.roofline(cfg, flops, bench.up_gemm_bytes(cfg, kept), 1.5, PEAKS, "measured", None)
+    nbytes = bench.up_gemm_bytes(cfg, kept)
+    # a timed region under a second: the burst peak, the sustained one beside it
+    r = bench.roofline(cfg, flops, nbytes, 1.5, PEAKS, "measured", None, 0.12)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(flops / 1.5e-3 / 1e12)
-    # timed inside the loop of forwards: the sustained peak, the burst one beside it
+    assert r["peak"] == PEAKS["bf16_tflops"] and "burst" in r["peak_source"]
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
+    assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
+    # a timed region of seconds runs under the power limit: the sustained peak
+    r = bench.roofline(cfg, flops, nbytes, 1.5, PEAKS, "measured", None, 3.0)
     assert r["peak"] == PEAKS["bf16_tflops_sustained"] and "sustained" in r["peak_source"]
-    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
     assert r["frac_of_burst"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
     burst_only = {k: v for k, v in PEAKS.items() if k != "bf16_tflops_sustained"}
-    r = bench.roofline(cfg, flops, bench.up_gemm_bytes(cfg, kept), 1.5, burst_only, "fallback", None)
+    r = bench.roofline(cfg, flops, nbytes, 1.5, burst_only, "fallback", None, 3.0)
     assert r["peak"] == PEAKS["bf16_tflops"] and "burst" in r["peak_source"]
 
 
@@ -40,7 +45,7 @@ def test_roofline_is_hbm_bound_when_weights_dominate():
     kept = [2] * cfg.n_experts          # a few rows per expert: weight streaming
     flops = bench.algorithmic_flops(cfg, sum(kept))["up"]
     nbytes = bench.up_gemm_bytes(cfg, kept)
-    r = bench.roofline(cfg, flops, nbytes, 0.5, PEAKS, "fallback", None)
+    r = bench.roofline(cfg, flops, nbytes, 0.5, PEAKS, "fallback", None, 0.04)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(nbytes / 0.5e-3 / 1e9)
     assert r["peak"] == PEAKS["hbm_gbs"] and "fallback" in r["peak_source"]

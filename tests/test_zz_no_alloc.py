@@ -20,6 +20,11 @@ CASES = [
               capacity_factor=1.25, dtype="bf16", seed=31),
     MoeConfig("na_zen", T=1000, d_model=256, n_experts=128, top_k=8, d_ff=128, n_shared=0,
               capacity_factor=1.0, dtype="bf16", seed=32, bias_range=0.1),
+    # above the fused scan+rank limit (ceil(T/256)^2 * E > 2^22): the separate
+    # scan kernel writes the chunk bases into the second half of the array
+    # (2 * 257 * 64 = 32896 of its 262144 words)
+    MoeConfig("na_two_kernel_scan", T=65537, d_model=64, n_experts=64, top_k=4, d_ff=64, n_shared=0,
+              capacity_factor=1.0, dtype="bf16", seed=33),
 ]
 
 
