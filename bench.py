@@ -296,6 +296,28 @@ def roofline(cfg, flops: float, nbytes: float, launch_ms: float, peaks: dict, pe
     return r
 
 
+def stage_spans(rows) -> dict:
+    """Mean per-stage device spans in us from moe_layer_forward_clocked's
+    clocks (one row of 2 * NUM_CLOCKS per forward); dispatch+gather runs from
+    the dispatch kernels' first start to the gather's last end."""
+    names = _lib.CLOCK_NAMES
+    acc = {}
+
+    def span(row, a, b):
+        s, e = row[2 * names.index(a)] & 0xFFFFFFFFFFFFFFFF, row[2 * names.index(b) + 1] & 0xFFFFFFFFFFFFFFFF
+        if s == 0 or e == 0:
+            return None
+        return (e - ((~s) & 0xFFFFFFFFFFFFFFFF)) / 1e3
+
+    for row in rows:
+        vals = {n: span(row, n, n) for n in names}
+        vals["dispatch+gather"] = span(row, "dispatch", "gather")
+        for k, v in vals.items():
+            if v is not None:
+                acc.setdefault(k, []).append(v)
+    return {k: statistics.mean(v) for k, v in acc.items()}
+
+
 def dispatch_bytes(cfg, kept_pairs: int) -> float:
     """topk_idx read twice (histogram, rank) + slot_of / perm written + x rows read + x_perm written."""
     es = 2 if cfg.dtype == "bf16" else 4
@@ -452,6 +474,18 @@ def run_ours(args, cfg):
     for j in range(1, _lib.NUM_EVENTS):
         stage[_lib.EVENT_NAMES[j]] = sum(evs[i][j - 1].elapsed_time(evs[i][j]) for i in range(n_prof)) / n_prof
 
+    # device-stamped stage spans (moe_layer_forward_clocked): the forwards run back to
+    # back with no events between their kernels; every stage kernel stamps the global
+    # timer when it may start reading its inputs (after the programmatic-launch wait)
+    # and when its last CTA ends
+    n_clk = min(args.steps, 20)
+    clocks = torch.zeros((n_clk, 2 * _lib.NUM_CLOCKS), dtype=torch.int64, device="cuda")
+    for i in range(n_clk):
+        api.moe_layer_forward_clocked(layer.prob, xs[i % n_x], layer.weights, y, layer.routing, layer.stats,
+                                      layer.ws, clocks[i], stream)
+    torch.cuda.synchronize()
+    clock_spans = stage_spans(clocks.cpu().tolist())
+
     # end to end through the public API (MoeLayer.forward_host): every step copies
     # its x from pinned host memory and its y and statistics back; the copies of
     # neighbouring steps overlap the kernels (separate streams, double buffers).
@@ -583,9 +617,19 @@ def run_ours(args, cfg):
                         timed_s, kernel="routed + shared up/gate GEMM with SwiGLU epilogue, one launch (tcgen05)")
     else:
         roof = roofline(cfg, flops["up"], up_bytes, up_ms, peaks, peak_src, ncu_traffic(cfg.name), timed_s)
-    disp_gbs = dispatch_bytes(cfg, kept) / (stage["dispatched"] * 1e-3) / 1e9
-    router_gbs = router_bytes(cfg) / (stage["routed"] * 1e-3) / 1e9
-    combine_gbs = combine_bytes(cfg, kept) / (stage["end"] * 1e-3) / 1e9
+    # HBM fractions of the memory-bound stages from the device-stamped spans
+    # (first CTA start to last CTA end of the stage's kernels), and from the
+    # event pass beside them (which adds a launch gap at every stage boundary)
+    mem_bytes = {"router": router_bytes(cfg), "dispatch": dispatch_bytes(cfg, kept),
+                 "combine": combine_bytes(cfg, kept)}
+    span_key = {"router": "route", "dispatch": "dispatch+gather", "combine": "combine"}
+    event_key = {"router": "routed", "dispatch": "dispatched", "combine": "end"}
+    gbs_clock = {k: (mem_bytes[k] / (clock_spans[span_key[k]] * 1e-6) / 1e9
+                     if clock_spans.get(span_key[k]) else None) for k in mem_bytes}
+    gbs_event = {k: mem_bytes[k] / (stage[event_key[k]] * 1e-3) / 1e9 for k in mem_bytes}
+    disp_gbs = gbs_clock["dispatch"] or gbs_event["dispatch"]
+    router_gbs = gbs_clock["router"] or gbs_event["router"]
+    combine_gbs = gbs_clock["combine"] or gbs_event["combine"]
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -623,8 +667,12 @@ def run_ours(args, cfg):
         "dispatch_gbs": disp_gbs, "router_gbs": router_gbs, "combine_gbs": combine_gbs,
         "hbm_frac": {"router": router_gbs / peaks["hbm_gbs"], "dispatch": disp_gbs / peaks["hbm_gbs"],
                      "combine": combine_gbs / peaks["hbm_gbs"],
-                     "note": "algorithmic bytes / stage time (the bench's separate pass with an event at "
-                             "every stage boundary) / the measured HBM copy bandwidth"},
+                     "note": "algorithmic bytes / the stage's device-stamped span (moe_layer_forward_clocked: "
+                             "first CTA start to last CTA end of the stage's kernels, dispatch = scan+rank "
+                             "start to gather end, mean of back-to-back forwards) / the measured HBM copy "
+                             "bandwidth"},
+        "stage_clock_us": clock_spans,
+        "hbm_frac_event_stages": {k: gbs_event[k] / peaks["hbm_gbs"] for k in gbs_event},
         "layer_tflops": total_flops / (ms * 1e-3) / 1e12,
         "backward": bwd,
         "expert_parallel": epl,

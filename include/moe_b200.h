@@ -391,6 +391,35 @@ int moe_layer_forward_profiled(const moe_problem_t* p, const void* x, const moe_
                                void* ws, size_t ws_bytes, moe_stream_t stream,
                                void* const* events, int32_t* n_kernels);
 
+/* Stages whose kernels moe_layer_forward_clocked times on the device. */
+#define MOE_CLOCK_ROUTE 0    /* gate logits, selection, chunk statistics (the fused router) */
+#define MOE_CLOCK_DISPATCH 1 /* scan, capacity, ranks, slots (histogram on moe_dispatch) */
+#define MOE_CLOCK_GATHER 2   /* x rows into expert order */
+#define MOE_CLOCK_UP 3       /* routed up/gate projection + SwiGLU (and the shared experts'
+                                when they share its launch) */
+#define MOE_CLOCK_DOWN 4     /* routed down projection (ditto) */
+#define MOE_CLOCK_SHARED 5   /* the shared experts' own launches, when they run separately */
+#define MOE_CLOCK_COMBINE 6  /* gate-weighted combine */
+#define MOE_NUM_CLOCKS 7
+
+/* moe_layer_forward, timed on the device: every BF16 kernel of a stage
+ * stamps the global timer (ns) into clocks[2s] and clocks[2s + 1], so that
+ * after the forward completes
+ *     start_s = ~clocks[2s]   (bitwise complement: the earliest start)
+ *     end_s   =  clocks[2s + 1] (the latest end)
+ * span the stage's kernels from the first CTA that could read its inputs to
+ * the last CTA's end, without the launch gaps an event pair would include.
+ *   clocks: DEVICE array of 2 * MOE_NUM_CLOCKS uint64, 8-byte aligned, filled
+ *           with zeros by the caller before the call (every stamp is an atomic
+ *           max); a stage that did not run, or whose kernels do not stamp
+ *           (the FP32 expert GEMMs and gate logits), leaves its pair at zero.
+ * Kernel work and results are those of moe_layer_forward; each CTA adds two
+ * atomics.  Same arguments and errors, plus MOE_ERR_INVALID_ARG for clocks.
+ * This is measurement support, not a step of the pages' method. */
+int moe_layer_forward_clocked(const moe_problem_t* p, const void* x, const moe_weights_t* w,
+                              void* y, const moe_routing_t* routing, float* stats,
+                              void* ws, size_t ws_bytes, moe_stream_t stream, uint64_t* clocks);
+
 /* Expert-parallel exchange plan.  "Scaling with experts", What you still pay
  * for (experts partitioned over devices: a token travels to the device that
  * holds its expert, the output travels back); Zen MoDE §7.2 Communication

@@ -27,10 +27,13 @@ DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
 EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
             "moe_reset_device_status", "moe_read_device_status", "moe_route", "moe_dispatch",
             "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
+            "moe_layer_forward_clocked",
             "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update", "moe_backward_workspace_size",
             "moe_layer_backward", "moe_ep_plan")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
+NUM_CLOCKS = 7  # MOE_CLOCK_ROUTE .. MOE_CLOCK_COMBINE
+CLOCK_NAMES = ("route", "dispatch", "gather", "up", "down", "shared", "combine")
 
 
 class MoeProblem(ctypes.Structure):
@@ -98,6 +101,9 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_forward_profiled.argtypes = [PP, P, ctypes.POINTER(MoeWeights), P, ctypes.POINTER(MoeRouting), P,
                                              P, sz, P, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(i32)]
     L.moe_layer_forward_profiled.restype = ctypes.c_int
+    L.moe_layer_forward_clocked.argtypes = [PP, P, ctypes.POINTER(MoeWeights), P, ctypes.POINTER(MoeRouting), P,
+                                            P, sz, P, P]
+    L.moe_layer_forward_clocked.restype = ctypes.c_int
     L.moe_dispatch_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P]
     L.moe_dispatch_noalloc.restype = ctypes.c_int
     L.moe_dispatch_capacity.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, sz, P]

@@ -18,7 +18,7 @@ from ._lib import (BIAS_UPDATE_PROPORTIONAL, BIAS_UPDATE_SIGN, DTYPE_BF16, DTYPE
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
            "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
-           "moe_layer_forward_profiled", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
+           "moe_layer_forward_profiled", "moe_layer_forward_clocked", "stage_clock_us", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
            "moe_layer_backward", "backward_workspace_size", "alloc_backward_workspace", "moe_ep_plan",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
            "FLAG_EXTENDED_STATS", "FLAG_EXPERT_CAPACITY", "FLAG_SAVE_GU", "EXTENDED_STATS", "stats_size",
@@ -173,6 +173,34 @@ def moe_layer_forward_profiled(prob, x, weights: dict, y, routing: dict | None, 
                                                ws.numel(), _stream(stream), handles, ctypes.byref(n))
     _lib.check("moe_layer_forward_profiled", rc)
     return int(n.value)
+
+
+def moe_layer_forward_clocked(prob, x, weights: dict, y, routing: dict | None, stats, ws, clocks, stream=None):
+    """moe_layer_forward with device stage clocks: `clocks` is a zero-filled
+    int64 device tensor of 2 * NUM_CLOCKS entries (see stage_clock_us)."""
+    assert clocks.dtype == torch.int64 and clocks.numel() >= 2 * _lib.NUM_CLOCKS and clocks.is_cuda
+    w = _weights_struct(weights)
+    r = _routing_struct(routing)
+    rc = _lib.lib().moe_layer_forward_clocked(ctypes.byref(prob), _p(x), ctypes.byref(w), _p(y),
+                                              ctypes.byref(r) if r is not None else None, _p(stats), _p(ws),
+                                              ws.numel(), _stream(stream), _p(clocks))
+    _lib.check("moe_layer_forward_clocked", rc)
+
+
+def stage_clock_us(clocks) -> dict:
+    """Per-stage device time in us from one forward's clocks (host copy, any
+    integer sequence of 2 * NUM_CLOCKS): end - start for each stage that
+    stamped, None for the others."""
+    out = {}
+    vals = [int(v) & 0xFFFFFFFFFFFFFFFF for v in clocks]
+    for s, name in enumerate(_lib.CLOCK_NAMES):
+        start_c, end = vals[2 * s], vals[2 * s + 1]
+        if start_c == 0 or end == 0:
+            out[name] = None
+            continue
+        start = (~start_c) & 0xFFFFFFFFFFFFFFFF
+        out[name] = (end - start) / 1e3
+    return out
 
 
 def backward_workspace_size(prob: MoeProblem) -> int:

@@ -56,10 +56,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const T* __res
                                                                   const float* __restrict__ topk_w,
                                                                   const T* __restrict__ y_shared,
                                                                   T* __restrict__ y, int64_t Tn, int d, int K,
-                                                                  int64_t n_perm_rows) {
+                                                                  int64_t n_perm_rows, unsigned long long* clk) {
   constexpr int V = Pack16<T>::N;
   pdl_wait();
   pdl_trigger();
+  stage_clock_start(clk);
   const int nvec = d / V;
   const int v0 = blockIdx.x * (kCombineThreads * kCombineVPT) + threadIdx.x;
   for (int64_t t = blockIdx.y; t < Tn; t += gridDim.y) {
@@ -93,10 +94,14 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const T* __res
       if (v < nvec) Pack16<T>::store(y + t * d + v * V, acc[j]);
     }
   }
+  if (clk) {
+    __syncthreads();
+    stage_clock_end(clk);
+  }
 }
 
 cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
-                           const void* y_shared, void* y, cudaStream_t st) {
+                           const void* y_shared, void* y, cudaStream_t st, unsigned long long* clk) {
   const int V = p.dtype == kBF16 ? 8 : 4;
   const int nvec = p.d / V;
   const unsigned gx = static_cast<unsigned>((nvec + kCombineThreads * kCombineVPT - 1) / (kCombineThreads * kCombineVPT));
@@ -107,11 +112,11 @@ cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* 
     return launch_k(combine_kernel<__nv_bfloat16>, grid, dim3(kCombineThreads), 0, st,
                     static_cast<const __nv_bfloat16*>(y_perm), slot_of, topk_w,
                     static_cast<const __nv_bfloat16*>(y_shared), static_cast<__nv_bfloat16*>(y), p.T, p.d, p.K,
-                    p.max_rows);
+                    p.max_rows, clk);
   else
     return launch_k(combine_kernel<float>, grid, dim3(kCombineThreads), 0, st, static_cast<const float*>(y_perm),
                     slot_of, topk_w, static_cast<const float*>(y_shared), static_cast<float*>(y), p.T, p.d, p.K,
-                    p.max_rows);
+                    p.max_rows, clk);
   return cudaGetLastError();
 }
 

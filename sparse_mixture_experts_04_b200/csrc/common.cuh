@@ -70,21 +70,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase of `bar` with the given parity has completed.  Bounded:
-// gives up when `abort` is raised by another role, or after kWaitLimitNs (then
+// gives up when `abort` is raised by another role, or after limit_ns (then
 // raises `abort` itself).  Returns false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
+}
+
+// Test hook of the bounded-wait abort path (stall_ns > 0, see
+// test_stall_ns() in internal.h): the MMA-issuing thread first waits for a
+// barrier phase that nothing completes (`bar`'s first phase, before anything
+// arrives on it), gives up after stall_ns, raises `abort`, and the kernel then
+// takes its abort path: every role drains what it started and returns.
+__device__ __forceinline__ bool test_stall(uint64_t* bar, volatile int* abort, unsigned long long stall_ns) {
+  return stall_ns == 0 || mbar_wait_for(bar, 0, abort, stall_ns);
 }
 
 // -------------------------------------------------------------- TMA copies
@@ -361,6 +375,20 @@ __device__ __forceinline__ void balance_loss(const double* fp, int E, float alph
   double acc = 0.0;
   for (int e = 0; e < E; ++e) acc += fp[e];
   stats[2 * E] = static_cast<float>(static_cast<double>(alpha) * E * acc);
+}
+
+// ----------------------------------------------------------- stage clocks
+// moe_layer_forward_clocked: each kernel of a stage raises clk[0] to the
+// bitwise complement of its start and clk[1] to its end (ns of the global
+// timer), so a zero-filled pair ends up holding the stage's earliest start
+// (complemented) and latest end whatever the order of the CTAs.  Thread 0 of
+// every CTA stamps: the start once the predecessor's outputs may be read
+// (after pdl_wait), the end after the CTA's last barrier.
+__device__ __forceinline__ void stage_clock_start(unsigned long long* clk) {
+  if (clk && threadIdx.x == 0) atomicMax(clk, ~global_ns());
+}
+__device__ __forceinline__ void stage_clock_end(unsigned long long* clk) {
+  if (clk && threadIdx.x == 0) atomicMax(clk + 1, global_ns());
 }
 
 // ------------------------------------------- programmatic dependent launch

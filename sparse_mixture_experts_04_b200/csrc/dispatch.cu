@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
                                                              const unsigned long long* __restrict__ chunk_psum,
                                                              float* __restrict__ stats, int64_t T, int K,
                                                              float alpha, const float* __restrict__ zpart,
-                                                             int n_zpart, const int32_t* __restrict__ expert_cap) {
+                                                             int n_zpart, const int32_t* __restrict__ expert_cap,
+                                                             unsigned long long* clk) {
   __shared__ int part[1024];
   __shared__ unsigned long long ppart[1024];
   __shared__ int s_kept[kMaxExperts];
@@ -75,6 +76,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
   __shared__ double s_zsum[1024];
   pdl_wait();
   pdl_trigger();
+  stage_clock_start(clk);
   int S = 1024 / E;
   if (S > n_chunks) S = n_chunks;
   if (S < 1) S = 1;
@@ -162,6 +164,10 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(const int32_t* __re
     }
     if (tid == 31) seg_off[E] = incl;
   }
+  if (clk) {
+    __syncthreads();
+    stage_clock_end(clk);
+  }
 }
 
 __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __restrict__ idx, int64_t T, int K,
@@ -169,11 +175,12 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
                                                             const int32_t* __restrict__ kept,
                                                             const int32_t* __restrict__ seg_off,
                                                             int32_t* __restrict__ slot_of,
-                                                            int32_t* __restrict__ perm) {
+                                                            int32_t* __restrict__ perm, unsigned long long* clk) {
   __shared__ uint32_t mask[8][kMaxExperts];
   __shared__ int wbase[8][kMaxExperts];
   pdl_wait();
   pdl_trigger();
+  stage_clock_start(clk);
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) mask[i / E][i % E] = 0u;
@@ -212,6 +219,10 @@ __global__ void __launch_bounds__(256) dispatch_rank_kernel(const int32_t* __res
       slot_of[pair] = slot;
     }
   }
+  if (clk) {
+    __syncthreads();
+    stage_clock_end(clk);
+  }
 }
 
 // Fused scan+rank reads n_chunks^2 * E histogram words from L2 in all (every
@@ -234,7 +245,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
     int n_chunks, long long cap, const int32_t* __restrict__ expert_cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ kept_out, int32_t* __restrict__ seg_off_out, int32_t* __restrict__ slot_of,
     int32_t* __restrict__ perm, const unsigned long long* __restrict__ chunk_psum, float* __restrict__ stats,
-    float alpha, const float* __restrict__ zpart, int n_zpart) {
+    float alpha, const float* __restrict__ zpart, int n_zpart, unsigned long long* clk) {
   __shared__ int s_tot_part[256];
   __shared__ int s_pre_part[256];
   __shared__ int s_tot[kMaxExperts];
@@ -247,6 +258,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
   __shared__ double s_red[256];
   pdl_wait();
   pdl_trigger();
+  stage_clock_start(clk);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -374,6 +386,10 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
       if (zpart) utilisation_stats(s_tot, s_kept, E, T, s_red[0], stats);
     }
   }
+  if (clk) {
+    __syncthreads();
+    stage_clock_end(clk);
+  }
 }
 
 bool dispatch_fused(const Problem& p) {
@@ -385,7 +401,7 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready,
                             const unsigned long long* chunk_psum, float* stats, const float* zpart, int n_zpart,
-                            const int32_t* expert_cap) {
+                            const int32_t* expert_cap, unsigned long long* clk) {
   const int n_chunks = static_cast<int>((p.T + kDispatchChunk - 1) / kDispatchChunk);
   if (!counts_ready) {
     if (cudaError_t e = launch_k(dispatch_hist_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
@@ -396,15 +412,15 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
     return launch_k(dispatch_scan_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
                     static_cast<const int32_t*>(chunk_counts), n_chunks, static_cast<long long>(p.cap), expert_cap,
                     counts, kept, seg_off, slot_of, perm, chunk_psum, chunk_psum ? stats : nullptr, p.alpha, zpart,
-                    n_zpart);
+                    n_zpart, clk);
   if (cudaError_t e = launch_k(dispatch_scan_kernel, dim3(1), dim3(1024), 0, st,
                                static_cast<const int32_t*>(chunk_counts), n_chunks, p.E, static_cast<long long>(p.cap),
                                chunk_base, counts, kept, seg_off, chunk_psum, chunk_psum ? stats : nullptr, p.T,
-                               p.K, p.alpha, zpart, n_zpart, expert_cap))
+                               p.K, p.alpha, zpart, n_zpart, expert_cap, clk))
     return e;
   return launch_k(dispatch_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
                   static_cast<const int32_t*>(chunk_base), static_cast<const int32_t*>(kept),
-                  static_cast<const int32_t*>(seg_off), slot_of, perm);
+                  static_cast<const int32_t*>(seg_off), slot_of, perm, clk);
 }
 
 constexpr int kGatherUnroll = 8;
@@ -415,10 +431,11 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ seg_off, int E, int K,
                                                           int64_t T, int vec_per_row, int64_t max_rows,
-                                                          uint4* __restrict__ x_perm) {
+                                                          uint4* __restrict__ x_perm, unsigned long long* clk) {
   const int lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
+  stage_clock_start(clk);
   const int64_t n_rows = seg_off[E];
   const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -438,10 +455,14 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
         if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = buf[j];
     }
   }
+  if (clk) {
+    __syncthreads();
+    stage_clock_end(clk);
+  }
 }
 
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
-                          void* x_perm, cudaStream_t st) {
+                          void* x_perm, cudaStream_t st, unsigned long long* clk) {
   if (p.max_rows <= 0) return cudaSuccess;
   const int vec_per_row = static_cast<int>(p.d * p.esize() / 16);
   int64_t blocks = (p.max_rows + 7) / 8;
@@ -449,7 +470,7 @@ cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, 
   if (blocks > cap_blocks) blocks = cap_blocks;
   return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
                   static_cast<const uint4*>(x), perm, seg_off, p.E, p.K, p.T, vec_per_row, p.max_rows,
-                  static_cast<uint4*>(x_perm));
+                  static_cast<uint4*>(x_perm), clk);
 }
 
 }  // namespace moe

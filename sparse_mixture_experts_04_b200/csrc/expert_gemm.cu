@@ -85,6 +85,10 @@ struct GemmArgs {
   // pair kernel, merged maps: swap tiles of at most 64 token rows take
   // 192-deep stages (tokens and weights of three chunks in one stage slot)
   int deep_swap;
+  // stage clock of the launch (moe_layer_forward_clocked), or nullptr
+  unsigned long long* clk;
+  // single-CTA kernel: abort-path test hook (test_stall), 0 normally
+  unsigned long long stall_ns;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -379,6 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   pdl_wait();  // everything above is local set-up; from here on the predecessor's outputs are read
   pdl_trigger();
+  stage_clock_start(args.clk);
   if (warp == 2) tile_prefix_warp<kBM>(args, n_tiles_n, prefix, lane);
   if (warp == 3) {
     if (args2.n_groups > 0)
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      bool ok = test_stall(drain, abort_flag, args.stall_ns);
       int it = 0;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
@@ -517,6 +522,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   __syncthreads();
+  stage_clock_end(args.clk);
   if (threadIdx.x == 0 && *abort_flag) raise_status(args.status, kDevWaitTimeout);
   if (warp == 1) {
     __syncwarp();
@@ -750,6 +756,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
   pdl_wait();  // everything above is local set-up; from here on the predecessor's outputs are read
   pdl_trigger();
+  stage_clock_start(args.clk);
   if (warp == 2) tile_prefix_warp<kPairBM>(args, n_tiles_n, prefix, lane);
   if (warp == 3) {
     if (args2.n_groups > 0)
@@ -951,6 +958,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   __syncwarp();
   tc_fence_before_sync();
   cluster_sync();  // no CTA leaves while its peer may still touch its shared memory or TMEM
+  stage_clock_end(args.clk);
   if (threadIdx.x == 0 && *abort_flag) raise_status(args.status, kDevWaitTimeout);
   if (warp == 1) {
     __syncwarp();
@@ -1230,7 +1238,7 @@ int router_k_splits(const Problem& p) {
 // s writes its partial logits at out + s*T*E (the offset goes into slice 0) and
 // the selection kernel adds the slices in order.
 int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset, float* out,
-                          int n_splits, unsigned* status, cudaStream_t st) {
+                          int n_splits, unsigned* status, cudaStream_t st, unsigned long long* clk) {
   CUtensorMap ta, tb;
   const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.T)};
   const uint32_t ba[2] = {kBK, kBM};
@@ -1240,6 +1248,7 @@ int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, c
   const uint32_t bb[3] = {kBK, static_cast<uint32_t>(bn), 1};
   if (!make_map(&tb, w_gate, 3, db, bb)) return -3;
   GemmArgs a{};
+  a.stall_ns = test_stall_ns();
   a.n_groups = n_splits;
   a.seg_off = nullptr;
   a.n_rows = static_cast<int>(p.T);
@@ -1253,6 +1262,7 @@ int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, c
   a.status = status;
   a.k_split = n_splits > 1 ? static_cast<int>(cdiv(cdiv(p.d, n_splits), kBK) * kBK) : 0;
   a.out_group_stride = p.T * p.E;
+  a.clk = clk;
   const int64_t tiles = cdiv(p.T, kBM) * n_splits;
   switch (bn) {
     case 32: return run_gemm<EPI_F32, 32, 8>(ta, tb, a, tiles, st);
@@ -1502,6 +1512,7 @@ static bool up_single_problem(const Problem& p, bool routed, const void* x_rows,
   if (!make_map(&q->ta, x_rows, 2, da, ba) || !make_map(&q->tb, w13, 3, db, bb)) return false;
   GemmArgs& a = q->a;
   a = GemmArgs{};
+  a.stall_ns = test_stall_ns();
   a.n_groups = G;
   a.seg_off = routed ? seg_off : nullptr;
   a.n_rows = static_cast<int>(n_rows);
@@ -1535,6 +1546,7 @@ static bool down_single_problem(const Problem& p, bool routed, const void* h, in
   if (!make_map(&q->ta, h, 2, da, ba) || !make_map(&q->tb, w2, 3, db, bb)) return false;
   GemmArgs& a = q->a;
   a = GemmArgs{};
+  a.stall_ns = test_stall_ns();
   a.n_groups = routed ? G : 1;
   a.seg_off = routed ? seg_off : nullptr;
   a.n_rows = static_cast<int>(n_rows);
@@ -1556,7 +1568,8 @@ static bool down_single_problem(const Problem& p, bool routed, const void* h, in
 // [n_rows, N_s * F] (shared).
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status, cudaStream_t st,
-                      cudaEvent_t after_up, int* n_kernels, void* gu) {
+                      cudaEvent_t after_up, int* n_kernels, void* gu, unsigned long long* clk_up,
+                      unsigned long long* clk_down) {
   if (n_rows <= 0) return 0;
   if (p.dtype == kF32) {
     if (n_kernels) *n_kernels += 2;
@@ -1580,6 +1593,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     if (pair) {
       PairProblem q;
       if (!up_pair_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, tail, &q)) return -3;
+      q.a.clk = clk_up;
       int rc = run_pair_gemm<EPI_SWIGLU>(q, nullptr, st);
       if (rc) return rc;
       if (tail) {
@@ -1594,6 +1608,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     } else {
       SingleProblem q;
       if (!up_single_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, &q)) return -3;
+      q.a.clk = clk_up;
       const int rc = run_gemm<EPI_SWIGLU, 256, 4>(q.ta, q.tb, q.a, q.tile_bound, st);
       if (rc) return rc;
     }
@@ -1610,6 +1625,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     if (pair) {
       PairProblem q;
       if (!down_pair_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, tail, &q)) return -3;
+      q.a.clk = clk_down;
       int rc = run_pair_gemm<EPI_BF16>(q, nullptr, st);
       if (rc) return rc;
       if (tail) {
@@ -1623,6 +1639,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     } else {
       SingleProblem q;
       if (!down_single_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, &q)) return -3;
+      q.a.clk = clk_down;
       const int rc = run_gemm<EPI_BF16, 256, 4>(q.ta, q.tb, q.a, q.tile_bound, st);
       if (rc) return rc;
     }
@@ -1645,7 +1662,8 @@ bool expert_ffn_mixed_ok(const Problem& p) {
 int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t* seg_off, const void* w13,
                             const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
                             const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
-                            cudaStream_t st, cudaEvent_t after_up, int* n_kernels) {
+                            cudaStream_t st, cudaEvent_t after_up, int* n_kernels, unsigned long long* clk_up,
+                            unsigned long long* clk_down) {
   if (!expert_ffn_mixed_ok(p)) return -3;
   if (n_kernels) *n_kernels += 2;
   if (ffn_tile_mode(p, true, p.max_rows) == kTileSingle) {
@@ -1653,23 +1671,27 @@ int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t*
     if (!up_single_problem(p, true, x_perm, p.max_rows, seg_off, w13, h, gu, status, &r) ||
         !up_single_problem(p, false, x, p.T, nullptr, w13_shared, h_shared, gu_shared, status, &s))
       return -3;
+    r.a.clk = clk_up;
     if (int rc = run_gemm<EPI_SWIGLU, 256, 4>(r.ta, r.tb, r.a, r.tile_bound, st, &s.ta, &s.tb, &s.a, s.tile_bound))
       return rc;
     if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
     if (!down_single_problem(p, true, h, p.max_rows, seg_off, w2, y_perm, status, &r) ||
         !down_single_problem(p, false, h_shared, p.T, nullptr, w2_shared, y_shared, status, &s))
       return -3;
+    r.a.clk = clk_down;
     return run_gemm<EPI_BF16, 256, 4>(r.ta, r.tb, r.a, r.tile_bound, st, &s.ta, &s.tb, &s.a, s.tile_bound);
   }
   PairProblem r, s;
   if (!up_pair_problem(p, true, x_perm, p.max_rows, seg_off, w13, h, gu, status, false, &r) ||
       !up_pair_problem(p, false, x, p.T, nullptr, w13_shared, h_shared, gu_shared, status, false, &s))
     return -3;
+  r.a.clk = clk_up;
   if (int rc = run_pair_gemm<EPI_SWIGLU>(r, &s, st)) return rc;
   if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
   if (!down_pair_problem(p, true, h, p.max_rows, seg_off, w2, y_perm, status, false, &r) ||
       !down_pair_problem(p, false, h_shared, p.T, nullptr, w2_shared, y_shared, status, false, &s))
     return -3;
+  r.a.clk = clk_down;
   return run_pair_gemm<EPI_BF16>(r, &s, st);
 }
 

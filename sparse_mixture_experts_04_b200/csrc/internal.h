@@ -56,9 +56,12 @@ cudaError_t launch_gate_logits_simt(const Problem& p, const void* x, const void*
 // zpart (or nullptr): [route_select_zparts(p)] partial sums of logsumexp^2
 // (router z-loss), at most n_sel_blocks of them
 int route_select_zparts(const Problem& p);
+// clk (all launchers below; or nullptr): the stage clock the kernels stamp
+// (moe_layer_forward_clocked)
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
                                 const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
-                                unsigned long long* chunk_psum, float* zpart, cudaStream_t st);
+                                unsigned long long* chunk_psum, float* zpart, cudaStream_t st,
+                                unsigned long long* clk = nullptr);
 // f, P and the loss from those chunk totals (moe_route's statistics); with
 // zpart also the extended statistics (kept = min(counts, cap))
 cudaError_t launch_route_stats(const Problem& p, const int32_t* chunk_counts, const unsigned long long* chunk_psum,
@@ -80,9 +83,10 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* 
                             int32_t* seg_off, int32_t* slot_of, int32_t* perm, int32_t* chunk_counts,
                             int32_t* chunk_base, unsigned* status, cudaStream_t st, bool counts_ready = false,
                             const unsigned long long* chunk_psum = nullptr, float* stats = nullptr,
-                            const float* zpart = nullptr, int n_zpart = 0, const int32_t* expert_cap = nullptr);
+                            const float* zpart = nullptr, int n_zpart = 0, const int32_t* expert_cap = nullptr,
+                            unsigned long long* clk = nullptr);
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
-                          void* x_perm, cudaStream_t st);
+                          void* x_perm, cudaStream_t st, unsigned long long* clk = nullptr);
 
 // balance.cu: selection-bias update and adaptive capacity from one step's
 // counts (see moe_balance_update).  bias / caps may be nullptr.
@@ -90,14 +94,27 @@ cudaError_t launch_balance_update(const Problem& p, const int32_t* counts, float
                                   int32_t* hist, int hist_slot, int hist_rows, float c_base, float gamma,
                                   int32_t* caps, cudaStream_t st);
 
+// router_fused.cu: gate GEMM (tcgen05, split-K over a thread-block cluster)
+// and the selection of route_select in one launch; BF16, logits computed
+// (router_fused_ok).  Writes logits, topk_idx, topk_w, adds the chunk
+// histogram and chunk p sums, and (zpart) *n_zpart z-loss partials, at most
+// router_fused_zparts(p) <= ceil(T/128) * 8 of them.
+bool router_fused_ok(const Problem& p);
+int router_fused_zparts(const Problem& p);
+cudaError_t launch_router_fused(const Problem& p, const void* x, const void* w_gate, const float* offset,
+                                const float* sel_bias, float* logits, int32_t* topk_idx, float* topk_w,
+                                int32_t* chunk_counts, unsigned long long* chunk_psum, float* zpart,
+                                unsigned* status, cudaStream_t st, int* n_zpart, unsigned long long* clk = nullptr);
+
 // expert_gemm.cu -- returns a moe_status value
 int router_k_splits(const Problem& p);  // slices of the tensor-core gate GEMM's reduction
 int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset, float* out,
-                          int n_splits, unsigned* status, cudaStream_t st);
+                          int n_splits, unsigned* status, cudaStream_t st, unsigned long long* clk = nullptr);
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
                       cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr,
-                      void* gu = nullptr);
+                      void* gu = nullptr, unsigned long long* clk_up = nullptr,
+                      unsigned long long* clk_down = nullptr);
 // Routed (x_perm over seg_off, p.max_rows rows) and shared (x, T rows)
 // experts in the same two launches, their tiles interleaved: requires
 // expert_ffn_mixed_ok(p) (BF16, shared experts, both on the same tile shape:
@@ -107,7 +124,8 @@ bool expert_ffn_mixed_ok(const Problem& p);
 int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t* seg_off, const void* w13,
                             const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
                             const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
-                            cudaStream_t st, cudaEvent_t after_up, int* n_kernels);
+                            cudaStream_t st, cudaEvent_t after_up, int* n_kernels,
+                            unsigned long long* clk_up = nullptr, unsigned long long* clk_down = nullptr);
 
 // expert_gemm.cu: gu = x W13^T (gate | up projections, BF16) for the backward
 int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
@@ -130,12 +148,19 @@ int launch_router_wgrad(const Problem& p, const void* dl16, int e_pad, const voi
 
 // combine.cu
 cudaError_t launch_combine(const Problem& p, const void* y_perm, const int32_t* slot_of, const float* topk_w,
-                           const void* y_shared, void* y, cudaStream_t st);
+                           const void* y_shared, void* y, cudaStream_t st, unsigned long long* clk = nullptr);
 
 // device properties (cached per device)
 int num_sms();
 
 // moe_api.cu: the moe_status value reported for a CUDA error (MOE_OK for cudaSuccess)
 int cuda_rc(cudaError_t e);
+
+// moe_api.cu: test hook of the bounded-wait abort path.  MOE_B200_TEST_STALL_NS
+// (read at every launch of the fused router and the single-CTA expert GEMM;
+// unset or 0 normally) makes those kernels' MMA thread wait that long for a
+// barrier phase that never completes, so the kernel records
+// MOE_DEV_WAIT_TIMEOUT and returns through its abort path.
+unsigned long long test_stall_ns();
 
 }  // namespace moe

@@ -6,6 +6,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -70,7 +71,9 @@ WsLayout make_layout(const Problem& p) {
   L.chunk_base = take(static_cast<size_t>(L.n_chunks) * p.E * 4);
   const int splits = (p.dtype == kBF16) ? router_k_splits(p) : 1;
   L.logit_parts = take(splits > 1 ? static_cast<size_t>(splits) * p.T * p.E * 4 : 0);
-  L.zpart = take(static_cast<size_t>(L.n_sel_blocks) * 4);
+  // z-loss partials: one per selection block, or one per CTA of the fused router
+  const size_t n_zp = std::max<size_t>(static_cast<size_t>(L.n_sel_blocks), static_cast<size_t>((p.T + 127) / 128) * 8);
+  L.zpart = take(n_zp * 4);
   L.x_perm = take(R * p.d * es);
   L.h_routed = take(R * p.F * es);
   L.y_perm = take(R * p.d * es);
@@ -144,6 +147,13 @@ static T* at(void* ws, size_t off) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+unsigned long long test_stall_ns() {
+  const char* e = getenv("MOE_B200_TEST_STALL_NS");
+  if (!e || !e[0]) return 0;
+  const unsigned long long v = strtoull(e, nullptr, 10);
+  return v > kWaitLimitNs ? kWaitLimitNs : v;
+}
+
 // Router body shared by moe_route and moe_layer_forward.
 // chunk_totals_cleared: the caller already zeroed the chunk totals;
 // stats_in_route: finalise the statistics here (else the dispatch scan does).
@@ -152,7 +162,7 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 static int route_impl(const Problem& p, const void* x, const void* w_gate, const float* offset,
                       const float* sel_bias, float* logits, int32_t* idx, float* w, float* stats, void* ws,
                       const WsLayout& L, cudaStream_t st, bool chunk_totals_cleared, bool stats_in_route,
-                      int* n_zpart, int* n_kernels) {
+                      int* n_zpart, int* n_kernels, unsigned long long* clk = nullptr) {
   unsigned* status = at<unsigned>(ws, L.status);
   // the chunk totals start at zero: the layer forward clears them with the
   // status word; a standalone call clears them here
@@ -164,7 +174,12 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
   unsigned long long* chunk_psum = at<unsigned long long>(ws, L.chunk_psum);
   float* zpart = (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr;
   int kernels = 0;
-  {
+  if (router_fused_ok(p)) {
+    if (cudaError_t e = launch_router_fused(p, x, w_gate, offset, sel_bias, logits, idx, w, chunk_counts, chunk_psum,
+                                            zpart, status, st, n_zpart, clk))
+      return cuda_rc(e);
+    kernels += 1;
+  } else {
     int n_parts = 0;
     float* parts = nullptr;
     if (!(p.flags & MOE_FLAG_LOGITS_GIVEN)) {
@@ -174,7 +189,8 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
           parts = at<float>(ws, L.logit_parts);
           n_parts = splits;
         }
-        const int rc = launch_gate_logits_tc(p, x, w_gate, offset, splits > 1 ? parts : logits, splits, status, st);
+        const int rc =
+            launch_gate_logits_tc(p, x, w_gate, offset, splits > 1 ? parts : logits, splits, status, st, clk);
         if (rc) return MOE_ERR_CUDA;
       } else {
         if (cudaError_t e = launch_gate_logits_simt(p, x, w_gate, offset, logits, st)) return cuda_rc(e);
@@ -182,7 +198,7 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
       kernels += 1;
     }
     if (cudaError_t e = launch_route_select(p, logits, parts, n_parts, sel_bias, idx, w, chunk_counts, chunk_psum,
-                                            zpart, st))
+                                            zpart, st, clk))
       return cuda_rc(e);
     kernels += 1;
     *n_zpart = route_select_zparts(p);
@@ -361,7 +377,8 @@ int moe_combine(const moe_problem_t* q, const void* y_perm, const int32_t* slot_
 
 static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
                               const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes,
-                              moe_stream_t stream, void* const* events, int32_t* n_kernels) {
+                              moe_stream_t stream, void* const* events, int32_t* n_kernels,
+                              unsigned long long* clocks) {
   Problem p;
   if (int rc = to_problem(q, &p)) return rc;
   if (int rc = check_ws(p, ws, ws_bytes)) return rc;
@@ -383,6 +400,8 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st);
   };
   int kernels = 0;
+  // the stage clock of stage s, or nullptr
+  auto clk = [&](int s) -> unsigned long long* { return clocks ? clocks + 2 * s : nullptr; };
   moe_routing_t r{};
   if (routing) r = *routing;
   float* logits = r.logits ? r.logits : at<float>(ws, L.logits);
@@ -403,7 +422,8 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
   if (cudaError_t e = mark(MOE_EV_START)) return cuda_rc(e);
   int n_zpart = 0;
   if (int rc = route_impl(p, x, w->w_gate, given ? nullptr : w->logit_offset, w->sel_bias, logits, idx, gw, stats,
-                          ws, L, st, /*chunk_totals_cleared=*/true, /*stats_in_route=*/false, &n_zpart, &kernels))
+                          ws, L, st, /*chunk_totals_cleared=*/true, /*stats_in_route=*/false, &n_zpart, &kernels,
+                          clk(MOE_CLOCK_ROUTE)))
     return rc;
   if (cudaError_t e = mark(MOE_EV_ROUTED)) return cuda_rc(e);
   // scan+rank (the histogram came from the selection kernel); the scan also
@@ -412,11 +432,11 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
                                       at<int32_t>(ws, L.chunk_base), status, st, /*counts_ready=*/true,
                                       at<unsigned long long>(ws, L.chunk_psum), stats,
                                       (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr,
-                                      n_zpart, expert_cap))
+                                      n_zpart, expert_cap, clk(MOE_CLOCK_DISPATCH)))
     return cuda_rc(e);
   kernels += dispatch_fused(p) ? 1 : 2;
   if (p.max_rows > 0) {
-    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st)) return cuda_rc(e);
+    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st, clk(MOE_CLOCK_GATHER))) return cuda_rc(e);
     kernels += 1;
   }
   if (cudaError_t e = mark(MOE_EV_DISPATCHED)) return cuda_rc(e);
@@ -428,13 +448,14 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     if (launch_expert_ffn_mixed(p, x_perm, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed), y_perm,
                                 save_gu ? at<void>(ws, L.gu_routed) : nullptr, x, w->w13_shared, w->w2_shared,
                                 at<void>(ws, L.h_shared), y_sh, save_gu ? at<void>(ws, L.gu_shared) : nullptr,
-                                status, st, up_ev, &kernels))
+                                status, st, up_ev, &kernels, clk(MOE_CLOCK_UP), clk(MOE_CLOCK_DOWN)))
       return MOE_ERR_CUDA;
     if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
   } else {
     if (p.max_rows > 0) {
       if (launch_expert_ffn(p, MOE_FFN_ROUTED, x_perm, p.max_rows, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed),
-                            y_perm, status, st, up_ev, &kernels, save_gu ? at<void>(ws, L.gu_routed) : nullptr))
+                            y_perm, status, st, up_ev, &kernels, save_gu ? at<void>(ws, L.gu_routed) : nullptr,
+                            clk(MOE_CLOCK_UP), clk(MOE_CLOCK_DOWN)))
         return MOE_ERR_CUDA;
     } else if (cudaError_t e = mark(MOE_EV_UP)) {
       return cuda_rc(e);
@@ -443,12 +464,13 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     if (p.Ns > 0) {
       if (launch_expert_ffn(p, MOE_FFN_SHARED, x, p.T, nullptr, w->w13_shared, w->w2_shared,
                             at<void>(ws, L.h_shared), y_sh, status, st, nullptr, &kernels,
-                            save_gu ? at<void>(ws, L.gu_shared) : nullptr))
+                            save_gu ? at<void>(ws, L.gu_shared) : nullptr, clk(MOE_CLOCK_SHARED),
+                            clk(MOE_CLOCK_SHARED)))
         return MOE_ERR_CUDA;
     }
   }
   if (cudaError_t e = mark(MOE_EV_SHARED)) return cuda_rc(e);
-  if (cudaError_t e = launch_combine(p, y_perm, slot_of, gw, y_sh, y, st)) return cuda_rc(e);
+  if (cudaError_t e = launch_combine(p, y_perm, slot_of, gw, y_sh, y, st, clk(MOE_CLOCK_COMBINE))) return cuda_rc(e);
   kernels += 1;
   if (cudaError_t e = mark(MOE_EV_END)) return cuda_rc(e);
   if (n_kernels) *n_kernels = kernels;
@@ -457,13 +479,22 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
 
 int moe_layer_forward(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
                       const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes, moe_stream_t stream) {
-  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, nullptr, nullptr);
+  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, nullptr, nullptr, nullptr);
 }
 
 int moe_layer_forward_profiled(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
                                const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes,
                                moe_stream_t stream, void* const* events, int32_t* n_kernels) {
-  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, events, n_kernels);
+  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, events, n_kernels, nullptr);
+}
+
+int moe_layer_forward_clocked(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,
+                              const moe_routing_t* routing, float* stats, void* ws, size_t ws_bytes,
+                              moe_stream_t stream, uint64_t* clocks) {
+  if (!clocks || (reinterpret_cast<uintptr_t>(clocks) & 7u)) return MOE_ERR_INVALID_ARG;
+  static_assert(sizeof(unsigned long long) == sizeof(uint64_t), "64-bit clocks");
+  return layer_forward_impl(q, x, w, y, routing, stats, ws, ws_bytes, stream, nullptr, nullptr,
+                            reinterpret_cast<unsigned long long*>(clocks));
 }
 
 }  // extern "C"

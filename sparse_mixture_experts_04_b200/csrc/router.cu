@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "router_select.cuh"
 
 namespace moe {
 
@@ -148,7 +149,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
                                                            float* __restrict__ topk_w, int64_t T, int E, int K,
                                                            int32_t* __restrict__ chunk_counts,
                                                            unsigned long long* __restrict__ chunk_psum,
-                                                           double pscale, float* __restrict__ zpart) {
+                                                           double pscale, float* __restrict__ zpart,
+                                                           unsigned long long* clk) {
   __shared__ float s_psum[8][32 * EPL];
   __shared__ int s_count[32 * EPL];
   __shared__ float s_z[8];
@@ -158,6 +160,7 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
   const int warp = threadIdx.x >> 5;
   pdl_wait();
   pdl_trigger();
+  stage_clock_start(clk);
   for (int e = threadIdx.x; e < 32 * EPL; e += blockDim.x) s_count[e] = 0;
   __syncthreads();
 
@@ -204,208 +207,8 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
         bias[i] = (sel_bias && e < E) ? sel_bias[e] : 0.f;
       }
     }
-    float mloc = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) mloc = fmaxf(mloc, lg[i]);
-    const float m = warp_max(mloc);
-    float ex[EPL];
-    float zloc = 0.f;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      ex[i] = (e < E) ? expf(lg[i] - m) : 0.f;
-      zloc += ex[i];
-    }
-    const float Z = warp_sum(zloc);
-    const float invZ = 1.0f / Z;
-    const float lse = m + logf(Z);
-    zacc += lse * lse;
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) pacc[i] += ex[i] * invZ;
-
-    int my_e = -1;
-    float my_ex = 0.f;
-    bool done = false;
-    if (sel_bias == nullptr || !bias_on_logit) {
-      // Ranked on 32-bit keys of float32 scores.  Without a bias the score is
-      // the float32 logit itself, so this ranking is the exact one (K rounds).
-      // Bias on p: the float32 scores s = ex/Z + b (K+1 rounds).  Each is
-      // within d = (E+8) eps p + eps (|s| + 1) of the exact p + b (eps =
-      // 2^-23; terms: expf's 2 ulp, the sum Z, 1/Z, the product, the add, and
-      // the rounding of l - m, whose effect on p is at most eps |l - m| p / 2
-      // <= eps / (2e)); if every gap between consecutive ones of the best K+1
-      // exceeds 2d, the exact ranking of the top K is the same, else the
-      // token is ranked again in float64 below.
-      const bool biased = sel_bias != nullptr;
-      unsigned k32[EPL];
-      float s32[EPL];
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        const int e = lane + 32 * i;
-        float sc = (e < E) ? (biased ? ex[i] * invZ + bias[i] : lg[i]) : 0.f;
-        if (sc != sc) sc = -INFINITY;
-        sc += 0.0f;
-        s32[i] = sc;
-        const unsigned b = __float_as_uint(sc);
-        k32[i] = e >= E ? 0u : ((b >> 31) ? ~b : (b | 0x80000000u));
-      }
-      // this lane's keys in descending order with their slots (equal keys:
-      // the lower slot, i.e. expert, first): a round only pops the winner's head
-      unsigned hk[EPL];
-      int hs[EPL];
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        hk[i] = k32[i];
-        hs[i] = i;
-      }
-#pragma unroll
-      for (int pass = 0; pass < EPL; ++pass)
-#pragma unroll
-        for (int i = pass & 1; i + 1 < EPL; i += 2)
-          if (hk[i + 1] > hk[i]) {  // slots start ascending and equal keys never swap
-            const unsigned tk = hk[i];
-            hk[i] = hk[i + 1];
-            hk[i + 1] = tk;
-            const int ts = hs[i];
-            hs[i] = hs[i + 1];
-            hs[i + 1] = ts;
-          }
-      const int rounds = biased ? K + 1 : K;
-      for (int r = 0; r < rounds && r < 32; ++r) {
-        const unsigned kmax = __reduce_max_sync(0xffffffffu, hk[0]);
-        const int best_e =
-            __reduce_min_sync(0xffffffffu, (hk[0] != 0u && hk[0] == kmax) ? lane + 32 * hs[0] : 0x7fffffff);
-        if (lane == (best_e & 31)) {
-#pragma unroll
-          for (int i = 0; i + 1 < EPL; ++i) {
-            hk[i] = hk[i + 1];
-            hs[i] = hs[i + 1];
-          }
-          hk[EPL - 1] = 0u;
-        }
-        if (lane == r) my_e = best_e;
-        if (best_e == 0x7fffffff) break;  // fewer than K+1 experts (K == E)
-      }
-      // the winners' ex and score: expert e sits in lane e & 31, slot e >> 5
-      float my_s = 0.f;
-      {
-        const int src = my_e & 31, slot = my_e >> 5;
-#pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const float a = __shfl_sync(0xffffffffu, ex[i], src);
-          const float b = __shfl_sync(0xffffffffu, s32[i], src);
-          if (i == slot) {
-            my_ex = a;
-            my_s = b;
-          }
-        }
-      }
-      const float my_p = my_ex * invZ;
-      const float s_next = __shfl_down_sync(0xffffffffu, my_s, 1);
-      const float p_next = __shfl_down_sync(0xffffffffu, my_p, 1);
-      const float eps = 1.1920928955078125e-7f;  // 2^-23
-      const float d = (static_cast<float>(E) + 8.0f) * eps * fmaxf(my_p, p_next) +
-                      eps * (fmaxf(fabsf(my_s), fabsf(s_next)) + 1.0f);
-      // with K == E there is no (K+1)-th score: the last gap only orders the set
-      const bool last_ok = lane == K - 1 && K == E;
-      const bool gap_ok = !biased || lane >= K || last_ok || (my_s - s_next > 2.0f * d);
-      done = __all_sync(0xffffffffu, gap_ok);
-      if (!done) {
-        my_e = -1;
-        my_ex = 0.f;
-      }
-    }
-    if (!done) {
-      double score[EPL];
-      if (sel_bias == nullptr) {
-  #pragma unroll
-        for (int i = 0; i < EPL; ++i) score[i] = static_cast<double>(lg[i]);
-      } else if (bias_on_logit) {
-  #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          score[i] = (e < E) ? static_cast<double>(lg[i]) + static_cast<double>(bias[i]) : -INFINITY;
-        }
-      } else {
-        const double m64 = static_cast<double>(m);
-        double ex64[EPL];
-        double z64loc = 0.0;
-  #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          ex64[i] = (e < E) ? exp(static_cast<double>(lg[i]) - m64) : 0.0;
-          z64loc += ex64[i];
-        }
-        const double z64 = warp_sum(z64loc);
-  #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-          const int e = lane + 32 * i;
-          score[i] = (e < E) ? ex64[i] / z64 + static_cast<double>(bias[i]) : -INFINITY;
-        }
-      }
-
-      // Order-preserving 64-bit keys: a larger key is a larger score (NaN ranks
-      // as -inf, -0 as +0); padding lanes and chosen experts get key 0, below
-      // every real score.  (key, index ascending) is a total order, so every
-      // lane agrees on each round's winner, which is always a valid expert.
-      unsigned long long key[EPL];
-  #pragma unroll
-      for (int i = 0; i < EPL; ++i) {
-        double sc = score[i];
-        if (sc != sc) sc = -INFINITY;
-        sc += 0.0;
-        const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(sc));
-        key[i] = (lane + 32 * i) >= E ? 0ull : ((b >> 63) ? ~b : (b | 0x8000000000000000ull));
-      }
-      // this lane's best remaining entry (equal keys: the lower slot, i.e. expert)
-      unsigned long long bk = 0;
-      int bi = 0;
-  #pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (key[i] > bk) {
-          bk = key[i];
-          bi = i;
-        }
-      for (int k = 0; k < K; ++k) {
-        // warp arg-max: high word, then low word among the maxima, then the
-        // lowest expert index among equal keys
-        const unsigned hi = static_cast<unsigned>(bk >> 32), lo = static_cast<unsigned>(bk);
-        const unsigned hmax = __reduce_max_sync(0xffffffffu, hi);
-        const unsigned lmax = __reduce_max_sync(0xffffffffu, hi == hmax ? lo : 0u);
-        const bool cand = bk != 0ull && hi == hmax && lo == lmax;
-        const int best_e = __reduce_min_sync(0xffffffffu, cand ? lane + 32 * bi : 0x7fffffff);
-        const int wl = best_e & 31;
-        float ex_mine = 0.f;
-  #pragma unroll
-        for (int i = 0; i < EPL; ++i)
-          if (i == bi) ex_mine = ex[i];
-        const float ex_sel = __shfl_sync(0xffffffffu, ex_mine, wl);
-        if (lane == wl) {  // the winner's lane drops it and finds its next best
-          bk = 0;
-  #pragma unroll
-          for (int i = 0; i < EPL; ++i) {
-            if (i == bi) key[i] = 0ull;
-          }
-          bi = 0;
-  #pragma unroll
-          for (int i = 0; i < EPL; ++i)
-            if (key[i] > bk) {
-              bk = key[i];
-              bi = i;
-            }
-        }
-        if (lane == k) {
-          my_e = best_e;
-          my_ex = ex_sel;
-        }
-      }
-    }
-    const float wsum = warp_sum(lane < K ? my_ex : 0.f);
-    if (lane < K) {
-      topk_idx[t * K + lane] = my_e;
-      topk_w[t * K + lane] = my_ex / wsum;
-      if (static_cast<unsigned>(my_e) < static_cast<unsigned>(E)) atomicAdd(&s_count[my_e], 1);
-    }
+    select_token_group<EPL, 32>(lg, bias, sel_bias != nullptr, bias_on_logit, E, K, lane, pacc, zacc, topk_idx + t * K,
+                           topk_w + t * K, s_count);
   }
 #pragma unroll
   for (int i = 0; i < EPL; ++i) s_psum[warp][lane + 32 * i] = pacc[i];
@@ -429,27 +232,32 @@ __global__ void __launch_bounds__(256) route_select_kernel(float* __restrict__ l
     if (s_count[e]) atomicAdd(&chunk_counts[chunk * E + e], s_count[e]);
     if (s > 0.f) atomicAdd(&chunk_psum[chunk * E + e], __double2ull_rn(static_cast<double>(s) * pscale));
   }
+  if (clk) {
+    __syncthreads();
+    stage_clock_end(clk);
+  }
 }
 
 int route_select_zparts(const Problem& p) { return static_cast<int>((p.T + kSelectTokens - 1) / kSelectTokens); }
 
 cudaError_t launch_route_select(const Problem& p, float* logits, const float* parts, int n_parts,
                                 const float* sel_bias, int32_t* topk_idx, float* topk_w, int32_t* chunk_counts,
-                                unsigned long long* chunk_psum, float* zpart, cudaStream_t st) {
+                                unsigned long long* chunk_psum, float* zpart, cudaStream_t st,
+                                unsigned long long* clk) {
   const unsigned blocks = static_cast<unsigned>((p.T + kSelectTokens - 1) / kSelectTokens);
   const int bias_on_logit = (p.flags & 0x2u) ? 1 : 0;
   if (p.E <= 32)
     return launch_k(route_select_kernel<1>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart, clk);
   else if (p.E <= 64)
     return launch_k(route_select_kernel<2>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart, clk);
   else if (p.E <= 128)
     return launch_k(route_select_kernel<4>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart, clk);
   else
     return launch_k(route_select_kernel<8>, dim3(blocks), dim3(256), 0, st, logits, parts, n_parts, sel_bias,
-                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart);
+                    bias_on_logit, topk_idx, topk_w, p.T, p.E, p.K, chunk_counts, chunk_psum, p_fixed_scale(p.T), zpart, clk);
 }
 
 // ----------------------------------------------------------------------------

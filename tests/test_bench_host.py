@@ -86,3 +86,31 @@ def test_shared_up_bytes_counts_weights_x_and_h():
     cfg = CONFIGS["zen_fine"]
     d, F, Ns, T = cfg.d_model, cfg.d_ff, cfg.n_shared, cfg.T
     assert bench.shared_up_bytes(cfg) == 2 * (Ns * 2 * F * d + T * d + T * Ns * F)
+
+
+def test_stage_spans_from_device_clocks():
+    """Each stage's pair holds (~earliest start, latest end); dispatch+gather
+    runs from the dispatch kernels' start to the gather's end; stages left at
+    zero (not run, or not stamped) are absent."""
+    from sparse_mixture_experts_04_b200 import _lib
+    n = _lib.NUM_CLOCKS
+    names = _lib.CLOCK_NAMES
+    row = [0] * (2 * n)
+    mask = (1 << 64) - 1
+
+    def put(name, start_ns, end_ns):
+        i = names.index(name)
+        c = (~start_ns) & mask
+        row[2 * i] = c - (1 << 64) if c >= 1 << 63 else c   # int64 as torch returns it
+        row[2 * i + 1] = end_ns
+
+    put("route", 1_000, 9_000)
+    put("dispatch", 10_000, 14_000)
+    put("gather", 14_500, 35_000)
+    put("combine", 40_000, 60_000)
+    spans = bench.stage_spans([row, row])
+    assert spans["route"] == pytest.approx(8.0)
+    assert spans["dispatch+gather"] == pytest.approx(25.0)
+    assert spans["gather"] == pytest.approx(20.5)
+    assert spans["combine"] == pytest.approx(20.0)
+    assert "up" not in spans and "shared" not in spans

@@ -391,6 +391,39 @@ def test_layer_forward_is_deterministic():
         assert torch.equal(r1[k], v), k
 
 
+@pytest.mark.parametrize("name", ["mini_mixtral", "mini_zen", "mini_decode", "ragged_bf16"])
+def test_clocked_forward_equals_the_plain_forward_and_stamps_its_stages(name):
+    """moe_layer_forward_clocked runs the same kernels (plus two atomics per
+    CTA): outputs, routing and statistics bit-identical to moe_layer_forward,
+    and every BF16 stage that ran has a span, in order along the stream."""
+    from sparse_mixture_experts_04_b200 import _lib
+    inp = inputs(name)
+    layer = MoeLayer.from_inputs(inp)
+    x = dev(inp["x"])
+    y1 = layer.forward(x).clone()
+    s1 = layer.stats.clone()
+    r1 = {k: v.clone() for k, v in layer.routing.items()}
+    clocks = torch.zeros(2 * _lib.NUM_CLOCKS, dtype=torch.int64, device="cuda")
+    y2 = torch.empty_like(y1)
+    api.moe_layer_forward_clocked(layer.prob, x, layer.weights, y2, layer.routing, layer.stats, layer.ws, clocks)
+    torch.cuda.synchronize()
+    assert api.read_device_status(layer.ws) == 0
+    assert torch.equal(y1, y2) and torch.equal(s1, layer.stats)
+    for k, v in layer.routing.items():
+        assert torch.equal(r1[k], v), k
+    us = api.stage_clock_us(clocks.cpu().tolist())
+    for st in ("route", "dispatch", "gather", "up", "down", "combine"):
+        assert us[st] is not None and 0.0 < us[st] < 1e5, (st, us)
+    c = [int(v) & 0xFFFFFFFFFFFFFFFF for v in clocks.cpu().tolist()]
+    names = _lib.CLOCK_NAMES
+    start = lambda n: (~c[2 * names.index(n)]) & 0xFFFFFFFFFFFFFFFF
+    end = lambda n: c[2 * names.index(n) + 1]
+    # each stage starts reading only after its predecessor's last CTA ended
+    order = ["route", "dispatch", "gather", "up", "down", "combine"]
+    for a, b in zip(order, order[1:]):
+        assert end(a) <= start(b), (a, b)
+
+
 def test_layer_stats_match_oracle_and_uniform_routing_gives_alpha():
     # all-equal logits: P_e = 1/E for every expert; with K = E every expert is
     # chosen by every token, so f_e = 1/E too, and the loss is exactly alpha
