@@ -235,6 +235,26 @@ int moe_expert_ffn(const moe_problem_t* p, int32_t mode, const void* x_rows, int
                    const int32_t* seg_off, const void* w13, const void* w2, void* y_rows,
                    void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_expert_ffn (ROUTED) over n_segments row segments instead of E: rows
+ * [seg_off[s], seg_off[s+1]) go through expert s % E.  This is the layout of
+ * the expert-parallel receive buffer, where every source rank's rows for the
+ * local experts arrive as one block (segments source-major, experts in order
+ * within each source), so a single message per peer needs no regrouping.
+ *   seg_off [n_segments + 1] int32 device, non-decreasing, seg_off[0] = 0,
+ *           seg_off[n_segments] <= n_rows <= moe_max_rows(p);
+ *   1 <= n_segments <= 256 (else MOE_ERR_UNSUPPORTED).
+ * With more segments than experts the rows are first copied into expert order
+ * in the workspace (each expert's rows one group, so its tiles are full and
+ * its weights stream once per tile column) and the outputs copied back to the
+ * segment order of x_rows; the result is that of computing segment by segment.
+ * Everything else (weights [E, ...], y_rows, workspace, errors) as
+ * moe_expert_ffn; FP32 problems use the CUDA-core path with the same rule.
+ * The pages state expert parallelism ("Scaling with experts", What you still
+ * pay for); this layout of its receive buffer is this library's. */
+int moe_expert_ffn_segments(const moe_problem_t* p, const void* x_rows, int64_t n_rows,
+                            const int32_t* seg_off, int32_t n_segments, const void* w13, const void* w2,
+                            void* y_rows, void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* Gate-weighted combine back to token order ("Scaling with experts", The
  * gating network: y = g1 E1(x) + g2 E2(x); A budget: dropped pairs add 0).
  *   y[t] = y_shared[t] + sum_{k: slot_of[t,k] >= 0} topk_w[t,k] * y_perm[slot_of[t,k]]
@@ -435,19 +455,21 @@ int moe_layer_forward_clocked(const moe_problem_t* p, const void* x, const moe_w
  * x_perm[seg_off[e] .. seg_off[e+1]).
  *   seg_off_all   [G, E+1] in: row s = rank s's seg_off (each starts at 0 and
  *                 never decreases)
- *   send          [E, 3] out: chunk e = {peer e / E_l, first row in this rank's
- *                 x_perm (and, on the way back, y_perm), rows}
- *   recv          [E_l * G, 3] out: chunk el*G + s = {peer s, first row in the
- *                 local buffer, rows} for local expert el from source rank s
- *   local_seg_off [E_l + 1] out: local expert el owns local rows
- *                 [local_seg_off[el], local_seg_off[el+1]) -- sources in rank
- *                 order inside each expert -- ready for moe_expert_ffn (ROUTED)
- *                 with the rank's E_l expert weights
- * Forward: send chunk e of x_perm to its peer, receive chunk (el, s) into the
- * local buffer; back: send local chunk (el, s) of the expert outputs to s,
- * receive chunk e into y_perm.  Between two ranks both sides list their chunks
- * in ascending expert order, so point-to-point messages match in posting
- * order.  Chunks with 0 rows may be skipped by both sides.
+ *   send          [G, 3] out: chunk q = {peer q, first row in this rank's
+ *                 x_perm (and, on the way back, y_perm), rows}: the rows of
+ *                 the experts peer q holds are contiguous in x_perm, from
+ *                 seg_off[q E_l] to seg_off[(q+1) E_l]
+ *   recv          [G, 3] out: chunk s = {peer s, first row in the local
+ *                 buffer, rows}: source s's block, blocks in rank order
+ *   local_seg_off [G * E_l + 1] out: segment s*E_l + el = the rows of local
+ *                 expert el from source s, [local_seg_off[i], local_seg_off[i+1])
+ *                 -- ready for moe_expert_ffn_segments with n_segments = G E_l
+ *                 and the rank's E_l expert weights (segment i uses expert
+ *                 i % E_l)
+ * Forward: send chunk q of x_perm to peer q, receive chunk s into the local
+ * buffer; back: send local chunk s of the expert outputs to s, receive chunk q
+ * into y_perm.  One message each way per pair of ranks.  Chunks with 0 rows
+ * may be skipped by both sides.
  * Errors: MOE_ERR_INVALID_ARG for NULL pointers, G < 1, rank out of range,
  * E % G != 0, offsets not starting at 0 or decreasing, more than INT32_MAX
  * local rows. */

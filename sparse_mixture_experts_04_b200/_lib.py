@@ -27,7 +27,7 @@ DEV_BAD_EXPERT, DEV_WAIT_TIMEOUT = 0x1, 0x2
 EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_rows", "moe_workspace_size",
             "moe_reset_device_status", "moe_read_device_status", "moe_route", "moe_dispatch",
             "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
-            "moe_layer_forward_clocked",
+            "moe_layer_forward_clocked", "moe_expert_ffn_segments",
             "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update", "moe_backward_workspace_size",
             "moe_layer_backward", "moe_ep_plan")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
@@ -94,6 +94,8 @@ def lib() -> ctypes.CDLL:
     L.moe_dispatch.restype = ctypes.c_int
     L.moe_expert_ffn.argtypes = [PP, i32, P, i64, P, P, P, P, P, sz, P]
     L.moe_expert_ffn.restype = ctypes.c_int
+    L.moe_expert_ffn_segments.argtypes = [PP, P, i64, P, i32, P, P, P, P, sz, P]
+    L.moe_expert_ffn_segments.restype = ctypes.c_int
     L.moe_combine.argtypes = [PP, P, P, P, P, P, P, sz, P]
     L.moe_combine.restype = ctypes.c_int
     L.moe_layer_forward.argtypes = [PP, P, ctypes.POINTER(MoeWeights), P, ctypes.POINTER(MoeRouting), P, P, sz, P]

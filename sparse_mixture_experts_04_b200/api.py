@@ -17,7 +17,7 @@ from ._lib import (BIAS_UPDATE_PROPORTIONAL, BIAS_UPDATE_SIGN, DTYPE_BF16, DTYPE
                    MoeError, MoeGrads, MoeProblem, MoeRouting, MoeWeights)
 
 __all__ = ["MoeError", "MoeProblem", "make_problem", "workspace_size", "capacity", "max_rows", "alloc_workspace",
-           "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_forward",
+           "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_expert_ffn_segments", "moe_combine", "moe_layer_forward",
            "moe_layer_forward_profiled", "moe_layer_forward_clocked", "stage_clock_us", "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update",
            "moe_layer_backward", "backward_workspace_size", "alloc_backward_workspace", "moe_ep_plan",
            "reset_device_status", "read_device_status", "FLAG_LOGITS_GIVEN", "FLAG_BIAS_LOGIT",
@@ -132,6 +132,14 @@ def moe_expert_ffn(prob, mode, x_rows, n_rows, seg_off, w13, w2, y_rows, ws, str
     _lib.check("moe_expert_ffn", rc)
 
 
+def moe_expert_ffn_segments(prob, x_rows, n_rows, seg_off, n_segments, w13, w2, y_rows, ws, stream=None):
+    """Routed experts over n_segments row segments; segment i uses expert i % E."""
+    _lib.check("moe_expert_ffn_segments",
+               _lib.lib().moe_expert_ffn_segments(ctypes.byref(prob), _p(x_rows), int(n_rows), _p(seg_off),
+                                                  int(n_segments), _p(w13), _p(w2), _p(y_rows), _p(ws), ws.numel(),
+                                                  _stream(stream)))
+
+
 def moe_combine(prob, y_perm, slot_of, topk_w, y_shared, y, ws, stream=None):
     rc = _lib.lib().moe_combine(ctypes.byref(prob), _p(y_perm), _p(slot_of), _p(topk_w), _p(y_shared), _p(y),
                                 _p(ws), ws.numel(), _stream(stream))
@@ -230,18 +238,18 @@ def moe_layer_backward(prob, x, weights: dict, routing: dict | None, fwd_ws, dy,
 
 def moe_ep_plan(n_ranks: int, rank: int, n_experts: int, seg_off_all) -> tuple:
     """Expert-parallel exchange plan (host function, no device).  seg_off_all
-    [n_ranks, E+1] int32 (CPU) -> (send [E, 3], recv [E_l*n_ranks, 3],
-    local_seg_off [E_l+1]) int32 CPU tensors; see include/moe_b200.h."""
+    [n_ranks, E+1] int32 (CPU) -> (send [G, 3], recv [G, 3],
+    local_seg_off [G*E_l+1]) int32 CPU tensors; see include/moe_b200.h."""
     so = torch.as_tensor(seg_off_all, dtype=torch.int32).contiguous()
     if so.device.type != "cpu":
         raise ValueError("moe_ep_plan takes host (CPU) segment offsets")
     G, E = int(n_ranks), int(n_experts)
     El = E // G if G > 0 else 0
-    send = torch.empty((max(E, 1), 3), dtype=torch.int32)
-    recv = torch.empty((max(El * G, 1), 3), dtype=torch.int32)
-    local = torch.empty(El + 1, dtype=torch.int32)
+    send = torch.empty((max(G, 1), 3), dtype=torch.int32)
+    recv = torch.empty((max(G, 1), 3), dtype=torch.int32)
+    local = torch.empty(G * El + 1, dtype=torch.int32)
     if so.numel() != G * (E + 1):
         raise ValueError(f"seg_off_all has {so.numel()} entries, expected {G}x{E + 1}")
     rc = _lib.lib().moe_ep_plan(G, int(rank), E, so.data_ptr(), send.data_ptr(), recv.data_ptr(), local.data_ptr())
     _lib.check("moe_ep_plan", rc)
-    return send[:E], recv[:El * G], local
+    return send[:G], recv[:G], local

@@ -473,4 +473,77 @@ cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, 
                   static_cast<uint4*>(x_perm), clk);
 }
 
+// Segment regrouping (moe_expert_ffn_segments): segment s holds expert s % E
+// (source s / E); expert-major order lists every source's rows of expert 0,
+// then of expert 1, ... (sources ascending inside each expert).  One thread:
+// n_seg <= kMaxSegments.
+__global__ void segment_regroup_plan_kernel(const int32_t* __restrict__ seg_off, int n_seg, int E,
+                                            int32_t* __restrict__ dst_off, int32_t* __restrict__ expert_off) {
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x != 0) return;
+  const int n_src = (n_seg + E - 1) / E;
+  int run = 0;
+  for (int e = 0; e < E; ++e) {
+    expert_off[e] = run;
+    for (int s = 0; s < n_src; ++s) {
+      const int seg = s * E + e;
+      if (seg >= n_seg) continue;
+      dst_off[seg] = run;
+      run += seg_off[seg + 1] - seg_off[seg];
+    }
+  }
+  expert_off[E] = run;
+}
+
+// Row r of segment s (segment order) <-> row dst_off[s] + (r - seg_off[s])
+// (expert-major order); one warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) segment_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                           const int32_t* __restrict__ seg_off,
+                                                           const int32_t* __restrict__ dst_off, int n_seg,
+                                                           int64_t n_rows, int vec_per_row, int to_expert) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t rows = min(n_rows, static_cast<int64_t>(seg_off[n_seg]));
+  for (int64_t r = warp0; r < rows; r += n_warps) {
+    int lo = 0, hi = n_seg - 1;  // the segment holding row r: largest s with seg_off[s] <= r
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (seg_off[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int64_t q = dst_off[lo] + (r - seg_off[lo]);
+    if (q < 0 || q >= n_rows) continue;
+    const uint4* from = src + (to_expert ? r : q) * vec_per_row;
+    uint4* to = dst + (to_expert ? q : r) * vec_per_row;
+    for (int v0 = lane; v0 < vec_per_row; v0 += 32 * kGatherUnroll) {
+      uint4 buf[kGatherUnroll];
+#pragma unroll
+      for (int j = 0; j < kGatherUnroll; ++j)
+        if (v0 + 32 * j < vec_per_row) buf[j] = from[v0 + 32 * j];
+#pragma unroll
+      for (int j = 0; j < kGatherUnroll; ++j)
+        if (v0 + 32 * j < vec_per_row) to[v0 + 32 * j] = buf[j];
+    }
+  }
+}
+
+cudaError_t launch_segment_regroup_plan(const int32_t* seg_off, int n_seg, int E, int32_t* dst_off,
+                                        int32_t* expert_off, cudaStream_t st) {
+  return launch_k(segment_regroup_plan_kernel, dim3(1), dim3(32), 0, st, seg_off, n_seg, E, dst_off, expert_off);
+}
+
+cudaError_t launch_segment_copy(const void* src, void* dst, const int32_t* seg_off, const int32_t* dst_off, int n_seg,
+                                int64_t n_rows, int row_bytes, bool to_expert, cudaStream_t st) {
+  if (n_rows <= 0) return cudaSuccess;
+  int64_t blocks = (n_rows + 7) / 8;
+  const int64_t cap_blocks = static_cast<int64_t>(num_sms()) * 16;
+  if (blocks > cap_blocks) blocks = cap_blocks;
+  return launch_k(segment_copy_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                  static_cast<const uint4*>(src), static_cast<uint4*>(dst), seg_off, dst_off, n_seg, n_rows,
+                  row_bytes / 16, to_expert ? 1 : 0);
+}
+
 }  // namespace moe

@@ -9,15 +9,16 @@
 // Rank q of G holds the global experts [q*E_l, (q+1)*E_l), E_l = E/G.  Every
 // rank routes and dispatches its own tokens exactly as a single device would
 // (so its capacity cut and statistics are its own batch's), which leaves the
-// kept rows of global expert e at x_perm[seg_off[e] .. seg_off[e+1]).  The plan
-// turns all ranks' segment offsets into
-//   - one send chunk per global expert (to the expert's owner), and
-//   - one receive chunk per (local expert, source rank), placed so that the
-//     local buffer is grouped by local expert, sources in rank order inside
-//     each expert: the grouped expert GEMM then runs on it unchanged.
-// The return trip is the same table read backwards.  Between one pair of
-// ranks, both sides list their chunks in ascending expert order, so
-// point-to-point messages between the pair match in posting order.
+// kept rows of global expert e at x_perm[seg_off[e] .. seg_off[e+1]): the rows
+// for the experts of peer q are ONE contiguous block of x_perm.  So the plan is
+//   - one send chunk per peer (that block),
+//   - one receive chunk per source rank, the blocks laid end to end in rank
+//     order (source-major), and
+//   - G * E_l row segments over that buffer, segment s*E_l + el holding source
+//     s's rows for local expert el, which the grouped expert GEMM runs as
+//     they lie (moe_expert_ffn_segments: segment i uses expert i % E_l).
+// The return trip is the same table read backwards.  One message each way
+// per pair of ranks.
 
 #include <cstdint>
 
@@ -37,26 +38,24 @@ extern "C" int moe_ep_plan(int32_t n_ranks, int32_t rank, int32_t n_experts, con
       if (so[e + 1] < so[e]) return MOE_ERR_INVALID_ARG;
   }
   const int32_t* mine = seg_off_all + static_cast<int64_t>(rank) * (E + 1);
-  for (int e = 0; e < E; ++e) {
-    send[3 * e + 0] = e / El;
-    send[3 * e + 1] = mine[e];
-    send[3 * e + 2] = mine[e + 1] - mine[e];
+  for (int q = 0; q < G; ++q) {
+    send[3 * q + 0] = q;
+    send[3 * q + 1] = mine[q * El];
+    send[3 * q + 2] = mine[(q + 1) * El] - mine[q * El];
   }
   int64_t off = 0;
-  for (int el = 0; el < El; ++el) {
-    local_seg_off[el] = static_cast<int32_t>(off);
-    const int e = rank * El + el;
-    for (int s = 0; s < G; ++s) {
-      const int32_t* so = seg_off_all + static_cast<int64_t>(s) * (E + 1);
-      const int32_t rows = so[e + 1] - so[e];
-      int32_t* c = recv + 3 * (static_cast<int64_t>(el) * G + s);
-      c[0] = s;
-      c[1] = static_cast<int32_t>(off);
-      c[2] = rows;
-      off += rows;
-      if (off > INT32_MAX) return MOE_ERR_INVALID_ARG;
+  for (int s = 0; s < G; ++s) {
+    const int32_t* so = seg_off_all + static_cast<int64_t>(s) * (E + 1);
+    const int32_t first = so[rank * El];
+    recv[3 * s + 0] = s;
+    recv[3 * s + 1] = static_cast<int32_t>(off);
+    recv[3 * s + 2] = so[(rank + 1) * El] - first;
+    for (int el = 0; el < El; ++el) {
+      local_seg_off[s * El + el] = static_cast<int32_t>(off + (so[rank * El + el] - first));
     }
+    off += so[(rank + 1) * El] - first;
+    if (off > INT32_MAX) return MOE_ERR_INVALID_ARG;
   }
-  local_seg_off[El] = static_cast<int32_t>(off);
+  local_seg_off[G * El] = static_cast<int32_t>(off);
   return MOE_OK;
 }

@@ -89,6 +89,10 @@ struct GemmArgs {
   unsigned long long* clk;
   // single-CTA kernel: abort-path test hook (test_stall), 0 normally
   unsigned long long stall_ns;
+  // > 0: group g is computed with the weights of expert g % weight_mod (row
+  // segments that repeat the experts, e.g. one run of experts per source rank
+  // in the expert-parallel receive buffer); 0: expert g
+  int weight_mod;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -124,6 +128,7 @@ constexpr int gemm_smem_bytes() {
 
 struct TileInfo {
   int g, row0, row_end, n0;
+  int w;        // expert whose weights the tile uses (g, or g % weight_mod)
   bool swap;    // operand-swapped remainder tile (pair kernel only)
   bool second;  // tile of the pair kernel's second problem
 };
@@ -156,6 +161,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   }
   TileInfo ti;
   ti.g = lo;
+  ti.w = a.weight_mod > 0 ? lo % a.weight_mod : lo;
   int base;
   const int rows = group_rows(a, lo, &base);
   const int mt = (rows + BM - 1) / BM;
@@ -425,10 +431,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           tma_load_2d(a_dst, mA, &full[stage], kg * A.K + kk, ti.row0);
           if (EPI == EPI_SWIGLU) {
-            tma_load_3d(b_dst, mB, &full[stage], kk, ti.n0, 2 * ti.g);
-            tma_load_3d(b_dst + C::kBBytes / 2, mB, &full[stage], kk, ti.n0, 2 * ti.g + 1);
+            tma_load_3d(b_dst, mB, &full[stage], kk, ti.n0, 2 * ti.w);
+            tma_load_3d(b_dst + C::kBBytes / 2, mB, &full[stage], kk, ti.n0, 2 * ti.w + 1);
           } else if (EPI == EPI_BF16) {
-            tma_load_3d(b_dst, mB, &full[stage], kk, ti.n0, ti.g * A.k_groups + kg);
+            tma_load_3d(b_dst, mB, &full[stage], kk, ti.n0, ti.w * A.k_groups + kg);
           } else {
             tma_load_3d(b_dst, mB, &full[stage], kk, 0, 0);
           }
@@ -826,9 +832,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (merge) {
             const CUtensorMap* wmap = deep ? (ti.second ? &tmB64d_2 : &tmB64d) : mB64;
             if (EPI == EPI_SWIGLU)  // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
-              tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.g, kk0 / kBK);
+              tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.w, kk0 / kBK);
             else
-              tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.g * A.k_groups + kg,
+              tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 128 * static_cast<int>(rank), ti.w * A.k_groups + kg,
                                kk0 / kBK);
           } else {
 #pragma unroll
@@ -837,12 +843,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               uint8_t* bc = b_dst + c * kPairChunk;
               if (EPI == EPI_SWIGLU && ti.swap) {
                 const int f = ti.n0 + 64 * static_cast<int>(rank);
-                tma_load_3d_pair(bc, mB64, bar, kk, f, 2 * ti.g);
-                tma_load_3d_pair(bc + kPairChunk / 2, mB64, bar, kk, f, 2 * ti.g + 1);
+                tma_load_3d_pair(bc, mB64, bar, kk, f, 2 * ti.w);
+                tma_load_3d_pair(bc + kPairChunk / 2, mB64, bar, kk, f, 2 * ti.w + 1);
               } else if (EPI == EPI_SWIGLU) {
-                tma_load_3d_pair(bc, mB, bar, kk, ti.n0, 2 * ti.g + static_cast<int>(rank));
+                tma_load_3d_pair(bc, mB, bar, kk, ti.n0, 2 * ti.w + static_cast<int>(rank));
               } else {
-                tma_load_3d_pair(bc, mB, bar, kk, ti.n0 + 128 * static_cast<int>(rank), ti.g * A.k_groups + kg);
+                tma_load_3d_pair(bc, mB, bar, kk, ti.n0 + 128 * static_cast<int>(rank), ti.w * A.k_groups + kg);
               }
             }
           }
@@ -1296,7 +1302,8 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const float* __restrict__
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // ty: 8 row groups of 4 rows
   float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
   for (int kg = 0; kg < args.k_groups; ++kg) {
-    const float* Bm = B + static_cast<int64_t>(g * args.k_groups + kg) * b_group_stride;
+    const int wg = args.weight_mod > 0 ? g % args.weight_mod : g;
+    const float* Bm = B + static_cast<int64_t>(wg * args.k_groups + kg) * b_group_stride;
     for (int k0 = 0; k0 < args.K; k0 += 32) {
       for (int i = threadIdx.x; i < 32 * 32; i += 256) {
         const int rr = i / 32, kc = i % 32;
@@ -1337,14 +1344,17 @@ __global__ void __launch_bounds__(256) ffn_simt_kernel(const float* __restrict__
 }
 
 static int ffn_simt(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
-                    const void* w13, const void* w2, void* h, void* y_rows, cudaStream_t st, cudaEvent_t after_up) {
+                    const void* w13, const void* w2, void* h, void* y_rows, cudaStream_t st, cudaEvent_t after_up,
+                    int n_seg) {
   const bool routed = mode == 0;
-  const int G = routed ? p.E : p.Ns;
+  const int G = routed ? (n_seg > 0 ? n_seg : p.E) : p.Ns;
   int64_t max_group_rows = routed ? (p.cap < 0 ? p.T : (p.cap < p.T ? p.cap : p.T)) : n_rows;
+  if (n_seg > 0) max_group_rows = n_rows;  // a segment may hold any number of the rows
   if (max_group_rows > n_rows) max_group_rows = n_rows;
   if (max_group_rows <= 0) return 0;
   GemmArgs up{};
   up.n_groups = G;
+  up.weight_mod = routed && n_seg > 0 ? p.E : 0;
   up.seg_off = routed ? seg_off : nullptr;
   up.n_rows = static_cast<int>(n_rows);
   up.N = p.F;
@@ -1359,7 +1369,8 @@ static int ffn_simt(const Problem& p, int mode, const void* x_rows, int64_t n_ro
     return -3;
   if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
   GemmArgs dn{};
-  dn.n_groups = routed ? p.E : 1;
+  dn.n_groups = routed ? G : 1;
+  dn.weight_mod = up.weight_mod;
   dn.seg_off = routed ? seg_off : nullptr;
   dn.n_rows = static_cast<int>(n_rows);
   dn.N = p.d;
@@ -1417,7 +1428,7 @@ static int ffn_tile_mode(const Problem& p, bool routed, int64_t n_rows) {
 // at 2g+1; swap tiles take 64 gate and the same 64 up rows per CTA.
 static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, int64_t n_rows,
                             const int32_t* seg_off, const void* w13, void* h, void* gu, unsigned* status, bool tail,
-                            PairProblem* q) {
+                            PairProblem* q, int n_seg = 0) {
   const int G = routed ? p.E : p.Ns;
   const bool merged = merged_k_ok(p.d);
   if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, x_rows, p.d, n_rows, merged) ||
@@ -1431,7 +1442,8 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
   }
   GemmArgs& a = q->a;
   a = GemmArgs{};
-  a.n_groups = G;
+  a.n_groups = n_seg > 0 ? n_seg : G;  // routed row segments (n_seg: expert = segment % E)
+  a.weight_mod = n_seg > 0 ? G : 0;
   a.seg_off = routed ? seg_off : nullptr;
   a.n_rows = static_cast<int>(n_rows);
   a.N = p.F;
@@ -1448,8 +1460,8 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
   a.row_mode = tail ? 1 : 0;  // 1: full 256-row blocks only
   a.merged_k = merged ? 1 : 0;
   a.deep_swap = merged && deep_swap_on() ? 1 : 0;
-  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
-  q->tile_bound = (mt / 2 + G) * cdiv(p.F, 128);
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + a.n_groups : G * cdiv(n_rows, kBM);
+  q->tile_bound = (mt / 2 + a.n_groups) * cdiv(p.F, 128);
   return true;
 }
 
@@ -1457,7 +1469,8 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
 // B = w2 [G, d, F] viewed as (F, d, G); a pair CTA stages half of the 256 B
 // rows.  Shared: one group whose reduction runs over all N_s experts.
 static bool down_pair_problem(const Problem& p, bool routed, const void* h, int64_t n_rows, const int32_t* seg_off,
-                              const void* w2, void* y_rows, unsigned* status, bool tail, PairProblem* q) {
+                              const void* w2, void* y_rows, unsigned* status, bool tail, PairProblem* q,
+                              int n_seg = 0) {
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
   const bool merged = merged_k_ok(p.F);
@@ -1472,7 +1485,8 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   }
   GemmArgs& a = q->a;
   a = GemmArgs{};
-  a.n_groups = routed ? G : 1;
+  a.n_groups = routed ? (n_seg > 0 ? n_seg : G) : 1;
+  a.weight_mod = routed && n_seg > 0 ? G : 0;
   a.seg_off = routed ? seg_off : nullptr;
   a.n_rows = static_cast<int>(n_rows);
   a.N = p.d;
@@ -1486,7 +1500,7 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   a.row_mode = tail ? 1 : 0;
   a.merged_k = merged ? 1 : 0;
   a.deep_swap = merged && deep_swap_on() ? 1 : 0;
-  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + a.n_groups : cdiv(n_rows, kBM);
   q->tile_bound = (mt / 2 + a.n_groups) * cdiv(p.d, 256);
   return true;
 }
@@ -1503,7 +1517,7 @@ struct SingleProblem {
 // 2g, up rows at 2g+1).
 static bool up_single_problem(const Problem& p, bool routed, const void* x_rows, int64_t n_rows,
                               const int32_t* seg_off, const void* w13, void* h, void* gu, unsigned* status,
-                              SingleProblem* q) {
+                              SingleProblem* q, int n_seg = 0) {
   const int G = routed ? p.E : p.Ns;
   const uint64_t da[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(n_rows)};
   const uint32_t ba[2] = {kBK, kBM};
@@ -1513,7 +1527,8 @@ static bool up_single_problem(const Problem& p, bool routed, const void* x_rows,
   GemmArgs& a = q->a;
   a = GemmArgs{};
   a.stall_ns = test_stall_ns();
-  a.n_groups = G;
+  a.n_groups = n_seg > 0 ? n_seg : G;
+  a.weight_mod = n_seg > 0 ? G : 0;
   a.seg_off = routed ? seg_off : nullptr;
   a.n_rows = static_cast<int>(n_rows);
   a.N = p.F;
@@ -1527,7 +1542,7 @@ static bool up_single_problem(const Problem& p, bool routed, const void* x_rows,
   a.gu = gu;
   a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
   a.gu_col_stride = routed ? 0 : 2 * p.F;
-  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : G * cdiv(n_rows, kBM);
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + a.n_groups : G * cdiv(n_rows, kBM);
   q->tile_bound = mt * cdiv(p.F, 128);
   return true;
 }
@@ -1536,7 +1551,7 @@ static bool up_single_problem(const Problem& p, bool routed, const void* x_rows,
 // viewed as (F, d, G) with 256-row boxes.
 static bool down_single_problem(const Problem& p, bool routed, const void* h, int64_t n_rows,
                                 const int32_t* seg_off, const void* w2, void* y_rows, unsigned* status,
-                                SingleProblem* q) {
+                                SingleProblem* q, int n_seg = 0) {
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
   const uint64_t da[2] = {static_cast<uint64_t>(h_cols), static_cast<uint64_t>(n_rows)};
@@ -1547,7 +1562,8 @@ static bool down_single_problem(const Problem& p, bool routed, const void* h, in
   GemmArgs& a = q->a;
   a = GemmArgs{};
   a.stall_ns = test_stall_ns();
-  a.n_groups = routed ? G : 1;
+  a.n_groups = routed ? (n_seg > 0 ? n_seg : G) : 1;
+  a.weight_mod = routed && n_seg > 0 ? G : 0;
   a.seg_off = routed ? seg_off : nullptr;
   a.n_rows = static_cast<int>(n_rows);
   a.N = p.d;
@@ -1558,7 +1574,7 @@ static bool down_single_problem(const Problem& p, bool routed, const void* h, in
   a.out_col_stride = 0;
   a.status = status;
   a.swap_max = swap_max_rows();
-  const int64_t mt = routed ? cdiv(n_rows, kBM) + G : cdiv(n_rows, kBM);
+  const int64_t mt = routed ? cdiv(n_rows, kBM) + a.n_groups : cdiv(n_rows, kBM);
   q->tile_bound = mt * cdiv(p.d, 256);
   return true;
 }
@@ -1569,11 +1585,11 @@ static bool down_single_problem(const Problem& p, bool routed, const void* h, in
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status, cudaStream_t st,
                       cudaEvent_t after_up, int* n_kernels, void* gu, unsigned long long* clk_up,
-                      unsigned long long* clk_down) {
+                      unsigned long long* clk_down, int n_seg) {
   if (n_rows <= 0) return 0;
   if (p.dtype == kF32) {
     if (n_kernels) *n_kernels += 2;
-    return ffn_simt(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, st, after_up);
+    return ffn_simt(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, st, after_up, n_seg);
   }
   const bool routed = mode == 0;
   const int G = routed ? p.E : p.Ns;
@@ -1592,7 +1608,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     CUtensorMap ta, tb;
     if (pair) {
       PairProblem q;
-      if (!up_pair_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, tail, &q)) return -3;
+      if (!up_pair_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, tail, &q, n_seg)) return -3;
       q.a.clk = clk_up;
       int rc = run_pair_gemm<EPI_SWIGLU>(q, nullptr, st);
       if (rc) return rc;
@@ -1602,12 +1618,12 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
         a.swap_max = 0;
         a.merged_k = 0;
         if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
-        rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, 2 * G * cdiv(p.F, 128), st);
+        rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.F, 128), st);
         if (rc) return rc;
       }
     } else {
       SingleProblem q;
-      if (!up_single_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, &q)) return -3;
+      if (!up_single_problem(p, routed, x_rows, n_rows, seg_off, w13, h, gu, status, &q, n_seg)) return -3;
       q.a.clk = clk_up;
       const int rc = run_gemm<EPI_SWIGLU, 256, 4>(q.ta, q.tb, q.a, q.tile_bound, st);
       if (rc) return rc;
@@ -1624,7 +1640,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
     if (pair) {
       PairProblem q;
-      if (!down_pair_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, tail, &q)) return -3;
+      if (!down_pair_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, tail, &q, n_seg)) return -3;
       q.a.clk = clk_down;
       int rc = run_pair_gemm<EPI_BF16>(q, nullptr, st);
       if (rc) return rc;
@@ -1638,7 +1654,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
       }
     } else {
       SingleProblem q;
-      if (!down_single_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, &q)) return -3;
+      if (!down_single_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, &q, n_seg)) return -3;
       q.a.clk = clk_down;
       const int rc = run_gemm<EPI_BF16, 256, 4>(q.ta, q.tb, q.a, q.tile_bound, st);
       if (rc) return rc;

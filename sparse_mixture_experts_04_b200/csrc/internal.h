@@ -15,6 +15,7 @@ constexpr int kMaxTopK = 32;
 constexpr int kDispatchChunk = 256;  // tokens per block in the dispatch kernels
 constexpr int kSelectTokens = 8;     // tokens per block in the selection kernel (one per warp)
 constexpr int kMaxLogitParts = 8;    // most slices of the split-K gate GEMM
+constexpr int kMaxSegments = 256;    // moe_expert_ffn_segments
 
 enum Dtype { kBF16 = 0, kF32 = 1 };
 
@@ -34,6 +35,7 @@ struct Problem {
 struct WsLayout {
   size_t status, logits, topk_idx, topk_w, counts, kept, seg_off, slot_of, perm;
   size_t chunk_counts, chunk_psum, chunk_base, logit_parts, zpart;
+  size_t seg_map;  // moe_expert_ffn_segments: [kMaxSegments] destinations + [kMaxSegments + 1] expert offsets
   size_t zero_bytes;  // status word + chunk histogram + chunk p sums: cleared together at offset 0
   size_t x_perm, h_routed, y_perm, h_shared, y_shared;
   size_t gu_routed, gu_shared;  // with MOE_FLAG_SAVE_GU: the gate/up projections for the backward
@@ -88,23 +90,36 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* 
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
                           void* x_perm, cudaStream_t st, unsigned long long* clk = nullptr);
 
+// dispatch.cu: rows of n_seg segments (segment s = source s / E, expert s % E)
+// moved into expert-major order and back: segment_regroup_plan writes each
+// segment's first row in expert-major order (dst_off [n_seg]) and the experts'
+// offsets (expert_off [E + 1]); segment_copy copies rows src -> dst with
+// to_expert (segment order -> expert-major) or back (expert-major -> segment order).
+cudaError_t launch_segment_regroup_plan(const int32_t* seg_off, int n_seg, int E, int32_t* dst_off,
+                                        int32_t* expert_off, cudaStream_t st);
+cudaError_t launch_segment_copy(const void* src, void* dst, const int32_t* seg_off, const int32_t* dst_off, int n_seg,
+                                int64_t n_rows, int row_bytes, bool to_expert, cudaStream_t st);
+
 // balance.cu: selection-bias update and adaptive capacity from one step's
 // counts (see moe_balance_update).  bias / caps may be nullptr.
 cudaError_t launch_balance_update(const Problem& p, const int32_t* counts, float* bias, float rate, int mode,
                                   int32_t* hist, int hist_slot, int hist_rows, float c_base, float gamma,
                                   int32_t* caps, cudaStream_t st);
 
-// router_fused.cu: gate GEMM (tcgen05, split-K over a thread-block cluster)
-// and the selection of route_select in one launch; BF16, logits computed
-// (router_fused_ok).  Writes logits, topk_idx, topk_w, adds the chunk
-// histogram and chunk p sums, and (zpart) *n_zpart z-loss partials, at most
+// router_fused.cu: gate GEMM (tcgen05, split-K over a thread-block cluster,
+// partials summed through distributed shared memory); BF16, logits computed
+// (router_fused_ok).  Writes the logits; with select (router_selects(p)) also
+// ranks the tokens like route_select: topk_idx, topk_w, the chunk histogram
+// and chunk p sums, and (zpart) *n_zpart z-loss partials, at most
 // router_fused_zparts(p) <= ceil(T/128) * 8 of them.
 bool router_fused_ok(const Problem& p);
+bool router_selects(const Problem& p);
 int router_fused_zparts(const Problem& p);
 cudaError_t launch_router_fused(const Problem& p, const void* x, const void* w_gate, const float* offset,
                                 const float* sel_bias, float* logits, int32_t* topk_idx, float* topk_w,
                                 int32_t* chunk_counts, unsigned long long* chunk_psum, float* zpart,
-                                unsigned* status, cudaStream_t st, int* n_zpart, unsigned long long* clk = nullptr);
+                                unsigned* status, cudaStream_t st, int* n_zpart, unsigned long long* clk,
+                                bool select);
 
 // expert_gemm.cu -- returns a moe_status value
 int router_k_splits(const Problem& p);  // slices of the tensor-core gate GEMM's reduction
@@ -114,7 +129,9 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
                       cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr,
                       void* gu = nullptr, unsigned long long* clk_up = nullptr,
-                      unsigned long long* clk_down = nullptr);
+                      unsigned long long* clk_down = nullptr, int n_seg = 0);
+// (routed mode) n_seg > 0: seg_off has n_seg + 1 entries and row segment s is
+// computed with expert s % p.E (moe_expert_ffn_segments).
 // Routed (x_perm over seg_off, p.max_rows rows) and shared (x, T rows)
 // experts in the same two launches, their tiles interleaved: requires
 // expert_ffn_mixed_ok(p) (BF16, shared experts, both on the same tile shape:

@@ -74,6 +74,7 @@ WsLayout make_layout(const Problem& p) {
   // z-loss partials: one per selection block, or one per CTA of the fused router
   const size_t n_zp = std::max<size_t>(static_cast<size_t>(L.n_sel_blocks), static_cast<size_t>((p.T + 127) / 128) * 8);
   L.zpart = take(n_zp * 4);
+  L.seg_map = take(static_cast<size_t>(2 * kMaxSegments + 1) * 4);
   L.x_perm = take(R * p.d * es);
   L.h_routed = take(R * p.F * es);
   L.y_perm = take(R * p.d * es);
@@ -175,10 +176,20 @@ static int route_impl(const Problem& p, const void* x, const void* w_gate, const
   float* zpart = (stats && (p.flags & MOE_FLAG_EXTENDED_STATS)) ? at<float>(ws, L.zpart) : nullptr;
   int kernels = 0;
   if (router_fused_ok(p)) {
+    // the gate GEMM with its split reduction summed on chip; the tokens are
+    // ranked in the same kernel, or by the selection kernel right after it
+    const bool sel_here = router_selects(p);
     if (cudaError_t e = launch_router_fused(p, x, w_gate, offset, sel_bias, logits, idx, w, chunk_counts, chunk_psum,
-                                            zpart, status, st, n_zpart, clk))
+                                            zpart, status, st, n_zpart, clk, sel_here))
       return cuda_rc(e);
     kernels += 1;
+    if (!sel_here) {
+      if (cudaError_t e = launch_route_select(p, logits, nullptr, 0, sel_bias, idx, w, chunk_counts, chunk_psum, zpart,
+                                              st, clk))
+        return cuda_rc(e);
+      kernels += 1;
+      *n_zpart = route_select_zparts(p);
+    }
   } else {
     int n_parts = 0;
     float* parts = nullptr;
@@ -361,6 +372,42 @@ int moe_expert_ffn(const moe_problem_t* q, int32_t mode, const void* x_rows, int
   const int rc = launch_expert_ffn(p, mode, x_rows, n_rows, seg_off, w13, w2, h, y_rows, at<unsigned>(ws, L.status),
                                    reinterpret_cast<cudaStream_t>(stream));
   return rc ? MOE_ERR_CUDA : MOE_OK;
+}
+
+int moe_expert_ffn_segments(const moe_problem_t* q, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
+                            int32_t n_segments, const void* w13, const void* w2, void* y_rows, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+  Problem p;
+  if (int rc = to_problem(q, &p)) return rc;
+  if (int rc = check_ws(p, ws, ws_bytes)) return rc;
+  if (n_segments < 1 || !seg_off || !x_rows || !w13 || !w2 || !y_rows || n_rows < 1) return MOE_ERR_INVALID_ARG;
+  if (n_segments > 256) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x_rows) || !aligned16(w13) || !aligned16(w2) || !aligned16(y_rows)) return MOE_ERR_INVALID_ARG;
+  if (n_rows > p.max_rows) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(p);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  unsigned* status = at<unsigned>(ws, L.status);
+  if (n_segments <= p.E) {  // at most one segment per expert: run them as they lie
+    const int rc = launch_expert_ffn(p, MOE_FFN_ROUTED, x_rows, n_rows, seg_off, w13, w2, at<void>(ws, L.h_routed),
+                                     y_rows, status, st, nullptr, nullptr, nullptr, nullptr, nullptr, n_segments);
+    return rc ? MOE_ERR_CUDA : MOE_OK;
+  }
+  // Several segments per expert (a few dozen rows each in the expert-parallel
+  // receive buffer): each would end in a part tile that streams the expert's
+  // weights again.  So the rows go into expert-major order in the workspace
+  // (one group per expert, full tiles), and the outputs back to segment order.
+  int32_t* dst_off = at<int32_t>(ws, L.seg_map);
+  int32_t* expert_off = dst_off + kMaxSegments;
+  const int row_bytes = static_cast<int>(p.d * p.esize());
+  if (cudaError_t e = launch_segment_regroup_plan(seg_off, n_segments, p.E, dst_off, expert_off, st)) return cuda_rc(e);
+  if (cudaError_t e = launch_segment_copy(x_rows, at<void>(ws, L.x_perm), seg_off, dst_off, n_segments, n_rows,
+                                          row_bytes, true, st))
+    return cuda_rc(e);
+  if (launch_expert_ffn(p, MOE_FFN_ROUTED, at<void>(ws, L.x_perm), n_rows, expert_off, w13, w2,
+                        at<void>(ws, L.h_routed), at<void>(ws, L.y_perm), status, st))
+    return MOE_ERR_CUDA;
+  return cuda_rc(launch_segment_copy(at<void>(ws, L.y_perm), y_rows, seg_off, dst_off, n_segments, n_rows, row_bytes,
+                                     false, st));
 }
 
 int moe_combine(const moe_problem_t* q, const void* y_perm, const int32_t* slot_of, const float* topk_w,

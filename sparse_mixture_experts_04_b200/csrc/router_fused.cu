@@ -73,6 +73,7 @@ struct RouterArgs {
   unsigned* status;
   unsigned long long* clk;  // stage clock, or nullptr
   unsigned long long stall_ns;  // abort-path test hook (test_stall), 0 normally
+  int select;  // 1: rank the tokens here; 0: only write the logits (a selection kernel follows)
 };
 
 // Shared-memory carve-up (bytes from the 1024-aligned base), the same on host
@@ -247,7 +248,28 @@ __global__ void __launch_bounds__(kRtThreads, 2)
   // every CTA's partial is in its shared memory and visible cluster-wide
   cluster_sync();
 
-  {
+  if (!a.select) {
+    // --------------------------------------------- the logits only (warp per row)
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    const float* peer[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) peer[q] = q < C ? cluster.map_shared_rank(part, static_cast<unsigned>(q)) : part;
+    for (int tl = warp; tl < TPC; tl += kRtWarps) {
+      const int64_t t = row0 + static_cast<int64_t>(rank) * TPC + tl;
+      if (t >= a.T) break;
+      const int row = (static_cast<int>(rank) * TPC + tl) * L.part_stride;
+      for (int e = lane; e < a.E; e += 32) {
+        float pv[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) pv[q] = q < C ? peer[q][row + e] : 0.f;
+        float v = pv[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < C) v += pv[q];
+        a.logits[t * a.E + e] = v + s_off[e];
+      }
+    }
+  } else {
     // ------------------------------------------------------------ selection
     // every warp: the TMA and MMA warps are idle from here on
     constexpr int NW = kRtWarps;
@@ -440,15 +462,17 @@ bool router_fused_ok(const Problem& p) {
          p.T <= (static_cast<int64_t>(1) << 31) - kRtBM;
 }
 
-// 64 or 128 experts: a group of 16 lanes per token (two tokens per warp at a
-// time) when the K + 1 ranking rounds fit in it (MOE_B200_ROUTER_GROUP=32:
-// always a whole warp per token).
-static bool rt_group16(const Problem& p) {
-  static const bool warp_only = [] {
-    const char* e = getenv("MOE_B200_ROUTER_GROUP");
-    return e && e[0] == '3';
-  }();
-  return !warp_only && p.K + 1 <= 16;
+// Where the tokens are ranked: in this kernel, unless MOE_B200_ROUTER_SPLIT=1
+// (then it only writes the logits and the selection kernel ranks them, with
+// more warps per SM).  In place on all four BF16 workloads the single launch
+// was the faster (device-stamped spans, same box: 17.4 / 25.8 / 32.4 / 12.1 us
+// against 23.5 / 32.3 / 38.3 / 17.0 us for mixtral / zen_fine / skewed /
+// decode): the second launch and the logits' round trip through L2 cost more
+// than the extra warps save.
+bool router_selects(const Problem& p) {
+  (void)p;
+  const char* e = getenv("MOE_B200_ROUTER_SPLIT");
+  return !(e && e[0] == '1');
 }
 
 int router_fused_zparts(const Problem& p) {
@@ -459,7 +483,8 @@ int router_fused_zparts(const Problem& p) {
 cudaError_t launch_router_fused(const Problem& p, const void* x, const void* w_gate, const float* offset,
                                 const float* sel_bias, float* logits, int32_t* topk_idx, float* topk_w,
                                 int32_t* chunk_counts, unsigned long long* chunk_psum, float* zpart,
-                                unsigned* status, cudaStream_t st, int* n_zpart, unsigned long long* clk) {
+                                unsigned* status, cudaStream_t st, int* n_zpart, unsigned long long* clk,
+                                bool select) {
   const int epad = rt_epad(p.E);
   CUtensorMap tx, tw;
   const uint64_t dx[2] = {static_cast<uint64_t>(p.d), static_cast<uint64_t>(p.T)};
@@ -486,15 +511,13 @@ cudaError_t launch_router_fused(const Problem& p, const void* x, const void* w_g
   a.status = status;
   a.clk = clk;
   a.stall_ns = test_stall_ns();
+  a.select = select ? 1 : 0;
   switch (epad) {
     case 16:  // one expert per lane, a group of 8 or 16 lanes per token
       return p.E <= 8 ? run_router<16, 8>(p, tx, tw, a, st, n_zpart) : run_router<16, 16>(p, tx, tw, a, st, n_zpart);
     case 32: return run_router<32, 32>(p, tx, tw, a, st, n_zpart);
-    case 64:
-      return rt_group16(p) ? run_router<64, 16>(p, tx, tw, a, st, n_zpart) : run_router<64, 32>(p, tx, tw, a, st, n_zpart);
-    case 128:
-      return rt_group16(p) ? run_router<128, 16>(p, tx, tw, a, st, n_zpart)
-                           : run_router<128, 32>(p, tx, tw, a, st, n_zpart);
+    case 64: return run_router<64, 32>(p, tx, tw, a, st, n_zpart);
+    case 128: return run_router<128, 32>(p, tx, tw, a, st, n_zpart);
     default: return run_router<256, 32>(p, tx, tw, a, st, n_zpart);
   }
 }

@@ -13,11 +13,13 @@ of the router and of the shared experts.  One forward on rank q:
      seg_off[e] .. seg_off[e+1];
   2. all-gather of the G segment-offset vectors (E+1 int32 each) and
      moe_ep_plan (host): which rows go where;
-  3. exchange: chunk e of x_perm goes to the owner of expert e; the chunks
-     received land grouped by local expert, sources in rank order;
-  4. moe_expert_ffn (ROUTED) with the local E_l experts on the received rows;
-  5. exchange back: each output chunk returns to its source's y_perm, in the
-     place its input came from;
+  3. exchange: the rows for peer q's experts are one contiguous block of
+     x_perm (seg_off[q E_l] .. seg_off[(q+1) E_l]), sent as one message; the
+     blocks received lie end to end in rank order (source-major);
+  4. moe_expert_ffn_segments with the local E_l experts over the G E_l row
+     segments of that buffer (segment s E_l + el: source s, local expert el);
+  5. exchange back: each source's block of outputs returns as one message to
+     its y_perm, in the place its input came from;
   6. shared experts (local; `forward` runs them while the rows of step 3 are
      in flight) and moe_combine, as on one device.
 
@@ -86,6 +88,10 @@ class CudaExperts:
         self.x_loc = torch.empty((self.max_local_rows, d), dtype=self.dtype, device=dev)
         self.y_loc = torch.empty((self.max_local_rows, d), dtype=self.dtype, device=dev)
         self.stats = torch.empty(api.stats_size(prob), dtype=torch.float32, device=dev)
+        # segment offsets of the receive buffer: host plan -> pinned staging -> device, without a host wait
+        self.seg_host = torch.empty(n_ranks * self.n_local + 1, dtype=torch.int32,
+                                    pin_memory=self.device.type == "cuda")
+        self.seg_dev = torch.empty(n_ranks * self.n_local + 1, **i32)
         self.y_shared = torch.empty((T, d), dtype=self.dtype, device=dev) if prob.n_shared > 0 else None
 
     def route_dispatch(self, x: torch.Tensor) -> torch.Tensor:
@@ -101,10 +107,16 @@ class CudaExperts:
         return self.seg_off
 
     def experts(self, n_rows: int, local_seg_off: torch.Tensor) -> None:
+        """The local experts over the receive buffer's G E_l source-major
+        segments (segment i: local expert i % E_l).  The offsets reach the
+        device by an asynchronous copy from pinned memory; the next plan is
+        made only after the next step's all-gather has been read on the host,
+        which orders it after this copy."""
         if n_rows > 0:
-            seg = local_seg_off.to(self.device, non_blocking=False)
-            api.moe_expert_ffn(self.prob_local, api.FFN_ROUTED, self.x_loc, n_rows, seg, self.weights["w13"],
-                               self.weights["w2"], self.y_loc, self.ws_local)
+            self.seg_host.copy_(local_seg_off)
+            self.seg_dev.copy_(self.seg_host, non_blocking=True)
+            api.moe_expert_ffn_segments(self.prob_local, self.x_loc, n_rows, self.seg_dev, self.seg_dev.numel() - 1,
+                                        self.weights["w13"], self.weights["w2"], self.y_loc, self.ws_local)
 
     def shared(self, x: torch.Tensor) -> None:
         """The shared experts on this rank's batch (no routed rows needed)."""

@@ -39,48 +39,55 @@ def _random_seg_off(rng, G, E, T, K):
 
 @pytest.mark.parametrize("G,E", [(1, 4), (2, 4), (2, 8), (4, 8), (8, 8), (3, 6)])
 def test_plan_tables_match_their_definition(G, E):
+    """One chunk per peer each way: the block of x_perm holding peer q's
+    experts goes to q; the blocks received lie end to end in source order, and
+    segment s*E_l + el covers source s's rows for local expert el."""
     rng = np.random.default_rng(G * 100 + E)
     so = _random_seg_off(rng, G, E, T=20, K=2)
     El = E // G
     for rank in range(G):
         send, recv, local = (t.numpy() for t in api.moe_ep_plan(G, rank, E, torch.from_numpy(so)))
-        for e in range(E):
-            assert tuple(send[e]) == (e // El, so[rank, e], so[rank, e + 1] - so[rank, e])
+        assert send.shape == (G, 3) and recv.shape == (G, 3) and local.shape == (G * El + 1,)
+        for q in range(G):
+            assert tuple(send[q]) == (q, so[rank, q * El], so[rank, (q + 1) * El] - so[rank, q * El])
         off = 0
-        for el in range(El):
-            assert local[el] == off
-            for s in range(G):
-                rows = so[s, rank * El + el + 1] - so[s, rank * El + el]
-                assert tuple(recv[el * G + s]) == (s, off, rows)
-                off += rows
-        assert local[El] == off
+        for s in range(G):
+            rows = so[s, (rank + 1) * El] - so[s, rank * El]
+            assert tuple(recv[s]) == (s, off, rows)
+            for el in range(El):
+                assert local[s * El + el] == off + so[s, rank * El + el] - so[s, rank * El]
+            off += rows
+        assert local[G * El] == off
+        assert (np.diff(local) >= 0).all()
 
 
 @pytest.mark.parametrize("G,E", [(2, 4), (4, 8), (3, 6), (8, 8)])
 def test_plan_moves_every_kept_row_to_its_expert_and_back(G, E):
     """Simulate the exchange with labelled rows: each row of rank s's x_perm is
-    (s, slot).  After the forward exchange, rank q's local buffer holds, for
-    each local expert in order, exactly the rows the ranks kept for it; after
-    the return exchange every y_perm slot holds its own label again."""
+    (s, slot).  After the forward exchange, segment s*E_l + el of rank q's
+    local buffer holds exactly the rows rank s kept for q's local expert el;
+    after the return exchange every y_perm slot holds its own label again."""
     rng = np.random.default_rng(7 * G + E)
     so = _random_seg_off(rng, G, E, T=16, K=2)
     El = E // G
     plans = [tuple(t.numpy() for t in api.moe_ep_plan(G, r, E, torch.from_numpy(so))) for r in range(G)]
     x_perm = [np.array([(s, i) for i in range(so[s, E])], dtype=np.int64).reshape(-1, 2) for s in range(G)]
-    x_loc = [np.full((plans[q][2][El], 2), -1, np.int64) for q in range(G)]
-    for s in range(G):          # forward: sender s's chunks to q, in order, meet q's receive slots from s, in order
+    x_loc = [np.full((plans[q][2][-1], 2), -1, np.int64) for q in range(G)]
+    for s in range(G):          # forward: one message s -> q
         for q in range(G):
             out = [(o, n) for p, o, n in plans[s][0] if p == q and n > 0]
             inn = [(o, n) for p, o, n in plans[q][1] if p == s and n > 0]
-            assert [n for _, n in out] == [n for _, n in inn]
+            assert [n for _, n in out] == [n for _, n in inn] and len(out) <= 1
             for (o1, n), (o2, _) in zip(out, inn):
                 x_loc[q][o2:o2 + n] = x_perm[s][o1:o1 + n]
     for q in range(G):
         local = plans[q][2]
-        for el in range(El):
-            e = q * El + el
-            want = [(s, i) for s in range(G) for i in range(so[s, e], so[s, e + 1])]
-            assert [tuple(r) for r in x_loc[q][local[el]:local[el + 1]]] == want
+        for s in range(G):
+            for el in range(El):
+                e = q * El + el
+                want = [(s, i) for i in range(so[s, e], so[s, e + 1])]
+                seg = s * El + el
+                assert [tuple(r) for r in x_loc[q][local[seg]:local[seg + 1]]] == want
     y_perm = [np.full((so[s, E], 2), -1, np.int64) for s in range(G)]
     for q in range(G):          # back: the expert outputs (here: the labels) return to their sources
         for s in range(G):
@@ -138,8 +145,9 @@ class OracleExperts:
 
     def experts(self, n_rows, local_seg_off):
         lso = local_seg_off.tolist()
-        for el in range(self.n_local):
-            for r in range(lso[el], lso[el + 1]):
+        for seg in range(len(lso) - 1):      # segment i: local expert i % E_l
+            el = seg % self.n_local
+            for r in range(lso[seg], lso[seg + 1]):
                 self.y_loc[r] = torch.from_numpy(oracle.swiglu(self.x_loc[r].numpy(), self.w13[el], self.w2[el]))
 
     def shared(self, x):

@@ -105,3 +105,43 @@ def test_one_rank_nccl_group_matches_single_device():
     assert rel_err(got, want) <= tol(cfg)
     # one rank: the local rows are x_perm itself, in the same order and tiles
     assert torch.equal(y, y_one)
+
+
+@pytest.mark.parametrize("tile", ["256all", "128"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_expert_ffn_segments_repeat_the_experts(dtype, tile, monkeypatch):
+    """moe_expert_ffn_segments: segment i of the rows uses expert i % E (the
+    expert-parallel receive buffer: one block per source, experts in order
+    inside it), checked row by row against the oracle, empty segments and
+    segments of several hundred rows included."""
+    import oracle
+    from helpers import host_np
+    if tile:
+        monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
+    E, S, d, F = 4, 12, 256, 192
+    rng = np.random.default_rng(31)
+    rows = rng.integers(0, 120, size=S)
+    rows[[2, 7]] = 0
+    rows[5] = 300
+    seg = np.concatenate([[0], np.cumsum(rows)]).astype(np.int32)
+    n = int(seg[-1])
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    x = torch.from_numpy(rng.normal(size=(n, d)).astype(np.float32)).to(tdt)
+    w13 = torch.from_numpy((rng.normal(size=(E, 2 * F, d)) / np.sqrt(d)).astype(np.float32)).to(tdt)
+    w2 = torch.from_numpy((rng.normal(size=(E, d, F)) / np.sqrt(F)).astype(np.float32)).to(tdt)
+    prob = api.make_problem(n, d, E, 1, F, 0, 0.0, dtype)
+    ws = api.alloc_workspace(prob)
+    y = torch.zeros((n, d), dtype=tdt, device="cuda")
+    api.reset_device_status(ws)
+    api.moe_expert_ffn_segments(prob, dev(x), n, dev(seg), S, dev(w13), dev(w2), y, ws)
+    assert api.read_device_status(ws) == 0
+    xs, a, b = host_np(x), host_np(w13), host_np(w2)
+    if dtype == "bf16":
+        x64 = (xs.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    else:
+        x64 = xs.astype(np.float64)
+    e_of = np.repeat(np.arange(S) % E, rows)
+    pick = np.unique(np.concatenate([seg[:-1][rows > 0], seg[1:][rows > 0] - 1, rng.choice(n, 48, replace=False)]))
+    want = np.stack([oracle.swiglu(x64[r], a[e_of[r]], b[e_of[r]]) for r in pick])
+    got = y.float().cpu().numpy()[pick]
+    assert rel_err(got, want) <= (2e-2 if dtype == "bf16" else 1e-4)
