@@ -263,6 +263,21 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int b = blockIdx.x;
+  // Every global load that does not depend on another is issued here, before
+  // the first barrier, so that their latencies overlap (the kernel is a chain
+  // of dependent steps, not bandwidth): this thread's token's experts, its
+  // share of the chunk histogram and, in block 0, the chunk p sums.
+  const int64_t t = static_cast<int64_t>(b) * kDispatchChunk + tid;
+  const bool tok_ok = t < T;
+  constexpr int kKReg = 8;  // the first experts of the token stay in registers
+  int my_e[kKReg];
+#pragma unroll
+  for (int k = 0; k < kKReg; ++k) my_e[k] = (tok_ok && k < K) ? idx[t * K + k] : -1;
+  unsigned long long ps_mine = 0;  // block 0: sum of expert tid's chunk p sums
+  if (b == 0 && stats && tid < E) {
+#pragma unroll 8
+    for (int c = 0; c < n_chunks; ++c) ps_mine += chunk_psum[static_cast<int64_t>(c) * E + tid];
+  }
   // 1. per expert: total over all chunks and the count in chunks before b.
   //    Thread (e, sl) sums a strided set of chunks; E <= 256 experts, S slices.
   int S = 256 / E;
@@ -272,7 +287,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
     const int e = tid % E, sl = tid / E;
     int tot = 0, pre = 0;
     if (tid < E * S) {
-#pragma unroll 4
+#pragma unroll 16
       for (int c = sl; c < n_chunks; c += S) {
         const int v = chunk_counts[static_cast<int64_t>(c) * E + e];
         tot += v;
@@ -323,10 +338,13 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
     if (lane == 31) s_seg[E] = incl;
   }
   // 3. this chunk's lane masks
-  const int64_t t = static_cast<int64_t>(b) * kDispatchChunk + warp * 32 + lane;
-  const bool tok_ok = t < T;
   if (tok_ok) {
-    for (int k = 0; k < K; ++k) {
+#pragma unroll
+    for (int k = 0; k < kKReg; ++k) {
+      const int e = my_e[k];
+      if (k < K && static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicOr(&mask[warp][e], 1u << lane);
+    }
+    for (int k = kKReg; k < K; ++k) {
       const int e = idx[t * K + k];
       if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) atomicOr(&mask[warp][e], 1u << lane);
     }
@@ -351,9 +369,8 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
   // 4. ranks and slots
   if (tok_ok) {
     const uint32_t lower = (1u << lane) - 1u;
-    for (int k = 0; k < K; ++k) {
+    auto rank_pair = [&](int k, int e) {
       const int64_t pair = t * K + k;
-      const int e = idx[pair];
       int slot = -1;
       if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) {
         const int rank = wbase[warp][e] + __popc(mask[warp][e] & lower);
@@ -363,15 +380,15 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
         }
       }
       slot_of[pair] = slot;
-    }
+    };
+#pragma unroll
+    for (int k = 0; k < kKReg; ++k)
+      if (k < K) rank_pair(k, my_e[k]);
+    for (int k = kKReg; k < K; ++k) rank_pair(k, idx[t * K + k]);
   }
   // 5. block 0: the balance statistics (f, P, loss; z-loss and utilisation with zpart)
   if (b == 0 && stats) {
-    for (int e = tid; e < E; e += blockDim.x) {
-      unsigned long long ps = 0;
-      for (int c = 0; c < n_chunks; ++c) ps += chunk_psum[static_cast<int64_t>(c) * E + e];
-      s_fp[e] = balance_stats_expert(s_tot[e], ps, T, E, K, e, stats);
-    }
+    for (int e = tid; e < E; e += blockDim.x) s_fp[e] = balance_stats_expert(s_tot[e], ps_mine, T, E, K, e, stats);
     double z = 0.0;
     if (zpart)
       for (int i = tid; i < n_zpart; i += blockDim.x) z += zpart[i];
