@@ -72,9 +72,6 @@ struct GemmArgs {
   // pair kernel: a group's last row tile with at most swap_max rows (0: never)
   // is computed operand-swapped (see grouped_gemm_pair_kernel)
   int swap_max;
-  // pair kernel: a group whose rows exceed a multiple of 256 by 1..fold_max
-  // computes those rows inside its last full tile (0: never)
-  int fold_max;
   // EPI_SWIGLU: when not null, the gate and up projections are also stored
   // (BF16): row r, group g: g at gu + r*ld_gu + g*gu_col_stride + col, u at
   // N columns further
@@ -133,7 +130,6 @@ struct TileInfo {
   int g, row0, row_end, n0;
   int w;        // expert whose weights the tile uses (g, or g % weight_mod)
   bool swap;    // operand-swapped remainder tile (pair kernel only)
-  int fold;     // pair kernel: rows past this full tile computed inside it (0: none)
   bool second;  // tile of the pair kernel's second problem
 };
 
@@ -156,19 +152,6 @@ __device__ __forceinline__ int group_rows(const GemmArgs& a, int g, int* base) {
   return rows;
 }
 
-// Row tiles of a group with `rows` rows.  *fold: the rows past the last full
-// tile that it computes as well (1..fold_max, pair kernel), else 0.
-template <int BM>
-__device__ __forceinline__ int row_tiles(const GemmArgs& a, int rows, int* fold) {
-  const int full = rows / BM, rem = rows - full * BM;
-  if (full > 0 && rem > 0 && rem <= a.fold_max) {
-    *fold = rem;
-    return full;
-  }
-  *fold = 0;
-  return (rows + BM - 1) / BM;
-}
-
 template <int BM>
 __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, const GemmArgs& a, int out_cols) {
   int lo = 0, hi = a.n_groups - 1;
@@ -181,16 +164,14 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
   ti.w = a.weight_mod > 0 ? lo % a.weight_mod : lo;
   int base;
   const int rows = group_rows(a, lo, &base);
-  int fold;
-  const int mt = row_tiles<BM>(a, rows, &fold);
+  const int mt = (rows + BM - 1) / BM;
   const int local = tile - prefix[lo];
   const int n_idx = local / mt;
   const int m_idx = local - n_idx * mt;
   ti.row0 = base + m_idx * BM;
   ti.row_end = base + rows;
   ti.n0 = n_idx * out_cols;
-  ti.fold = m_idx == mt - 1 ? fold : 0;
-  ti.swap = ti.fold == 0 && m_idx == mt - 1 && rows - m_idx * BM <= a.swap_max;
+  ti.swap = m_idx == mt - 1 && rows - m_idx * BM <= a.swap_max;
   ti.second = false;
   return ti;
 }
@@ -204,8 +185,8 @@ __device__ __forceinline__ void tile_prefix_warp(const GemmArgs& args, int n_til
   for (int i = 0; i < per; ++i) {
     const int g = lane * per + i;
     if (g < args.n_groups) {
-      int base, fold;
-      local += row_tiles<BM>(args, group_rows(args, g, &base), &fold) * n_tiles_n;
+      int base;
+      local += ((group_rows(args, g, &base) + BM - 1) / BM) * n_tiles_n;
     }
   }
   int incl = local;
@@ -219,8 +200,8 @@ __device__ __forceinline__ void tile_prefix_warp(const GemmArgs& args, int n_til
     const int g = lane * per + i;
     if (g < args.n_groups) {
       prefix[g] = run;
-      int base, fold;
-      run += row_tiles<BM>(args, group_rows(args, g, &base), &fold) * n_tiles_n;
+      int base;
+      run += ((group_rows(args, g, &base) + BM - 1) / BM) * n_tiles_n;
     }
   }
   if (lane == 31) prefix[args.n_groups] = incl;
@@ -245,21 +226,17 @@ __device__ __forceinline__ TileInfo decode_mixed_tile(int tile, int t1, int tota
 // Drain one accumulator (this warp's 32 TMEM lanes, BN columns starting at
 // t_row) and store the thread's row.  Every lane must call it (the TMEM loads
 // are warp-collective); row_ok masks only the stores.
-// SwiGLU: gate features n0 + c in columns c, up features in c + BN/2; with
-// il64 (BN = 256, weights staged 64 gate + 64 up rows per CTA of a pair) the
-// columns hold [gate 0..63 | up 0..63 | gate 64..127 | up 64..127].
 template <int EPI, int BN>
 __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int row, bool row_ok, int n0,
-                                              uint32_t t_row, bool il64 = false) {
+                                              uint32_t t_row) {
   if (EPI == EPI_SWIGLU) {
     __nv_bfloat16* out_row = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * args.ldo +
                              static_cast<int64_t>(g) * args.out_col_stride;
 #pragma unroll 1
     for (int c = 0; c < BN / 2; c += 32) {
       uint32_t gr[32], ur[32];
-      const int gc = il64 ? (c & 32) + (c >= 64 ? 128 : 0) : c;
-      tmem_load_32x32(t_row + gc, gr);
-      tmem_load_32x32(t_row + (il64 ? gc + 64 : BN / 2 + c), ur);
+      tmem_load_32x32(t_row + c, gr);
+      tmem_load_32x32(t_row + BN / 2 + c, ur);
       tmem_load_wait();
       if (row_ok) {
 #pragma unroll
@@ -571,12 +548,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //   empty[s]  (each)    one arrive from the leader's multicast commit
 //   tfull[a]  (each)    one arrive from the leader's multicast commit
 //   tempty[a] (leader)  8 arrives: 4 epilogue warps in each CTA
-// Tiles are 256 rows; a group with r rows spans ceil(r/256) row tiles, or
-// floor(r/256) when its last full tile folds in the rest (fold tiles, below).
-// Stage s occupies [s * 64 KB, (s + 1) * 64 KB): the token / A rows first,
-// then the weights (32 KB each; a deep swap stage: tokens, then 48 KB of
-// weights); a fold tile's remainder tokens for stage s sit in a ring of their
-// own after the stages.
+// Tiles are 256 rows; a group with r rows spans ceil(r/256) row tiles.  Stage
+// s occupies [s * 64 KB, (s + 1) * 64 KB): the token / A rows first, then the
+// weights (32 KB each; a deep swap stage: tokens, then 48 KB of weights).
 // ============================================================================
 constexpr int kPairBM = 256;
 constexpr int kPairBN = 256;  // MMA N: both halves of B
@@ -596,30 +570,16 @@ constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
 constexpr int kDeepKC = 3;
 constexpr int kDeepWOffset = kPairStageBytes - kDeepKC * kPairChunk;
 static_assert(kDeepKC * 32 * kBK * 2 <= kDeepWOffset, "deep swap tokens overlap the weights");
-// Fold tiles: a group of 256 h + r rows with 1 <= r <= kFoldMax computes its
-// last r rows inside its last full tile.  Per stage the tile's MMAs use the
-// staged weights twice: as B against the 256 full-tile token rows, and as A
-// (M = 256) against the r remainder tokens (N = r rounded up to 16, half per
-// CTA), so the weights cross into shared memory once instead of once more for
-// a swap tile of r rows, which costs nearly a full tile's copies.  The
-// remainder accumulator borrows the first N columns of the other TMEM slot.
-// Its tokens come in boxes of kFoldBox rows (N/2 <= 24 per CTA).
-constexpr int kFoldMax = 48;
-constexpr int kFoldBox = 24;
-constexpr int kFoldChunk = kFoldBox * kBK * 2;  // 3 KB, a whole number of 1 KB swizzle atoms
-constexpr int kFoldStageBytes = kPairKC * kFoldChunk;
-static_assert(kFoldChunk % 1024 == 0, "fold chunks must keep the 128-byte swizzle atoms aligned");
 
 // 64-deep chunks per stage of a tile whose token box is a_box rows
 __device__ __forceinline__ int pair_tile_kc(const GemmArgs& a, const TileInfo& ti, int a_box) {
   return (a.deep_swap && a.merged_k && ti.swap && a_box <= 32) ? kDeepKC : kPairKC;
 }
 
-// Swap-tile epilogues transpose through shared memory, 16 tokens at a time:
+// Swap-tile epilogues transpose through shared memory, 32 tokens at a time:
 // xbuf[token][TMEM lane] (row stride 132 floats keeps 16-byte alignment).
-constexpr int kSwapXTokens = 16;
 constexpr int kSwapXStride = 132;
-constexpr int kSwapXBytes = kSwapXTokens * kSwapXStride * 4;
+constexpr int kSwapXBytes = 32 * kSwapXStride * 4;
 // A swap tile loads its tokens with the smallest box (16, 32, 64 or 128
 // rows) that holds its N/2 tokens per CTA.
 __device__ __forceinline__ int swap_box_rows(int half_n) {
@@ -627,9 +587,8 @@ __device__ __forceinline__ int swap_box_rows(int half_n) {
 }
 
 constexpr int pair_smem_bytes() {
-  return kPairStages * (kPairStageBytes + kFoldStageBytes) + 256 + 8 * (kMaxGroups + 1) + kSwapXBytes + 1024;
+  return kPairStages * kPairStageBytes + 256 + 8 * (kMaxGroups + 1) + kSwapXBytes + 1024;
 }
-static_assert(pair_smem_bytes() <= 227 * 1024, "pair kernel shared memory above the per-CTA limit");
 
 __device__ __forceinline__ TileInfo decode_pair_tile(int tile, int t1, int total, const int* prefix,
                                                      const int* prefix2, const GemmArgs& a1, const GemmArgs& a2,
@@ -647,8 +606,8 @@ __device__ __forceinline__ int swap_n(int rows) { return (rows + 15) & ~15; }
 
 // Epilogue of a swap tile (all four epilogue warps, uniform control flow):
 // TMEM lane = weight row of this CTA, column = token of the tile.  Each
-// 32-token chunk of columns goes through xbuf 16 tokens at a time so that
-// every thread then stores 8 consecutive outputs of one token (16 bytes).
+// 32-token chunk goes through xbuf so that every thread then stores 8
+// consecutive outputs of one token (16 bytes).
 //   SwiGLU: lanes 0..63 hold gate features n0 + 64*rank + (0..63), lanes
 //   64..127 the same up features: h = silu(g) * u.
 //   BF16: lane = output column n0 + 128*rank + lane.
@@ -666,18 +625,16 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileIn
     tmem_load_32x32(t_lane + c, v);
     tmem_load_wait();
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int c0 = c + half * kSwapXTokens;  // first token of this pass (n is a multiple of 16)
-      if (c0 >= n) break;
+    for (int j = 0; j < 32; ++j) xbuf[j * kSwapXStride + my_lane] = __uint_as_float(v[j]);
+    named_bar_sync(1, 128);
+    if (EPI == EPI_SWIGLU) {
+      // 64 features = 8 groups of 8: 16 tokens per pass
+      const int fg = et & 7;
+      const int f = ti.n0 + 64 * static_cast<int>(rank) + 8 * fg;
 #pragma unroll
-      for (int j = 0; j < kSwapXTokens; ++j) xbuf[j * kSwapXStride + my_lane] = __uint_as_float(v[half * kSwapXTokens + j]);
-      named_bar_sync(1, 128);
-      if (EPI == EPI_SWIGLU) {
-        // 64 features = 8 groups of 8: the 16 tokens in one pass
-        const int fg = et & 7;
-        const int f = ti.n0 + 64 * static_cast<int>(rank) + 8 * fg;
-        const int j = et >> 3;
-        if (c0 + j < rows && f < args.N) {
+      for (int pass = 0; pass < 2; ++pass) {
+        const int j = pass * 16 + (et >> 3);
+        if (c + j < rows && f < args.N) {
           const float4* gp = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 8 * fg);
           const float4* up = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 64 + 8 * fg);
           const float4 g0 = gp[0], g1 = gp[1], u0 = up[0], u1 = up[1];
@@ -690,11 +647,11 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileIn
             const float h1 = __fdividef(g[2 * q + 1], 1.0f + __expf(-g[2 * q + 1])) * u[2 * q + 1];
             pk[q] = pack_bf16x2(h0, h1);
           }
-          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c0 + j) * args.ldo + f) =
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c + j) * args.ldo + f) =
               make_uint4(pk[0], pk[1], pk[2], pk[3]);
           if (args.gu) {
             __nv_bfloat16* gu_row = static_cast<__nv_bfloat16*>(args.gu) +
-                                    static_cast<int64_t>(ti.row0 + c0 + j) * args.ld_gu +
+                                    static_cast<int64_t>(ti.row0 + c + j) * args.ld_gu +
                                     static_cast<int64_t>(ti.g) * args.gu_col_stride;
             *reinterpret_cast<uint4*>(gu_row + f) =
                 make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]), pack_bf16x2(g[4], g[5]),
@@ -704,24 +661,23 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileIn
                            pack_bf16x2(u[6], u[7]));
           }
         }
-      } else {
-        // 128 columns = 16 groups of 8: 8 tokens per pass, two passes
-        const int fg = et & 15;
-        const int col = ti.n0 + 128 * static_cast<int>(rank) + 8 * fg;
+      }
+    } else {
+      // 128 columns = 16 groups of 8: 8 tokens per pass
+      const int fg = et & 15;
+      const int col = ti.n0 + 128 * static_cast<int>(rank) + 8 * fg;
 #pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-          const int j = pass * 8 + (et >> 4);
-          if (c0 + j < rows && col < args.N) {
-            const float4* vp = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 8 * fg);
-            const float4 a = vp[0], b = vp[1];
-            *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c0 + j) * args.ldo + col) =
-                make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
-                           pack_bf16x2(b.z, b.w));
-          }
+      for (int pass = 0; pass < 4; ++pass) {
+        const int j = pass * 8 + (et >> 4);
+        if (c + j < rows && col < args.N) {
+          const float4* vp = reinterpret_cast<const float4*>(xbuf + j * kSwapXStride + 8 * fg);
+          const float4 a = vp[0], b = vp[1];
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c + j) * args.ldo + col) =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
         }
       }
-      named_bar_sync(1, 128);
     }
+    named_bar_sync(1, 128);
   }
 }
 
@@ -737,15 +693,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                              const __grid_constant__ GemmArgs args2,
                              const __grid_constant__ CUtensorMap tmA32d, const __grid_constant__ CUtensorMap tmA16d,
                              const __grid_constant__ CUtensorMap tmB64d, const __grid_constant__ CUtensorMap tmA32d_2,
-                             const __grid_constant__ CUtensorMap tmA16d_2, const __grid_constant__ CUtensorMap tmB64d_2,
-                             const __grid_constant__ CUtensorMap tmAf, const __grid_constant__ CUtensorMap tmAf_2) {
+                             const __grid_constant__ CUtensorMap tmA16d_2, const __grid_constant__ CUtensorMap tmB64d_2) {
   constexpr int kOutCols = (EPI == EPI_SWIGLU) ? kPairBN / 2 : kPairBN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // stage s: smem + s * kPairStageBytes (tokens / A rows first, then weights);
-  // its fold tokens at fold_ring + s * kFoldStageBytes
-  uint8_t* fold_ring = smem + kPairStages * kPairStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(fold_ring + kPairStages * kFoldStageBytes);
+  // stage s: smem + s * kPairStageBytes (tokens / A rows first, then weights)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kPairStages * kPairStageBytes);
   uint64_t* empty = full + kPairStages;
   uint64_t* tfull = empty + kPairStages;
   uint64_t* tempty = tfull + 2;
@@ -792,8 +745,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       prefetch_tensormap(&tmA16_2);
       prefetch_tensormap(&tmB64_2);
     }
-    if (args.fold_max > 0) prefetch_tensormap(&tmAf);
-    if (args2.n_groups > 0 && args2.fold_max > 0) prefetch_tensormap(&tmAf_2);
     if (args.deep_swap) {
       prefetch_tensormap(&tmA32d);
       prefetch_tensormap(&tmA16d);
@@ -846,10 +797,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int a_box = ti.swap ? swap_box_rows(half_n) : 128;
         const int kc = pair_tile_kc(A, ti, a_box);
         const bool deep = kc == kDeepKC;
-        // fold tile: this CTA's half of the remainder tokens, and (SwiGLU) the
-        // weights in the swap tiles' layout, which both MMAs can use
-        const int fold_row = ti.row_end - ti.fold + static_cast<int>(rank) * (swap_n(ti.fold) / 2);
-        const bool swap_w = ti.swap || (EPI == EPI_SWIGLU && ti.fold > 0);
         const int nkb_g = (A.K + kBK * kc - 1) / (kBK * kc);
         const int nkb = nkb_g * A.k_groups;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -864,9 +811,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                      : a_box == 32 ? (deep ? (ti.second ? &tmA32d_2 : &tmA32d) : (ti.second ? &tmA32_2 : &tmA32))
                                      : a_box == 64 ? (ti.second ? &tmA64_2 : &tmA64)
                                                    : mA;
-          if (rank == 0)
-            mbar_arrive_expect_tx(&full[stage],
-                                  2 * kc * (kPairChunk + a_box * kBK * 2 + (ti.fold > 0 ? kFoldChunk : 0)));
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kc * (kPairChunk + a_box * kBK * 2));
           const int a_row = ti.row0 + static_cast<int>(rank) * half_n;
           uint8_t* a_dst = smem + stage * kPairStageBytes;
           uint8_t* b_dst = a_dst + (deep ? kDeepWOffset : kPairABytes);
@@ -884,14 +829,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               tma_load_2d_pair(a_dst + c * a_box * kBK * 2, a_box == 128 ? mA : a_map, bar, kg * A.K + kk0 + c * kBK,
                                a_row);
           }
-          if (ti.fold > 0) {
-            uint8_t* f_dst = fold_ring + stage * kFoldStageBytes;
-#pragma unroll
-            for (int c = 0; c < kPairKC; ++c)
-              tma_load_2d_pair(f_dst + c * kFoldChunk, ti.second ? &tmAf_2 : &tmAf, bar, kg * A.K + kk0 + c * kBK,
-                               fold_row);
-          }
-          if (A.merged_k && swap_w) {
+          if (merge) {
             const CUtensorMap* wmap = deep ? (ti.second ? &tmB64d_2 : &tmB64d) : mB64;
             if (EPI == EPI_SWIGLU)  // weights are the M operand: this CTA's 64 gate rows, then the same 64 up rows
               tma_load_4d_pair(b_dst, wmap, bar, 0, ti.n0 + 64 * static_cast<int>(rank), 2 * ti.w, kk0 / kBK);
@@ -903,7 +841,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < kPairKC; ++c) {
               const int kk = kk0 + c * kBK;
               uint8_t* bc = b_dst + c * kPairChunk;
-              if (EPI == EPI_SWIGLU && swap_w) {
+              if (EPI == EPI_SWIGLU && ti.swap) {
                 const int f = ti.n0 + 64 * static_cast<int>(rank);
                 tma_load_3d_pair(bc, mB64, bar, kk, f, 2 * ti.w);
                 tma_load_3d_pair(bc + kPairChunk / 2, mB64, bar, kk, f, 2 * ti.w + 1);
@@ -941,9 +879,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      // uses of each TMEM slot so far: a tile's own slot (it & 1), and the
-      // other one too when a fold tile borrows it for its remainder
-      uint32_t uses0 = 0u, uses1 = 0u;
       for (int tile = pair; ok && tile < total_tiles; tile += n_pairs, ++it) {
         const TileInfo ti = decode_pair_tile(tile, tiles1, total_tiles, prefix, prefix2, args, args2, kOutCols);
         const int a_box = ti.swap ? swap_box_rows(swap_n(ti.row_end - ti.row0) / 2) : 128;
@@ -956,25 +891,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // the token operand's chunks sit a_box rows apart (see the producer)
         const int a_chunk = a_box * kBK * 2;
         const int acc = it & 1;
-        uint32_t& use_own = acc ? uses1 : uses0;
-        uint32_t& use_other = acc ? uses0 : uses1;
-        if (!mbar_wait(&tempty[acc], (use_own & 1u) ^ 1u, abort_flag)) {
+        const uint32_t acc_par = static_cast<uint32_t>(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
-        ++use_own;
-        if (ti.fold > 0) {
-          if (!mbar_wait(&tempty[acc ^ 1], (use_other & 1u) ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          ++use_other;
-        }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kPairBN);
-        // fold tile: A = the staged weight rows (M = 256), B = the remainder tokens
-        const uint32_t d_fold = tmem_base + static_cast<uint32_t>((acc ^ 1) * kPairBN);
-        const uint32_t idesc_fold = idesc_bf16_f32(kPairBM, swap_n(ti.fold > 0 ? ti.fold : 16));
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) {
             ok = false;
@@ -992,12 +915,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k)
               umma_bf16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | c | k) != 0 ? 1u : 0u);
-            if (ti.fold > 0) {
-              const uint64_t fdesc = smem_desc_k128(smem_addr(fold_ring + stage * kFoldStageBytes + c * kFoldChunk));
-#pragma unroll
-              for (int k = 0; k < kBK / 16; ++k)
-                umma_bf16_pair(d_fold, wdesc + 2 * k, fdesc + 2 * k, idesc_fold, (kb | c | k) != 0 ? 1u : 0u);
-            }
           }
           umma_commit_pair_multicast(&empty[stage], 0x3);
           if (++stage == kPairStages) {
@@ -1034,18 +951,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kPairBN);
       if (ti.swap) {
         epilogue_swap<EPI>(A, ti, rank, quarter, lane, (warp - 2) * 32 + lane, t_row, xbuf);
-      } else if (ti.fold > 0) {
-        // the remainder first, from the borrowed slot, which is then released
-        TileInfo tr = ti;
-        tr.row0 = ti.row_end - ti.fold;
-        const uint32_t t_fold = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                static_cast<uint32_t>((acc ^ 1) * kPairBN);
-        epilogue_swap<EPI>(A, tr, rank, quarter, lane, (warp - 2) * 32 + lane, t_fold, xbuf);
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tempty_leader + static_cast<uint32_t>((acc ^ 1) * 8));
-        const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
-        epilogue_rows<EPI, kPairBN>(A, ti.g, row, true, ti.n0, t_row, EPI == EPI_SWIGLU);
       } else {
         const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
         epilogue_rows<EPI, kPairBN>(A, ti.g, row, row < ti.row_end, ti.n0, t_row);
@@ -1127,17 +1032,15 @@ bool make_map_strided(CUtensorMap* m, const void* base, int rank, const uint64_t
 }
 
 // Token maps of the pair kernel: a 2-D (cols, rows) map with 128-row boxes,
-// a 2-D map with the fold tiles' kFoldBox-row boxes, and swap-tile maps with
-// 64-, 32- and 16-row boxes: 2-D as well, or with merged chunks one box
-// spanning both 64-deep chunks of a stage, (64, rows, cols/64) with the chunk
-// stride 128 bytes.
-static bool make_token_maps(CUtensorMap* t128, CUtensorMap* tf, CUtensorMap* t64, CUtensorMap* t32,
-                            CUtensorMap* t16, CUtensorMap* t32d, CUtensorMap* t16d, const void* base, int64_t cols,
-                            int64_t rows, bool merged) {
+// and swap-tile maps with 64-, 32- and 16-row boxes: 2-D as well, or with
+// merged chunks one box spanning both 64-deep chunks of a stage,
+// (64, rows, cols/64) with the chunk stride 128 bytes.
+static bool make_token_maps(CUtensorMap* t128, CUtensorMap* t64, CUtensorMap* t32, CUtensorMap* t16,
+                            CUtensorMap* t32d, CUtensorMap* t16d, const void* base, int64_t cols, int64_t rows,
+                            bool merged) {
   const uint64_t d2[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
   const uint32_t b128[2] = {kBK, 128};
-  const uint32_t bf[2] = {kBK, kFoldBox};
-  if (!make_map(t128, base, 2, d2, b128) || !make_map(tf, base, 2, d2, bf)) return false;
+  if (!make_map(t128, base, 2, d2, b128)) return false;
   CUtensorMap* maps[3] = {t64, t32, t16};
   const uint32_t heights[3] = {64, 32, 16};
   for (int i = 0; i < 3; ++i) {
@@ -1232,7 +1135,6 @@ static int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs
 struct PairProblem {
   CUtensorMap ta, tb, ta64, tb64, ta32, ta16;
   CUtensorMap ta32d, ta16d, tb64d;  // deep swap stages (three chunks per box)
-  CUtensorMap taf;                  // fold tiles' remainder tokens
   GemmArgs a;
   int64_t tile_bound;
 };
@@ -1276,9 +1178,7 @@ static int run_pair_gemm(const PairProblem& p1, const PairProblem* p2, cudaStrea
   if (!p2) a2.n_groups = 0;
   return launch_k(grouped_gemm_pair_kernel<EPI>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kGemmThreads), smem,
                   st, p1.ta, p1.tb, p1.ta64, p1.tb64, p1.ta32, p1.ta16, p1.a, q.ta, q.tb, q.ta64, q.tb64, q.ta32,
-                  q.ta16, a2, p1.ta32d, p1.ta16d, p1.tb64d, q.ta32d, q.ta16d, q.tb64d, p1.taf, q.taf) == cudaSuccess
-             ? 0
-             : -3;
+                  q.ta16, a2, p1.ta32d, p1.ta16d, p1.tb64d, q.ta32d, q.ta16d, q.tb64d) == cudaSuccess ? 0 : -3;
 }
 
 static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -1317,20 +1217,6 @@ static int swap_max_rows() {
     return v < 0 ? 0 : v > 255 ? 255 : v;
   }
   return 128;
-}
-
-// Largest remainder (rows past a multiple of 256) that the pair kernel folds
-// into the group's last full tile (see the kernel); off unless
-// MOE_B200_FOLD_MAX (1..48) asks for it.  Measured: no faster than swap tiles
-// (a fold tile's second MMA reads the staged weights from shared memory again,
-// and its borrowed accumulator slot waits for the previous tile's epilogue).
-static int fold_max_rows() {
-  const char* e = getenv("MOE_B200_FOLD_MAX");
-  if (e && *e) {
-    const int v = atoi(e);
-    return v < 0 ? 0 : v > kFoldMax ? kFoldMax : v;
-  }
-  return 0;
 }
 
 static int tile_mode(int64_t expected_rows_per_group) {
@@ -1545,8 +1431,7 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
                             PairProblem* q, int n_seg = 0) {
   const int G = routed ? p.E : p.Ns;
   const bool merged = merged_k_ok(p.d);
-  if (!make_token_maps(&q->ta, &q->taf, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, x_rows, p.d, n_rows,
-                       merged) ||
+  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, x_rows, p.d, n_rows, merged) ||
       !make_weight_map(&q->tb, w13, p.d, p.F, 2 * G, 128, 1, false) ||
       !make_weight_map(&q->tb64, w13, p.d, p.F, 2 * G, 64, merged ? 2 : 1, merged))
     return false;
@@ -1569,7 +1454,6 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
   a.out_col_stride = routed ? 0 : p.F;
   a.status = status;
   a.swap_max = swap_max_rows();
-  a.fold_max = fold_max_rows();
   a.gu = gu;  // kept for the backward (routed [rows, 2F]; shared [rows, N_s 2F])
   a.ld_gu = 2 * static_cast<int64_t>(p.F) * (routed ? 1 : p.Ns);
   a.gu_col_stride = routed ? 0 : 2 * p.F;
@@ -1590,8 +1474,7 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
   const bool merged = merged_k_ok(p.F);
-  if (!make_token_maps(&q->ta, &q->taf, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, h, h_cols, n_rows,
-                       merged) ||
+  if (!make_token_maps(&q->ta, &q->ta64, &q->ta32, &q->ta16, &q->ta32d, &q->ta16d, h, h_cols, n_rows, merged) ||
       !make_weight_map(&q->tb, w2, p.F, p.d, G, 128, 1, false) ||
       !make_weight_map(&q->tb64, w2, p.F, p.d, G, 128, 1, merged))
     return false;
@@ -1614,7 +1497,6 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   a.out_col_stride = 0;
   a.status = status;
   a.swap_max = swap_max_rows();
-  a.fold_max = fold_max_rows();
   a.row_mode = tail ? 1 : 0;
   a.merged_k = merged ? 1 : 0;
   a.deep_swap = merged && deep_swap_on() ? 1 : 0;
@@ -1734,7 +1616,6 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
         GemmArgs a = q.a;
         a.row_mode = 2;  // the rest (under 256 rows per group) on single CTAs
         a.swap_max = 0;
-        a.fold_max = 0;
         a.merged_k = 0;
         if (!make_map(&ta, x_rows, 2, da, ba) || !make_map(&tb, w13, 3, db, bb)) return -3;
         rc = run_gemm<EPI_SWIGLU, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.F, 128), st);
@@ -1767,7 +1648,6 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
         GemmArgs a = q.a;
         a.row_mode = 2;
         a.swap_max = 0;
-        a.fold_max = 0;
         a.merged_k = 0;
         rc = run_gemm<EPI_BF16, 256, 4>(ta, tb, a, 2 * a.n_groups * cdiv(p.d, 256), st);
         if (rc) return rc;

@@ -247,7 +247,7 @@ def test_routed_expert_ffn_matches_oracle(name):
 
 
 # last-tile row counts: every swap-tile MMA width class and token-box height,
-# and groups of 256 h + r rows with r on both sides of the fold limit (48)
+# and groups of 256 h + r rows with small r (16, 17, 32, 33, 48, 49, 1)
 REMAINDER_SIZES = [1, 15, 16, 17, 31, 33, 100, 128, 129, 200, 255, 256, 257, 300, 513, 0, 48,
                    272, 273, 288, 289, 304, 305, 560, 561]
 
@@ -271,18 +271,16 @@ def _remainder_ffn(F, sizes=REMAINDER_SIZES):
 
 
 @pytest.mark.parametrize("F", [200, 320])
-@pytest.mark.parametrize("tile,swap,fold", [("256all", "", ""), ("256all", "", "48"), ("256all", "0", ""),
-                                            ("256all", "100", "48"), ("128", "", "")])
-def test_routed_ffn_every_remainder_shape(tile, swap, fold, F, monkeypatch):
+@pytest.mark.parametrize("tile,swap", [("256all", ""), ("256all", "0"), ("256all", "100"), ("128", "")])
+def test_routed_ffn_every_remainder_shape(tile, swap, F, monkeypatch):
     """Groups whose last 256-row tile holds 1..256 rows (every swap-tile MMA
-    width class and token-box height, ragged F across two column tiles) and
-    groups whose last 1..48 rows fold into their last full tile, every row
-    against the oracle's SwiGLU of its expert.  F = 320 (a multiple of 64)
-    takes the down projection's chunk-merged swap-tile boxes, F = 200 the
-    per-chunk ones (the up projection, d = 256, always merged)."""
+    width class and token-box height, ragged F across two column tiles), after
+    zero to two full tiles, every row against the oracle's SwiGLU of its
+    expert.  F = 320 (a multiple of 64) takes the down projection's
+    chunk-merged swap-tile boxes, F = 200 the per-chunk ones (the up
+    projection, d = 256, always merged)."""
     monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
     monkeypatch.setenv("MOE_B200_SWAP_MAX", swap)
-    monkeypatch.setenv("MOE_B200_FOLD_MAX", fold)
     y, (x_rows, w13, w2, seg_off) = _remainder_ffn(F)
     sizes = REMAINDER_SIZES
     E, T = len(sizes), sum(sizes)
@@ -295,20 +293,6 @@ def test_routed_ffn_every_remainder_shape(tile, swap, fold, F, monkeypatch):
         lo, hi = seg_off[e], seg_off[e + 1]
         if hi > lo:
             assert rel_err(got[lo:hi], want[lo:hi]) <= 2e-2, (e, sizes[e])
-
-
-@pytest.mark.parametrize("F", [200, 320])
-def test_fold_tiles_are_bit_identical_to_swap_tiles(F, monkeypatch):
-    """A remainder folded into its group's last full tile runs the MMAs of the
-    swap tile it replaces (weights as the 256-row operand, the same k order),
-    and the full tile's own MMAs are unchanged, so every output row is the same
-    bytes with fold tiles on (MOE_B200_FOLD_MAX=48) and off (the default)."""
-    monkeypatch.setenv("MOE_B200_GEMM_TILE", "256all")
-    outs = []
-    for fold in ("48", "0"):
-        monkeypatch.setenv("MOE_B200_FOLD_MAX", fold)
-        outs.append(_remainder_ffn(F)[0])
-    assert torch.equal(outs[0], outs[1])
 
 
 def _row64(xs, t, dtype):
