@@ -643,6 +643,17 @@ def run_ours(args, cfg):
         cpu = {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": f"{n} tokens of the {cfg.name} workload through the float64 oracle's full pipeline "
                          f"(no capacity limit within the sample), one thread, {dt:.1f} s", **host_cpu()}
+        # the same source built with OpenMP on every host core (same bits; a second baseline)
+        import oracle
+        cores = oracle.set_threads(os.cpu_count() or 1)
+        try:
+            n_omp = n * cores
+            v_omp, dt_omp = oracle_tokens_per_s(cfg, inp, n_omp)
+        finally:
+            oracle.set_threads(1)
+        cpu["openmp"] = {"value": v_omp, "unit": "tokens/s", "cores": cores,
+                         "sample": f"{n_omp} tokens, the oracle built with -fopenmp (gate logits and layer rows "
+                                   f"split over {cores} threads), {dt_omp:.1f} s"}
     total_flops = sum(flops.values())
     line = {
         "metric": METRIC, "value": world * T / (ms_max * 1e-3), "unit": "tokens/s", "n_gpus": world,

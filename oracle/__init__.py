@@ -4,7 +4,10 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product path (the CUDA library in
 ``sparse_mixture_experts_04_b200``) never imports, links or calls it, and the
 two share no code.  The arithmetic lives in ``moe_oracle.c`` (plain loops,
-float64, one thread); this module only marshals numpy arrays into it.
+float64); this module only marshals numpy arrays into it.  It runs on one
+thread unless ``set_threads(n)`` with n > 1 switches to the same source built
+with OpenMP (outer loops of the gate logits and layer rows split over
+threads, every output still summed in the same order: the same bits).
 
 Every function here names the passage it follows (page title and section /
 equation); see the header of ``moe_oracle.c`` for the source list.
@@ -45,29 +48,41 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "libmoe_oracle.so")
+_LIB_OMP = os.path.join(_HERE, "libmoe_oracle_omp.so")
 
 F64, F32, BF16 = 0, 1, 2
 BIAS_PROB, BIAS_LOGIT = 0, 1
 
 
-def build(force: bool = False) -> str:
-    """Compile moe_oracle.c with gcc (plain -O2: no fast-math, no reassociation)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile moe_oracle.c with gcc (plain -O2: no fast-math, no reassociation);
+    openmp: the -fopenmp build of the same source."""
+    path = _LIB_OMP if openmp else _LIB
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        tmp = path + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared",
-                               "-fno-fast-math", "-ffp-contract=off",
+                               "-fno-fast-math", "-ffp-contract=off", *(["-fopenmp"] if openmp else []),
                                "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _LIB)
-    return _LIB
+        os.replace(tmp, path)
+    return path
 
 
-_lib = None
+_libs = {}
+_use_omp = False
+
+
+def set_threads(n: int) -> int:
+    """n == 1: the single-thread build (the default); n > 1: the OpenMP build
+    on n threads.  Returns the threads the oracle now uses."""
+    global _use_omp
+    _use_omp = n > 1
+    return int(_L().oracle_set_threads(n))
 
 
 def _L():
-    global _lib
-    if _lib is None:
-        lib = ctypes.CDLL(build())
+    key = "omp" if _use_omp else "seq"
+    if key not in _libs:
+        lib = ctypes.CDLL(build(openmp=_use_omp))
         P = ctypes.c_void_p
         i64, i32, f32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_double
         lib.oracle_gate_logits.argtypes = [i64, i32, i32, P, i32, P, i32, P, P]
@@ -104,8 +119,10 @@ def _L():
         lib.oracle_utilization.restype = None
         lib.oracle_flops.argtypes = [i64, i32, i32, i32, i32, i64, P]
         lib.oracle_flops.restype = None
-        _lib = lib
-    return _lib
+        lib.oracle_set_threads.argtypes = [i32]
+        lib.oracle_set_threads.restype = ctypes.c_int
+        _libs[key] = lib
+    return _libs[key]
 
 
 def _ptr(a):

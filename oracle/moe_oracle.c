@@ -7,9 +7,15 @@
  * never links, loads or calls it, and the two share no code.
  *
  * Style rules this file keeps so that a reader can check it against the pages:
- *   - one plain loop nest per formula, single thread, no blocking, no fusion;
+ *   - one plain loop nest per formula, no blocking, no fusion;
  *   - every sum runs in ascending order of its reduction index;
  *   - all arithmetic is float64; BF16 / FP32 inputs are upcast exactly.
+ *
+ * Threads: the default build (no -fopenmp) runs on one thread.  The same
+ * source compiled with -fopenmp (libmoe_oracle_omp.so, a CPU-baseline build)
+ * splits the outer loops of the gate logits and of the layer rows over
+ * threads: each output is still one thread's sum in the same order, so both
+ * builds give the same bits.
  *
  * Sources (page title, section / equation):
  *   [ZM]  "Zen MoDE: Mixture of Distilled Experts Architecture"
@@ -28,6 +34,21 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Threads the OpenMP build uses from now on (n >= 1); returns the number it
+ * will use.  The default build always returns 1. */
+int oracle_set_threads(int32_t n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* Element type codes for inputs handed to the oracle. */
 enum { ORC_F64 = 0, ORC_F32 = 1, ORC_BF16 = 2 };
@@ -60,6 +81,7 @@ void oracle_gate_logits(int64_t T, int32_t d, int32_t E,
                         const void* x, int32_t x_dt,
                         const void* wg, int32_t wg_dt,
                         const float* offset, double* logits) {
+#pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
         for (int32_t e = 0; e < E; ++e) {
             double acc = 0.0;
@@ -301,6 +323,34 @@ void oracle_swiglu_accumulate(int32_t d, int32_t F, const double* x,
     }
 }
 
+/* One row of oracle_layer_rows (below): token t into yr (d doubles); xr, h scratch.
+ * Returns -1 on an out-of-range token or expert, else 0. */
+static int layer_row(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32_t n_shared,
+                     const void* x, int32_t x_dt, const void* w13, const void* w2,
+                     const void* w13_sh, const void* w2_sh, int32_t w_dt,
+                     const int32_t* idx, const double* w, const int32_t* slot_of,
+                     int64_t t, double* xr, double* h, double* yr) {
+    const int64_t w13_stride = 2 * (int64_t)F * d;
+    const int64_t w2_stride = (int64_t)d * F;
+    if (t < 0 || t >= T) return -1;
+    for (int32_t j = 0; j < d; ++j) xr[j] = ld(x, x_dt, t * d + j);
+    for (int32_t i = 0; i < d; ++i) yr[i] = 0.0;
+    for (int32_t s = 0; s < n_shared; ++s) {
+        const char* a = (const char*)w13_sh + (size_t)(s * w13_stride) * esz(w_dt);
+        const char* b = (const char*)w2_sh + (size_t)(s * w2_stride) * esz(w_dt);
+        oracle_swiglu_accumulate(d, F, xr, a, b, w_dt, 1.0, h, yr);
+    }
+    for (int32_t k = 0; k < K; ++k) {
+        if (slot_of[t * K + k] < 0) continue;
+        int32_t e = idx[t * K + k];
+        if (e < 0 || e >= E) return -1;
+        const char* a = (const char*)w13 + (size_t)(e * w13_stride) * esz(w_dt);
+        const char* b = (const char*)w2 + (size_t)(e * w2_stride) * esz(w_dt);
+        oracle_swiglu_accumulate(d, F, xr, a, b, w_dt, w[t * K + k], h, yr);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------------------
  * The layer output for a list of tokens, given the routing.
  *   y[t] = sum_{s < N_s} Expert^shared_s(x_t)
@@ -321,34 +371,22 @@ int oracle_layer_rows(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int
                       const void* w13_sh, const void* w2_sh, int32_t w_dt,
                       const int32_t* idx, const double* w, const int32_t* slot_of,
                       int64_t n_rows, const int64_t* rows, double* y) {
-    double* xr = (double*)malloc(sizeof(double) * (size_t)d);
-    double* h = (double*)malloc(sizeof(double) * (size_t)F);
-    const int64_t w13_stride = 2 * (int64_t)F * d;
-    const int64_t w2_stride = (int64_t)d * F;
     int rc = 0;
-    for (int64_t r = 0; r < n_rows; ++r) {
-        int64_t t = rows[r];
-        if (t < 0 || t >= T) { rc = -1; break; }
-        for (int32_t j = 0; j < d; ++j) xr[j] = ld(x, x_dt, t * d + j);
-        double* yr = y + r * d;
-        for (int32_t i = 0; i < d; ++i) yr[i] = 0.0;
-        for (int32_t s = 0; s < n_shared; ++s) {
-            const char* a = (const char*)w13_sh + (size_t)(s * w13_stride) * esz(w_dt);
-            const char* b = (const char*)w2_sh + (size_t)(s * w2_stride) * esz(w_dt);
-            oracle_swiglu_accumulate(d, F, xr, a, b, w_dt, 1.0, h, yr);
+#pragma omp parallel
+    {
+        double* xr = (double*)malloc(sizeof(double) * (size_t)d);
+        double* h = (double*)malloc(sizeof(double) * (size_t)F);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            if (layer_row(T, d, E, K, F, n_shared, x, x_dt, w13, w2, w13_sh, w2_sh, w_dt, idx, w, slot_of,
+                          rows[r], xr, h, y + r * d) != 0) {
+#pragma omp atomic write
+                rc = -1;
+            }
         }
-        for (int32_t k = 0; k < K; ++k) {
-            if (slot_of[t * K + k] < 0) continue;
-            int32_t e = idx[t * K + k];
-            if (e < 0 || e >= E) { rc = -1; break; }
-            const char* a = (const char*)w13 + (size_t)(e * w13_stride) * esz(w_dt);
-            const char* b = (const char*)w2 + (size_t)(e * w2_stride) * esz(w_dt);
-            oracle_swiglu_accumulate(d, F, xr, a, b, w_dt, w[t * K + k], h, yr);
-        }
-        if (rc) break;
+        free(xr);
+        free(h);
     }
-    free(xr);
-    free(h);
     return rc;
 }
 

@@ -672,3 +672,40 @@ def test_layer_backward_logit_gradient_matches_finite_differences():
         fd[i] = (J(lp) - J(lm)) / 2e-6
     assert np.max(np.abs(fd - g["dlogits"])) <= 1e-6 * max(1.0, float(np.max(np.abs(fd))))
     assert np.allclose(g["dlogits"].sum(0), g["doff"], rtol=0, atol=1e-12)
+
+
+def test_openmp_build_gives_the_same_bits():
+    """The -fopenmp build of the oracle (the CPU baseline's second figure)
+    splits the outer loops of the gate logits and the layer rows over threads;
+    each output is still one thread's sum in the same order, so every value is
+    the same bits as the single-thread build's (shared experts, drops and a
+    bias included)."""
+    rng = np.random.default_rng(7)
+    T, d, E, K, F, Ns = 37, 48, 6, 2, 40, 1
+    bf = lambda a: (np.asarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    x = bf(rng.normal(size=(T, d)))
+    wg = bf(rng.normal(size=(E, d)) / np.sqrt(d))
+    w13 = bf(rng.normal(size=(E, 2 * F, d)) / np.sqrt(d))
+    w2 = bf(rng.normal(size=(E, d, F)) / np.sqrt(F))
+    w13s = bf(rng.normal(size=(Ns, 2 * F, d)) / np.sqrt(d))
+    w2s = bf(rng.normal(size=(Ns, d, F)) / np.sqrt(F))
+    bias = rng.uniform(-0.05, 0.05, size=E).astype(np.float32)
+    offset = rng.normal(size=E).astype(np.float32)
+
+    def run():
+        l = oracle.gate_logits(x, wg, offset)
+        idx, w, p = oracle.select(l, K, bias=bias)
+        disp = oracle.dispatch(idx, E, 9)
+        y = oracle.layer_rows(x, w13, w2, idx, w, disp["slot_of"], w13_shared=w13s, w2_shared=w2s)
+        return l, idx, w, disp["slot_of"], y
+
+    seq = run()
+    try:
+        n = oracle.set_threads(4)
+        omp = run()
+    finally:
+        assert oracle.set_threads(1) == 1
+    assert n == 4
+    assert (seq[3] < 0).any()          # some pairs dropped
+    for a, b in zip(seq, omp):
+        assert a.dtype == b.dtype and np.array_equal(a.view(np.uint8), b.view(np.uint8))
