@@ -234,10 +234,13 @@ constexpr long long kFusedScanMaxReads = 1ll << 22;
 // on another): every block reads the whole [n_chunks, E] histogram (E x
 // n_chunks int32, a few KB, from L2) to get each expert's total and the count
 // in the chunks before its own, derives kept and seg_off itself, and ranks its
-// 256 tokens.  Block 0 also writes counts / kept / seg_off and, with stats !=
-// nullptr, finalises the balance statistics from the histogram and the chunk
-// probability sums (fixed point) that the selection kernel added: f_e, P_e,
-// the loss, and with zpart the z-loss and utilisation statistics.
+// 256 tokens.  Block 0 also writes counts / kept / seg_off.  With stats !=
+// nullptr one more block (number n_chunks) finalises the balance statistics
+// from the histogram and the chunk probability sums (fixed point) that the
+// selection kernel added: f_e, P_e, the loss, and with zpart the z-loss and
+// utilisation statistics.  It runs beside the ranking blocks: a ranking block
+// that also did the statistics took 2.5x as long as the others (instrumented
+// copy, fine-grained layer: 11.6 vs 4.7 us) and set the kernel's duration.
 //   rank(t,k) = (tokens of earlier chunks for e) + (earlier warps of this
 //   chunk, by popcount of their lane masks) + popcount of the lower lanes
 __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
   __shared__ int wbase[8][kMaxExperts];
   __shared__ double s_fp[kMaxExperts];
   __shared__ double s_red[256];
+  __shared__ unsigned long long s_ps_part[256];
   pdl_wait();
   pdl_trigger();
   stage_clock_start(clk);
@@ -263,21 +267,69 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int b = blockIdx.x;
+  if (b == n_chunks) {  // the statistics block (launched only with stats)
+    // per expert: its count and fixed-point p sum over all chunks (integers,
+    // so the sums do not depend on the order); thread (e, sl) takes the
+    // chunks c = sl (mod S) with all its loads in flight
+    int S = 256 / E;
+    if (S > n_chunks) S = n_chunks;
+    if (S < 1) S = 1;
+    const int e = tid % E, sl = tid / E;
+    int tot = 0;
+    unsigned long long ps = 0;
+    if (tid < E * S) {
+#pragma unroll 16
+      for (int c = sl; c < n_chunks; c += S) {
+        tot += chunk_counts[static_cast<int64_t>(c) * E + e];
+        ps += chunk_psum[static_cast<int64_t>(c) * E + e];
+      }
+    }
+    double z = 0.0;
+    if (zpart)
+      for (int i = tid; i < n_zpart; i += blockDim.x) z += zpart[i];
+    s_tot_part[tid] = tot;
+    s_ps_part[tid] = ps;
+    s_red[tid] = z;
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int tt = 0;
+      unsigned long long pp = 0;
+      for (int q = 0; q < S; ++q) {
+        tt += s_tot_part[q * E + ee];
+        pp += s_ps_part[q * E + ee];
+      }
+      const long long ce = expert_cap ? static_cast<long long>(expert_cap[ee]) : cap;  // Zen MoDE §5.3
+      s_tot[ee] = tt;
+      s_kept[ee] = (ce < 0 || tt < ce) ? tt : static_cast<int>(ce);
+      s_fp[ee] = balance_stats_expert(tt, pp, T, E, K, ee, stats);
+    }
+    if (zpart) {
+      for (int w = 128; w > 0; w >>= 1) {  // fixed-shape tree
+        if (tid < w) s_red[tid] += s_red[tid + w];
+        __syncthreads();
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      balance_loss(s_fp, E, alpha, stats);
+      if (zpart) utilisation_stats(s_tot, s_kept, E, T, s_red[0], stats);
+    }
+    if (clk) {
+      __syncthreads();
+      stage_clock_end(clk);
+    }
+    return;
+  }
   // Every global load that does not depend on another is issued here, before
   // the first barrier, so that their latencies overlap (the kernel is a chain
   // of dependent steps, not bandwidth): this thread's token's experts, its
-  // share of the chunk histogram and, in block 0, the chunk p sums.
+  // share of the chunk histogram.
   const int64_t t = static_cast<int64_t>(b) * kDispatchChunk + tid;
   const bool tok_ok = t < T;
   constexpr int kKReg = 8;  // the first experts of the token stay in registers
   int my_e[kKReg];
 #pragma unroll
   for (int k = 0; k < kKReg; ++k) my_e[k] = (tok_ok && k < K) ? idx[t * K + k] : -1;
-  unsigned long long ps_mine = 0;  // block 0: sum of expert tid's chunk p sums
-  if (b == 0 && stats && tid < E) {
-#pragma unroll 8
-    for (int c = 0; c < n_chunks; ++c) ps_mine += chunk_psum[static_cast<int64_t>(c) * E + tid];
-  }
   // 1. per expert: total over all chunks and the count in chunks before b.
   //    Thread (e, sl) sums a strided set of chunks; E <= 256 experts, S slices.
   int S = 256 / E;
@@ -386,23 +438,6 @@ __global__ void __launch_bounds__(256) dispatch_scan_rank_kernel(
       if (k < K) rank_pair(k, my_e[k]);
     for (int k = kKReg; k < K; ++k) rank_pair(k, idx[t * K + k]);
   }
-  // 5. block 0: the balance statistics (f, P, loss; z-loss and utilisation with zpart)
-  if (b == 0 && stats) {
-    for (int e = tid; e < E; e += blockDim.x) s_fp[e] = balance_stats_expert(s_tot[e], ps_mine, T, E, K, e, stats);
-    double z = 0.0;
-    if (zpart)
-      for (int i = tid; i < n_zpart; i += blockDim.x) z += zpart[i];
-    s_red[tid] = z;
-    __syncthreads();
-    for (int w = 128; w > 0; w >>= 1) {  // fixed-shape tree
-      if (tid < w) s_red[tid] += s_red[tid + w];
-      __syncthreads();
-    }
-    if (tid == 0) {
-      balance_loss(s_fp, E, alpha, stats);
-      if (zpart) utilisation_stats(s_tot, s_kept, E, T, s_red[0], stats);
-    }
-  }
   if (clk) {
     __syncthreads();
     stage_clock_end(clk);
@@ -426,7 +461,8 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* idx, int32_t* count
       return e;
   }
   if (dispatch_fused(p))
-    return launch_k(dispatch_scan_rank_kernel, dim3(n_chunks), dim3(256), 0, st, idx, p.T, p.K, p.E,
+    return launch_k(dispatch_scan_rank_kernel, dim3(n_chunks + (chunk_psum && stats ? 1 : 0)), dim3(256), 0, st,
+                    idx, p.T, p.K, p.E,
                     static_cast<const int32_t*>(chunk_counts), n_chunks, static_cast<long long>(p.cap), expert_cap,
                     counts, kept, seg_off, slot_of, perm, chunk_psum, chunk_psum ? stats : nullptr, p.alpha, zpart,
                     n_zpart, clk);
