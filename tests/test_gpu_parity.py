@@ -40,6 +40,9 @@ SMALL = {
                                capacity_factor=0.05, dtype="bf16", seed=19),
     "wide_e256": MoeConfig("wide_e256", T=200, d_model=128, n_experts=256, top_k=6, d_ff=64, n_shared=0,
                            capacity_factor=2.0, dtype="bf16", seed=20, bias_range=0.01),
+    # the largest top-K of this build (32, with a bias on p: K + 1 ranking rounds exceed the warp)
+    "max_k32": MoeConfig("max_k32", T=96, d_model=128, n_experts=256, top_k=32, d_ff=64, n_shared=1,
+                         capacity_factor=1.0, dtype="bf16", seed=23, bias_range=0.01),
 }
 
 

@@ -27,6 +27,8 @@ CASES = [  # T, d, E, K, bias ("none" | "prob" | "logit"), offset
     (32, 4096, 128, 8, "prob", False),
     (1, 64, 4, 4, "none", True),
     (64, 1024, 64, 8, "logit", False),
+    (100, 128, 256, 32, "prob", False),   # the largest top-K: K + 1 rounds exceed a warp's lanes
+    (65, 64, 64, 32, "none", True),
 ]
 
 
