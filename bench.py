@@ -593,7 +593,26 @@ def run_ours(args, cfg):
         out_rows = [sum(n for p_, o_, n in rk.send.tolist() if p_ != rk.k.rank) +
                     sum(n for p_, o_, n in rk.recv.tolist() if p_ != rk.k.rank) for rk in ranks]
         xbytes = max(out_rows) * row_bytes
+        # the same ranks with the exchange inside the kernels (moe_ep_scatter into the experts'
+        # ranks' receive buffers, moe_ep_combine from their output buffers, device plan)
+        peers = [ep.PeerRank(rk.k) for rk in ranks]
+        ep.connect_emulated(peers)
+        for _ in range(2):
+            ep.forward_emulated_p2p(peers, xb)
+        torch.cuda.synchronize()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for _ in range(n_ep):
+            ep.forward_emulated_p2p(peers, xb)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        p2p_ms = p0.elapsed_time(p1) / n_ep
+        del peers
         epl = {"ranks": G, "emulated_on_one_gpu": True, "ms_per_step_all_ranks": ep_ms,
+               "peer_memory": {"ms_per_step_all_ranks": p2p_ms, "tokens_per_s_on_one_gpu": G * T / (p2p_ms * 1e-3),
+                               "note": "the exchange inside the kernels: rows scattered into the experts' ranks' "
+                                       "receive buffers, outputs read back by the combine, plan on the device, no "
+                                       "host wait (ep.forward_emulated_p2p)"},
                "tokens_per_step": G * T, "tokens_per_s_on_one_gpu": G * T / (ep_ms * 1e-3),
                "exchange_bytes_per_rank_per_direction_max": xbytes,
                "modelled_exchange_ms_at_770GBps": xbytes / 770e9 * 1e3,

@@ -476,6 +476,75 @@ int moe_layer_forward_clocked(const moe_problem_t* p, const void* x, const moe_w
 int moe_ep_plan(int32_t n_ranks, int32_t rank, int32_t n_experts, const int32_t* seg_off_all,
                 int32_t* send, int32_t* recv, int32_t* local_seg_off);
 
+/* Expert-parallel exchange over peer memory (the rows and the outputs cross
+ * between devices inside the kernels, as loads and stores to peer memory;
+ * no copy and no collective on the data path).  Same sources and the same
+ * expert placement as moe_ep_plan: rank q of G holds the global experts
+ * [q E_l, (q+1) E_l), E_l = E / G; every rank routes and ranks its own T
+ * tokens (moe_route, then moe_dispatch with x_perm = NULL).
+ *
+ * A rank's receive buffer (and its output buffer, row for row) is
+ * expert-major: local expert el's rows from source rank 0, then from source 1,
+ * ... -- the grouped expert GEMM's order.  Slot j of rank r for global expert
+ * e lies at row j + delta_r[e] of the buffers of rank e / E_l.
+ *
+ * moe_ep_peer_plan (one small kernel on `stream`; no host synchronisation):
+ *   seg_off_all   [G, E+1] int32 device in: row s = rank s's seg_off (the
+ *                 all-gathered segment offsets; each starts at 0, never
+ *                 decreases)
+ *   delta         [E] int64 device out: delta_r[e] for rank `rank`
+ *   local_seg_off [E_l + 1] int32 device out: the groups of rank `rank`'s
+ *                 receive buffer (local expert el: rows [local_seg_off[el],
+ *                 local_seg_off[el+1])), ready for moe_expert_ffn (ROUTED) of a
+ *                 problem with E_l experts and those weights.
+ *   Errors: MOE_ERR_INVALID_ARG for NULL pointers, G < 1, rank out of range,
+ *   E > 256 or E % G != 0. */
+int moe_ep_peer_plan(int32_t n_ranks, int32_t rank, int32_t n_experts, const int32_t* seg_off_all,
+                     int64_t* delta, int32_t* local_seg_off, moe_stream_t stream);
+
+/* moe_ep_scatter: the dispatch's row gather, each kept row written straight
+ * into the receive buffer of the rank that holds its expert:
+ *   for every slot j < seg_off[E] of this rank, expert e of that slot:
+ *     recv_bufs[e / E_l][(j + delta[e]) * d ...] = x[(perm[j] / K) * d ...]
+ *   x          [T, d] device in (16-byte aligned); perm, seg_off from this
+ *              rank's moe_dispatch; delta [E] int64 device from moe_ep_peer_plan
+ *   recv_bufs  [G] device array of device pointers: rank q's receive buffer
+ *              (peer memory mapped into this process for q != rank, e.g. by
+ *              moe_ipc_open), each [rows q receives, d]
+ * The receiving rank may read its buffer once every rank's scatter has
+ * completed (the caller orders that, e.g. with a barrier on the stream). */
+int moe_ep_scatter(const moe_problem_t* p, int32_t n_ranks, const void* x, const int32_t* perm,
+                   const int32_t* seg_off, void* const* recv_bufs, const int64_t* delta,
+                   moe_stream_t stream);
+
+/* moe_ep_combine: moe_combine with each kept pair's expert output read from
+ * the rank that computed it:
+ *   y[t] = y_shared[t] + sum_{k: slot_of[t,k] >= 0} topk_w[t,k] *
+ *          out_bufs[e / E_l][(slot_of[t,k] + delta[e]) * d ...],  e = topk_idx[t,k]
+ * in moe_combine's order and rounding (shared first, then k ascending, FP32
+ * sums, one rounding).  out_bufs [G] device array of device pointers (rank
+ * q's output buffer, row for row its receive buffer); y_shared as in
+ * moe_combine (NULL iff n_shared == 0); y [T, d] out.  Every rank's expert
+ * GEMM must have completed before the call's kernel starts. */
+int moe_ep_combine(const moe_problem_t* p, int32_t n_ranks, const void* const* out_bufs,
+                   const int64_t* delta, const int32_t* topk_idx, const int32_t* slot_of,
+                   const float* topk_w, const void* y_shared, void* y, moe_stream_t stream);
+
+/* Buffers another process can map (CUDA IPC), for the receive and output
+ * buffers of moe_ep_scatter / moe_ep_combine across processes:
+ *   moe_ipc_malloc  a whole device allocation of `bytes` (so a peer that opens
+ *                   its handle maps it at offset 0); free with moe_ipc_free
+ *   moe_ipc_handle  its handle, MOE_IPC_HANDLE_BYTES bytes, into `handle` (host)
+ *   moe_ipc_open    maps a handle from another process (peer access enabled
+ *                   lazily); unmap with moe_ipc_close
+ * Errors: MOE_ERR_INVALID_ARG for NULL pointers or 0 bytes; MOE_ERR_CUDA. */
+#define MOE_IPC_HANDLE_BYTES 64
+int moe_ipc_malloc(size_t bytes, void** ptr);
+int moe_ipc_free(void* ptr);
+int moe_ipc_handle(const void* ptr, void* handle);
+int moe_ipc_open(const void* handle, void** ptr);
+int moe_ipc_close(void* ptr);
+
 #ifdef __cplusplus
 }
 #endif

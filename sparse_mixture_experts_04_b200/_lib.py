@@ -29,7 +29,8 @@ EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_row
             "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_layer_forward_profiled",
             "moe_layer_forward_clocked", "moe_expert_ffn_segments",
             "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update", "moe_backward_workspace_size",
-            "moe_layer_backward", "moe_ep_plan")
+            "moe_layer_backward", "moe_ep_plan", "moe_ep_peer_plan", "moe_ep_scatter", "moe_ep_combine",
+            "moe_ipc_malloc", "moe_ipc_free", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
 NUM_CLOCKS = 7  # MOE_CLOCK_ROUTE .. MOE_CLOCK_COMBINE
@@ -120,6 +121,22 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_backward.restype = ctypes.c_int
     L.moe_ep_plan.argtypes = [i32, i32, i32, P, P, P, P]
     L.moe_ep_plan.restype = ctypes.c_int
+    L.moe_ep_peer_plan.argtypes = [i32, i32, i32, P, P, P, P]
+    L.moe_ep_peer_plan.restype = ctypes.c_int
+    L.moe_ep_scatter.argtypes = [PP, i32, P, P, P, P, P, P]
+    L.moe_ep_scatter.restype = ctypes.c_int
+    L.moe_ep_combine.argtypes = [PP, i32, P, P, P, P, P, P, P, P]
+    L.moe_ep_combine.restype = ctypes.c_int
+    L.moe_ipc_malloc.argtypes = [sz, ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_ipc_malloc.restype = ctypes.c_int
+    L.moe_ipc_free.argtypes = [P]
+    L.moe_ipc_free.restype = ctypes.c_int
+    L.moe_ipc_handle.argtypes = [P, P]
+    L.moe_ipc_handle.restype = ctypes.c_int
+    L.moe_ipc_open.argtypes = [P, ctypes.POINTER(ctypes.c_void_p)]
+    L.moe_ipc_open.restype = ctypes.c_int
+    L.moe_ipc_close.argtypes = [P]
+    L.moe_ipc_close.restype = ctypes.c_int
     if L.moe_abi_version() != ABI_VERSION:
         raise RuntimeError(f"{LIB_PATH} has ABI version {L.moe_abi_version()}, this binding expects {ABI_VERSION}: "
                            "rebuild it")

@@ -253,3 +253,75 @@ def moe_ep_plan(n_ranks: int, rank: int, n_experts: int, seg_off_all) -> tuple:
     rc = _lib.lib().moe_ep_plan(G, int(rank), E, so.data_ptr(), send.data_ptr(), recv.data_ptr(), local.data_ptr())
     _lib.check("moe_ep_plan", rc)
     return send[:G], recv[:G], local
+
+
+# ----------------------------------------------------- expert parallel over peer memory
+IPC_HANDLE_BYTES = 64
+
+
+def moe_ep_peer_plan(n_ranks: int, rank: int, n_experts: int, seg_off_all, delta, local_seg_off, stream=None):
+    """Device plan of the peer-memory exchange (one kernel, no host wait):
+    seg_off_all [G, E+1] int32 (device) -> delta [E] int64 and
+    local_seg_off [E/G + 1] int32 (device); see include/moe_b200.h."""
+    rc = _lib.lib().moe_ep_peer_plan(int(n_ranks), int(rank), int(n_experts), _p(seg_off_all), _p(delta),
+                                     _p(local_seg_off), _stream(stream))
+    _lib.check("moe_ep_peer_plan", rc)
+
+
+def moe_ep_scatter(prob, n_ranks: int, x, perm, seg_off, recv_bufs, delta, stream=None):
+    """Each kept row of this rank written into the receive buffer of its
+    expert's rank; recv_bufs: [G] int64 device tensor of device pointers."""
+    rc = _lib.lib().moe_ep_scatter(ctypes.byref(prob), int(n_ranks), _p(x), _p(perm), _p(seg_off), _p(recv_bufs),
+                                   _p(delta), _stream(stream))
+    _lib.check("moe_ep_scatter", rc)
+
+
+def moe_ep_combine(prob, n_ranks: int, out_bufs, delta, topk_idx, slot_of, topk_w, y_shared, y, stream=None):
+    """moe_combine reading each kept pair's output from its expert's rank;
+    out_bufs: [G] int64 device tensor of device pointers."""
+    rc = _lib.lib().moe_ep_combine(ctypes.byref(prob), int(n_ranks), _p(out_bufs), _p(delta), _p(topk_idx),
+                                   _p(slot_of), _p(topk_w), _p(y_shared), _p(y), _stream(stream))
+    _lib.check("moe_ep_combine", rc)
+
+
+class IpcBuffer:
+    """A whole device allocation (moe_ipc_malloc) another process can map,
+    or the mapping of one (moe_ipc_open); `tensor` views it as a torch tensor
+    (through __cuda_array_interface__).  release() frees / unmaps it."""
+
+    def __init__(self, shape, dtype, handle: bytes | None = None):
+        self.shape, self.dtype = tuple(int(n) for n in shape), dtype
+        nbytes = max(1, int(torch.tensor([], dtype=dtype).element_size()))
+        for n in self.shape:
+            nbytes *= n
+        ptr = ctypes.c_void_p()
+        if handle is None:
+            _lib.check("moe_ipc_malloc", _lib.lib().moe_ipc_malloc(max(nbytes, 16), ctypes.byref(ptr)))
+            self.opened = False
+        else:
+            buf = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+            _lib.check("moe_ipc_open", _lib.lib().moe_ipc_open(buf, ctypes.byref(ptr)))
+            self.opened = True
+        self.ptr = int(ptr.value)
+        # BF16 has no array-interface type code: viewed as int16, then as BF16
+        typestr = {torch.bfloat16: "<i2", torch.float32: "<f4", torch.int32: "<i4", torch.int64: "<i8"}[dtype]
+        t = torch.as_tensor(_Iface(self.shape, typestr, self.ptr), device="cuda")
+        self.tensor = t.view(torch.bfloat16) if dtype == torch.bfloat16 else t
+
+    def handle(self) -> bytes:
+        buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+        _lib.check("moe_ipc_handle", _lib.lib().moe_ipc_handle(self.ptr, buf))
+        return buf.raw
+
+    def release(self) -> None:
+        if self.ptr:
+            self.tensor = None
+            fn = _lib.lib().moe_ipc_close if self.opened else _lib.lib().moe_ipc_free
+            _lib.check("moe_ipc_release", fn(self.ptr))
+            self.ptr = 0
+
+
+class _Iface:
+    def __init__(self, shape, typestr, ptr):
+        self.__cuda_array_interface__ = {"shape": shape, "typestr": typestr, "data": (ptr, False), "version": 3,
+                                         "strides": None}

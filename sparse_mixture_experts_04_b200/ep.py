@@ -28,6 +28,11 @@ buffers, computes nothing and moves rows with torch.distributed point-to-point
 operations (NCCL between GPUs, gloo between CPU processes), or with device
 copies for the chunks a rank keeps for itself.  `forward_emulated` runs the
 same schedule for G ranks held in one process (every exchange a copy).
+
+The second schedule (`PeerRank`, `forward_p2p`, `forward_emulated_p2p`, at the
+end of this module) moves the rows inside the kernels instead: the dispatch
+writes them into the experts' ranks' memory and the combine reads the outputs
+from there, with a device-side plan and no host round trip.
 """
 from __future__ import annotations
 
@@ -104,6 +109,20 @@ class CudaExperts:
         else:
             api.moe_dispatch(P, self.topk_idx, x, self.counts, self.kept, self.seg_off, self.slot_of, self.perm,
                              self.x_perm, self.ws)
+        return self.seg_off
+
+    def route_rank(self, x: torch.Tensor) -> torch.Tensor:
+        """Routing and the dispatch's ranks only (no gather): the peer-memory
+        exchange moves the rows itself; returns this rank's seg_off [E+1]."""
+        w, P = self.weights, self.prob
+        api.moe_route(P, x, w.get("w_gate"), w.get("logit_offset"), w.get("sel_bias"), self.logits, self.topk_idx,
+                      self.topk_w, self.stats, self.ws)
+        if self.capacity_flag:
+            api.moe_dispatch_capacity(P, self.topk_idx, w["expert_capacity"], x, self.counts, self.kept,
+                                      self.seg_off, self.slot_of, self.perm, None, self.ws)
+        else:
+            api.moe_dispatch(P, self.topk_idx, x, self.counts, self.kept, self.seg_off, self.slot_of, self.perm,
+                             None, self.ws)
         return self.seg_off
 
     def experts(self, n_rows: int, local_seg_off: torch.Tensor) -> None:
@@ -278,3 +297,162 @@ def split_weights(weights: dict, n_ranks: int, rank: int) -> dict:
     out["w13"] = weights["w13"][rank * El:(rank + 1) * El].contiguous()
     out["w2"] = weights["w2"][rank * El:(rank + 1) * El].contiguous()
     return out
+
+
+# ------------------------------------------------------------------------------------------
+# The exchange over peer memory: the dispatch writes each kept row straight into the
+# receive buffer of its expert's rank (moe_ep_scatter), and the combine reads each
+# expert output from the rank that computed it (moe_ep_combine) -- loads and stores to
+# peer memory inside the kernels.  The receive buffer is expert-major (local expert el's
+# rows from source 0, then source 1, ...), so the local experts run as one group each
+# (moe_expert_ffn over E_l groups, no regrouping), and the plan is a device kernel
+# (moe_ep_peer_plan) on the all-gathered segment offsets: no host round trip.
+
+
+class PeerRank:
+    """One rank of the peer-memory schedule.  `kernels` (CudaExperts) holds the
+    rank's routing buffers and its receive / output buffers x_loc / y_loc;
+    connect() gives it every rank's x_loc and y_loc addresses (rank q's
+    buffers at index q: local tensors in one process, mapped peer memory
+    across processes)."""
+
+    def __init__(self, kernels: CudaExperts):
+        k = self.k = kernels
+        dev = k.device
+        self.delta = torch.empty(k.prob.n_experts, dtype=torch.int64, device=dev)
+        self.local_seg_off = torch.empty(k.n_local + 1, dtype=torch.int32, device=dev)
+        self.recv_ptrs = self.out_ptrs = None
+        self.ipc = []
+
+    def connect(self, recv_ptrs, out_ptrs) -> None:
+        G = self.k.n_ranks
+        if len(recv_ptrs) != G or len(out_ptrs) != G:
+            raise ValueError(f"{G} ranks need {G} receive and {G} output buffers")
+        self.recv_ptrs = torch.tensor([int(p) for p in recv_ptrs], dtype=torch.int64, device=self.k.device)
+        self.out_ptrs = torch.tensor([int(p) for p in out_ptrs], dtype=torch.int64, device=self.k.device)
+
+    def route(self, x: torch.Tensor) -> torch.Tensor:
+        return self.k.route_rank(x)
+
+    def plan(self, seg_off_all: torch.Tensor) -> None:
+        """seg_off_all [G, E+1] int32 on the device (every rank's seg_off)."""
+        k = self.k
+        api.moe_ep_peer_plan(k.n_ranks, k.rank, k.prob.n_experts, seg_off_all, self.delta, self.local_seg_off)
+
+    def scatter(self, x: torch.Tensor) -> None:
+        k = self.k
+        api.moe_ep_scatter(k.prob, k.n_ranks, x, k.perm, k.seg_off, self.recv_ptrs, self.delta)
+
+    def experts(self) -> None:
+        k = self.k
+        api.moe_expert_ffn(k.prob_local, api.FFN_ROUTED, k.x_loc, k.max_local_rows, self.local_seg_off,
+                           k.weights["w13"], k.weights["w2"], k.y_loc, k.ws_local)
+
+    def shared(self, x: torch.Tensor) -> None:
+        self.k.shared(x)
+
+    def combine(self, y: torch.Tensor | None = None) -> torch.Tensor:
+        k = self.k
+        if y is None:
+            y = torch.empty((k.prob.T, k.d_model), dtype=k.dtype, device=k.device)
+        api.moe_ep_combine(k.prob, k.n_ranks, self.out_ptrs, self.delta, k.topk_idx, k.slot_of, k.topk_w,
+                           k.y_shared, y)
+        return y
+
+    def release(self) -> None:
+        """Unmap the peers' buffers and free this rank's own (open_peer_buffers)."""
+        for b in self.ipc:
+            b.release()
+        self.ipc = []
+
+
+def connect_emulated(ranks: list) -> None:
+    """G PeerRanks held in one process: every rank's table points at the
+    others' local buffers."""
+    recv = [rk.k.x_loc.data_ptr() for rk in ranks]
+    out = [rk.k.y_loc.data_ptr() for rk in ranks]
+    for rk in ranks:
+        rk.connect(recv, out)
+
+
+def forward_emulated_p2p(ranks: list, xs: list) -> list:
+    """The peer-memory schedule for G ranks held in one process (connect_emulated
+    first): route and rank every batch, one device plan per rank, every rank's
+    scatter into the others' receive buffers, the local experts, and every
+    rank's combine from the others' output buffers -- in stream order, which
+    orders the phases as the barriers of `forward_p2p` do.  No host wait.
+    Returns the G layer outputs."""
+    if len(ranks) != len(xs):
+        raise ValueError("one batch per rank")
+    seg_all = torch.stack([rk.route(x) for rk, x in zip(ranks, xs)])
+    for rk in ranks:
+        rk.plan(seg_all)
+    for rk, x in zip(ranks, xs):
+        rk.scatter(x)
+    for rk, x in zip(ranks, xs):
+        rk.shared(x)
+        rk.experts()
+    return [rk.combine() for rk in ranks]
+
+
+def open_peer_buffers(rank_state: PeerRank, group=None) -> None:
+    """Across processes (one per GPU, torch.distributed initialised): give the
+    rank receive and output buffers other processes can map (CUDA IPC), swap
+    handles with every rank, map the peers' and connect the tables.  Release
+    with rank_state.release() before the process group is destroyed."""
+    import torch.distributed as dist
+    k = rank_state.k
+    G, rank = dist.get_world_size(group), dist.get_rank(group)
+    if G != k.n_ranks or rank != k.rank:
+        raise RuntimeError(f"process group rank {rank}/{G} but the experts were placed for {k.rank}/{k.n_ranks}")
+    shape = (k.max_local_rows, k.d_model)
+    xb, yb = api.IpcBuffer(shape, k.dtype), api.IpcBuffer(shape, k.dtype)
+    k.x_loc, k.y_loc = xb.tensor, yb.tensor
+    rank_state.ipc = [xb, yb]
+    handles = [None] * G
+    dist.all_gather_object(handles, (xb.handle(), yb.handle()), group=group)
+    recv, out = [], []
+    for q, (hx, hy) in enumerate(handles):
+        if q == rank:
+            recv.append(xb.ptr)
+            out.append(yb.ptr)
+            continue
+        px, py = api.IpcBuffer(shape, k.dtype, handle=hx), api.IpcBuffer(shape, k.dtype, handle=hy)
+        rank_state.ipc += [px, py]
+        recv.append(px.ptr)
+        out.append(py.ptr)
+    rank_state.connect(recv, out)
+
+
+def _stream_barrier(group=None) -> None:
+    """Every rank's work enqueued so far has completed before any rank's
+    next kernel starts: a one-element all-reduce ordered on the current stream."""
+    import torch.distributed as dist
+    flag = torch.zeros(1, dtype=torch.float32, device=torch.cuda.current_device())
+    dist.all_reduce(flag, group=group)
+
+
+def forward_p2p(rank_state: PeerRank, x: torch.Tensor, y: torch.Tensor | None = None, group=None) -> torch.Tensor:
+    """One expert-parallel forward with the exchange over peer memory
+    (open_peer_buffers first).  Per rank: route and rank; all-gather of the
+    segment offsets into device memory; device plan; scatter of the kept rows
+    into their experts' ranks; barrier; shared and local experts; barrier;
+    combine from the ranks that computed the outputs.  The barriers also
+    order consecutive forwards: a rank scatters into a peer's receive buffer
+    only after that peer's experts have read it, and computes into its output
+    buffer only after every peer's combine has read it."""
+    import torch.distributed as dist
+    k = rank_state.k
+    G = dist.get_world_size(group)
+    if G != k.n_ranks or dist.get_rank(group) != k.rank:
+        raise RuntimeError("the process group does not match the expert placement")
+    seg = rank_state.route(x)
+    seg_all = torch.empty((G, seg.numel()), dtype=seg.dtype, device=seg.device)
+    dist.all_gather_into_tensor(seg_all, seg, group=group)
+    rank_state.plan(seg_all)
+    rank_state.scatter(x)
+    _stream_barrier(group)
+    rank_state.shared(x)
+    rank_state.experts()
+    _stream_barrier(group)
+    return rank_state.combine(y)

@@ -145,3 +145,131 @@ def test_expert_ffn_segments_repeat_the_experts(dtype, tile, monkeypatch):
     want = np.stack([oracle.swiglu(x64[r], a[e_of[r]], b[e_of[r]]) for r in pick])
     got = y.float().cpu().numpy()[pick]
     assert rel_err(got, want) <= (2e-2 if dtype == "bf16" else 1e-4)
+
+
+# ------------------------------------------------------------ the exchange over peer memory
+def _plan_reference(seg_all, rank):
+    """The receive layout written out: expert-major receive buffers, source
+    ranks in order within an expert; returns (delta [E], local_seg_off)."""
+    G, E1 = seg_all.shape
+    E, El = E1 - 1, (E1 - 1) // G
+    rows = seg_all[:, 1:].astype(np.int64) - seg_all[:, :-1]          # [G, E]
+    tot = rows.sum(axis=0)
+    delta = np.zeros(E, np.int64)
+    for e in range(E):
+        q = e // El
+        base = tot[q * El:e].sum()
+        delta[e] = base + rows[:rank, e].sum() - seg_all[rank, e]
+    own = tot[rank * El:(rank + 1) * El]
+    local = np.concatenate([[0], np.cumsum(own)]).astype(np.int32)
+    return delta, local
+
+
+@pytest.mark.parametrize("G,E", [(1, 8), (2, 8), (4, 64), (8, 256), (8, 8)])
+def test_peer_plan_matches_its_definition(G, E):
+    rng = np.random.default_rng(G * 1000 + E)
+    counts = rng.integers(0, 40, size=(G, E))
+    counts[:, rng.integers(0, E)] = 0                                   # an expert nobody chose
+    seg_all = np.concatenate([np.zeros((G, 1), np.int64), np.cumsum(counts, axis=1)], axis=1).astype(np.int32)
+    sa = torch.as_tensor(seg_all).cuda()
+    for rank in range(G):
+        delta = torch.empty(E, dtype=torch.int64, device="cuda")
+        local = torch.empty(E // G + 1, dtype=torch.int32, device="cuda")
+        api.moe_ep_peer_plan(G, rank, E, sa, delta, local)
+        want_d, want_l = _plan_reference(seg_all, rank)
+        assert (delta.cpu().numpy() == want_d).all()
+        assert (local.cpu().numpy() == want_l).all()
+    # every slot of every rank lands on a distinct row of its owner's buffer
+    El = E // G
+    for q in range(G):
+        seen = []
+        for r in range(G):
+            d_r, _ = _plan_reference(seg_all, r)
+            for e in range(q * El, (q + 1) * El):
+                seen += [j + d_r[e] for j in range(seg_all[r, e], seg_all[r, e + 1])]
+        assert sorted(seen) == list(range(int(counts[:, q * El:(q + 1) * El].sum())))
+
+
+def _peer_ranks(cfg, inp, G):
+    ranks = [ep.PeerRank(rk.k) for rk in _ranks(cfg, inp, G)]
+    ep.connect_emulated(ranks)
+    return ranks
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("name", list(CFGS))
+def test_emulated_peer_exchange_equals_the_copy_schedule(name, G):
+    """Scatter into the experts' ranks' buffers, local experts over the
+    expert-major buffer, combine from the owners' outputs: the rows reach the
+    expert GEMM in the order the copy schedule's regrouping gives them, and the
+    combine adds the same terms in the same order, so every rank's output is
+    the same bytes as ep.forward_emulated's; and within the layer's tolerance
+    of the oracle."""
+    cfg = CFGS[name]
+    inp = generate(cfg)
+    xs = [dev(x) for x in extra_activations(cfg, G)]
+    ys_copy = [y.clone() for y in ep.forward_emulated(_ranks(cfg, inp, G), xs)]
+    ranks = _peer_ranks(cfg, inp, G)
+    ys = ep.forward_emulated_p2p(ranks, xs)
+    torch.cuda.synchronize()
+    for r in range(G):
+        k = ranks[r].k
+        assert api.read_device_status(k.ws) == 0 and api.read_device_status(k.ws_local) == 0
+        assert torch.equal(ys[r], ys_copy[r]), r
+        want = _reference(inp, xs[r].cpu(), k)
+        assert rel_err(ys[r].float().cpu().numpy(), want) <= tol(cfg)
+    # the receive buffers hold every kept row once
+    assert sum(int(rk.local_seg_off[-1]) for rk in ranks) == sum(int(rk.k.seg_off[-1]) for rk in ranks)
+    # a second forward on the same buffers gives the same outputs
+    ys2 = ep.forward_emulated_p2p(ranks, xs)
+    for r in range(G):
+        assert torch.equal(ys2[r], ys[r])
+
+
+def test_one_rank_nccl_group_peer_exchange():
+    """forward_p2p through a one-rank NCCL group: IPC-allocated receive and
+    output buffers, the all-gather into device memory, the device plan and
+    the two stream barriers; equal to the copy schedule's ep.forward."""
+    import torch.distributed as dist
+    cfg = CFGS["small"]
+    inp = generate(cfg)
+    x = dev(extra_activations(cfg, 1)[0])
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    rk = None
+    try:
+        y_copy = ep.forward(_ranks(cfg, inp, 1)[0], x).clone()
+        rk = ep.PeerRank(_ranks(cfg, inp, 1)[0].k)
+        ep.open_peer_buffers(rk)
+        y = ep.forward_p2p(rk, x).clone()
+        y2 = ep.forward_p2p(rk, x).clone()
+        torch.cuda.synchronize()
+    finally:
+        if rk is not None:
+            rk.release()
+        dist.destroy_process_group()
+    assert torch.equal(y, y_copy) and torch.equal(y2, y)
+    assert rel_err(y.float().cpu().numpy(), _reference(inp, x.cpu(), rk.k)) <= tol(cfg)
+
+
+def test_scatter_into_a_buffer_mapped_from_another_process():
+    """CUDA IPC on one GPU: this process allocates a receive buffer
+    (moe_ipc_malloc) and hands its handle to a second process, which maps it
+    (moe_ipc_open) and runs moe_ep_scatter into it; the rows arrive here."""
+    import subprocess
+    import sys
+    n, d, seed = 300, 264, 5
+    buf = api.IpcBuffer((n, d), torch.bfloat16)
+    try:
+        buf.tensor.zero_()
+        torch.cuda.synchronize()
+        child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "ep_ipc_child.py")
+        r = subprocess.run([sys.executable, child, buf.handle().hex(), str(n), str(d), str(seed)],
+                           capture_output=True, text=True, timeout=300)
+        assert r.returncode == 0, r.stderr[-2000:]
+        g = torch.Generator().manual_seed(seed)
+        want = torch.randn((n, d), generator=g).to(torch.bfloat16)
+        assert torch.equal(buf.tensor.cpu(), want)
+    finally:
+        buf.release()
