@@ -233,3 +233,82 @@ def test_gloo_ranks_equal_the_single_device_layer(world):
     assert [o[0] for o in out] == list(range(world))
     assert all(o[1] for o in out), out
     assert all(o[2] > 0 for o in out)
+
+
+# ------------------------------------------- the peer-memory form: buffer tables across processes
+class _FakeIpc:
+    """Stands in for api.IpcBuffer on CPU: an allocation gets an address that
+    encodes (owner rank, buffer kind) and a handle that carries it; mapping a
+    handle gives the owner's address back, as CUDA IPC maps the same memory."""
+    rank = 0
+    made = []
+
+    def __init__(self, shape, dtype, handle=None):
+        if handle is None:
+            kind = sum(1 for b in _FakeIpc.made if not b.opened)
+            self.ptr = 1_000_000 * (_FakeIpc.rank + 1) + kind
+            self.opened = False
+        else:
+            self.ptr = int.from_bytes(handle[:8], "little")
+            self.opened = True
+        self.tensor = torch.zeros(shape, dtype=dtype)
+        self.released = False
+        _FakeIpc.made.append(self)
+
+    def handle(self):
+        return self.ptr.to_bytes(8, "little") + bytes(api.IPC_HANDLE_BYTES - 8)
+
+    def release(self):
+        self.released = True
+
+
+class _Kernels:
+    def __init__(self, world, rank):
+        self.n_ranks, self.rank, self.prob = world, rank, api.make_problem(8, 16, 2 * world, 1, 16)
+        self.n_local, self.max_local_rows, self.d_model = 2, 5, 16
+        self.dtype, self.device = torch.float32, torch.device("cpu")
+        self.x_loc = self.y_loc = None
+
+
+def _peer_table_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        _FakeIpc.rank = rank
+        api.IpcBuffer = _FakeIpc          # this process only (spawned)
+        rk = ep.PeerRank(_Kernels(world, rank))
+        ep.open_peer_buffers(rk)
+        own = [b.ptr for b in _FakeIpc.made if not b.opened]
+        q.put((rank, rk.recv_ptrs.tolist(), rk.out_ptrs.tolist(), own,
+               tuple(rk.k.x_loc.shape), len(rk.ipc)))
+        rk.release()
+        assert all(b.released for b in _FakeIpc.made)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_open_peer_buffers_tables_list_every_rank_in_order(world):
+    """ep.open_peer_buffers on gloo ranks with a stand-in for the IPC calls:
+    every rank's receive and output tables hold, at index q, rank q's own
+    buffers (its own allocations at its own index, the peers' mapped from
+    their handles), and each rank keeps 2 + 2 (G - 1) mappings to release."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_peer_table_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=300) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    owners = {r: own for r, _, _, own, _, _ in out}
+    for r, recv, outp, own, shape, n_ipc in out:
+        assert recv == [owners[s][0] for s in range(world)]
+        assert outp == [owners[s][1] for s in range(world)]
+        assert shape == (5, 16) and n_ipc == 2 * world
