@@ -26,6 +26,9 @@ CFGS = {
     # groups of a few hundred rows (pair tiles), no capacity limit, no shared expert
     "pairs": MoeConfig("ep_pairs", T=1536, d_model=512, n_experts=8, top_k=2, d_ff=1024, n_shared=0,
                        capacity_factor=0.0, dtype="bf16", seed=22, x_std=1.0),
+    # FP32 (CUDA-core expert GEMMs), ragged d and F
+    "f32": MoeConfig("ep_f32", T=200, d_model=72, n_experts=8, top_k=2, d_ff=40, n_shared=1,
+                     capacity_factor=1.0, dtype="f32", seed=23, x_std=0.5),
 }
 
 
@@ -273,3 +276,38 @@ def test_scatter_into_a_buffer_mapped_from_another_process():
         assert torch.equal(buf.tensor.cpu(), want)
     finally:
         buf.release()
+
+
+@pytest.mark.parametrize("G", [2, 8])
+def test_emulated_peer_exchange_with_per_expert_capacity(G):
+    """MOE_FLAG_EXPERT_CAPACITY (Zen MoDE §5.3, a capacity per expert, some 0):
+    each rank ranks with moe_dispatch_capacity; the peer-memory schedule equals
+    the copy schedule byte for byte and the oracle on the rows each rank kept."""
+    cfg = CFGS["small"]
+    inp = generate(cfg)
+    xs = [dev(x) for x in extra_activations(cfg, G)]
+    rng = np.random.default_rng(G)
+    caps = rng.integers(0, 3 * cfg.T * cfg.top_k // cfg.n_experts, size=cfg.n_experts).astype(np.int32)
+    caps[1] = 0
+
+    def ranks(peer):
+        P = api.make_problem(cfg.T, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.n_shared,
+                             cfg.capacity_factor, cfg.dtype, api.FLAG_EXPERT_CAPACITY, cfg.alpha)
+        full = {k: dev(inp[k]) for k in ("w_gate", "w13", "w2", "w13_shared", "w2_shared")}
+        full["expert_capacity"] = torch.as_tensor(caps).cuda()
+        ks = [ep.CudaExperts(P, ep.split_weights(full, G, r), G, r) for r in range(G)]
+        if not peer:
+            return [ep.EpRank(k) for k in ks]
+        out = [ep.PeerRank(k) for k in ks]
+        ep.connect_emulated(out)
+        return out
+
+    ys_copy = [y.clone() for y in ep.forward_emulated(ranks(False), xs)]
+    rk = ranks(True)
+    ys = ep.forward_emulated_p2p(rk, xs)
+    torch.cuda.synchronize()
+    for r in range(G):
+        k = rk[r].k
+        assert (k.kept.cpu().numpy() <= caps).all() and int(k.kept[1]) == 0
+        assert torch.equal(ys[r], ys_copy[r]), r
+        assert rel_err(ys[r].float().cpu().numpy(), _reference(inp, xs[r].cpu(), k)) <= tol(cfg)
