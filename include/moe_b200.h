@@ -31,9 +31,11 @@
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers, row-major, densely packed, owned
- *     by the caller.  The library never allocates or frees device memory and
- *     keeps no state between calls; scratch space is the caller's workspace
- *     `ws` of `ws_bytes` bytes (size from moe_workspace_size; 256-byte aligned).
+ *     by the caller.  The library never allocates or frees device memory
+ *     (except moe_ipc_malloc / moe_ipc_free, which exist to do so for buffers
+ *     other processes map) and keeps no state between calls; scratch space is
+ *     the caller's workspace `ws` of `ws_bytes` bytes (size from
+ *     moe_workspace_size; 256-byte aligned).
  *   - Every call only enqueues work on `stream` and returns; nothing
  *     synchronises with the host (except moe_read_device_status).
  *   - Activations and weights are BF16 (MOE_DTYPE_BF16) or FP32 (MOE_DTYPE_F32);
