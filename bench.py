@@ -639,11 +639,8 @@ def run_ours(args, cfg):
     # HBM fractions of the memory-bound stages from the device-stamped spans
     # (first CTA start to last CTA end of the stage's kernels), and from the
     # event pass beside them (which adds a launch gap at every stage boundary)
-    # with the combine inside the down projection's epilogue there is no combine stage of its own
-    fused = api.layer_combine_fused(layer.prob)
-    mem_bytes = {"router": router_bytes(cfg), "dispatch": dispatch_bytes(cfg, kept)}
-    if not fused:
-        mem_bytes["combine"] = combine_bytes(cfg, kept)
+    mem_bytes = {"router": router_bytes(cfg), "dispatch": dispatch_bytes(cfg, kept),
+                 "combine": combine_bytes(cfg, kept)}
     span_key = {"router": "route", "dispatch": "dispatch+gather", "combine": "combine"}
     event_key = {"router": "routed", "dispatch": "dispatched", "combine": "end"}
     gbs_clock = {k: (mem_bytes[k] / (clock_spans[span_key[k]] * 1e-6) / 1e9
@@ -651,7 +648,7 @@ def run_ours(args, cfg):
     gbs_event = {k: mem_bytes[k] / (stage[event_key[k]] * 1e-3) / 1e9 for k in mem_bytes}
     disp_gbs = gbs_clock["dispatch"] or gbs_event["dispatch"]
     router_gbs = gbs_clock["router"] or gbs_event["router"]
-    combine_gbs = None if fused else (gbs_clock["combine"] or gbs_event["combine"])
+    combine_gbs = gbs_clock["combine"] or gbs_event["combine"]
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -698,9 +695,8 @@ def run_ours(args, cfg):
         "expert_gemm_pct_sustained_peak": (100.0 * gemm_tflops / peaks["bf16_tflops_sustained"]
                                            if peaks.get("bf16_tflops_sustained") else None),
         "dispatch_gbs": disp_gbs, "router_gbs": router_gbs, "combine_gbs": combine_gbs,
-        "combine_fused_into_down": fused,
         "hbm_frac": {"router": router_gbs / peaks["hbm_gbs"], "dispatch": disp_gbs / peaks["hbm_gbs"],
-                     "combine": None if fused else combine_gbs / peaks["hbm_gbs"],
+                     "combine": combine_gbs / peaks["hbm_gbs"],
                      "note": "algorithmic bytes / the stage's device-stamped span (moe_layer_forward_clocked: "
                              "first CTA start to last CTA end of the stage's kernels, dispatch = scan+rank "
                              "start to gather end, mean of back-to-back forwards) / the measured HBM copy "

@@ -267,19 +267,6 @@ int moe_combine(const moe_problem_t* p, const void* y_perm, const int32_t* slot_
                 const float* topk_w, const void* y_shared, void* y,
                 void* ws, size_t ws_bytes, moe_stream_t stream);
 
-/* Whether moe_layer_forward computes the combine inside the down
- * projection's epilogue for this problem (1) or with the separate combine
- * kernel (0); negative for an invalid problem.  HOST function.  Fused: BF16,
- * the routed (and shared) down projections on CTA-pair tiles in one launch,
- * with MOE_B200_FUSED_COMBINE=1 (off by default).  Each down tile that writes an expert row
- * adds its column halves to a per-(token, 256-column tile) counter after a
- * fence; the writer that completes the token's count (2 per kept pair, 2 for
- * the shared experts) combines those columns in the separate kernel's order
- * and rounding, so the output bytes are the same either way ("Scaling with
- * experts", The gating network, A budget, A shared expert).  Rows of tokens
- * with no kept pair and no shared experts are zeroed by the gather. */
-int moe_layer_combine_fused(const moe_problem_t* p);
-
 /* The whole layer: route -> dispatch -> routed experts -> shared experts ->
  * combine, plus statistics, enqueued on one stream with no host sync.
  *   x [T, d] in; w weights; y [T, d] out;

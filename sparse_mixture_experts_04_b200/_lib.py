@@ -30,8 +30,7 @@ EXPORTED = ("moe_abi_version", "moe_status_string", "moe_capacity", "moe_max_row
             "moe_layer_forward_clocked", "moe_expert_ffn_segments",
             "moe_dispatch_noalloc", "moe_dispatch_capacity", "moe_balance_update", "moe_backward_workspace_size",
             "moe_layer_backward", "moe_ep_plan", "moe_ep_peer_plan", "moe_ep_scatter", "moe_ep_combine",
-            "moe_ipc_malloc", "moe_ipc_free", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close",
-            "moe_layer_combine_fused")
+            "moe_ipc_malloc", "moe_ipc_free", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close")
 NUM_EVENTS = 7  # MOE_EV_START .. MOE_EV_END
 EVENT_NAMES = ("start", "routed", "dispatched", "up", "down", "shared", "end")
 NUM_CLOCKS = 7  # MOE_CLOCK_ROUTE .. MOE_CLOCK_COMBINE
@@ -122,8 +121,6 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_backward.restype = ctypes.c_int
     L.moe_ep_plan.argtypes = [i32, i32, i32, P, P, P, P]
     L.moe_ep_plan.restype = ctypes.c_int
-    L.moe_layer_combine_fused.argtypes = [PP]
-    L.moe_layer_combine_fused.restype = ctypes.c_int
     L.moe_ep_peer_plan.argtypes = [i32, i32, i32, P, P, P, P]
     L.moe_ep_peer_plan.restype = ctypes.c_int
     L.moe_ep_scatter.argtypes = [PP, i32, P, P, P, P, P, P]

@@ -325,12 +325,3 @@ class _Iface:
     def __init__(self, shape, typestr, ptr):
         self.__cuda_array_interface__ = {"shape": shape, "typestr": typestr, "data": (ptr, False), "version": 3,
                                          "strides": None}
-
-
-def layer_combine_fused(prob) -> bool:
-    """Whether moe_layer_forward does the combine inside the down projection
-    for this problem (see include/moe_b200.h, moe_layer_combine_fused)."""
-    rc = _lib.lib().moe_layer_combine_fused(ctypes.byref(prob))
-    if rc < 0:
-        _lib.check("moe_layer_combine_fused", rc)
-    return rc == 1

@@ -484,9 +484,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ seg_off, int E, int K,
                                                           int64_t T, int vec_per_row, int64_t max_rows,
-                                                          uint4* __restrict__ x_perm, unsigned long long* clk,
-                                                          uint4* __restrict__ zero_y,
-                                                          const int32_t* __restrict__ slot_of) {
+                                                          uint4* __restrict__ x_perm, unsigned long long* clk) {
   const int lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
@@ -510,17 +508,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
         if (v0 + 32 * j < vec_per_row) dst[v0 + 32 * j] = buf[j];
     }
   }
-  // the layer output of a token with no kept pair (and no shared experts) is
-  // zero; the combine fused into the down projection writes every other row
-  if (zero_y) {
-    for (int64_t t = warp0; t < T; t += n_warps) {
-      bool kept = false;
-      for (int k = lane; k < K; k += 32) kept |= slot_of[t * K + k] >= 0;
-      if (__any_sync(0xffffffffu, kept)) continue;
-      uint4* dst = zero_y + t * vec_per_row;
-      for (int v = lane; v < vec_per_row; v += 32) dst[v] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
   if (clk) {
     __syncthreads();
     stage_clock_end(clk);
@@ -528,8 +515,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
 }
 
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
-                          void* x_perm, cudaStream_t st, unsigned long long* clk, void* zero_y,
-                          const int32_t* slot_of) {
+                          void* x_perm, cudaStream_t st, unsigned long long* clk) {
   if (p.max_rows <= 0) return cudaSuccess;
   const int vec_per_row = static_cast<int>(p.d * p.esize() / 16);
   int64_t blocks = (p.max_rows + 7) / 8;
@@ -537,7 +523,7 @@ cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, 
   if (blocks > cap_blocks) blocks = cap_blocks;
   return launch_k(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
                   static_cast<const uint4*>(x), perm, seg_off, p.E, p.K, p.T, vec_per_row, p.max_rows,
-                  static_cast<uint4*>(x_perm), clk, static_cast<uint4*>(zero_y), slot_of);
+                  static_cast<uint4*>(x_perm), clk);
 }
 
 // Segment regrouping (moe_expert_ffn_segments): segment s holds expert s % E

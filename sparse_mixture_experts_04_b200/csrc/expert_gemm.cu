@@ -93,18 +93,6 @@ struct GemmArgs {
   // segments that repeat the experts, e.g. one run of experts per source rank
   // in the expert-parallel receive buffer); 0: expert g
   int weight_mod;
-  // pair kernel, EPI_BF16 (the layer's down projection): the combine as well
-  // (fc_contribute); fc_perm: routed rows (slot -> pair, token = pair / K),
-  // nullptr for the shared experts' rows (row = token)
-  int fc;
-  int* fc_count;  // [fc_T, fc_ntn] 128-column halves written so far (zeroed before the launch)
-  const int32_t* fc_slot_of;
-  const float* fc_w;
-  const int32_t* fc_perm;
-  const void* fc_yperm;
-  const void* fc_yshared;
-  void* fc_y;
-  int fc_T, fc_K, fc_ntn, fc_has_shared;
 };
 
 // Reduction range of a tile of group g: first k, number of 64-wide k-blocks.
@@ -316,86 +304,6 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& args, int g, int r
         }
       }
     }
-  }
-}
-
-// The combine fused into the down projection's epilogue ("Scaling with
-// experts", The gating network: y = sum of the gate-weighted expert outputs;
-// "A shared expert": its output added unweighted; "A budget": a dropped pair
-// adds nothing).  Every writer of 128 output columns of a token's expert row
-// (a routed slot or the shared experts' row) fences its stores and adds its
-// halves to the token's counter for this 256-column tile; the writer that
-// completes the count -- 2 halves per kept pair, 2 for the shared experts --
-// combines the tile's columns of that token from global memory: the shared
-// output first, then the kept pairs in k order, FP32, one rounding (the order
-// and rounding of the separate combine kernel, so the bytes are the same).
-// Called by all 32 lanes of a warp (lane: one row, `valid` if it wrote one);
-// the tokens the warp completes are then combined by the whole warp, lane l
-// taking columns n0 + 8 l .. + 7 with up to 4 expert rows in flight.
-__device__ __noinline__ void fc_contribute_warp(const GemmArgs& a, bool valid, int row, int n0, int units,
-                                                int lane) {
-  int t = -1;
-  bool last = false;
-  if (valid) {
-    t = a.fc_perm ? a.fc_perm[row] / a.fc_K : row;
-    if (t >= 0 && t < a.fc_T) {
-      const int32_t* so = a.fc_slot_of + static_cast<int64_t>(t) * a.fc_K;
-      int kept = 0;
-      for (int k = 0; k < a.fc_K; ++k) kept += so[k] >= 0 ? 1 : 0;
-      const int target = 2 * (kept + a.fc_has_shared);
-      __threadfence();
-      const int old = atomicAdd(a.fc_count + static_cast<int64_t>(t) * a.fc_ntn + n0 / 256, units);
-      last = old + units == target;
-    }
-  }
-  unsigned todo = __ballot_sync(0xffffffffu, last);
-  if (!todo) return;
-  __threadfence();
-  const int d = a.N;
-  const int col = n0 + 8 * lane;
-  const bool col_ok = col < d;
-  const __nv_bfloat16* yp = static_cast<const __nv_bfloat16*>(a.fc_yperm);
-  const __nv_bfloat16* ys = static_cast<const __nv_bfloat16*>(a.fc_yshared);
-  while (todo) {
-    const int src = __ffs(todo) - 1;
-    todo &= todo - 1;
-    const int tt = __shfl_sync(0xffffffffu, t, src);
-    const int my_slot = lane < a.fc_K ? a.fc_slot_of[static_cast<int64_t>(tt) * a.fc_K + lane] : -1;
-    const float my_w = lane < a.fc_K ? a.fc_w[static_cast<int64_t>(tt) * a.fc_K + lane] : 0.f;
-    float acc[8];
-    if (ys && col_ok) {
-      const uint4 q = __ldcg(reinterpret_cast<const uint4*>(ys + static_cast<int64_t>(tt) * d + col));
-      acc[0] = bf16_lo(q.x); acc[1] = bf16_hi(q.x); acc[2] = bf16_lo(q.y); acc[3] = bf16_hi(q.y);
-      acc[4] = bf16_lo(q.z); acc[5] = bf16_hi(q.z); acc[6] = bf16_lo(q.w); acc[7] = bf16_hi(q.w);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    }
-    for (int k0 = 0; k0 < a.fc_K; k0 += 4) {
-      uint4 q[4];
-      float wk[4];
-      bool ok[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int slot = __shfl_sync(0xffffffffu, my_slot, (k0 + j) & 31);
-        wk[j] = __shfl_sync(0xffffffffu, my_w, (k0 + j) & 31);
-        ok[j] = k0 + j < a.fc_K && slot >= 0 && col_ok;
-        q[j] = ok[j] ? __ldcg(reinterpret_cast<const uint4*>(yp + static_cast<int64_t>(slot) * d + col))
-                     : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (ok[j]) {
-          const float r[8] = {bf16_lo(q[j].x), bf16_hi(q[j].x), bf16_lo(q[j].y), bf16_hi(q[j].y),
-                              bf16_lo(q[j].z), bf16_hi(q[j].z), bf16_lo(q[j].w), bf16_hi(q[j].w)};
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(wk[j], r[i], acc[i]);
-        }
-    }
-    if (col_ok)
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.fc_y) + static_cast<int64_t>(tt) * d + col) =
-          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
-                     pack_bf16x2(acc[6], acc[7]));
   }
 }
 
@@ -768,11 +676,8 @@ __device__ __forceinline__ void epilogue_swap(const GemmArgs& args, const TileIn
               make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
         }
       }
-      if (args.fc) __threadfence();  // this CTA's half of the 32 tokens' rows, before the count
     }
     named_bar_sync(1, 128);
-    // the first epilogue warp adds this CTA's half of the chunk's 32 tokens (lane = token)
-    if (EPI == EPI_BF16 && args.fc && et < 32) fc_contribute_warp(args, c + et < rows, ti.row0 + c + et, ti.n0, 1, et);
   }
 }
 
@@ -1049,7 +954,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       } else {
         const int row = ti.row0 + 128 * static_cast<int>(rank) + r;
         epilogue_rows<EPI, kPairBN>(A, ti.g, row, row < ti.row_end, ti.n0, t_row);
-        if (EPI == EPI_BF16 && A.fc) fc_contribute_warp(A, row < ti.row_end, row, ti.n0, 2, lane);
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -1566,7 +1470,7 @@ static bool up_pair_problem(const Problem& p, bool routed, const void* x_rows, i
 // rows.  Shared: one group whose reduction runs over all N_s experts.
 static bool down_pair_problem(const Problem& p, bool routed, const void* h, int64_t n_rows, const int32_t* seg_off,
                               const void* w2, void* y_rows, unsigned* status, bool tail, PairProblem* q,
-                              int n_seg = 0, const FusedCombine* fc = nullptr) {
+                              int n_seg = 0) {
   const int G = routed ? p.E : p.Ns;
   const int64_t h_cols = routed ? p.F : static_cast<int64_t>(p.Ns) * p.F;
   const bool merged = merged_k_ok(p.F);
@@ -1596,20 +1500,6 @@ static bool down_pair_problem(const Problem& p, bool routed, const void* h, int6
   a.row_mode = tail ? 1 : 0;
   a.merged_k = merged ? 1 : 0;
   a.deep_swap = merged && deep_swap_on() ? 1 : 0;
-  if (fc && !tail) {
-    a.fc = 1;
-    a.fc_count = fc->count;
-    a.fc_slot_of = fc->slot_of;
-    a.fc_w = fc->topk_w;
-    a.fc_perm = routed ? fc->perm : nullptr;
-    a.fc_yperm = fc->y_perm;
-    a.fc_yshared = fc->y_shared;
-    a.fc_y = fc->y;
-    a.fc_T = static_cast<int>(p.T);
-    a.fc_K = p.K;
-    a.fc_ntn = static_cast<int>(cdiv(p.d, 256));
-    a.fc_has_shared = p.Ns > 0 ? 1 : 0;
-  }
   const int64_t mt = routed ? cdiv(n_rows, kBM) + a.n_groups : cdiv(n_rows, kBM);
   q->tile_bound = (mt / 2 + a.n_groups) * cdiv(p.d, 256);
   return true;
@@ -1695,7 +1585,7 @@ static bool down_single_problem(const Problem& p, bool routed, const void* h, in
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status, cudaStream_t st,
                       cudaEvent_t after_up, int* n_kernels, void* gu, unsigned long long* clk_up,
-                      unsigned long long* clk_down, int n_seg, const FusedCombine* fc) {
+                      unsigned long long* clk_down, int n_seg) {
   if (n_rows <= 0) return 0;
   if (p.dtype == kF32) {
     if (n_kernels) *n_kernels += 2;
@@ -1750,9 +1640,7 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
     if (!make_map(&ta, h, 2, da, ba) || !make_map(&tb, w2, 3, db, bb)) return -3;
     if (pair) {
       PairProblem q;
-      if (!down_pair_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, tail, &q, n_seg,
-                             routed && !tail ? fc : nullptr))
-        return -3;
+      if (!down_pair_problem(p, routed, h, n_rows, seg_off, w2, y_rows, status, tail, &q, n_seg)) return -3;
       q.a.clk = clk_down;
       int rc = run_pair_gemm<EPI_BF16>(q, nullptr, st);
       if (rc) return rc;
@@ -1775,15 +1663,6 @@ int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_
   return 0;
 }
 
-bool fused_combine_ok(const Problem& p) {
-  // opt-in (MOE_B200_FUSED_COMBINE=1): measured slower than the separate combine
-  const char* e = getenv("MOE_B200_FUSED_COMBINE");
-  if (!(e && e[0] == '1')) return false;
-  if (p.dtype != kBF16 || p.max_rows <= 0 || p.d % 8 != 0) return false;
-  if (ffn_tile_mode(p, true, p.max_rows) != kTilePair) return false;
-  return p.Ns == 0 || expert_ffn_mixed_ok(p);
-}
-
 bool expert_ffn_mixed_ok(const Problem& p) {
   const char* e = getenv("MOE_B200_MIX_SHARED");
   if (e && e[0] == '0') return false;
@@ -1800,7 +1679,7 @@ int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t*
                             const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
                             const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
                             cudaStream_t st, cudaEvent_t after_up, int* n_kernels, unsigned long long* clk_up,
-                            unsigned long long* clk_down, const FusedCombine* fc) {
+                            unsigned long long* clk_down) {
   if (!expert_ffn_mixed_ok(p)) return -3;
   if (n_kernels) *n_kernels += 2;
   if (ffn_tile_mode(p, true, p.max_rows) == kTileSingle) {
@@ -1825,8 +1704,8 @@ int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t*
   r.a.clk = clk_up;
   if (int rc = run_pair_gemm<EPI_SWIGLU>(r, &s, st)) return rc;
   if (after_up && cudaEventRecord(after_up, st) != cudaSuccess) return -3;
-  if (!down_pair_problem(p, true, h, p.max_rows, seg_off, w2, y_perm, status, false, &r, 0, fc) ||
-      !down_pair_problem(p, false, h_shared, p.T, nullptr, w2_shared, y_shared, status, false, &s, 0, fc))
+  if (!down_pair_problem(p, true, h, p.max_rows, seg_off, w2, y_perm, status, false, &r) ||
+      !down_pair_problem(p, false, h_shared, p.T, nullptr, w2_shared, y_shared, status, false, &s))
     return -3;
   r.a.clk = clk_down;
   return run_pair_gemm<EPI_BF16>(r, &s, st);

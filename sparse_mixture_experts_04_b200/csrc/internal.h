@@ -36,8 +36,7 @@ struct WsLayout {
   size_t status, logits, topk_idx, topk_w, counts, kept, seg_off, slot_of, perm;
   size_t chunk_counts, chunk_psum, chunk_base, logit_parts, zpart;
   size_t seg_map;  // moe_expert_ffn_segments: [kMaxSegments] destinations + [kMaxSegments + 1] expert offsets
-  size_t fc_count;  // BF16: [T, ceil(d / 256)] int32 counters of the combine fused into the down projection
-  size_t zero_bytes;  // status word + chunk histogram + chunk p sums + fc_count: cleared together at offset 0
+  size_t zero_bytes;  // status word + chunk histogram + chunk p sums: cleared together at offset 0
   size_t x_perm, h_routed, y_perm, h_shared, y_shared;
   size_t gu_routed, gu_shared;  // with MOE_FLAG_SAVE_GU: the gate/up projections for the backward
   size_t total;
@@ -88,11 +87,8 @@ cudaError_t launch_dispatch(const Problem& p, const int32_t* topk_idx, int32_t* 
                             const unsigned long long* chunk_psum = nullptr, float* stats = nullptr,
                             const float* zpart = nullptr, int n_zpart = 0, const int32_t* expert_cap = nullptr,
                             unsigned long long* clk = nullptr);
-// zero_y (or nullptr): [T, d] rows of tokens whose pairs were all dropped are
-// zeroed as well (the fused combine's output with no shared experts)
 cudaError_t launch_gather(const Problem& p, const void* x, const int32_t* perm, const int32_t* seg_off,
-                          void* x_perm, cudaStream_t st, unsigned long long* clk = nullptr,
-                          void* zero_y = nullptr, const int32_t* slot_of = nullptr);
+                          void* x_perm, cudaStream_t st, unsigned long long* clk = nullptr);
 
 // dispatch.cu: rows of n_seg segments (segment s = source s / E, expert s % E)
 // moved into expert-major order and back: segment_regroup_plan writes each
@@ -129,27 +125,11 @@ cudaError_t launch_router_fused(const Problem& p, const void* x, const void* w_g
 int router_k_splits(const Problem& p);  // slices of the tensor-core gate GEMM's reduction
 int launch_gate_logits_tc(const Problem& p, const void* x, const void* w_gate, const float* offset, float* out,
                           int n_splits, unsigned* status, cudaStream_t st, unsigned long long* clk = nullptr);
-// The layer's combine done by the down projection's epilogue (CTA-pair
-// tiles): the counter array is zeroed before the launch; y rows of tokens with
-// no kept pair and no shared experts are written by the gather (launch_gather
-// with zero_y).
-struct FusedCombine {
-  int* count;              // [T, ceil(d / 256)] int32
-  const int32_t* slot_of;  // [T, K]
-  const float* topk_w;     // [T, K]
-  const int32_t* perm;     // [rows] slot -> pair
-  const void* y_perm;      // routed outputs
-  const void* y_shared;    // shared outputs, or nullptr
-  void* y;                 // [T, d] layer output
-};
-// The layer forward can fuse the combine (BF16, routed (and shared) down
-// projections on CTA pairs in one launch; MOE_B200_FUSED_COMBINE=0 turns it off).
-bool fused_combine_ok(const Problem& p);
 int launch_expert_ffn(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,
                       const void* w13, const void* w2, void* h, void* y_rows, unsigned* status,
                       cudaStream_t st, cudaEvent_t after_up = nullptr, int* n_kernels = nullptr,
                       void* gu = nullptr, unsigned long long* clk_up = nullptr,
-                      unsigned long long* clk_down = nullptr, int n_seg = 0, const FusedCombine* fc = nullptr);
+                      unsigned long long* clk_down = nullptr, int n_seg = 0);
 // (routed mode) n_seg > 0: seg_off has n_seg + 1 entries and row segment s is
 // computed with expert s % p.E (moe_expert_ffn_segments).
 // Routed (x_perm over seg_off, p.max_rows rows) and shared (x, T rows)
@@ -162,8 +142,7 @@ int launch_expert_ffn_mixed(const Problem& p, const void* x_perm, const int32_t*
                             const void* w2, void* h, void* y_perm, void* gu, const void* x, const void* w13_shared,
                             const void* w2_shared, void* h_shared, void* y_shared, void* gu_shared, unsigned* status,
                             cudaStream_t st, cudaEvent_t after_up, int* n_kernels,
-                            unsigned long long* clk_up = nullptr, unsigned long long* clk_down = nullptr,
-                            const FusedCombine* fc = nullptr);
+                            unsigned long long* clk_up = nullptr, unsigned long long* clk_down = nullptr);
 
 // expert_gemm.cu: gu = x W13^T (gate | up projections, BF16) for the backward
 int launch_up_projections(const Problem& p, int mode, const void* x_rows, int64_t n_rows, const int32_t* seg_off,

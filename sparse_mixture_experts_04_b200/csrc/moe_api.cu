@@ -58,8 +58,7 @@ WsLayout make_layout(const Problem& p) {
   L.status = 0;
   L.chunk_psum = 256;                              // 8-byte entries
   L.chunk_counts = align256(L.chunk_psum + ce * 8);
-  L.fc_count = align256(L.chunk_counts + ce * 4);
-  L.zero_bytes = L.fc_count + (p.dtype == kBF16 ? static_cast<size_t>(p.T) * ((p.d + 255) / 256) * 4 : 0);
+  L.zero_bytes = L.chunk_counts + ce * 4;
   off = align256(L.zero_bytes);
   L.logits = take(static_cast<size_t>(p.T) * p.E * 4);
   L.topk_idx = take(TK * 4);
@@ -483,15 +482,8 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
                                       n_zpart, expert_cap, clk(MOE_CLOCK_DISPATCH)))
     return cuda_rc(e);
   kernels += dispatch_fused(p) ? 1 : 2;
-  // the combine inside the down projection's epilogue (counters in the zeroed
-  // prefix of the workspace); rows of tokens with nothing kept and no shared
-  // experts are zeroed by the gather
-  const bool fuse = fused_combine_ok(p);
-  FusedCombine fc{at<int>(ws, L.fc_count), slot_of, gw, perm, y_perm, y_sh, y};
   if (p.max_rows > 0) {
-    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st, clk(MOE_CLOCK_GATHER),
-                                      fuse && p.Ns == 0 ? y : nullptr, slot_of))
-      return cuda_rc(e);
+    if (cudaError_t e = launch_gather(p, x, perm, seg_off, x_perm, st, clk(MOE_CLOCK_GATHER))) return cuda_rc(e);
     kernels += 1;
   }
   if (cudaError_t e = mark(MOE_EV_DISPATCHED)) return cuda_rc(e);
@@ -503,15 +495,14 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     if (launch_expert_ffn_mixed(p, x_perm, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed), y_perm,
                                 save_gu ? at<void>(ws, L.gu_routed) : nullptr, x, w->w13_shared, w->w2_shared,
                                 at<void>(ws, L.h_shared), y_sh, save_gu ? at<void>(ws, L.gu_shared) : nullptr,
-                                status, st, up_ev, &kernels, clk(MOE_CLOCK_UP), clk(MOE_CLOCK_DOWN),
-                                fuse ? &fc : nullptr))
+                                status, st, up_ev, &kernels, clk(MOE_CLOCK_UP), clk(MOE_CLOCK_DOWN)))
       return MOE_ERR_CUDA;
     if (cudaError_t e = mark(MOE_EV_DOWN)) return cuda_rc(e);
   } else {
     if (p.max_rows > 0) {
       if (launch_expert_ffn(p, MOE_FFN_ROUTED, x_perm, p.max_rows, seg_off, w->w13, w->w2, at<void>(ws, L.h_routed),
                             y_perm, status, st, up_ev, &kernels, save_gu ? at<void>(ws, L.gu_routed) : nullptr,
-                            clk(MOE_CLOCK_UP), clk(MOE_CLOCK_DOWN), 0, fuse ? &fc : nullptr))
+                            clk(MOE_CLOCK_UP), clk(MOE_CLOCK_DOWN)))
         return MOE_ERR_CUDA;
     } else if (cudaError_t e = mark(MOE_EV_UP)) {
       return cuda_rc(e);
@@ -526,20 +517,11 @@ static int layer_forward_impl(const moe_problem_t* q, const void* x, const moe_w
     }
   }
   if (cudaError_t e = mark(MOE_EV_SHARED)) return cuda_rc(e);
-  if (!fuse) {
-    if (cudaError_t e = launch_combine(p, y_perm, slot_of, gw, y_sh, y, st, clk(MOE_CLOCK_COMBINE)))
-      return cuda_rc(e);
-    kernels += 1;
-  }
+  if (cudaError_t e = launch_combine(p, y_perm, slot_of, gw, y_sh, y, st, clk(MOE_CLOCK_COMBINE))) return cuda_rc(e);
+  kernels += 1;
   if (cudaError_t e = mark(MOE_EV_END)) return cuda_rc(e);
   if (n_kernels) *n_kernels = kernels;
   return MOE_OK;
-}
-
-int moe_layer_combine_fused(const moe_problem_t* q) {
-  Problem p;
-  if (int rc = to_problem(q, &p)) return rc;
-  return fused_combine_ok(p) ? 1 : 0;
 }
 
 int moe_layer_forward(const moe_problem_t* q, const void* x, const moe_weights_t* w, void* y,

@@ -346,36 +346,6 @@ def test_combine_matches_oracle(name):
     assert np.all(np.abs(got - want) <= ulp * np.abs(want) + 1e-6 * np.max(np.abs(want)))
 
 
-@pytest.mark.parametrize("name,tile", [("mini_mixtral", "256all"), ("mini_zen", "256all"), ("mini_skewed", "256all"),
-                                       ("ragged_bf16", "256all"), ("tiny_capacity", "256all"),
-                                       ("max_k32", "256all"), ("wide_e256", "256all")])
-def test_combine_in_the_down_projection_is_bit_identical(name, tile, monkeypatch):
-    """The layer with the combine inside the down projection's epilogue (per
-    token and 256-column tile, the writer that completes the count combines)
-    against the separate combine kernel (MOE_B200_FUSED_COMBINE=0): the same
-    output bytes, routing and statistics -- shared experts, dropped pairs and
-    tokens with every pair dropped, swap tiles, ragged d included; and the
-    oracle's layer."""
-    monkeypatch.setenv("MOE_B200_GEMM_TILE", tile)
-    cfg = SMALL[name]
-    inp = inputs(name)
-    logits32 = given_logits(cfg)
-    outs = []
-    for fuse in ("1", "0"):
-        monkeypatch.setenv("MOE_B200_FUSED_COMBINE", fuse)
-        layer = MoeLayer.from_inputs(inp, flags=api.FLAG_LOGITS_GIVEN)
-        assert api.layer_combine_fused(layer.prob) == (fuse == "1")
-        layer.routing["logits"].copy_(torch.as_tensor(logits32))
-        y = layer.forward(dev(inp["x"]))
-        y2 = layer.forward(dev(inp["x"]))   # the counters start from zero every forward
-        assert api.read_device_status(layer.ws) == 0
-        assert torch.equal(y, y2)
-        outs.append((y.clone(), layer.stats.clone()))
-    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
-    ref = oracle_routing(cfg, logits32.astype(np.float64), inp["sel_bias"])
-    assert rel_err(outs[0][0].float().cpu().numpy(), oracle_layer(inp, ref)) <= tol(cfg)
-
-
 # ------------------------------------------------------------- whole layer
 @pytest.mark.parametrize("name", list(SMALL))
 def test_layer_forward_given_logits_matches_oracle(name):
@@ -458,18 +428,14 @@ def test_clocked_forward_equals_the_plain_forward_and_stamps_its_stages(name):
     for k, v in layer.routing.items():
         assert torch.equal(r1[k], v), k
     us = api.stage_clock_us(clocks.cpu().tolist())
-    # with the combine inside the down projection's epilogue there is no combine launch
-    fused = api.layer_combine_fused(layer.prob)
-    order = ["route", "dispatch", "gather", "up", "down"] + ([] if fused else ["combine"])
-    for st in order:
+    for st in ("route", "dispatch", "gather", "up", "down", "combine"):
         assert us[st] is not None and 0.0 < us[st] < 1e5, (st, us)
-    if fused:
-        assert us["combine"] is None
     c = [int(v) & 0xFFFFFFFFFFFFFFFF for v in clocks.cpu().tolist()]
     names = _lib.CLOCK_NAMES
     start = lambda n: (~c[2 * names.index(n)]) & 0xFFFFFFFFFFFFFFFF
     end = lambda n: c[2 * names.index(n) + 1]
     # each stage starts reading only after its predecessor's last CTA ended
+    order = ["route", "dispatch", "gather", "up", "down", "combine"]
     for a, b in zip(order, order[1:]):
         assert end(a) <= start(b), (a, b)
 
