@@ -359,9 +359,19 @@ class PeerRank:
                            k.y_shared, y)
         return y
 
-    def release(self) -> None:
-        """Unmap the peers' buffers and free this rank's own (open_peer_buffers)."""
-        for b in self.ipc:
+    def release(self, group=None) -> None:
+        """Unmap the peers' buffers, wait until every rank has unmapped this
+        rank's (a barrier of the process group, when one is initialised), then
+        free this rank's own (open_peer_buffers).  Every rank calls it."""
+        opened = [b for b in self.ipc if b.opened]
+        own = [b for b in self.ipc if not b.opened]
+        for b in opened:
+            b.release()
+        if own:
+            import torch.distributed as dist
+            if dist.is_available() and dist.is_initialized():
+                dist.barrier(group=group)
+        for b in own:
             b.release()
         self.ipc = []
 

@@ -242,6 +242,7 @@ class _FakeIpc:
     handle gives the owner's address back, as CUDA IPC maps the same memory."""
     rank = 0
     made = []
+    release_order = []
 
     def __init__(self, shape, dtype, handle=None):
         if handle is None:
@@ -260,6 +261,7 @@ class _FakeIpc:
 
     def release(self):
         self.released = True
+        _FakeIpc.release_order.append(self)
 
 
 class _Kernels:
@@ -285,6 +287,9 @@ def _peer_table_worker(rank, world, port, q):
                tuple(rk.k.x_loc.shape), len(rk.ipc)))
         rk.release()
         assert all(b.released for b in _FakeIpc.made)
+        # the peers' mappings were closed before this rank's own buffers were freed
+        order = [b.opened for b in _FakeIpc.release_order]
+        assert order == sorted(order, reverse=True)
         dist.barrier()
     finally:
         dist.destroy_process_group()
