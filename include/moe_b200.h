@@ -514,7 +514,10 @@ int moe_ep_peer_plan(int32_t n_ranks, int32_t rank, int32_t n_experts, const int
  *              (peer memory mapped into this process for q != rank, e.g. by
  *              moe_ipc_open), each [rows q receives, d]
  * The receiving rank may read its buffer once every rank's scatter has
- * completed (the caller orders that, e.g. with a barrier on the stream). */
+ * completed (the caller orders that, e.g. with a barrier on the stream).
+ * Errors: the problem's checks (as moe_dispatch); MOE_ERR_INVALID_ARG for
+ * NULL pointers, an x not 16-byte aligned, n_ranks < 1 or E % n_ranks != 0;
+ * MOE_ERR_CUDA for a failed launch. */
 int moe_ep_scatter(const moe_problem_t* p, int32_t n_ranks, const void* x, const int32_t* perm,
                    const int32_t* seg_off, void* const* recv_bufs, const int64_t* delta,
                    moe_stream_t stream);
@@ -527,7 +530,10 @@ int moe_ep_scatter(const moe_problem_t* p, int32_t n_ranks, const void* x, const
  * sums, one rounding).  out_bufs [G] device array of device pointers (rank
  * q's output buffer, row for row its receive buffer); y_shared as in
  * moe_combine (NULL iff n_shared == 0); y [T, d] out.  Every rank's expert
- * GEMM must have completed before the call's kernel starts. */
+ * GEMM must have completed before the call's kernel starts.
+ * Errors: the problem's checks; MOE_ERR_INVALID_ARG for NULL pointers, y or
+ * y_shared not 16-byte aligned, y_shared given iff n_shared == 0, n_ranks < 1
+ * or E % n_ranks != 0; MOE_ERR_CUDA for a failed launch. */
 int moe_ep_combine(const moe_problem_t* p, int32_t n_ranks, const void* const* out_bufs,
                    const int64_t* delta, const int32_t* topk_idx, const int32_t* slot_of,
                    const float* topk_w, const void* y_shared, void* y, moe_stream_t stream);
