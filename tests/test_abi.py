@@ -213,3 +213,30 @@ def test_backward_rejects_bad_arguments_before_launching(L):
     assert call(prob_=f32) == -2
     given = api.make_problem(64, 64, 8, 2, 128, flags=api.FLAG_LOGITS_GIVEN)
     assert call(prob_=given) == -1   # dw_gate requested although the logits are given
+
+
+def test_peer_exchange_entry_points_reject_bad_arguments_before_launching(L):
+    """moe_ep_peer_plan / moe_ep_scatter / moe_ep_combine and the IPC calls
+    refuse bad arguments on the host, before any launch or CUDA call."""
+    prob = api.make_problem(64, 64, 8, 2, 128, n_shared=0)
+    P = ctypes.byref(prob)
+    fake = 4096
+    # plan: rank out of range, E not divisible by G, E above 256, NULL outputs
+    assert L.moe_ep_peer_plan(2, 2, 8, fake, fake, fake, None) == -1
+    assert L.moe_ep_peer_plan(3, 0, 8, fake, fake, fake, None) == -1
+    assert L.moe_ep_peer_plan(1, 0, 512, fake, fake, fake, None) == -1
+    assert L.moe_ep_peer_plan(2, 0, 8, fake, None, fake, None) == -1
+    # scatter: G does not divide E; misaligned x; NULL table
+    assert L.moe_ep_scatter(P, 3, fake, fake, fake, fake, fake, None) == -1
+    assert L.moe_ep_scatter(P, 2, fake + 4, fake, fake, fake, fake, None) == -1
+    assert L.moe_ep_scatter(P, 2, fake, fake, fake, None, fake, None) == -1
+    # combine: y_shared given although n_shared == 0; misaligned y; G does not divide E
+    assert L.moe_ep_combine(P, 2, fake, fake, fake, fake, fake, fake, fake, None) == -1
+    assert L.moe_ep_combine(P, 2, fake, fake, fake, fake, fake, None, fake + 8, None) == -1
+    assert L.moe_ep_combine(P, 3, fake, fake, fake, fake, fake, None, fake, None) == -1
+    # IPC: NULL arguments, zero bytes
+    p = ctypes.c_void_p()
+    assert L.moe_ipc_malloc(0, ctypes.byref(p)) == -1
+    assert L.moe_ipc_handle(None, fake) == -1
+    assert L.moe_ipc_open(None, ctypes.byref(p)) == -1
+    assert L.moe_ipc_close(None) == -1 and L.moe_ipc_free(None) == -1
